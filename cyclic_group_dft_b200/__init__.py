@@ -1,0 +1,44 @@
+"""B200-native (sm_100a) EQ-Linear forward over the cyclic group C_G.
+
+y[n,o,g] = bias[o] + sum_{i,h} w[o,i,(g-h) mod G] x[n,i,h], computed as a real
+DFT over the group axis, per-frequency contractions on tcgen05 tensor cores
+(half spectrum) and an inverse DFT, fused in one kernel.
+
+Usage::
+
+    import cyclic_group_dft_b200 as eq
+    h = eq.prepare(w, bias)          # w [Cout, Cin, G] CUDA tensor (bf16 or fp32)
+    y = h.forward(x)                 # x [N, Cin, G] -> y [N, Cout, G]
+
+The functions with the C ABI's names (eqlin_prepare_weights, eqlin_forward,
+eqlin_destroy, ...) are the same calls with explicit arguments.
+"""
+from ._capi import (  # noqa: F401
+    ATTRS,
+    EQLIN_BF16,
+    EQLIN_ERR_CUDA,
+    EQLIN_ERR_INVALID_ARG,
+    EQLIN_ERR_MISALIGNED,
+    EQLIN_ERR_OOM,
+    EQLIN_ERR_TIMEOUT,
+    EQLIN_ERR_UNSUPPORTED,
+    EQLIN_F32,
+    EQLIN_OK,
+    LIB_PATH,
+    PATH_NAMES,
+    EqlinError,
+    Handle,
+    eqlin_check_shape,
+    eqlin_copy_freq_weights,
+    eqlin_destroy,
+    eqlin_device_status,
+    eqlin_forward,
+    eqlin_last_error,
+    eqlin_prepare_weights,
+    eqlin_status_string,
+    eqlin_version,
+    header_functions,
+    library,
+)
+
+prepare = eqlin_prepare_weights

@@ -1,0 +1,253 @@
+"""ctypes binding of libeqlin.so (C ABI in include/eqlin.h).
+
+Argument marshalling only: every step of the forward runs in the library's
+kernels.  torch supplies device memory and streams.  Importing this module
+fails loudly if the library has not been built -- there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libeqlin.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "eqlin.h")
+
+EQLIN_F32 = 0
+EQLIN_BF16 = 1
+
+EQLIN_OK = 0
+EQLIN_ERR_INVALID_ARG = -1
+EQLIN_ERR_UNSUPPORTED = -2
+EQLIN_ERR_MISALIGNED = -3
+EQLIN_ERR_CUDA = -4
+EQLIN_ERR_OOM = -5
+EQLIN_ERR_TIMEOUT = -6
+
+ATTRS = {
+    "G": 0, "Cin": 1, "Cout": 2, "io_dtype": 3, "path": 4, "tokens_per_tile": 5,
+    "stages": 6, "smem_bytes": 7, "max_grid": 8, "weight_bytes": 9,
+}
+PATH_NAMES = {0: "tcgen05_resident_weights", 1: "tcgen05_streamed_weights", 2: "fp32_ffma"}
+
+_TORCH_TO_EQLIN = {torch.float32: EQLIN_F32, torch.bfloat16: EQLIN_BF16}
+_EQLIN_TO_TORCH = {v: k for k, v in _TORCH_TO_EQLIN.items()}
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build the CUDA library first "
+        "(python -m cyclic_group_dft_b200.build); there is no fallback path")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_vp, _i64, _int = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+_lib.eqlin_prepare_weights.argtypes = [_vp, _vp, _i64, _i64, _i64, _int, _int, _vp, ctypes.POINTER(_vp)]
+_lib.eqlin_forward.argtypes = [_vp, _vp, _vp, _i64, _vp]
+_lib.eqlin_destroy.argtypes = [_vp]
+_lib.eqlin_device_status.argtypes = [_vp, ctypes.POINTER(_int)]
+_lib.eqlin_get_attr.argtypes = [_vp, _int, ctypes.POINTER(_i64)]
+_lib.eqlin_copy_freq_weights.argtypes = [_vp, ctypes.POINTER(ctypes.c_float), _i64]
+_lib.eqlin_check_shape.argtypes = [_i64, _i64, _i64, _int, _int]
+_lib.eqlin_status_string.argtypes = [_int]
+_lib.eqlin_status_string.restype = ctypes.c_char_p
+_lib.eqlin_last_error.argtypes = []
+_lib.eqlin_last_error.restype = ctypes.c_char_p
+_lib.eqlin_version.argtypes = []
+for _f in ("eqlin_prepare_weights", "eqlin_forward", "eqlin_destroy", "eqlin_device_status",
+           "eqlin_get_attr", "eqlin_copy_freq_weights", "eqlin_check_shape", "eqlin_version"):
+    getattr(_lib, _f).restype = _int
+
+
+class EqlinError(RuntimeError):
+    """A C-ABI call returned a negative eqlin_status."""
+
+    def __init__(self, status: int, what: str):
+        self.status = status
+        msg = _lib.eqlin_last_error().decode(errors="replace")
+        super().__init__(f"{what}: {eqlin_status_string(status)} ({status}): {msg}")
+
+
+def _check(status: int, what: str) -> None:
+    if status != EQLIN_OK:
+        raise EqlinError(status, what)
+
+
+def library() -> ctypes.CDLL:
+    """The loaded libeqlin.so."""
+    return _lib
+
+
+def header_functions() -> list[str]:
+    """Names of the functions include/eqlin.h declares."""
+    with open(HEADER_PATH) as f:
+        text = f.read()
+    return re.findall(r"^EQLIN_API\s+[\w\s\*]+?\b(eqlin_\w+)\s*\(", text, flags=re.M)
+
+
+def eqlin_status_string(status: int) -> str:
+    return _lib.eqlin_status_string(int(status)).decode()
+
+
+def eqlin_last_error() -> str:
+    return _lib.eqlin_last_error().decode(errors="replace")
+
+
+def eqlin_version() -> int:
+    return int(_lib.eqlin_version())
+
+
+def eqlin_check_shape(Cout: int, Cin: int, G: int, w_dtype=EQLIN_BF16, io_dtype=EQLIN_BF16) -> int:
+    """Host-only shape check; returns the status prepare's validation would give."""
+    return int(_lib.eqlin_check_shape(Cout, Cin, G, _as_code(w_dtype), _as_code(io_dtype)))
+
+
+def _as_code(dt) -> int:
+    if isinstance(dt, torch.dtype):
+        return _TORCH_TO_EQLIN[dt]
+    return int(dt)
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+class Handle:
+    """Frequency-domain weights prepared on one device (owns device memory)."""
+
+    def __init__(self, ptr: int, device: torch.device):
+        self._ptr = ptr
+        self.device = device
+        self.G = self.attr("G")
+        self.Cin = self.attr("Cin")
+        self.Cout = self.attr("Cout")
+        self.io_dtype = _EQLIN_TO_TORCH[self.attr("io_dtype")]
+
+    @property
+    def ptr(self) -> int:
+        if not self._ptr:
+            raise EqlinError(EQLIN_ERR_INVALID_ARG, "handle already destroyed")
+        return self._ptr
+
+    def attr(self, name: str) -> int:
+        v = ctypes.c_int64()
+        _check(_lib.eqlin_get_attr(self.ptr, ATTRS[name], ctypes.byref(v)), f"eqlin_get_attr({name})")
+        return int(v.value)
+
+    @property
+    def path(self) -> str:
+        return PATH_NAMES[self.attr("path")]
+
+    def forward(self, x: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        return eqlin_forward(self, x, out, stream)
+
+    def forward_host(self, x_host: torch.Tensor, out_host: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
+        """Forward from and to host memory: copy x in, run, copy y back (synchronous)."""
+        if x_host.device.type != "cpu":
+            raise ValueError("forward_host takes a CPU tensor")
+        with torch.cuda.device(self.device):
+            s = torch.cuda.current_stream() if stream is None else stream
+            with torch.cuda.stream(s):
+                xd = x_host.to(self.device, non_blocking=True)
+                yd = eqlin_forward(self, xd, None, s)
+                if out_host is None:
+                    out_host = torch.empty(yd.shape, dtype=yd.dtype, pin_memory=x_host.is_pinned())
+                out_host.copy_(yd, non_blocking=True)
+            s.synchronize()
+        return out_host
+
+    def device_status(self) -> int:
+        return eqlin_device_status(self)
+
+    def freq_weights(self) -> torch.Tensor:
+        return eqlin_copy_freq_weights(self)
+
+    def close(self) -> None:
+        if self._ptr:
+            p, self._ptr = self._ptr, None
+            _check(_lib.eqlin_destroy(p), "eqlin_destroy")
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def __del__(self):
+        try:
+            if self._ptr and _lib is not None:
+                _lib.eqlin_destroy(self._ptr)
+                self._ptr = None
+        except Exception:
+            pass
+
+
+def eqlin_prepare_weights(w: torch.Tensor, bias: torch.Tensor | None = None,
+                          io_dtype: torch.dtype | None = None, stream=None) -> Handle:
+    """Transform w [Cout, Cin, G] (and bias [Cout]) to the frequency domain on w's device."""
+    if w.dim() != 3:
+        raise ValueError("w must be [Cout, Cin, G]")
+    if w.device.type != "cuda":
+        raise ValueError("w must be a CUDA tensor")
+    if w.dtype not in _TORCH_TO_EQLIN:
+        raise ValueError(f"unsupported weight dtype {w.dtype}")
+    w = w.contiguous()
+    Cout, Cin, G = w.shape
+    if bias is not None:
+        if bias.shape != (Cout,) or bias.device != w.device:
+            raise ValueError("bias must be [Cout] on w's device")
+        bias = bias.to(w.dtype).contiguous()
+    io = _TORCH_TO_EQLIN[w.dtype if io_dtype is None else io_dtype]
+    out = ctypes.c_void_p()
+    with torch.cuda.device(w.device):
+        st = _lib.eqlin_prepare_weights(
+            w.data_ptr(), None if bias is None else bias.data_ptr(), Cout, Cin, G,
+            _TORCH_TO_EQLIN[w.dtype], io, _stream_ptr(stream), ctypes.byref(out))
+    _check(st, "eqlin_prepare_weights")
+    return Handle(out.value, w.device)
+
+
+def eqlin_forward(h: Handle, x: torch.Tensor, y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y [N, Cout, G] = EQ-Linear(x [N, Cin, G]) on the handle's device."""
+    if x.dim() != 3 or x.shape[1] != h.Cin or x.shape[2] != h.G:
+        raise ValueError(f"x must be [N, {h.Cin}, {h.G}], got {tuple(x.shape)}")
+    if x.device != h.device or x.dtype != h.io_dtype:
+        raise ValueError(f"x must be {h.io_dtype} on {h.device}")
+    if not x.is_contiguous():
+        raise ValueError("x must be contiguous")
+    N = x.shape[0]
+    if y is None:
+        y = torch.empty((N, h.Cout, h.G), dtype=h.io_dtype, device=h.device)
+    elif y.shape != (N, h.Cout, h.G) or y.dtype != h.io_dtype or y.device != h.device \
+            or not y.is_contiguous():
+        raise ValueError("y has the wrong shape, dtype, device or layout")
+    with torch.cuda.device(h.device):
+        _check(_lib.eqlin_forward(h.ptr, x.data_ptr(), y.data_ptr(), N, _stream_ptr(stream)),
+               "eqlin_forward")
+    return y
+
+
+def eqlin_destroy(h: Handle) -> None:
+    h.close()
+
+
+def eqlin_device_status(h: Handle) -> int:
+    v = ctypes.c_int()
+    with torch.cuda.device(h.device):
+        _check(_lib.eqlin_device_status(h.ptr, ctypes.byref(v)), "eqlin_device_status")
+    return int(v.value)
+
+
+def eqlin_copy_freq_weights(h: Handle) -> torch.Tensor:
+    """fp32 frequency-domain weights [G, Cin, Cout] (scaled; see include/eqlin.h)."""
+    out = torch.empty((h.G, h.Cin, h.Cout), dtype=torch.float32)
+    with torch.cuda.device(h.device):
+        dst = ctypes.cast(out.data_ptr(), ctypes.POINTER(ctypes.c_float))
+        _check(_lib.eqlin_copy_freq_weights(h.ptr, dst, out.numel()), "eqlin_copy_freq_weights")
+    return out

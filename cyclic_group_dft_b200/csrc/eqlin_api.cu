@@ -1,0 +1,476 @@
+// eqlin_api.cu -- host side of the C ABI declared in include/eqlin.h: argument
+// validation, kernel planning (shared-memory budget, ring depth), ownership of the
+// frequency-domain weights, TMA descriptor encoding and launches.
+#include "eqlin.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstdlib>
+#include <mutex>
+#include <new>
+#include <string>
+
+#include "eqlin_fwd_tc.cuh"
+#include "eqlin_layout.h"
+#include "eqlin_prep.cuh"
+
+using eqlin::TcParams;
+
+namespace {
+
+constexpr size_t kB200SmemOptin = 232448;   // 227 KB opt-in shared memory per CTA on sm_100
+constexpr size_t kSmemAlignSlack = 1024;    // the kernel rounds its smem base up to 1 KB
+constexpr size_t kSmemCtlBytes = 256;       // mbarriers + control block
+constexpr int kMaxStages = 8;
+constexpr int64_t kMaxChannels = 1 << 16;
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per bounded wait
+
+enum Path { kPathResident = 0, kPathStreamed = 1, kPathF32 = 2 };
+
+thread_local std::string g_last_error;
+
+int fail(int code, const std::string& msg) {
+    g_last_error = msg;
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+    return fail(EQLIN_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+struct Plan {
+    int path = kPathF32;
+    int nK = 0, rows = 0, n_oc = 0, BN = 0, stages = 0;
+    uint32_t w_region_bytes = 0, w_img_bytes = 0;
+    size_t smem_bytes = 0;
+    size_t img_alloc_bytes = 0;
+};
+
+template <int G>
+int plan_tc_g(int64_t Cout, int64_t Cin, size_t max_smem, Plan* pl) {
+    using S = eqlin::tc::Shape<G>;
+    pl->nK = static_cast<int>((Cin + eqlin::kChunkK - 1) / eqlin::kChunkK);
+    pl->n_oc = static_cast<int>((Cout + eqlin::kMmaM - 1) / eqlin::kMmaM);
+    pl->BN = S::BN;
+    const size_t fixed = kSmemAlignSlack + kSmemCtlBytes;
+    if (pl->n_oc == 1) {
+        // weights resident in shared memory for the whole kernel
+        const int rows = static_cast<int>((Cout + 7) / 8 * 8);
+        const size_t img = static_cast<size_t>(G) * pl->nK * rows * eqlin::kPlaneRowBytes;
+        // the A operand always reads 128 rows: keep the overrun of the last block inside
+        const size_t region = (img + static_cast<size_t>(eqlin::kMmaM - rows) * eqlin::kPlaneRowBytes +
+                               1023) / 1024 * 1024;
+        if (max_smem > fixed + region) {
+            const size_t stages = std::min<size_t>(kMaxStages, (max_smem - fixed - region) / S::XCHUNK_BYTES);
+            if (stages >= 2) {
+                pl->path = kPathResident;
+                pl->rows = rows;
+                pl->stages = static_cast<int>(stages);
+                pl->w_region_bytes = static_cast<uint32_t>(region);
+                pl->w_img_bytes = static_cast<uint32_t>(img);
+                pl->img_alloc_bytes = img;
+                pl->smem_bytes = fixed + region + stages * S::XCHUNK_BYTES;
+                return EQLIN_OK;
+            }
+        }
+    }
+    // weights streamed chunk by chunk next to each x chunk
+    const size_t stage = static_cast<size_t>(S::XCHUNK_BYTES) + S::WSTAGE_BYTES;
+    const size_t stages = max_smem > fixed ? std::min<size_t>(kMaxStages, (max_smem - fixed) / stage) : 0;
+    if (stages < 1) return fail(EQLIN_ERR_UNSUPPORTED, "shape does not fit in shared memory");
+    pl->path = kPathStreamed;
+    pl->rows = eqlin::kMmaM;
+    pl->stages = static_cast<int>(stages);
+    pl->w_region_bytes = 0;
+    pl->w_img_bytes = 0;
+    pl->img_alloc_bytes = static_cast<size_t>(pl->n_oc) * pl->nK * S::WSTAGE_BYTES;
+    pl->smem_bytes = fixed + stages * stage;
+    return EQLIN_OK;
+}
+
+int plan_for(int64_t Cout, int64_t Cin, int64_t G, int io_dtype, size_t max_smem, Plan* pl) {
+    if (io_dtype == EQLIN_F32) {
+        const size_t smem = static_cast<size_t>(eqlin::kF32Tokens) * G * Cin * sizeof(float);
+        if (smem > max_smem) return fail(EQLIN_ERR_UNSUPPORTED, "Cin*G too large for the fp32 path");
+        pl->path = kPathF32;
+        pl->BN = eqlin::kF32Tokens;
+        pl->smem_bytes = smem;
+        return EQLIN_OK;
+    }
+    switch (G) {
+        case 2: return plan_tc_g<2>(Cout, Cin, max_smem, pl);
+        case 4: return plan_tc_g<4>(Cout, Cin, max_smem, pl);
+        case 8: return plan_tc_g<8>(Cout, Cin, max_smem, pl);
+        case 16: return plan_tc_g<16>(Cout, Cin, max_smem, pl);
+        default: return fail(EQLIN_ERR_UNSUPPORTED, "G must be 2, 4, 8 or 16");
+    }
+}
+
+int check_shape_impl(int64_t Cout, int64_t Cin, int64_t G, int w_dtype, int io_dtype) {
+    if (w_dtype != EQLIN_F32 && w_dtype != EQLIN_BF16) return fail(EQLIN_ERR_INVALID_ARG, "unknown w_dtype");
+    if (io_dtype != EQLIN_F32 && io_dtype != EQLIN_BF16) return fail(EQLIN_ERR_INVALID_ARG, "unknown io_dtype");
+    if (Cout <= 0 || Cin <= 0 || G <= 0) return fail(EQLIN_ERR_INVALID_ARG, "sizes must be positive");
+    if (G != 2 && G != 4 && G != 8 && G != 16) return fail(EQLIN_ERR_UNSUPPORTED, "G must be 2, 4, 8 or 16");
+    if (Cout > kMaxChannels || Cin > kMaxChannels) return fail(EQLIN_ERR_UNSUPPORTED, "channel count above 65536");
+    if (io_dtype == EQLIN_BF16 && (Cin * G) % 8 != 0)
+        return fail(EQLIN_ERR_UNSUPPORTED, "bf16 I/O needs Cin*G to be a multiple of 8 (16-byte rows)");
+    return EQLIN_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+template <int G, bool STREAM>
+void* tc_kernel_ptr() {
+    return reinterpret_cast<void*>(&eqlin::eqlin_fwd_tc_kernel<G, STREAM>);
+}
+
+void* tc_kernel_for(int G, bool stream) {
+    switch (G) {
+        case 2: return stream ? tc_kernel_ptr<2, true>() : tc_kernel_ptr<2, false>();
+        case 4: return stream ? tc_kernel_ptr<4, true>() : tc_kernel_ptr<4, false>();
+        case 8: return stream ? tc_kernel_ptr<8, true>() : tc_kernel_ptr<8, false>();
+        case 16: return stream ? tc_kernel_ptr<16, true>() : tc_kernel_ptr<16, false>();
+        default: return nullptr;
+    }
+}
+
+void* f32_kernel_for(int G) {
+    switch (G) {
+        case 2: return reinterpret_cast<void*>(&eqlin::eqlin_fwd_f32_kernel<2>);
+        case 4: return reinterpret_cast<void*>(&eqlin::eqlin_fwd_f32_kernel<4>);
+        case 8: return reinterpret_cast<void*>(&eqlin::eqlin_fwd_f32_kernel<8>);
+        case 16: return reinterpret_cast<void*>(&eqlin::eqlin_fwd_f32_kernel<16>);
+        default: return nullptr;
+    }
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+template <int G>
+int box_elems() { return eqlin::tc::Shape<G>::BOX_ELEMS; }
+
+int tc_box_elems(int G) {
+    switch (G) {
+        case 2: return box_elems<2>();
+        case 4: return box_elems<4>();
+        case 8: return box_elems<8>();
+        default: return box_elems<16>();
+    }
+}
+
+}  // namespace
+
+struct eqlin_handle {
+    int device = 0;
+    int sm_count = 0;
+    int64_t Cout = 0, Cin = 0, G = 0;
+    int w_dtype = 0, io_dtype = 0;
+    Plan plan;
+    uint8_t* w_img = nullptr;
+    float* w_f32 = nullptr;
+    float* bias_f32 = nullptr;
+    int* status = nullptr;
+    bool has_bias = false;
+    bool sync_check = false;
+    unsigned long long timeout_ns = kDefaultTimeoutNs;
+};
+
+namespace {
+
+void free_handle(eqlin_handle* h) {
+    if (!h) return;
+    if (h->w_img) cudaFree(h->w_img);
+    if (h->w_f32) cudaFree(h->w_f32);
+    if (h->bias_f32) cudaFree(h->bias_f32);
+    if (h->status) cudaFree(h->status);
+    delete h;
+}
+
+int launch_prep(eqlin_handle* h, const void* w, const void* bias, cudaStream_t st) {
+    const int64_t pairs = h->Cout * h->Cin;
+    const int threads = 256;
+    const unsigned blocks = static_cast<unsigned>((pairs + threads - 1) / threads);
+    const int Cout = static_cast<int>(h->Cout), Cin = static_cast<int>(h->Cin), G = static_cast<int>(h->G);
+    if (h->w_dtype == EQLIN_F32) {
+        eqlin::eqlin_prep_freq_kernel<float><<<blocks, threads, 0, st>>>(
+            static_cast<const float*>(w), static_cast<const float*>(bias), Cout, Cin, G, h->w_f32, h->bias_f32);
+    } else {
+        eqlin::eqlin_prep_freq_kernel<__nv_bfloat16><<<blocks, threads, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(w), static_cast<const __nv_bfloat16*>(bias), Cout, Cin, G,
+            h->w_f32, h->bias_f32);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "weight transform launch");
+    if (h->w_img) {
+        const size_t n = h->plan.img_alloc_bytes / 2;
+        const unsigned b2 = static_cast<unsigned>((n + threads - 1) / threads);
+        eqlin::eqlin_prep_image_kernel<<<b2, threads, 0, st>>>(h->w_f32, Cout, Cin, G, h->plan.nK, h->plan.rows,
+                                                                n, h->w_img);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "weight image launch");
+    }
+    e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "weight transform");
+    return EQLIN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int eqlin_check_shape(int64_t Cout, int64_t Cin, int64_t G, int w_dtype, int io_dtype) {
+    int s = check_shape_impl(Cout, Cin, G, w_dtype, io_dtype);
+    if (s != EQLIN_OK) return s;
+    Plan pl;
+    return plan_for(Cout, Cin, G, io_dtype, kB200SmemOptin, &pl);
+}
+
+int eqlin_prepare_weights(const void* w, const void* bias, int64_t Cout, int64_t Cin, int64_t G, int w_dtype,
+                          int io_dtype, void* stream, eqlin_handle** out) {
+    if (!out) return fail(EQLIN_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    if (!w) return fail(EQLIN_ERR_INVALID_ARG, "w is NULL");
+    int s = check_shape_impl(Cout, Cin, G, w_dtype, io_dtype);
+    if (s != EQLIN_OK) return s;
+    const size_t welt = w_dtype == EQLIN_F32 ? 4 : 2;
+    if (!aligned(w, welt) || (bias && !aligned(bias, welt)))
+        return fail(EQLIN_ERR_MISALIGNED, "w / bias not aligned to their element size");
+
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    int major = 0, minor = 0, sms = 0, optin = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
+        return cuda_fail(e, "device query");
+    if (major != 10 || minor != 0)
+        return fail(EQLIN_ERR_UNSUPPORTED, "needs a compute capability 10.0 (sm_100a) device");
+
+    Plan plan;
+    s = plan_for(Cout, Cin, G, io_dtype, static_cast<size_t>(optin), &plan);
+    if (s != EQLIN_OK) return s;
+
+    eqlin_handle* h = new (std::nothrow) eqlin_handle();
+    if (!h) return fail(EQLIN_ERR_OOM, "host allocation");
+    h->device = dev;
+    h->sm_count = sms;
+    h->Cout = Cout;
+    h->Cin = Cin;
+    h->G = G;
+    h->w_dtype = w_dtype;
+    h->io_dtype = io_dtype;
+    h->plan = plan;
+    h->has_bias = bias != nullptr;
+    const char* sc = std::getenv("EQLIN_SYNC_CHECK");
+    h->sync_check = sc && sc[0] == '1';
+    if (const char* t = std::getenv("EQLIN_WAIT_TIMEOUT_MS")) {
+        const long long ms = std::atoll(t);
+        if (ms > 0) h->timeout_ns = static_cast<unsigned long long>(ms) * 1000000ull;
+    }
+
+    const size_t wf_bytes = static_cast<size_t>(G) * Cin * Cout * sizeof(float);
+    if (cudaMalloc(&h->w_f32, wf_bytes) != cudaSuccess ||
+        cudaMalloc(&h->bias_f32, static_cast<size_t>(Cout) * sizeof(float)) != cudaSuccess ||
+        cudaMalloc(&h->status, 256) != cudaSuccess ||
+        (plan.img_alloc_bytes && cudaMalloc(&h->w_img, plan.img_alloc_bytes) != cudaSuccess)) {
+        cudaGetLastError();
+        free_handle(h);
+        return fail(EQLIN_ERR_OOM, "device allocation for the transformed weights");
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((e = cudaMemsetAsync(h->status, 0, 256, st)) != cudaSuccess) {
+        free_handle(h);
+        return cuda_fail(e, "status init");
+    }
+    s = launch_prep(h, w, bias, st);
+    if (s != EQLIN_OK) {
+        free_handle(h);
+        return s;
+    }
+    void* k = plan.path == kPathF32 ? f32_kernel_for(static_cast<int>(G))
+                                    : tc_kernel_for(static_cast<int>(G), plan.path == kPathStreamed);
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(plan.smem_bytes));
+    if (e != cudaSuccess) {
+        free_handle(h);
+        return cuda_fail(e, "cudaFuncSetAttribute");
+    }
+    *out = h;
+    return EQLIN_OK;
+}
+
+int eqlin_forward(const eqlin_handle* h, const void* x, void* y, int64_t N, void* stream) {
+    if (!h) return fail(EQLIN_ERR_INVALID_ARG, "handle is NULL");
+    if (N < 0) return fail(EQLIN_ERR_INVALID_ARG, "N < 0");
+    if (N == 0) return EQLIN_OK;
+    if (!x || !y) return fail(EQLIN_ERR_INVALID_ARG, "x or y is NULL");
+    if (N >= (int64_t(1) << 31)) return fail(EQLIN_ERR_UNSUPPORTED, "N must be below 2^31");
+    if (!aligned(x, 16) || !aligned(y, 16)) return fail(EQLIN_ERR_MISALIGNED, "x and y must be 16-byte aligned");
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev != h->device) return fail(EQLIN_ERR_INVALID_ARG, "current device differs from the handle's device");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const Plan& pl = h->plan;
+    const int G = static_cast<int>(h->G);
+
+    if (pl.path == kPathF32) {
+        dim3 grid(static_cast<unsigned>((N + eqlin::kF32Tokens - 1) / eqlin::kF32Tokens),
+                  static_cast<unsigned>((h->Cout + 31) / 32));
+        void* args_x = const_cast<void*>(x);
+        const float* xf = static_cast<const float*>(args_x);
+        float* yf = static_cast<float*>(y);
+        const long long n = N;
+        const int Cin = static_cast<int>(h->Cin), Cout = static_cast<int>(h->Cout);
+        switch (G) {
+            case 2: eqlin::eqlin_fwd_f32_kernel<2><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, h->w_f32, h->bias_f32, yf, n, Cin, Cout); break;
+            case 4: eqlin::eqlin_fwd_f32_kernel<4><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, h->w_f32, h->bias_f32, yf, n, Cin, Cout); break;
+            case 8: eqlin::eqlin_fwd_f32_kernel<8><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, h->w_f32, h->bias_f32, yf, n, Cin, Cout); break;
+            default: eqlin::eqlin_fwd_f32_kernel<16><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, h->w_f32, h->bias_f32, yf, n, Cin, Cout); break;
+        }
+    } else {
+        auto encode = tensor_map_encoder();
+        if (!encode) return fail(EQLIN_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+        const int box = tc_box_elems(G);
+        CUtensorMap map;
+        cuuint64_t dims[2] = {static_cast<cuuint64_t>(h->Cin * G), static_cast<cuuint64_t>(N)};
+        cuuint64_t strides[1] = {static_cast<cuuint64_t>(h->Cin * G * 2)};
+        cuuint32_t boxdim[2] = {static_cast<cuuint32_t>(box), static_cast<cuuint32_t>(pl.BN)};
+        cuuint32_t estr[2] = {1, 1};
+        CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, boxdim,
+                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return fail(EQLIN_ERR_CUDA, "cuTensorMapEncodeTiled failed for x");
+        TcParams p;
+        p.w_img = h->w_img;
+        p.bias = h->has_bias ? h->bias_f32 : nullptr;
+        p.y = static_cast<__nv_bfloat16*>(y);
+        p.status = h->status;
+        p.N = N;
+        p.Cout = static_cast<int>(h->Cout);
+        p.nK = pl.nK;
+        p.rows = pl.rows;
+        p.n_oc = pl.n_oc;
+        const long long n_tiles = (N + pl.BN - 1) / pl.BN;
+        p.n_work = static_cast<int>(n_tiles * pl.n_oc);
+        p.stages = pl.stages;
+        p.w_region_bytes = pl.w_region_bytes;
+        p.w_img_bytes = pl.w_img_bytes;
+        p.timeout_ns = h->timeout_ns;
+        const unsigned grid = static_cast<unsigned>(std::min<long long>(p.n_work, h->sm_count));
+        const bool streamed = pl.path == kPathStreamed;
+        switch (G) {
+#define EQLIN_LAUNCH(GG)                                                                                     \
+    case GG:                                                                                                 \
+        if (streamed)                                                                                        \
+            eqlin::eqlin_fwd_tc_kernel<GG, true><<<grid, eqlin::tc::kThreads, pl.smem_bytes, st>>>(map, p);  \
+        else                                                                                                 \
+            eqlin::eqlin_fwd_tc_kernel<GG, false><<<grid, eqlin::tc::kThreads, pl.smem_bytes, st>>>(map, p); \
+        break;
+            EQLIN_LAUNCH(2)
+            EQLIN_LAUNCH(4)
+            EQLIN_LAUNCH(8)
+            EQLIN_LAUNCH(16)
+#undef EQLIN_LAUNCH
+            default: return fail(EQLIN_ERR_UNSUPPORTED, "G");
+        }
+    }
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "forward launch");
+    if (h->sync_check) {
+        int dst = 0;
+        e = cudaStreamSynchronize(st);
+        if (e != cudaSuccess) return cuda_fail(e, "forward (EQLIN_SYNC_CHECK)");
+        e = cudaMemcpy(&dst, h->status, sizeof(int), cudaMemcpyDeviceToHost);
+        if (e != cudaSuccess) return cuda_fail(e, "status read");
+        if (dst != 0) return fail(dst, "device reported an error (status word)");
+    }
+    return EQLIN_OK;
+}
+
+int eqlin_destroy(eqlin_handle* h) {
+    if (!h) return EQLIN_OK;
+    free_handle(h);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFree");
+    return EQLIN_OK;
+}
+
+int eqlin_device_status(eqlin_handle* h, int* status_out) {
+    if (!h || !status_out) return fail(EQLIN_ERR_INVALID_ARG, "NULL argument");
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    int v = 0;
+    if ((e = cudaMemcpy(&v, h->status, sizeof(int), cudaMemcpyDeviceToHost)) != cudaSuccess)
+        return cuda_fail(e, "status read");
+    if ((e = cudaMemset(h->status, 0, sizeof(int))) != cudaSuccess) return cuda_fail(e, "status clear");
+    *status_out = v;
+    return EQLIN_OK;
+}
+
+int eqlin_get_attr(const eqlin_handle* h, int attr, int64_t* value) {
+    if (!h || !value) return fail(EQLIN_ERR_INVALID_ARG, "NULL argument");
+    const Plan& pl = h->plan;
+    switch (attr) {
+        case EQLIN_ATTR_G: *value = h->G; break;
+        case EQLIN_ATTR_CIN: *value = h->Cin; break;
+        case EQLIN_ATTR_COUT: *value = h->Cout; break;
+        case EQLIN_ATTR_IO_DTYPE: *value = h->io_dtype; break;
+        case EQLIN_ATTR_PATH: *value = pl.path; break;
+        case EQLIN_ATTR_TOKENS_PER_TILE: *value = pl.BN; break;
+        case EQLIN_ATTR_STAGES: *value = pl.stages; break;
+        case EQLIN_ATTR_SMEM_BYTES: *value = static_cast<int64_t>(pl.smem_bytes); break;
+        case EQLIN_ATTR_MAX_GRID: *value = pl.path == kPathF32 ? -1 : h->sm_count; break;
+        case EQLIN_ATTR_WEIGHT_BYTES:
+            *value = pl.path == kPathF32 ? static_cast<int64_t>(h->G * h->Cin * h->Cout * 4)
+                                         : static_cast<int64_t>(pl.img_alloc_bytes);
+            break;
+        default: return fail(EQLIN_ERR_INVALID_ARG, "unknown attribute");
+    }
+    return EQLIN_OK;
+}
+
+int eqlin_copy_freq_weights(const eqlin_handle* h, float* dst, int64_t count) {
+    if (!h || !dst) return fail(EQLIN_ERR_INVALID_ARG, "NULL argument");
+    const int64_t need = h->G * h->Cin * h->Cout;
+    if (count < need) return fail(EQLIN_ERR_INVALID_ARG, "destination too small");
+    cudaError_t e = cudaMemcpy(dst, h->w_f32, static_cast<size_t>(need) * sizeof(float), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "copy of frequency-domain weights");
+    return EQLIN_OK;
+}
+
+const char* eqlin_status_string(int status) {
+    switch (status) {
+        case EQLIN_OK: return "ok";
+        case EQLIN_ERR_INVALID_ARG: return "invalid argument";
+        case EQLIN_ERR_UNSUPPORTED: return "unsupported";
+        case EQLIN_ERR_MISALIGNED: return "misaligned pointer";
+        case EQLIN_ERR_CUDA: return "CUDA error";
+        case EQLIN_ERR_OOM: return "out of memory";
+        case EQLIN_ERR_TIMEOUT: return "device wait timed out";
+        default: return "unknown status";
+    }
+}
+
+const char* eqlin_last_error(void) { return g_last_error.c_str(); }
+
+int eqlin_version(void) { return 100; }
+
+}  // extern "C"

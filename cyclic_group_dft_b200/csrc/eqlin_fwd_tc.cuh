@@ -1,0 +1,451 @@
+// eqlin_fwd_tc.cuh -- fused EQ-Linear forward for bf16 I/O on sm_100a.
+//
+// Operation (page "Flash EQ-Linear: Accelerating Equivariant Linear Layers via
+// Group-wise Discrete Fourier Transform", sections "Percepcion Central" and
+// "Enfoque Algoritmico"):
+//     y[n,o,g] = bias[o] + sum_{i,h} w[o,i,(g-h) mod G] x[n,i,h]
+// computed as  X^ = rDFT_G(x)  ->  Y^_k = W^_k X^_k  (k = 0..G/2)  ->  y = irDFT_G(Y^) + bias,
+// all in one persistent kernel; nothing is written to global memory between the steps
+// (section "Implementacion": fused dataflow, Fourier fragments kept on chip).
+//
+// Per CTA (one per SM, persistent over work items = (token tile, 128-row output chunk)):
+//   warp 8     TMA producer: x chunks [BN tokens x 32 channels x G] into a smem ring
+//              (plus the weight chunk when the weights are streamed).
+//   warps 4-7  DFT: read a landed x chunk, real DFT over G in fp32 registers, write the
+//              G frequency planes [BN x 32] bf16 back IN PLACE in the UMMA K-major
+//              SWIZZLE_64B layout (the x chunk and its spectrum have the same size).
+//   warp 9     MMA issuer (one thread) + TMEM owner: per chunk and frequency,
+//              tcgen05.mma with A = W^ plane [128 out-rows x 32], B = X^ plane [BN x 32],
+//              D in TMEM (lane = output channel, column = token).  Complex frequencies
+//              use four real products; the -Im(W)Im(X) term uses the descriptor's
+//              negate-A bit, so only Re and Im of W^ are stored.
+//   warps 0-3  epilogue: tcgen05.ld of all G planes of a token group, inverse real DFT
+//              (1/G and 2/G are folded into W^), + bias, round to bf16 and store
+//              y[n, o, 0..G-1] directly: a warp writes 32 consecutive o -> one
+//              contiguous run of 32*G*2 bytes per token.
+// All waits are bounded (globaltimer); on expiry the kernel records EQLIN_ERR_TIMEOUT
+// in the status word, every role leaves its loop, in-flight copies and MMAs are
+// drained with bounded waits, and TMEM is freed before exit.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "eqlin_layout.h"
+#include "group_dft.cuh"
+#include "sm100_ptx.cuh"
+
+namespace eqlin {
+
+struct TcParams {
+    const uint8_t* w_img;   // frequency-domain weight image (layout: eqlin_layout.h)
+    const float* bias;      // [Cout] fp32, or nullptr
+    __nv_bfloat16* y;       // [N, Cout, G]
+    int* status;            // device status word (first error wins)
+    long long N;
+    int Cout;
+    int nK;                 // 32-channel chunks along Cin
+    int rows;               // weight rows per sub-block (resident: Cout rounded to 8; streamed: 128)
+    int n_oc;               // 128-row output chunks
+    int n_work;             // n_tiles * n_oc
+    int stages;             // smem ring depth
+    uint32_t w_region_bytes;  // smem reserved for resident weights (0 when streamed)
+    uint32_t w_img_bytes;     // bytes of the resident image to copy
+    unsigned long long timeout_ns;
+};
+
+namespace tc {
+
+constexpr int kThreads = 320;
+constexpr int kWarpProducer = 8;
+constexpr int kWarpMma = 9;
+constexpr int kBarDft = 1;   // named barrier ids (0 is __syncthreads)
+constexpr int kBarEpi = 2;
+
+template <int G>
+struct Shape {
+    static constexpr int BN = (512 / G) < 128 ? (512 / G) : 128;    // tokens per tile (MMA N)
+    static constexpr int PLANE_BYTES = BN * kPlaneRowBytes;          // one frequency plane
+    static constexpr int XCHUNK_BYTES = G * PLANE_BYTES;             // == BN * 32 * G * 2
+    static constexpr int XROW_ELEMS = kChunkK * G;                   // one token row of a chunk
+    static constexpr int BOX_ELEMS = XROW_ELEMS < 256 ? XROW_ELEMS : 256;
+    static constexpr int NBOX = XROW_ELEMS / BOX_ELEMS;
+    static constexpr int WSTAGE_BYTES = G * kMmaM * kPlaneRowBytes;  // streamed weight chunk
+    static constexpr int TMEM_COLS = (G * BN <= 256) ? 256 : 512;
+    static constexpr int TG = (64 / G) < BN ? (64 / G) : BN;         // tokens per epilogue group
+    static_assert(XCHUNK_BYTES % 1024 == 0, "stage alignment");
+    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N");
+    static_assert(G * BN <= TMEM_COLS, "TMEM columns");
+};
+
+struct Ctl {
+    volatile int abort;
+    uint32_t tmem_base;
+};
+
+// Bounded mbarrier wait.  Returns false (after flagging) on timeout or abort.
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, Ctl* ctl,
+                                             int* status, unsigned long long timeout_ns) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = ptx::globaltimer_ns();
+    for (uint32_t spin = 1;; ++spin) {
+        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if ((spin & 63u) == 0) {
+            if (ctl->abort) return false;
+            if (ptx::globaltimer_ns() - t0 > timeout_ns) {
+                ctl->abort = 1;
+                atomicCAS(status, 0, kDeviceErrTimeout);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// ---------------------------------------------------------------- DFT role
+// 128 threads.  Unit = one token row x two adjacent channels (2*G bf16).
+// Lanes 0-15 take row r, lanes 16-31 row r+1; lane&15 selects the channel pair.
+template <int G>
+__device__ __forceinline__ void dft_chunk(uint8_t* xs, int dft_tid) {
+    using S = Shape<G>;
+    constexpr int WORDS = G;                         // 32-bit words per unit (2 ch x G x 2 B / 4)
+    constexpr int STEPS = S::BN / 8;                 // 2 rows per step, 4 warps
+    const int warp = dft_tid >> 5, lane = dft_tid & 31;
+    const int pair = lane & 15;
+    const int row0 = warp * (S::BN / 4) + (lane >> 4);
+    // element offset of the unit inside a token row, and the TMA box it lives in
+    constexpr int UNIT_ELEMS = 2 * G;
+    const int e = pair * UNIT_ELEMS;
+    const int box = e / S::BOX_ELEMS;
+    const int e_in = e % S::BOX_ELEMS;
+    const uint8_t* src0 = xs + box * (S::BN * S::BOX_ELEMS * 2) + e_in * 2;
+
+    uint32_t w[STEPS][WORDS];
+#pragma unroll
+    for (int s = 0; s < STEPS; ++s) {
+        const int r = row0 + 2 * s;
+        const uint8_t* src = src0 + r * (S::BOX_ELEMS * 2);
+        if constexpr (WORDS == 2) {
+            const uint2 v = *reinterpret_cast<const uint2*>(src);
+            w[s][0] = v.x;
+            w[s][1] = v.y;
+        } else {
+#pragma unroll
+            for (int c = 0; c < WORDS / 4; ++c) {
+                const uint4 v = *reinterpret_cast<const uint4*>(src + 16 * c);
+                w[s][4 * c + 0] = v.x;
+                w[s][4 * c + 1] = v.y;
+                w[s][4 * c + 2] = v.z;
+                w[s][4 * c + 3] = v.w;
+            }
+        }
+    }
+    // every read of this chunk happens before any in-place write
+    ptx::named_bar_sync(kBarDft, 128);
+
+    const int chunk = pair >> 2;              // 16-B chunk of the 64-B plane row
+    const int in_chunk = (pair & 3) * 4;      // byte inside it
+#pragma unroll
+    for (int s = 0; s < STEPS; ++s) {
+        const int r = row0 + 2 * s;
+        float xa[G], xb[G];
+#pragma unroll
+        for (int h = 0; h < G / 2; ++h) {
+            const uint32_t ua = w[s][h], ub = w[s][G / 2 + h];
+            xa[2 * h] = __uint_as_float(ua << 16);
+            xa[2 * h + 1] = __uint_as_float(ua & 0xFFFF0000u);
+            xb[2 * h] = __uint_as_float(ub << 16);
+            xb[2 * h + 1] = __uint_as_float(ub & 0xFFFF0000u);
+        }
+        float pa[G], pb[G];
+        rdft_planes<G>(xa, pa);
+        rdft_planes<G>(xb, pb);
+        const int phys = (chunk ^ ((r >> 1) & 3)) * 16 + in_chunk;   // SWIZZLE_64B
+        uint8_t* dst = xs + r * kPlaneRowBytes + phys;
+#pragma unroll
+        for (int p = 0; p < G; ++p) {
+            *reinterpret_cast<uint32_t*>(dst + p * S::PLANE_BYTES) = pack_bf16x2(pa[p], pb[p]);
+        }
+    }
+}
+
+// ------------------------------------------------------------ epilogue role
+template <int G>
+__device__ __forceinline__ void epilogue_tile(const TcParams& p, uint32_t tmem_base, int q,
+                                              int lane, long long n0, int oc) {
+    using S = Shape<G>;
+    constexpr int TG = S::TG;
+    const int o_local = q * 32 + lane;
+    const int o = oc * kMmaM + o_local;
+    const bool valid_o = o < p.Cout;
+    const float b = (p.bias != nullptr && valid_o) ? p.bias[o] : 0.0f;
+    const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+    for (int j = 0; j < S::BN / TG; ++j) {
+        uint32_t r[G][TG];
+#pragma unroll
+        for (int pl = 0; pl < G; ++pl) ptx::tmem_ld_32x32b<TG>(lane_addr + pl * S::BN + j * TG, r[pl]);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int t = 0; t < TG; ++t) {
+            const long long n = n0 + j * TG + t;
+            float z[G], yv[G];
+#pragma unroll
+            for (int pl = 0; pl < G; ++pl) z[pl] = __uint_as_float(r[pl][t]);
+            z[0] += b;  // the DC term appears with weight 1 in every output
+            RealIdft<G>::run(z, yv);
+            if (valid_o && n < p.N) {
+                __nv_bfloat16* dst = p.y + (n * p.Cout + o) * G;
+                if constexpr (G == 2) {
+                    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(yv[0], yv[1]);
+                } else if constexpr (G == 4) {
+                    *reinterpret_cast<uint2*>(dst) =
+                        make_uint2(pack_bf16x2(yv[0], yv[1]), pack_bf16x2(yv[2], yv[3]));
+                } else {
+#pragma unroll
+                    for (int c = 0; c < G / 8; ++c) {
+                        *reinterpret_cast<uint4*>(dst + 8 * c) = make_uint4(
+                            pack_bf16x2(yv[8 * c + 0], yv[8 * c + 1]),
+                            pack_bf16x2(yv[8 * c + 2], yv[8 * c + 3]),
+                            pack_bf16x2(yv[8 * c + 4], yv[8 * c + 5]),
+                            pack_bf16x2(yv[8 * c + 6], yv[8 * c + 7]));
+                    }
+                }
+            }
+        }
+    }
+}
+
+}  // namespace tc
+
+template <int G, bool STREAM_W>
+__global__ void __launch_bounds__(tc::kThreads, 1)
+    eqlin_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const TcParams p) {
+    using S = tc::Shape<G>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+
+    constexpr uint32_t STAGE_BYTES = S::XCHUNK_BYTES + (STREAM_W ? S::WSTAGE_BYTES : 0);
+    constexpr uint32_t STAGE_TX = STAGE_BYTES;   // every byte of a stage arrives by copy
+    const int NS = p.stages;
+    uint8_t* stage0 = smem + p.w_region_bytes;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(stage0 + static_cast<size_t>(NS) * STAGE_BYTES);
+    tc::Ctl* ctl = reinterpret_cast<tc::Ctl*>(bars + 3 * NS + 4);
+
+    const uint32_t s_w = ptx::smem_u32(smem);
+    const uint32_t s_stage0 = ptx::smem_u32(stage0);
+    auto bar_full = [&](int s) { return ptx::smem_u32(bars + s); };
+    auto bar_xhat = [&](int s) { return ptx::smem_u32(bars + NS + s); };
+    auto bar_empty = [&](int s) { return ptx::smem_u32(bars + 2 * NS + s); };
+    const uint32_t bar_acc_full = ptx::smem_u32(bars + 3 * NS + 0);
+    const uint32_t bar_acc_empty = ptx::smem_u32(bars + 3 * NS + 1);
+    const uint32_t bar_w_full = ptx::smem_u32(bars + 3 * NS + 2);
+    const uint32_t bar_drain = ptx::smem_u32(bars + 3 * NS + 3);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; ++s) {
+            ptx::mbar_init(bar_full(s), 1);
+            ptx::mbar_init(bar_xhat(s), 128);
+            ptx::mbar_init(bar_empty(s), 1);
+        }
+        ptx::mbar_init(bar_acc_full, 1);
+        ptx::mbar_init(bar_acc_empty, 128);
+        ptx::mbar_init(bar_w_full, 1);
+        ptx::mbar_init(bar_drain, 1);
+        ctl->abort = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == tc::kWarpMma) {
+        ptx::tmem_alloc(ptx::smem_u32(&ctl->tmem_base), S::TMEM_COLS);
+        ptx::tmem_relinquish();
+    }
+    if (warp == tc::kWarpProducer && lane == 0) ptx::prefetch_tmap(&tmap_x);
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = ctl->tmem_base;
+
+    if (warp == tc::kWarpProducer) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            if constexpr (!STREAM_W) {
+                ptx::mbar_arrive_expect_tx(bar_w_full, p.w_img_bytes);
+                for (uint32_t off = 0; off < p.w_img_bytes; off += 32768u) {
+                    const uint32_t n = min(32768u, p.w_img_bytes - off);
+                    ptx::bulk_load(s_w + off, p.w_img + off, n, bar_w_full);
+                }
+            }
+            int stage = 0;
+            uint32_t phase = 0;
+            long long issued = 0;
+            bool ok = true;
+            for (int wk = blockIdx.x; ok && wk < p.n_work; wk += gridDim.x) {
+                const int tile = wk / p.n_oc, oc = wk % p.n_oc;
+                const int n0 = tile * S::BN;
+                for (int c = 0; c < p.nK; ++c) {
+                    if (!tc::wait_bounded(bar_empty(stage), phase ^ 1u, ctl, p.status, p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t dst = s_stage0 + stage * STAGE_BYTES;
+                    ptx::mbar_arrive_expect_tx(bar_full(stage), STAGE_TX);
+#pragma unroll
+                    for (int bx = 0; bx < S::NBOX; ++bx) {
+                        ptx::tma_load_2d(dst + bx * (S::BN * S::BOX_ELEMS * 2), &tmap_x,
+                                         c * S::XROW_ELEMS + bx * S::BOX_ELEMS, n0, bar_full(stage));
+                    }
+                    if constexpr (STREAM_W) {
+                        ptx::bulk_load(dst + S::XCHUNK_BYTES,
+                                       p.w_img + static_cast<size_t>(oc * p.nK + c) * S::WSTAGE_BYTES,
+                                       S::WSTAGE_BYTES, bar_full(stage));
+                    }
+                    ++issued;
+                    if (++stage == NS) { stage = 0; phase ^= 1u; }
+                }
+            }
+            // drain: every copy this thread started must land before the CTA exits
+            for (int s = 0; s < NS; ++s) {
+                const long long times = issued > s ? (issued - s + NS - 1) / NS : 0;
+                if (times > 0) {
+                    const uint32_t par = static_cast<uint32_t>((times - 1) & 1);
+                    // bounded, and deliberately blind to the abort flag: a copy in
+                    // flight must land before its shared memory is released
+                    const uint64_t t0 = ptx::globaltimer_ns();
+                    while (!ptx::mbar_try_wait(bar_full(s), par)) {
+                        if (ptx::globaltimer_ns() - t0 > p.timeout_ns) {
+                            atomicCAS(p.status, 0, kDeviceErrTimeout);
+                            break;
+                        }
+                    }
+                }
+            }
+            if constexpr (!STREAM_W) {
+                const uint64_t t0 = ptx::globaltimer_ns();
+                while (!ptx::mbar_try_wait(bar_w_full, 0)) {
+                    if (ptx::globaltimer_ns() - t0 > p.timeout_ns) {
+                        atomicCAS(p.status, 0, kDeviceErrTimeout);
+                        break;
+                    }
+                }
+            }
+        }
+    } else if (warp == tc::kWarpMma) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            bool ok = true;
+            if constexpr (!STREAM_W) ok = tc::wait_bounded(bar_w_full, 0, ctl, p.status, p.timeout_ns);
+            constexpr uint32_t ID = idesc_bf16_f32(kMmaM, S::BN, false);
+            constexpr uint32_t ID_NEG = idesc_bf16_f32(kMmaM, S::BN, true);
+            int stage = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            for (int wk = blockIdx.x; ok && wk < p.n_work; wk += gridDim.x) {
+                if (!tc::wait_bounded(bar_acc_empty, acc_phase ^ 1u, ctl, p.status, p.timeout_ns)) {
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+                for (int c = 0; c < p.nK; ++c) {
+                    if (!tc::wait_bounded(bar_xhat(stage), phase, ctl, p.status, p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint32_t xb = s_stage0 + stage * STAGE_BYTES;
+                    uint32_t wb, wsub;
+                    if constexpr (STREAM_W) {
+                        wb = xb + S::XCHUNK_BYTES;
+                        wsub = kMmaM * kPlaneRowBytes;
+                    } else {
+                        wsub = static_cast<uint32_t>(p.rows) * kPlaneRowBytes;
+                        wb = s_w + static_cast<uint32_t>(c * G) * wsub;
+                    }
+#pragma unroll
+                    for (int ks = 0; ks < kChunkK / 16; ++ks) {
+                        const uint32_t acc0 = (c > 0 || ks > 0) ? 1u : 0u;
+                        auto A = [&](int pl) { return ptx::sdesc_kmajor_sw64(wb + pl * wsub + ks * 32); };
+                        auto B = [&](int pl) {
+                            return ptx::sdesc_kmajor_sw64(xb + pl * S::PLANE_BYTES + ks * 32);
+                        };
+                        auto D = [&](int pl) { return tmem_base + static_cast<uint32_t>(pl * S::BN); };
+                        // real frequencies k = 0 and k = G/2
+                        ptx::umma_f16(D(0), A(0), B(0), ID, acc0);
+                        ptx::umma_f16(D(1), A(1), B(1), ID, acc0);
+                        // complex frequencies: (Wr + i Wi)(Xr + i Xi)
+#pragma unroll
+                        for (int k = 1; k < G / 2; ++k) {
+                            const int pr = 2 * k, pi = 2 * k + 1;
+                            ptx::umma_f16(D(pr), A(pr), B(pr), ID, acc0);      // + Wr Xr
+                            ptx::umma_f16(D(pr), A(pi), B(pi), ID_NEG, 1u);    // - Wi Xi
+                            ptx::umma_f16(D(pi), A(pi), B(pr), ID, acc0);      // + Wi Xr
+                            ptx::umma_f16(D(pi), A(pr), B(pi), ID, 1u);        // + Wr Xi
+                        }
+                    }
+                    ptx::umma_commit(bar_empty(stage));   // stage reusable once these finish
+                    if (++stage == NS) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                ptx::umma_commit(bar_acc_full);
+                acc_phase ^= 1u;
+            }
+            // drain: all MMAs done before TMEM is released
+            ptx::umma_commit(bar_drain);
+            const uint64_t t0 = ptx::globaltimer_ns();
+            while (!ptx::mbar_try_wait(bar_drain, 0)) {
+                if (ptx::globaltimer_ns() - t0 > p.timeout_ns) {
+                    atomicCAS(p.status, 0, kDeviceErrTimeout);
+                    break;
+                }
+            }
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ DFT warps
+        const int dft_tid = threadIdx.x - 128;
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int wk = blockIdx.x; wk < p.n_work; wk += gridDim.x) {
+            bool ok = true;
+            for (int c = 0; c < p.nK; ++c) {
+                const bool got = tc::wait_bounded(bar_full(stage), phase, ctl, p.status, p.timeout_ns);
+                if (!ptx::named_bar_and(tc::kBarDft, 128, got)) {
+                    ok = false;
+                    break;
+                }
+                tc::dft_chunk<G>(stage0 + static_cast<size_t>(stage) * STAGE_BYTES, dft_tid);
+                ptx::fence_proxy_async_smem();
+                ptx::mbar_arrive(bar_xhat(stage));
+                if (++stage == NS) { stage = 0; phase ^= 1u; }
+            }
+            if (!ok) break;
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue warps
+        uint32_t acc_phase = 0;
+        for (int wk = blockIdx.x; wk < p.n_work; wk += gridDim.x) {
+            const bool got = tc::wait_bounded(bar_acc_full, acc_phase, ctl, p.status, p.timeout_ns);
+            if (!ptx::named_bar_and(tc::kBarEpi, 128, got)) break;
+            ptx::tc_fence_after();
+            const int tile = wk / p.n_oc, oc = wk % p.n_oc;
+            tc::epilogue_tile<G>(p, tmem_base, warp, lane, static_cast<long long>(tile) * S::BN, oc);
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(bar_acc_empty);
+            acc_phase ^= 1u;
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == tc::kWarpMma) {
+        __syncwarp();
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem_base, S::TMEM_COLS);
+    }
+}
+
+}  // namespace eqlin

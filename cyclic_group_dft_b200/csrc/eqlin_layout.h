@@ -1,0 +1,41 @@
+// eqlin_layout.h -- data layout of the frequency-domain weights shared by the
+// weight pre-transform kernel (writer) and the fused forward kernels (readers).
+//
+// Frequency components ("planes") of a real length-G signal, G even:
+//   plane 0 = Re X_0,  plane 1 = Re X_{G/2},  plane 2k = Re X_k,  plane 2k+1 = Im X_k
+// for 0 < k < G/2, with X_k = sum_m v_m exp(-2 pi i m k / G).  The stored weight
+// planes carry the inverse-DFT scale: 1/G on planes 0 and 1, 2/G on the complex
+// planes (the conjugate partner k' = G-k is folded into the factor 2).
+//
+// fp32 planes (always built; used by the fp32 path and for inspection):
+//   w_f32[p][i][o], p < G, i < Cin, o < Cout  (output channel fastest)
+//
+// bf16 tensor-core image (bf16 I/O only): the exact shared-memory image the UMMA
+// A operand reads, so a plain bulk copy stages it:
+//   [oc][c][p][r][32]  with oc < n_oc (128-row output chunks), c < nK (32-channel
+//   chunks of Cin, zero padded), p < G, r < rows (output rows of the chunk, zero
+//   padded), 32 bf16 = one 64-byte row, K-major, SWIZZLE_64B: the 16-byte piece j
+//   of row r is stored at piece j ^ ((r >> 1) & 3).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+namespace eqlin {
+
+constexpr int kChunkK = 32;          // input channels per K chunk
+constexpr int kPlaneRowBytes = 64;   // one K chunk of one row in bf16
+constexpr int kMmaM = 128;           // UMMA M (output rows per chunk)
+
+// device status word values (mirrors EQLIN_ERR_TIMEOUT in eqlin.h)
+constexpr int kDeviceErrTimeout = -6;
+
+// byte offset of element (row r, column col) of sub-block `sub` (each sub-block
+// holds `rows` rows of 64 bytes)
+__host__ __device__ inline size_t image_offset(size_t sub, int rows, int r, int col) {
+    const int piece = (col >> 3) ^ ((r >> 1) & 3);
+    return sub * static_cast<size_t>(rows) * kPlaneRowBytes + static_cast<size_t>(r) * kPlaneRowBytes +
+           static_cast<size_t>(piece) * 16 + static_cast<size_t>(col & 7) * 2;
+}
+
+}  // namespace eqlin

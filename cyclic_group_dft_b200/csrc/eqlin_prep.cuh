@@ -1,0 +1,139 @@
+// eqlin_prep.cuh -- weight pre-transform (run once per weight update) and the fp32
+// fused forward.
+//
+// Page "Flash EQ-Linear: Accelerating Equivariant Linear Layers via Group-wise
+// Discrete Fourier Transform", section "Enfoque Algoritmico": in the frequency
+// domain the group convolution is a pointwise product, so the weights are moved to
+// the frequency domain once (W^_k = sum_m w_m exp(-2 pi i m k / G), k = 0..G/2) and
+// reused by every forward.  Layouts: eqlin_layout.h.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "eqlin_layout.h"
+#include "group_dft.cuh"
+
+namespace eqlin {
+
+template <typename T>
+__device__ __forceinline__ double load_as_double(const T* p, size_t i);
+template <>
+__device__ __forceinline__ double load_as_double<float>(const float* p, size_t i) {
+    return static_cast<double>(p[i]);
+}
+template <>
+__device__ __forceinline__ double load_as_double<__nv_bfloat16>(const __nv_bfloat16* p, size_t i) {
+    return static_cast<double>(__bfloat162float(p[i]));
+}
+
+// One thread per (o, i): real DFT of w[o, i, :] in float64, scaled for the folded
+// inverse (1/G real planes, 2/G complex planes), stored to w_f32[p][i][o].
+// Thread (o, i = 0) also converts bias[o] (or writes 0 when bias is null).
+template <typename T>
+__global__ void eqlin_prep_freq_kernel(const T* __restrict__ w, const T* __restrict__ bias, int Cout,
+                                       int Cin, int G, float* __restrict__ w_f32,
+                                       float* __restrict__ bias_f32) {
+    const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx >= static_cast<long long>(Cout) * Cin) return;
+    const int o = static_cast<int>(idx / Cin), i = static_cast<int>(idx % Cin);
+    const size_t base = static_cast<size_t>(idx) * G;
+    for (int p = 0; p < G; ++p) {
+        const int k = p == 0 ? 0 : (p == 1 ? G / 2 : p / 2);
+        const bool imag = p >= 2 && (p & 1);
+        const double scale = (p < 2 ? 1.0 : 2.0) / G;
+        double acc = 0.0;
+        for (int m = 0; m < G; ++m) {
+            double s, c;
+            sincospi(2.0 * static_cast<double>((m * k) % G) / G, &s, &c);
+            acc += load_as_double(w, base + m) * (imag ? -s : c);
+        }
+        w_f32[(static_cast<size_t>(p) * Cin + i) * Cout + o] = static_cast<float>(scale * acc);
+    }
+    if (i == 0) bias_f32[o] = bias != nullptr ? static_cast<float>(load_as_double(bias, o)) : 0.0f;
+}
+
+// One thread per element of the bf16 tensor-core image (see eqlin_layout.h).
+// `rows` rows per sub-block; output chunk oc covers o = oc*128 + r.
+__global__ void eqlin_prep_image_kernel(const float* __restrict__ w_f32, int Cout, int Cin, int G,
+                                        int nK, int rows, size_t n_elems, uint8_t* __restrict__ img) {
+    const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx >= n_elems) return;
+    const int col = static_cast<int>(idx % kChunkK);
+    const int r = static_cast<int>((idx / kChunkK) % rows);
+    const size_t sub = idx / (static_cast<size_t>(kChunkK) * rows);
+    const int p = static_cast<int>(sub % G);
+    const int c = static_cast<int>((sub / G) % nK);
+    const int oc = static_cast<int>(sub / (static_cast<size_t>(G) * nK));
+    const int o = oc * kMmaM + r;
+    const int i = c * kChunkK + col;
+    float v = 0.0f;
+    if (o < Cout && i < Cin) v = w_f32[(static_cast<size_t>(p) * Cin + i) * Cout + o];
+    *reinterpret_cast<__nv_bfloat16*>(img + image_offset(sub, rows, r, col)) = __float2bfloat16_rn(v);
+}
+
+// ------------------------------------------------------------------ fp32 path
+// Fused forward for fp32 I/O on CUDA cores (FFMA): the tensor-core kinds that take
+// fp32 operands round them to tf32 (10-bit mantissa), too coarse for a 1e-5 bound.
+// Block = 8 warps; block (bx, by) handles tokens [8 bx, 8 bx + 8) and outputs
+// [32 by, 32 by + 32); warp = token, lane = output channel.
+constexpr int kF32Tokens = 8;
+constexpr int kF32Threads = 256;
+
+template <int G>
+__global__ void __launch_bounds__(kF32Threads)
+    eqlin_fwd_f32_kernel(const float* __restrict__ x, const float* __restrict__ w_f32,
+                         const float* __restrict__ bias_f32, float* __restrict__ y, long long N,
+                         int Cin, int Cout) {
+    extern __shared__ float xs[];  // [kF32Tokens][G][Cin] spectrum of the block's tokens
+    const long long n0 = static_cast<long long>(blockIdx.x) * kF32Tokens;
+    for (int idx = threadIdx.x; idx < kF32Tokens * Cin; idx += kF32Threads) {
+        const int t = idx / Cin, i = idx % Cin;
+        const long long n = n0 + t;
+        float v[G], pl[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) v[h] = n < N ? x[(n * Cin + i) * G + h] : 0.0f;
+        rdft_planes<G>(v, pl);
+#pragma unroll
+        for (int p = 0; p < G; ++p) xs[(t * G + p) * Cin + i] = pl[p];
+    }
+    __syncthreads();
+    const int t = threadIdx.x >> 5;
+    const long long n = n0 + t;
+    const int o = blockIdx.y * 32 + (threadIdx.x & 31);
+    if (n >= N || o >= Cout) return;
+    float z[G];
+#pragma unroll
+    for (int p = 0; p < G; ++p) z[p] = 0.0f;
+    const float* xt = xs + t * G * Cin;
+    for (int i = 0; i < Cin; ++i) {
+        float xv[G], wv[G];
+#pragma unroll
+        for (int p = 0; p < G; ++p) {
+            xv[p] = xt[p * Cin + i];
+            wv[p] = w_f32[(static_cast<size_t>(p) * Cin + i) * Cout + o];
+        }
+        z[0] = fmaf(wv[0], xv[0], z[0]);
+        z[1] = fmaf(wv[1], xv[1], z[1]);
+#pragma unroll
+        for (int k = 1; k < G / 2; ++k) {
+            const int pr = 2 * k, pi = 2 * k + 1;
+            z[pr] = fmaf(wv[pr], xv[pr], fmaf(-wv[pi], xv[pi], z[pr]));
+            z[pi] = fmaf(wv[pi], xv[pr], fmaf(wv[pr], xv[pi], z[pi]));
+        }
+    }
+    z[0] += bias_f32[o];
+    float yv[G];
+    RealIdft<G>::run(z, yv);
+    float* dst = y + (n * Cout + o) * G;
+    if constexpr (G % 4 == 0) {
+#pragma unroll
+        for (int g = 0; g < G; g += 4) {
+            *reinterpret_cast<float4*>(dst + g) = make_float4(yv[g], yv[g + 1], yv[g + 2], yv[g + 3]);
+        }
+    } else {
+        *reinterpret_cast<float2*>(dst) = make_float2(yv[0], yv[1]);
+    }
+}
+
+}  // namespace eqlin

@@ -18,6 +18,17 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 GPU and the built CUDA library")
+    # build (if stale) the oracle and the CUDA library before test modules import them
+    # (the package's build script is loaded by path: importing the package
+    # itself requires the built library)
+    import importlib.util
+    from oracle import build as oracle_build
+    oracle_build.build()
+    spec = importlib.util.spec_from_file_location(
+        "_eqlin_build", os.path.join(ROOT, "cyclic_group_dft_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
 
 
 @pytest.fixture(scope="session")

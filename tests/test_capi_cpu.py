@@ -1,0 +1,111 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/eqlin.h declares, and rejects bad arguments on the host before any
+CUDA work (so these return codes are the same with or without a device)."""
+from __future__ import annotations
+
+import ctypes
+import subprocess
+
+import pytest
+import torch
+
+import cyclic_group_dft_b200 as eq
+from cyclic_group_dft_b200 import _capi
+
+
+def test_exports_every_declared_function():
+    declared = eq.header_functions()
+    assert len(declared) >= 10
+    lib = eq.library()
+    for name in declared:
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", eq.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    assert exported == set(declared), exported ^ set(declared)
+
+
+def test_version_and_status_strings():
+    assert eq.eqlin_version() >= 100
+    assert eq.eqlin_status_string(0) == "ok"
+    for code in range(-6, 0):
+        assert eq.eqlin_status_string(code) not in ("", "unknown status")
+    assert eq.eqlin_status_string(-99) == "unknown status"
+
+
+@pytest.mark.parametrize("shape,expected", [
+    ((96, 96, 4, eq.EQLIN_BF16, eq.EQLIN_BF16), eq.EQLIN_OK),
+    ((768, 192, 4, eq.EQLIN_BF16, eq.EQLIN_BF16), eq.EQLIN_OK),
+    ((64, 64, 8, eq.EQLIN_BF16, eq.EQLIN_BF16), eq.EQLIN_OK),
+    ((32, 32, 16, eq.EQLIN_BF16, eq.EQLIN_BF16), eq.EQLIN_OK),
+    ((16, 16, 4, eq.EQLIN_F32, eq.EQLIN_F32), eq.EQLIN_OK),
+    ((16, 16, 2, eq.EQLIN_F32, eq.EQLIN_BF16), eq.EQLIN_OK),
+    ((96, 96, 3, eq.EQLIN_BF16, eq.EQLIN_BF16), eq.EQLIN_ERR_UNSUPPORTED),
+    ((96, 96, 32, eq.EQLIN_BF16, eq.EQLIN_BF16), eq.EQLIN_ERR_UNSUPPORTED),
+    ((3, 3, 2, eq.EQLIN_BF16, eq.EQLIN_BF16), eq.EQLIN_ERR_UNSUPPORTED),   # Cin*G % 8
+    ((3, 3, 2, eq.EQLIN_F32, eq.EQLIN_F32), eq.EQLIN_OK),                  # fine for fp32
+    ((0, 4, 4, eq.EQLIN_BF16, eq.EQLIN_BF16), eq.EQLIN_ERR_INVALID_ARG),
+    ((4, -1, 4, eq.EQLIN_BF16, eq.EQLIN_BF16), eq.EQLIN_ERR_INVALID_ARG),
+    ((4, 4, 4, 7, eq.EQLIN_BF16), eq.EQLIN_ERR_INVALID_ARG),
+    ((4, 4, 4, eq.EQLIN_BF16, 9), eq.EQLIN_ERR_INVALID_ARG),
+    ((1 << 17, 8, 4, eq.EQLIN_BF16, eq.EQLIN_BF16), eq.EQLIN_ERR_UNSUPPORTED),
+])
+def test_check_shape(shape, expected):
+    assert eq.eqlin_check_shape(*shape) == expected
+
+
+def _prepare_raw(w_ptr, Cout=8, Cin=8, G=4, wd=eq.EQLIN_BF16, io=eq.EQLIN_BF16, out=True):
+    h = ctypes.c_void_p(1234)
+    st = eq.library().eqlin_prepare_weights(w_ptr, None, Cout, Cin, G, wd, io, None,
+                                            ctypes.byref(h) if out else None)
+    return st, h.value
+
+
+def test_prepare_rejects_bad_arguments_on_host():
+    lib = eq.library()
+    assert _prepare_raw(None)[0] == eq.EQLIN_ERR_INVALID_ARG
+    st, h = _prepare_raw(None)
+    assert h is None  # *out cleared on failure
+    assert _prepare_raw(16, out=False)[0] == eq.EQLIN_ERR_INVALID_ARG
+    assert _prepare_raw(16, G=5)[0] == eq.EQLIN_ERR_UNSUPPORTED
+    assert _prepare_raw(16, Cout=0)[0] == eq.EQLIN_ERR_INVALID_ARG
+    assert _prepare_raw(17)[0] == eq.EQLIN_ERR_MISALIGNED        # bf16 w at an odd address
+    assert _prepare_raw(18, wd=eq.EQLIN_F32, io=eq.EQLIN_F32)[0] == eq.EQLIN_ERR_MISALIGNED
+    assert "aligned" in eq.eqlin_last_error()
+    assert lib.eqlin_destroy(None) == eq.EQLIN_OK
+
+
+def test_forward_rejects_bad_arguments_on_host():
+    lib = eq.library()
+    assert lib.eqlin_forward(None, 16, 16, 4, None) == eq.EQLIN_ERR_INVALID_ARG
+    assert "NULL" in eq.eqlin_last_error()
+    v = ctypes.c_int64()
+    assert lib.eqlin_get_attr(None, 0, ctypes.byref(v)) == eq.EQLIN_ERR_INVALID_ARG
+    s = ctypes.c_int()
+    assert lib.eqlin_device_status(None, ctypes.byref(s)) == eq.EQLIN_ERR_INVALID_ARG
+    assert lib.eqlin_copy_freq_weights(None, None, 0) == eq.EQLIN_ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks behaviour without a GPU")
+def test_prepare_without_gpu_reports_cuda_error():
+    # an aligned fake pointer passes host validation; the device query then fails
+    st, h = _prepare_raw(256)
+    assert st == eq.EQLIN_ERR_CUDA
+    assert h is None
+
+
+def test_binding_validates_before_calling():
+    with pytest.raises(ValueError):
+        eq.eqlin_prepare_weights(torch.zeros(4, 4))          # not 3-D
+    with pytest.raises(ValueError):
+        eq.eqlin_prepare_weights(torch.zeros(4, 4, 4))       # not on a GPU
+
+
+def test_header_matches_binding_constants():
+    text = open(_capi.HEADER_PATH).read()
+    for name in ("EQLIN_ERR_INVALID_ARG = -1", "EQLIN_ERR_UNSUPPORTED = -2", "EQLIN_ERR_MISALIGNED = -3",
+                 "EQLIN_ERR_CUDA = -4", "EQLIN_ERR_OOM = -5", "EQLIN_ERR_TIMEOUT = -6",
+                 "EQLIN_F32 = 0", "EQLIN_BF16 = 1"):
+        assert name in text
+    for attr, code in eq.ATTRS.items():
+        assert f"= {code}" in text
