@@ -243,9 +243,13 @@ def main() -> None:
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override the workload's token count (profiling a smaller case)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     wl = workloads.WORKLOADS[args.workload]
+    if args.tokens is not None:
+        wl = wl.with_n(args.tokens)
 
     if args.impl == "reference":
         run_reference(args, wl)
@@ -314,25 +318,30 @@ def main() -> None:
 
     # ----------------------------------------------------------- end to end
     E = args.e2e_steps
-    x_pin = x_cpu.pin_memory()
-    y_pin = torch.empty(N, wl.Cout, wl.G, dtype=wl.torch_dtype).pin_memory()
-    h.forward_host(x_pin, y_pin)  # warm the path
-    barrier()
-    torch.cuda.synchronize(dev)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(E):
-        h.forward_host(x_pin, y_pin, stream=stream)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * E * N / (e2e_ms / 1e3)
+    e2e = None
+    if E > 0:
+        x_pin = x_cpu.pin_memory()
+        y_pin = torch.empty(N, wl.Cout, wl.G, dtype=wl.torch_dtype).pin_memory()
+        h.forward_host(x_pin, y_pin)  # warm the path
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(E):
+            h.forward_host(x_pin, y_pin, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e2e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": world * E * N / (e2e_ms / 1e3), "unit": "tokens/s", "steps": E,
+               "h2d_bytes_per_step": x_pin.numel() * x_pin.element_size(),
+               "d2h_bytes_per_step": y_pin.numel() * y_pin.element_size(),
+               "api": "Handle.forward_host (pinned host x -> device -> eqlin_forward -> pinned host y)"}
 
     # ----------------------------------------------------------- CPU baseline
     cpu = None
@@ -394,10 +403,7 @@ def main() -> None:
         "launch_us": {"mean": 1e3 * statistics.mean(launch_ms), "median": 1e3 * statistics.median(launch_ms),
                       "min": 1e3 * min(launch_ms), "max": 1e3 * max(launch_ms)},
         "clocks": clocks.summary(),
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "steps": E,
-                "h2d_bytes_per_step": x_pin.numel() * x_pin.element_size(),
-                "d2h_bytes_per_step": y_pin.numel() * y_pin.element_size(),
-                "api": "Handle.forward_host (pinned host x -> device -> eqlin_forward -> pinned host y)"},
+        "e2e": e2e,
         "gpu_launches": K,
         "device_status": status,
         "cpu_baseline": cpu,

@@ -24,8 +24,8 @@ namespace {
 
 constexpr size_t kB200SmemOptin = 232448;   // 227 KB opt-in shared memory per CTA on sm_100
 constexpr size_t kSmemAlignSlack = 1024;    // the kernel rounds its smem base up to 1 KB
-constexpr size_t kSmemCtlBytes = 256;       // mbarriers + control block
-constexpr int kMaxStages = 8;
+constexpr size_t kSmemCtlBytes = 512;       // mbarriers + control block
+constexpr int kMaxStages = 12;
 constexpr int64_t kMaxChannels = 1 << 16;
 constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per bounded wait
 
@@ -94,7 +94,7 @@ int plan_tc_g(int64_t Cout, int64_t Cin, size_t max_smem, Plan* pl) {
 
 int plan_for(int64_t Cout, int64_t Cin, int64_t G, int io_dtype, size_t max_smem, Plan* pl) {
     if (io_dtype == EQLIN_F32) {
-        const size_t smem = static_cast<size_t>(eqlin::kF32Tokens) * G * Cin * sizeof(float);
+        const size_t smem = static_cast<size_t>(eqlin::kF32Tokens) * G * Cin * sizeof(double);
         if (smem > max_smem) return fail(EQLIN_ERR_UNSUPPORTED, "Cin*G too large for the fp32 path");
         pl->path = kPathF32;
         pl->BN = eqlin::kF32Tokens;
@@ -185,6 +185,8 @@ struct eqlin_handle {
     uint8_t* w_img = nullptr;
     float* w_f32 = nullptr;
     float* bias_f32 = nullptr;
+    double* w_f64 = nullptr;     // fp32-I/O path only
+    double* bias_f64 = nullptr;  // fp32-I/O path only
     int* status = nullptr;
     bool has_bias = false;
     bool sync_check = false;
@@ -198,6 +200,8 @@ void free_handle(eqlin_handle* h) {
     if (h->w_img) cudaFree(h->w_img);
     if (h->w_f32) cudaFree(h->w_f32);
     if (h->bias_f32) cudaFree(h->bias_f32);
+    if (h->w_f64) cudaFree(h->w_f64);
+    if (h->bias_f64) cudaFree(h->bias_f64);
     if (h->status) cudaFree(h->status);
     delete h;
 }
@@ -209,11 +213,12 @@ int launch_prep(eqlin_handle* h, const void* w, const void* bias, cudaStream_t s
     const int Cout = static_cast<int>(h->Cout), Cin = static_cast<int>(h->Cin), G = static_cast<int>(h->G);
     if (h->w_dtype == EQLIN_F32) {
         eqlin::eqlin_prep_freq_kernel<float><<<blocks, threads, 0, st>>>(
-            static_cast<const float*>(w), static_cast<const float*>(bias), Cout, Cin, G, h->w_f32, h->bias_f32);
+            static_cast<const float*>(w), static_cast<const float*>(bias), Cout, Cin, G, h->w_f32, h->bias_f32,
+            h->w_f64, h->bias_f64);
     } else {
         eqlin::eqlin_prep_freq_kernel<__nv_bfloat16><<<blocks, threads, 0, st>>>(
             static_cast<const __nv_bfloat16*>(w), static_cast<const __nv_bfloat16*>(bias), Cout, Cin, G,
-            h->w_f32, h->bias_f32);
+            h->w_f32, h->bias_f32, h->w_f64, h->bias_f64);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "weight transform launch");
@@ -290,6 +295,8 @@ int eqlin_prepare_weights(const void* w, const void* bias, int64_t Cout, int64_t
     if (cudaMalloc(&h->w_f32, wf_bytes) != cudaSuccess ||
         cudaMalloc(&h->bias_f32, static_cast<size_t>(Cout) * sizeof(float)) != cudaSuccess ||
         cudaMalloc(&h->status, 256) != cudaSuccess ||
+        (plan.path == kPathF32 && (cudaMalloc(&h->w_f64, wf_bytes * 2) != cudaSuccess ||
+                                   cudaMalloc(&h->bias_f64, static_cast<size_t>(Cout) * sizeof(double)) != cudaSuccess)) ||
         (plan.img_alloc_bytes && cudaMalloc(&h->w_img, plan.img_alloc_bytes) != cudaSuccess)) {
         cudaGetLastError();
         free_handle(h);
@@ -340,10 +347,10 @@ int eqlin_forward(const eqlin_handle* h, const void* x, void* y, int64_t N, void
         const long long n = N;
         const int Cin = static_cast<int>(h->Cin), Cout = static_cast<int>(h->Cout);
         switch (G) {
-            case 2: eqlin::eqlin_fwd_f32_kernel<2><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, h->w_f32, h->bias_f32, yf, n, Cin, Cout); break;
-            case 4: eqlin::eqlin_fwd_f32_kernel<4><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, h->w_f32, h->bias_f32, yf, n, Cin, Cout); break;
-            case 8: eqlin::eqlin_fwd_f32_kernel<8><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, h->w_f32, h->bias_f32, yf, n, Cin, Cout); break;
-            default: eqlin::eqlin_fwd_f32_kernel<16><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, h->w_f32, h->bias_f32, yf, n, Cin, Cout); break;
+            case 2: eqlin::eqlin_fwd_f32_kernel<2><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, h->w_f64, h->bias_f64, yf, n, Cin, Cout); break;
+            case 4: eqlin::eqlin_fwd_f32_kernel<4><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, h->w_f64, h->bias_f64, yf, n, Cin, Cout); break;
+            case 8: eqlin::eqlin_fwd_f32_kernel<8><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, h->w_f64, h->bias_f64, yf, n, Cin, Cout); break;
+            default: eqlin::eqlin_fwd_f32_kernel<16><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, h->w_f64, h->bias_f64, yf, n, Cin, Cout); break;
         }
     } else {
         auto encode = tensor_map_encoder();
@@ -439,7 +446,7 @@ int eqlin_get_attr(const eqlin_handle* h, int attr, int64_t* value) {
         case EQLIN_ATTR_SMEM_BYTES: *value = static_cast<int64_t>(pl.smem_bytes); break;
         case EQLIN_ATTR_MAX_GRID: *value = pl.path == kPathF32 ? -1 : h->sm_count; break;
         case EQLIN_ATTR_WEIGHT_BYTES:
-            *value = pl.path == kPathF32 ? static_cast<int64_t>(h->G * h->Cin * h->Cout * 4)
+            *value = pl.path == kPathF32 ? static_cast<int64_t>(h->G * h->Cin * h->Cout * 8)
                                          : static_cast<int64_t>(pl.img_alloc_bytes);
             break;
         default: return fail(EQLIN_ERR_INVALID_ARG, "unknown attribute");

@@ -9,20 +9,23 @@
 // (section "Implementacion": fused dataflow, Fourier fragments kept on chip).
 //
 // Per CTA (one per SM, persistent over work items = (token tile, 128-row output chunk)):
-//   warp 8     TMA producer: x chunks [BN tokens x 32 channels x G] into a smem ring
-//              (plus the weight chunk when the weights are streamed).
-//   warps 4-7  DFT: read a landed x chunk, real DFT over G in fp32 registers, write the
-//              G frequency planes [BN x 32] bf16 back IN PLACE in the UMMA K-major
-//              SWIZZLE_64B layout (the x chunk and its spectrum have the same size).
-//   warp 9     MMA issuer (one thread) + TMEM owner: per chunk and frequency,
-//              tcgen05.mma with A = W^ plane [128 out-rows x 32], B = X^ plane [BN x 32],
-//              D in TMEM (lane = output channel, column = token).  Complex frequencies
-//              use four real products; the -Im(W)Im(X) term uses the descriptor's
-//              negate-A bit, so only Re and Im of W^ are stored.
-//   warps 0-3  epilogue: tcgen05.ld of all G planes of a token group, inverse real DFT
-//              (1/G and 2/G are folded into W^), + bias, round to bf16 and store
-//              y[n, o, 0..G-1] directly: a warp writes 32 consecutive o -> one
-//              contiguous run of 32*G*2 bytes per token.
+//   warp 12     TMA producer: x chunks [BN tokens x 32 channels x G] (16 KB) into a smem
+//               ring (plus the weight chunk when the weights are streamed).
+//   warps 8-11  DFT: read a landed x chunk, real DFT over G in fp32 registers, write the
+//               G frequency planes [BN x 32] bf16 back IN PLACE in the UMMA K-major
+//               SWIZZLE_64B layout (the x chunk and its spectrum have the same size).
+//   warp 13     MMA issuer (one thread) + TMEM owner: per chunk and frequency,
+//               tcgen05.mma with A = W^ plane [128 out-rows x 32], B = X^ plane [BN x 32],
+//               D in TMEM (lane = output channel, column = token).  Complex frequencies
+//               use four real products; the -Im(W)Im(X) term uses the descriptor's
+//               negate-A bit, so only Re and Im of W^ are stored.  Two accumulators
+//               (G*BN = 256 columns each) alternate between work items, so the MMAs of
+//               one tile overlap the epilogue of the previous one.
+//   warps 0-7   epilogue: tcgen05.ld of all G planes of a token group, inverse real DFT
+//               (1/G and 2/G are folded into W^), + bias, round to bf16 and store
+//               y[n, o, 0..G-1] directly: a warp writes 32 consecutive o -> one
+//               contiguous run of 32*G*2 bytes per token.  Warps w and w+4 share TMEM
+//               lane quarter w and split the tile's tokens.
 // All waits are bounded (globaltimer); on expiry the kernel records EQLIN_ERR_TIMEOUT
 // in the status word, every role leaves its loop, in-flight copies and MMAs are
 // drained with bounded waits, and TMEM is freed before exit.
@@ -56,26 +59,32 @@ struct TcParams {
 
 namespace tc {
 
-constexpr int kThreads = 320;
-constexpr int kWarpProducer = 8;
-constexpr int kWarpMma = 9;
+constexpr int kThreads = 448;
+constexpr int kEpiWarps = 8;
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kWarpDft0 = 8;
+constexpr int kWarpProducer = 12;
+constexpr int kWarpMma = 13;
+constexpr int kNumAcc = 2;       // TMEM accumulator buffers
 constexpr int kBarDft = 1;   // named barrier ids (0 is __syncthreads)
 constexpr int kBarEpi = 2;
 
 template <int G>
 struct Shape {
-    static constexpr int BN = (512 / G) < 128 ? (512 / G) : 128;    // tokens per tile (MMA N)
+    static constexpr int BN = (256 / G) < 128 ? (256 / G) : 128;    // tokens per tile (MMA N)
     static constexpr int PLANE_BYTES = BN * kPlaneRowBytes;          // one frequency plane
     static constexpr int XCHUNK_BYTES = G * PLANE_BYTES;             // == BN * 32 * G * 2
     static constexpr int XROW_ELEMS = kChunkK * G;                   // one token row of a chunk
     static constexpr int BOX_ELEMS = XROW_ELEMS < 256 ? XROW_ELEMS : 256;
     static constexpr int NBOX = XROW_ELEMS / BOX_ELEMS;
     static constexpr int WSTAGE_BYTES = G * kMmaM * kPlaneRowBytes;  // streamed weight chunk
-    static constexpr int TMEM_COLS = (G * BN <= 256) ? 256 : 512;
-    static constexpr int TG = (64 / G) < BN ? (64 / G) : BN;         // tokens per epilogue group
+    static constexpr int ACC_COLS = G * BN;                          // one accumulator
+    static constexpr int TMEM_COLS = 512;
+    static constexpr int TG = (64 / G) < BN / 2 ? (64 / G) : BN / 2;  // tokens per epilogue group
     static_assert(XCHUNK_BYTES % 1024 == 0, "stage alignment");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N");
-    static_assert(G * BN <= TMEM_COLS, "TMEM columns");
+    static_assert(kNumAcc * ACC_COLS <= TMEM_COLS, "TMEM columns");
+    static_assert((BN / 2) % TG == 0, "epilogue groups");
 };
 
 struct Ctl {
@@ -174,8 +183,10 @@ __device__ __forceinline__ void dft_chunk(uint8_t* xs, int dft_tid) {
 }
 
 // ------------------------------------------------------------ epilogue role
+// Warp (q, half): TMEM lane quarter q (output rows 32q..32q+31 of the chunk), tokens
+// [half*BN/2, (half+1)*BN/2) of the tile held in accumulator `acc` (column base).
 template <int G>
-__device__ __forceinline__ void epilogue_tile(const TcParams& p, uint32_t tmem_base, int q,
+__device__ __forceinline__ void epilogue_tile(const TcParams& p, uint32_t acc, int q, int half,
                                               int lane, long long n0, int oc) {
     using S = Shape<G>;
     constexpr int TG = S::TG;
@@ -183,16 +194,17 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, uint32_t tmem_b
     const int o = oc * kMmaM + o_local;
     const bool valid_o = o < p.Cout;
     const float b = (p.bias != nullptr && valid_o) ? p.bias[o] : 0.0f;
-    const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    const uint32_t lane_addr = acc + (static_cast<uint32_t>(q * 32) << 16);
+    const int t0 = half * (S::BN / 2);
 #pragma unroll 1
-    for (int j = 0; j < S::BN / TG; ++j) {
+    for (int j = 0; j < S::BN / 2 / TG; ++j) {
         uint32_t r[G][TG];
 #pragma unroll
-        for (int pl = 0; pl < G; ++pl) ptx::tmem_ld_32x32b<TG>(lane_addr + pl * S::BN + j * TG, r[pl]);
+        for (int pl = 0; pl < G; ++pl) ptx::tmem_ld_32x32b<TG>(lane_addr + pl * S::BN + t0 + j * TG, r[pl]);
         ptx::tmem_wait_ld();
 #pragma unroll
         for (int t = 0; t < TG; ++t) {
-            const long long n = n0 + j * TG + t;
+            const long long n = n0 + t0 + j * TG + t;
             float z[G], yv[G];
 #pragma unroll
             for (int pl = 0; pl < G; ++pl) z[pl] = __uint_as_float(r[pl][t]);
@@ -235,17 +247,17 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     const int NS = p.stages;
     uint8_t* stage0 = smem + p.w_region_bytes;
     uint64_t* bars = reinterpret_cast<uint64_t*>(stage0 + static_cast<size_t>(NS) * STAGE_BYTES);
-    tc::Ctl* ctl = reinterpret_cast<tc::Ctl*>(bars + 3 * NS + 4);
+    tc::Ctl* ctl = reinterpret_cast<tc::Ctl*>(bars + 3 * NS + 2 * tc::kNumAcc + 2);
 
     const uint32_t s_w = ptx::smem_u32(smem);
     const uint32_t s_stage0 = ptx::smem_u32(stage0);
     auto bar_full = [&](int s) { return ptx::smem_u32(bars + s); };
     auto bar_xhat = [&](int s) { return ptx::smem_u32(bars + NS + s); };
     auto bar_empty = [&](int s) { return ptx::smem_u32(bars + 2 * NS + s); };
-    const uint32_t bar_acc_full = ptx::smem_u32(bars + 3 * NS + 0);
-    const uint32_t bar_acc_empty = ptx::smem_u32(bars + 3 * NS + 1);
-    const uint32_t bar_w_full = ptx::smem_u32(bars + 3 * NS + 2);
-    const uint32_t bar_drain = ptx::smem_u32(bars + 3 * NS + 3);
+    auto bar_acc_full = [&](int a) { return ptx::smem_u32(bars + 3 * NS + a); };
+    auto bar_acc_empty = [&](int a) { return ptx::smem_u32(bars + 3 * NS + tc::kNumAcc + a); };
+    const uint32_t bar_w_full = ptx::smem_u32(bars + 3 * NS + 2 * tc::kNumAcc);
+    const uint32_t bar_drain = ptx::smem_u32(bars + 3 * NS + 2 * tc::kNumAcc + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -255,8 +267,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
             ptx::mbar_init(bar_xhat(s), 128);
             ptx::mbar_init(bar_empty(s), 1);
         }
-        ptx::mbar_init(bar_acc_full, 1);
-        ptx::mbar_init(bar_acc_empty, 128);
+        for (int a = 0; a < tc::kNumAcc; ++a) {
+            ptx::mbar_init(bar_acc_full(a), 1);
+            ptx::mbar_init(bar_acc_empty(a), tc::kEpiThreads);
+        }
         ptx::mbar_init(bar_w_full, 1);
         ptx::mbar_init(bar_drain, 1);
         ctl->abort = 0;
@@ -344,13 +358,17 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
             constexpr uint32_t ID = idesc_bf16_f32(kMmaM, S::BN, false);
             constexpr uint32_t ID_NEG = idesc_bf16_f32(kMmaM, S::BN, true);
             int stage = 0;
-            uint32_t phase = 0, acc_phase = 0;
-            for (int wk = blockIdx.x; ok && wk < p.n_work; wk += gridDim.x) {
-                if (!tc::wait_bounded(bar_acc_empty, acc_phase ^ 1u, ctl, p.status, p.timeout_ns)) {
+            uint32_t phase = 0;
+            int it = 0;
+            for (int wk = blockIdx.x; ok && wk < p.n_work; wk += gridDim.x, ++it) {
+                const int abuf = it & 1;
+                const uint32_t acc_phase = static_cast<uint32_t>(it >> 1) & 1u;
+                if (!tc::wait_bounded(bar_acc_empty(abuf), acc_phase ^ 1u, ctl, p.status, p.timeout_ns)) {
                     ok = false;
                     break;
                 }
                 ptx::tc_fence_after();
+                const uint32_t acc_base = tmem_base + static_cast<uint32_t>(abuf * S::ACC_COLS);
                 for (int c = 0; c < p.nK; ++c) {
                     if (!tc::wait_bounded(bar_xhat(stage), phase, ctl, p.status, p.timeout_ns)) {
                         ok = false;
@@ -373,7 +391,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                         auto B = [&](int pl) {
                             return ptx::sdesc_kmajor_sw64(xb + pl * S::PLANE_BYTES + ks * 32);
                         };
-                        auto D = [&](int pl) { return tmem_base + static_cast<uint32_t>(pl * S::BN); };
+                        auto D = [&](int pl) { return acc_base + static_cast<uint32_t>(pl * S::BN); };
                         // real frequencies k = 0 and k = G/2
                         ptx::umma_f16(D(0), A(0), B(0), ID, acc0);
                         ptx::umma_f16(D(1), A(1), B(1), ID, acc0);
@@ -391,8 +409,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                     if (++stage == NS) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
-                ptx::umma_commit(bar_acc_full);
-                acc_phase ^= 1u;
+                ptx::umma_commit(bar_acc_full(abuf));
             }
             // drain: all MMAs done before TMEM is released
             ptx::umma_commit(bar_drain);
@@ -404,9 +421,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                 }
             }
         }
-    } else if (warp >= 4) {
+    } else if (warp >= tc::kWarpDft0) {
         // ------------------------------------------------------------ DFT warps
-        const int dft_tid = threadIdx.x - 128;
+        const int dft_tid = threadIdx.x - tc::kWarpDft0 * 32;
         int stage = 0;
         uint32_t phase = 0;
         for (int wk = blockIdx.x; wk < p.n_work; wk += gridDim.x) {
@@ -426,16 +443,18 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue warps
-        uint32_t acc_phase = 0;
-        for (int wk = blockIdx.x; wk < p.n_work; wk += gridDim.x) {
-            const bool got = tc::wait_bounded(bar_acc_full, acc_phase, ctl, p.status, p.timeout_ns);
-            if (!ptx::named_bar_and(tc::kBarEpi, 128, got)) break;
+        int it = 0;
+        for (int wk = blockIdx.x; wk < p.n_work; wk += gridDim.x, ++it) {
+            const int abuf = it & 1;
+            const uint32_t acc_phase = static_cast<uint32_t>(it >> 1) & 1u;
+            const bool got = tc::wait_bounded(bar_acc_full(abuf), acc_phase, ctl, p.status, p.timeout_ns);
+            if (!ptx::named_bar_and(tc::kBarEpi, tc::kEpiThreads, got)) break;
             ptx::tc_fence_after();
             const int tile = wk / p.n_oc, oc = wk % p.n_oc;
-            tc::epilogue_tile<G>(p, tmem_base, warp, lane, static_cast<long long>(tile) * S::BN, oc);
+            tc::epilogue_tile<G>(p, tmem_base + static_cast<uint32_t>(abuf * S::ACC_COLS), warp & 3,
+                                 warp >> 2, lane, static_cast<long long>(tile) * S::BN, oc);
             ptx::tc_fence_before();
-            ptx::mbar_arrive(bar_acc_empty);
-            acc_phase ^= 1u;
+            ptx::mbar_arrive(bar_acc_empty(abuf));
         }
     }
 

@@ -28,12 +28,14 @@ __device__ __forceinline__ double load_as_double<__nv_bfloat16>(const __nv_bfloa
 }
 
 // One thread per (o, i): real DFT of w[o, i, :] in float64, scaled for the folded
-// inverse (1/G real planes, 2/G complex planes), stored to w_f32[p][i][o].
-// Thread (o, i = 0) also converts bias[o] (or writes 0 when bias is null).
+// inverse (1/G real planes, 2/G complex planes), stored to w_f32[p][i][o] and, when
+// w_f64 is not null, to w_f64[p][i][o].  Thread (o, i = 0) also converts bias[o]
+// (0 when bias is null) to bias_f32[o] and, when requested, bias_f64[o].
 template <typename T>
 __global__ void eqlin_prep_freq_kernel(const T* __restrict__ w, const T* __restrict__ bias, int Cout,
                                        int Cin, int G, float* __restrict__ w_f32,
-                                       float* __restrict__ bias_f32) {
+                                       float* __restrict__ bias_f32, double* __restrict__ w_f64,
+                                       double* __restrict__ bias_f64) {
     const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (idx >= static_cast<long long>(Cout) * Cin) return;
     const int o = static_cast<int>(idx / Cin), i = static_cast<int>(idx % Cin);
@@ -48,9 +50,15 @@ __global__ void eqlin_prep_freq_kernel(const T* __restrict__ w, const T* __restr
             sincospi(2.0 * static_cast<double>((m * k) % G) / G, &s, &c);
             acc += load_as_double(w, base + m) * (imag ? -s : c);
         }
-        w_f32[(static_cast<size_t>(p) * Cin + i) * Cout + o] = static_cast<float>(scale * acc);
+        const size_t dst = (static_cast<size_t>(p) * Cin + i) * Cout + o;
+        w_f32[dst] = static_cast<float>(scale * acc);
+        if (w_f64 != nullptr) w_f64[dst] = scale * acc;
     }
-    if (i == 0) bias_f32[o] = bias != nullptr ? static_cast<float>(load_as_double(bias, o)) : 0.0f;
+    if (i == 0) {
+        const double b = bias != nullptr ? load_as_double(bias, o) : 0.0;
+        bias_f32[o] = static_cast<float>(b);
+        if (bias_f64 != nullptr) bias_f64[o] = b;
+    }
 }
 
 // One thread per element of the bf16 tensor-core image (see eqlin_layout.h).
@@ -73,8 +81,10 @@ __global__ void eqlin_prep_image_kernel(const float* __restrict__ w_f32, int Cou
 }
 
 // ------------------------------------------------------------------ fp32 path
-// Fused forward for fp32 I/O on CUDA cores (FFMA): the tensor-core kinds that take
-// fp32 operands round them to tf32 (10-bit mantissa), too coarse for a 1e-5 bound.
+// Fused forward for fp32 I/O on CUDA cores.  The tensor-core kinds that take fp32
+// operands round them to tf32 (10-bit mantissa), far from a 1e-5 bound, so this
+// path keeps x, the spectra, the weights and the accumulation in float64 and
+// rounds once, when y is stored (elementwise relative error ~2^-24).
 // Block = 8 warps; block (bx, by) handles tokens [8 bx, 8 bx + 8) and outputs
 // [32 by, 32 by + 32); warp = token, lane = output channel.
 constexpr int kF32Tokens = 8;
@@ -82,18 +92,18 @@ constexpr int kF32Threads = 256;
 
 template <int G>
 __global__ void __launch_bounds__(kF32Threads)
-    eqlin_fwd_f32_kernel(const float* __restrict__ x, const float* __restrict__ w_f32,
-                         const float* __restrict__ bias_f32, float* __restrict__ y, long long N,
+    eqlin_fwd_f32_kernel(const float* __restrict__ x, const double* __restrict__ w_f64,
+                         const double* __restrict__ bias_f64, float* __restrict__ y, long long N,
                          int Cin, int Cout) {
-    extern __shared__ float xs[];  // [kF32Tokens][G][Cin] spectrum of the block's tokens
+    extern __shared__ double xs[];  // [kF32Tokens][G][Cin] spectrum of the block's tokens
     const long long n0 = static_cast<long long>(blockIdx.x) * kF32Tokens;
     for (int idx = threadIdx.x; idx < kF32Tokens * Cin; idx += kF32Threads) {
         const int t = idx / Cin, i = idx % Cin;
         const long long n = n0 + t;
-        float v[G], pl[G];
+        double v[G], pl[G];
 #pragma unroll
-        for (int h = 0; h < G; ++h) v[h] = n < N ? x[(n * Cin + i) * G + h] : 0.0f;
-        rdft_planes<G>(v, pl);
+        for (int h = 0; h < G; ++h) v[h] = n < N ? static_cast<double>(x[(n * Cin + i) * G + h]) : 0.0;
+        rdft_planes<G, double>(v, pl);
 #pragma unroll
         for (int p = 0; p < G; ++p) xs[(t * G + p) * Cin + i] = pl[p];
     }
@@ -102,37 +112,39 @@ __global__ void __launch_bounds__(kF32Threads)
     const long long n = n0 + t;
     const int o = blockIdx.y * 32 + (threadIdx.x & 31);
     if (n >= N || o >= Cout) return;
-    float z[G];
+    double z[G];
 #pragma unroll
-    for (int p = 0; p < G; ++p) z[p] = 0.0f;
-    const float* xt = xs + t * G * Cin;
+    for (int p = 0; p < G; ++p) z[p] = 0.0;
+    const double* xt = xs + t * G * Cin;
     for (int i = 0; i < Cin; ++i) {
-        float xv[G], wv[G];
+        double xv[G], wv[G];
 #pragma unroll
         for (int p = 0; p < G; ++p) {
             xv[p] = xt[p * Cin + i];
-            wv[p] = w_f32[(static_cast<size_t>(p) * Cin + i) * Cout + o];
+            wv[p] = w_f64[(static_cast<size_t>(p) * Cin + i) * Cout + o];
         }
-        z[0] = fmaf(wv[0], xv[0], z[0]);
-        z[1] = fmaf(wv[1], xv[1], z[1]);
+        z[0] = fma(wv[0], xv[0], z[0]);
+        z[1] = fma(wv[1], xv[1], z[1]);
 #pragma unroll
         for (int k = 1; k < G / 2; ++k) {
             const int pr = 2 * k, pi = 2 * k + 1;
-            z[pr] = fmaf(wv[pr], xv[pr], fmaf(-wv[pi], xv[pi], z[pr]));
-            z[pi] = fmaf(wv[pi], xv[pr], fmaf(wv[pr], xv[pi], z[pi]));
+            z[pr] = fma(wv[pr], xv[pr], fma(-wv[pi], xv[pi], z[pr]));
+            z[pi] = fma(wv[pi], xv[pr], fma(wv[pr], xv[pi], z[pi]));
         }
     }
-    z[0] += bias_f32[o];
-    float yv[G];
-    RealIdft<G>::run(z, yv);
+    z[0] += bias_f64[o];
+    double yv[G];
+    RealIdft<G, double>::run(z, yv);
     float* dst = y + (n * Cout + o) * G;
     if constexpr (G % 4 == 0) {
 #pragma unroll
         for (int g = 0; g < G; g += 4) {
-            *reinterpret_cast<float4*>(dst + g) = make_float4(yv[g], yv[g + 1], yv[g + 2], yv[g + 3]);
+            *reinterpret_cast<float4*>(dst + g) =
+                make_float4(static_cast<float>(yv[g]), static_cast<float>(yv[g + 1]),
+                            static_cast<float>(yv[g + 2]), static_cast<float>(yv[g + 3]));
         }
     } else {
-        *reinterpret_cast<float2*>(dst) = make_float2(yv[0], yv[1]);
+        *reinterpret_cast<float2*>(dst) = make_float2(static_cast<float>(yv[0]), static_cast<float>(yv[1]));
     }
 }
 

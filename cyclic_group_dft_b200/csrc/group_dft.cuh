@@ -9,6 +9,8 @@
 // subtractions (section "Especializacion para el Grupo de Rotacion p4"); the
 // recursion below reproduces that: G = 4 costs 8 add/sub forward, 8 inverse.
 //
+// T is float (bf16 path) or double (fp32-I/O path).
+//
 // Frequency components are kept in "plane order":
 //   plane 0      = Re X_0          (real)
 //   plane 1      = Re X_{G/2}      (real, Nyquist)
@@ -22,33 +24,38 @@
 namespace eqlin {
 
 // cos(2*pi*j/16), exact closed forms: cos(pi/8) = sqrt(2+sqrt(2))/2,
-// cos(pi/4) = sqrt(2)/2, cos(3pi/8) = sqrt(2-sqrt(2))/2, rounded to float.
-__host__ __device__ constexpr float cos16(int j) {
-    constexpr float c1 = 0.923879532511286756128f;
-    constexpr float c2 = 0.707106781186547524401f;
-    constexpr float c3 = 0.382683432365089771728f;
+// cos(pi/4) = sqrt(2)/2, cos(3pi/8) = sqrt(2-sqrt(2))/2, rounded to T.
+template <typename T = float>
+__host__ __device__ constexpr T cos16(int j) {
+    constexpr T c1 = static_cast<T>(0.923879532511286756128183189396788933);
+    constexpr T c2 = static_cast<T>(0.707106781186547524400844362104849039);
+    constexpr T c3 = static_cast<T>(0.382683432365089771728459984030398867);
     j &= 15;
     switch (j) {
-        case 0: return 1.0f;
+        case 0: return T(1);
         case 1: return c1;
         case 2: return c2;
         case 3: return c3;
-        case 4: return 0.0f;
+        case 4: return T(0);
         case 5: return -c3;
         case 6: return -c2;
         case 7: return -c1;
-        case 8: return -1.0f;
+        case 8: return T(-1);
         case 9: return -c1;
         case 10: return -c2;
         case 11: return -c3;
-        case 12: return 0.0f;
+        case 12: return T(0);
         case 13: return c3;
         case 14: return c2;
         default: return c1;
     }
 }
 // sin(2*pi*j/16) = cos(2*pi*(j-4)/16)
-__host__ __device__ constexpr float sin16(int j) { return cos16(j - 4); }
+template <typename T = float>
+__host__ __device__ constexpr T sin16(int j) { return cos16<T>(j - 4); }
+
+__device__ __forceinline__ float fma_t(float a, float b, float c) { return fmaf(a, b, c); }
+__device__ __forceinline__ double fma_t(double a, double b, double c) { return fma(a, b, c); }
 
 template <int N, class F, int... Is>
 __device__ __forceinline__ void static_for_impl(F&& f, std::integer_sequence<int, Is...>) {
@@ -62,8 +69,8 @@ __device__ __forceinline__ void static_for(F&& f) {
 
 // acc += v * cos(2 pi J / 16) and accI -= v * sin(2 pi J / 16), with the trivial
 // angles (multiples of pi/2) done as plain adds.
-template <int J>
-__device__ __forceinline__ void twiddle_acc(float v, float& re, float& im) {
+template <int J, typename T>
+__device__ __forceinline__ void twiddle_acc(T v, T& re, T& im) {
     constexpr int j = J & 15;
     if constexpr (j == 0) {
         re += v;
@@ -74,14 +81,14 @@ __device__ __forceinline__ void twiddle_acc(float v, float& re, float& im) {
     } else if constexpr (j == 12) {
         im += v;
     } else {
-        re = fmaf(v, cos16(j), re);
-        im = fmaf(-v, sin16(j), im);
+        re = fma_t(v, cos16<T>(j), re);
+        im = fma_t(-v, sin16<T>(j), im);
     }
 }
 
 // re*cos(2 pi J/16) - im*sin(2 pi J/16), trivial angles without multiplies.
-template <int J>
-__device__ __forceinline__ float rotate_real(float re, float im) {
+template <int J, typename T>
+__device__ __forceinline__ T rotate_real(T re, T im) {
     constexpr int j = J & 15;
     if constexpr (j == 0) {
         return re;
@@ -92,7 +99,7 @@ __device__ __forceinline__ float rotate_real(float re, float im) {
     } else if constexpr (j == 12) {
         return im;
     } else {
-        return fmaf(re, cos16(j), -im * sin16(j));
+        return fma_t(re, cos16<T>(j), -im * sin16<T>(j));
     }
 }
 
@@ -100,20 +107,19 @@ __device__ __forceinline__ float rotate_real(float re, float im) {
 // (im[0] and im[G/2] are zero and not written).  Decimation in frequency:
 // u_h = x_h + x_{h+G/2} carries the even frequencies (a length-G/2 real DFT),
 // v_h = x_h - x_{h+G/2} the odd ones.
-template <int G>
+template <int G, typename T = float>
 struct RealDft {
     static_assert(G >= 4 && (G & (G - 1)) == 0, "G must be a power of two >= 4");
-    __device__ __forceinline__ static void run(const float (&x)[G], float (&re)[G / 2 + 1],
-                                               float (&im)[G / 2 + 1]) {
+    __device__ __forceinline__ static void run(const T (&x)[G], T (&re)[G / 2 + 1], T (&im)[G / 2 + 1]) {
         constexpr int H = G / 2;
-        float u[H], v[H];
+        T u[H], v[H];
 #pragma unroll
         for (int h = 0; h < H; ++h) {
             u[h] = x[h] + x[h + H];
             v[h] = x[h] - x[h + H];
         }
-        float ure[H / 2 + 1], uim[H / 2 + 1];
-        RealDft<H>::run(u, ure, uim);
+        T ure[H / 2 + 1], uim[H / 2 + 1];
+        RealDft<H, T>::run(u, ure, uim);
         static_for<H / 2 + 1>([&](auto kk) {
             constexpr int k = decltype(kk)::value;
             re[2 * k] = ure[k];
@@ -122,19 +128,19 @@ struct RealDft {
         // odd frequencies k = 1, 3, ..., H-1
         static_for<H / 2>([&](auto jj) {
             constexpr int k = 2 * decltype(jj)::value + 1;
-            float r = 0.0f, i = 0.0f;
+            T r = T(0), i = T(0);
             static_for<H>([&](auto hh) {
                 constexpr int h = decltype(hh)::value;
-                twiddle_acc<((h * k) % G) * (16 / G)>(v[h], r, i);
+                twiddle_acc<((h * k) % G) * (16 / G), T>(v[h], r, i);
             });
             re[k] = r;
             im[k] = i;
         });
     }
 };
-template <>
-struct RealDft<2> {
-    __device__ __forceinline__ static void run(const float (&x)[2], float (&re)[2], float (&im)[2]) {
+template <typename T>
+struct RealDft<2, T> {
+    __device__ __forceinline__ static void run(const T (&x)[2], T (&re)[2], T (&im)[2]) {
         re[0] = x[0] + x[1];
         re[1] = x[0] - x[1];
         (void)im;
@@ -145,13 +151,13 @@ struct RealDft<2> {
 //   y_g = z[0] + (-1)^g z[1] + sum_{0<k<G/2} (z[2k] cos(2pi gk/G) - z[2k+1] sin(2pi gk/G))
 // (i.e. 1/G folded into the real planes and 2/G into the complex ones).
 // Even/odd split over k: y_g = E_g + O_g, y_{g+G/2} = E_g - O_g.
-template <int G>
+template <int G, typename T = float>
 struct RealIdft {
     static_assert(G >= 4 && (G & (G - 1)) == 0, "G must be a power of two >= 4");
-    __device__ __forceinline__ static void run(const float (&z)[G], float (&y)[G]) {
+    __device__ __forceinline__ static void run(const T (&z)[G], T (&y)[G]) {
         constexpr int H = G / 2;
         // even frequencies form a length-H spectrum in plane order
-        float ze[H];
+        T ze[H];
         ze[0] = z[0];
         ze[1] = z[1];
         static_for<H / 2 - 1>([&](auto jj) {
@@ -159,33 +165,33 @@ struct RealIdft {
             ze[2 * k2] = z[4 * k2];
             ze[2 * k2 + 1] = z[4 * k2 + 1];
         });
-        float e[H];
-        RealIdft<H>::run(ze, e);
+        T e[H];
+        RealIdft<H, T>::run(ze, e);
         static_for<H>([&](auto gg) {
             constexpr int g = decltype(gg)::value;
-            float o = 0.0f;
+            T o = T(0);
             static_for<H / 2>([&](auto jj) {
                 constexpr int k = 2 * decltype(jj)::value + 1;
-                o += rotate_real<((g * k) % G) * (16 / G)>(z[2 * k], z[2 * k + 1]);
+                o += rotate_real<((g * k) % G) * (16 / G), T>(z[2 * k], z[2 * k + 1]);
             });
             y[g] = e[g] + o;
             y[g + H] = e[g] - o;
         });
     }
 };
-template <>
-struct RealIdft<2> {
-    __device__ __forceinline__ static void run(const float (&z)[2], float (&y)[2]) {
+template <typename T>
+struct RealIdft<2, T> {
+    __device__ __forceinline__ static void run(const T (&z)[2], T (&y)[2]) {
         y[0] = z[0] + z[1];
         y[1] = z[0] - z[1];
     }
 };
 
 // Forward transform straight into plane order.
-template <int G>
-__device__ __forceinline__ void rdft_planes(const float (&x)[G], float (&p)[G]) {
-    float re[G / 2 + 1], im[G / 2 + 1];
-    RealDft<G>::run(x, re, im);
+template <int G, typename T>
+__device__ __forceinline__ void rdft_planes(const T (&x)[G], T (&p)[G]) {
+    T re[G / 2 + 1], im[G / 2 + 1];
+    RealDft<G, T>::run(x, re, im);
     p[0] = re[0];
     p[1] = re[G / 2];
 #pragma unroll
