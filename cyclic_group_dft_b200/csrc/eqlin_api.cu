@@ -44,8 +44,8 @@ int cuda_fail(cudaError_t e, const char* what) {
 
 struct Plan {
     int path = kPathF32;
-    int nK = 0, rows = 0, n_oc = 0, BN = 0, stages = 0;
-    uint32_t w_region_bytes = 0, w_img_bytes = 0;
+    int nK = 0, rows = 0, n_oc = 0, BN = 0, stages = 0, TG = 0, ycols_pad = 0;
+    uint32_t w_region_bytes = 0, w_img_bytes = 0, ystage_bytes = 0;
     size_t smem_bytes = 0;
     size_t img_alloc_bytes = 0;
 };
@@ -56,7 +56,13 @@ int plan_tc_g(int64_t Cout, int64_t Cin, size_t max_smem, Plan* pl) {
     pl->nK = static_cast<int>((Cin + eqlin::kChunkK - 1) / eqlin::kChunkK);
     pl->n_oc = static_cast<int>((Cout + eqlin::kMmaM - 1) / eqlin::kMmaM);
     pl->BN = S::BN;
-    const size_t fixed = kSmemAlignSlack + kSmemCtlBytes;
+    pl->TG = S::TG;
+    // y staging: 4 buffers (2 per epilogue half) of TG rows x the chunk's y columns
+    const int64_t chunk_rows = std::min<int64_t>(Cout, eqlin::kMmaM);
+    pl->ycols_pad = static_cast<int>((chunk_rows * G + eqlin::tc::kYBoxCols - 1) / eqlin::tc::kYBoxCols *
+                                     eqlin::tc::kYBoxCols);
+    pl->ystage_bytes = static_cast<uint32_t>(S::TG * pl->ycols_pad * 2);
+    const size_t fixed = kSmemAlignSlack + kSmemCtlBytes + 4 * static_cast<size_t>(pl->ystage_bytes);
     if (pl->n_oc == 1) {
         // weights resident in shared memory for the whole kernel
         const int rows = static_cast<int>((Cout + 7) / 8 * 8);
@@ -116,8 +122,8 @@ int check_shape_impl(int64_t Cout, int64_t Cin, int64_t G, int w_dtype, int io_d
     if (Cout <= 0 || Cin <= 0 || G <= 0) return fail(EQLIN_ERR_INVALID_ARG, "sizes must be positive");
     if (G != 2 && G != 4 && G != 8 && G != 16) return fail(EQLIN_ERR_UNSUPPORTED, "G must be 2, 4, 8 or 16");
     if (Cout > kMaxChannels || Cin > kMaxChannels) return fail(EQLIN_ERR_UNSUPPORTED, "channel count above 65536");
-    if (io_dtype == EQLIN_BF16 && (Cin * G) % 8 != 0)
-        return fail(EQLIN_ERR_UNSUPPORTED, "bf16 I/O needs Cin*G to be a multiple of 8 (16-byte rows)");
+    if (io_dtype == EQLIN_BF16 && ((Cin * G) % 8 != 0 || (Cout * G) % 8 != 0))
+        return fail(EQLIN_ERR_UNSUPPORTED, "bf16 I/O needs Cin*G and Cout*G to be multiples of 8 (16-byte rows)");
     return EQLIN_OK;
 }
 
@@ -365,6 +371,14 @@ int eqlin_forward(const eqlin_handle* h, const void* x, void* y, int64_t N, void
                             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return fail(EQLIN_ERR_CUDA, "cuTensorMapEncodeTiled failed for x");
+        CUtensorMap ymap;
+        cuuint64_t ydims[2] = {static_cast<cuuint64_t>(h->Cout * G), static_cast<cuuint64_t>(N)};
+        cuuint64_t ystrides[1] = {static_cast<cuuint64_t>(h->Cout * G * 2)};
+        cuuint32_t ybox[2] = {static_cast<cuuint32_t>(eqlin::tc::kYBoxCols), static_cast<cuuint32_t>(pl.TG)};
+        r = encode(&ymap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, ydims, ystrides, ybox, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return fail(EQLIN_ERR_CUDA, "cuTensorMapEncodeTiled failed for y");
         TcParams p;
         p.w_img = h->w_img;
         p.bias = h->has_bias ? h->bias_f32 : nullptr;
@@ -379,6 +393,8 @@ int eqlin_forward(const eqlin_handle* h, const void* x, void* y, int64_t N, void
         p.n_work = static_cast<int>(n_tiles * pl.n_oc);
         p.stages = pl.stages;
         p.w_region_bytes = pl.w_region_bytes;
+        p.ystage_bytes = pl.ystage_bytes;
+        p.ycols_pad = pl.ycols_pad;
         p.w_img_bytes = pl.w_img_bytes;
         p.timeout_ns = h->timeout_ns;
         const unsigned grid = static_cast<unsigned>(std::min<long long>(p.n_work, h->sm_count));
@@ -387,9 +403,9 @@ int eqlin_forward(const eqlin_handle* h, const void* x, void* y, int64_t N, void
 #define EQLIN_LAUNCH(GG)                                                                                     \
     case GG:                                                                                                 \
         if (streamed)                                                                                        \
-            eqlin::eqlin_fwd_tc_kernel<GG, true><<<grid, eqlin::tc::kThreads, pl.smem_bytes, st>>>(map, p);  \
+            eqlin::eqlin_fwd_tc_kernel<GG, true><<<grid, eqlin::tc::kThreads, pl.smem_bytes, st>>>(map, ymap, p); \
         else                                                                                                 \
-            eqlin::eqlin_fwd_tc_kernel<GG, false><<<grid, eqlin::tc::kThreads, pl.smem_bytes, st>>>(map, p); \
+            eqlin::eqlin_fwd_tc_kernel<GG, false><<<grid, eqlin::tc::kThreads, pl.smem_bytes, st>>>(map, ymap, p); \
         break;
             EQLIN_LAUNCH(2)
             EQLIN_LAUNCH(4)

@@ -22,10 +22,13 @@
 //               (G*BN = 256 columns each) alternate between work items, so the MMAs of
 //               one tile overlap the epilogue of the previous one.
 //   warps 0-7   epilogue: tcgen05.ld of all G planes of a token group, inverse real DFT
-//               (1/G and 2/G are folded into W^), + bias, round to bf16 and store
-//               y[n, o, 0..G-1] directly: a warp writes 32 consecutive o -> one
-//               contiguous run of 32*G*2 bytes per token.  Warps w and w+4 share TMEM
-//               lane quarter w and split the tile's tokens.
+//               (1/G and 2/G are folded into W^), + bias, round to bf16, write the
+//               group's y rows [TG tokens x Cout*G] into a shared-memory staging tile
+//               (a warp writes 32 consecutive o -> one contiguous 32*G*2-byte run), and
+//               one thread per half stores the tile with TMA (rows past N and columns
+//               past Cout*G are clipped by the tensor map).  Warps w and w+4 share TMEM
+//               lane quarter w and split the tile's tokens; each half double-buffers
+//               its staging tile so the TMA store of one group overlaps the next.
 // All waits are bounded (globaltimer); on expiry the kernel records EQLIN_ERR_TIMEOUT
 // in the status word, every role leaves its loop, in-flight copies and MMAs are
 // drained with bounded waits, and TMEM is freed before exit.
@@ -53,6 +56,8 @@ struct TcParams {
     int n_work;             // n_tiles * n_oc
     int stages;             // smem ring depth
     uint32_t w_region_bytes;  // smem reserved for resident weights (0 when streamed)
+    uint32_t ystage_bytes;    // one y staging buffer (TG rows x ycols_pad bf16)
+    int ycols_pad;            // staged y columns per group, multiple of kYBoxCols
     uint32_t w_img_bytes;     // bytes of the resident image to copy
     unsigned long long timeout_ns;
 };
@@ -68,6 +73,8 @@ constexpr int kWarpMma = 13;
 constexpr int kNumAcc = 2;       // TMEM accumulator buffers
 constexpr int kBarDft = 1;   // named barrier ids (0 is __syncthreads)
 constexpr int kBarEpi = 2;
+constexpr int kBarEpiHalf0 = 3;  // 3 and 4: one per epilogue half (128 threads)
+constexpr int kYBoxCols = 128;   // y TMA store box: 128 bf16 columns (256 B) x TG rows
 
 template <int G>
 struct Shape {
@@ -185,9 +192,13 @@ __device__ __forceinline__ void dft_chunk(uint8_t* xs, int dft_tid) {
 // ------------------------------------------------------------ epilogue role
 // Warp (q, half): TMEM lane quarter q (output rows 32q..32q+31 of the chunk), tokens
 // [half*BN/2, (half+1)*BN/2) of the tile held in accumulator `acc` (column base).
+// `active`: this warp's quarter holds valid output rows (inactive warps still take part
+// in the half's barriers).  `ystage`: this half's two staging buffers; `ybuf` alternates.
+// `leader`: the one thread of the half that issues and tracks the TMA stores.
 template <int G>
-__device__ __forceinline__ void epilogue_tile(const TcParams& p, uint32_t acc, int q, int half,
-                                              int lane, long long n0, int oc) {
+__device__ __forceinline__ void epilogue_tile(const TcParams& p, const CUtensorMap* tmap_y, uint32_t acc,
+                                              int q, int half, int lane, long long n0, int oc, bool active,
+                                              uint8_t* ystage, int& ybuf, bool leader) {
     using S = Shape<G>;
     constexpr int TG = S::TG;
     const int o_local = q * 32 + lane;
@@ -196,39 +207,74 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, uint32_t acc, i
     const float b = (p.bias != nullptr && valid_o) ? p.bias[o] : 0.0f;
     const uint32_t lane_addr = acc + (static_cast<uint32_t>(q * 32) << 16);
     const int t0 = half * (S::BN / 2);
+    const uint32_t bar_half = kBarEpiHalf0 + half;
+    // column of this lane's first output inside the staged rows, and its box / offset
+    const int col = o_local * G;
+    const int box = col / kYBoxCols, col_in = col % kYBoxCols;
+    const int valid_rows = min(kMmaM, p.Cout - oc * kMmaM);
+    const int n_boxes = (valid_rows * G + kYBoxCols - 1) / kYBoxCols;
 #pragma unroll 1
     for (int j = 0; j < S::BN / 2 / TG; ++j) {
         uint32_t r[G][TG];
+        if (active) {
 #pragma unroll
-        for (int pl = 0; pl < G; ++pl) ptx::tmem_ld_32x32b<TG>(lane_addr + pl * S::BN + t0 + j * TG, r[pl]);
-        ptx::tmem_wait_ld();
+            for (int pl = 0; pl < G; ++pl) ptx::tmem_ld_32x32b<TG>(lane_addr + pl * S::BN + t0 + j * TG, r[pl]);
+            ptx::tmem_wait_ld();
 #pragma unroll
-        for (int t = 0; t < TG; ++t) {
-            const long long n = n0 + t0 + j * TG + t;
-            float z[G], yv[G];
+            for (int pl = 0; pl < G; ++pl) ptx::tmem_regs_ready<TG>(r[pl]);
+        }
+        // the buffer about to be written was last stored two groups ago: wait until the
+        // TMA engine has read it, then release the half
+        if (leader) ptx::bulk_wait_group_read<1>();
+        ptx::named_bar_sync(bar_half, 128);
+        uint8_t* buf = ystage + static_cast<size_t>(ybuf) * p.ystage_bytes;
+        if (active && valid_o) {
 #pragma unroll
-            for (int pl = 0; pl < G; ++pl) z[pl] = __uint_as_float(r[pl][t]);
-            z[0] += b;  // the DC term appears with weight 1 in every output
-            RealIdft<G>::run(z, yv);
-            if (valid_o && n < p.N) {
-                __nv_bfloat16* dst = p.y + (n * p.Cout + o) * G;
-                if constexpr (G == 2) {
-                    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(yv[0], yv[1]);
-                } else if constexpr (G == 4) {
-                    *reinterpret_cast<uint2*>(dst) =
-                        make_uint2(pack_bf16x2(yv[0], yv[1]), pack_bf16x2(yv[2], yv[3]));
+            for (int t = 0; t < TG; ++t) {
+                float z[G], yv[G];
+#pragma unroll
+                for (int pl = 0; pl < G; ++pl) z[pl] = __uint_as_float(r[pl][t]);
+                z[0] += b;  // the DC term appears with weight 1 in every output
+                RealIdft<G>::run(z, yv);
+                if constexpr (G <= 4) {
+                    // the lane's 2G bytes sit inside one box (128 % G == 0)
+                    uint8_t* dst = buf + box * (TG * kYBoxCols * 2) + t * (kYBoxCols * 2) + col_in * 2;
+                    if constexpr (G == 2) {
+                        *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(yv[0], yv[1]);
+                    } else {
+                        *reinterpret_cast<uint2*>(dst) =
+                            make_uint2(pack_bf16x2(yv[0], yv[1]), pack_bf16x2(yv[2], yv[3]));
+                    }
                 } else {
+                    // G/8 pieces of 16 B (8 columns); a piece never straddles a box
 #pragma unroll
                     for (int c = 0; c < G / 8; ++c) {
-                        *reinterpret_cast<uint4*>(dst + 8 * c) = make_uint4(
-                            pack_bf16x2(yv[8 * c + 0], yv[8 * c + 1]),
-                            pack_bf16x2(yv[8 * c + 2], yv[8 * c + 3]),
-                            pack_bf16x2(yv[8 * c + 4], yv[8 * c + 5]),
-                            pack_bf16x2(yv[8 * c + 6], yv[8 * c + 7]));
+                        const int cc = col + 8 * c;
+                        uint8_t* dst = buf + (cc / kYBoxCols) * (TG * kYBoxCols * 2) + t * (kYBoxCols * 2) +
+                                       (cc % kYBoxCols) * 2;
+                        *reinterpret_cast<uint4*>(dst) = make_uint4(
+                            pack_bf16x2(yv[8 * c + 0], yv[8 * c + 1]), pack_bf16x2(yv[8 * c + 2], yv[8 * c + 3]),
+                            pack_bf16x2(yv[8 * c + 4], yv[8 * c + 5]), pack_bf16x2(yv[8 * c + 6], yv[8 * c + 7]));
                     }
                 }
             }
         }
+        ptx::fence_proxy_async_smem();
+        ptx::named_bar_sync(bar_half, 128);
+        if (leader) {
+            // every store starts inside the tensor: rows past N and columns past Cout*G
+            // of a started box are clipped by the tensor map, boxes that would start
+            // outside are not issued
+            const long long row = n0 + t0 + j * TG;
+            if (row < p.N) {
+                const uint32_t src = ptx::smem_u32(buf);
+                for (int bx = 0; bx < n_boxes; ++bx)
+                    ptx::tma_store_2d(tmap_y, src + bx * (TG * kYBoxCols * 2), oc * kMmaM * G + bx * kYBoxCols,
+                                      static_cast<int>(row));
+            }
+            ptx::bulk_commit_group();
+        }
+        ybuf ^= 1;
     }
 }
 
@@ -236,7 +282,8 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, uint32_t acc, i
 
 template <int G, bool STREAM_W>
 __global__ void __launch_bounds__(tc::kThreads, 1)
-    eqlin_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const TcParams p) {
+    eqlin_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_y,
+                        const TcParams p) {
     using S = tc::Shape<G>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -245,7 +292,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     constexpr uint32_t STAGE_BYTES = S::XCHUNK_BYTES + (STREAM_W ? S::WSTAGE_BYTES : 0);
     constexpr uint32_t STAGE_TX = STAGE_BYTES;   // every byte of a stage arrives by copy
     const int NS = p.stages;
-    uint8_t* stage0 = smem + p.w_region_bytes;
+    uint8_t* ystage0 = smem + p.w_region_bytes;                 // 4 y staging buffers (2 per half)
+    uint8_t* stage0 = ystage0 + 4 * static_cast<size_t>(p.ystage_bytes);
     uint64_t* bars = reinterpret_cast<uint64_t*>(stage0 + static_cast<size_t>(NS) * STAGE_BYTES);
     tc::Ctl* ctl = reinterpret_cast<tc::Ctl*>(bars + 3 * NS + 2 * tc::kNumAcc + 2);
 
@@ -280,7 +328,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         ptx::tmem_alloc(ptx::smem_u32(&ctl->tmem_base), S::TMEM_COLS);
         ptx::tmem_relinquish();
     }
-    if (warp == tc::kWarpProducer && lane == 0) ptx::prefetch_tmap(&tmap_x);
+    if (warp == tc::kWarpProducer && lane == 0) {
+        ptx::prefetch_tmap(&tmap_x);
+        ptx::prefetch_tmap(&tmap_y);
+    }
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
@@ -384,12 +435,19 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                         wsub = static_cast<uint32_t>(p.rows) * kPlaneRowBytes;
                         wb = s_w + static_cast<uint32_t>(c * G) * wsub;
                     }
+                    // descriptors differ only in their start-address field: build each
+                    // one as (constant high half, low half + byte offset / 16)
+                    const uint32_t a_lo = ptx::sdesc_sw64_lo(wb), b_lo = ptx::sdesc_sw64_lo(xb);
+                    const uint32_t wsub16 = wsub >> 4;
+                    const uint32_t acc_first = c > 0 ? 1u : 0u;
 #pragma unroll
                     for (int ks = 0; ks < kChunkK / 16; ++ks) {
-                        const uint32_t acc0 = (c > 0 || ks > 0) ? 1u : 0u;
-                        auto A = [&](int pl) { return ptx::sdesc_kmajor_sw64(wb + pl * wsub + ks * 32); };
+                        const uint32_t acc0 = ks > 0 ? 1u : acc_first;
+                        auto A = [&](int pl) {
+                            return ptx::sdesc_sw64_from_lo(a_lo + static_cast<uint32_t>(pl) * wsub16 + ks * 2);
+                        };
                         auto B = [&](int pl) {
-                            return ptx::sdesc_kmajor_sw64(xb + pl * S::PLANE_BYTES + ks * 32);
+                            return ptx::sdesc_sw64_from_lo(b_lo + (pl * S::PLANE_BYTES + ks * 32) / 16);
                         };
                         auto D = [&](int pl) { return acc_base + static_cast<uint32_t>(pl * S::BN); };
                         // real frequencies k = 0 and k = G/2
@@ -443,6 +501,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue warps
+        const int half = warp >> 2;
+        const bool leader = (warp & 3) == 0 && lane == 0;
+        uint8_t* ystage = ystage0 + static_cast<size_t>(2 * half) * p.ystage_bytes;
+        int ybuf = 0;
         int it = 0;
         for (int wk = blockIdx.x; wk < p.n_work; wk += gridDim.x, ++it) {
             const int abuf = it & 1;
@@ -451,11 +513,15 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
             if (!ptx::named_bar_and(tc::kBarEpi, tc::kEpiThreads, got)) break;
             ptx::tc_fence_after();
             const int tile = wk / p.n_oc, oc = wk % p.n_oc;
-            tc::epilogue_tile<G>(p, tmem_base + static_cast<uint32_t>(abuf * S::ACC_COLS), warp & 3,
-                                 warp >> 2, lane, static_cast<long long>(tile) * S::BN, oc);
+            // warps whose lane quarter holds no valid output row skip the math
+            const bool active = oc * kMmaM + (warp & 3) * 32 < p.Cout;
+            tc::epilogue_tile<G>(p, &tmap_y, tmem_base + static_cast<uint32_t>(abuf * S::ACC_COLS), warp & 3,
+                                 half, lane, static_cast<long long>(tile) * S::BN, oc, active, ystage, ybuf, leader);
             ptx::tc_fence_before();
             ptx::mbar_arrive(bar_acc_empty(abuf));
         }
+        // the y stores must be complete (not only read) before the CTA exits
+        if (leader) ptx::bulk_wait_group<0>();
     }
 
     ptx::tc_fence_before();

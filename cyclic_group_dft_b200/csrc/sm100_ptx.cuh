@@ -85,6 +85,27 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* m, 
         "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(bar)
         : "memory");
 }
+// 2-D tiled TMA store shared -> global (bulk async-group completion).  Rows or columns
+// of the box outside the tensor are not written.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, uint32_t src, int32_t c0, int32_t c1) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                     reinterpret_cast<uint64_t>(m)),
+                 "r"(c0), "r"(c1), "r"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until at most N committed bulk groups of this thread still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Wait until at most N committed bulk groups of this thread are incomplete.
+template <int N>
+__device__ __forceinline__ void bulk_wait_group() {
+    asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
 // Plain bulk copy global -> shared (16-B aligned addresses, size multiple of 16).
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
                                           uint32_t bar) {
@@ -138,6 +159,14 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
 }
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+// Ties registers filled by tcgen05.ld to a preceding tmem_wait_ld(): an empty volatile
+// asm per register stays ordered after the wait, and every later use of the register
+// depends on it, so no use can be scheduled before the data is valid.
+template <int N>
+__device__ __forceinline__ void tmem_regs_ready(uint32_t (&r)[N]) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
 }
 
 // 32 lanes x 32 bits x N consecutive columns: thread t gets lane (base+t), columns [col, col+N).
@@ -193,6 +222,15 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_sw64(uint32_t start) {
     d |= static_cast<uint64_t>(1) << 46;                 // [46,48): descriptor version 1 (sm_100)
     d |= static_cast<uint64_t>(4) << 61;                 // [61,64): layout 4 = SWIZZLE_64B
     return d;                                            // base offset 0, LBO mode 0
+}
+
+// The same descriptor split in halves: only the start-address field (low 14 bits)
+// varies between operands, so the issuing loop adds (byte offset >> 4) to the low
+// half and pairs it with the constant high half.
+__device__ __forceinline__ uint32_t sdesc_sw64_lo(uint32_t start) { return (1u << 16) | (start >> 4); }
+constexpr uint32_t kSdescSw64Hi = (512u >> 4) | (1u << 14) | (4u << 29);
+__device__ __forceinline__ uint64_t sdesc_sw64_from_lo(uint32_t lo) {
+    return (static_cast<uint64_t>(kSdescSw64Hi) << 32) | lo;
 }
 
 }  // namespace ptx

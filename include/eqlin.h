@@ -28,8 +28,8 @@
  *     a failed call launches nothing and changes nothing.  Nothing throws, aborts
  *     or prints.  eqlin_last_error() describes the latest failure of the
  *     calling thread.
- *   - Supported: G in {2, 4, 8, 16}; Cin, Cout >= 1; Cin*G a multiple of 8
- *     (16-byte rows for the TMA engine).  io_dtype EQLIN_BF16 runs the fused
+ *   - Supported: G in {2, 4, 8, 16}; Cin, Cout >= 1; for bf16 I/O Cin*G and
+ *     Cout*G multiples of 8 (16-byte rows for the TMA engine).  io_dtype EQLIN_BF16 runs the fused
  *     tcgen05 (tensor-core) kernel; EQLIN_F32 runs a fused FFMA kernel.
  *   - Requires a compute-capability 10.0 device (B200).
  */
@@ -83,7 +83,7 @@ typedef enum {
  * The handle owns device memory for the transformed weights (bf16 tensor-core
  * image and/or fp32 planes), an fp32 copy of the bias and a device status word.
  * Errors: INVALID_ARG (null w/out, non-positive sizes, unknown dtype),
- * UNSUPPORTED (G not in {2,4,8,16}, Cin*G not a multiple of 8 for bf16 I/O,
+ * UNSUPPORTED (G not in {2,4,8,16}, Cin*G or Cout*G not a multiple of 8 for bf16 I/O,
  * not an sm_100 device, shape too large for shared memory), MISALIGNED (w or
  * bias not aligned to its element size), OOM, CUDA.
  */

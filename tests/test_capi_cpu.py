@@ -44,6 +44,7 @@ def test_version_and_status_strings():
     ((96, 96, 32, eq.EQLIN_BF16, eq.EQLIN_BF16), eq.EQLIN_ERR_UNSUPPORTED),
     ((3, 3, 2, eq.EQLIN_BF16, eq.EQLIN_BF16), eq.EQLIN_ERR_UNSUPPORTED),   # Cin*G % 8
     ((3, 3, 2, eq.EQLIN_F32, eq.EQLIN_F32), eq.EQLIN_OK),                  # fine for fp32
+    ((3, 8, 2, eq.EQLIN_BF16, eq.EQLIN_BF16), eq.EQLIN_ERR_UNSUPPORTED),   # Cout*G % 8
     ((0, 4, 4, eq.EQLIN_BF16, eq.EQLIN_BF16), eq.EQLIN_ERR_INVALID_ARG),
     ((4, -1, 4, eq.EQLIN_BF16, eq.EQLIN_BF16), eq.EQLIN_ERR_INVALID_ARG),
     ((4, 4, 4, 7, eq.EQLIN_BF16), eq.EQLIN_ERR_INVALID_ARG),
