@@ -44,15 +44,17 @@ int cuda_fail(cudaError_t e, const char* what) {
 
 struct Plan {
     int path = kPathF32;
+    int nacc = 2;  // TMEM accumulator buffers (tcgen05 path)
     int nK = 0, rows = 0, n_oc = 0, BN = 0, stages = 0, TG = 0, ycols_pad = 0;
     uint32_t w_region_bytes = 0, w_img_bytes = 0, ystage_bytes = 0;
     size_t smem_bytes = 0;
     size_t img_alloc_bytes = 0;
 };
 
-template <int G>
+template <int G, int NACC>
 int plan_tc_g(int64_t Cout, int64_t Cin, size_t max_smem, Plan* pl) {
-    using S = eqlin::tc::Shape<G>;
+    using S = eqlin::tc::Shape<G, NACC>;
+    pl->nacc = NACC;
     pl->nK = static_cast<int>((Cin + eqlin::kChunkK - 1) / eqlin::kChunkK);
     pl->n_oc = static_cast<int>((Cout + eqlin::kMmaM - 1) / eqlin::kMmaM);
     pl->BN = S::BN;
@@ -98,6 +100,12 @@ int plan_tc_g(int64_t Cout, int64_t Cin, size_t max_smem, Plan* pl) {
     return EQLIN_OK;
 }
 
+// Accumulator buffers per group order (measured on B200; see the design notes).
+int default_acc_buffers(int G) {
+    (void)G;
+    return 2;
+}
+
 int plan_for(int64_t Cout, int64_t Cin, int64_t G, int io_dtype, size_t max_smem, Plan* pl) {
     if (io_dtype == EQLIN_F32) {
         const size_t smem = static_cast<size_t>(eqlin::kF32Tokens) * G * Cin * sizeof(double);
@@ -107,11 +115,16 @@ int plan_for(int64_t Cout, int64_t Cin, int64_t G, int io_dtype, size_t max_smem
         pl->smem_bytes = smem;
         return EQLIN_OK;
     }
+    int nacc = default_acc_buffers(static_cast<int>(G));
+    if (const char* e = std::getenv("EQLIN_ACC_BUFFERS")) {
+        if (e[0] == '1') nacc = 1;
+        if (e[0] == '2') nacc = 2;
+    }
     switch (G) {
-        case 2: return plan_tc_g<2>(Cout, Cin, max_smem, pl);
-        case 4: return plan_tc_g<4>(Cout, Cin, max_smem, pl);
-        case 8: return plan_tc_g<8>(Cout, Cin, max_smem, pl);
-        case 16: return plan_tc_g<16>(Cout, Cin, max_smem, pl);
+        case 2: return nacc == 1 ? plan_tc_g<2, 1>(Cout, Cin, max_smem, pl) : plan_tc_g<2, 2>(Cout, Cin, max_smem, pl);
+        case 4: return nacc == 1 ? plan_tc_g<4, 1>(Cout, Cin, max_smem, pl) : plan_tc_g<4, 2>(Cout, Cin, max_smem, pl);
+        case 8: return nacc == 1 ? plan_tc_g<8, 1>(Cout, Cin, max_smem, pl) : plan_tc_g<8, 2>(Cout, Cin, max_smem, pl);
+        case 16: return nacc == 1 ? plan_tc_g<16, 1>(Cout, Cin, max_smem, pl) : plan_tc_g<16, 2>(Cout, Cin, max_smem, pl);
         default: return fail(EQLIN_ERR_UNSUPPORTED, "G must be 2, 4, 8 or 16");
     }
 }
@@ -141,18 +154,38 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-template <int G, bool STREAM>
-void* tc_kernel_ptr() {
-    return reinterpret_cast<void*>(&eqlin::eqlin_fwd_tc_kernel<G, STREAM>);
+using TcLaunch = void (*)(unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& mx,
+                          const CUtensorMap& my, const TcParams& p);
+
+template <int G, bool STREAM, int NACC>
+void tc_launch(unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& mx, const CUtensorMap& my,
+               const TcParams& p) {
+    eqlin::eqlin_fwd_tc_kernel<G, STREAM, NACC><<<grid, eqlin::tc::kThreads, smem, st>>>(mx, my, p);
 }
 
-void* tc_kernel_for(int G, bool stream) {
+struct TcEntry {
+    TcLaunch launch = nullptr;
+    void* kernel = nullptr;
+};
+
+template <int G, bool STREAM, int NACC>
+TcEntry tc_entry() {
+    return {&tc_launch<G, STREAM, NACC>, reinterpret_cast<void*>(&eqlin::eqlin_fwd_tc_kernel<G, STREAM, NACC>)};
+}
+
+template <int G>
+TcEntry tc_entry_g(bool stream, int nacc) {
+    if (stream) return nacc == 1 ? tc_entry<G, true, 1>() : tc_entry<G, true, 2>();
+    return nacc == 1 ? tc_entry<G, false, 1>() : tc_entry<G, false, 2>();
+}
+
+TcEntry tc_entry_for(int G, bool stream, int nacc) {
     switch (G) {
-        case 2: return stream ? tc_kernel_ptr<2, true>() : tc_kernel_ptr<2, false>();
-        case 4: return stream ? tc_kernel_ptr<4, true>() : tc_kernel_ptr<4, false>();
-        case 8: return stream ? tc_kernel_ptr<8, true>() : tc_kernel_ptr<8, false>();
-        case 16: return stream ? tc_kernel_ptr<16, true>() : tc_kernel_ptr<16, false>();
-        default: return nullptr;
+        case 2: return tc_entry_g<2>(stream, nacc);
+        case 4: return tc_entry_g<4>(stream, nacc);
+        case 8: return tc_entry_g<8>(stream, nacc);
+        case 16: return tc_entry_g<16>(stream, nacc);
+        default: return {};
     }
 }
 
@@ -169,7 +202,7 @@ void* f32_kernel_for(int G) {
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 template <int G>
-int box_elems() { return eqlin::tc::Shape<G>::BOX_ELEMS; }
+int box_elems() { return eqlin::tc::Shape<G, 2>::BOX_ELEMS; }  // independent of the accumulator count
 
 int tc_box_elems(int G) {
     switch (G) {
@@ -318,8 +351,9 @@ int eqlin_prepare_weights(const void* w, const void* bias, int64_t Cout, int64_t
         free_handle(h);
         return s;
     }
-    void* k = plan.path == kPathF32 ? f32_kernel_for(static_cast<int>(G))
-                                    : tc_kernel_for(static_cast<int>(G), plan.path == kPathStreamed);
+    void* k = plan.path == kPathF32
+                  ? f32_kernel_for(static_cast<int>(G))
+                  : tc_entry_for(static_cast<int>(G), plan.path == kPathStreamed, plan.nacc).kernel;
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(plan.smem_bytes));
     if (e != cudaSuccess) {
         free_handle(h);
@@ -398,22 +432,9 @@ int eqlin_forward(const eqlin_handle* h, const void* x, void* y, int64_t N, void
         p.w_img_bytes = pl.w_img_bytes;
         p.timeout_ns = h->timeout_ns;
         const unsigned grid = static_cast<unsigned>(std::min<long long>(p.n_work, h->sm_count));
-        const bool streamed = pl.path == kPathStreamed;
-        switch (G) {
-#define EQLIN_LAUNCH(GG)                                                                                     \
-    case GG:                                                                                                 \
-        if (streamed)                                                                                        \
-            eqlin::eqlin_fwd_tc_kernel<GG, true><<<grid, eqlin::tc::kThreads, pl.smem_bytes, st>>>(map, ymap, p); \
-        else                                                                                                 \
-            eqlin::eqlin_fwd_tc_kernel<GG, false><<<grid, eqlin::tc::kThreads, pl.smem_bytes, st>>>(map, ymap, p); \
-        break;
-            EQLIN_LAUNCH(2)
-            EQLIN_LAUNCH(4)
-            EQLIN_LAUNCH(8)
-            EQLIN_LAUNCH(16)
-#undef EQLIN_LAUNCH
-            default: return fail(EQLIN_ERR_UNSUPPORTED, "G");
-        }
+        const TcEntry entry = tc_entry_for(G, pl.path == kPathStreamed, pl.nacc);
+        if (!entry.launch) return fail(EQLIN_ERR_UNSUPPORTED, "G");
+        entry.launch(grid, pl.smem_bytes, st, map, ymap, p);
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "forward launch");

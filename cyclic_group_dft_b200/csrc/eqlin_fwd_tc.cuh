@@ -70,15 +70,18 @@ constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kWarpDft0 = 8;
 constexpr int kWarpProducer = 12;
 constexpr int kWarpMma = 13;
-constexpr int kNumAcc = 2;       // TMEM accumulator buffers
 constexpr int kBarDft = 1;   // named barrier ids (0 is __syncthreads)
 constexpr int kBarEpi = 2;
 constexpr int kBarEpiHalf0 = 3;  // 3 and 4: one per epilogue half (128 threads)
 constexpr int kYBoxCols = 128;   // y TMA store box: 128 bf16 columns (256 B) x TG rows
 
-template <int G>
+// NACC accumulator buffers of G*BN TMEM columns each share the 512 columns: with two,
+// the MMAs of one tile overlap the epilogue of the previous one; with one, each MMA
+// covers twice the tokens (half the weight-operand traffic and MMA count per token).
+template <int G, int NACC = 2>
 struct Shape {
-    static constexpr int BN = (256 / G) < 128 ? (256 / G) : 128;    // tokens per tile (MMA N)
+    static constexpr int kNumAcc = NACC;
+    static constexpr int BN = (512 / (G * NACC)) < 128 ? (512 / (G * NACC)) : 128;  // tokens per tile (MMA N)
     static constexpr int PLANE_BYTES = BN * kPlaneRowBytes;          // one frequency plane
     static constexpr int XCHUNK_BYTES = G * PLANE_BYTES;             // == BN * 32 * G * 2
     static constexpr int XROW_ELEMS = kChunkK * G;                   // one token row of a chunk
@@ -90,9 +93,12 @@ struct Shape {
     static constexpr int TG = (64 / G) < BN / 2 ? (64 / G) : BN / 2;  // tokens per epilogue group
     static_assert(XCHUNK_BYTES % 1024 == 0, "stage alignment");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N");
-    static_assert(kNumAcc * ACC_COLS <= TMEM_COLS, "TMEM columns");
+    static_assert(NACC * ACC_COLS <= TMEM_COLS, "TMEM columns");
     static_assert((BN / 2) % TG == 0, "epilogue groups");
 };
+
+// suspend-time hint of a waiting thread (it wakes as soon as the phase completes)
+constexpr uint32_t kWaitSleepNs = 20000;
 
 struct Ctl {
     volatile int abort;
@@ -105,8 +111,8 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, Ctl*
     if (ptx::mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = ptx::globaltimer_ns();
     for (uint32_t spin = 1;; ++spin) {
-        if (ptx::mbar_try_wait(bar, parity)) return true;
-        if ((spin & 63u) == 0) {
+        if (ptx::mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
+        if ((spin & 7u) == 0) {
             if (ctl->abort) return false;
             if (ptx::globaltimer_ns() - t0 > timeout_ns) {
                 ctl->abort = 1;
@@ -125,9 +131,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // ---------------------------------------------------------------- DFT role
 // 128 threads.  Unit = one token row x two adjacent channels (2*G bf16).
 // Lanes 0-15 take row r, lanes 16-31 row r+1; lane&15 selects the channel pair.
-template <int G>
+template <int G, int NACC>
 __device__ __forceinline__ void dft_chunk(uint8_t* xs, int dft_tid) {
-    using S = Shape<G>;
+    using S = Shape<G, NACC>;
     constexpr int WORDS = G;                         // 32-bit words per unit (2 ch x G x 2 B / 4)
     constexpr int STEPS = S::BN / 8;                 // 2 rows per step, 4 warps
     const int warp = dft_tid >> 5, lane = dft_tid & 31;
@@ -195,11 +201,11 @@ __device__ __forceinline__ void dft_chunk(uint8_t* xs, int dft_tid) {
 // `active`: this warp's quarter holds valid output rows (inactive warps still take part
 // in the half's barriers).  `ystage`: this half's two staging buffers; `ybuf` alternates.
 // `leader`: the one thread of the half that issues and tracks the TMA stores.
-template <int G>
+template <int G, int NACC>
 __device__ __forceinline__ void epilogue_tile(const TcParams& p, const CUtensorMap* tmap_y, uint32_t acc,
                                               int q, int half, int lane, long long n0, int oc, bool active,
                                               uint8_t* ystage, int& ybuf, bool leader) {
-    using S = Shape<G>;
+    using S = Shape<G, NACC>;
     constexpr int TG = S::TG;
     const int o_local = q * 32 + lane;
     const int o = oc * kMmaM + o_local;
@@ -280,11 +286,11 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, const CUtensorM
 
 }  // namespace tc
 
-template <int G, bool STREAM_W>
+template <int G, bool STREAM_W, int NACC>
 __global__ void __launch_bounds__(tc::kThreads, 1)
     eqlin_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_y,
                         const TcParams p) {
-    using S = tc::Shape<G>;
+    using S = tc::Shape<G, NACC>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -295,7 +301,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     uint8_t* ystage0 = smem + p.w_region_bytes;                 // 4 y staging buffers (2 per half)
     uint8_t* stage0 = ystage0 + 4 * static_cast<size_t>(p.ystage_bytes);
     uint64_t* bars = reinterpret_cast<uint64_t*>(stage0 + static_cast<size_t>(NS) * STAGE_BYTES);
-    tc::Ctl* ctl = reinterpret_cast<tc::Ctl*>(bars + 3 * NS + 2 * tc::kNumAcc + 2);
+    tc::Ctl* ctl = reinterpret_cast<tc::Ctl*>(bars + 3 * NS + 2 * NACC + 2);
 
     const uint32_t s_w = ptx::smem_u32(smem);
     const uint32_t s_stage0 = ptx::smem_u32(stage0);
@@ -303,9 +309,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     auto bar_xhat = [&](int s) { return ptx::smem_u32(bars + NS + s); };
     auto bar_empty = [&](int s) { return ptx::smem_u32(bars + 2 * NS + s); };
     auto bar_acc_full = [&](int a) { return ptx::smem_u32(bars + 3 * NS + a); };
-    auto bar_acc_empty = [&](int a) { return ptx::smem_u32(bars + 3 * NS + tc::kNumAcc + a); };
-    const uint32_t bar_w_full = ptx::smem_u32(bars + 3 * NS + 2 * tc::kNumAcc);
-    const uint32_t bar_drain = ptx::smem_u32(bars + 3 * NS + 2 * tc::kNumAcc + 1);
+    auto bar_acc_empty = [&](int a) { return ptx::smem_u32(bars + 3 * NS + NACC + a); };
+    const uint32_t bar_w_full = ptx::smem_u32(bars + 3 * NS + 2 * NACC);
+    const uint32_t bar_drain = ptx::smem_u32(bars + 3 * NS + 2 * NACC + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -315,7 +321,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
             ptx::mbar_init(bar_xhat(s), 128);
             ptx::mbar_init(bar_empty(s), 1);
         }
-        for (int a = 0; a < tc::kNumAcc; ++a) {
+        for (int a = 0; a < NACC; ++a) {
             ptx::mbar_init(bar_acc_full(a), 1);
             ptx::mbar_init(bar_acc_empty(a), tc::kEpiThreads);
         }
@@ -412,8 +418,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
             uint32_t phase = 0;
             int it = 0;
             for (int wk = blockIdx.x; ok && wk < p.n_work; wk += gridDim.x, ++it) {
-                const int abuf = it & 1;
-                const uint32_t acc_phase = static_cast<uint32_t>(it >> 1) & 1u;
+                const int abuf = it % NACC;
+                const uint32_t acc_phase = static_cast<uint32_t>(it / NACC) & 1u;
                 if (!tc::wait_bounded(bar_acc_empty(abuf), acc_phase ^ 1u, ctl, p.status, p.timeout_ns)) {
                     ok = false;
                     break;
@@ -492,7 +498,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                     ok = false;
                     break;
                 }
-                tc::dft_chunk<G>(stage0 + static_cast<size_t>(stage) * STAGE_BYTES, dft_tid);
+                tc::dft_chunk<G, NACC>(stage0 + static_cast<size_t>(stage) * STAGE_BYTES, dft_tid);
                 ptx::fence_proxy_async_smem();
                 ptx::mbar_arrive(bar_xhat(stage));
                 if (++stage == NS) { stage = 0; phase ^= 1u; }
@@ -507,15 +513,15 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         int ybuf = 0;
         int it = 0;
         for (int wk = blockIdx.x; wk < p.n_work; wk += gridDim.x, ++it) {
-            const int abuf = it & 1;
-            const uint32_t acc_phase = static_cast<uint32_t>(it >> 1) & 1u;
+            const int abuf = it % NACC;
+            const uint32_t acc_phase = static_cast<uint32_t>(it / NACC) & 1u;
             const bool got = tc::wait_bounded(bar_acc_full(abuf), acc_phase, ctl, p.status, p.timeout_ns);
             if (!ptx::named_bar_and(tc::kBarEpi, tc::kEpiThreads, got)) break;
             ptx::tc_fence_after();
             const int tile = wk / p.n_oc, oc = wk % p.n_oc;
             // warps whose lane quarter holds no valid output row skip the math
             const bool active = oc * kMmaM + (warp & 3) * 32 < p.Cout;
-            tc::epilogue_tile<G>(p, &tmap_y, tmem_base + static_cast<uint32_t>(abuf * S::ACC_COLS), warp & 3,
+            tc::epilogue_tile<G, NACC>(p, &tmap_y, tmem_base + static_cast<uint32_t>(abuf * S::ACC_COLS), warp & 3,
                                  half, lane, static_cast<long long>(tile) * S::BN, oc, active, ystage, ybuf, leader);
             ptx::tc_fence_before();
             ptx::mbar_arrive(bar_acc_empty(abuf));
