@@ -50,13 +50,15 @@ _lib.eqlin_device_status.argtypes = [_vp, ctypes.POINTER(_int)]
 _lib.eqlin_get_attr.argtypes = [_vp, _int, ctypes.POINTER(_i64)]
 _lib.eqlin_copy_freq_weights.argtypes = [_vp, ctypes.POINTER(ctypes.c_float), _i64]
 _lib.eqlin_check_shape.argtypes = [_i64, _i64, _i64, _int, _int]
+_lib.eqlin_forward_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _int, _vp]
 _lib.eqlin_status_string.argtypes = [_int]
 _lib.eqlin_status_string.restype = ctypes.c_char_p
 _lib.eqlin_last_error.argtypes = []
 _lib.eqlin_last_error.restype = ctypes.c_char_p
 _lib.eqlin_version.argtypes = []
 for _f in ("eqlin_prepare_weights", "eqlin_forward", "eqlin_destroy", "eqlin_device_status",
-           "eqlin_get_attr", "eqlin_copy_freq_weights", "eqlin_check_shape", "eqlin_version"):
+           "eqlin_get_attr", "eqlin_copy_freq_weights", "eqlin_check_shape", "eqlin_version",
+           "eqlin_forward_noalloc"):
     getattr(_lib, _f).restype = _int
 
 
@@ -251,3 +253,28 @@ def eqlin_copy_freq_weights(h: Handle) -> torch.Tensor:
         dst = ctypes.cast(out.data_ptr(), ctypes.POINTER(ctypes.c_float))
         _check(_lib.eqlin_copy_freq_weights(h.ptr, dst, out.numel()), "eqlin_copy_freq_weights")
     return out
+
+
+def eqlin_forward_noalloc(x: torch.Tensor, w: torch.Tensor, bias: torch.Tensor | None = None,
+                          y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Weight transform + forward in one call that allocates no device memory in the
+    library (for callers that must not allocate); x, w, bias and y share one dtype.
+    Calls that overlap on the GPU share the library's fixed scratch array: serialise
+    them.  (The y tensor, when not given, is allocated here by torch.)"""
+    if w.dim() != 3 or x.dim() != 3 or x.shape[1:] != w.shape[1:]:
+        raise ValueError("x must be [N, Cin, G] and w [Cout, Cin, G]")
+    if x.dtype not in _TORCH_TO_EQLIN or w.dtype != x.dtype or x.device != w.device:
+        raise ValueError("x and w must share a supported dtype and a device")
+    if not (x.is_contiguous() and w.is_contiguous()):
+        raise ValueError("x and w must be contiguous")
+    N, Cin, G = x.shape
+    Cout = w.shape[0]
+    if bias is not None and (bias.shape != (Cout,) or bias.dtype != x.dtype or not bias.is_contiguous()):
+        raise ValueError("bias must be a contiguous [Cout] tensor of x's dtype")
+    if y is None:
+        y = torch.empty((N, Cout, G), dtype=x.dtype, device=x.device)
+    with torch.cuda.device(x.device):
+        _check(_lib.eqlin_forward_noalloc(x.data_ptr(), w.data_ptr(), None if bias is None else bias.data_ptr(),
+                                          y.data_ptr(), N, Cout, Cin, G, _TORCH_TO_EQLIN[x.dtype],
+                                          _stream_ptr(stream)), "eqlin_forward_noalloc")
+    return y

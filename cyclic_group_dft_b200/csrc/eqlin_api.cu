@@ -518,3 +518,217 @@ const char* eqlin_last_error(void) { return g_last_error.c_str(); }
 int eqlin_version(void) { return 100; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------
+// Allocation-free forward (eqlin_forward_noalloc).
+//
+// For callers that must not allocate device memory: a framework whose device memory
+// is owned by its own pool (a stray cudaMalloc fragments it or is refused), or a host
+// loop that cannot afford the implicit device-wide synchronisation and latency of
+// cudaMalloc / cudaFree.  Such a caller passes only its inputs (x, w, bias) and its
+// output (y); everything else the computation needs -- the device status word and the
+// frequency-domain weights that eqlin_prepare_weights would keep in a handle -- lives
+// in the fixed array below.  The array is part of the library image: every GPU that
+// loads the library holds it until the process exits.
+//
+// In host code the array's name is only a host-side stand-in, never a device
+// address, so its device address is looked up once per device (cudaGetSymbolAddress)
+// and handed to the kernels as a pointer.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[EQLIN_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kNoAllocMaxDevices = 64;
+
+struct NoAllocDevice {
+    bool ready = false;
+    uint8_t* scratch = nullptr;  // device address of g_noalloc_scratch on this device
+    int sm_count = 0;
+    int optin = 0;
+    bool cc_ok = false;
+    uint32_t attr_done[2][4][2][2] = {};  // [f32?][G index][stream][nacc-1]: smem attribute set
+};
+
+std::mutex g_noalloc_mutex;
+NoAllocDevice g_noalloc_dev[kNoAllocMaxDevices];
+
+size_t align256(size_t v) { return (v + 255) / 256 * 256; }
+
+int g_index(int64_t G) { return G == 2 ? 0 : G == 4 ? 1 : G == 8 ? 2 : 3; }
+
+// First call on a device, with that device current: resolve the scratch array's
+// device address and read the device limits.  Later calls reuse them.
+int noalloc_setup(int dev, NoAllocDevice** out) {
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(EQLIN_ERR_UNSUPPORTED, "device index above 63");
+    NoAllocDevice& d = g_noalloc_dev[dev];
+    if (!d.ready) {
+        void* ptr = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+        int major = 0, minor = 0;
+        if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&d.optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
+            return cuda_fail(e, "device query");
+        d.cc_ok = major == 10 && minor == 0;
+        d.scratch = static_cast<uint8_t*>(ptr);
+        d.ready = true;
+    }
+    if (!d.cc_ok) return fail(EQLIN_ERR_UNSUPPORTED, "needs a compute capability 10.0 (sm_100a) device");
+    *out = &d;
+    return EQLIN_OK;
+}
+
+}  // namespace
+
+extern "C" int eqlin_forward_noalloc(const void* x, const void* w, const void* bias, void* y, int64_t N,
+                                     int64_t Cout, int64_t Cin, int64_t G, int dtype, void* stream) {
+    int s = check_shape_impl(Cout, Cin, G, dtype, dtype);
+    if (s != EQLIN_OK) return s;
+    if (N < 0) return fail(EQLIN_ERR_INVALID_ARG, "N < 0");
+    if (!w) return fail(EQLIN_ERR_INVALID_ARG, "w is NULL");
+    if (N == 0) return EQLIN_OK;
+    if (!x || !y) return fail(EQLIN_ERR_INVALID_ARG, "x or y is NULL");
+    if (N >= (int64_t(1) << 31)) return fail(EQLIN_ERR_UNSUPPORTED, "N must be below 2^31");
+    const size_t elt = dtype == EQLIN_F32 ? 4 : 2;
+    if (!aligned(x, 16) || !aligned(y, 16)) return fail(EQLIN_ERR_MISALIGNED, "x and y must be 16-byte aligned");
+    if (!aligned(w, elt) || (bias && !aligned(bias, elt)))
+        return fail(EQLIN_ERR_MISALIGNED, "w / bias not aligned to their element size");
+
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    NoAllocDevice* d = nullptr;
+    Plan plan;
+    {
+        std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+        s = noalloc_setup(dev, &d);
+        if (s != EQLIN_OK) return s;
+        s = plan_for(Cout, Cin, G, dtype, static_cast<size_t>(d->optin), &plan);
+        if (s != EQLIN_OK) return s;
+        // kernel shared-memory attribute, once per kernel and device
+        const int fi = plan.path == kPathF32 ? 1 : 0, gi = g_index(G);
+        const int si = plan.path == kPathStreamed ? 1 : 0, ai = plan.nacc == 1 ? 0 : 1;
+        if (!d->attr_done[fi][gi][si][ai]) {
+            void* k = plan.path == kPathF32 ? f32_kernel_for(static_cast<int>(G))
+                                            : tc_entry_for(static_cast<int>(G), si == 1, plan.nacc).kernel;
+            e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(plan.smem_bytes));
+            if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+            d->attr_done[fi][gi][si][ai] = 1;
+        }
+    }
+
+    // scratch layout: status word | fp32 bias | fp32 planes | (bf16 image | fp64 planes + bias)
+    const size_t planes = static_cast<size_t>(G) * Cin * Cout;
+    size_t off = 0;
+    const size_t off_status = off;
+    off += 256;
+    const size_t off_bias = off;
+    off = align256(off + static_cast<size_t>(Cout) * sizeof(float));
+    const size_t off_wf = off;
+    off = align256(off + planes * sizeof(float));
+    size_t off_img = 0, off_wd = 0, off_bd = 0;
+    if (plan.path == kPathF32) {
+        off_wd = off;
+        off = align256(off + planes * sizeof(double));
+        off_bd = off;
+        off = align256(off + static_cast<size_t>(Cout) * sizeof(double));
+    } else {
+        off_img = off;
+        off = align256(off + plan.img_alloc_bytes);
+    }
+    if (off > EQLIN_NOALLOC_SCRATCH_BYTES)
+        return fail(EQLIN_ERR_UNSUPPORTED, "shape needs " + std::to_string(off) +
+                                               " bytes of scratch; eqlin_forward_noalloc is limited to " +
+                                               std::to_string(EQLIN_NOALLOC_SCRATCH_BYTES));
+    uint8_t* sc = d->scratch;
+    int* status = reinterpret_cast<int*>(sc + off_status);
+    float* bias_f32 = reinterpret_cast<float*>(sc + off_bias);
+    float* w_f32 = reinterpret_cast<float*>(sc + off_wf);
+    double* w_f64 = plan.path == kPathF32 ? reinterpret_cast<double*>(sc + off_wd) : nullptr;
+    double* bias_f64 = plan.path == kPathF32 ? reinterpret_cast<double*>(sc + off_bd) : nullptr;
+    uint8_t* img = plan.path == kPathF32 ? nullptr : sc + off_img;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    // the status word keeps the previous call's value: clear it
+    if ((e = cudaMemsetAsync(status, 0, sizeof(int), st)) != cudaSuccess) return cuda_fail(e, "status clear");
+
+    // weight transform into the scratch (same kernels as eqlin_prepare_weights)
+    const int threads = 256;
+    const unsigned blocks = static_cast<unsigned>((Cout * Cin + threads - 1) / threads);
+    const int iCout = static_cast<int>(Cout), iCin = static_cast<int>(Cin), iG = static_cast<int>(G);
+    if (dtype == EQLIN_F32) {
+        eqlin::eqlin_prep_freq_kernel<float><<<blocks, threads, 0, st>>>(
+            static_cast<const float*>(w), static_cast<const float*>(bias), iCout, iCin, iG, w_f32, bias_f32, w_f64,
+            bias_f64);
+    } else {
+        eqlin::eqlin_prep_freq_kernel<__nv_bfloat16><<<blocks, threads, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(w), static_cast<const __nv_bfloat16*>(bias), iCout, iCin, iG, w_f32,
+            bias_f32, w_f64, bias_f64);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "weight transform launch");
+    if (img) {
+        const size_t n = plan.img_alloc_bytes / 2;
+        eqlin::eqlin_prep_image_kernel<<<static_cast<unsigned>((n + threads - 1) / threads), threads, 0, st>>>(
+            w_f32, iCout, iCin, iG, plan.nK, plan.rows, n, img);
+        if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "weight image launch");
+    }
+
+    // the forward itself (same kernels as eqlin_forward)
+    if (plan.path == kPathF32) {
+        dim3 grid(static_cast<unsigned>((N + eqlin::kF32Tokens - 1) / eqlin::kF32Tokens),
+                  static_cast<unsigned>((Cout + 31) / 32));
+        const float* xf = static_cast<const float*>(x);
+        float* yf = static_cast<float*>(y);
+        switch (G) {
+            case 2: eqlin::eqlin_fwd_f32_kernel<2><<<grid, eqlin::kF32Threads, plan.smem_bytes, st>>>(xf, w_f64, bias_f64, yf, N, iCin, iCout); break;
+            case 4: eqlin::eqlin_fwd_f32_kernel<4><<<grid, eqlin::kF32Threads, plan.smem_bytes, st>>>(xf, w_f64, bias_f64, yf, N, iCin, iCout); break;
+            case 8: eqlin::eqlin_fwd_f32_kernel<8><<<grid, eqlin::kF32Threads, plan.smem_bytes, st>>>(xf, w_f64, bias_f64, yf, N, iCin, iCout); break;
+            default: eqlin::eqlin_fwd_f32_kernel<16><<<grid, eqlin::kF32Threads, plan.smem_bytes, st>>>(xf, w_f64, bias_f64, yf, N, iCin, iCout); break;
+        }
+    } else {
+        auto encode = tensor_map_encoder();
+        if (!encode) return fail(EQLIN_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+        CUtensorMap map, ymap;
+        cuuint64_t dims[2] = {static_cast<cuuint64_t>(Cin * G), static_cast<cuuint64_t>(N)};
+        cuuint64_t strides[1] = {static_cast<cuuint64_t>(Cin * G * 2)};
+        cuuint32_t boxdim[2] = {static_cast<cuuint32_t>(tc_box_elems(iG)), static_cast<cuuint32_t>(plan.BN)};
+        cuuint32_t estr[2] = {1, 1};
+        CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, boxdim,
+                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return fail(EQLIN_ERR_CUDA, "cuTensorMapEncodeTiled failed for x");
+        cuuint64_t ydims[2] = {static_cast<cuuint64_t>(Cout * G), static_cast<cuuint64_t>(N)};
+        cuuint64_t ystrides[1] = {static_cast<cuuint64_t>(Cout * G * 2)};
+        cuuint32_t ybox[2] = {static_cast<cuuint32_t>(eqlin::tc::kYBoxCols), static_cast<cuuint32_t>(plan.TG)};
+        r = encode(&ymap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, ydims, ystrides, ybox, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return fail(EQLIN_ERR_CUDA, "cuTensorMapEncodeTiled failed for y");
+        TcParams p;
+        p.w_img = img;
+        p.bias = bias ? bias_f32 : nullptr;
+        p.y = static_cast<__nv_bfloat16*>(y);
+        p.status = status;
+        p.N = N;
+        p.Cout = iCout;
+        p.nK = plan.nK;
+        p.rows = plan.rows;
+        p.n_oc = plan.n_oc;
+        p.n_work = static_cast<int>((N + plan.BN - 1) / plan.BN * plan.n_oc);
+        p.stages = plan.stages;
+        p.w_region_bytes = plan.w_region_bytes;
+        p.ystage_bytes = plan.ystage_bytes;
+        p.ycols_pad = plan.ycols_pad;
+        p.w_img_bytes = plan.w_img_bytes;
+        p.timeout_ns = kDefaultTimeoutNs;
+        const TcEntry entry = tc_entry_for(iG, plan.path == kPathStreamed, plan.nacc);
+        if (!entry.launch) return fail(EQLIN_ERR_UNSUPPORTED, "G");
+        const unsigned grid = static_cast<unsigned>(std::min<long long>(p.n_work, d->sm_count));
+        entry.launch(grid, plan.smem_bytes, st, map, ymap, p);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "forward launch");
+    return EQLIN_OK;
+}

@@ -165,6 +165,44 @@ EQLIN_API int eqlin_copy_freq_weights(const eqlin_handle* h, float* dst, int64_t
  */
 EQLIN_API int eqlin_check_shape(int64_t Cout, int64_t Cin, int64_t G, int w_dtype, int io_dtype);
 
+/*
+ * eqlin_forward_noalloc -- the same forward as eqlin_prepare_weights followed by
+ * eqlin_forward, in one call that allocates no device memory.  (Not a step of the
+ * method: the source page has no counterpart; it exists for callers that cannot
+ * allocate.)
+ *
+ * It is meant for callers that must not call cudaMalloc: a framework whose device
+ * memory is owned by its own pool (a stray driver allocation fragments the pool or is
+ * refused outright), or a host loop that cannot take the device-wide synchronisation
+ * and latency an allocation or free can imply.  The caller passes its inputs and its
+ * output; the device status word and the frequency-domain weights (which the handle
+ * API keeps in memory it allocates) live instead in one fixed array of
+ * EQLIN_NOALLOC_SCRATCH_BYTES (4 MiB) that is part of the library image, so every GPU
+ * that loads the library holds it until the process exits.
+ *
+ *   x, y     device, [N, Cin, G] / [N, Cout, G] of dtype, 16-byte aligned.
+ *   w, bias  device, [Cout, Cin, G] / [Cout] of dtype (bias may be NULL).
+ *   dtype    EQLIN_BF16 or EQLIN_F32, for all four tensors.
+ *   stream   every step (weight transform, forward) is enqueued on it; nothing is
+ *            synchronised.
+ *
+ * Each call re-transforms the weights (a small kernel, O(Cout*Cin*G^2)).  Every call
+ * on a device shares the one array and leaves its contents there; the status word is
+ * cleared at the start of each call.  Calls whose work overlaps on the GPU (other
+ * streams, other host threads) race on the array: serialise them.  The first call on
+ * a device sets up (it looks up the array's device address and sets kernel
+ * attributes) and must be made with that device current and before any stream
+ * capture that will contain this call.
+ *
+ * Errors: as eqlin_prepare_weights / eqlin_forward; UNSUPPORTED also when the shape's
+ * transformed weights do not fit in the array (the message gives the bytes needed).
+ * Kernel-side wait timeouts are recorded in the array's status word and are not
+ * reported to the caller.
+ */
+#define EQLIN_NOALLOC_SCRATCH_BYTES (4u * 1024u * 1024u)
+EQLIN_API int eqlin_forward_noalloc(const void* x, const void* w, const void* bias, void* y, int64_t N,
+                                    int64_t Cout, int64_t Cin, int64_t G, int dtype, void* stream);
+
 /* Static description of a status code ("ok", "invalid argument", ...). */
 EQLIN_API const char* eqlin_status_string(int status);
 
