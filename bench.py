@@ -189,6 +189,23 @@ def oracle_rate(wl: workloads.Workload, target_s: float, seed: int = 0, cap_toke
 
 
 # ------------------------------------------------------------------ helpers
+def reduce_max(value: float, device) -> float:
+    """Max of `value` over all ranks (identity without a process group).  Every rank
+    must call it at the same point."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tokens_per_s(world: int, steps: int, tokens_per_rank: int, max_elapsed_ms: float) -> float:
+    """Whole-job throughput: every rank processes `tokens_per_rank` tokens per step
+    (replicas, weak scaling); the job takes as long as its slowest rank."""
+    return world * steps * tokens_per_rank / (max_elapsed_ms / 1e3)
+
+
 def dist_info():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -308,12 +325,8 @@ def main() -> None:
     launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     status = h.device_status()
 
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
-
-    value = world * K * N / (elapsed_ms / 1e3)
+    elapsed_ms = reduce_max(elapsed_ms, dev)
+    value = aggregate_tokens_per_s(world, K, N, elapsed_ms)
     avg_launch_s = statistics.mean(launch_ms) / 1e3
 
     # ----------------------------------------------------------- end to end
@@ -333,12 +346,8 @@ def main() -> None:
         e1.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-        e2e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": world * E * N / (e2e_ms / 1e3), "unit": "tokens/s", "steps": E,
+        e2e_ms = reduce_max(e0.elapsed_time(e1), dev)
+        e2e = {"value": aggregate_tokens_per_s(world, E, N, e2e_ms), "unit": "tokens/s", "steps": E,
                "h2d_bytes_per_step": x_pin.numel() * x_pin.element_size(),
                "d2h_bytes_per_step": y_pin.numel() * y_pin.element_size(),
                "api": "Handle.forward_host (pinned host x -> device -> eqlin_forward -> pinned host y)"}
