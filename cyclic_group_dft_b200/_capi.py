@@ -31,7 +31,9 @@ ATTRS = {
     "G": 0, "Cin": 1, "Cout": 2, "io_dtype": 3, "path": 4, "tokens_per_tile": 5,
     "stages": 6, "smem_bytes": 7, "max_grid": 8, "weight_bytes": 9,
 }
-PATH_NAMES = {0: "tcgen05_resident_weights", 1: "tcgen05_streamed_weights", 2: "fp32_ffma"}
+PATH_NAMES = {0: "tcgen05_tokens_on_n_resident_weights", 1: "tcgen05_tokens_on_n_streamed_weights",
+              2: "fp32_fp64_arithmetic", 3: "tcgen05_tokens_on_m_resident_weights",
+              4: "tcgen05_tokens_on_m_streamed_weights"}
 
 _TORCH_TO_EQLIN = {torch.float32: EQLIN_F32, torch.bfloat16: EQLIN_BF16}
 _EQLIN_TO_TORCH = {v: k for k, v in _TORCH_TO_EQLIN.items()}

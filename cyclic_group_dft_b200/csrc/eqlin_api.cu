@@ -1,6 +1,6 @@
 // eqlin_api.cu -- host side of the C ABI declared in include/eqlin.h: argument
-// validation, kernel planning (shared-memory budget, ring depth), ownership of the
-// frequency-domain weights, TMA descriptor encoding and launches.
+// validation, kernel planning (shared-memory budget, ring depth, kernel variant),
+// ownership of the frequency-domain weights, TMA descriptor encoding and launches.
 #include "eqlin.h"
 
 #include <cuda.h>
@@ -10,26 +10,33 @@
 #include <algorithm>
 #include <cstdint>
 #include <cstdlib>
+#include <cstring>
 #include <mutex>
 #include <new>
 #include <string>
 
 #include "eqlin_fwd_tc.cuh"
+#include "eqlin_fwd_tm.cuh"
 #include "eqlin_layout.h"
 #include "eqlin_prep.cuh"
 
 using eqlin::TcParams;
+using eqlin::TmParams;
 
 namespace {
 
 constexpr size_t kB200SmemOptin = 232448;   // 227 KB opt-in shared memory per CTA on sm_100
-constexpr size_t kSmemAlignSlack = 1024;    // the kernel rounds its smem base up to 1 KB
+constexpr size_t kSmemAlignSlack = 1024;    // the kernels round their smem base up to 1 KB
 constexpr size_t kSmemCtlBytes = 512;       // mbarriers + control block
 constexpr int kMaxStages = 12;
 constexpr int64_t kMaxChannels = 1 << 16;
 constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per bounded wait
 
-enum Path { kPathResident = 0, kPathStreamed = 1, kPathF32 = 2 };
+// Kernel variants (EQLIN_ATTR_PATH):
+//   0/1  tcgen05, tokens on the MMA N dimension, weights resident / streamed
+//   2    fp32 I/O, float64 CUDA-core kernel
+//   3/4  tcgen05, tokens on the MMA M dimension, weights resident / streamed
+enum Path { kPathResident = 0, kPathStreamed = 1, kPathF32 = 2, kPathTmResident = 3, kPathTmStreamed = 4 };
 
 thread_local std::string g_last_error;
 
@@ -44,21 +51,32 @@ int cuda_fail(cudaError_t e, const char* what) {
 
 struct Plan {
     int path = kPathF32;
-    int nacc = 2;  // TMEM accumulator buffers (tcgen05 path)
-    int nK = 0, rows = 0, n_oc = 0, BN = 0, stages = 0, TG = 0, ycols_pad = 0;
+    int nacc = 2;        // TMEM accumulator buffers (tokens-on-N kernel)
+    int nK = 0;          // input-channel chunks
+    int rows = 0;        // weight rows per image sub-block (tokens-on-M: NO, the MMA N)
+    int n_oc = 0;        // output chunks
+    int BN = 0;          // tokens per work item
+    int stages = 0;
+    int TG = 0;          // y TMA store box rows (tokens-on-N)
+    int ycols_pad = 0;   // staged y columns per group (tokens-on-N)
+    int box_elems = 0;   // x TMA box columns
     uint32_t w_region_bytes = 0, w_img_bytes = 0, ystage_bytes = 0;
     size_t smem_bytes = 0;
     size_t img_alloc_bytes = 0;
+    bool tm() const { return path == kPathTmResident || path == kPathTmStreamed; }
+    bool streamed() const { return path == kPathStreamed || path == kPathTmStreamed; }
 };
 
+// ----------------------------------------------------------------- planning
 template <int G, int NACC>
-int plan_tc_g(int64_t Cout, int64_t Cin, size_t max_smem, Plan* pl) {
+int plan_tn_g(int64_t Cout, int64_t Cin, size_t max_smem, Plan* pl) {
     using S = eqlin::tc::Shape<G, NACC>;
     pl->nacc = NACC;
     pl->nK = static_cast<int>((Cin + eqlin::kChunkK - 1) / eqlin::kChunkK);
     pl->n_oc = static_cast<int>((Cout + eqlin::kMmaM - 1) / eqlin::kMmaM);
     pl->BN = S::BN;
     pl->TG = S::TG;
+    pl->box_elems = S::BOX_ELEMS;
     // y staging: 4 buffers (2 per epilogue half) of TG rows x the chunk's y columns
     const int64_t chunk_rows = std::min<int64_t>(Cout, eqlin::kMmaM);
     pl->ycols_pad = static_cast<int>((chunk_rows * G + eqlin::tc::kYBoxCols - 1) / eqlin::tc::kYBoxCols *
@@ -100,11 +118,51 @@ int plan_tc_g(int64_t Cout, int64_t Cin, size_t max_smem, Plan* pl) {
     return EQLIN_OK;
 }
 
-// Accumulator buffers per group order (measured on B200; see the design notes).
-int default_acc_buffers(int G) {
-    (void)G;
-    return 2;
+template <int G>
+int plan_tm_g(int64_t Cout, int64_t Cin, size_t max_smem, Plan* pl) {
+    using C = eqlin::tm::Cfg<G>;
+    const int64_t no = std::min<int64_t>((Cout + 31) / 32 * 32, C::NMAX);  // MMA N, multiple of 32
+    pl->rows = static_cast<int>(no);
+    pl->nK = static_cast<int>((Cin + eqlin::kChunkK16 - 1) / eqlin::kChunkK16);
+    pl->n_oc = static_cast<int>((Cout + no - 1) / no);
+    pl->BN = eqlin::tm::kM;
+    pl->box_elems = C::XROW_ELEMS;
+    const size_t wchunk = static_cast<size_t>(G) * no * eqlin::kRowBytes32;   // one (oc, c) weight chunk
+    const size_t fixed = kSmemAlignSlack + kSmemCtlBytes +
+                         static_cast<size_t>(eqlin::tm::kYBufs) * eqlin::tm::kYBufBytes;
+    if (pl->n_oc == 1) {
+        const size_t img = wchunk * pl->nK;
+        const size_t region = (img + 1023) / 1024 * 1024;
+        if (max_smem > fixed + region) {
+            const size_t stages = std::min<size_t>(kMaxStages, (max_smem - fixed - region) / C::XCHUNK_BYTES);
+            if (stages >= 2) {
+                pl->path = kPathTmResident;
+                pl->stages = static_cast<int>(stages);
+                pl->w_region_bytes = static_cast<uint32_t>(region);
+                pl->w_img_bytes = static_cast<uint32_t>(img);
+                pl->img_alloc_bytes = img;
+                pl->smem_bytes = fixed + region + stages * C::XCHUNK_BYTES;
+                return EQLIN_OK;
+            }
+        }
+    }
+    const size_t stage = C::XCHUNK_BYTES + wchunk;
+    const size_t stages = max_smem > fixed ? std::min<size_t>(kMaxStages, (max_smem - fixed) / stage) : 0;
+    if (stages < 1) return fail(EQLIN_ERR_UNSUPPORTED, "shape does not fit in shared memory");
+    pl->path = kPathTmStreamed;
+    pl->stages = static_cast<int>(stages);
+    pl->w_region_bytes = 0;
+    pl->w_img_bytes = 0;
+    pl->img_alloc_bytes = wchunk * pl->nK * pl->n_oc;
+    pl->smem_bytes = fixed + stages * stage;
+    return EQLIN_OK;
 }
+
+// Kernel variant per group order, from B200 measurements: with tokens on M the MMA
+// count per token no longer grows with the padding of a small Cout to 128 rows, which
+// wins for G >= 8 (C16 C32: 358 -> 166 us, p8 C64: 30.9 -> 28.1 us); for G = 4 the
+// double-buffered tokens-on-N kernel stays ahead (p4 C96: 70.1 vs 76.6 us).
+bool default_tokens_on_m(int G) { return G >= 8; }
 
 int plan_for(int64_t Cout, int64_t Cin, int64_t G, int io_dtype, size_t max_smem, Plan* pl) {
     if (io_dtype == EQLIN_F32) {
@@ -115,16 +173,30 @@ int plan_for(int64_t Cout, int64_t Cin, int64_t G, int io_dtype, size_t max_smem
         pl->smem_bytes = smem;
         return EQLIN_OK;
     }
-    int nacc = default_acc_buffers(static_cast<int>(G));
+    bool tm = default_tokens_on_m(static_cast<int>(G));
+    if (const char* e = std::getenv("EQLIN_KERNEL")) {
+        if (std::strcmp(e, "tm") == 0) tm = true;
+        if (std::strcmp(e, "tn") == 0) tm = false;
+    }
+    if (tm) {
+        switch (G) {
+            case 2: return plan_tm_g<2>(Cout, Cin, max_smem, pl);
+            case 4: return plan_tm_g<4>(Cout, Cin, max_smem, pl);
+            case 8: return plan_tm_g<8>(Cout, Cin, max_smem, pl);
+            case 16: return plan_tm_g<16>(Cout, Cin, max_smem, pl);
+            default: return fail(EQLIN_ERR_UNSUPPORTED, "G must be 2, 4, 8 or 16");
+        }
+    }
+    int nacc = 2;
     if (const char* e = std::getenv("EQLIN_ACC_BUFFERS")) {
         if (e[0] == '1') nacc = 1;
         if (e[0] == '2') nacc = 2;
     }
     switch (G) {
-        case 2: return nacc == 1 ? plan_tc_g<2, 1>(Cout, Cin, max_smem, pl) : plan_tc_g<2, 2>(Cout, Cin, max_smem, pl);
-        case 4: return nacc == 1 ? plan_tc_g<4, 1>(Cout, Cin, max_smem, pl) : plan_tc_g<4, 2>(Cout, Cin, max_smem, pl);
-        case 8: return nacc == 1 ? plan_tc_g<8, 1>(Cout, Cin, max_smem, pl) : plan_tc_g<8, 2>(Cout, Cin, max_smem, pl);
-        case 16: return nacc == 1 ? plan_tc_g<16, 1>(Cout, Cin, max_smem, pl) : plan_tc_g<16, 2>(Cout, Cin, max_smem, pl);
+        case 2: return nacc == 1 ? plan_tn_g<2, 1>(Cout, Cin, max_smem, pl) : plan_tn_g<2, 2>(Cout, Cin, max_smem, pl);
+        case 4: return nacc == 1 ? plan_tn_g<4, 1>(Cout, Cin, max_smem, pl) : plan_tn_g<4, 2>(Cout, Cin, max_smem, pl);
+        case 8: return nacc == 1 ? plan_tn_g<8, 1>(Cout, Cin, max_smem, pl) : plan_tn_g<8, 2>(Cout, Cin, max_smem, pl);
+        case 16: return nacc == 1 ? plan_tn_g<16, 1>(Cout, Cin, max_smem, pl) : plan_tn_g<16, 2>(Cout, Cin, max_smem, pl);
         default: return fail(EQLIN_ERR_UNSUPPORTED, "G must be 2, 4, 8 or 16");
     }
 }
@@ -154,17 +226,29 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
+// ------------------------------------------------------------- kernel tables
 using TcLaunch = void (*)(unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& mx,
                           const CUtensorMap& my, const TcParams& p);
+using TmLaunch = void (*)(unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& mx,
+                          const CUtensorMap& my, const TmParams& p);
 
 template <int G, bool STREAM, int NACC>
 void tc_launch(unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& mx, const CUtensorMap& my,
                const TcParams& p) {
     eqlin::eqlin_fwd_tc_kernel<G, STREAM, NACC><<<grid, eqlin::tc::kThreads, smem, st>>>(mx, my, p);
 }
+template <int G, bool STREAM>
+void tm_launch(unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& mx, const CUtensorMap& my,
+               const TmParams& p) {
+    eqlin::eqlin_fwd_tm_kernel<G, STREAM><<<grid, eqlin::tm::Cfg<G>::kThreads, smem, st>>>(mx, my, p);
+}
 
 struct TcEntry {
     TcLaunch launch = nullptr;
+    void* kernel = nullptr;
+};
+struct TmEntry {
+    TmLaunch launch = nullptr;
     void* kernel = nullptr;
 };
 
@@ -172,19 +256,31 @@ template <int G, bool STREAM, int NACC>
 TcEntry tc_entry() {
     return {&tc_launch<G, STREAM, NACC>, reinterpret_cast<void*>(&eqlin::eqlin_fwd_tc_kernel<G, STREAM, NACC>)};
 }
-
 template <int G>
 TcEntry tc_entry_g(bool stream, int nacc) {
     if (stream) return nacc == 1 ? tc_entry<G, true, 1>() : tc_entry<G, true, 2>();
     return nacc == 1 ? tc_entry<G, false, 1>() : tc_entry<G, false, 2>();
 }
-
 TcEntry tc_entry_for(int G, bool stream, int nacc) {
     switch (G) {
         case 2: return tc_entry_g<2>(stream, nacc);
         case 4: return tc_entry_g<4>(stream, nacc);
         case 8: return tc_entry_g<8>(stream, nacc);
         case 16: return tc_entry_g<16>(stream, nacc);
+        default: return {};
+    }
+}
+
+template <int G, bool STREAM>
+TmEntry tm_entry() {
+    return {&tm_launch<G, STREAM>, reinterpret_cast<void*>(&eqlin::eqlin_fwd_tm_kernel<G, STREAM>)};
+}
+TmEntry tm_entry_for(int G, bool stream) {
+    switch (G) {
+        case 2: return stream ? tm_entry<2, true>() : tm_entry<2, false>();
+        case 4: return stream ? tm_entry<4, true>() : tm_entry<4, false>();
+        case 8: return stream ? tm_entry<8, true>() : tm_entry<8, false>();
+        case 16: return stream ? tm_entry<16, true>() : tm_entry<16, false>();
         default: return {};
     }
 }
@@ -199,18 +295,150 @@ void* f32_kernel_for(int G) {
     }
 }
 
+void* kernel_for(const Plan& pl, int G) {
+    if (pl.path == kPathF32) return f32_kernel_for(G);
+    if (pl.tm()) return tm_entry_for(G, pl.streamed()).kernel;
+    return tc_entry_for(G, pl.streamed(), pl.nacc).kernel;
+}
+
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-template <int G>
-int box_elems() { return eqlin::tc::Shape<G, 2>::BOX_ELEMS; }  // independent of the accumulator count
+// ------------------------------------------------------------------ launches
+// Buffers of the frequency-domain weights (owned by a handle or carved from the
+// allocation-free scratch array).
+struct WeightBuffers {
+    uint8_t* img = nullptr;       // bf16 tensor-core image (bf16 I/O)
+    float* w_f32 = nullptr;       // [G][Cin][Cout]
+    float* bias_f32 = nullptr;    // [Cout]
+    double* w_f64 = nullptr;      // fp32-I/O path only
+    double* bias_f64 = nullptr;   // fp32-I/O path only
+    int* status = nullptr;
+    bool has_bias = false;
+};
 
-int tc_box_elems(int G) {
-    switch (G) {
-        case 2: return box_elems<2>();
-        case 4: return box_elems<4>();
-        case 8: return box_elems<8>();
-        default: return box_elems<16>();
+int launch_prep(const Plan& pl, int w_dtype, const void* w, const void* bias, int64_t Cout, int64_t Cin,
+                int64_t G, const WeightBuffers& b, cudaStream_t st) {
+    const int threads = 256;
+    const unsigned blocks = static_cast<unsigned>((Cout * Cin + threads - 1) / threads);
+    const int iCout = static_cast<int>(Cout), iCin = static_cast<int>(Cin), iG = static_cast<int>(G);
+    if (w_dtype == EQLIN_F32) {
+        eqlin::eqlin_prep_freq_kernel<float><<<blocks, threads, 0, st>>>(
+            static_cast<const float*>(w), static_cast<const float*>(bias), iCout, iCin, iG, b.w_f32, b.bias_f32,
+            b.w_f64, b.bias_f64);
+    } else {
+        eqlin::eqlin_prep_freq_kernel<__nv_bfloat16><<<blocks, threads, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(w), static_cast<const __nv_bfloat16*>(bias), iCout, iCin, iG,
+            b.w_f32, b.bias_f32, b.w_f64, b.bias_f64);
     }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "weight transform launch");
+    if (b.img) {
+        const size_t n = pl.img_alloc_bytes / 2;
+        const unsigned b2 = static_cast<unsigned>((n + threads - 1) / threads);
+        if (pl.tm()) {
+            eqlin::eqlin_prep_image_k16_kernel<<<b2, threads, 0, st>>>(b.w_f32, iCout, iCin, iG, pl.nK, pl.rows, n,
+                                                                        b.img);
+        } else {
+            eqlin::eqlin_prep_image_kernel<<<b2, threads, 0, st>>>(b.w_f32, iCout, iCin, iG, pl.nK, pl.rows, n,
+                                                                    b.img);
+        }
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "weight image launch");
+    }
+    return EQLIN_OK;
+}
+
+int launch_forward(const Plan& pl, int64_t Cout, int64_t Cin, int64_t G, int sm_count, const void* x, void* y,
+                   int64_t N, const WeightBuffers& b, unsigned long long timeout_ns, cudaStream_t st) {
+    const int iG = static_cast<int>(G);
+    if (pl.path == kPathF32) {
+        dim3 grid(static_cast<unsigned>((N + eqlin::kF32Tokens - 1) / eqlin::kF32Tokens),
+                  static_cast<unsigned>((Cout + 31) / 32));
+        const float* xf = static_cast<const float*>(x);
+        float* yf = static_cast<float*>(y);
+        const int iCin = static_cast<int>(Cin), iCout = static_cast<int>(Cout);
+        switch (iG) {
+            case 2: eqlin::eqlin_fwd_f32_kernel<2><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, b.w_f64, b.bias_f64, yf, N, iCin, iCout); break;
+            case 4: eqlin::eqlin_fwd_f32_kernel<4><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, b.w_f64, b.bias_f64, yf, N, iCin, iCout); break;
+            case 8: eqlin::eqlin_fwd_f32_kernel<8><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, b.w_f64, b.bias_f64, yf, N, iCin, iCout); break;
+            default: eqlin::eqlin_fwd_f32_kernel<16><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, b.w_f64, b.bias_f64, yf, N, iCin, iCout); break;
+        }
+    } else {
+        auto encode = tensor_map_encoder();
+        if (!encode) return fail(EQLIN_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+        CUtensorMap map, ymap;
+        cuuint32_t estr[2] = {1, 1};
+        cuuint64_t dims[2] = {static_cast<cuuint64_t>(Cin * G), static_cast<cuuint64_t>(N)};
+        cuuint64_t strides[1] = {static_cast<cuuint64_t>(Cin * G * 2)};
+        cuuint32_t boxdim[2] = {static_cast<cuuint32_t>(pl.box_elems), static_cast<cuuint32_t>(pl.BN)};
+        CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, boxdim,
+                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return fail(EQLIN_ERR_CUDA, "cuTensorMapEncodeTiled failed for x");
+        cuuint64_t ydims[2] = {static_cast<cuuint64_t>(Cout * G), static_cast<cuuint64_t>(N)};
+        cuuint64_t ystrides[1] = {static_cast<cuuint64_t>(Cout * G * 2)};
+        cuuint32_t ybox[2];
+        CUtensorMapSwizzle yswz;
+        if (pl.tm()) {
+            ybox[0] = eqlin::tm::kYCols;
+            ybox[1] = eqlin::tm::kM;
+            yswz = CU_TENSOR_MAP_SWIZZLE_64B;
+        } else {
+            ybox[0] = eqlin::tc::kYBoxCols;
+            ybox[1] = static_cast<cuuint32_t>(pl.TG);
+            yswz = CU_TENSOR_MAP_SWIZZLE_NONE;
+        }
+        r = encode(&ymap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, ydims, ystrides, ybox, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, yswz, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return fail(EQLIN_ERR_CUDA, "cuTensorMapEncodeTiled failed for y");
+        const long long n_tiles = (N + pl.BN - 1) / pl.BN;
+        const int n_work = static_cast<int>(n_tiles * pl.n_oc);
+        const unsigned grid = static_cast<unsigned>(std::min<long long>(n_work, sm_count));
+        if (pl.tm()) {
+            TmParams p;
+            p.w_img = b.img;
+            p.bias = b.has_bias ? b.bias_f32 : nullptr;
+            p.status = b.status;
+            p.N = N;
+            p.Cout = static_cast<int>(Cout);
+            p.nK = pl.nK;
+            p.NO = pl.rows;
+            p.n_oc = pl.n_oc;
+            p.n_work = n_work;
+            p.stages = pl.stages;
+            p.w_region_bytes = pl.w_region_bytes;
+            p.w_img_bytes = pl.w_img_bytes;
+            p.timeout_ns = timeout_ns;
+            const TmEntry entry = tm_entry_for(iG, pl.streamed());
+            if (!entry.launch) return fail(EQLIN_ERR_UNSUPPORTED, "G");
+            entry.launch(grid, pl.smem_bytes, st, map, ymap, p);
+        } else {
+            TcParams p;
+            p.w_img = b.img;
+            p.bias = b.has_bias ? b.bias_f32 : nullptr;
+            p.y = static_cast<__nv_bfloat16*>(y);
+            p.status = b.status;
+            p.N = N;
+            p.Cout = static_cast<int>(Cout);
+            p.nK = pl.nK;
+            p.rows = pl.rows;
+            p.n_oc = pl.n_oc;
+            p.n_work = n_work;
+            p.stages = pl.stages;
+            p.w_region_bytes = pl.w_region_bytes;
+            p.ystage_bytes = pl.ystage_bytes;
+            p.ycols_pad = pl.ycols_pad;
+            p.w_img_bytes = pl.w_img_bytes;
+            p.timeout_ns = timeout_ns;
+            const TcEntry entry = tc_entry_for(iG, pl.streamed(), pl.nacc);
+            if (!entry.launch) return fail(EQLIN_ERR_UNSUPPORTED, "G");
+            entry.launch(grid, pl.smem_bytes, st, map, ymap, p);
+        }
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "forward launch");
+    return EQLIN_OK;
 }
 
 }  // namespace
@@ -221,13 +449,7 @@ struct eqlin_handle {
     int64_t Cout = 0, Cin = 0, G = 0;
     int w_dtype = 0, io_dtype = 0;
     Plan plan;
-    uint8_t* w_img = nullptr;
-    float* w_f32 = nullptr;
-    float* bias_f32 = nullptr;
-    double* w_f64 = nullptr;     // fp32-I/O path only
-    double* bias_f64 = nullptr;  // fp32-I/O path only
-    int* status = nullptr;
-    bool has_bias = false;
+    WeightBuffers buf;   // device memory owned by the handle
     bool sync_check = false;
     unsigned long long timeout_ns = kDefaultTimeoutNs;
 };
@@ -236,42 +458,13 @@ namespace {
 
 void free_handle(eqlin_handle* h) {
     if (!h) return;
-    if (h->w_img) cudaFree(h->w_img);
-    if (h->w_f32) cudaFree(h->w_f32);
-    if (h->bias_f32) cudaFree(h->bias_f32);
-    if (h->w_f64) cudaFree(h->w_f64);
-    if (h->bias_f64) cudaFree(h->bias_f64);
-    if (h->status) cudaFree(h->status);
+    if (h->buf.img) cudaFree(h->buf.img);
+    if (h->buf.w_f32) cudaFree(h->buf.w_f32);
+    if (h->buf.bias_f32) cudaFree(h->buf.bias_f32);
+    if (h->buf.w_f64) cudaFree(h->buf.w_f64);
+    if (h->buf.bias_f64) cudaFree(h->buf.bias_f64);
+    if (h->buf.status) cudaFree(h->buf.status);
     delete h;
-}
-
-int launch_prep(eqlin_handle* h, const void* w, const void* bias, cudaStream_t st) {
-    const int64_t pairs = h->Cout * h->Cin;
-    const int threads = 256;
-    const unsigned blocks = static_cast<unsigned>((pairs + threads - 1) / threads);
-    const int Cout = static_cast<int>(h->Cout), Cin = static_cast<int>(h->Cin), G = static_cast<int>(h->G);
-    if (h->w_dtype == EQLIN_F32) {
-        eqlin::eqlin_prep_freq_kernel<float><<<blocks, threads, 0, st>>>(
-            static_cast<const float*>(w), static_cast<const float*>(bias), Cout, Cin, G, h->w_f32, h->bias_f32,
-            h->w_f64, h->bias_f64);
-    } else {
-        eqlin::eqlin_prep_freq_kernel<__nv_bfloat16><<<blocks, threads, 0, st>>>(
-            static_cast<const __nv_bfloat16*>(w), static_cast<const __nv_bfloat16*>(bias), Cout, Cin, G,
-            h->w_f32, h->bias_f32, h->w_f64, h->bias_f64);
-    }
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "weight transform launch");
-    if (h->w_img) {
-        const size_t n = h->plan.img_alloc_bytes / 2;
-        const unsigned b2 = static_cast<unsigned>((n + threads - 1) / threads);
-        eqlin::eqlin_prep_image_kernel<<<b2, threads, 0, st>>>(h->w_f32, Cout, Cin, G, h->plan.nK, h->plan.rows,
-                                                                n, h->w_img);
-        e = cudaGetLastError();
-        if (e != cudaSuccess) return cuda_fail(e, "weight image launch");
-    }
-    e = cudaStreamSynchronize(st);
-    if (e != cudaSuccess) return cuda_fail(e, "weight transform");
-    return EQLIN_OK;
 }
 
 }  // namespace
@@ -322,7 +515,7 @@ int eqlin_prepare_weights(const void* w, const void* bias, int64_t Cout, int64_t
     h->w_dtype = w_dtype;
     h->io_dtype = io_dtype;
     h->plan = plan;
-    h->has_bias = bias != nullptr;
+    h->buf.has_bias = bias != nullptr;
     const char* sc = std::getenv("EQLIN_SYNC_CHECK");
     h->sync_check = sc && sc[0] == '1';
     if (const char* t = std::getenv("EQLIN_WAIT_TIMEOUT_MS")) {
@@ -331,30 +524,30 @@ int eqlin_prepare_weights(const void* w, const void* bias, int64_t Cout, int64_t
     }
 
     const size_t wf_bytes = static_cast<size_t>(G) * Cin * Cout * sizeof(float);
-    if (cudaMalloc(&h->w_f32, wf_bytes) != cudaSuccess ||
-        cudaMalloc(&h->bias_f32, static_cast<size_t>(Cout) * sizeof(float)) != cudaSuccess ||
-        cudaMalloc(&h->status, 256) != cudaSuccess ||
-        (plan.path == kPathF32 && (cudaMalloc(&h->w_f64, wf_bytes * 2) != cudaSuccess ||
-                                   cudaMalloc(&h->bias_f64, static_cast<size_t>(Cout) * sizeof(double)) != cudaSuccess)) ||
-        (plan.img_alloc_bytes && cudaMalloc(&h->w_img, plan.img_alloc_bytes) != cudaSuccess)) {
+    WeightBuffers& b = h->buf;
+    if (cudaMalloc(&b.w_f32, wf_bytes) != cudaSuccess ||
+        cudaMalloc(&b.bias_f32, static_cast<size_t>(Cout) * sizeof(float)) != cudaSuccess ||
+        cudaMalloc(&b.status, 256) != cudaSuccess ||
+        (plan.path == kPathF32 && (cudaMalloc(&b.w_f64, wf_bytes * 2) != cudaSuccess ||
+                                   cudaMalloc(&b.bias_f64, static_cast<size_t>(Cout) * sizeof(double)) != cudaSuccess)) ||
+        (plan.img_alloc_bytes && cudaMalloc(&b.img, plan.img_alloc_bytes) != cudaSuccess)) {
         cudaGetLastError();
         free_handle(h);
         return fail(EQLIN_ERR_OOM, "device allocation for the transformed weights");
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if ((e = cudaMemsetAsync(h->status, 0, 256, st)) != cudaSuccess) {
+    if ((e = cudaMemsetAsync(b.status, 0, 256, st)) != cudaSuccess) {
         free_handle(h);
         return cuda_fail(e, "status init");
     }
-    s = launch_prep(h, w, bias, st);
+    s = launch_prep(plan, w_dtype, w, bias, Cout, Cin, G, b, st);
+    if (s == EQLIN_OK && (e = cudaStreamSynchronize(st)) != cudaSuccess) s = cuda_fail(e, "weight transform");
     if (s != EQLIN_OK) {
         free_handle(h);
         return s;
     }
-    void* k = plan.path == kPathF32
-                  ? f32_kernel_for(static_cast<int>(G))
-                  : tc_entry_for(static_cast<int>(G), plan.path == kPathStreamed, plan.nacc).kernel;
-    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(plan.smem_bytes));
+    e = cudaFuncSetAttribute(kernel_for(plan, static_cast<int>(G)), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(plan.smem_bytes));
     if (e != cudaSuccess) {
         free_handle(h);
         return cuda_fail(e, "cudaFuncSetAttribute");
@@ -375,74 +568,13 @@ int eqlin_forward(const eqlin_handle* h, const void* x, void* y, int64_t N, void
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     if (dev != h->device) return fail(EQLIN_ERR_INVALID_ARG, "current device differs from the handle's device");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const Plan& pl = h->plan;
-    const int G = static_cast<int>(h->G);
-
-    if (pl.path == kPathF32) {
-        dim3 grid(static_cast<unsigned>((N + eqlin::kF32Tokens - 1) / eqlin::kF32Tokens),
-                  static_cast<unsigned>((h->Cout + 31) / 32));
-        void* args_x = const_cast<void*>(x);
-        const float* xf = static_cast<const float*>(args_x);
-        float* yf = static_cast<float*>(y);
-        const long long n = N;
-        const int Cin = static_cast<int>(h->Cin), Cout = static_cast<int>(h->Cout);
-        switch (G) {
-            case 2: eqlin::eqlin_fwd_f32_kernel<2><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, h->w_f64, h->bias_f64, yf, n, Cin, Cout); break;
-            case 4: eqlin::eqlin_fwd_f32_kernel<4><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, h->w_f64, h->bias_f64, yf, n, Cin, Cout); break;
-            case 8: eqlin::eqlin_fwd_f32_kernel<8><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, h->w_f64, h->bias_f64, yf, n, Cin, Cout); break;
-            default: eqlin::eqlin_fwd_f32_kernel<16><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, h->w_f64, h->bias_f64, yf, n, Cin, Cout); break;
-        }
-    } else {
-        auto encode = tensor_map_encoder();
-        if (!encode) return fail(EQLIN_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
-        const int box = tc_box_elems(G);
-        CUtensorMap map;
-        cuuint64_t dims[2] = {static_cast<cuuint64_t>(h->Cin * G), static_cast<cuuint64_t>(N)};
-        cuuint64_t strides[1] = {static_cast<cuuint64_t>(h->Cin * G * 2)};
-        cuuint32_t boxdim[2] = {static_cast<cuuint32_t>(box), static_cast<cuuint32_t>(pl.BN)};
-        cuuint32_t estr[2] = {1, 1};
-        CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, boxdim,
-                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        if (r != CUDA_SUCCESS) return fail(EQLIN_ERR_CUDA, "cuTensorMapEncodeTiled failed for x");
-        CUtensorMap ymap;
-        cuuint64_t ydims[2] = {static_cast<cuuint64_t>(h->Cout * G), static_cast<cuuint64_t>(N)};
-        cuuint64_t ystrides[1] = {static_cast<cuuint64_t>(h->Cout * G * 2)};
-        cuuint32_t ybox[2] = {static_cast<cuuint32_t>(eqlin::tc::kYBoxCols), static_cast<cuuint32_t>(pl.TG)};
-        r = encode(&ymap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, ydims, ystrides, ybox, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        if (r != CUDA_SUCCESS) return fail(EQLIN_ERR_CUDA, "cuTensorMapEncodeTiled failed for y");
-        TcParams p;
-        p.w_img = h->w_img;
-        p.bias = h->has_bias ? h->bias_f32 : nullptr;
-        p.y = static_cast<__nv_bfloat16*>(y);
-        p.status = h->status;
-        p.N = N;
-        p.Cout = static_cast<int>(h->Cout);
-        p.nK = pl.nK;
-        p.rows = pl.rows;
-        p.n_oc = pl.n_oc;
-        const long long n_tiles = (N + pl.BN - 1) / pl.BN;
-        p.n_work = static_cast<int>(n_tiles * pl.n_oc);
-        p.stages = pl.stages;
-        p.w_region_bytes = pl.w_region_bytes;
-        p.ystage_bytes = pl.ystage_bytes;
-        p.ycols_pad = pl.ycols_pad;
-        p.w_img_bytes = pl.w_img_bytes;
-        p.timeout_ns = h->timeout_ns;
-        const unsigned grid = static_cast<unsigned>(std::min<long long>(p.n_work, h->sm_count));
-        const TcEntry entry = tc_entry_for(G, pl.path == kPathStreamed, pl.nacc);
-        if (!entry.launch) return fail(EQLIN_ERR_UNSUPPORTED, "G");
-        entry.launch(grid, pl.smem_bytes, st, map, ymap, p);
-    }
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "forward launch");
+    int s = launch_forward(h->plan, h->Cout, h->Cin, h->G, h->sm_count, x, y, N, h->buf, h->timeout_ns, st);
+    if (s != EQLIN_OK) return s;
     if (h->sync_check) {
         int dst = 0;
         e = cudaStreamSynchronize(st);
         if (e != cudaSuccess) return cuda_fail(e, "forward (EQLIN_SYNC_CHECK)");
-        e = cudaMemcpy(&dst, h->status, sizeof(int), cudaMemcpyDeviceToHost);
+        e = cudaMemcpy(&dst, h->buf.status, sizeof(int), cudaMemcpyDeviceToHost);
         if (e != cudaSuccess) return cuda_fail(e, "status read");
         if (dst != 0) return fail(dst, "device reported an error (status word)");
     }
@@ -462,9 +594,9 @@ int eqlin_device_status(eqlin_handle* h, int* status_out) {
     cudaError_t e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
     int v = 0;
-    if ((e = cudaMemcpy(&v, h->status, sizeof(int), cudaMemcpyDeviceToHost)) != cudaSuccess)
+    if ((e = cudaMemcpy(&v, h->buf.status, sizeof(int), cudaMemcpyDeviceToHost)) != cudaSuccess)
         return cuda_fail(e, "status read");
-    if ((e = cudaMemset(h->status, 0, sizeof(int))) != cudaSuccess) return cuda_fail(e, "status clear");
+    if ((e = cudaMemset(h->buf.status, 0, sizeof(int))) != cudaSuccess) return cuda_fail(e, "status clear");
     *status_out = v;
     return EQLIN_OK;
 }
@@ -495,7 +627,7 @@ int eqlin_copy_freq_weights(const eqlin_handle* h, float* dst, int64_t count) {
     if (!h || !dst) return fail(EQLIN_ERR_INVALID_ARG, "NULL argument");
     const int64_t need = h->G * h->Cin * h->Cout;
     if (count < need) return fail(EQLIN_ERR_INVALID_ARG, "destination too small");
-    cudaError_t e = cudaMemcpy(dst, h->w_f32, static_cast<size_t>(need) * sizeof(float), cudaMemcpyDeviceToHost);
+    cudaError_t e = cudaMemcpy(dst, h->buf.w_f32, static_cast<size_t>(need) * sizeof(float), cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return cuda_fail(e, "copy of frequency-domain weights");
     return EQLIN_OK;
 }
@@ -539,6 +671,7 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[EQLIN_NOALLOC_S
 namespace {
 
 constexpr int kNoAllocMaxDevices = 64;
+constexpr int kNumPaths = 5;
 
 struct NoAllocDevice {
     bool ready = false;
@@ -546,7 +679,7 @@ struct NoAllocDevice {
     int sm_count = 0;
     int optin = 0;
     bool cc_ok = false;
-    uint32_t attr_done[2][4][2][2] = {};  // [f32?][G index][stream][nacc-1]: smem attribute set
+    uint8_t attr_done[kNumPaths][4][2] = {};  // [path][G index][nacc-1]: smem attribute set
 };
 
 std::mutex g_noalloc_mutex;
@@ -608,15 +741,12 @@ extern "C" int eqlin_forward_noalloc(const void* x, const void* w, const void* b
         s = plan_for(Cout, Cin, G, dtype, static_cast<size_t>(d->optin), &plan);
         if (s != EQLIN_OK) return s;
         // kernel shared-memory attribute, once per kernel and device
-        const int fi = plan.path == kPathF32 ? 1 : 0, gi = g_index(G);
-        const int si = plan.path == kPathStreamed ? 1 : 0, ai = plan.nacc == 1 ? 0 : 1;
-        if (!d->attr_done[fi][gi][si][ai]) {
-            void* k = plan.path == kPathF32 ? f32_kernel_for(static_cast<int>(G))
-                                            : tc_entry_for(static_cast<int>(G), si == 1, plan.nacc).kernel;
-            e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     static_cast<int>(plan.smem_bytes));
+        uint8_t& done = d->attr_done[plan.path][g_index(G)][plan.nacc == 1 ? 0 : 1];
+        if (!done) {
+            e = cudaFuncSetAttribute(kernel_for(plan, static_cast<int>(G)),
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(plan.smem_bytes));
             if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-            d->attr_done[fi][gi][si][ai] = 1;
+            done = 1;
         }
     }
 
@@ -644,91 +774,20 @@ extern "C" int eqlin_forward_noalloc(const void* x, const void* w, const void* b
                                                " bytes of scratch; eqlin_forward_noalloc is limited to " +
                                                std::to_string(EQLIN_NOALLOC_SCRATCH_BYTES));
     uint8_t* sc = d->scratch;
-    int* status = reinterpret_cast<int*>(sc + off_status);
-    float* bias_f32 = reinterpret_cast<float*>(sc + off_bias);
-    float* w_f32 = reinterpret_cast<float*>(sc + off_wf);
-    double* w_f64 = plan.path == kPathF32 ? reinterpret_cast<double*>(sc + off_wd) : nullptr;
-    double* bias_f64 = plan.path == kPathF32 ? reinterpret_cast<double*>(sc + off_bd) : nullptr;
-    uint8_t* img = plan.path == kPathF32 ? nullptr : sc + off_img;
+    WeightBuffers b;
+    b.status = reinterpret_cast<int*>(sc + off_status);
+    b.bias_f32 = reinterpret_cast<float*>(sc + off_bias);
+    b.w_f32 = reinterpret_cast<float*>(sc + off_wf);
+    b.w_f64 = plan.path == kPathF32 ? reinterpret_cast<double*>(sc + off_wd) : nullptr;
+    b.bias_f64 = plan.path == kPathF32 ? reinterpret_cast<double*>(sc + off_bd) : nullptr;
+    b.img = plan.path == kPathF32 ? nullptr : sc + off_img;
+    b.has_bias = bias != nullptr;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
     // the status word keeps the previous call's value: clear it
-    if ((e = cudaMemsetAsync(status, 0, sizeof(int), st)) != cudaSuccess) return cuda_fail(e, "status clear");
-
-    // weight transform into the scratch (same kernels as eqlin_prepare_weights)
-    const int threads = 256;
-    const unsigned blocks = static_cast<unsigned>((Cout * Cin + threads - 1) / threads);
-    const int iCout = static_cast<int>(Cout), iCin = static_cast<int>(Cin), iG = static_cast<int>(G);
-    if (dtype == EQLIN_F32) {
-        eqlin::eqlin_prep_freq_kernel<float><<<blocks, threads, 0, st>>>(
-            static_cast<const float*>(w), static_cast<const float*>(bias), iCout, iCin, iG, w_f32, bias_f32, w_f64,
-            bias_f64);
-    } else {
-        eqlin::eqlin_prep_freq_kernel<__nv_bfloat16><<<blocks, threads, 0, st>>>(
-            static_cast<const __nv_bfloat16*>(w), static_cast<const __nv_bfloat16*>(bias), iCout, iCin, iG, w_f32,
-            bias_f32, w_f64, bias_f64);
-    }
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "weight transform launch");
-    if (img) {
-        const size_t n = plan.img_alloc_bytes / 2;
-        eqlin::eqlin_prep_image_kernel<<<static_cast<unsigned>((n + threads - 1) / threads), threads, 0, st>>>(
-            w_f32, iCout, iCin, iG, plan.nK, plan.rows, n, img);
-        if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "weight image launch");
-    }
-
-    // the forward itself (same kernels as eqlin_forward)
-    if (plan.path == kPathF32) {
-        dim3 grid(static_cast<unsigned>((N + eqlin::kF32Tokens - 1) / eqlin::kF32Tokens),
-                  static_cast<unsigned>((Cout + 31) / 32));
-        const float* xf = static_cast<const float*>(x);
-        float* yf = static_cast<float*>(y);
-        switch (G) {
-            case 2: eqlin::eqlin_fwd_f32_kernel<2><<<grid, eqlin::kF32Threads, plan.smem_bytes, st>>>(xf, w_f64, bias_f64, yf, N, iCin, iCout); break;
-            case 4: eqlin::eqlin_fwd_f32_kernel<4><<<grid, eqlin::kF32Threads, plan.smem_bytes, st>>>(xf, w_f64, bias_f64, yf, N, iCin, iCout); break;
-            case 8: eqlin::eqlin_fwd_f32_kernel<8><<<grid, eqlin::kF32Threads, plan.smem_bytes, st>>>(xf, w_f64, bias_f64, yf, N, iCin, iCout); break;
-            default: eqlin::eqlin_fwd_f32_kernel<16><<<grid, eqlin::kF32Threads, plan.smem_bytes, st>>>(xf, w_f64, bias_f64, yf, N, iCin, iCout); break;
-        }
-    } else {
-        auto encode = tensor_map_encoder();
-        if (!encode) return fail(EQLIN_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
-        CUtensorMap map, ymap;
-        cuuint64_t dims[2] = {static_cast<cuuint64_t>(Cin * G), static_cast<cuuint64_t>(N)};
-        cuuint64_t strides[1] = {static_cast<cuuint64_t>(Cin * G * 2)};
-        cuuint32_t boxdim[2] = {static_cast<cuuint32_t>(tc_box_elems(iG)), static_cast<cuuint32_t>(plan.BN)};
-        cuuint32_t estr[2] = {1, 1};
-        CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, boxdim,
-                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        if (r != CUDA_SUCCESS) return fail(EQLIN_ERR_CUDA, "cuTensorMapEncodeTiled failed for x");
-        cuuint64_t ydims[2] = {static_cast<cuuint64_t>(Cout * G), static_cast<cuuint64_t>(N)};
-        cuuint64_t ystrides[1] = {static_cast<cuuint64_t>(Cout * G * 2)};
-        cuuint32_t ybox[2] = {static_cast<cuuint32_t>(eqlin::tc::kYBoxCols), static_cast<cuuint32_t>(plan.TG)};
-        r = encode(&ymap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, ydims, ystrides, ybox, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        if (r != CUDA_SUCCESS) return fail(EQLIN_ERR_CUDA, "cuTensorMapEncodeTiled failed for y");
-        TcParams p;
-        p.w_img = img;
-        p.bias = bias ? bias_f32 : nullptr;
-        p.y = static_cast<__nv_bfloat16*>(y);
-        p.status = status;
-        p.N = N;
-        p.Cout = iCout;
-        p.nK = plan.nK;
-        p.rows = plan.rows;
-        p.n_oc = plan.n_oc;
-        p.n_work = static_cast<int>((N + plan.BN - 1) / plan.BN * plan.n_oc);
-        p.stages = plan.stages;
-        p.w_region_bytes = plan.w_region_bytes;
-        p.ystage_bytes = plan.ystage_bytes;
-        p.ycols_pad = plan.ycols_pad;
-        p.w_img_bytes = plan.w_img_bytes;
-        p.timeout_ns = kDefaultTimeoutNs;
-        const TcEntry entry = tc_entry_for(iG, plan.path == kPathStreamed, plan.nacc);
-        if (!entry.launch) return fail(EQLIN_ERR_UNSUPPORTED, "G");
-        const unsigned grid = static_cast<unsigned>(std::min<long long>(p.n_work, d->sm_count));
-        entry.launch(grid, plan.smem_bytes, st, map, ymap, p);
-    }
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "forward launch");
-    return EQLIN_OK;
+    if ((e = cudaMemsetAsync(b.status, 0, sizeof(int), st)) != cudaSuccess) return cuda_fail(e, "status clear");
+    // weight transform into the scratch, then the forward (same kernels as the handle API)
+    s = launch_prep(plan, dtype, w, bias, Cout, Cin, G, b, st);
+    if (s != EQLIN_OK) return s;
+    return launch_forward(plan, Cout, Cin, G, d->sm_count, x, y, N, b, kDefaultTimeoutNs, st);
 }

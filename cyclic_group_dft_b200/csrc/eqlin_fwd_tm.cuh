@@ -1,0 +1,422 @@
+// eqlin_fwd_tm.cuh -- fused EQ-Linear forward with tokens on the MMA M dimension.
+//
+// Same operation and steps as eqlin_fwd_tc.cuh (page "Flash EQ-Linear: Accelerating
+// Equivariant Linear Layers via Group-wise Discrete Fourier Transform", sections
+// "Enfoque Algoritmico" and "Implementacion"), with the operand roles of the
+// per-frequency products swapped:
+//   A = X^ plane [128 tokens x 16 channels]  (M = 128 tokens)
+//   B = W^ plane [NO output channels x 16]   (N = NO <= 512/G, a multiple of 32)
+//   D = TMEM, lane = token, column = output channel, one plane per frequency component
+// A work item (128 tokens, NO output channels) needs 2G-2 MMAs per 16 input channels,
+// independent of how many output channels it covers, so small Cout configurations
+// issue 4-8x fewer MMAs than with tokens on N.  G*NO <= 512 TMEM columns leaves room for
+// one accumulator: the MMAs of a tile wait for the epilogue of the previous tile to
+// release it (the epilogue releases it as soon as its last TMEM load has landed).
+//
+// Roles per CTA (one per SM, persistent):
+//   producer warp    TMA loads of x chunks [128 tokens x 16 channels x G] (+ the weight
+//                    chunk when the weights are streamed) into a smem ring
+//   DW DFT warps     in-place real DFT over G: x chunk -> G planes, K-major SWIZZLE_32B
+//   MMA warp         one thread issues tcgen05.mma (2 real + 4 per complex frequency)
+//   8 epilogue warps lane = token; per group of 32/G output channels: tcgen05.ld of the
+//                    G planes, inverse real DFT + bias, bf16, into a SWIZZLE_64B staging
+//                    tile [128 tokens x 32 columns], TMA store (rows past N and columns
+//                    past Cout*G clipped); warps w and w+4 split the output channels
+// Waits are bounded as in eqlin_fwd_tc.cuh.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "eqlin_fwd_tc.cuh"
+#include "eqlin_layout.h"
+#include "group_dft.cuh"
+#include "sm100_ptx.cuh"
+
+namespace eqlin {
+
+struct TmParams {
+    const uint8_t* w_img;   // weight image, image_offset_k16 layout with NO rows per sub-block
+    const float* bias;      // [Cout] fp32, or nullptr
+    int* status;
+    long long N;
+    int Cout;
+    int nK;                 // 16-channel chunks along Cin
+    int NO;                 // output channels per work item (MMA N)
+    int n_oc;               // output chunks
+    int n_work;             // token tiles * n_oc
+    int stages;
+    uint32_t w_region_bytes;  // resident weights (0 when streamed)
+    uint32_t w_img_bytes;
+    unsigned long long timeout_ns;
+};
+
+namespace tm {
+
+constexpr int kM = 128;                          // tokens per tile (MMA M)
+constexpr int kEpiWarps = 8;
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kBarDft = 1;
+constexpr int kBarEpi = 2;
+constexpr int kBarEpiHalf0 = 3;                  // 3 and 4
+constexpr int kYCols = 32;                       // staged y columns per group (64 B rows)
+constexpr int kYBufBytes = kM * kYCols * 2;      // 8 KB
+constexpr int kYBufs = 4;                        // 2 per epilogue half
+
+template <int G>
+struct Cfg {
+    static constexpr int DW = G == 16 ? 8 : 4;               // DFT warps
+    static constexpr int kDftThreads = DW * 32;
+    static constexpr int kWarpDft0 = kEpiWarps;
+    static constexpr int kWarpProducer = kEpiWarps + DW;
+    static constexpr int kWarpMma = kEpiWarps + DW + 1;
+    static constexpr int kThreads = (kEpiWarps + DW + 2) * 32;
+    static constexpr int PLANE_BYTES = kM * kRowBytes32;      // 4 KB
+    static constexpr int XCHUNK_BYTES = G * PLANE_BYTES;      // 128 tokens x 16 ch x G x 2
+    static constexpr int XROW_ELEMS = kChunkK16 * G;          // <= 256 (one TMA box)
+    static constexpr int NMAX = (512 / G) < 256 ? (512 / G) : 256;
+    static constexpr int OG = 32 / G;                         // output channels per group
+    static_assert(XROW_ELEMS <= 256, "x box");
+    static_assert(XCHUNK_BYTES % 1024 == 0, "stage alignment");
+};
+
+// --------------------------------------------------------------- DFT role
+// Unit = one token row x two adjacent channels (2*G bf16).  Lane l: row offset l/8,
+// channel pair l%8; a warp covers 4 rows per step.
+template <int G>
+__device__ __forceinline__ void dft_chunk(uint8_t* xs, int dft_tid) {
+    using C = Cfg<G>;
+    constexpr int WORDS = G;
+    constexpr int ROWS_PER_STEP = C::kDftThreads / 8;
+    constexpr int STEPS = kM / ROWS_PER_STEP;
+    const int warp = dft_tid >> 5, lane = dft_tid & 31;
+    const int pair = lane & 7;
+    const int row0 = warp * 4 + (lane >> 3);
+    const uint8_t* src0 = xs + pair * (4 * G);
+    uint32_t w[STEPS][WORDS];
+#pragma unroll
+    for (int s = 0; s < STEPS; ++s) {
+        const uint8_t* src = src0 + (row0 + s * ROWS_PER_STEP) * (C::XROW_ELEMS * 2);
+        if constexpr (WORDS == 2) {
+            const uint2 v = *reinterpret_cast<const uint2*>(src);
+            w[s][0] = v.x;
+            w[s][1] = v.y;
+        } else {
+#pragma unroll
+            for (int c = 0; c < WORDS / 4; ++c) {
+                const uint4 v = *reinterpret_cast<const uint4*>(src + 16 * c);
+                w[s][4 * c + 0] = v.x;
+                w[s][4 * c + 1] = v.y;
+                w[s][4 * c + 2] = v.z;
+                w[s][4 * c + 3] = v.w;
+            }
+        }
+    }
+    ptx::named_bar_sync(kBarDft, C::kDftThreads);   // all reads before any in-place write
+    const int in_piece = (pair & 3) * 4;
+#pragma unroll
+    for (int s = 0; s < STEPS; ++s) {
+        const int r = row0 + s * ROWS_PER_STEP;
+        float xa[G], xb[G];
+#pragma unroll
+        for (int h = 0; h < G / 2; ++h) {
+            const uint32_t ua = w[s][h], ub = w[s][G / 2 + h];
+            xa[2 * h] = __uint_as_float(ua << 16);
+            xa[2 * h + 1] = __uint_as_float(ua & 0xFFFF0000u);
+            xb[2 * h] = __uint_as_float(ub << 16);
+            xb[2 * h + 1] = __uint_as_float(ub & 0xFFFF0000u);
+        }
+        float pa[G], pb[G];
+        rdft_planes<G>(xa, pa);
+        rdft_planes<G>(xb, pb);
+        const int phys = ((pair >> 2) ^ ((r >> 2) & 1)) * 16 + in_piece;   // SWIZZLE_32B
+        uint8_t* dst = xs + r * kRowBytes32 + phys;
+#pragma unroll
+        for (int p = 0; p < G; ++p)
+            *reinterpret_cast<uint32_t*>(dst + p * C::PLANE_BYTES) = tc::pack_bf16x2(pa[p], pb[p]);
+    }
+}
+
+// ------------------------------------------------------------ epilogue role
+// Warp (q, half): tokens 32q..32q+31 (TMEM lane quarter q), output channels
+// [half*NO/2, (half+1)*NO/2) of the work item, in groups of OG = 32/G channels.
+// Arrives on `acc_empty` once its last TMEM load has landed.
+template <int G>
+__device__ __forceinline__ void epilogue_tile(const TmParams& p, const CUtensorMap* tmap_y, uint32_t tmem,
+                                              int q, int half, int lane, long long n0, int oc, uint8_t* ystage,
+                                              int& ybuf, bool leader, uint32_t acc_empty) {
+    using C = Cfg<G>;
+    constexpr int OG = C::OG;
+    const int n_groups = (p.NO / 2) / OG;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    const uint32_t bar_half = kBarEpiHalf0 + half;
+    const int row = q * 32 + lane;                 // token row inside the tile
+    const int swz = (row >> 1) & 3;                // SWIZZLE_64B of the staging rows
+#pragma unroll 1
+    for (int g = 0; g < n_groups; ++g) {
+        const int o_loc0 = half * (p.NO / 2) + g * OG;
+        uint32_t r[G][OG];
+#pragma unroll
+        for (int pl = 0; pl < G; ++pl) ptx::tmem_ld_32x32b<OG>(lane_addr + pl * p.NO + o_loc0, r[pl]);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int pl = 0; pl < G; ++pl) ptx::tmem_regs_ready<OG>(r[pl]);
+        if (g == n_groups - 1) {
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(acc_empty);           // TMEM no longer needed by this thread
+        }
+        const int o0 = oc * p.NO + o_loc0;
+        float yv[OG * G];
+#pragma unroll
+        for (int j = 0; j < OG; ++j) {
+            float z[G], y1[G];
+#pragma unroll
+            for (int pl = 0; pl < G; ++pl) z[pl] = __uint_as_float(r[pl][j]);
+            const int o = o0 + j;
+            z[0] += (p.bias != nullptr && o < p.Cout) ? __ldg(p.bias + o) : 0.0f;
+            RealIdft<G>::run(z, y1);
+#pragma unroll
+            for (int gg = 0; gg < G; ++gg) yv[j * G + gg] = y1[gg];
+        }
+        // the buffer was last stored two groups ago: wait until the TMA engine read it
+        if (leader) ptx::bulk_wait_group_read<1>();
+        ptx::named_bar_sync(bar_half, 128);
+        uint8_t* buf = ystage + static_cast<size_t>(ybuf) * kYBufBytes;
+        uint8_t* rowp = buf + row * (kYCols * 2);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            *reinterpret_cast<uint4*>(rowp + ((k ^ swz) * 16)) =
+                make_uint4(tc::pack_bf16x2(yv[8 * k + 0], yv[8 * k + 1]), tc::pack_bf16x2(yv[8 * k + 2], yv[8 * k + 3]),
+                           tc::pack_bf16x2(yv[8 * k + 4], yv[8 * k + 5]), tc::pack_bf16x2(yv[8 * k + 6], yv[8 * k + 7]));
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::named_bar_sync(bar_half, 128);
+        if (leader) {
+            // a store only starts inside the tensor; its clipped parts are not written
+            if (n0 < p.N && o0 < p.Cout)
+                ptx::tma_store_2d(tmap_y, ptx::smem_u32(buf), o0 * G, static_cast<int>(n0));
+            ptx::bulk_commit_group();
+        }
+        ybuf ^= 1;
+    }
+}
+
+}  // namespace tm
+
+template <int G, bool STREAM_W>
+__global__ void __launch_bounds__(tm::Cfg<G>::kThreads, 1)
+    eqlin_fwd_tm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_y,
+                        const TmParams p) {
+    using C = tm::Cfg<G>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+
+    const uint32_t wstage_bytes = STREAM_W ? static_cast<uint32_t>(G * p.NO * kRowBytes32) : 0u;
+    const uint32_t stage_bytes = C::XCHUNK_BYTES + wstage_bytes;
+    const int NS = p.stages;
+    uint8_t* ystage0 = smem + p.w_region_bytes;
+    uint8_t* stage0 = ystage0 + tm::kYBufs * tm::kYBufBytes;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(stage0 + static_cast<size_t>(NS) * stage_bytes);
+    tc::Ctl* ctl = reinterpret_cast<tc::Ctl*>(bars + 3 * NS + 4);
+
+    const uint32_t s_w = ptx::smem_u32(smem);
+    const uint32_t s_stage0 = ptx::smem_u32(stage0);
+    auto bar_full = [&](int s) { return ptx::smem_u32(bars + s); };
+    auto bar_xhat = [&](int s) { return ptx::smem_u32(bars + NS + s); };
+    auto bar_empty = [&](int s) { return ptx::smem_u32(bars + 2 * NS + s); };
+    const uint32_t bar_acc_full = ptx::smem_u32(bars + 3 * NS + 0);
+    const uint32_t bar_acc_empty = ptx::smem_u32(bars + 3 * NS + 1);
+    const uint32_t bar_w_full = ptx::smem_u32(bars + 3 * NS + 2);
+    const uint32_t bar_drain = ptx::smem_u32(bars + 3 * NS + 3);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; ++s) {
+            ptx::mbar_init(bar_full(s), 1);
+            ptx::mbar_init(bar_xhat(s), C::kDftThreads);
+            ptx::mbar_init(bar_empty(s), 1);
+        }
+        ptx::mbar_init(bar_acc_full, 1);
+        ptx::mbar_init(bar_acc_empty, tm::kEpiThreads);
+        ptx::mbar_init(bar_w_full, 1);
+        ptx::mbar_init(bar_drain, 1);
+        ctl->abort = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == C::kWarpMma) {
+        ptx::tmem_alloc(ptx::smem_u32(&ctl->tmem_base), 512);
+        ptx::tmem_relinquish();
+    }
+    if (warp == C::kWarpProducer && lane == 0) {
+        ptx::prefetch_tmap(&tmap_x);
+        ptx::prefetch_tmap(&tmap_y);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = ctl->tmem_base;
+
+    if (warp == C::kWarpProducer) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            if constexpr (!STREAM_W) {
+                ptx::mbar_arrive_expect_tx(bar_w_full, p.w_img_bytes);
+                for (uint32_t off = 0; off < p.w_img_bytes; off += 32768u)
+                    ptx::bulk_load(s_w + off, p.w_img + off, min(32768u, p.w_img_bytes - off), bar_w_full);
+            }
+            int stage = 0;
+            uint32_t phase = 0;
+            long long issued = 0;
+            bool ok = true;
+            for (int wk = blockIdx.x; ok && wk < p.n_work; wk += gridDim.x) {
+                const int tile = wk / p.n_oc, oc = wk % p.n_oc;
+                const int n0 = tile * tm::kM;
+                for (int c = 0; c < p.nK; ++c) {
+                    if (!tc::wait_bounded(bar_empty(stage), phase ^ 1u, ctl, p.status, p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t dst = s_stage0 + stage * stage_bytes;
+                    ptx::mbar_arrive_expect_tx(bar_full(stage), stage_bytes);
+                    ptx::tma_load_2d(dst, &tmap_x, c * C::XROW_ELEMS, n0, bar_full(stage));
+                    if constexpr (STREAM_W) {
+                        ptx::bulk_load(dst + C::XCHUNK_BYTES,
+                                       p.w_img + static_cast<size_t>(oc * p.nK + c) * wstage_bytes, wstage_bytes,
+                                       bar_full(stage));
+                    }
+                    ++issued;
+                    if (++stage == NS) { stage = 0; phase ^= 1u; }
+                }
+            }
+            // drain: every copy started here lands before the CTA exits (bounded)
+            for (int s = 0; s < NS; ++s) {
+                const long long times = issued > s ? (issued - s + NS - 1) / NS : 0;
+                if (times > 0) {
+                    const uint32_t par = static_cast<uint32_t>((times - 1) & 1);
+                    const uint64_t t0 = ptx::globaltimer_ns();
+                    while (!ptx::mbar_try_wait(bar_full(s), par)) {
+                        if (ptx::globaltimer_ns() - t0 > p.timeout_ns) {
+                            atomicCAS(p.status, 0, kDeviceErrTimeout);
+                            break;
+                        }
+                    }
+                }
+            }
+            if constexpr (!STREAM_W) {
+                const uint64_t t0 = ptx::globaltimer_ns();
+                while (!ptx::mbar_try_wait(bar_w_full, 0)) {
+                    if (ptx::globaltimer_ns() - t0 > p.timeout_ns) {
+                        atomicCAS(p.status, 0, kDeviceErrTimeout);
+                        break;
+                    }
+                }
+            }
+        }
+    } else if (warp == C::kWarpMma) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            bool ok = true;
+            if constexpr (!STREAM_W) ok = tc::wait_bounded(bar_w_full, 0, ctl, p.status, p.timeout_ns);
+            const uint32_t ID = idesc_bf16_f32(tm::kM, p.NO, false, false);
+            const uint32_t ID_NEG = idesc_bf16_f32(tm::kM, p.NO, false, true);
+            const uint32_t wplane = static_cast<uint32_t>(p.NO) * kRowBytes32;
+            int stage = 0;
+            uint32_t phase = 0;
+            int it = 0;
+            for (int wk = blockIdx.x; ok && wk < p.n_work; wk += gridDim.x, ++it) {
+                if (!tc::wait_bounded(bar_acc_empty, (static_cast<uint32_t>(it) & 1u) ^ 1u, ctl, p.status,
+                                      p.timeout_ns)) {
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+                for (int c = 0; c < p.nK; ++c) {
+                    if (!tc::wait_bounded(bar_xhat(stage), phase, ctl, p.status, p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint32_t xb = s_stage0 + stage * stage_bytes;
+                    const uint32_t wb = STREAM_W ? xb + C::XCHUNK_BYTES
+                                                 : s_w + static_cast<uint32_t>(c * G) * wplane;
+                    const uint32_t a_lo = ptx::sdesc_sw32_lo(xb), b_lo = ptx::sdesc_sw32_lo(wb);
+                    const uint32_t wplane16 = wplane >> 4;
+                    const uint32_t acc0 = c > 0 ? 1u : 0u;
+                    auto A = [&](int pl) { return ptx::sdesc_sw32_from_lo(a_lo + (pl * C::PLANE_BYTES) / 16); };
+                    auto B = [&](int pl) { return ptx::sdesc_sw32_from_lo(b_lo + static_cast<uint32_t>(pl) * wplane16); };
+                    auto D = [&](int pl) { return tmem_base + static_cast<uint32_t>(pl * p.NO); };
+                    ptx::umma_f16(D(0), A(0), B(0), ID, acc0);          // k = 0
+                    ptx::umma_f16(D(1), A(1), B(1), ID, acc0);          // k = G/2
+#pragma unroll
+                    for (int k = 1; k < G / 2; ++k) {                   // (Xr + i Xi)(Wr + i Wi)
+                        const int pr = 2 * k, pi = 2 * k + 1;
+                        ptx::umma_f16(D(pr), A(pr), B(pr), ID, acc0);       // + Xr Wr
+                        ptx::umma_f16(D(pr), A(pi), B(pi), ID_NEG, 1u);     // - Xi Wi
+                        ptx::umma_f16(D(pi), A(pr), B(pi), ID, acc0);       // + Xr Wi
+                        ptx::umma_f16(D(pi), A(pi), B(pr), ID, 1u);         // + Xi Wr
+                    }
+                    ptx::umma_commit(bar_empty(stage));
+                    if (++stage == NS) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                ptx::umma_commit(bar_acc_full);
+            }
+            ptx::umma_commit(bar_drain);
+            const uint64_t t0 = ptx::globaltimer_ns();
+            while (!ptx::mbar_try_wait(bar_drain, 0)) {
+                if (ptx::globaltimer_ns() - t0 > p.timeout_ns) {
+                    atomicCAS(p.status, 0, kDeviceErrTimeout);
+                    break;
+                }
+            }
+        }
+    } else if (warp >= C::kWarpDft0) {
+        // ------------------------------------------------------------ DFT warps
+        const int dft_tid = threadIdx.x - C::kWarpDft0 * 32;
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int wk = blockIdx.x; wk < p.n_work; wk += gridDim.x) {
+            bool ok = true;
+            for (int c = 0; c < p.nK; ++c) {
+                const bool got = tc::wait_bounded(bar_full(stage), phase, ctl, p.status, p.timeout_ns);
+                if (!ptx::named_bar_and(tm::kBarDft, C::kDftThreads, got)) {
+                    ok = false;
+                    break;
+                }
+                tm::dft_chunk<G>(stage0 + static_cast<size_t>(stage) * stage_bytes, dft_tid);
+                ptx::fence_proxy_async_smem();
+                ptx::mbar_arrive(bar_xhat(stage));
+                if (++stage == NS) { stage = 0; phase ^= 1u; }
+            }
+            if (!ok) break;
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue warps
+        const int half = warp >> 2;
+        const bool leader = (warp & 3) == 0 && lane == 0;
+        uint8_t* ystage = ystage0 + static_cast<size_t>(2 * half) * tm::kYBufBytes;
+        int ybuf = 0;
+        int it = 0;
+        for (int wk = blockIdx.x; wk < p.n_work; wk += gridDim.x, ++it) {
+            const bool got = tc::wait_bounded(bar_acc_full, static_cast<uint32_t>(it) & 1u, ctl, p.status,
+                                              p.timeout_ns);
+            if (!ptx::named_bar_and(tm::kBarEpi, tm::kEpiThreads, got)) break;
+            ptx::tc_fence_after();
+            const int tile = wk / p.n_oc, oc = wk % p.n_oc;
+            tm::epilogue_tile<G>(p, &tmap_y, tmem_base, warp & 3, half, lane,
+                                 static_cast<long long>(tile) * tm::kM, oc, ystage, ybuf, leader, bar_acc_empty);
+        }
+        if (leader) ptx::bulk_wait_group<0>();
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == C::kWarpMma) {
+        __syncwarp();
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem_base, 512);
+    }
+}
+
+}  // namespace eqlin

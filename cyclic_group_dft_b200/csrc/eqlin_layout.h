@@ -38,4 +38,15 @@ __host__ __device__ inline size_t image_offset(size_t sub, int rows, int r, int 
            static_cast<size_t>(piece) * 16 + static_cast<size_t>(col & 7) * 2;
 }
 
+// Tokens-on-M kernel variant: 16-channel K chunks, rows of 32 bytes, SWIZZLE_32B
+// (16-byte piece j of row r stored at piece j ^ ((r >> 2) & 1)).  Image layout
+// [oc][c][p][r < rows][16].
+constexpr int kChunkK16 = 16;
+constexpr int kRowBytes32 = 32;
+__host__ __device__ inline size_t image_offset_k16(size_t sub, int rows, int r, int col) {
+    const int piece = (col >> 3) ^ ((r >> 2) & 1);
+    return sub * static_cast<size_t>(rows) * kRowBytes32 + static_cast<size_t>(r) * kRowBytes32 +
+           static_cast<size_t>(piece) * 16 + static_cast<size_t>(col & 7) * 2;
+}
+
 }  // namespace eqlin

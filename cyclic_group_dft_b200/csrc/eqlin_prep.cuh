@@ -80,6 +80,25 @@ __global__ void eqlin_prep_image_kernel(const float* __restrict__ w_f32, int Cou
     *reinterpret_cast<__nv_bfloat16*>(img + image_offset(sub, rows, r, col)) = __float2bfloat16_rn(v);
 }
 
+// Image for the tokens-on-M kernel (layout: image_offset_k16).  `rows` rows per
+// sub-block; output chunk oc covers o = oc*rows + r.
+__global__ void eqlin_prep_image_k16_kernel(const float* __restrict__ w_f32, int Cout, int Cin, int G,
+                                            int nK, int rows, size_t n_elems, uint8_t* __restrict__ img) {
+    const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx >= n_elems) return;
+    const int col = static_cast<int>(idx % kChunkK16);
+    const int r = static_cast<int>((idx / kChunkK16) % rows);
+    const size_t sub = idx / (static_cast<size_t>(kChunkK16) * rows);
+    const int p = static_cast<int>(sub % G);
+    const int c = static_cast<int>((sub / G) % nK);
+    const int oc = static_cast<int>(sub / (static_cast<size_t>(G) * nK));
+    const int o = oc * rows + r;
+    const int i = c * kChunkK16 + col;
+    float v = 0.0f;
+    if (o < Cout && i < Cin) v = w_f32[(static_cast<size_t>(p) * Cin + i) * Cout + o];
+    *reinterpret_cast<__nv_bfloat16*>(img + image_offset_k16(sub, rows, r, col)) = __float2bfloat16_rn(v);
+}
+
 // ------------------------------------------------------------------ fp32 path
 // Fused forward for fp32 I/O on CUDA cores.  The tensor-core kinds that take fp32
 // operands round them to tf32 (10-bit mantissa), far from a 1e-5 bound, so this

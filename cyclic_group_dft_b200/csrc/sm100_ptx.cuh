@@ -188,6 +188,10 @@ template <int N>
 __device__ __forceinline__ void tmem_ld_32x32b(uint32_t taddr, uint32_t (&r)[N]);
 
 template <>
+__device__ __forceinline__ void tmem_ld_32x32b<2>(uint32_t taddr, uint32_t (&r)[2]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(taddr));
+}
+template <>
 __device__ __forceinline__ void tmem_ld_32x32b<4>(uint32_t taddr, uint32_t (&r)[4]) {
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
@@ -238,6 +242,14 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_sw64(uint32_t start) {
     return d;                                            // base offset 0, LBO mode 0
 }
 
+// K-major operand with 32-byte swizzle: rows of 32 B (16 bf16 along K = one MMA K
+// step), 8-row atoms of 256 B stacked along M/N.
+__device__ __forceinline__ uint32_t sdesc_sw32_lo(uint32_t start) { return (1u << 16) | (start >> 4); }
+constexpr uint32_t kSdescSw32Hi = (256u >> 4) | (1u << 14) | (6u << 29);
+__device__ __forceinline__ uint64_t sdesc_sw32_from_lo(uint32_t lo) {
+    return (static_cast<uint64_t>(kSdescSw32Hi) << 32) | lo;
+}
+
 // The same descriptor split in halves: only the start-address field (low 14 bits)
 // varies between operands, so the issuing loop adds (byte offset >> 4) to the low
 // half and pairs it with the constant high half.
@@ -251,11 +263,12 @@ __device__ __forceinline__ uint64_t sdesc_sw64_from_lo(uint32_t lo) {
 
 // Instruction descriptor for tcgen05.mma kind::f16 with bf16 A/B, fp32 D, both
 // operands K-major.  M in {64,128}, N a multiple of 16 up to 256.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool negate_a) {
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool negate_a, bool negate_b = false) {
     return (1u << 4)                                  // D format: F32
            | (1u << 7)                                // A format: BF16
            | (1u << 10)                               // B format: BF16
            | ((negate_a ? 1u : 0u) << 13)             // negate A
+           | ((negate_b ? 1u : 0u) << 14)             // negate B
            | (static_cast<uint32_t>(N >> 3) << 17)    // N >> 3
            | (static_cast<uint32_t>(M >> 4) << 24);   // M >> 4
 }
