@@ -17,6 +17,9 @@ module only marshals numpy arrays to it.  Functions:
   half spectrum (section "Enfoque Algoritmico", conjugate symmetry);
 * :func:`forward_fourier`  -- the method's algorithm: DFT, per-frequency
   complex contraction, inverse DFT, bias (section "Enfoque Algoritmico");
+* :func:`backward_dx`, :func:`backward_dw` -- the gradients of a loss with
+  respect to x, and to w and bias, by the chain rule on the definition (the
+  backward pass of section "Implementacion");
 * :func:`dense_flops`, :func:`fourier_flops` -- the operation counts of the
   naive and the Fourier-domain contraction (sections "Enfoque Algoritmico",
   "Especializacion para el Grupo de Rotacion p4").
@@ -44,12 +47,15 @@ def _load():
         lib.eqlin_oracle_dense_weight_f64.argtypes = [dp, i64, i64, i64, dp]
         lib.eqlin_oracle_rdft_f64.argtypes = [dp, i64, i64, dp, dp]
         lib.eqlin_oracle_irdft_f64.argtypes = [dp, dp, i64, i64, dp]
+        lib.eqlin_oracle_backward_dx_f64.argtypes = [dp, dp, i64, i64, i64, i64, dp, ip]
+        lib.eqlin_oracle_backward_dw_f64.argtypes = [dp, dp, i64, i64, i64, i64, dp, dp, ip]
         lib.eqlin_oracle_num_freqs.argtypes = [i64]
         lib.eqlin_oracle_num_freqs.restype = i64
         lib.eqlin_oracle_max_threads.restype = ctypes.c_int
         for f in ("eqlin_oracle_forward_f64", "eqlin_oracle_forward_fourier_f64",
                   "eqlin_oracle_dense_weight_f64", "eqlin_oracle_rdft_f64",
-                  "eqlin_oracle_irdft_f64"):
+                  "eqlin_oracle_irdft_f64", "eqlin_oracle_backward_dx_f64",
+                  "eqlin_oracle_backward_dw_f64"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -107,6 +113,41 @@ def forward_fourier(x, w, bias=None, threads: int = 0) -> np.ndarray:
         _ptr(x), _ptr(w), None if b is None else _ptr(b), N, Cin, Cout, G, _ptr(y), int(threads))
     _check(st, "forward_fourier")
     return y
+
+
+def backward_dx(dy, w, threads: int = 0) -> np.ndarray:
+    """Gradient with respect to x: dx[n,i,h] = sum_{o,g} w[o,i,(g-h) mod G] dy[n,o,g].
+
+    dy [N, Cout, G], w [Cout, Cin, G] -> dx [N, Cin, G], float64.
+    """
+    dy, w = _f64(dy), _f64(w)
+    N, Cout, G = dy.shape
+    Cin = w.shape[1]
+    if w.shape != (Cout, Cin, G):
+        raise ValueError(f"w shape {w.shape} does not match dy shape {dy.shape}")
+    dx = np.empty((N, Cin, G), dtype=np.float64)
+    st = _load().eqlin_oracle_backward_dx_f64(_ptr(dy), _ptr(w), N, Cin, Cout, G, _ptr(dx), int(threads))
+    _check(st, "backward_dx")
+    return dx
+
+
+def backward_dw(dy, x, threads: int = 0) -> tuple[np.ndarray, np.ndarray]:
+    """Gradients with respect to w and bias:
+    dw[o,i,m] = sum_{n,g} dy[n,o,g] x[n,i,(g-m) mod G], dbias[o] = sum_{n,g} dy[n,o,g].
+
+    dy [N, Cout, G], x [N, Cin, G] -> (dw [Cout, Cin, G], dbias [Cout]), float64.
+    """
+    dy, x = _f64(dy), _f64(x)
+    N, Cout, G = dy.shape
+    if x.shape[0] != N or x.shape[2] != G:
+        raise ValueError(f"x shape {x.shape} does not match dy shape {dy.shape}")
+    Cin = x.shape[1]
+    dw = np.empty((Cout, Cin, G), dtype=np.float64)
+    db = np.empty((Cout,), dtype=np.float64)
+    st = _load().eqlin_oracle_backward_dw_f64(_ptr(dy), _ptr(x), N, Cin, Cout, G, _ptr(dw), _ptr(db),
+                                              int(threads))
+    _check(st, "backward_dw")
+    return dw, db
 
 
 def dense_weight(w) -> np.ndarray:
