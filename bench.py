@@ -39,8 +39,13 @@ from cyclic_group_dft_b200 import workloads  # noqa: E402
 METRIC = "EQ-Linear tokens/s and % of roofline (HBM vs bf16 TC), p4 Cin=Cout=96"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_BYTES = 126 * 1024 * 1024
-KERNEL_SOURCES = ["eqlin_fwd_tc.cuh", "group_dft.cuh", "sm100_ptx.cuh", "eqlin_layout.h", "eqlin_api.cu"]
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "eqlin_fwd_tc_traffic.json")
+# device code of each fused kernel: a recorded ncu traffic figure is reported only
+# while these files are unchanged since the capture
+KERNEL_SOURCES = {
+    "eqlin_fwd_tc": ["eqlin_fwd_tc.cuh", "group_dft.cuh", "sm100_ptx.cuh", "eqlin_layout.h"],
+    "eqlin_fwd_tm": ["eqlin_fwd_tm.cuh", "group_dft.cuh", "sm100_ptx.cuh", "eqlin_layout.h"],
+}
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "eqlin_fwd_traffic.json")
 
 # NVML clock-event reason bits
 REASON_BITS = {
@@ -78,9 +83,9 @@ def load_peaks() -> tuple[dict, str]:
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
-    for name in KERNEL_SOURCES:
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "cyclic_group_dft_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -94,7 +99,9 @@ def recorded_traffic(workload: str):
     except (OSError, ValueError):
         return None
     entry = d.get(workload)
-    if not entry or entry.get("source_hash") != kernel_source_hash():
+    if not entry or entry.get("kernel") not in KERNEL_SOURCES:
+        return None
+    if entry.get("source_hash") != kernel_source_hash(entry["kernel"]):
         return None
     return entry.get("dram_bytes_per_launch")
 

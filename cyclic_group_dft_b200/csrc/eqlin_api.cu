@@ -58,7 +58,7 @@ struct Plan {
     int BN = 0;          // tokens per work item
     int stages = 0;
     int TG = 0;          // y TMA store box rows (tokens-on-N)
-    int ycols_pad = 0;   // staged y columns per group (tokens-on-N)
+    int ybufs = 0;       // y staging buffers per epilogue warp (tokens-on-N)
     int box_elems = 0;   // x TMA box columns
     uint32_t w_region_bytes = 0, w_img_bytes = 0, ystage_bytes = 0;
     size_t smem_bytes = 0;
@@ -68,8 +68,19 @@ struct Plan {
 };
 
 // ----------------------------------------------------------------- planning
+// Tuning overrides read from the environment: EQLIN_MAX_STAGES caps the ring depth,
+// EQLIN_YBUFS (1 or 2) fixes the tokens-on-N y staging depth.
+int env_int(const char* name, int dflt) {
+    const char* e = std::getenv(name);
+    if (!e || !*e) return dflt;
+    const int v = std::atoi(e);
+    return v > 0 ? v : dflt;
+}
+
 template <int G, int NACC>
 int plan_tn_g(int64_t Cout, int64_t Cin, size_t max_smem, Plan* pl) {
+    const int max_stages = std::min(kMaxStages, env_int("EQLIN_MAX_STAGES", kMaxStages));
+    const int ybufs_env = env_int("EQLIN_YBUFS", 0);
     using S = eqlin::tc::Shape<G, NACC>;
     pl->nacc = NACC;
     pl->nK = static_cast<int>((Cin + eqlin::kChunkK - 1) / eqlin::kChunkK);
@@ -77,50 +88,63 @@ int plan_tn_g(int64_t Cout, int64_t Cin, size_t max_smem, Plan* pl) {
     pl->BN = S::BN;
     pl->TG = S::TG;
     pl->box_elems = S::BOX_ELEMS;
-    // y staging: 4 buffers (2 per epilogue half) of TG rows x the chunk's y columns
-    const int64_t chunk_rows = std::min<int64_t>(Cout, eqlin::kMmaM);
-    pl->ycols_pad = static_cast<int>((chunk_rows * G + eqlin::tc::kYBoxCols - 1) / eqlin::tc::kYBoxCols *
-                                     eqlin::tc::kYBoxCols);
-    pl->ystage_bytes = static_cast<uint32_t>(S::TG * pl->ycols_pad * 2);
-    const size_t fixed = kSmemAlignSlack + kSmemCtlBytes + 4 * static_cast<size_t>(pl->ystage_bytes);
-    if (pl->n_oc == 1) {
-        // weights resident in shared memory for the whole kernel
-        const int rows = static_cast<int>((Cout + 7) / 8 * 8);
-        const size_t img = static_cast<size_t>(G) * pl->nK * rows * eqlin::kPlaneRowBytes;
-        // the A operand always reads 128 rows: keep the overrun of the last block inside
-        const size_t region = (img + static_cast<size_t>(eqlin::kMmaM - rows) * eqlin::kPlaneRowBytes +
-                               1023) / 1024 * 1024;
-        if (max_smem > fixed + region) {
-            const size_t stages = std::min<size_t>(kMaxStages, (max_smem - fixed - region) / S::XCHUNK_BYTES);
-            if (stages >= 2) {
-                pl->path = kPathResident;
-                pl->rows = rows;
+    // y staging: per epilogue warp, ybufs buffers of TG rows x 32*G bf16 columns (4 KB);
+    // double-buffered when at least 5 ring stages still fit
+    const size_t ybuf = static_cast<size_t>(S::TG) * 32 * G * 2;
+    auto fixed_for = [&](int nb) {
+        return kSmemAlignSlack + kSmemCtlBytes + static_cast<size_t>(eqlin::tc::kEpiWarps) * nb * ybuf;
+    };
+    pl->ybufs = 2;
+    for (int nb = 2; nb >= 1; --nb) {
+        if (ybufs_env && nb != ybufs_env) continue;
+        const size_t fixed = fixed_for(nb);
+        pl->ybufs = nb;
+        pl->ystage_bytes = static_cast<uint32_t>(nb * ybuf);
+        if (pl->n_oc == 1) {
+            // weights resident in shared memory for the whole kernel
+            const int rows = static_cast<int>((Cout + 7) / 8 * 8);
+            const size_t img = static_cast<size_t>(G) * pl->nK * rows * eqlin::kPlaneRowBytes;
+            // the A operand always reads 128 rows: keep the overrun of the last block inside
+            const size_t region = (img + static_cast<size_t>(eqlin::kMmaM - rows) * eqlin::kPlaneRowBytes +
+                                   1023) / 1024 * 1024;
+            if (max_smem > fixed + region) {
+                const size_t stages =
+                    std::min<size_t>(max_stages, (max_smem - fixed - region) / S::XCHUNK_BYTES);
+                if (stages >= static_cast<size_t>(nb == 2 && !ybufs_env ? 5 : 2)) {
+                    pl->path = kPathResident;
+                    pl->rows = rows;
+                    pl->stages = static_cast<int>(stages);
+                    pl->w_region_bytes = static_cast<uint32_t>(region);
+                    pl->w_img_bytes = static_cast<uint32_t>(img);
+                    pl->img_alloc_bytes = img;
+                    pl->smem_bytes = fixed + region + stages * S::XCHUNK_BYTES;
+                    return EQLIN_OK;
+                }
+            }
+        }
+        // weights streamed chunk by chunk next to each x chunk
+        if (pl->n_oc > 1 || nb == 1) {
+            const size_t stage = static_cast<size_t>(S::XCHUNK_BYTES) + S::WSTAGE_BYTES;
+            const size_t stages = max_smem > fixed ? std::min<size_t>(max_stages, (max_smem - fixed) / stage) : 0;
+            if (stages >= static_cast<size_t>(nb == 2 && !ybufs_env ? 3 : 1)) {
+                pl->path = kPathStreamed;
+                pl->rows = eqlin::kMmaM;
                 pl->stages = static_cast<int>(stages);
-                pl->w_region_bytes = static_cast<uint32_t>(region);
-                pl->w_img_bytes = static_cast<uint32_t>(img);
-                pl->img_alloc_bytes = img;
-                pl->smem_bytes = fixed + region + stages * S::XCHUNK_BYTES;
+                pl->w_region_bytes = 0;
+                pl->w_img_bytes = 0;
+                pl->img_alloc_bytes = static_cast<size_t>(pl->n_oc) * pl->nK * S::WSTAGE_BYTES;
+                pl->smem_bytes = fixed + stages * stage;
                 return EQLIN_OK;
             }
         }
     }
-    // weights streamed chunk by chunk next to each x chunk
-    const size_t stage = static_cast<size_t>(S::XCHUNK_BYTES) + S::WSTAGE_BYTES;
-    const size_t stages = max_smem > fixed ? std::min<size_t>(kMaxStages, (max_smem - fixed) / stage) : 0;
-    if (stages < 1) return fail(EQLIN_ERR_UNSUPPORTED, "shape does not fit in shared memory");
-    pl->path = kPathStreamed;
-    pl->rows = eqlin::kMmaM;
-    pl->stages = static_cast<int>(stages);
-    pl->w_region_bytes = 0;
-    pl->w_img_bytes = 0;
-    pl->img_alloc_bytes = static_cast<size_t>(pl->n_oc) * pl->nK * S::WSTAGE_BYTES;
-    pl->smem_bytes = fixed + stages * stage;
-    return EQLIN_OK;
+    return fail(EQLIN_ERR_UNSUPPORTED, "shape does not fit in shared memory");
 }
 
 template <int G>
 int plan_tm_g(int64_t Cout, int64_t Cin, size_t max_smem, Plan* pl) {
     using C = eqlin::tm::Cfg<G>;
+    const int kMaxStages = std::min(::kMaxStages, env_int("EQLIN_MAX_STAGES", ::kMaxStages));
     const int64_t no = std::min<int64_t>((Cout + 31) / 32 * 32, C::NMAX);  // MMA N, multiple of 32
     pl->rows = static_cast<int>(no);
     pl->nK = static_cast<int>((Cin + eqlin::kChunkK16 - 1) / eqlin::kChunkK16);
@@ -232,15 +256,43 @@ using TcLaunch = void (*)(unsigned grid, size_t smem, cudaStream_t st, const CUt
 using TmLaunch = void (*)(unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& mx,
                           const CUtensorMap& my, const TmParams& p);
 
+// The fused kernels are launched with programmatic stream serialization (PDL): a
+// forward's CTAs may start while the previous kernel of the stream drains, and wait in
+// griddepcontrol.wait before touching global memory.  Grids never exceed one CTA per
+// SM, so a waiting dependent cannot starve its predecessor.  EQLIN_PDL=0 disables it.
+bool use_pdl() {
+    static const bool on = [] {
+        const char* e = std::getenv("EQLIN_PDL");
+        return !(e && e[0] == '0');
+    }();
+    return on;
+}
+
+template <class Kernel, class Params>
+void launch_fused(Kernel k, unsigned grid, unsigned threads, size_t smem, cudaStream_t st, const CUtensorMap& mx,
+                  const CUtensorMap& my, const Params& p) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = use_pdl() ? 1 : 0;
+    cudaLaunchKernelEx(&cfg, k, mx, my, p);
+}
+
 template <int G, bool STREAM, int NACC>
 void tc_launch(unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& mx, const CUtensorMap& my,
                const TcParams& p) {
-    eqlin::eqlin_fwd_tc_kernel<G, STREAM, NACC><<<grid, eqlin::tc::kThreads, smem, st>>>(mx, my, p);
+    launch_fused(eqlin::eqlin_fwd_tc_kernel<G, STREAM, NACC>, grid, eqlin::tc::kThreads, smem, st, mx, my, p);
 }
 template <int G, bool STREAM>
 void tm_launch(unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& mx, const CUtensorMap& my,
                const TmParams& p) {
-    eqlin::eqlin_fwd_tm_kernel<G, STREAM><<<grid, eqlin::tm::Cfg<G>::kThreads, smem, st>>>(mx, my, p);
+    launch_fused(eqlin::eqlin_fwd_tm_kernel<G, STREAM>, grid, eqlin::tm::Cfg<G>::kThreads, smem, st, mx, my, p);
 }
 
 struct TcEntry {
@@ -384,7 +436,7 @@ int launch_forward(const Plan& pl, int64_t Cout, int64_t Cin, int64_t G, int sm_
             ybox[1] = eqlin::tm::kM;
             yswz = CU_TENSOR_MAP_SWIZZLE_64B;
         } else {
-            ybox[0] = eqlin::tc::kYBoxCols;
+            ybox[0] = static_cast<cuuint32_t>(std::min<int64_t>(32 * G, eqlin::tc::kYBoxCols2));
             ybox[1] = static_cast<cuuint32_t>(pl.TG);
             yswz = CU_TENSOR_MAP_SWIZZLE_NONE;
         }
@@ -428,7 +480,7 @@ int launch_forward(const Plan& pl, int64_t Cout, int64_t Cin, int64_t G, int sm_
             p.stages = pl.stages;
             p.w_region_bytes = pl.w_region_bytes;
             p.ystage_bytes = pl.ystage_bytes;
-            p.ycols_pad = pl.ycols_pad;
+            p.ybufs = pl.ybufs;
             p.w_img_bytes = pl.w_img_bytes;
             p.timeout_ns = timeout_ns;
             const TcEntry entry = tc_entry_for(iG, pl.streamed(), pl.nacc);

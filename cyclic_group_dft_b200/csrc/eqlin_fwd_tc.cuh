@@ -23,12 +23,11 @@
 //               one tile overlap the epilogue of the previous one.
 //   warps 0-7   epilogue: tcgen05.ld of all G planes of a token group, inverse real DFT
 //               (1/G and 2/G are folded into W^), + bias, round to bf16, write the
-//               group's y rows [TG tokens x Cout*G] into a shared-memory staging tile
-//               (a warp writes 32 consecutive o -> one contiguous 32*G*2-byte run), and
-//               one thread per half stores the tile with TMA (rows past N and columns
-//               past Cout*G are clipped by the tensor map).  Warps w and w+4 share TMEM
-//               lane quarter w and split the tile's tokens; each half double-buffers
-//               its staging tile so the TMA store of one group overlaps the next.
+//               group's y block [TG tokens x 32*G columns] into the warp's own staging
+//               tile (a warp writes 32 consecutive o -> one contiguous 32*G*2-byte run
+//               per token) and lane 0 stores it with TMA (rows past N and columns past
+//               Cout*G are clipped by the tensor map).  Warps w and w+4 share TMEM lane
+//               quarter w and split the tile's tokens.
 // All waits are bounded (globaltimer); on expiry the kernel records EQLIN_ERR_TIMEOUT
 // in the status word, every role leaves its loop, in-flight copies and MMAs are
 // drained with bounded waits, and TMEM is freed before exit.
@@ -56,8 +55,8 @@ struct TcParams {
     int n_work;             // n_tiles * n_oc
     int stages;             // smem ring depth
     uint32_t w_region_bytes;  // smem reserved for resident weights (0 when streamed)
-    uint32_t ystage_bytes;    // one y staging buffer (TG rows x ycols_pad bf16)
-    int ycols_pad;            // staged y columns per group, multiple of kYBoxCols
+    uint32_t ystage_bytes;    // y staging per epilogue warp (ybufs buffers of TG x 32*G bf16)
+    int ybufs;                // 1 or 2 staging buffers per epilogue warp
     uint32_t w_img_bytes;     // bytes of the resident image to copy
     unsigned long long timeout_ns;
 };
@@ -72,8 +71,7 @@ constexpr int kWarpProducer = 12;
 constexpr int kWarpMma = 13;
 constexpr int kBarDft = 1;   // named barrier ids (0 is __syncthreads)
 constexpr int kBarEpi = 2;
-constexpr int kBarEpiHalf0 = 3;  // 3 and 4: one per epilogue half (128 threads)
-constexpr int kYBoxCols = 128;   // y TMA store box: 128 bf16 columns (256 B) x TG rows
+constexpr int kYBoxCols2 = 256;  // widest y TMA store box (bf16 columns)
 
 // NACC accumulator buffers of G*BN TMEM columns each share the 512 columns: with two,
 // the MMAs of one tile overlap the epilogue of the previous one; with one, each MMA
@@ -198,43 +196,43 @@ __device__ __forceinline__ void dft_chunk(uint8_t* xs, int dft_tid) {
 // ------------------------------------------------------------ epilogue role
 // Warp (q, half): TMEM lane quarter q (output rows 32q..32q+31 of the chunk), tokens
 // [half*BN/2, (half+1)*BN/2) of the tile held in accumulator `acc` (column base).
-// `active`: this warp's quarter holds valid output rows (inactive warps still take part
-// in the half's barriers).  `ystage`: this half's two staging buffers; `ybuf` alternates.
-// `leader`: the one thread of the half that issues and tracks the TMA stores.
+// The warp stages each group of TG tokens x its 32 output channels (32*G columns,
+// 4 KB) in its own buffer and lane 0 stores it with TMA, so the epilogue warps never
+// wait for one another.  `wstage`: this warp's p.ybufs buffers; `ybuf` alternates.
 template <int G, int NACC>
 __device__ __forceinline__ void epilogue_tile(const TcParams& p, const CUtensorMap* tmap_y, uint32_t acc,
-                                              int q, int half, int lane, long long n0, int oc, bool active,
-                                              uint8_t* ystage, int& ybuf, bool leader) {
+                                              int q, int half, int lane, long long n0, int oc, uint8_t* wstage,
+                                              int& ybuf) {
     using S = Shape<G, NACC>;
     constexpr int TG = S::TG;
+    constexpr int WCOLS = 32 * G;                           // y columns of the warp's 32 outputs
+    constexpr int YBC = WCOLS < kYBoxCols2 ? WCOLS : kYBoxCols2;  // TMA box columns
+    constexpr int NYB = WCOLS / YBC;
+    constexpr int BOX_BYTES = TG * YBC * 2;
     const int o_local = q * 32 + lane;
     const int o = oc * kMmaM + o_local;
     const bool valid_o = o < p.Cout;
     const float b = (p.bias != nullptr && valid_o) ? p.bias[o] : 0.0f;
     const uint32_t lane_addr = acc + (static_cast<uint32_t>(q * 32) << 16);
     const int t0 = half * (S::BN / 2);
-    const uint32_t bar_half = kBarEpiHalf0 + half;
-    // column of this lane's first output inside the staged rows, and its box / offset
-    const int col = o_local * G;
-    const int box = col / kYBoxCols, col_in = col % kYBoxCols;
-    const int valid_rows = min(kMmaM, p.Cout - oc * kMmaM);
-    const int n_boxes = (valid_rows * G + kYBoxCols - 1) / kYBoxCols;
+    const int col = lane * G;                               // first staged column of this lane
+    uint8_t* lane_off0 = wstage + (col / YBC) * BOX_BYTES + (col % YBC) * 2;
 #pragma unroll 1
     for (int j = 0; j < S::BN / 2 / TG; ++j) {
         uint32_t r[G][TG];
-        if (active) {
 #pragma unroll
-            for (int pl = 0; pl < G; ++pl) ptx::tmem_ld_32x32b<TG>(lane_addr + pl * S::BN + t0 + j * TG, r[pl]);
-            ptx::tmem_wait_ld();
+        for (int pl = 0; pl < G; ++pl) ptx::tmem_ld_32x32b<TG>(lane_addr + pl * S::BN + t0 + j * TG, r[pl]);
+        ptx::tmem_wait_ld();
 #pragma unroll
-            for (int pl = 0; pl < G; ++pl) ptx::tmem_regs_ready<TG>(r[pl]);
+        for (int pl = 0; pl < G; ++pl) ptx::tmem_regs_ready<TG>(r[pl]);
+        // the buffer about to be written was stored p.ybufs groups ago: wait until read
+        if (lane == 0) {
+            if (p.ybufs == 2) ptx::bulk_wait_group_read<1>();
+            else ptx::bulk_wait_group_read<0>();
         }
-        // the buffer about to be written was last stored two groups ago: wait until the
-        // TMA engine has read it, then release the half
-        if (leader) ptx::bulk_wait_group_read<1>();
-        ptx::named_bar_sync(bar_half, 128);
-        uint8_t* buf = ystage + static_cast<size_t>(ybuf) * p.ystage_bytes;
-        if (active && valid_o) {
+        __syncwarp();
+        uint8_t* lane_off = lane_off0 + static_cast<size_t>(ybuf) * (NYB * BOX_BYTES);
+        if (valid_o) {
 #pragma unroll
             for (int t = 0; t < TG; ++t) {
                 float z[G], yv[G];
@@ -242,23 +240,16 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, const CUtensorM
                 for (int pl = 0; pl < G; ++pl) z[pl] = __uint_as_float(r[pl][t]);
                 z[0] += b;  // the DC term appears with weight 1 in every output
                 RealIdft<G>::run(z, yv);
-                if constexpr (G <= 4) {
-                    // the lane's 2G bytes sit inside one box (128 % G == 0)
-                    uint8_t* dst = buf + box * (TG * kYBoxCols * 2) + t * (kYBoxCols * 2) + col_in * 2;
-                    if constexpr (G == 2) {
-                        *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(yv[0], yv[1]);
-                    } else {
-                        *reinterpret_cast<uint2*>(dst) =
-                            make_uint2(pack_bf16x2(yv[0], yv[1]), pack_bf16x2(yv[2], yv[3]));
-                    }
+                uint8_t* dst = lane_off + t * (YBC * 2);
+                if constexpr (G == 2) {
+                    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(yv[0], yv[1]);
+                } else if constexpr (G == 4) {
+                    *reinterpret_cast<uint2*>(dst) =
+                        make_uint2(pack_bf16x2(yv[0], yv[1]), pack_bf16x2(yv[2], yv[3]));
                 } else {
-                    // G/8 pieces of 16 B (8 columns); a piece never straddles a box
 #pragma unroll
                     for (int c = 0; c < G / 8; ++c) {
-                        const int cc = col + 8 * c;
-                        uint8_t* dst = buf + (cc / kYBoxCols) * (TG * kYBoxCols * 2) + t * (kYBoxCols * 2) +
-                                       (cc % kYBoxCols) * 2;
-                        *reinterpret_cast<uint4*>(dst) = make_uint4(
+                        *reinterpret_cast<uint4*>(dst + 16 * c) = make_uint4(
                             pack_bf16x2(yv[8 * c + 0], yv[8 * c + 1]), pack_bf16x2(yv[8 * c + 2], yv[8 * c + 3]),
                             pack_bf16x2(yv[8 * c + 4], yv[8 * c + 5]), pack_bf16x2(yv[8 * c + 6], yv[8 * c + 7]));
                     }
@@ -266,21 +257,23 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, const CUtensorM
             }
         }
         ptx::fence_proxy_async_smem();
-        ptx::named_bar_sync(bar_half, 128);
-        if (leader) {
+        __syncwarp();
+        if (lane == 0) {
             // every store starts inside the tensor: rows past N and columns past Cout*G
-            // of a started box are clipped by the tensor map, boxes that would start
-            // outside are not issued
+            // of a started box are clipped, boxes that would start outside are skipped
             const long long row = n0 + t0 + j * TG;
             if (row < p.N) {
-                const uint32_t src = ptx::smem_u32(buf);
-                for (int bx = 0; bx < n_boxes; ++bx)
-                    ptx::tma_store_2d(tmap_y, src + bx * (TG * kYBoxCols * 2), oc * kMmaM * G + bx * kYBoxCols,
-                                      static_cast<int>(row));
+                const uint32_t src = ptx::smem_u32(wstage + static_cast<size_t>(ybuf) * (NYB * BOX_BYTES));
+#pragma unroll
+                for (int bx = 0; bx < NYB; ++bx) {
+                    const int o_first = oc * kMmaM + q * 32 + bx * (YBC / G);
+                    if (o_first < p.Cout)
+                        ptx::tma_store_2d(tmap_y, src + bx * BOX_BYTES, o_first * G, static_cast<int>(row));
+                }
             }
             ptx::bulk_commit_group();
         }
-        ybuf ^= 1;
+        if (p.ybufs == 2) ybuf ^= 1;
     }
 }
 
@@ -298,8 +291,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     constexpr uint32_t STAGE_BYTES = S::XCHUNK_BYTES + (STREAM_W ? S::WSTAGE_BYTES : 0);
     constexpr uint32_t STAGE_TX = STAGE_BYTES;   // every byte of a stage arrives by copy
     const int NS = p.stages;
-    uint8_t* ystage0 = smem + p.w_region_bytes;                 // 4 y staging buffers (2 per half)
-    uint8_t* stage0 = ystage0 + 4 * static_cast<size_t>(p.ystage_bytes);
+    uint8_t* ystage0 = smem + p.w_region_bytes;                 // y staging, one area per epilogue warp
+    uint8_t* stage0 = ystage0 + tc::kEpiWarps * static_cast<size_t>(p.ystage_bytes);
     uint64_t* bars = reinterpret_cast<uint64_t*>(stage0 + static_cast<size_t>(NS) * STAGE_BYTES);
     tc::Ctl* ctl = reinterpret_cast<tc::Ctl*>(bars + 3 * NS + 2 * NACC + 2);
 
@@ -342,6 +335,11 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem_base = ctl->tmem_base;
+    // The next forward of the stream may begin launching (its CTAs take an SM as one of
+    // ours exits); every global access below waits until the previous kernel of the
+    // stream has completed, so y / x aliasing between consecutive calls stays safe.
+    ptx::grid_launch_dependents();
+    ptx::grid_dependency_wait();
 
     if (warp == tc::kWarpProducer) {
         // ------------------------------------------------------------ producer
@@ -508,8 +506,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     } else {
         // ------------------------------------------------------------ epilogue warps
         const int half = warp >> 2;
-        const bool leader = (warp & 3) == 0 && lane == 0;
-        uint8_t* ystage = ystage0 + static_cast<size_t>(2 * half) * p.ystage_bytes;
+        uint8_t* wstage = ystage0 + static_cast<size_t>(warp) * p.ystage_bytes;
         int ybuf = 0;
         int it = 0;
         for (int wk = blockIdx.x; wk < p.n_work; wk += gridDim.x, ++it) {
@@ -519,15 +516,17 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
             if (!ptx::named_bar_and(tc::kBarEpi, tc::kEpiThreads, got)) break;
             ptx::tc_fence_after();
             const int tile = wk / p.n_oc, oc = wk % p.n_oc;
-            // warps whose lane quarter holds no valid output row skip the math
-            const bool active = oc * kMmaM + (warp & 3) * 32 < p.Cout;
-            tc::epilogue_tile<G, NACC>(p, &tmap_y, tmem_base + static_cast<uint32_t>(abuf * S::ACC_COLS), warp & 3,
-                                 half, lane, static_cast<long long>(tile) * S::BN, oc, active, ystage, ybuf, leader);
+            // warps whose lane quarter holds no valid output row skip the work
+            if (oc * kMmaM + (warp & 3) * 32 < p.Cout) {
+                tc::epilogue_tile<G, NACC>(p, &tmap_y, tmem_base + static_cast<uint32_t>(abuf * S::ACC_COLS),
+                                           warp & 3, half, lane, static_cast<long long>(tile) * S::BN, oc, wstage,
+                                           ybuf);
+            }
             ptx::tc_fence_before();
             ptx::mbar_arrive(bar_acc_empty(abuf));
         }
         // the y stores must be complete (not only read) before the CTA exits
-        if (leader) ptx::bulk_wait_group<0>();
+        if (lane == 0) ptx::bulk_wait_group<0>();
     }
 
     ptx::tc_fence_before();

@@ -256,6 +256,11 @@ __global__ void __launch_bounds__(tm::Cfg<G>::kThreads, 1)
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem_base = ctl->tmem_base;
+    // The next forward of the stream may begin launching (its CTAs take an SM as one of
+    // ours exits); every global access below waits until the previous kernel of the
+    // stream has completed, so y / x aliasing between consecutive calls stays safe.
+    ptx::grid_launch_dependents();
+    ptx::grid_dependency_wait();
 
     if (warp == C::kWarpProducer) {
         // ------------------------------------------------------------ producer

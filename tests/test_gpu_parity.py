@@ -100,6 +100,35 @@ def test_shapes_every_group_order(Cout, Cin, G, io):
     h.close()
 
 
+@pytest.mark.parametrize("kernel", ["tn", "tm"])
+@pytest.mark.parametrize("Cout,Cin,G", SHAPES)
+def test_shapes_both_fused_kernels(Cout, Cin, G, kernel, monkeypatch):
+    """Each fused bf16 kernel (tokens on N, tokens on M) is correct for every
+    shape, whichever one the planner would pick by default."""
+    monkeypatch.setenv("EQLIN_KERNEL", kernel)
+    gen = torch.Generator().manual_seed(Cout * 1000 + Cin * 10 + G + 5)
+    N = 517
+    x = torch.randn(N, Cin, G, generator=gen).to(torch.bfloat16)
+    w = (torch.randn(Cout, Cin, G, generator=gen) / np.sqrt(Cin * G)).to(torch.bfloat16)
+    bias = (torch.randn(Cout, generator=gen) * 0.3).to(torch.bfloat16)
+    y, h = _run(x, w, bias, torch.bfloat16)
+    assert f"tokens_on_{kernel[1]}" in h.path, h.path
+    _assert_parity(torch.bfloat16, y, _ref(x, w, bias), f"Cout={Cout} Cin={Cin} G={G} {kernel}")
+    h.close()
+
+
+@pytest.mark.parametrize("kernel", ["tn", "tm"])
+@pytest.mark.parametrize("name", ["p4_c96_bf16", "p8_c64_bf16", "p4_mlp_bf16", "c16_c32_bf16"])
+def test_workloads_both_fused_kernels(name, kernel, monkeypatch):
+    monkeypatch.setenv("EQLIN_KERNEL", kernel)
+    wl = workloads.WORKLOADS[name]
+    x, w, bias = workloads.make_inputs(wl, seed=11, N=2 * 148 * 128 + 77)
+    y, h = _run(x, w, bias, wl.torch_dtype)
+    idx = workloads.sample_tokens(x.shape[0], 512, seed=13)
+    _assert_parity(wl.torch_dtype, y[idx], _ref(x[idx], w, bias), f"{name} {kernel} path={h.path}")
+    h.close()
+
+
 @pytest.mark.parametrize("G", [2, 4, 8, 16])
 def test_fp32_weights_bf16_io(G):
     gen = torch.Generator().manual_seed(G)
