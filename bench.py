@@ -64,6 +64,16 @@ def algorithmic_bytes(wl: workloads.Workload, N: int) -> int:
     return N * wl.Cin * wl.G * e + N * wl.Cout * wl.G * e + wl.G * wl.Cin * wl.Cout * e + bias
 
 
+def backward_bytes(wl: workloads.Workload, N: int) -> dict:
+    """Algorithmic bytes of the two backward calls.  Input gradient: read dy once,
+    write dx once, read its weights once.  Weight gradient: read x and dy once,
+    write dw and dbias once (fp32)."""
+    e = wl.elem_bytes
+    act = N * (wl.Cin + wl.Cout) * wl.G * e
+    return {"dx": act + wl.G * wl.Cin * wl.Cout * e,
+            "dw": act + 4 * (wl.G * wl.Cin * wl.Cout + wl.Cout)}
+
+
 def fourier_flops(wl: workloads.Workload, N: int) -> int:
     """Per-frequency real products: 2 real + 4 per complex frequency = 2G-2 blocks."""
     return 2 * N * wl.Cin * wl.Cout * (2 * wl.G - 2)
@@ -267,6 +277,8 @@ def main() -> None:
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip the extra measurement of the backward calls (input and weight gradients)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override the workload's token count (profiling a smaller case)")
     args = ap.parse_args()
@@ -291,7 +303,8 @@ def main() -> None:
     torch.cuda.set_device(dev)
 
     x_cpu, w, bias = workloads.make_inputs(wl)
-    h = eq.prepare(w.to(dev), None if bias is None else bias.to(dev), io_dtype=wl.torch_dtype)
+    h = eq.prepare(w.to(dev), None if bias is None else bias.to(dev), io_dtype=wl.torch_dtype,
+                   backward=not args.no_backward)
     N = wl.N
     set_bytes = N * (wl.Cin + wl.Cout) * wl.G * wl.elem_bytes
     n_sets = max(2, math.ceil(2 * L2_BYTES / set_bytes))
@@ -359,6 +372,44 @@ def main() -> None:
                "d2h_bytes_per_step": y_pin.numel() * y_pin.element_size(),
                "api": "Handle.forward_host (pinned host x -> device -> eqlin_forward -> pinned host y)"}
 
+    # ----------------------------------------------------------- backward calls
+    # Measured after the forward's timed region, on the same rotating buffer sets
+    # (the forward outputs stand in for dy): us per call from CUDA events around
+    # Kb back-to-back calls, against the same roofline model as the forward.
+    bwd = None
+    if not args.no_backward:
+        Kb = max(10, min(K, 200))
+        dxs = [torch.empty(N, wl.Cin, wl.G, dtype=wl.torch_dtype, device=dev) for _ in range(n_sets)]
+        dw_t = torch.empty(wl.Cout, wl.Cin, wl.G, dtype=torch.float32, device=dev)
+        db_t = torch.empty(wl.Cout, dtype=torch.float32, device=dev)
+        ws_t = torch.empty(max(16, eq.eqlin_backward_dw_workspace_size(h, N)), dtype=torch.uint8, device=dev)
+        calls = {
+            "dx": lambda i: h.backward_dx(ys[i % n_sets], out=dxs[i % n_sets], stream=stream),
+            "dw": lambda i: eq.eqlin_backward_dw(h, xs[i % n_sets], ys[i % n_sets], stream=stream,
+                                                 dw=dw_t, dbias=db_t, workspace=ws_t),
+        }
+        bwd = {}
+        for key, fn in calls.items():
+            for i in range(max(3, args.warmup)):
+                fn(i)
+            barrier()
+            torch.cuda.synchronize(dev)
+            b0 = torch.cuda.Event(enable_timing=True)
+            b1 = torch.cuda.Event(enable_timing=True)
+            b0.record(stream)
+            for i in range(Kb):
+                fn(i)
+            b1.record(stream)
+            torch.cuda.synchronize(dev)
+            barrier()
+            bwd[key] = {"us_per_call": 1e3 * reduce_max(b0.elapsed_time(b1), dev) / Kb, "calls": Kb}
+        bwd["device_status"] = h.device_status()
+        bwd["kernels"] = {"dx": "fused forward kernel on the adjoint operator (1 launch)",
+                          "dw": "tcgen05 contraction over tokens + deterministic reduction / inverse DFT "
+                                "(2 launches)" if wl.io_dtype == "bf16" else
+                                "float64 CUDA-core kernel (clear + kernel + convert)"}
+        del dxs
+
     # ----------------------------------------------------------- CPU baseline
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -395,6 +446,16 @@ def main() -> None:
     roof["tensor_tflops"] = tflops
     roof["tensor_frac"] = tflops / peaks["bf16_tflops"]
 
+    if bwd is not None:
+        bb = backward_bytes(wl, N)
+        for key in ("dx", "dw"):
+            t = bwd[key]["us_per_call"] * 1e-6
+            t_h = bb[key] / (peaks["hbm_gbs"] * 1e9)
+            t_roof = max(t_h, t_tc)
+            bwd[key].update({"bytes": bb[key], "roofline_time_us": 1e6 * t_roof,
+                             "bound": "hbm" if t_h >= t_tc else "tensor",
+                             "frac_of_roofline_time": t_roof / t, "tokens_per_s": N / t})
+
     emit({
         "metric": METRIC,
         "value": value,
@@ -423,6 +484,7 @@ def main() -> None:
         "gpu_launches": K,
         "device_status": status,
         "cpu_baseline": cpu,
+        "backward": bwd,
     })
     h.close()
 

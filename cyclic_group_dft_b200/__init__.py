@@ -2,13 +2,18 @@
 
 y[n,o,g] = bias[o] + sum_{i,h} w[o,i,(g-h) mod G] x[n,i,h], computed as a real
 DFT over the group axis, per-frequency contractions on tcgen05 tensor cores
-(half spectrum) and an inverse DFT, fused in one kernel.
+(half spectrum) and an inverse DFT, fused in one kernel; and its backward
+(input, weight and bias gradients) the same way.
 
 Usage::
 
     import cyclic_group_dft_b200 as eq
     h = eq.prepare(w, bias)          # w [Cout, Cin, G] CUDA tensor (bf16 or fp32)
     y = h.forward(x)                 # x [N, Cin, G] -> y [N, Cout, G]
+
+    hb = eq.prepare(w, bias, backward=True)
+    dx = hb.backward_dx(dy)          # dy [N, Cout, G] -> dx [N, Cin, G]
+    dw, dbias = hb.backward_dw(x, dy)  # fp32 [Cout, Cin, G], [Cout]
 
 The functions with the C ABI's names (eqlin_prepare_weights, eqlin_forward,
 eqlin_destroy, ...) are the same calls with explicit arguments.
@@ -24,10 +29,14 @@ from ._capi import (  # noqa: F401
     EQLIN_ERR_UNSUPPORTED,
     EQLIN_F32,
     EQLIN_OK,
+    EQLIN_PREPARE_BACKWARD,
     LIB_PATH,
     PATH_NAMES,
     EqlinError,
     Handle,
+    eqlin_backward_dw,
+    eqlin_backward_dw_workspace_size,
+    eqlin_backward_dx,
     eqlin_check_shape,
     eqlin_copy_freq_weights,
     eqlin_destroy,

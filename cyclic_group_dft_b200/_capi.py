@@ -1,7 +1,7 @@
 """ctypes binding of libeqlin.so (C ABI in include/eqlin.h).
 
-Argument marshalling only: every step of the forward runs in the library's
-kernels.  torch supplies device memory and streams.  Importing this module
+Argument marshalling only: every step of the forward and backward runs in the
+library's kernels.  torch supplies device memory and streams.  Importing this module
 fails loudly if the library has not been built -- there is no fallback.
 """
 from __future__ import annotations
@@ -26,6 +26,8 @@ EQLIN_ERR_MISALIGNED = -3
 EQLIN_ERR_CUDA = -4
 EQLIN_ERR_OOM = -5
 EQLIN_ERR_TIMEOUT = -6
+
+EQLIN_PREPARE_BACKWARD = 1
 
 ATTRS = {
     "G": 0, "Cin": 1, "Cout": 2, "io_dtype": 3, "path": 4, "tokens_per_tile": 5,
@@ -53,6 +55,11 @@ _lib.eqlin_get_attr.argtypes = [_vp, _int, ctypes.POINTER(_i64)]
 _lib.eqlin_copy_freq_weights.argtypes = [_vp, ctypes.POINTER(ctypes.c_float), _i64]
 _lib.eqlin_check_shape.argtypes = [_i64, _i64, _i64, _int, _int]
 _lib.eqlin_forward_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _int, _vp]
+_lib.eqlin_prepare_weights_ex.argtypes = [_vp, _vp, _i64, _i64, _i64, _int, _int, ctypes.c_uint, _vp,
+                                          ctypes.POINTER(_vp)]
+_lib.eqlin_backward_dx.argtypes = [_vp, _vp, _vp, _i64, _vp]
+_lib.eqlin_backward_dw_workspace_size.argtypes = [_vp, _i64, ctypes.POINTER(ctypes.c_size_t)]
+_lib.eqlin_backward_dw.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _vp, ctypes.c_size_t, _vp]
 _lib.eqlin_status_string.argtypes = [_int]
 _lib.eqlin_status_string.restype = ctypes.c_char_p
 _lib.eqlin_last_error.argtypes = []
@@ -60,7 +67,8 @@ _lib.eqlin_last_error.restype = ctypes.c_char_p
 _lib.eqlin_version.argtypes = []
 for _f in ("eqlin_prepare_weights", "eqlin_forward", "eqlin_destroy", "eqlin_device_status",
            "eqlin_get_attr", "eqlin_copy_freq_weights", "eqlin_check_shape", "eqlin_version",
-           "eqlin_forward_noalloc"):
+           "eqlin_forward_noalloc", "eqlin_prepare_weights_ex", "eqlin_backward_dx",
+           "eqlin_backward_dw_workspace_size", "eqlin_backward_dw"):
     getattr(_lib, _f).restype = _int
 
 
@@ -150,6 +158,15 @@ class Handle:
     def forward(self, x: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
         return eqlin_forward(self, x, out, stream)
 
+    def backward_dx(self, dy: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        """dx = dL/dx from dy (the handle must be prepared with backward=True)."""
+        return eqlin_backward_dx(self, dy, out, stream)
+
+    def backward_dw(self, x: torch.Tensor, dy: torch.Tensor, with_bias: bool = True,
+                    stream=None) -> tuple[torch.Tensor, torch.Tensor | None]:
+        """(dw [Cout, Cin, G], dbias [Cout] or None) = dL/dw, dL/dbias, both fp32."""
+        return eqlin_backward_dw(self, x, dy, with_bias, stream)
+
     def forward_host(self, x_host: torch.Tensor, out_host: torch.Tensor | None = None,
                      stream=None) -> torch.Tensor:
         """Forward from and to host memory: copy x in, run, copy y back (synchronous)."""
@@ -193,8 +210,10 @@ class Handle:
 
 
 def eqlin_prepare_weights(w: torch.Tensor, bias: torch.Tensor | None = None,
-                          io_dtype: torch.dtype | None = None, stream=None) -> Handle:
-    """Transform w [Cout, Cin, G] (and bias [Cout]) to the frequency domain on w's device."""
+                          io_dtype: torch.dtype | None = None, stream=None, backward: bool = False) -> Handle:
+    """Transform w [Cout, Cin, G] (and bias [Cout]) to the frequency domain on w's device.
+    backward=True also prepares the input-gradient weights (eqlin_prepare_weights_ex with
+    EQLIN_PREPARE_BACKWARD), for Handle.backward_dx."""
     if w.dim() != 3:
         raise ValueError("w must be [Cout, Cin, G]")
     if w.device.type != "cuda":
@@ -210,10 +229,11 @@ def eqlin_prepare_weights(w: torch.Tensor, bias: torch.Tensor | None = None,
     io = _TORCH_TO_EQLIN[w.dtype if io_dtype is None else io_dtype]
     out = ctypes.c_void_p()
     with torch.cuda.device(w.device):
-        st = _lib.eqlin_prepare_weights(
+        st = _lib.eqlin_prepare_weights_ex(
             w.data_ptr(), None if bias is None else bias.data_ptr(), Cout, Cin, G,
-            _TORCH_TO_EQLIN[w.dtype], io, _stream_ptr(stream), ctypes.byref(out))
-    _check(st, "eqlin_prepare_weights")
+            _TORCH_TO_EQLIN[w.dtype], io, EQLIN_PREPARE_BACKWARD if backward else 0,
+            _stream_ptr(stream), ctypes.byref(out))
+    _check(st, "eqlin_prepare_weights_ex")
     return Handle(out.value, w.device)
 
 
@@ -235,6 +255,64 @@ def eqlin_forward(h: Handle, x: torch.Tensor, y: torch.Tensor | None = None, str
         _check(_lib.eqlin_forward(h.ptr, x.data_ptr(), y.data_ptr(), N, _stream_ptr(stream)),
                "eqlin_forward")
     return y
+
+
+def _check_rows(t: torch.Tensor, name: str, C: int, h: Handle) -> None:
+    if t.dim() != 3 or t.shape[1] != C or t.shape[2] != h.G:
+        raise ValueError(f"{name} must be [N, {C}, {h.G}], got {tuple(t.shape)}")
+    if t.device != h.device or t.dtype != h.io_dtype:
+        raise ValueError(f"{name} must be {h.io_dtype} on {h.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def eqlin_backward_dx(h: Handle, dy: torch.Tensor, dx: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """dx [N, Cin, G] = dL/dx for the upstream gradient dy [N, Cout, G]."""
+    _check_rows(dy, "dy", h.Cout, h)
+    N = dy.shape[0]
+    if dx is None:
+        dx = torch.empty((N, h.Cin, h.G), dtype=h.io_dtype, device=h.device)
+    elif dx.shape != (N, h.Cin, h.G) or dx.dtype != h.io_dtype or dx.device != h.device \
+            or not dx.is_contiguous():
+        raise ValueError("dx has the wrong shape, dtype, device or layout")
+    with torch.cuda.device(h.device):
+        _check(_lib.eqlin_backward_dx(h.ptr, dy.data_ptr(), dx.data_ptr(), N, _stream_ptr(stream)),
+               "eqlin_backward_dx")
+    return dx
+
+
+def eqlin_backward_dw_workspace_size(h: Handle, N: int) -> int:
+    v = ctypes.c_size_t()
+    _check(_lib.eqlin_backward_dw_workspace_size(h.ptr, N, ctypes.byref(v)), "eqlin_backward_dw_workspace_size")
+    return int(v.value)
+
+
+def eqlin_backward_dw(h: Handle, x: torch.Tensor, dy: torch.Tensor, with_bias: bool = True,
+                      stream=None, dw: torch.Tensor | None = None, dbias: torch.Tensor | None = None,
+                      workspace: torch.Tensor | None = None) -> tuple[torch.Tensor, torch.Tensor | None]:
+    """(dw [Cout, Cin, G] fp32, dbias [Cout] fp32 or None) for the forward input x and
+    the upstream gradient dy.  The workspace (a uint8 CUDA tensor) is allocated by torch
+    when not given."""
+    _check_rows(x, "x", h.Cin, h)
+    _check_rows(dy, "dy", h.Cout, h)
+    N = x.shape[0]
+    if dy.shape[0] != N:
+        raise ValueError("x and dy must have the same number of tokens")
+    if dw is None:
+        dw = torch.empty((h.Cout, h.Cin, h.G), dtype=torch.float32, device=h.device)
+    elif dw.shape != (h.Cout, h.Cin, h.G) or dw.dtype != torch.float32 or not dw.is_contiguous():
+        raise ValueError("dw must be a contiguous fp32 [Cout, Cin, G] tensor")
+    if with_bias and dbias is None:
+        dbias = torch.empty((h.Cout,), dtype=torch.float32, device=h.device)
+    need = eqlin_backward_dw_workspace_size(h, N)
+    if workspace is None:
+        workspace = torch.empty((max(need, 16),), dtype=torch.uint8, device=h.device)
+    with torch.cuda.device(h.device):
+        _check(_lib.eqlin_backward_dw(h.ptr, x.data_ptr(), dy.data_ptr(), dw.data_ptr(),
+                                      None if dbias is None else dbias.data_ptr(), N,
+                                      workspace.data_ptr(), workspace.numel(), _stream_ptr(stream)),
+               "eqlin_backward_dw")
+    return dw, dbias
 
 
 def eqlin_destroy(h: Handle) -> None:

@@ -15,6 +15,7 @@
 #include <new>
 #include <string>
 
+#include "eqlin_bwd_dw.cuh"
 #include "eqlin_fwd_tc.cuh"
 #include "eqlin_fwd_tm.cuh"
 #include "eqlin_layout.h"
@@ -368,19 +369,21 @@ struct WeightBuffers {
     bool has_bias = false;
 };
 
+// Cout x Cin is the operator's shape.  adjoint: the operator is the layer's input
+// gradient (the layer's w is then [Cin, Cout, G] in these names, and bias is NULL).
 int launch_prep(const Plan& pl, int w_dtype, const void* w, const void* bias, int64_t Cout, int64_t Cin,
-                int64_t G, const WeightBuffers& b, cudaStream_t st) {
+                int64_t G, const WeightBuffers& b, cudaStream_t st, bool adjoint = false) {
     const int threads = 256;
     const unsigned blocks = static_cast<unsigned>((Cout * Cin + threads - 1) / threads);
     const int iCout = static_cast<int>(Cout), iCin = static_cast<int>(Cin), iG = static_cast<int>(G);
     if (w_dtype == EQLIN_F32) {
         eqlin::eqlin_prep_freq_kernel<float><<<blocks, threads, 0, st>>>(
             static_cast<const float*>(w), static_cast<const float*>(bias), iCout, iCin, iG, b.w_f32, b.bias_f32,
-            b.w_f64, b.bias_f64);
+            b.w_f64, b.bias_f64, adjoint);
     } else {
         eqlin::eqlin_prep_freq_kernel<__nv_bfloat16><<<blocks, threads, 0, st>>>(
             static_cast<const __nv_bfloat16*>(w), static_cast<const __nv_bfloat16*>(bias), iCout, iCin, iG,
-            b.w_f32, b.bias_f32, b.w_f64, b.bias_f64);
+            b.w_f32, b.bias_f32, b.w_f64, b.bias_f64, adjoint);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "weight transform launch");
@@ -493,6 +496,204 @@ int launch_forward(const Plan& pl, int64_t Cout, int64_t Cin, int64_t G, int sm_
     return EQLIN_OK;
 }
 
+// ------------------------------------------------------ weight gradient (dW)
+// Tiling of the weight-gradient kernel: a unit is an (MO-row, NI-column) tile of the
+// [Cout x Cin] gradient; the grid is units x token splits (see eqlin_bwd_dw.cuh).
+struct DwPlan {
+    int MO = 0, NI = 0, n_ot = 0, n_it = 0, max_splits = 0;
+    int cpb_dy = 0, cpb_x = 0;
+    uint32_t dy_bytes = 0, raw_bytes = 0, a_bytes = 0, b_bytes = 0, tmem_cols = 0;
+    size_t smem_bytes = 0, slab_floats = 0;
+    int units() const { return n_ot * n_it; }
+};
+
+uint32_t round_kb(size_t v) { return static_cast<uint32_t>((v + 1023) / 1024 * 1024); }
+int round16(int64_t v) { return static_cast<int>((v + 15) / 16 * 16); }
+
+// Channels per TMA box: the largest divisor d of C with d*G <= 256 elements and
+// 16-byte box rows (C is a multiple of 16, so d = 16 always qualifies).
+int box_channels(int C, int G) {
+    for (int d = C; d >= 1; --d)
+        if (C % d == 0 && d * G <= 256 && (d * G * 2) % 16 == 0) return d;
+    return 0;
+}
+
+size_t dw_smem(int MO, int NI, int G, DwPlan* out) {
+    const size_t raw = round_kb(static_cast<size_t>(eqlin::dw::kTok) * (MO + NI) * G * 2);
+    const size_t a = round_kb(static_cast<size_t>(G * MO + (eqlin::kMmaM - MO)) * eqlin::kPlaneRowBytes);
+    const size_t b = round_kb(static_cast<size_t>(G) * NI * eqlin::kPlaneRowBytes);
+    const size_t total = kSmemAlignSlack + eqlin::dw::kRawStages * raw + eqlin::dw::kSpecBufs * (a + b) +
+                         static_cast<size_t>(4 * MO) * 4 + 256;
+    if (out) {
+        out->dy_bytes = static_cast<uint32_t>(eqlin::dw::kTok) * MO * G * 2;
+        out->raw_bytes = static_cast<uint32_t>(raw);
+        out->a_bytes = static_cast<uint32_t>(a);
+        out->b_bytes = static_cast<uint32_t>(b);
+        out->smem_bytes = total;
+    }
+    return total;
+}
+
+// Pick the tile with the fewest units that fits shared memory (fewer units = fewer
+// re-reads of x and dy); ties go to the larger MO (less MMA padding), then larger NI.
+int plan_dw(int64_t Cout, int64_t Cin, int G, size_t max_smem, int sm_count, DwPlan* pl) {
+    const int mo_max = std::min(eqlin::kMmaM, round16(Cout));
+    const int ni_cap = std::min(256, (512 / G) / 16 * 16);
+    const int ni_max = std::min(ni_cap, round16(Cin));
+    long long best_units = -1;
+    int best_mo = 0, best_ni = 0;
+    for (int mo = mo_max; mo >= 16; mo -= 16) {
+        for (int ni = ni_max; ni >= 16; ni -= 16) {
+            if (dw_smem(mo, ni, G, nullptr) > max_smem) continue;
+            const long long units = ((Cout + mo - 1) / mo) * ((Cin + ni - 1) / ni);
+            if (best_units < 0 || units < best_units) {
+                best_units = units;
+                best_mo = mo;
+                best_ni = ni;
+            }
+        }
+    }
+    if (best_units < 0) return fail(EQLIN_ERR_UNSUPPORTED, "no weight-gradient tile fits shared memory");
+    pl->MO = best_mo;
+    pl->NI = best_ni;
+    pl->n_ot = static_cast<int>((Cout + best_mo - 1) / best_mo);
+    pl->n_it = static_cast<int>((Cin + best_ni - 1) / best_ni);
+    pl->max_splits = std::max(1, sm_count / pl->units());
+    pl->cpb_dy = box_channels(best_mo, G);
+    pl->cpb_x = box_channels(best_ni, G);
+    dw_smem(best_mo, best_ni, G, pl);
+    int cols = 32;
+    while (cols < G * best_ni) cols *= 2;
+    pl->tmem_cols = static_cast<uint32_t>(cols);
+    pl->slab_floats = static_cast<size_t>(G) * best_ni * best_mo;
+    return EQLIN_OK;
+}
+
+// Workspace of one weight-gradient call: per CTA a [G][NI][MO] slab plus [MO] bias sums
+// (bf16 path), or a float64 [Cout][Cin][G] + [Cout] accumulator (fp32 path).
+size_t dw_workspace_bytes(const DwPlan& pl, bool f32_path, int64_t Cout, int64_t Cin, int64_t G, int64_t N) {
+    if (f32_path) return static_cast<size_t>(Cout * Cin * G + Cout) * sizeof(double);
+    const long long n_chunks = (N + eqlin::dw::kTok - 1) / eqlin::dw::kTok;
+    const long long splits = std::max<long long>(1, std::min<long long>(pl.max_splits, n_chunks));
+    const size_t grid = static_cast<size_t>(pl.units()) * static_cast<size_t>(splits);
+    return grid * (pl.slab_floats + static_cast<size_t>(pl.MO)) * sizeof(float);
+}
+
+template <int G>
+void dw_launch(unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& mdy, const CUtensorMap& mx,
+               const eqlin::DwParams& p) {
+    launch_fused(eqlin::eqlin_dw_tc_kernel<G>, grid, eqlin::dw::kThreads, smem, st, mdy, mx, p);
+}
+
+void* dw_kernel_for(int G) {
+    switch (G) {
+        case 2: return reinterpret_cast<void*>(&eqlin::eqlin_dw_tc_kernel<2>);
+        case 4: return reinterpret_cast<void*>(&eqlin::eqlin_dw_tc_kernel<4>);
+        case 8: return reinterpret_cast<void*>(&eqlin::eqlin_dw_tc_kernel<8>);
+        case 16: return reinterpret_cast<void*>(&eqlin::eqlin_dw_tc_kernel<16>);
+        default: return nullptr;
+    }
+}
+
+int encode_rows_map(CUtensorMap* map, const void* base, int64_t cols, int64_t rows, int box_cols, int box_rows) {
+    auto encode = tensor_map_encoder();
+    if (!encode) return fail(EQLIN_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    cuuint32_t estr[2] = {1, 1};
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols * 2)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+    CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(EQLIN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+    return EQLIN_OK;
+}
+
+int launch_dw(const DwPlan& pl, bool f32_path, int64_t Cout, int64_t Cin, int64_t G, const void* x, const void* dy,
+              float* dw, float* dbias, int64_t N, void* ws, int* status, unsigned long long timeout_ns,
+              cudaStream_t st) {
+    const int iG = static_cast<int>(G), iCout = static_cast<int>(Cout), iCin = static_cast<int>(Cin);
+    cudaError_t e;
+    if (f32_path) {
+        double* acc = static_cast<double*>(ws);
+        const size_t n_w = static_cast<size_t>(Cout * Cin * G);
+        if ((e = cudaMemsetAsync(acc, 0, (n_w + Cout) * sizeof(double), st)) != cudaSuccess)
+            return cuda_fail(e, "weight-gradient accumulator clear");
+        const long long pairs = Cout * Cin;
+        const long long per = 512;
+        const unsigned slices = static_cast<unsigned>(std::min<long long>((N + per - 1) / per, 65535));
+        const long long tps = (N + slices - 1) / slices;
+        dim3 grid(static_cast<unsigned>((pairs + 255) / 256), slices);
+        const float* xf = static_cast<const float*>(x);
+        const float* dyf = static_cast<const float*>(dy);
+        switch (iG) {
+            case 2: eqlin::eqlin_dw_f64_kernel<2><<<grid, 256, 0, st>>>(xf, dyf, acc, N, iCin, iCout, tps); break;
+            case 4: eqlin::eqlin_dw_f64_kernel<4><<<grid, 256, 0, st>>>(xf, dyf, acc, N, iCin, iCout, tps); break;
+            case 8: eqlin::eqlin_dw_f64_kernel<8><<<grid, 256, 0, st>>>(xf, dyf, acc, N, iCin, iCout, tps); break;
+            default: eqlin::eqlin_dw_f64_kernel<16><<<grid, 256, 0, st>>>(xf, dyf, acc, N, iCin, iCout, tps); break;
+        }
+        if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "weight-gradient launch");
+        const size_t n_conv = std::max(n_w, static_cast<size_t>(Cout));
+        eqlin::eqlin_dw_f64_convert_kernel<<<static_cast<unsigned>((n_conv + 255) / 256), 256, 0, st>>>(
+            acc, dw, dbias, n_w, iCout);
+        if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "weight-gradient convert launch");
+        return EQLIN_OK;
+    }
+    CUtensorMap mdy, mx;
+    int s = encode_rows_map(&mdy, dy, Cout * G, N, pl.cpb_dy * iG, eqlin::dw::kTok);
+    if (s != EQLIN_OK) return s;
+    s = encode_rows_map(&mx, x, Cin * G, N, pl.cpb_x * iG, eqlin::dw::kTok);
+    if (s != EQLIN_OK) return s;
+    eqlin::DwParams p;
+    p.ws = static_cast<float*>(ws);
+    p.status = status;
+    p.N = N;
+    p.MO = pl.MO;
+    p.NI = pl.NI;
+    p.n_it = pl.n_it;
+    p.n_chunks = (N + eqlin::dw::kTok - 1) / eqlin::dw::kTok;
+    p.n_splits = static_cast<int>(std::max<long long>(1, std::min<long long>(pl.max_splits, p.n_chunks)));
+    p.cpb_dy = pl.cpb_dy;
+    p.cpb_x = pl.cpb_x;
+    p.dy_bytes = pl.dy_bytes;
+    p.raw_bytes = pl.raw_bytes;
+    p.a_bytes = pl.a_bytes;
+    p.b_bytes = pl.b_bytes;
+    p.tmem_cols = pl.tmem_cols;
+    p.slab_floats = pl.slab_floats;
+    const unsigned grid = static_cast<unsigned>(pl.units() * p.n_splits);
+    p.bias_offset = static_cast<size_t>(grid) * pl.slab_floats;
+    p.timeout_ns = timeout_ns;
+    switch (iG) {
+        case 2: dw_launch<2>(grid, pl.smem_bytes, st, mdy, mx, p); break;
+        case 4: dw_launch<4>(grid, pl.smem_bytes, st, mdy, mx, p); break;
+        case 8: dw_launch<8>(grid, pl.smem_bytes, st, mdy, mx, p); break;
+        default: dw_launch<16>(grid, pl.smem_bytes, st, mdy, mx, p); break;
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "weight-gradient launch");
+    eqlin::DwFinalParams f;
+    f.ws = p.ws;
+    f.dw = dw;
+    f.dbias = dbias;
+    f.Cout = iCout;
+    f.Cin = iCin;
+    f.MO = pl.MO;
+    f.NI = pl.NI;
+    f.n_it = pl.n_it;
+    f.n_splits = p.n_splits;
+    f.slab_floats = pl.slab_floats;
+    f.bias_offset = p.bias_offset;
+    const unsigned fgrid = static_cast<unsigned>(pl.units() * pl.NI * ((pl.MO + 31) / 32));
+    switch (iG) {
+        case 2: eqlin::eqlin_dw_finalize_kernel<2><<<fgrid, 256, 0, st>>>(f); break;
+        case 4: eqlin::eqlin_dw_finalize_kernel<4><<<fgrid, 256, 0, st>>>(f); break;
+        case 8: eqlin::eqlin_dw_finalize_kernel<8><<<fgrid, 256, 0, st>>>(f); break;
+        default: eqlin::eqlin_dw_finalize_kernel<16><<<fgrid, 256, 0, st>>>(f); break;
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "weight-gradient finalize launch");
+    return EQLIN_OK;
+}
+
 }  // namespace
 
 struct eqlin_handle {
@@ -502,6 +703,10 @@ struct eqlin_handle {
     int w_dtype = 0, io_dtype = 0;
     Plan plan;
     WeightBuffers buf;   // device memory owned by the handle
+    bool has_dx = false; // prepared with EQLIN_PREPARE_BACKWARD
+    Plan plan_dx;        // input-gradient operator: [Cin x Cout], adjoint filters
+    WeightBuffers buf_dx;  // its weights (status word shared with buf)
+    DwPlan dwp;          // weight-gradient tiling (bf16 I/O)
     bool sync_check = false;
     unsigned long long timeout_ns = kDefaultTimeoutNs;
 };
@@ -516,6 +721,11 @@ void free_handle(eqlin_handle* h) {
     if (h->buf.w_f64) cudaFree(h->buf.w_f64);
     if (h->buf.bias_f64) cudaFree(h->buf.bias_f64);
     if (h->buf.status) cudaFree(h->buf.status);
+    if (h->buf_dx.img) cudaFree(h->buf_dx.img);
+    if (h->buf_dx.w_f32) cudaFree(h->buf_dx.w_f32);
+    if (h->buf_dx.bias_f32) cudaFree(h->buf_dx.bias_f32);
+    if (h->buf_dx.w_f64) cudaFree(h->buf_dx.w_f64);
+    if (h->buf_dx.bias_f64) cudaFree(h->buf_dx.bias_f64);
     delete h;
 }
 
@@ -532,8 +742,14 @@ int eqlin_check_shape(int64_t Cout, int64_t Cin, int64_t G, int w_dtype, int io_
 
 int eqlin_prepare_weights(const void* w, const void* bias, int64_t Cout, int64_t Cin, int64_t G, int w_dtype,
                           int io_dtype, void* stream, eqlin_handle** out) {
+    return eqlin_prepare_weights_ex(w, bias, Cout, Cin, G, w_dtype, io_dtype, 0u, stream, out);
+}
+
+int eqlin_prepare_weights_ex(const void* w, const void* bias, int64_t Cout, int64_t Cin, int64_t G, int w_dtype,
+                             int io_dtype, unsigned flags, void* stream, eqlin_handle** out) {
     if (!out) return fail(EQLIN_ERR_INVALID_ARG, "out is NULL");
     *out = nullptr;
+    if (flags & ~static_cast<unsigned>(EQLIN_PREPARE_BACKWARD)) return fail(EQLIN_ERR_INVALID_ARG, "unknown flags");
     if (!w) return fail(EQLIN_ERR_INVALID_ARG, "w is NULL");
     int s = check_shape_impl(Cout, Cin, G, w_dtype, io_dtype);
     if (s != EQLIN_OK) return s;
@@ -604,7 +820,129 @@ int eqlin_prepare_weights(const void* w, const void* bias, int64_t Cout, int64_t
         free_handle(h);
         return cuda_fail(e, "cudaFuncSetAttribute");
     }
+    if (flags & EQLIN_PREPARE_BACKWARD) {
+        // input gradient: the same fused forward on the adjoint operator [Cin x Cout]
+        s = plan_for(Cin, Cout, G, io_dtype, static_cast<size_t>(optin), &h->plan_dx);
+        if (s != EQLIN_OK) {
+            free_handle(h);
+            return s;
+        }
+        WeightBuffers& d = h->buf_dx;
+        const Plan& pd = h->plan_dx;
+        d.status = b.status;
+        d.has_bias = false;
+        if (cudaMalloc(&d.w_f32, wf_bytes) != cudaSuccess ||
+            cudaMalloc(&d.bias_f32, static_cast<size_t>(Cin) * sizeof(float)) != cudaSuccess ||
+            (pd.path == kPathF32 && (cudaMalloc(&d.w_f64, wf_bytes * 2) != cudaSuccess ||
+                                     cudaMalloc(&d.bias_f64, static_cast<size_t>(Cin) * sizeof(double)) != cudaSuccess)) ||
+            (pd.img_alloc_bytes && cudaMalloc(&d.img, pd.img_alloc_bytes) != cudaSuccess)) {
+            cudaGetLastError();
+            free_handle(h);
+            return fail(EQLIN_ERR_OOM, "device allocation for the input-gradient weights");
+        }
+        s = launch_prep(pd, w_dtype, w, nullptr, Cin, Cout, G, d, st, /*adjoint=*/true);
+        if (s == EQLIN_OK && (e = cudaStreamSynchronize(st)) != cudaSuccess) s = cuda_fail(e, "input-gradient transform");
+        if (s == EQLIN_OK &&
+            (e = cudaFuncSetAttribute(kernel_for(pd, static_cast<int>(G)), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      static_cast<int>(pd.smem_bytes))) != cudaSuccess)
+            s = cuda_fail(e, "cudaFuncSetAttribute");
+        if (s != EQLIN_OK) {
+            free_handle(h);
+            return s;
+        }
+        h->has_dx = true;
+    }
+    if (io_dtype == EQLIN_BF16) {
+        // weight-gradient tiling (host only); a shape without one fails only in eqlin_backward_dw
+        if (plan_dw(Cout, Cin, static_cast<int>(G), static_cast<size_t>(optin), sms, &h->dwp) == EQLIN_OK) {
+            e = cudaFuncSetAttribute(dw_kernel_for(static_cast<int>(G)), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(h->dwp.smem_bytes));
+            if (e != cudaSuccess) {
+                free_handle(h);
+                return cuda_fail(e, "cudaFuncSetAttribute");
+            }
+        } else {
+            h->dwp = DwPlan();
+        }
+        g_last_error.clear();
+    }
     *out = h;
+    return EQLIN_OK;
+}
+
+int eqlin_backward_dx(const eqlin_handle* h, const void* dy, void* dx, int64_t N, void* stream) {
+    if (!h) return fail(EQLIN_ERR_INVALID_ARG, "handle is NULL");
+    if (!h->has_dx) return fail(EQLIN_ERR_INVALID_ARG, "handle was prepared without EQLIN_PREPARE_BACKWARD");
+    if (N < 0) return fail(EQLIN_ERR_INVALID_ARG, "N < 0");
+    if (N == 0) return EQLIN_OK;
+    if (!dy || !dx) return fail(EQLIN_ERR_INVALID_ARG, "dy or dx is NULL");
+    if (N >= (int64_t(1) << 31)) return fail(EQLIN_ERR_UNSUPPORTED, "N must be below 2^31");
+    if (!aligned(dy, 16) || !aligned(dx, 16)) return fail(EQLIN_ERR_MISALIGNED, "dy and dx must be 16-byte aligned");
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev != h->device) return fail(EQLIN_ERR_INVALID_ARG, "current device differs from the handle's device");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int s = launch_forward(h->plan_dx, h->Cin, h->Cout, h->G, h->sm_count, dy, dx, N, h->buf_dx, h->timeout_ns, st);
+    if (s != EQLIN_OK) return s;
+    if (h->sync_check) {
+        int dst = 0;
+        if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return cuda_fail(e, "backward_dx (EQLIN_SYNC_CHECK)");
+        if ((e = cudaMemcpy(&dst, h->buf.status, sizeof(int), cudaMemcpyDeviceToHost)) != cudaSuccess)
+            return cuda_fail(e, "status read");
+        if (dst != 0) return fail(dst, "device reported an error (status word)");
+    }
+    return EQLIN_OK;
+}
+
+int eqlin_backward_dw_workspace_size(const eqlin_handle* h, int64_t N, size_t* bytes) {
+    if (!h || !bytes) return fail(EQLIN_ERR_INVALID_ARG, "NULL argument");
+    if (N < 0) return fail(EQLIN_ERR_INVALID_ARG, "N < 0");
+    const bool f32_path = h->io_dtype == EQLIN_F32;
+    if (!f32_path && h->dwp.MO == 0) return fail(EQLIN_ERR_UNSUPPORTED, "no weight-gradient tile for this shape");
+    *bytes = N == 0 ? 0 : dw_workspace_bytes(h->dwp, f32_path, h->Cout, h->Cin, h->G, N);
+    return EQLIN_OK;
+}
+
+int eqlin_backward_dw(const eqlin_handle* h, const void* x, const void* dy, float* dw, float* dbias, int64_t N,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+    if (!h) return fail(EQLIN_ERR_INVALID_ARG, "handle is NULL");
+    if (!dw) return fail(EQLIN_ERR_INVALID_ARG, "dw is NULL");
+    if (N < 0) return fail(EQLIN_ERR_INVALID_ARG, "N < 0");
+    if (N >= (int64_t(1) << 31)) return fail(EQLIN_ERR_UNSUPPORTED, "N must be below 2^31");
+    if (!aligned(dw, 4) || (dbias && !aligned(dbias, 4)))
+        return fail(EQLIN_ERR_MISALIGNED, "dw and dbias must be 4-byte aligned");
+    const bool f32_path = h->io_dtype == EQLIN_F32;
+    if (!f32_path && h->dwp.MO == 0) return fail(EQLIN_ERR_UNSUPPORTED, "no weight-gradient tile for this shape");
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev != h->device) return fail(EQLIN_ERR_INVALID_ARG, "current device differs from the handle's device");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t n_w = static_cast<size_t>(h->Cout * h->Cin * h->G);
+    if (N == 0) {  // the gradient of an empty batch is zero
+        if ((e = cudaMemsetAsync(dw, 0, n_w * sizeof(float), st)) != cudaSuccess) return cuda_fail(e, "dw clear");
+        if (dbias && (e = cudaMemsetAsync(dbias, 0, static_cast<size_t>(h->Cout) * sizeof(float), st)) != cudaSuccess)
+            return cuda_fail(e, "dbias clear");
+        return EQLIN_OK;
+    }
+    if (!x || !dy) return fail(EQLIN_ERR_INVALID_ARG, "x or dy is NULL");
+    if (!aligned(x, 16) || !aligned(dy, 16)) return fail(EQLIN_ERR_MISALIGNED, "x and dy must be 16-byte aligned");
+    const size_t need = dw_workspace_bytes(h->dwp, f32_path, h->Cout, h->Cin, h->G, N);
+    if (!workspace || workspace_bytes < need)
+        return fail(EQLIN_ERR_INVALID_ARG, "workspace missing or smaller than eqlin_backward_dw_workspace_size (" +
+                                               std::to_string(need) + " bytes)");
+    if (!aligned(workspace, 16)) return fail(EQLIN_ERR_MISALIGNED, "workspace must be 16-byte aligned");
+    int s = launch_dw(h->dwp, f32_path, h->Cout, h->Cin, h->G, x, dy, dw, dbias, N, workspace, h->buf.status,
+                      h->timeout_ns, st);
+    if (s != EQLIN_OK) return s;
+    if (h->sync_check) {
+        int dst = 0;
+        if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return cuda_fail(e, "backward_dw (EQLIN_SYNC_CHECK)");
+        if ((e = cudaMemcpy(&dst, h->buf.status, sizeof(int), cudaMemcpyDeviceToHost)) != cudaSuccess)
+            return cuda_fail(e, "status read");
+        if (dst != 0) return fail(dst, "device reported an error (status word)");
+    }
     return EQLIN_OK;
 }
 

@@ -1,0 +1,533 @@
+// eqlin_bwd_dw.cuh -- weight and bias gradients of EQ-Linear (bf16 I/O) on sm_100a.
+//
+// The page "Flash EQ-Linear: Accelerating Equivariant Linear Layers via Group-wise
+// Discrete Fourier Transform" lists a backward pass among its kernels (section
+// "Implementacion").  For y[n,o,g] = bias[o] + sum_{i,h} w[o,i,(g-h) mod G] x[n,i,h]
+// and an upstream gradient dy, the chain rule gives
+//     dw[o,i,m] = sum_n sum_g dy[n,o,g] x[n,i,(g-m) mod G]     (a circular
+//                 cross-correlation along the group axis, summed over tokens)
+//     dbias[o]  = sum_n sum_g dy[n,o,g].
+// By the convolution theorem (section "Enfoque Algoritmico") the correlation is a
+// pointwise product of spectra, and with real data only the half spectrum is needed:
+//     dW_k[o,i] = sum_n DY_k[n,o] conj(X_k[n,i]),   k = 0 .. G/2,
+//     dw[o,i,:] = inverse real DFT of dW[o,i,:] (scale 1/G).
+// The sum over tokens is a GEMM with K = tokens: per frequency a [Cout x N] by [N x Cin]
+// product, 2G-2 real products per K step (4 per complex frequency, 1 per real one).
+//
+// Kernel eqlin_dw_tc_kernel<G>: the grid is units x token splits.  A unit is an
+// (MO-row output tile, NI-column input tile) pair; each CTA owns one unit and a
+// contiguous range of 32-token chunks, and keeps its partial dW in TMEM:
+//   warp 0      TMA producer: per chunk the dy tile [32 tokens x MO*G] and the x tile
+//               [32 tokens x NI*G] into a 2-stage raw ring (zero fill past N, Cout, Cin).
+//   warp 1      MMA issuer + TMEM owner: per chunk and 16-token K step, tcgen05.mma with
+//               A = DY^ plane [128 rows (MO valid) x 16 tokens], B = X^ plane [NI x 16],
+//               D plane in TMEM (lane = o, column = i):
+//                 D_0 += DY_0 X_0, D_1 += DY_{G/2} X_{G/2},
+//                 Re: D_2k   += DYr Xr + DYi Xi,   Im: D_2k+1 += DYi Xr - DYr Xi
+//               (the minus through the descriptor's negate-A bit).
+//   warps 2-9   transpose + DFT: a unit of work is one channel x 8 tokens; the thread
+//               loads the 8 tokens' G-vectors (lanes = 32 consecutive channels, so the
+//               loads are contiguous), runs the real DFT over G in fp32 registers, packs
+//               each plane's 8 values to bf16 and writes one 16-byte piece per plane
+//               into the K-major SWIZZLE_64B spectra (row = channel, 64-byte row = the
+//               chunk's 32 tokens).  The dy threads also sum plane 0 (the group sum) for
+//               dbias, in a fixed order.  Spectra are double-buffered.
+//               After the last chunk the same warps read the TMEM partial dW and write it
+//               to the CTA's slab of the workspace.
+// eqlin_dw_finalize_kernel<G> then sums the slabs of each unit over its token splits
+// in a fixed order (deterministic), runs the inverse real DFT over the planes in
+// float64 and writes dw (fp32) and dbias (fp32).
+//
+// The dy spectra of plane p start at row p*MO of the A region; an MMA reads 128 rows
+// from there, so rows MO..127 of its D are other planes' data (never read back).  The
+// A region holds G*MO + (128 - MO) rows, the tail zeroed once.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "eqlin_layout.h"
+#include "group_dft.cuh"
+#include "sm100_ptx.cuh"
+
+namespace eqlin {
+
+struct DwParams {
+    float* ws;                 // workspace: per CTA a slab [G][NI][MO] fp32, then per CTA [MO] bias sums
+    int* status;               // device status word (first error wins)
+    long long N;
+    int MO, NI;                // rows / columns of a unit (multiples of 16; MO <= 128, G*NI <= 512)
+    int n_it;                  // input tiles per output tile
+    int n_splits;              // CTAs per unit (token splits)
+    long long n_chunks;        // ceil(N / 32)
+    int cpb_dy, cpb_x;         // channels per TMA box of the dy / x tile
+    uint32_t dy_bytes;         // dy part of a raw stage: 32 * MO * G * 2
+    uint32_t raw_bytes;        // one raw stage: dy part + x part (multiple of 1 KB)
+    uint32_t a_bytes;          // A (dy spectra) region of one spectra buffer (multiple of 1 KB)
+    uint32_t b_bytes;          // B (x spectra) region (multiple of 1 KB)
+    uint32_t tmem_cols;        // power of two >= G * NI
+    size_t slab_floats;        // G * NI * MO
+    size_t bias_offset;        // float offset of the bias partials: gridDim.x * slab_floats
+    unsigned long long timeout_ns;
+};
+
+namespace dw {
+
+constexpr int kTok = 32;           // tokens per chunk (one 64-byte K-major row)
+constexpr int kRawStages = 2;
+constexpr int kSpecBufs = 2;
+constexpr int kDftWarps = 8;
+constexpr int kDftThreads = kDftWarps * 32;
+constexpr int kWarpProducer = 0;
+constexpr int kWarpMma = 1;
+constexpr int kWarpDft0 = 2;
+constexpr int kThreads = (2 + kDftWarps) * 32;
+constexpr int kBarDft = 1;         // named barrier among the DFT warps
+constexpr uint32_t kWaitSleepNs = 20000;
+
+struct Ctl {
+    volatile int abort;
+    uint32_t tmem_base;
+};
+
+// Bounded mbarrier wait; false (after flagging) on timeout or abort.
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, Ctl* ctl, int* status,
+                                             unsigned long long timeout_ns) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = ptx::globaltimer_ns();
+    for (uint32_t spin = 1;; ++spin) {
+        if (ptx::mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
+        if ((spin & 7u) == 0) {
+            if (ctl->abort) return false;
+            if (ptx::globaltimer_ns() - t0 > timeout_ns) {
+                ctl->abort = 1;
+                atomicCAS(status, 0, kDeviceErrTimeout);
+                return false;
+            }
+        }
+    }
+}
+
+// Wait that ignores the abort flag (for copies or MMAs in flight before exit).
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, int* status,
+                                           unsigned long long timeout_ns) {
+    const uint64_t t0 = ptx::globaltimer_ns();
+    while (!ptx::mbar_try_wait(bar, parity)) {
+        if (ptx::globaltimer_ns() - t0 > timeout_ns) {
+            atomicCAS(status, 0, kDeviceErrTimeout);
+            return;
+        }
+    }
+}
+
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// G bf16 values (one token's group vector of one channel) -> fp32.
+template <int G>
+__device__ __forceinline__ void load_group(const uint8_t* src, float (&v)[G]) {
+    if constexpr (G == 2) {
+        const uint32_t u = *reinterpret_cast<const uint32_t*>(src);
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u));
+        v[0] = f.x;
+        v[1] = f.y;
+    } else if constexpr (G == 4) {
+        const uint2 u = *reinterpret_cast<const uint2*>(src);
+        const uint32_t w[2] = {u.x, u.y};
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+            v[2 * j] = f.x;
+            v[2 * j + 1] = f.y;
+        }
+    } else {
+#pragma unroll
+        for (int q = 0; q < G / 8; ++q) {
+            const uint4 u = *reinterpret_cast<const uint4*>(src + 16 * q);
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+                v[8 * q + 2 * j] = f.x;
+                v[8 * q + 2 * j + 1] = f.y;
+            }
+        }
+    }
+}
+
+template <int G>
+__device__ __forceinline__ void planes_of(const float (&v)[G], float (&p)[G]) {
+    if constexpr (G == 2) {
+        p[0] = v[0] + v[1];
+        p[1] = v[0] - v[1];
+    } else {
+        rdft_planes<G, float>(v, p);
+    }
+}
+
+// One unit: channel c of the dy tile (is_dy) or of the x tile, tokens 8*tg .. 8*tg+7
+// of the chunk.  Raw tile layout: boxes of cpb channels, each [32 tokens][cpb*G] bf16.
+// Output: plane p of the channel at row r = p*rows_per_plane + c of `spec`, 16-byte
+// piece tg of the 64-byte row, SWIZZLE_64B (piece j of row r at j ^ ((r >> 1) & 3)).
+template <int G>
+__device__ __forceinline__ float transform_unit(const uint8_t* raw, int cpb, int c, int tg, uint8_t* spec,
+                                                int rows_per_plane) {
+    const int box = c / cpb, cc = c - box * cpb;
+    const int row_bytes = cpb * G * 2;
+    const uint8_t* src = raw + static_cast<size_t>(box) * (kTok * row_bytes) +
+                         static_cast<size_t>(tg * 8) * row_bytes + cc * G * 2;
+    uint32_t packed[G][4];
+    float s0 = 0.0f;
+#pragma unroll
+    for (int jp = 0; jp < 4; ++jp) {
+        float va[G], vb[G], pa[G], pb[G];
+        load_group<G>(src + (2 * jp) * row_bytes, va);
+        load_group<G>(src + (2 * jp + 1) * row_bytes, vb);
+        planes_of<G>(va, pa);
+        planes_of<G>(vb, pb);
+        s0 += pa[0] + pb[0];
+#pragma unroll
+        for (int p = 0; p < G; ++p) packed[p][jp] = pack2(pa[p], pb[p]);
+    }
+#pragma unroll
+    for (int p = 0; p < G; ++p) {
+        const int r = p * rows_per_plane + c;
+        uint8_t* dst = spec + static_cast<size_t>(r) * kPlaneRowBytes + ((tg ^ ((r >> 1) & 3)) << 4);
+        *reinterpret_cast<uint4*>(dst) = make_uint4(packed[p][0], packed[p][1], packed[p][2], packed[p][3]);
+    }
+    return s0;
+}
+
+}  // namespace dw
+
+template <int G>
+__global__ void __launch_bounds__(dw::kThreads, 1)
+    eqlin_dw_tc_kernel(const __grid_constant__ CUtensorMap tmap_dy, const __grid_constant__ CUtensorMap tmap_x,
+                       const DwParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t spec_bytes = p.a_bytes + p.b_bytes;
+    uint8_t* raw0 = base;
+    uint8_t* spec0 = raw0 + dw::kRawStages * p.raw_bytes;
+    float* bias_sm = reinterpret_cast<float*>(spec0 + dw::kSpecBufs * spec_bytes);
+    // bias_sm[tg][c]: group sums of dy channel c over token group tg of every chunk; each
+    // slot has a single writer (the unit -> thread map is the same for every chunk), so
+    // the per-CTA sums are formed in a fixed order
+    uint64_t* bars = reinterpret_cast<uint64_t*>(bias_sm + 4 * p.MO);
+    dw::Ctl* ctl = reinterpret_cast<dw::Ctl*>(bars + 2 * dw::kRawStages + 2 * dw::kSpecBufs + 2);
+
+    auto bar_raw_full = [&](int s) { return ptx::smem_u32(bars + s); };
+    auto bar_raw_empty = [&](int s) { return ptx::smem_u32(bars + dw::kRawStages + s); };
+    auto bar_spec_full = [&](int s) { return ptx::smem_u32(bars + 2 * dw::kRawStages + s); };
+    auto bar_spec_empty = [&](int s) { return ptx::smem_u32(bars + 2 * dw::kRawStages + dw::kSpecBufs + s); };
+    const uint32_t bar_acc_full = ptx::smem_u32(bars + 2 * dw::kRawStages + 2 * dw::kSpecBufs);
+    const uint32_t bar_drain = ptx::smem_u32(bars + 2 * dw::kRawStages + 2 * dw::kSpecBufs + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int unit = blockIdx.x / p.n_splits, split = blockIdx.x - unit * p.n_splits;
+    const int ot = unit / p.n_it, it = unit - ot * p.n_it;
+    const int o0 = ot * p.MO, i0 = it * p.NI;
+    const long long c_begin = p.n_chunks * split / p.n_splits;
+    const long long c_end = p.n_chunks * (split + 1) / p.n_splits;
+    const int n_mine = static_cast<int>(c_end - c_begin);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < dw::kRawStages; ++s) {
+            ptx::mbar_init(bar_raw_full(s), 1);
+            ptx::mbar_init(bar_raw_empty(s), dw::kDftThreads);
+        }
+        for (int s = 0; s < dw::kSpecBufs; ++s) {
+            ptx::mbar_init(bar_spec_full(s), dw::kDftThreads);
+            ptx::mbar_init(bar_spec_empty(s), 1);
+        }
+        ptx::mbar_init(bar_acc_full, 1);
+        ptx::mbar_init(bar_drain, 1);
+        ctl->abort = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == dw::kWarpMma) {
+        ptx::tmem_alloc(ptx::smem_u32(&ctl->tmem_base), p.tmem_cols);
+        ptx::tmem_relinquish();
+    }
+    if (warp == dw::kWarpProducer && lane == 0) {
+        ptx::prefetch_tmap(&tmap_dy);
+        ptx::prefetch_tmap(&tmap_x);
+    }
+    if (warp >= dw::kWarpDft0) {
+        const int t = threadIdx.x - dw::kWarpDft0 * 32;
+        for (int c = t; c < 4 * p.MO; c += dw::kDftThreads) bias_sm[c] = 0.0f;
+        // A-region tail rows (read by the MMA, never written by the transform): zero
+        const int tail0 = G * p.MO, tail1 = G * p.MO + (kMmaM - p.MO);
+        for (int b = 0; b < dw::kSpecBufs; ++b) {
+            uint8_t* a = spec0 + static_cast<size_t>(b) * spec_bytes;
+            for (int idx = tail0 * 4 + t; idx < tail1 * 4; idx += dw::kDftThreads)
+                reinterpret_cast<uint4*>(a)[idx] = make_uint4(0, 0, 0, 0);
+        }
+        ptx::fence_proxy_async_smem();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = ctl->tmem_base;
+    ptx::grid_launch_dependents();
+    ptx::grid_dependency_wait();
+
+    if (warp == dw::kWarpProducer) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            const int nb_dy = p.MO / p.cpb_dy, nb_x = p.NI / p.cpb_x;
+            const uint32_t box_dy = dw::kTok * p.cpb_dy * G * 2, box_x = dw::kTok * p.cpb_x * G * 2;
+            const uint32_t tx = p.dy_bytes + dw::kTok * p.NI * G * 2;
+            const uint32_t s_raw0 = ptx::smem_u32(raw0);
+            int issued = 0;
+            for (int j = 0; j < n_mine; ++j) {
+                const int s = j % dw::kRawStages;
+                const uint32_t ph = static_cast<uint32_t>(j / dw::kRawStages) & 1u;
+                if (!dw::wait_bounded(bar_raw_empty(s), ph ^ 1u, ctl, p.status, p.timeout_ns)) break;
+                const int n0 = static_cast<int>((c_begin + j) * dw::kTok);
+                const uint32_t dst = s_raw0 + s * p.raw_bytes;
+                ptx::mbar_arrive_expect_tx(bar_raw_full(s), tx);
+                for (int b = 0; b < nb_dy; ++b)
+                    ptx::tma_load_2d(dst + b * box_dy, &tmap_dy, (o0 + b * p.cpb_dy) * G, n0, bar_raw_full(s));
+                for (int b = 0; b < nb_x; ++b)
+                    ptx::tma_load_2d(dst + p.dy_bytes + b * box_x, &tmap_x, (i0 + b * p.cpb_x) * G, n0,
+                                     bar_raw_full(s));
+                ++issued;
+            }
+            // every copy issued must land before the CTA exits
+            for (int s = 0; s < dw::kRawStages && s < issued; ++s) {
+                const int last = ((issued - 1 - s) / dw::kRawStages) * dw::kRawStages + s;
+                dw::drain_wait(bar_raw_full(s), static_cast<uint32_t>(last / dw::kRawStages) & 1u, p.status,
+                               p.timeout_ns);
+            }
+        }
+    } else if (warp == dw::kWarpMma) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t ID = idesc_bf16_f32(kMmaM, p.NI, false);
+            const uint32_t ID_NEG = idesc_bf16_f32(kMmaM, p.NI, true);
+            const uint32_t s_spec0 = ptx::smem_u32(spec0);
+            const uint32_t a_plane16 = static_cast<uint32_t>(p.MO) * kPlaneRowBytes / 16;
+            const uint32_t b_plane16 = static_cast<uint32_t>(p.NI) * kPlaneRowBytes / 16;
+            bool ok = true;
+            for (int j = 0; j < n_mine; ++j) {
+                const int sb = j % dw::kSpecBufs;
+                const uint32_t ph = static_cast<uint32_t>(j / dw::kSpecBufs) & 1u;
+                if (!dw::wait_bounded(bar_spec_full(sb), ph, ctl, p.status, p.timeout_ns)) {
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+                const uint32_t a_addr = s_spec0 + sb * spec_bytes;
+                const uint32_t a_lo = ptx::sdesc_sw64_lo(a_addr), b_lo = ptx::sdesc_sw64_lo(a_addr + p.a_bytes);
+#pragma unroll
+                for (int ks = 0; ks < dw::kTok / 16; ++ks) {
+                    const uint32_t acc0 = (j > 0 || ks > 0) ? 1u : 0u;
+                    auto A = [&](int pl) { return ptx::sdesc_sw64_from_lo(a_lo + pl * a_plane16 + ks * 2); };
+                    auto B = [&](int pl) { return ptx::sdesc_sw64_from_lo(b_lo + pl * b_plane16 + ks * 2); };
+                    auto D = [&](int pl) { return tmem_base + static_cast<uint32_t>(pl * p.NI); };
+                    ptx::umma_f16(D(0), A(0), B(0), ID, acc0);
+                    ptx::umma_f16(D(1), A(1), B(1), ID, acc0);
+#pragma unroll
+                    for (int k = 1; k < G / 2; ++k) {
+                        const int pr = 2 * k, pi = 2 * k + 1;
+                        ptx::umma_f16(D(pr), A(pr), B(pr), ID, acc0);      // + DYr Xr
+                        ptx::umma_f16(D(pr), A(pi), B(pi), ID, 1u);        // + DYi Xi
+                        ptx::umma_f16(D(pi), A(pi), B(pr), ID, acc0);      // + DYi Xr
+                        ptx::umma_f16(D(pi), A(pr), B(pi), ID_NEG, 1u);    // - DYr Xi
+                    }
+                }
+                ptx::umma_commit(bar_spec_empty(sb));
+            }
+            if (ok) ptx::umma_commit(bar_acc_full);
+            ptx::umma_commit(bar_drain);
+            dw::drain_wait(bar_drain, 0, p.status, p.timeout_ns);
+        }
+    } else {
+        // ------------------------------------------------------------ transform warps
+        const int t = threadIdx.x - dw::kWarpDft0 * 32;
+        const int width = p.MO + p.NI;
+        const int n_units = 4 * width;
+        bool ok = true;
+        for (int j = 0; j < n_mine; ++j) {
+            const int s = j % dw::kRawStages, sb = j % dw::kSpecBufs;
+            const uint32_t ph_raw = static_cast<uint32_t>(j / dw::kRawStages) & 1u;
+            const uint32_t ph_spec = static_cast<uint32_t>(j / dw::kSpecBufs) & 1u;
+            bool got = dw::wait_bounded(bar_raw_full(s), ph_raw, ctl, p.status, p.timeout_ns);
+            if (got) got = dw::wait_bounded(bar_spec_empty(sb), ph_spec ^ 1u, ctl, p.status, p.timeout_ns);
+            if (!ptx::named_bar_and(dw::kBarDft, dw::kDftThreads, got)) {
+                ok = false;
+                break;
+            }
+            const uint8_t* raw = raw0 + static_cast<size_t>(s) * p.raw_bytes;
+            uint8_t* spec = spec0 + static_cast<size_t>(sb) * spec_bytes;
+            for (int u = t; u < n_units; u += dw::kDftThreads) {
+                const int tg = u / width, ch = u - tg * width;
+                if (ch < p.MO) {
+                    bias_sm[tg * p.MO + ch] += dw::transform_unit<G>(raw, p.cpb_dy, ch, tg, spec, p.MO);
+                } else {
+                    dw::transform_unit<G>(raw + p.dy_bytes, p.cpb_x, ch - p.MO, tg, spec + p.a_bytes, p.NI);
+                }
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::mbar_arrive(bar_raw_empty(s));
+            ptx::mbar_arrive(bar_spec_full(sb));
+        }
+        // partial dW: TMEM -> this CTA's workspace slab [G][NI][MO]
+        const bool got = ok && dw::wait_bounded(bar_acc_full, 0, ctl, p.status, p.timeout_ns);
+        const bool all = ptx::named_bar_and(dw::kBarDft, dw::kDftThreads, got);
+        float* slab = p.ws + static_cast<size_t>(blockIdx.x) * p.slab_floats;
+        if (all) {
+            ptx::tc_fence_after();
+            const int q = warp & 3, half = (warp - dw::kWarpDft0) >> 2;
+            const int row = q * 32 + lane;
+            if (q * 32 < p.MO) {
+                for (int pl = half * (G / 2); pl < (half + 1) * (G / 2); ++pl) {
+                    for (int cb = 0; cb < p.NI; cb += 16) {
+                        uint32_t v[16];
+                        ptx::tmem_ld_32x32b<16>(tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                                    static_cast<uint32_t>(pl * p.NI + cb),
+                                                v);
+                        ptx::tmem_wait_ld();
+                        if (row < p.MO) {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e)
+                                slab[(static_cast<size_t>(pl) * p.NI + cb + e) * p.MO + row] = __uint_as_float(v[e]);
+                        }
+                    }
+                }
+            }
+        }
+        // dbias partial of this CTA (every CTA writes it; the finalize reads input tile 0's)
+        ptx::named_bar_sync(dw::kBarDft, dw::kDftThreads);
+        for (int c = t; c < p.MO; c += dw::kDftThreads)
+            p.ws[p.bias_offset + static_cast<size_t>(blockIdx.x) * p.MO + c] =
+                (bias_sm[c] + bias_sm[p.MO + c]) + (bias_sm[2 * p.MO + c] + bias_sm[3 * p.MO + c]);
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == dw::kWarpMma) {
+        __syncwarp();
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem_base, p.tmem_cols);
+    }
+}
+
+// Sums each unit's slabs over its token splits (fixed order), then the inverse real
+// DFT over the planes: with P_k = sum_n DY_k conj(X_k) (unscaled transforms),
+//   dw[o,i,m] = (1/G) [P_0 + (-1)^m P_{G/2} + 2 sum_{0<k<G/2} Re(P_k e^{+2 pi i m k / G})].
+// Block = 32 output rows x one input column of one unit; warp w sums splits w, w+8, ...
+struct DwFinalParams {
+    const float* ws;
+    float* dw;            // [Cout, Cin, G]
+    float* dbias;         // [Cout] or nullptr
+    int Cout, Cin;
+    int MO, NI, n_it, n_splits;
+    size_t slab_floats, bias_offset;
+};
+
+template <int G>
+__global__ void __launch_bounds__(256) eqlin_dw_finalize_kernel(const DwFinalParams f) {
+    __shared__ double red[8][G + 1][32];
+    const int nob = (f.MO + 31) / 32;
+    const int ob = blockIdx.x % nob;
+    const int ii = (blockIdx.x / nob) % f.NI;
+    const int unit = blockIdx.x / (nob * f.NI);
+    const int ot = unit / f.n_it, it = unit - ot * f.n_it;
+    const int i = it * f.NI + ii;
+    if (i >= f.Cin) return;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int oo = ob * 32 + lane;
+    const bool valid = oo < f.MO;
+    const bool with_bias = f.dbias != nullptr && it == 0 && ii == 0;
+    double acc[G + 1];
+#pragma unroll
+    for (int q = 0; q <= G; ++q) acc[q] = 0.0;
+    if (valid) {
+        for (int s = warp; s < f.n_splits; s += 8) {
+            const size_t cta = static_cast<size_t>(unit) * f.n_splits + s;
+            const float* slab = f.ws + cta * f.slab_floats;
+#pragma unroll
+            for (int pl = 0; pl < G; ++pl) acc[pl] += slab[(static_cast<size_t>(pl) * f.NI + ii) * f.MO + oo];
+            if (with_bias) acc[G] += f.ws[f.bias_offset + cta * f.MO + oo];
+        }
+    }
+#pragma unroll
+    for (int q = 0; q <= G; ++q) red[warp][q][lane] = acc[q];
+    __syncthreads();
+    if (warp != 0) return;
+    const int o = ot * f.MO + oo;
+    if (!valid || o >= f.Cout) return;
+    double P[G + 1];
+#pragma unroll
+    for (int q = 0; q <= G; ++q) {
+        double v = 0.0;
+        for (int w = 0; w < 8; ++w) v += red[w][q][lane];
+        P[q] = v;
+    }
+    double z[G], out[G];
+    z[0] = P[0] / G;
+    z[1] = P[1] / G;
+#pragma unroll
+    for (int q = 2; q < G; ++q) z[q] = 2.0 * P[q] / G;
+    if constexpr (G == 2) {
+        out[0] = z[0] + z[1];
+        out[1] = z[0] - z[1];
+    } else {
+        RealIdft<G, double>::run(z, out);
+    }
+    float* dst = f.dw + (static_cast<size_t>(o) * f.Cin + i) * G;
+#pragma unroll
+    for (int m = 0; m < G; ++m) dst[m] = static_cast<float>(out[m]);
+    if (with_bias) f.dbias[o] = static_cast<float>(P[G]);
+}
+
+// ------------------------------------------------------------------ fp32 I/O
+// Weight and bias gradients for fp32 I/O on CUDA cores in float64, straight from the
+// definition: thread = (o, i) pair, blockIdx.y = token slice; partial sums are added
+// to a float64 accumulator [Cout][Cin][G] followed by [Cout] (zeroed by the caller),
+// which eqlin_dw_f64_convert_kernel rounds to fp32.
+template <int G>
+__global__ void __launch_bounds__(256)
+    eqlin_dw_f64_kernel(const float* __restrict__ x, const float* __restrict__ dy, double* __restrict__ acc,
+                        long long N, int Cin, int Cout, long long tokens_per_slice) {
+    const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx >= static_cast<long long>(Cout) * Cin) return;
+    const int o = static_cast<int>(idx / Cin), i = static_cast<int>(idx % Cin);
+    const long long n0 = static_cast<long long>(blockIdx.y) * tokens_per_slice;
+    const long long n1 = n0 + tokens_per_slice < N ? n0 + tokens_per_slice : N;
+    double s[G], b = 0.0;
+#pragma unroll
+    for (int m = 0; m < G; ++m) s[m] = 0.0;
+    for (long long n = n0; n < n1; ++n) {
+        double d[G], xv[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            d[g] = dy[(n * Cout + o) * G + g];
+            xv[g] = x[(n * Cin + i) * G + g];
+        }
+#pragma unroll
+        for (int m = 0; m < G; ++m) {
+#pragma unroll
+            for (int g = 0; g < G; ++g) s[m] = fma(d[g], xv[(g - m + G) % G], s[m]);
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g) b += d[g];
+    }
+    if (n1 <= n0) return;
+#pragma unroll
+    for (int m = 0; m < G; ++m) atomicAdd(acc + (static_cast<size_t>(o) * Cin + i) * G + m, s[m]);
+    if (i == 0) atomicAdd(acc + static_cast<size_t>(Cout) * Cin * G + o, b);
+}
+
+__global__ void eqlin_dw_f64_convert_kernel(const double* __restrict__ acc, float* __restrict__ dw,
+                                            float* __restrict__ dbias, size_t n_w, int Cout) {
+    const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx < n_w) dw[idx] = static_cast<float>(acc[idx]);
+    if (dbias != nullptr && idx < static_cast<size_t>(Cout)) dbias[idx] = static_cast<float>(acc[n_w + idx]);
+}
+
+}  // namespace eqlin

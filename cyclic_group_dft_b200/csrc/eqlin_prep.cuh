@@ -27,19 +27,27 @@ __device__ __forceinline__ double load_as_double<__nv_bfloat16>(const __nv_bfloa
     return static_cast<double>(__bfloat162float(p[i]));
 }
 
-// One thread per (o, i): real DFT of w[o, i, :] in float64, scaled for the folded
-// inverse (1/G real planes, 2/G complex planes), stored to w_f32[p][i][o] and, when
-// w_f64 is not null, to w_f64[p][i][o].  Thread (o, i = 0) also converts bias[o]
-// (0 when bias is null) to bias_f32[o] and, when requested, bias_f64[o].
+// One thread per (o, i) of the operator: real DFT of its filter f[o, i, :] in
+// float64, scaled for the folded inverse (1/G real planes, 2/G complex planes),
+// stored to w_f32[p][i][o] and, when w_f64 is not null, to w_f64[p][i][o].  Thread
+// (o, i = 0) also converts bias[o] (0 when bias is null) to bias_f32[o] and, when
+// requested, bias_f64[o].
+//
+// The operator is [Cout, Cin] with filter f = w (w is [Cout, Cin, G]) when
+// `adjoint` is false.  With `adjoint` true it is the input gradient of the layer:
+// dx[n,i,h] = sum_{o,g} w[o,i,(g-h) mod G] dy[n,o,g] is the same block-circulant
+// product with the channel axes swapped and the filter reflected,
+// f[i, o, m] = w[o, i, (-m) mod G]; then Cout and Cin here are the layer's Cin and
+// Cout and w is still the layer's [Cin_here, Cout_here, G] weight.
 template <typename T>
 __global__ void eqlin_prep_freq_kernel(const T* __restrict__ w, const T* __restrict__ bias, int Cout,
                                        int Cin, int G, float* __restrict__ w_f32,
                                        float* __restrict__ bias_f32, double* __restrict__ w_f64,
-                                       double* __restrict__ bias_f64) {
+                                       double* __restrict__ bias_f64, bool adjoint = false) {
     const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (idx >= static_cast<long long>(Cout) * Cin) return;
     const int o = static_cast<int>(idx / Cin), i = static_cast<int>(idx % Cin);
-    const size_t base = static_cast<size_t>(idx) * G;
+    const size_t base = adjoint ? (static_cast<size_t>(i) * Cout + o) * G : static_cast<size_t>(idx) * G;
     for (int p = 0; p < G; ++p) {
         const int k = p == 0 ? 0 : (p == 1 ? G / 2 : p / 2);
         const bool imag = p >= 2 && (p & 1);
@@ -48,7 +56,8 @@ __global__ void eqlin_prep_freq_kernel(const T* __restrict__ w, const T* __restr
         for (int m = 0; m < G; ++m) {
             double s, c;
             sincospi(2.0 * static_cast<double>((m * k) % G) / G, &s, &c);
-            acc += load_as_double(w, base + m) * (imag ? -s : c);
+            const int src = adjoint ? (G - m) % G : m;
+            acc += load_as_double(w, base + src) * (imag ? -s : c);
         }
         const size_t dst = (static_cast<size_t>(p) * Cin + i) * Cout + o;
         w_f32[dst] = static_cast<float>(scale * acc);

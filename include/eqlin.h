@@ -1,5 +1,6 @@
 /*
- * eqlin.h -- C ABI of the B200 (sm_100a) EQ-Linear forward over the cyclic group C_G.
+ * eqlin.h -- C ABI of the B200 (sm_100a) EQ-Linear over the cyclic group C_G:
+ * the forward pass and its backward (input, weight and bias gradients).
  *
  * The operation.  Page "Flash EQ-Linear: Accelerating Equivariant Linear Layers
  * via Group-wise Discrete Fourier Transform", section "Percepcion Central": an
@@ -204,6 +205,94 @@ EQLIN_API int eqlin_check_shape(int64_t Cout, int64_t Cin, int64_t G, int w_dtyp
 #define EQLIN_NOALLOC_SCRATCH_BYTES (4u * 1024u * 1024u)
 EQLIN_API int eqlin_forward_noalloc(const void* x, const void* w, const void* bias, void* y, int64_t N,
                                     int64_t Cout, int64_t Cin, int64_t G, int dtype, void* stream);
+
+/*
+ * Backward pass.  The page's section "Implementacion" lists backward kernels beside the
+ * forward; its results section ("Pasada Backward") reports their speed-ups.  By the chain
+ * rule on the definition above, for a loss L and its upstream gradient dy = dL/dy
+ * ([N, Cout, G]):
+ *
+ *     dx[n,i,h] = sum_{o<Cout} sum_{g<G} w[o,i,(g-h) mod G] * dy[n,o,g]
+ *     dw[o,i,m] = sum_{n<N}    sum_{g<G} dy[n,o,g] * x[n,i,(g-m) mod G]
+ *     dbias[o]  = sum_{n<N}    sum_{g<G} dy[n,o,g]
+ *
+ * Both gradients are circular correlations along the group axis.  In the frequency domain
+ * (section "Enfoque Algoritmico") they become per-frequency products on the half
+ * spectrum: dX_k = W^_k^H dY_k, and dW_k = sum_n dY_k conj(X_k).
+ *   - dx is the forward of the adjoint operator: the channel axes are swapped and the
+ *     filters reflected, f[i,o,m] = w[o,i,(-m) mod G], so the same fused kernels run it
+ *     with weights prepared for it.
+ *   - dw is a contraction over tokens: a [Cout x N] by [N x Cin] product per frequency,
+ *     on tcgen05 for bf16, then an inverse DFT over the group axis.
+ */
+
+/* eqlin_prepare_weights_ex flag: also prepare the input-gradient weights, so the
+ * handle can run eqlin_backward_dx.  They are about the same size as the forward
+ * weights. */
+#define EQLIN_PREPARE_BACKWARD 1u
+
+/*
+ * eqlin_prepare_weights_ex -- eqlin_prepare_weights with flags (0 or
+ * EQLIN_PREPARE_BACKWARD).  eqlin_prepare_weights(...) is this call with flags 0.
+ * Errors: as eqlin_prepare_weights; INVALID_ARG for an unknown flag bit.
+ */
+EQLIN_API int eqlin_prepare_weights_ex(const void* w, const void* bias, int64_t Cout, int64_t Cin, int64_t G,
+                                       int w_dtype, int io_dtype, unsigned flags, void* stream,
+                                       eqlin_handle** out);
+
+/*
+ * eqlin_backward_dx -- dx = dL/dx from dy, in one fused launch: the forward kernel on
+ * the adjoint operator (the weights were transformed by eqlin_prepare_weights_ex with
+ * EQLIN_PREPARE_BACKWARD).
+ *
+ *   h        handle prepared with EQLIN_PREPARE_BACKWARD.  Not modified.
+ *   dy       device, [N, Cout, G] of the handle's io_dtype, 16-byte aligned.
+ *   dx       device, [N, Cin, G] of io_dtype, 16-byte aligned; written, not
+ *            accumulated; must not overlap dy.
+ *   N        tokens; N == 0 is a no-op.  N < 2^31.
+ *   stream   asynchronous on this stream; allocates nothing.
+ *
+ * Errors: INVALID_ARG (null handle/pointers, N < 0, handle prepared without the flag,
+ * wrong current device), MISALIGNED, CUDA.  Kernel wait timeouts go to the device
+ * status word, as for eqlin_forward.
+ */
+EQLIN_API int eqlin_backward_dx(const eqlin_handle* h, const void* dy, void* dx, int64_t N, void* stream);
+
+/*
+ * eqlin_backward_dw_workspace_size -- bytes of device workspace eqlin_backward_dw needs
+ * for N tokens (0 for N == 0).  Host only.  Errors: INVALID_ARG, UNSUPPORTED (no
+ * weight-gradient tiling fits shared memory for this shape).
+ */
+EQLIN_API int eqlin_backward_dw_workspace_size(const eqlin_handle* h, int64_t N, size_t* bytes);
+
+/*
+ * eqlin_backward_dw -- dw = dL/dw and dbias = dL/dbias from x and dy.
+ *
+ *   h          any handle (no flag needed); gives the shape and the io_dtype.
+ *   x          device, [N, Cin, G] of io_dtype, 16-byte aligned (the forward's input).
+ *   dy         device, [N, Cout, G] of io_dtype, 16-byte aligned.
+ *   dw         device, [Cout, Cin, G] float32, written (not accumulated).
+ *   dbias      device, [Cout] float32, written; or NULL (not computed).
+ *   N          tokens; N == 0 writes zeros to dw (and dbias).  N < 2^31.
+ *   workspace  device, at least eqlin_backward_dw_workspace_size(h, N) bytes,
+ *              16-byte aligned, owned by the caller.  Its contents on entry do not
+ *              matter and on exit are unspecified.  Two calls whose work overlaps on
+ *              the GPU must not share it.
+ *   stream     asynchronous on this stream: 2 launches for bf16 (the tcgen05
+ *              contraction with a per-CTA partial sum, then a deterministic
+ *              reduction and inverse DFT); for fp32, a clear, a float64 CUDA-core
+ *              kernel and a conversion.  Allocates nothing.
+ *
+ * bf16: the spectra are rounded to bf16 for the tensor cores and accumulated in fp32;
+ * the partial sums are reduced in float64 in a fixed order, so repeated calls give
+ * identical results.  fp32: float64 arithmetic throughout (the order of the float64
+ * additions across token slices may vary).
+ * Errors: INVALID_ARG (null handle/dw, N < 0, null x/dy with N > 0, workspace missing or
+ * too small, wrong device), MISALIGNED, UNSUPPORTED, CUDA.  Kernel wait timeouts go to
+ * the device status word.
+ */
+EQLIN_API int eqlin_backward_dw(const eqlin_handle* h, const void* x, const void* dy, float* dw, float* dbias,
+                                int64_t N, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Static description of a status code ("ok", "invalid argument", ...). */
 EQLIN_API const char* eqlin_status_string(int status);

@@ -110,3 +110,25 @@ def test_header_matches_binding_constants():
         assert name in text
     for attr, code in eq.ATTRS.items():
         assert f"= {code}" in text
+
+
+def test_backward_entry_points_reject_bad_arguments_on_host():
+    lib = eq.library()
+    assert lib.eqlin_backward_dx(None, 16, 16, 4, None) == eq.EQLIN_ERR_INVALID_ARG
+    n = ctypes.c_size_t()
+    assert lib.eqlin_backward_dw_workspace_size(None, 4, ctypes.byref(n)) == eq.EQLIN_ERR_INVALID_ARG
+    assert lib.eqlin_backward_dw(None, 16, 16, 16, None, 4, 16, 1 << 20, None) == eq.EQLIN_ERR_INVALID_ARG
+    h = ctypes.c_void_p(1234)
+    # unknown flag bits are rejected before anything else is looked at
+    st = lib.eqlin_prepare_weights_ex(16, None, 8, 8, 4, eq.EQLIN_BF16, eq.EQLIN_BF16, 0x80, None,
+                                      ctypes.byref(h))
+    assert st == eq.EQLIN_ERR_INVALID_ARG and h.value is None
+    assert "flag" in eq.eqlin_last_error()
+    st = lib.eqlin_prepare_weights_ex(None, None, 8, 8, 4, eq.EQLIN_BF16, eq.EQLIN_BF16,
+                                      eq.EQLIN_PREPARE_BACKWARD, None, ctypes.byref(h))
+    assert st == eq.EQLIN_ERR_INVALID_ARG
+
+
+def test_header_declares_the_backward_flag():
+    text = open(_capi.HEADER_PATH).read()
+    assert f"#define EQLIN_PREPARE_BACKWARD {eq.EQLIN_PREPARE_BACKWARD}u" in text
