@@ -9,6 +9,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <cstdio>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -61,6 +62,7 @@ struct Plan {
     int TG = 0;          // y TMA store box rows (tokens-on-N)
     int ybufs = 0;       // y staging buffers per epilogue warp (tokens-on-N)
     int box_elems = 0;   // x TMA box columns
+    bool x_swizzle128 = false;  // x boxes land SWIZZLE_128B (tokens-on-M, G >= 8)
     uint32_t w_region_bytes = 0, w_img_bytes = 0, ystage_bytes = 0;
     size_t smem_bytes = 0;
     size_t img_alloc_bytes = 0;
@@ -151,10 +153,11 @@ int plan_tm_g(int64_t Cout, int64_t Cin, size_t max_smem, Plan* pl) {
     pl->nK = static_cast<int>((Cin + eqlin::kChunkK16 - 1) / eqlin::kChunkK16);
     pl->n_oc = static_cast<int>((Cout + no - 1) / no);
     pl->BN = eqlin::tm::kM;
-    pl->box_elems = C::XROW_ELEMS;
+    pl->box_elems = C::X_BOX;
+    pl->x_swizzle128 = C::X_SW128;
     const size_t wchunk = static_cast<size_t>(G) * no * eqlin::kRowBytes32;   // one (oc, c) weight chunk
     const size_t fixed = kSmemAlignSlack + kSmemCtlBytes +
-                         static_cast<size_t>(eqlin::tm::kYBufs) * eqlin::tm::kYBufBytes;
+                         static_cast<size_t>(eqlin::tm::kYStageBytes);
     if (pl->n_oc == 1) {
         const size_t img = wchunk * pl->nK;
         const size_t region = (img + 1023) / 1024 * 1024;
@@ -427,7 +430,8 @@ int launch_forward(const Plan& pl, int64_t Cout, int64_t Cin, int64_t G, int sm_
         cuuint64_t strides[1] = {static_cast<cuuint64_t>(Cin * G * 2)};
         cuuint32_t boxdim[2] = {static_cast<cuuint32_t>(pl.box_elems), static_cast<cuuint32_t>(pl.BN)};
         CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, boxdim,
-                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            pl.x_swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return fail(EQLIN_ERR_CUDA, "cuTensorMapEncodeTiled failed for x");
         cuuint64_t ydims[2] = {static_cast<cuuint64_t>(Cout * G), static_cast<cuuint64_t>(N)};
@@ -436,7 +440,7 @@ int launch_forward(const Plan& pl, int64_t Cout, int64_t Cin, int64_t G, int sm_
         CUtensorMapSwizzle yswz;
         if (pl.tm()) {
             ybox[0] = eqlin::tm::kYCols;
-            ybox[1] = eqlin::tm::kM;
+            ybox[1] = eqlin::tm::kYRows;
             yswz = CU_TENSOR_MAP_SWIZZLE_64B;
         } else {
             ybox[0] = static_cast<cuuint32_t>(std::min<int64_t>(32 * G, eqlin::tc::kYBoxCols2));
@@ -502,6 +506,7 @@ int launch_forward(const Plan& pl, int64_t Cout, int64_t Cin, int64_t G, int sm_
 struct DwPlan {
     int MO = 0, NI = 0, n_ot = 0, n_it = 0, max_splits = 0;
     int cpb_dy = 0, cpb_x = 0;
+    int raw_stages = 0, spec_bufs = 0;
     uint32_t dy_bytes = 0, raw_bytes = 0, a_bytes = 0, b_bytes = 0, tmem_cols = 0;
     size_t smem_bytes = 0, slab_floats = 0;
     int units() const { return n_ot * n_it; }
@@ -518,24 +523,30 @@ int box_channels(int C, int G) {
     return 0;
 }
 
-size_t dw_smem(int MO, int NI, int G, DwPlan* out) {
+size_t dw_smem(int MO, int NI, int G, int RS, int SB, DwPlan* out) {
     const size_t raw = round_kb(static_cast<size_t>(eqlin::dw::kTok) * (MO + NI) * G * 2);
     const size_t a = round_kb(static_cast<size_t>(G * MO + (eqlin::kMmaM - MO)) * eqlin::kPlaneRowBytes);
     const size_t b = round_kb(static_cast<size_t>(G) * NI * eqlin::kPlaneRowBytes);
-    const size_t total = kSmemAlignSlack + eqlin::dw::kRawStages * raw + eqlin::dw::kSpecBufs * (a + b) +
+    const size_t total = kSmemAlignSlack + static_cast<size_t>(RS) * raw + static_cast<size_t>(SB) * (a + b) +
                          static_cast<size_t>(4 * MO) * 4 + 256;
     if (out) {
         out->dy_bytes = static_cast<uint32_t>(eqlin::dw::kTok) * MO * G * 2;
         out->raw_bytes = static_cast<uint32_t>(raw);
         out->a_bytes = static_cast<uint32_t>(a);
         out->b_bytes = static_cast<uint32_t>(b);
+        out->raw_stages = RS;
+        out->spec_bufs = SB;
         out->smem_bytes = total;
     }
     return total;
 }
 
-// Pick the tile with the fewest units that fits shared memory (fewer units = fewer
-// re-reads of x and dy); ties go to the larger MO (less MMA padding), then larger NI.
+// Pick the tile with the fewest units that fits shared memory with the minimum
+// pipeline (2 raw stages, 1 spectra buffer); fewer units = fewer re-reads of x and dy.
+// Ties go to the larger MO (less MMA padding), then the larger NI.  Then the deepest
+// raw ring that fits: with two spectra buffers (the transform of one chunk overlaps the
+// MMAs of the previous one) when that still leaves >= 2 raw stages, else with one.  Tuning overrides: EQLIN_DW_TILE ("MO,NI"), EQLIN_DW_SPEC_BUFS,
+// EQLIN_DW_RAW_STAGES.
 int plan_dw(int64_t Cout, int64_t Cin, int G, size_t max_smem, int sm_count, DwPlan* pl) {
     const int mo_max = std::min(eqlin::kMmaM, round16(Cout));
     const int ni_cap = std::min(256, (512 / G) / 16 * 16);
@@ -544,7 +555,7 @@ int plan_dw(int64_t Cout, int64_t Cin, int G, size_t max_smem, int sm_count, DwP
     int best_mo = 0, best_ni = 0;
     for (int mo = mo_max; mo >= 16; mo -= 16) {
         for (int ni = ni_max; ni >= 16; ni -= 16) {
-            if (dw_smem(mo, ni, G, nullptr) > max_smem) continue;
+            if (dw_smem(mo, ni, G, 2, 1, nullptr) > max_smem) continue;
             const long long units = ((Cout + mo - 1) / mo) * ((Cin + ni - 1) / ni);
             if (best_units < 0 || units < best_units) {
                 best_units = units;
@@ -554,6 +565,25 @@ int plan_dw(int64_t Cout, int64_t Cin, int G, size_t max_smem, int sm_count, DwP
         }
     }
     if (best_units < 0) return fail(EQLIN_ERR_UNSUPPORTED, "no weight-gradient tile fits shared memory");
+    if (const char* e = std::getenv("EQLIN_DW_TILE")) {  // "MO,NI" tuning override
+        int mo = 0, ni = 0;
+        if (std::sscanf(e, "%d,%d", &mo, &ni) == 2 && mo >= 16 && mo <= mo_max && mo % 16 == 0 && ni >= 16 &&
+            ni <= ni_max && ni % 16 == 0 && dw_smem(mo, ni, G, 2, 1, nullptr) <= max_smem) {
+            best_mo = mo;
+            best_ni = ni;
+        }
+    }
+    auto max_rs = [&](int sb) {
+        int rs = 0;
+        while (rs < eqlin::dw::kMaxRawStages && dw_smem(best_mo, best_ni, G, rs + 1, sb, nullptr) <= max_smem) ++rs;
+        return rs;
+    };
+    int sb = max_rs(2) >= 2 ? 2 : 1;
+    const int sb_env = env_int("EQLIN_DW_SPEC_BUFS", 0);
+    if (sb_env == 1 || (sb_env == 2 && max_rs(2) >= 2)) sb = sb_env;
+    int rs = max_rs(sb);
+    const int rs_env = env_int("EQLIN_DW_RAW_STAGES", 0);
+    if (rs_env >= 2 && rs_env < rs) rs = rs_env;
     pl->MO = best_mo;
     pl->NI = best_ni;
     pl->n_ot = static_cast<int>((Cout + best_mo - 1) / best_mo);
@@ -561,7 +591,7 @@ int plan_dw(int64_t Cout, int64_t Cin, int G, size_t max_smem, int sm_count, DwP
     pl->max_splits = std::max(1, sm_count / pl->units());
     pl->cpb_dy = box_channels(best_mo, G);
     pl->cpb_x = box_channels(best_ni, G);
-    dw_smem(best_mo, best_ni, G, pl);
+    dw_smem(best_mo, best_ni, G, rs, sb, pl);
     int cols = 32;
     while (cols < G * best_ni) cols *= 2;
     pl->tmem_cols = static_cast<uint32_t>(cols);
@@ -660,6 +690,8 @@ int launch_dw(const DwPlan& pl, bool f32_path, int64_t Cout, int64_t Cin, int64_
     p.a_bytes = pl.a_bytes;
     p.b_bytes = pl.b_bytes;
     p.tmem_cols = pl.tmem_cols;
+    p.raw_stages = pl.raw_stages;
+    p.spec_bufs = pl.spec_bufs;
     p.slab_floats = pl.slab_floats;
     const unsigned grid = static_cast<unsigned>(pl.units() * p.n_splits);
     p.bias_offset = static_cast<size_t>(grid) * pl.slab_floats;

@@ -18,7 +18,8 @@
 // (MO-row output tile, NI-column input tile) pair; each CTA owns one unit and a
 // contiguous range of 32-token chunks, and keeps its partial dW in TMEM:
 //   warp 0      TMA producer: per chunk the dy tile [32 tokens x MO*G] and the x tile
-//               [32 tokens x NI*G] into a 2-stage raw ring (zero fill past N, Cout, Cin).
+//               [32 tokens x NI*G] into a raw ring of p.raw_stages stages (zero fill past
+//               N, Cout, Cin).
 //   warp 1      MMA issuer + TMEM owner: per chunk and 16-token K step, tcgen05.mma with
 //               A = DY^ plane [128 rows (MO valid) x 16 tokens], B = X^ plane [NI x 16],
 //               D plane in TMEM (lane = o, column = i):
@@ -26,12 +27,13 @@
 //                 Re: D_2k   += DYr Xr + DYi Xi,   Im: D_2k+1 += DYi Xr - DYr Xi
 //               (the minus through the descriptor's negate-A bit).
 //   warps 2-9   transpose + DFT: a unit of work is one channel x 8 tokens; the thread
-//               loads the 8 tokens' G-vectors (lanes = 32 consecutive channels, so the
-//               loads are contiguous), runs the real DFT over G in fp32 registers, packs
+//               loads the 8 tokens' G-vectors of all its units of the chunk first (lanes =
+//               32 consecutive channels, so the loads are contiguous), then runs the real
+//               DFT over G in fp32 registers (token pairs packed as fx2), packs
 //               each plane's 8 values to bf16 and writes one 16-byte piece per plane
 //               into the K-major SWIZZLE_64B spectra (row = channel, 64-byte row = the
 //               chunk's 32 tokens).  The dy threads also sum plane 0 (the group sum) for
-//               dbias, in a fixed order.  Spectra are double-buffered.
+//               dbias, in a fixed order.  Spectra use p.spec_bufs buffers.
 //               After the last chunk the same warps read the TMEM partial dW and write it
 //               to the CTA's slab of the workspace.
 // eqlin_dw_finalize_kernel<G> then sums the slabs of each unit over its token splits
@@ -66,6 +68,8 @@ struct DwParams {
     uint32_t a_bytes;          // A (dy spectra) region of one spectra buffer (multiple of 1 KB)
     uint32_t b_bytes;          // B (x spectra) region (multiple of 1 KB)
     uint32_t tmem_cols;        // power of two >= G * NI
+    int raw_stages;            // depth of the raw ring (2 .. kMaxRawStages)
+    int spec_bufs;             // spectra buffers (1 or 2)
     size_t slab_floats;        // G * NI * MO
     size_t bias_offset;        // float offset of the bias partials: gridDim.x * slab_floats
     unsigned long long timeout_ns;
@@ -74,8 +78,8 @@ struct DwParams {
 namespace dw {
 
 constexpr int kTok = 32;           // tokens per chunk (one 64-byte K-major row)
-constexpr int kRawStages = 2;
-constexpr int kSpecBufs = 2;
+constexpr int kMaxRawStages = 8;   // raw ring depth is a launch parameter (p.raw_stages)
+constexpr int kMaxSpecBufs = 2;
 constexpr int kDftWarps = 8;
 constexpr int kDftThreads = kDftWarps * 32;
 constexpr int kWarpProducer = 0;
@@ -125,71 +129,62 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// G bf16 values (one token's group vector of one channel) -> fp32.
+// One unit of the transform: one channel (of the dy tile or of the x tile) x 8 tokens
+// (token group tg of the chunk).  Raw tile layout: boxes of cpb channels, each
+// [32 tokens][cpb*G] bf16.  A thread first loads all of its units of a chunk (load_unit,
+// G/2 words per token) and then transforms and stores them (store_unit), so the shared
+// memory latency of the loads overlaps.
 template <int G>
-__device__ __forceinline__ void load_group(const uint8_t* src, float (&v)[G]) {
-    if constexpr (G == 2) {
-        const uint32_t u = *reinterpret_cast<const uint32_t*>(src);
-        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u));
-        v[0] = f.x;
-        v[1] = f.y;
-    } else if constexpr (G == 4) {
-        const uint2 u = *reinterpret_cast<const uint2*>(src);
-        const uint32_t w[2] = {u.x, u.y};
+struct UnitWords {
+    uint32_t w[8][G / 2];
+};
+
+template <int G>
+__device__ __forceinline__ void load_unit(const uint8_t* src, int row_bytes, UnitWords<G>& u) {
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
-            v[2 * j] = f.x;
-            v[2 * j + 1] = f.y;
-        }
-    } else {
+    for (int j = 0; j < 8; ++j) {
+        const uint8_t* q = src + j * row_bytes;
+        if constexpr (G == 2) {
+            u.w[j][0] = *reinterpret_cast<const uint32_t*>(q);
+        } else if constexpr (G == 4) {
+            const uint2 v = *reinterpret_cast<const uint2*>(q);
+            u.w[j][0] = v.x;
+            u.w[j][1] = v.y;
+        } else {
 #pragma unroll
-        for (int q = 0; q < G / 8; ++q) {
-            const uint4 u = *reinterpret_cast<const uint4*>(src + 16 * q);
-            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
-                v[8 * q + 2 * j] = f.x;
-                v[8 * q + 2 * j + 1] = f.y;
+            for (int c = 0; c < G / 8; ++c) {
+                const uint4 v = *reinterpret_cast<const uint4*>(q + 16 * c);
+                u.w[j][4 * c + 0] = v.x;
+                u.w[j][4 * c + 1] = v.y;
+                u.w[j][4 * c + 2] = v.z;
+                u.w[j][4 * c + 3] = v.w;
             }
         }
     }
 }
 
+// Real DFT over G of the unit's 8 tokens (token pairs packed as fx2), bf16 planes to
+// `spec`: plane p of channel c at row r = p*rows_per_plane + c, 16-byte piece tg of the
+// 64-byte row, SWIZZLE_64B (piece j of row r at j ^ ((r >> 1) & 3)).  Returns the sum of
+// plane 0 (the group sums) over the 8 tokens.
 template <int G>
-__device__ __forceinline__ void planes_of(const float (&v)[G], float (&p)[G]) {
-    if constexpr (G == 2) {
-        p[0] = v[0] + v[1];
-        p[1] = v[0] - v[1];
-    } else {
-        rdft_planes<G, float>(v, p);
-    }
-}
-
-// One unit: channel c of the dy tile (is_dy) or of the x tile, tokens 8*tg .. 8*tg+7
-// of the chunk.  Raw tile layout: boxes of cpb channels, each [32 tokens][cpb*G] bf16.
-// Output: plane p of the channel at row r = p*rows_per_plane + c of `spec`, 16-byte
-// piece tg of the 64-byte row, SWIZZLE_64B (piece j of row r at j ^ ((r >> 1) & 3)).
-template <int G>
-__device__ __forceinline__ float transform_unit(const uint8_t* raw, int cpb, int c, int tg, uint8_t* spec,
-                                                int rows_per_plane) {
-    const int box = c / cpb, cc = c - box * cpb;
-    const int row_bytes = cpb * G * 2;
-    const uint8_t* src = raw + static_cast<size_t>(box) * (kTok * row_bytes) +
-                         static_cast<size_t>(tg * 8) * row_bytes + cc * G * 2;
+__device__ __forceinline__ float store_unit(const UnitWords<G>& u, uint8_t* spec, int rows_per_plane, int c,
+                                            int tg) {
     uint32_t packed[G][4];
     float s0 = 0.0f;
 #pragma unroll
     for (int jp = 0; jp < 4; ++jp) {
-        float va[G], vb[G], pa[G], pb[G];
-        load_group<G>(src + (2 * jp) * row_bytes, va);
-        load_group<G>(src + (2 * jp + 1) * row_bytes, vb);
-        planes_of<G>(va, pa);
-        planes_of<G>(vb, pb);
-        s0 += pa[0] + pb[0];
+        fx2 v[G], pl[G];
 #pragma unroll
-        for (int p = 0; p < G; ++p) packed[p][jp] = pack2(pa[p], pb[p]);
+        for (int h = 0; h < G / 2; ++h) {
+            const uint32_t a = u.w[2 * jp][h], b = u.w[2 * jp + 1][h];
+            v[2 * h] = fx2(__uint_as_float(a << 16), __uint_as_float(b << 16));
+            v[2 * h + 1] = fx2(__uint_as_float(a & 0xFFFF0000u), __uint_as_float(b & 0xFFFF0000u));
+        }
+        rdft_planes<G>(v, pl);
+        s0 += pl[0].x + pl[0].y;
+#pragma unroll
+        for (int p = 0; p < G; ++p) packed[p][jp] = pack2(pl[p].x, pl[p].y);
     }
 #pragma unroll
     for (int p = 0; p < G; ++p) {
@@ -198,6 +193,12 @@ __device__ __forceinline__ float transform_unit(const uint8_t* raw, int cpb, int
         *reinterpret_cast<uint4*>(dst) = make_uint4(packed[p][0], packed[p][1], packed[p][2], packed[p][3]);
     }
     return s0;
+}
+
+// units a transform thread batches per pass (bounded by the registers of UnitWords)
+template <int G>
+constexpr int units_per_pass() {
+    return G <= 4 ? 4 : (G == 8 ? 2 : 1);
 }
 
 }  // namespace dw
@@ -210,20 +211,21 @@ __global__ void __launch_bounds__(dw::kThreads, 1)
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t spec_bytes = p.a_bytes + p.b_bytes;
     uint8_t* raw0 = base;
-    uint8_t* spec0 = raw0 + dw::kRawStages * p.raw_bytes;
-    float* bias_sm = reinterpret_cast<float*>(spec0 + dw::kSpecBufs * spec_bytes);
+    uint8_t* spec0 = raw0 + p.raw_stages * p.raw_bytes;
+    float* bias_sm = reinterpret_cast<float*>(spec0 + p.spec_bufs * spec_bytes);
     // bias_sm[tg][c]: group sums of dy channel c over token group tg of every chunk; each
     // slot has a single writer (the unit -> thread map is the same for every chunk), so
     // the per-CTA sums are formed in a fixed order
     uint64_t* bars = reinterpret_cast<uint64_t*>(bias_sm + 4 * p.MO);
-    dw::Ctl* ctl = reinterpret_cast<dw::Ctl*>(bars + 2 * dw::kRawStages + 2 * dw::kSpecBufs + 2);
+    const int RS = p.raw_stages, SB = p.spec_bufs;
+    dw::Ctl* ctl = reinterpret_cast<dw::Ctl*>(bars + 2 * RS + 2 * SB + 2);
 
     auto bar_raw_full = [&](int s) { return ptx::smem_u32(bars + s); };
-    auto bar_raw_empty = [&](int s) { return ptx::smem_u32(bars + dw::kRawStages + s); };
-    auto bar_spec_full = [&](int s) { return ptx::smem_u32(bars + 2 * dw::kRawStages + s); };
-    auto bar_spec_empty = [&](int s) { return ptx::smem_u32(bars + 2 * dw::kRawStages + dw::kSpecBufs + s); };
-    const uint32_t bar_acc_full = ptx::smem_u32(bars + 2 * dw::kRawStages + 2 * dw::kSpecBufs);
-    const uint32_t bar_drain = ptx::smem_u32(bars + 2 * dw::kRawStages + 2 * dw::kSpecBufs + 1);
+    auto bar_raw_empty = [&](int s) { return ptx::smem_u32(bars + RS + s); };
+    auto bar_spec_full = [&](int s) { return ptx::smem_u32(bars + 2 * RS + s); };
+    auto bar_spec_empty = [&](int s) { return ptx::smem_u32(bars + 2 * RS + SB + s); };
+    const uint32_t bar_acc_full = ptx::smem_u32(bars + 2 * RS + 2 * SB);
+    const uint32_t bar_drain = ptx::smem_u32(bars + 2 * RS + 2 * SB + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int unit = blockIdx.x / p.n_splits, split = blockIdx.x - unit * p.n_splits;
@@ -234,11 +236,11 @@ __global__ void __launch_bounds__(dw::kThreads, 1)
     const int n_mine = static_cast<int>(c_end - c_begin);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < dw::kRawStages; ++s) {
+        for (int s = 0; s < RS; ++s) {
             ptx::mbar_init(bar_raw_full(s), 1);
             ptx::mbar_init(bar_raw_empty(s), dw::kDftThreads);
         }
-        for (int s = 0; s < dw::kSpecBufs; ++s) {
+        for (int s = 0; s < SB; ++s) {
             ptx::mbar_init(bar_spec_full(s), dw::kDftThreads);
             ptx::mbar_init(bar_spec_empty(s), 1);
         }
@@ -260,7 +262,7 @@ __global__ void __launch_bounds__(dw::kThreads, 1)
         for (int c = t; c < 4 * p.MO; c += dw::kDftThreads) bias_sm[c] = 0.0f;
         // A-region tail rows (read by the MMA, never written by the transform): zero
         const int tail0 = G * p.MO, tail1 = G * p.MO + (kMmaM - p.MO);
-        for (int b = 0; b < dw::kSpecBufs; ++b) {
+        for (int b = 0; b < SB; ++b) {
             uint8_t* a = spec0 + static_cast<size_t>(b) * spec_bytes;
             for (int idx = tail0 * 4 + t; idx < tail1 * 4; idx += dw::kDftThreads)
                 reinterpret_cast<uint4*>(a)[idx] = make_uint4(0, 0, 0, 0);
@@ -283,8 +285,8 @@ __global__ void __launch_bounds__(dw::kThreads, 1)
             const uint32_t s_raw0 = ptx::smem_u32(raw0);
             int issued = 0;
             for (int j = 0; j < n_mine; ++j) {
-                const int s = j % dw::kRawStages;
-                const uint32_t ph = static_cast<uint32_t>(j / dw::kRawStages) & 1u;
+                const int s = j % RS;
+                const uint32_t ph = static_cast<uint32_t>(j / RS) & 1u;
                 if (!dw::wait_bounded(bar_raw_empty(s), ph ^ 1u, ctl, p.status, p.timeout_ns)) break;
                 const int n0 = static_cast<int>((c_begin + j) * dw::kTok);
                 const uint32_t dst = s_raw0 + s * p.raw_bytes;
@@ -297,9 +299,9 @@ __global__ void __launch_bounds__(dw::kThreads, 1)
                 ++issued;
             }
             // every copy issued must land before the CTA exits
-            for (int s = 0; s < dw::kRawStages && s < issued; ++s) {
-                const int last = ((issued - 1 - s) / dw::kRawStages) * dw::kRawStages + s;
-                dw::drain_wait(bar_raw_full(s), static_cast<uint32_t>(last / dw::kRawStages) & 1u, p.status,
+            for (int s = 0; s < RS && s < issued; ++s) {
+                const int last = ((issued - 1 - s) / RS) * RS + s;
+                dw::drain_wait(bar_raw_full(s), static_cast<uint32_t>(last / RS) & 1u, p.status,
                                p.timeout_ns);
             }
         }
@@ -313,8 +315,8 @@ __global__ void __launch_bounds__(dw::kThreads, 1)
             const uint32_t b_plane16 = static_cast<uint32_t>(p.NI) * kPlaneRowBytes / 16;
             bool ok = true;
             for (int j = 0; j < n_mine; ++j) {
-                const int sb = j % dw::kSpecBufs;
-                const uint32_t ph = static_cast<uint32_t>(j / dw::kSpecBufs) & 1u;
+                const int sb = j % SB;
+                const uint32_t ph = static_cast<uint32_t>(j / SB) & 1u;
                 if (!dw::wait_bounded(bar_spec_full(sb), ph, ctl, p.status, p.timeout_ns)) {
                     ok = false;
                     break;
@@ -352,9 +354,9 @@ __global__ void __launch_bounds__(dw::kThreads, 1)
         const int n_units = 4 * width;
         bool ok = true;
         for (int j = 0; j < n_mine; ++j) {
-            const int s = j % dw::kRawStages, sb = j % dw::kSpecBufs;
-            const uint32_t ph_raw = static_cast<uint32_t>(j / dw::kRawStages) & 1u;
-            const uint32_t ph_spec = static_cast<uint32_t>(j / dw::kSpecBufs) & 1u;
+            const int s = j % RS, sb = j % SB;
+            const uint32_t ph_raw = static_cast<uint32_t>(j / RS) & 1u;
+            const uint32_t ph_spec = static_cast<uint32_t>(j / SB) & 1u;
             bool got = dw::wait_bounded(bar_raw_full(s), ph_raw, ctl, p.status, p.timeout_ns);
             if (got) got = dw::wait_bounded(bar_spec_empty(sb), ph_spec ^ 1u, ctl, p.status, p.timeout_ns);
             if (!ptx::named_bar_and(dw::kBarDft, dw::kDftThreads, got)) {
@@ -363,12 +365,36 @@ __global__ void __launch_bounds__(dw::kThreads, 1)
             }
             const uint8_t* raw = raw0 + static_cast<size_t>(s) * p.raw_bytes;
             uint8_t* spec = spec0 + static_cast<size_t>(sb) * spec_bytes;
-            for (int u = t; u < n_units; u += dw::kDftThreads) {
-                const int tg = u / width, ch = u - tg * width;
-                if (ch < p.MO) {
-                    bias_sm[tg * p.MO + ch] += dw::transform_unit<G>(raw, p.cpb_dy, ch, tg, spec, p.MO);
-                } else {
-                    dw::transform_unit<G>(raw + p.dy_bytes, p.cpb_x, ch - p.MO, tg, spec + p.a_bytes, p.NI);
+            constexpr int UPT = dw::units_per_pass<G>();
+            for (int base = 0; base < n_units; base += dw::kDftThreads * UPT) {
+                dw::UnitWords<G> words[UPT];
+                int chs[UPT], tgs[UPT];
+#pragma unroll
+                for (int k = 0; k < UPT; ++k) {
+                    const int u = base + t + k * dw::kDftThreads;
+                    tgs[k] = -1;
+                    chs[k] = 0;
+                    if (u < n_units) {
+                        const int tg = u / width, ch = u - tg * width;
+                        const bool is_dy = ch < p.MO;
+                        const int c = is_dy ? ch : ch - p.MO, cpb = is_dy ? p.cpb_dy : p.cpb_x;
+                        const int box = c / cpb, row_bytes = cpb * G * 2;
+                        const uint8_t* src = raw + (is_dy ? 0u : p.dy_bytes) +
+                                             static_cast<size_t>(box) * (dw::kTok * row_bytes) +
+                                             static_cast<size_t>(tg * 8) * row_bytes + (c - box * cpb) * G * 2;
+                        dw::load_unit<G>(src, row_bytes, words[k]);
+                        tgs[k] = tg;
+                        chs[k] = ch;
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < UPT; ++k) {
+                    if (tgs[k] < 0) continue;
+                    if (chs[k] < p.MO) {
+                        bias_sm[tgs[k] * p.MO + chs[k]] += dw::store_unit<G>(words[k], spec, p.MO, chs[k], tgs[k]);
+                    } else {
+                        dw::store_unit<G>(words[k], spec + p.a_bytes, p.NI, chs[k] - p.MO, tgs[k]);
+                    }
                 }
             }
             ptx::fence_proxy_async_smem();

@@ -172,23 +172,22 @@ __device__ __forceinline__ void dft_chunk(uint8_t* xs, int dft_tid) {
 #pragma unroll
     for (int s = 0; s < STEPS; ++s) {
         const int r = row0 + 2 * s;
-        float xa[G], xb[G];
+        // the unit's two channels (a: words 0..G/2-1, b: words G/2..G-1) transformed as
+        // one packed pair
+        fx2 xab[G];
 #pragma unroll
         for (int h = 0; h < G / 2; ++h) {
             const uint32_t ua = w[s][h], ub = w[s][G / 2 + h];
-            xa[2 * h] = __uint_as_float(ua << 16);
-            xa[2 * h + 1] = __uint_as_float(ua & 0xFFFF0000u);
-            xb[2 * h] = __uint_as_float(ub << 16);
-            xb[2 * h + 1] = __uint_as_float(ub & 0xFFFF0000u);
+            xab[2 * h] = fx2(__uint_as_float(ua << 16), __uint_as_float(ub << 16));
+            xab[2 * h + 1] = fx2(__uint_as_float(ua & 0xFFFF0000u), __uint_as_float(ub & 0xFFFF0000u));
         }
-        float pa[G], pb[G];
-        rdft_planes<G>(xa, pa);
-        rdft_planes<G>(xb, pb);
+        fx2 pab[G];
+        rdft_planes<G>(xab, pab);
         const int phys = (chunk ^ ((r >> 1) & 3)) * 16 + in_chunk;   // SWIZZLE_64B
         uint8_t* dst = xs + r * kPlaneRowBytes + phys;
 #pragma unroll
         for (int p = 0; p < G; ++p) {
-            *reinterpret_cast<uint32_t*>(dst + p * S::PLANE_BYTES) = pack_bf16x2(pa[p], pb[p]);
+            *reinterpret_cast<uint32_t*>(dst + p * S::PLANE_BYTES) = pack_bf16x2(pab[p].x, pab[p].y);
         }
     }
 }

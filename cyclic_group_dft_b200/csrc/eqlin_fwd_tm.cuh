@@ -19,9 +19,10 @@
 //   DW DFT warps     in-place real DFT over G: x chunk -> G planes, K-major SWIZZLE_32B
 //   MMA warp         one thread issues tcgen05.mma (2 real + 4 per complex frequency)
 //   8 epilogue warps lane = token; per group of 32/G output channels: tcgen05.ld of the
-//                    G planes, inverse real DFT + bias, bf16, into a SWIZZLE_64B staging
-//                    tile [128 tokens x 32 columns], TMA store (rows past N and columns
-//                    past Cout*G clipped); warps w and w+4 split the output channels
+//                    G planes, inverse real DFT + bias, bf16, into the warp's own
+//                    SWIZZLE_64B staging tile [32 tokens x 32 columns], TMA store by the
+//                    warp (rows past N and columns past Cout*G clipped); warps w and w+4
+//                    split the output channels
 // Waits are bounded as in eqlin_fwd_tc.cuh.
 #pragma once
 
@@ -58,10 +59,11 @@ constexpr int kEpiWarps = 8;
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kBarDft = 1;
 constexpr int kBarEpi = 2;
-constexpr int kBarEpiHalf0 = 3;                  // 3 and 4
 constexpr int kYCols = 32;                       // staged y columns per group (64 B rows)
-constexpr int kYBufBytes = kM * kYCols * 2;      // 8 KB
-constexpr int kYBufs = 4;                        // 2 per epilogue half
+constexpr int kYRows = 32;                       // staged tokens per epilogue warp (TMA box rows)
+constexpr int kYWarpBufBytes = kYRows * kYCols * 2;   // 2 KB, 512-byte aligned
+constexpr int kYWarpBufs = 2;                    // per epilogue warp
+constexpr int kYStageBytes = kEpiWarps * kYWarpBufs * kYWarpBufBytes;   // 32 KB
 
 template <int G>
 struct Cfg {
@@ -73,7 +75,14 @@ struct Cfg {
     static constexpr int kThreads = (kEpiWarps + DW + 2) * 32;
     static constexpr int PLANE_BYTES = kM * kRowBytes32;      // 4 KB
     static constexpr int XCHUNK_BYTES = G * PLANE_BYTES;      // 128 tokens x 16 ch x G x 2
-    static constexpr int XROW_ELEMS = kChunkK16 * G;          // <= 256 (one TMA box)
+    static constexpr int XROW_ELEMS = kChunkK16 * G;          // <= 256 elements per token row
+    // G >= 8: the chunk lands as XROW_ELEMS/64 boxes of [128 rows x 128 B], SWIZZLE_128B,
+    // so the DFT's reads of 4G-byte units (lanes over 4 rows x 8 channel pairs) spread
+    // over all banks; G <= 4: one unswizzled box (its 16-byte units are conflict-free)
+    static constexpr bool X_SW128 = G >= 8;
+    static constexpr int X_BOX = X_SW128 ? 64 : XROW_ELEMS;
+    static constexpr int X_NBOX = XROW_ELEMS / X_BOX;
+    static constexpr int X_BOX_BYTES = kM * X_BOX * 2;
     static constexpr int NMAX = (512 / G) < 256 ? (512 / G) : 256;
     static constexpr int OG = 32 / G;                         // output channels per group
     static_assert(XROW_ELEMS <= 256, "x box");
@@ -97,7 +106,21 @@ __device__ __forceinline__ void dft_chunk(uint8_t* xs, int dft_tid) {
 #pragma unroll
     for (int s = 0; s < STEPS; ++s) {
         const uint8_t* src = src0 + (row0 + s * ROWS_PER_STEP) * (C::XROW_ELEMS * 2);
-        if constexpr (WORDS == 2) {
+        if constexpr (C::X_SW128) {
+            // 16-byte piece c of the unit: logical byte offset pair*4G + 16c in the row,
+            // box off/128, piece (off/16)%8 stored at piece ^ (row % 8)
+            const int r = row0 + s * ROWS_PER_STEP;
+#pragma unroll
+            for (int c = 0; c < WORDS / 4; ++c) {
+                const int off = pair * (4 * G) + 16 * c;
+                const uint8_t* q = xs + (off >> 7) * C::X_BOX_BYTES + r * 128 + ((((off >> 4) & 7) ^ (r & 7)) << 4);
+                const uint4 v = *reinterpret_cast<const uint4*>(q);
+                w[s][4 * c + 0] = v.x;
+                w[s][4 * c + 1] = v.y;
+                w[s][4 * c + 2] = v.z;
+                w[s][4 * c + 3] = v.w;
+            }
+        } else if constexpr (WORDS == 2) {
             const uint2 v = *reinterpret_cast<const uint2*>(src);
             w[s][0] = v.x;
             w[s][1] = v.y;
@@ -117,41 +140,43 @@ __device__ __forceinline__ void dft_chunk(uint8_t* xs, int dft_tid) {
 #pragma unroll
     for (int s = 0; s < STEPS; ++s) {
         const int r = row0 + s * ROWS_PER_STEP;
-        float xa[G], xb[G];
+        // the unit's two channels (a: words 0..G/2-1, b: words G/2..G-1) transformed as
+        // one packed pair
+        fx2 xab[G];
 #pragma unroll
         for (int h = 0; h < G / 2; ++h) {
             const uint32_t ua = w[s][h], ub = w[s][G / 2 + h];
-            xa[2 * h] = __uint_as_float(ua << 16);
-            xa[2 * h + 1] = __uint_as_float(ua & 0xFFFF0000u);
-            xb[2 * h] = __uint_as_float(ub << 16);
-            xb[2 * h + 1] = __uint_as_float(ub & 0xFFFF0000u);
+            xab[2 * h] = fx2(__uint_as_float(ua << 16), __uint_as_float(ub << 16));
+            xab[2 * h + 1] = fx2(__uint_as_float(ua & 0xFFFF0000u), __uint_as_float(ub & 0xFFFF0000u));
         }
-        float pa[G], pb[G];
-        rdft_planes<G>(xa, pa);
-        rdft_planes<G>(xb, pb);
+        fx2 pab[G];
+        rdft_planes<G>(xab, pab);
         const int phys = ((pair >> 2) ^ ((r >> 2) & 1)) * 16 + in_piece;   // SWIZZLE_32B
         uint8_t* dst = xs + r * kRowBytes32 + phys;
 #pragma unroll
         for (int p = 0; p < G; ++p)
-            *reinterpret_cast<uint32_t*>(dst + p * C::PLANE_BYTES) = tc::pack_bf16x2(pa[p], pb[p]);
+            *reinterpret_cast<uint32_t*>(dst + p * C::PLANE_BYTES) = tc::pack_bf16x2(pab[p].x, pab[p].y);
     }
 }
 
 // ------------------------------------------------------------ epilogue role
 // Warp (q, half): tokens 32q..32q+31 (TMEM lane quarter q), output channels
 // [half*NO/2, (half+1)*NO/2) of the work item, in groups of OG = 32/G channels.
-// Arrives on `acc_empty` once its last TMEM load has landed.
+// Per group: tcgen05.ld of the G planes, inverse real DFT + bias (channel pairs packed
+// as fx2), bf16, one 64-byte row per lane into the warp's own SWIZZLE_64B staging tile
+// [32 tokens x 32 columns] (double-buffered), and lane 0 stores it with TMA; the
+// epilogue warps never wait for one another.  Arrives on `acc_empty` once its last TMEM
+// load has landed.
 template <int G>
 __device__ __forceinline__ void epilogue_tile(const TmParams& p, const CUtensorMap* tmap_y, uint32_t tmem,
-                                              int q, int half, int lane, long long n0, int oc, uint8_t* ystage,
-                                              int& ybuf, bool leader, uint32_t acc_empty) {
+                                              int q, int half, int lane, long long n0, int oc, uint8_t* wstage,
+                                              int& ybuf, uint32_t acc_empty) {
     using C = Cfg<G>;
     constexpr int OG = C::OG;
     const int n_groups = (p.NO / 2) / OG;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
-    const uint32_t bar_half = kBarEpiHalf0 + half;
-    const int row = q * 32 + lane;                 // token row inside the tile
-    const int swz = (row >> 1) & 3;                // SWIZZLE_64B of the staging rows
+    const long long row0 = n0 + q * 32;            // first token of this warp's rows
+    const int swz = (lane >> 1) & 3;               // SWIZZLE_64B of the staging rows
 #pragma unroll 1
     for (int g = 0; g < n_groups; ++g) {
         const int o_loc0 = half * (p.NO / 2) + g * OG;
@@ -168,21 +193,26 @@ __device__ __forceinline__ void epilogue_tile(const TmParams& p, const CUtensorM
         const int o0 = oc * p.NO + o_loc0;
         float yv[OG * G];
 #pragma unroll
-        for (int j = 0; j < OG; ++j) {
-            float z[G], y1[G];
+        for (int j = 0; j < OG; j += 2) {
+            fx2 z[G], y2[G];
 #pragma unroll
-            for (int pl = 0; pl < G; ++pl) z[pl] = __uint_as_float(r[pl][j]);
+            for (int pl = 0; pl < G; ++pl) z[pl] = fx2(__uint_as_float(r[pl][j]), __uint_as_float(r[pl][j + 1]));
             const int o = o0 + j;
-            z[0] += (p.bias != nullptr && o < p.Cout) ? __ldg(p.bias + o) : 0.0f;
-            RealIdft<G>::run(z, y1);
+            if (p.bias != nullptr) {
+                z[0] += fx2(o < p.Cout ? __ldg(p.bias + o) : 0.0f, o + 1 < p.Cout ? __ldg(p.bias + o + 1) : 0.0f);
+            }
+            RealIdft<G, fx2>::run(z, y2);
 #pragma unroll
-            for (int gg = 0; gg < G; ++gg) yv[j * G + gg] = y1[gg];
+            for (int gg = 0; gg < G; ++gg) {
+                yv[j * G + gg] = y2[gg].x;
+                yv[(j + 1) * G + gg] = y2[gg].y;
+            }
         }
-        // the buffer was last stored two groups ago: wait until the TMA engine read it
-        if (leader) ptx::bulk_wait_group_read<1>();
-        ptx::named_bar_sync(bar_half, 128);
-        uint8_t* buf = ystage + static_cast<size_t>(ybuf) * kYBufBytes;
-        uint8_t* rowp = buf + row * (kYCols * 2);
+        // this buffer was last stored two groups ago: its TMA read must be complete
+        if (lane == 0) ptx::bulk_wait_group_read<1>();
+        __syncwarp();
+        uint8_t* buf = wstage + static_cast<size_t>(ybuf) * kYWarpBufBytes;
+        uint8_t* rowp = buf + lane * (kYCols * 2);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             *reinterpret_cast<uint4*>(rowp + ((k ^ swz) * 16)) =
@@ -190,11 +220,11 @@ __device__ __forceinline__ void epilogue_tile(const TmParams& p, const CUtensorM
                            tc::pack_bf16x2(yv[8 * k + 4], yv[8 * k + 5]), tc::pack_bf16x2(yv[8 * k + 6], yv[8 * k + 7]));
         }
         ptx::fence_proxy_async_smem();
-        ptx::named_bar_sync(bar_half, 128);
-        if (leader) {
+        __syncwarp();
+        if (lane == 0) {
             // a store only starts inside the tensor; its clipped parts are not written
-            if (n0 < p.N && o0 < p.Cout)
-                ptx::tma_store_2d(tmap_y, ptx::smem_u32(buf), o0 * G, static_cast<int>(n0));
+            if (row0 < p.N && o0 < p.Cout)
+                ptx::tma_store_2d(tmap_y, ptx::smem_u32(buf), o0 * G, static_cast<int>(row0));
             ptx::bulk_commit_group();
         }
         ybuf ^= 1;
@@ -216,7 +246,7 @@ __global__ void __launch_bounds__(tm::Cfg<G>::kThreads, 1)
     const uint32_t stage_bytes = C::XCHUNK_BYTES + wstage_bytes;
     const int NS = p.stages;
     uint8_t* ystage0 = smem + p.w_region_bytes;
-    uint8_t* stage0 = ystage0 + tm::kYBufs * tm::kYBufBytes;
+    uint8_t* stage0 = ystage0 + tm::kYStageBytes;
     uint64_t* bars = reinterpret_cast<uint64_t*>(stage0 + static_cast<size_t>(NS) * stage_bytes);
     tc::Ctl* ctl = reinterpret_cast<tc::Ctl*>(bars + 3 * NS + 4);
 
@@ -284,7 +314,10 @@ __global__ void __launch_bounds__(tm::Cfg<G>::kThreads, 1)
                     }
                     const uint32_t dst = s_stage0 + stage * stage_bytes;
                     ptx::mbar_arrive_expect_tx(bar_full(stage), stage_bytes);
-                    ptx::tma_load_2d(dst, &tmap_x, c * C::XROW_ELEMS, n0, bar_full(stage));
+#pragma unroll
+                    for (int bx = 0; bx < C::X_NBOX; ++bx)
+                        ptx::tma_load_2d(dst + bx * C::X_BOX_BYTES, &tmap_x, c * C::XROW_ELEMS + bx * C::X_BOX, n0,
+                                         bar_full(stage));
                     if constexpr (STREAM_W) {
                         ptx::bulk_load(dst + C::XCHUNK_BYTES,
                                        p.w_img + static_cast<size_t>(oc * p.nK + c) * wstage_bytes, wstage_bytes,
@@ -399,8 +432,7 @@ __global__ void __launch_bounds__(tm::Cfg<G>::kThreads, 1)
     } else {
         // ------------------------------------------------------------ epilogue warps
         const int half = warp >> 2;
-        const bool leader = (warp & 3) == 0 && lane == 0;
-        uint8_t* ystage = ystage0 + static_cast<size_t>(2 * half) * tm::kYBufBytes;
+        uint8_t* wstage = ystage0 + static_cast<size_t>(warp) * tm::kYWarpBufs * tm::kYWarpBufBytes;
         int ybuf = 0;
         int it = 0;
         for (int wk = blockIdx.x; wk < p.n_work; wk += gridDim.x, ++it) {
@@ -410,9 +442,10 @@ __global__ void __launch_bounds__(tm::Cfg<G>::kThreads, 1)
             ptx::tc_fence_after();
             const int tile = wk / p.n_oc, oc = wk % p.n_oc;
             tm::epilogue_tile<G>(p, &tmap_y, tmem_base, warp & 3, half, lane,
-                                 static_cast<long long>(tile) * tm::kM, oc, ystage, ybuf, leader, bar_acc_empty);
+                                 static_cast<long long>(tile) * tm::kM, oc, wstage, ybuf, bar_acc_empty);
         }
-        if (leader) ptx::bulk_wait_group<0>();
+        // the y stores must be complete (not only read) before the CTA exits
+        if (lane == 0) ptx::bulk_wait_group<0>();
     }
 
     ptx::tc_fence_before();

@@ -9,7 +9,8 @@
 // subtractions (section "Especializacion para el Grupo de Rotacion p4"); the
 // recursion below reproduces that: G = 4 costs 8 add/sub forward, 8 inverse.
 //
-// T is float (bf16 path) or double (fp32-I/O path).
+// T is float or fx2 (bf16 path: one or two transforms at a time) or double (fp32-I/O
+// path).
 //
 // Frequency components are kept in "plane order":
 //   plane 0      = Re X_0          (real)
@@ -56,6 +57,32 @@ __host__ __device__ constexpr T sin16(int j) { return cos16<T>(j - 4); }
 
 __device__ __forceinline__ float fma_t(float a, float b, float c) { return fmaf(a, b, c); }
 __device__ __forceinline__ double fma_t(double a, double b, double c) { return fma(a, b, c); }
+
+// Two fp32 lanes carried together, so that two independent transforms (two tokens or
+// two channels) run as one instruction stream on sm_100's packed FP32x2 add, multiply
+// and fused multiply-add (__fadd2_rn, __fmul2_rn, __ffma2_rn).  Each lane rounds
+// exactly as the scalar float operation would, so results are bit-identical to two
+// scalar transforms.
+struct fx2 {
+    float x, y;
+    __host__ __device__ constexpr fx2() : x(0.0f), y(0.0f) {}
+    __host__ __device__ constexpr fx2(double v) : x(static_cast<float>(v)), y(static_cast<float>(v)) {}
+    __host__ __device__ constexpr fx2(float a, float b) : x(a), y(b) {}
+};
+__device__ __forceinline__ float2 as_float2(fx2 a) { return make_float2(a.x, a.y); }
+__device__ __forceinline__ fx2 as_fx2(float2 a) { return fx2(a.x, a.y); }
+__device__ __forceinline__ fx2 operator+(fx2 a, fx2 b) { return as_fx2(__fadd2_rn(as_float2(a), as_float2(b))); }
+__device__ __forceinline__ fx2 operator-(fx2 a) { return fx2(-a.x, -a.y); }
+// a - b as a + b * (-1): the product is exact, so this rounds like a subtraction
+__device__ __forceinline__ fx2 operator-(fx2 a, fx2 b) {
+    return as_fx2(__ffma2_rn(as_float2(b), make_float2(-1.0f, -1.0f), as_float2(a)));
+}
+__device__ __forceinline__ fx2 operator*(fx2 a, fx2 b) { return as_fx2(__fmul2_rn(as_float2(a), as_float2(b))); }
+__device__ __forceinline__ fx2& operator+=(fx2& a, fx2 b) { return a = a + b; }
+__device__ __forceinline__ fx2& operator-=(fx2& a, fx2 b) { return a = a - b; }
+__device__ __forceinline__ fx2 fma_t(fx2 a, fx2 b, fx2 c) {
+    return as_fx2(__ffma2_rn(as_float2(a), as_float2(b), as_float2(c)));
+}
 
 template <int N, class F, int... Is>
 __device__ __forceinline__ void static_for_impl(F&& f, std::integer_sequence<int, Is...>) {
