@@ -599,20 +599,27 @@ int plan_dw(int64_t Cout, int64_t Cin, int G, size_t max_smem, int sm_count, DwP
     return EQLIN_OK;
 }
 
-// Workspace of one weight-gradient call: per CTA a [G][NI][MO] slab plus [MO] bias sums
-// (bf16 path), or a float64 [Cout][Cin][G] + [Cout] accumulator (fp32 path).
-size_t dw_workspace_bytes(const DwPlan& pl, bool f32_path, int64_t Cout, int64_t Cin, int64_t G, int64_t N) {
-    if (f32_path) return static_cast<size_t>(Cout * Cin * G + Cout) * sizeof(double);
+// Workspace of one weight-gradient call.  bf16 path: per CTA an fp32 slab ([G][NI][MO]
+// partial planes, then [MO] bias sums), followed (16-byte aligned) by the per-unit
+// float64 sums of those slabs.  fp32 path: a float64 [Cout][Cin][G] + [Cout] accumulator.
+size_t dw_slab_region_bytes(const DwPlan& pl, int64_t N) {
     const long long n_chunks = (N + eqlin::dw::kTok - 1) / eqlin::dw::kTok;
     const long long splits = std::max<long long>(1, std::min<long long>(pl.max_splits, n_chunks));
     const size_t grid = static_cast<size_t>(pl.units()) * static_cast<size_t>(splits);
-    return grid * (pl.slab_floats + static_cast<size_t>(pl.MO)) * sizeof(float);
+    const size_t bytes = grid * (pl.slab_floats + static_cast<size_t>(pl.MO)) * sizeof(float);
+    return (bytes + 15) / 16 * 16;
+}
+
+size_t dw_workspace_bytes(const DwPlan& pl, bool f32_path, int64_t Cout, int64_t Cin, int64_t G, int64_t N) {
+    if (f32_path) return static_cast<size_t>(Cout * Cin * G + Cout) * sizeof(double);
+    return dw_slab_region_bytes(pl, N) +
+           static_cast<size_t>(pl.units()) * (pl.slab_floats + static_cast<size_t>(pl.MO)) * sizeof(double);
 }
 
 template <int G>
 void dw_launch(unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& mdy, const CUtensorMap& mx,
                const eqlin::DwParams& p) {
-    launch_fused(eqlin::eqlin_dw_tc_kernel<G>, grid, eqlin::dw::kThreads, smem, st, mdy, mx, p);
+    launch_fused(eqlin::eqlin_dw_tc_kernel<G>, grid, eqlin::dw::Cfg<G>::kThreads, smem, st, mdy, mx, p);
 }
 
 void* dw_kernel_for(int G) {
@@ -694,7 +701,6 @@ int launch_dw(const DwPlan& pl, bool f32_path, int64_t Cout, int64_t Cin, int64_
     p.spec_bufs = pl.spec_bufs;
     p.slab_floats = pl.slab_floats;
     const unsigned grid = static_cast<unsigned>(pl.units() * p.n_splits);
-    p.bias_offset = static_cast<size_t>(grid) * pl.slab_floats;
     p.timeout_ns = timeout_ns;
     switch (iG) {
         case 2: dw_launch<2>(grid, pl.smem_bytes, st, mdy, mx, p); break;
@@ -705,6 +711,7 @@ int launch_dw(const DwPlan& pl, bool f32_path, int64_t Cout, int64_t Cin, int64_
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "weight-gradient launch");
     eqlin::DwFinalParams f;
     f.ws = p.ws;
+    f.P = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + dw_slab_region_bytes(pl, N));
     f.dw = dw;
     f.dbias = dbias;
     f.Cout = iCout;
@@ -714,15 +721,17 @@ int launch_dw(const DwPlan& pl, bool f32_path, int64_t Cout, int64_t Cin, int64_
     f.n_it = pl.n_it;
     f.n_splits = p.n_splits;
     f.slab_floats = pl.slab_floats;
-    f.bias_offset = p.bias_offset;
-    const unsigned fgrid = static_cast<unsigned>(pl.units() * pl.NI * ((pl.MO + 31) / 32));
+    const size_t per_unit = (pl.slab_floats + static_cast<size_t>(pl.MO) + 31) / 32;
+    eqlin::eqlin_dw_reduce_kernel<<<static_cast<unsigned>(pl.units() * per_unit), 256, 0, st>>>(f);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "weight-gradient reduction launch");
+    const unsigned igrid = static_cast<unsigned>((Cout * Cin + 255) / 256);
     switch (iG) {
-        case 2: eqlin::eqlin_dw_finalize_kernel<2><<<fgrid, 256, 0, st>>>(f); break;
-        case 4: eqlin::eqlin_dw_finalize_kernel<4><<<fgrid, 256, 0, st>>>(f); break;
-        case 8: eqlin::eqlin_dw_finalize_kernel<8><<<fgrid, 256, 0, st>>>(f); break;
-        default: eqlin::eqlin_dw_finalize_kernel<16><<<fgrid, 256, 0, st>>>(f); break;
+        case 2: eqlin::eqlin_dw_idft_kernel<2><<<igrid, 256, 0, st>>>(f); break;
+        case 4: eqlin::eqlin_dw_idft_kernel<4><<<igrid, 256, 0, st>>>(f); break;
+        case 8: eqlin::eqlin_dw_idft_kernel<8><<<igrid, 256, 0, st>>>(f); break;
+        default: eqlin::eqlin_dw_idft_kernel<16><<<igrid, 256, 0, st>>>(f); break;
     }
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "weight-gradient finalize launch");
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "weight-gradient inverse DFT launch");
     return EQLIN_OK;
 }
 

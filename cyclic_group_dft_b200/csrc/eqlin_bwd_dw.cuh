@@ -26,7 +26,8 @@
 //                 D_0 += DY_0 X_0, D_1 += DY_{G/2} X_{G/2},
 //                 Re: D_2k   += DYr Xr + DYi Xi,   Im: D_2k+1 += DYi Xr - DYr Xi
 //               (the minus through the descriptor's negate-A bit).
-//   warps 2-9   transpose + DFT: a unit of work is one channel x 8 tokens; the thread
+//   warps 2..    transpose + DFT (dw::Cfg<G>::kDftWarps warps): a unit of work is one
+//               channel x 8 tokens; the thread
 //               loads the 8 tokens' G-vectors of all its units of the chunk first (lanes =
 //               32 consecutive channels, so the loads are contiguous), then runs the real
 //               DFT over G in fp32 registers (token pairs packed as fx2), packs
@@ -36,9 +37,9 @@
 //               dbias, in a fixed order.  Spectra use p.spec_bufs buffers.
 //               After the last chunk the same warps read the TMEM partial dW and write it
 //               to the CTA's slab of the workspace.
-// eqlin_dw_finalize_kernel<G> then sums the slabs of each unit over its token splits
-// in a fixed order (deterministic), runs the inverse real DFT over the planes in
-// float64 and writes dw (fp32) and dbias (fp32).
+// eqlin_dw_reduce_kernel then sums the slabs of each unit over its token splits in a
+// fixed order (deterministic, float64) and eqlin_dw_idft_kernel<G> runs the inverse real
+// DFT over the planes in float64 and writes dw (fp32) and dbias (fp32).
 //
 // The dy spectra of plane p start at row p*MO of the A region; an MMA reads 128 rows
 // from there, so rows MO..127 of its D are other planes' data (never read back).  The
@@ -55,7 +56,7 @@
 namespace eqlin {
 
 struct DwParams {
-    float* ws;                 // workspace: per CTA a slab [G][NI][MO] fp32, then per CTA [MO] bias sums
+    float* ws;                 // workspace: per CTA a slab [G][NI][MO] fp32 followed by [MO] bias sums
     int* status;               // device status word (first error wins)
     long long N;
     int MO, NI;                // rows / columns of a unit (multiples of 16; MO <= 128, G*NI <= 512)
@@ -70,8 +71,7 @@ struct DwParams {
     uint32_t tmem_cols;        // power of two >= G * NI
     int raw_stages;            // depth of the raw ring (2 .. kMaxRawStages)
     int spec_bufs;             // spectra buffers (1 or 2)
-    size_t slab_floats;        // G * NI * MO
-    size_t bias_offset;        // float offset of the bias partials: gridDim.x * slab_floats
+    size_t slab_floats;        // G * NI * MO (a CTA's slab holds slab_floats + MO floats)
     unsigned long long timeout_ns;
 };
 
@@ -80,12 +80,20 @@ namespace dw {
 constexpr int kTok = 32;           // tokens per chunk (one 64-byte K-major row)
 constexpr int kMaxRawStages = 8;   // raw ring depth is a launch parameter (p.raw_stages)
 constexpr int kMaxSpecBufs = 2;
-constexpr int kDftWarps = 8;
-constexpr int kDftThreads = kDftWarps * 32;
 constexpr int kWarpProducer = 0;
 constexpr int kWarpMma = 1;
 constexpr int kWarpDft0 = 2;
-constexpr int kThreads = (2 + kDftWarps) * 32;
+
+// Transform warps per CTA: 12 (3 per SM sub-partition, to hide the latency of the
+// short dependent DFT chains) where the units of a chunk fill them and the registers
+// allow; 8 for G = 16 (256 units per chunk at most, and the DFT needs the registers).
+template <int G>
+struct Cfg {
+    static constexpr int kDftWarps = G == 16 ? 8 : 12;
+    static constexpr int kDftThreads = kDftWarps * 32;
+    static constexpr int kThreads = (2 + kDftWarps) * 32;
+    static constexpr int kUnitsPerPass = G >= 8 ? 1 : 2;    // units a thread batches per pass
+};
 constexpr int kBarDft = 1;         // named barrier among the DFT warps
 constexpr uint32_t kWaitSleepNs = 20000;
 
@@ -195,18 +203,13 @@ __device__ __forceinline__ float store_unit(const UnitWords<G>& u, uint8_t* spec
     return s0;
 }
 
-// units a transform thread batches per pass (bounded by the registers of UnitWords)
-template <int G>
-constexpr int units_per_pass() {
-    return G <= 4 ? 4 : (G == 8 ? 2 : 1);
-}
-
 }  // namespace dw
 
 template <int G>
-__global__ void __launch_bounds__(dw::kThreads, 1)
+__global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
     eqlin_dw_tc_kernel(const __grid_constant__ CUtensorMap tmap_dy, const __grid_constant__ CUtensorMap tmap_x,
                        const DwParams p) {
+    constexpr int kDftThreads = dw::Cfg<G>::kDftThreads;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t spec_bytes = p.a_bytes + p.b_bytes;
@@ -238,10 +241,10 @@ __global__ void __launch_bounds__(dw::kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < RS; ++s) {
             ptx::mbar_init(bar_raw_full(s), 1);
-            ptx::mbar_init(bar_raw_empty(s), dw::kDftThreads);
+            ptx::mbar_init(bar_raw_empty(s), kDftThreads);
         }
         for (int s = 0; s < SB; ++s) {
-            ptx::mbar_init(bar_spec_full(s), dw::kDftThreads);
+            ptx::mbar_init(bar_spec_full(s), kDftThreads);
             ptx::mbar_init(bar_spec_empty(s), 1);
         }
         ptx::mbar_init(bar_acc_full, 1);
@@ -259,12 +262,12 @@ __global__ void __launch_bounds__(dw::kThreads, 1)
     }
     if (warp >= dw::kWarpDft0) {
         const int t = threadIdx.x - dw::kWarpDft0 * 32;
-        for (int c = t; c < 4 * p.MO; c += dw::kDftThreads) bias_sm[c] = 0.0f;
+        for (int c = t; c < 4 * p.MO; c += kDftThreads) bias_sm[c] = 0.0f;
         // A-region tail rows (read by the MMA, never written by the transform): zero
         const int tail0 = G * p.MO, tail1 = G * p.MO + (kMmaM - p.MO);
         for (int b = 0; b < SB; ++b) {
             uint8_t* a = spec0 + static_cast<size_t>(b) * spec_bytes;
-            for (int idx = tail0 * 4 + t; idx < tail1 * 4; idx += dw::kDftThreads)
+            for (int idx = tail0 * 4 + t; idx < tail1 * 4; idx += kDftThreads)
                 reinterpret_cast<uint4*>(a)[idx] = make_uint4(0, 0, 0, 0);
         }
         ptx::fence_proxy_async_smem();
@@ -359,19 +362,19 @@ __global__ void __launch_bounds__(dw::kThreads, 1)
             const uint32_t ph_spec = static_cast<uint32_t>(j / SB) & 1u;
             bool got = dw::wait_bounded(bar_raw_full(s), ph_raw, ctl, p.status, p.timeout_ns);
             if (got) got = dw::wait_bounded(bar_spec_empty(sb), ph_spec ^ 1u, ctl, p.status, p.timeout_ns);
-            if (!ptx::named_bar_and(dw::kBarDft, dw::kDftThreads, got)) {
+            if (!ptx::named_bar_and(dw::kBarDft, kDftThreads, got)) {
                 ok = false;
                 break;
             }
             const uint8_t* raw = raw0 + static_cast<size_t>(s) * p.raw_bytes;
             uint8_t* spec = spec0 + static_cast<size_t>(sb) * spec_bytes;
-            constexpr int UPT = dw::units_per_pass<G>();
-            for (int base = 0; base < n_units; base += dw::kDftThreads * UPT) {
+            constexpr int UPT = dw::Cfg<G>::kUnitsPerPass;
+            for (int base = 0; base < n_units; base += kDftThreads * UPT) {
                 dw::UnitWords<G> words[UPT];
                 int chs[UPT], tgs[UPT];
 #pragma unroll
                 for (int k = 0; k < UPT; ++k) {
-                    const int u = base + t + k * dw::kDftThreads;
+                    const int u = base + t + k * kDftThreads;
                     tgs[k] = -1;
                     chs[k] = 0;
                     if (u < n_units) {
@@ -403,14 +406,16 @@ __global__ void __launch_bounds__(dw::kThreads, 1)
         }
         // partial dW: TMEM -> this CTA's workspace slab [G][NI][MO]
         const bool got = ok && dw::wait_bounded(bar_acc_full, 0, ctl, p.status, p.timeout_ns);
-        const bool all = ptx::named_bar_and(dw::kBarDft, dw::kDftThreads, got);
-        float* slab = p.ws + static_cast<size_t>(blockIdx.x) * p.slab_floats;
+        const bool all = ptx::named_bar_and(dw::kBarDft, kDftThreads, got);
+        float* slab = p.ws + static_cast<size_t>(blockIdx.x) * (p.slab_floats + p.MO);
         if (all) {
             ptx::tc_fence_after();
-            const int q = warp & 3, half = (warp - dw::kWarpDft0) >> 2;
+            // the warps of lane quarter q (warp % 4) share its planes round-robin
+            constexpr int kGroups = dw::Cfg<G>::kDftWarps / 4;
+            const int q = warp & 3, grp = (warp - dw::kWarpDft0) >> 2;
             const int row = q * 32 + lane;
             if (q * 32 < p.MO) {
-                for (int pl = half * (G / 2); pl < (half + 1) * (G / 2); ++pl) {
+                for (int pl = grp; pl < G; pl += kGroups) {
                     for (int cb = 0; cb < p.NI; cb += 16) {
                         uint32_t v[16];
                         ptx::tmem_ld_32x32b<16>(tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
@@ -426,11 +431,10 @@ __global__ void __launch_bounds__(dw::kThreads, 1)
                 }
             }
         }
-        // dbias partial of this CTA (every CTA writes it; the finalize reads input tile 0's)
-        ptx::named_bar_sync(dw::kBarDft, dw::kDftThreads);
-        for (int c = t; c < p.MO; c += dw::kDftThreads)
-            p.ws[p.bias_offset + static_cast<size_t>(blockIdx.x) * p.MO + c] =
-                (bias_sm[c] + bias_sm[p.MO + c]) + (bias_sm[2 * p.MO + c] + bias_sm[3 * p.MO + c]);
+        // dbias partial of this CTA (every CTA writes it; the inverse-DFT kernel reads input tile 0's)
+        ptx::named_bar_sync(dw::kBarDft, kDftThreads);
+        for (int c = t; c < p.MO; c += kDftThreads)
+            slab[p.slab_floats + c] = (bias_sm[c] + bias_sm[p.MO + c]) + (bias_sm[2 * p.MO + c] + bias_sm[3 * p.MO + c]);
     }
 
     ptx::tc_fence_before();
@@ -442,63 +446,74 @@ __global__ void __launch_bounds__(dw::kThreads, 1)
     }
 }
 
-// Sums each unit's slabs over its token splits (fixed order), then the inverse real
-// DFT over the planes: with P_k = sum_n DY_k conj(X_k) (unscaled transforms),
-//   dw[o,i,m] = (1/G) [P_0 + (-1)^m P_{G/2} + 2 sum_{0<k<G/2} Re(P_k e^{+2 pi i m k / G})].
-// Block = 32 output rows x one input column of one unit; warp w sums splits w, w+8, ...
+// Cross-CTA reduction, deterministic, in two small kernels:
+//  eqlin_dw_reduce_kernel  P[u][e] = sum over the unit's token splits s (in a fixed
+//                          order) of slab[u * n_splits + s][e], float64, for every slab
+//                          element e (the G planes and the bias sums).  Block = 32
+//                          consecutive elements; warp w sums splits w, w+8, ... with
+//                          several loads in flight; the 8 warp sums are added in order.
+//  eqlin_dw_idft_kernel    per (o, i): the inverse real DFT over the planes.  With
+//                          P_k = sum_n DY_k conj(X_k) (unscaled transforms),
+//   dw[o,i,m] = (1/G) [P_0 + (-1)^m P_{G/2} + 2 sum_{0<k<G/2} Re(P_k e^{+2 pi i m k / G})],
+//                          and dbias[o] from the bias sums of input tile 0.
 struct DwFinalParams {
-    const float* ws;
+    const float* ws;      // slabs: per CTA [G][NI][MO] then [MO]
+    double* P;            // per unit [G][NI][MO] then [MO]
     float* dw;            // [Cout, Cin, G]
     float* dbias;         // [Cout] or nullptr
     int Cout, Cin;
     int MO, NI, n_it, n_splits;
-    size_t slab_floats, bias_offset;
+    size_t slab_floats;   // G * NI * MO
 };
 
-template <int G>
-__global__ void __launch_bounds__(256) eqlin_dw_finalize_kernel(const DwFinalParams f) {
-    __shared__ double red[8][G + 1][32];
-    const int nob = (f.MO + 31) / 32;
-    const int ob = blockIdx.x % nob;
-    const int ii = (blockIdx.x / nob) % f.NI;
-    const int unit = blockIdx.x / (nob * f.NI);
-    const int ot = unit / f.n_it, it = unit - ot * f.n_it;
-    const int i = it * f.NI + ii;
-    if (i >= f.Cin) return;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int oo = ob * 32 + lane;
-    const bool valid = oo < f.MO;
-    const bool with_bias = f.dbias != nullptr && it == 0 && ii == 0;
-    double acc[G + 1];
-#pragma unroll
-    for (int q = 0; q <= G; ++q) acc[q] = 0.0;
-    if (valid) {
-        for (int s = warp; s < f.n_splits; s += 8) {
-            const size_t cta = static_cast<size_t>(unit) * f.n_splits + s;
-            const float* slab = f.ws + cta * f.slab_floats;
-#pragma unroll
-            for (int pl = 0; pl < G; ++pl) acc[pl] += slab[(static_cast<size_t>(pl) * f.NI + ii) * f.MO + oo];
-            if (with_bias) acc[G] += f.ws[f.bias_offset + cta * f.MO + oo];
+__global__ void __launch_bounds__(256) eqlin_dw_reduce_kernel(const DwFinalParams f) {
+    __shared__ double red[8][32];
+    const size_t stride = f.slab_floats + f.MO;
+    const size_t blocks_per_unit = (stride + 31) / 32;
+    const int unit = static_cast<int>(blockIdx.x / blocks_per_unit);
+    const size_t e = (blockIdx.x % blocks_per_unit) * 32 + (threadIdx.x & 31);
+    const int warp = threadIdx.x >> 5;
+    double acc = 0.0;
+    if (e < stride) {
+        const float* src = f.ws + static_cast<size_t>(unit) * f.n_splits * stride + e;
+        int s = warp;
+        for (; s + 24 < f.n_splits; s += 32) {   // four loads in flight, added in split order
+            const float v0 = src[static_cast<size_t>(s) * stride];
+            const float v1 = src[static_cast<size_t>(s + 8) * stride];
+            const float v2 = src[static_cast<size_t>(s + 16) * stride];
+            const float v3 = src[static_cast<size_t>(s + 24) * stride];
+            acc += v0;
+            acc += v1;
+            acc += v2;
+            acc += v3;
         }
+        for (; s < f.n_splits; s += 8) acc += src[static_cast<size_t>(s) * stride];
     }
-#pragma unroll
-    for (int q = 0; q <= G; ++q) red[warp][q][lane] = acc[q];
+    red[warp][threadIdx.x & 31] = acc;
     __syncthreads();
-    if (warp != 0) return;
-    const int o = ot * f.MO + oo;
-    if (!valid || o >= f.Cout) return;
-    double P[G + 1];
-#pragma unroll
-    for (int q = 0; q <= G; ++q) {
+    if (warp == 0 && e < stride) {
         double v = 0.0;
-        for (int w = 0; w < 8; ++w) v += red[w][q][lane];
-        P[q] = v;
-    }
-    double z[G], out[G];
-    z[0] = P[0] / G;
-    z[1] = P[1] / G;
 #pragma unroll
-    for (int q = 2; q < G; ++q) z[q] = 2.0 * P[q] / G;
+        for (int w = 0; w < 8; ++w) v += red[w][threadIdx.x];
+        f.P[static_cast<size_t>(unit) * stride + e] = v;
+    }
+}
+
+template <int G>
+__global__ void __launch_bounds__(256) eqlin_dw_idft_kernel(const DwFinalParams f) {
+    const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx >= static_cast<long long>(f.Cout) * f.Cin) return;
+    const int o = static_cast<int>(idx % f.Cout), i = static_cast<int>(idx / f.Cout);
+    const int ot = o / f.MO, oo = o - ot * f.MO;
+    const int it = i / f.NI, ii = i - it * f.NI;
+    const size_t stride = f.slab_floats + f.MO;
+    const double* P = f.P + static_cast<size_t>(ot * f.n_it + it) * stride;
+    double z[G], out[G];
+#pragma unroll
+    for (int pl = 0; pl < G; ++pl) {
+        const double v = P[(static_cast<size_t>(pl) * f.NI + ii) * f.MO + oo];
+        z[pl] = (pl < 2 ? v : 2.0 * v) / G;
+    }
     if constexpr (G == 2) {
         out[0] = z[0] + z[1];
         out[1] = z[0] - z[1];
@@ -508,7 +523,7 @@ __global__ void __launch_bounds__(256) eqlin_dw_finalize_kernel(const DwFinalPar
     float* dst = f.dw + (static_cast<size_t>(o) * f.Cin + i) * G;
 #pragma unroll
     for (int m = 0; m < G; ++m) dst[m] = static_cast<float>(out[m]);
-    if (with_bias) f.dbias[o] = static_cast<float>(P[G]);
+    if (f.dbias != nullptr && i == 0) f.dbias[o] = static_cast<float>(P[f.slab_floats + oo]);
 }
 
 // ------------------------------------------------------------------ fp32 I/O
