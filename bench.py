@@ -419,7 +419,7 @@ def main() -> None:
         bwd["device_status"] = h.device_status()
         bwd["kernels"] = {"dx": "fused forward kernel on the adjoint operator (1 launch)",
                           "dw": "tcgen05 contraction over tokens + deterministic reduction / inverse DFT "
-                                "(2 launches)" if wl.io_dtype == "bf16" else
+                                "(3 launches)" if wl.io_dtype != "f32" else
                                 "float64 CUDA-core kernel (clear + kernel + convert)"}
         del dxs
 
@@ -480,7 +480,7 @@ def main() -> None:
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16" if wl.io_dtype == "bf16" else "f32",
+        "dtype": wl.io_dtype,
         "data": "synthetic",
         "config": {
             "workload": wl.name, "N": N, "Cin": wl.Cin, "Cout": wl.Cout, "G": wl.G, "io": wl.io_dtype,

@@ -27,6 +27,7 @@ from ._capi import (  # noqa: F401
     EQLIN_ERR_OOM,
     EQLIN_ERR_TIMEOUT,
     EQLIN_ERR_UNSUPPORTED,
+    EQLIN_F16,
     EQLIN_F32,
     EQLIN_OK,
     EQLIN_PREPARE_BACKWARD,

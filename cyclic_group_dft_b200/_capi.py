@@ -18,6 +18,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "eqlin.h")
 
 EQLIN_F32 = 0
 EQLIN_BF16 = 1
+EQLIN_F16 = 2
 
 EQLIN_OK = 0
 EQLIN_ERR_INVALID_ARG = -1
@@ -37,7 +38,7 @@ PATH_NAMES = {0: "tcgen05_tokens_on_n_resident_weights", 1: "tcgen05_tokens_on_n
               2: "fp32_fp64_arithmetic", 3: "tcgen05_tokens_on_m_resident_weights",
               4: "tcgen05_tokens_on_m_streamed_weights"}
 
-_TORCH_TO_EQLIN = {torch.float32: EQLIN_F32, torch.bfloat16: EQLIN_BF16}
+_TORCH_TO_EQLIN = {torch.float32: EQLIN_F32, torch.bfloat16: EQLIN_BF16, torch.float16: EQLIN_F16}
 _EQLIN_TO_TORCH = {v: k for k, v in _TORCH_TO_EQLIN.items()}
 
 if not os.path.exists(LIB_PATH):

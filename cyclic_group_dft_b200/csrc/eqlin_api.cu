@@ -52,6 +52,7 @@ int cuda_fail(cudaError_t e, const char* what) {
 }
 
 struct Plan {
+    int io = EQLIN_BF16; // element type of x and y (EQLIN_BF16, EQLIN_F16 or EQLIN_F32)
     int path = kPathF32;
     int nacc = 2;        // TMEM accumulator buffers (tokens-on-N kernel)
     int nK = 0;          // input-channel chunks
@@ -193,6 +194,7 @@ int plan_tm_g(int64_t Cout, int64_t Cin, size_t max_smem, Plan* pl) {
 bool default_tokens_on_m(int G) { return G >= 8; }
 
 int plan_for(int64_t Cout, int64_t Cin, int64_t G, int io_dtype, size_t max_smem, Plan* pl) {
+    pl->io = io_dtype;
     if (io_dtype == EQLIN_F32) {
         const size_t smem = static_cast<size_t>(eqlin::kF32Tokens) * G * Cin * sizeof(double);
         if (smem > max_smem) return fail(EQLIN_ERR_UNSUPPORTED, "Cin*G too large for the fp32 path");
@@ -230,13 +232,16 @@ int plan_for(int64_t Cout, int64_t Cin, int64_t G, int io_dtype, size_t max_smem
 }
 
 int check_shape_impl(int64_t Cout, int64_t Cin, int64_t G, int w_dtype, int io_dtype) {
-    if (w_dtype != EQLIN_F32 && w_dtype != EQLIN_BF16) return fail(EQLIN_ERR_INVALID_ARG, "unknown w_dtype");
-    if (io_dtype != EQLIN_F32 && io_dtype != EQLIN_BF16) return fail(EQLIN_ERR_INVALID_ARG, "unknown io_dtype");
+    if (w_dtype != EQLIN_F32 && w_dtype != EQLIN_BF16 && w_dtype != EQLIN_F16)
+        return fail(EQLIN_ERR_INVALID_ARG, "unknown w_dtype");
+    if (io_dtype != EQLIN_F32 && io_dtype != EQLIN_BF16 && io_dtype != EQLIN_F16)
+        return fail(EQLIN_ERR_INVALID_ARG, "unknown io_dtype");
     if (Cout <= 0 || Cin <= 0 || G <= 0) return fail(EQLIN_ERR_INVALID_ARG, "sizes must be positive");
     if (G != 2 && G != 4 && G != 8 && G != 16) return fail(EQLIN_ERR_UNSUPPORTED, "G must be 2, 4, 8 or 16");
     if (Cout > kMaxChannels || Cin > kMaxChannels) return fail(EQLIN_ERR_UNSUPPORTED, "channel count above 65536");
-    if (io_dtype == EQLIN_BF16 && ((Cin * G) % 8 != 0 || (Cout * G) % 8 != 0))
-        return fail(EQLIN_ERR_UNSUPPORTED, "bf16 I/O needs Cin*G and Cout*G to be multiples of 8 (16-byte rows)");
+    if (io_dtype != EQLIN_F32 && ((Cin * G) % 8 != 0 || (Cout * G) % 8 != 0))
+        return fail(EQLIN_ERR_UNSUPPORTED,
+                     "16-bit I/O needs Cin*G and Cout*G to be multiples of 8 (16-byte rows)");
     return EQLIN_OK;
 }
 
@@ -288,15 +293,16 @@ void launch_fused(Kernel k, unsigned grid, unsigned threads, size_t smem, cudaSt
     cudaLaunchKernelEx(&cfg, k, mx, my, p);
 }
 
-template <int G, bool STREAM, int NACC>
+template <int G, bool STREAM, int NACC, class T16>
 void tc_launch(unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& mx, const CUtensorMap& my,
                const TcParams& p) {
-    launch_fused(eqlin::eqlin_fwd_tc_kernel<G, STREAM, NACC>, grid, eqlin::tc::kThreads, smem, st, mx, my, p);
+    launch_fused(eqlin::eqlin_fwd_tc_kernel<G, STREAM, NACC, T16>, grid, eqlin::tc::kThreads, smem, st, mx, my, p);
 }
-template <int G, bool STREAM>
+template <int G, bool STREAM, class T16>
 void tm_launch(unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& mx, const CUtensorMap& my,
                const TmParams& p) {
-    launch_fused(eqlin::eqlin_fwd_tm_kernel<G, STREAM>, grid, eqlin::tm::Cfg<G>::kThreads, smem, st, mx, my, p);
+    launch_fused(eqlin::eqlin_fwd_tm_kernel<G, STREAM, T16>, grid, eqlin::tm::Cfg<G>::kThreads, smem, st, mx, my,
+                 p);
 }
 
 struct TcEntry {
@@ -308,37 +314,46 @@ struct TmEntry {
     void* kernel = nullptr;
 };
 
-template <int G, bool STREAM, int NACC>
+template <int G, bool STREAM, int NACC, class T16>
 TcEntry tc_entry() {
-    return {&tc_launch<G, STREAM, NACC>, reinterpret_cast<void*>(&eqlin::eqlin_fwd_tc_kernel<G, STREAM, NACC>)};
+    return {&tc_launch<G, STREAM, NACC, T16>,
+            reinterpret_cast<void*>(&eqlin::eqlin_fwd_tc_kernel<G, STREAM, NACC, T16>)};
 }
-template <int G>
+template <int G, class T16>
 TcEntry tc_entry_g(bool stream, int nacc) {
-    if (stream) return nacc == 1 ? tc_entry<G, true, 1>() : tc_entry<G, true, 2>();
-    return nacc == 1 ? tc_entry<G, false, 1>() : tc_entry<G, false, 2>();
+    if (stream) return nacc == 1 ? tc_entry<G, true, 1, T16>() : tc_entry<G, true, 2, T16>();
+    return nacc == 1 ? tc_entry<G, false, 1, T16>() : tc_entry<G, false, 2, T16>();
 }
-TcEntry tc_entry_for(int G, bool stream, int nacc) {
+template <class T16>
+TcEntry tc_entry_t(int G, bool stream, int nacc) {
     switch (G) {
-        case 2: return tc_entry_g<2>(stream, nacc);
-        case 4: return tc_entry_g<4>(stream, nacc);
-        case 8: return tc_entry_g<8>(stream, nacc);
-        case 16: return tc_entry_g<16>(stream, nacc);
+        case 2: return tc_entry_g<2, T16>(stream, nacc);
+        case 4: return tc_entry_g<4, T16>(stream, nacc);
+        case 8: return tc_entry_g<8, T16>(stream, nacc);
+        case 16: return tc_entry_g<16, T16>(stream, nacc);
         default: return {};
     }
+}
+TcEntry tc_entry_for(int G, bool stream, int nacc, int io) {
+    return io == EQLIN_F16 ? tc_entry_t<__half>(G, stream, nacc) : tc_entry_t<__nv_bfloat16>(G, stream, nacc);
 }
 
-template <int G, bool STREAM>
+template <int G, bool STREAM, class T16>
 TmEntry tm_entry() {
-    return {&tm_launch<G, STREAM>, reinterpret_cast<void*>(&eqlin::eqlin_fwd_tm_kernel<G, STREAM>)};
+    return {&tm_launch<G, STREAM, T16>, reinterpret_cast<void*>(&eqlin::eqlin_fwd_tm_kernel<G, STREAM, T16>)};
 }
-TmEntry tm_entry_for(int G, bool stream) {
+template <class T16>
+TmEntry tm_entry_t(int G, bool stream) {
     switch (G) {
-        case 2: return stream ? tm_entry<2, true>() : tm_entry<2, false>();
-        case 4: return stream ? tm_entry<4, true>() : tm_entry<4, false>();
-        case 8: return stream ? tm_entry<8, true>() : tm_entry<8, false>();
-        case 16: return stream ? tm_entry<16, true>() : tm_entry<16, false>();
+        case 2: return stream ? tm_entry<2, true, T16>() : tm_entry<2, false, T16>();
+        case 4: return stream ? tm_entry<4, true, T16>() : tm_entry<4, false, T16>();
+        case 8: return stream ? tm_entry<8, true, T16>() : tm_entry<8, false, T16>();
+        case 16: return stream ? tm_entry<16, true, T16>() : tm_entry<16, false, T16>();
         default: return {};
     }
+}
+TmEntry tm_entry_for(int G, bool stream, int io) {
+    return io == EQLIN_F16 ? tm_entry_t<__half>(G, stream) : tm_entry_t<__nv_bfloat16>(G, stream);
 }
 
 void* f32_kernel_for(int G) {
@@ -353,8 +368,8 @@ void* f32_kernel_for(int G) {
 
 void* kernel_for(const Plan& pl, int G) {
     if (pl.path == kPathF32) return f32_kernel_for(G);
-    if (pl.tm()) return tm_entry_for(G, pl.streamed()).kernel;
-    return tc_entry_for(G, pl.streamed(), pl.nacc).kernel;
+    if (pl.tm()) return tm_entry_for(G, pl.streamed(), pl.io).kernel;
+    return tc_entry_for(G, pl.streamed(), pl.nacc, pl.io).kernel;
 }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -383,6 +398,10 @@ int launch_prep(const Plan& pl, int w_dtype, const void* w, const void* bias, in
         eqlin::eqlin_prep_freq_kernel<float><<<blocks, threads, 0, st>>>(
             static_cast<const float*>(w), static_cast<const float*>(bias), iCout, iCin, iG, b.w_f32, b.bias_f32,
             b.w_f64, b.bias_f64, adjoint);
+    } else if (w_dtype == EQLIN_F16) {
+        eqlin::eqlin_prep_freq_kernel<__half><<<blocks, threads, 0, st>>>(
+            static_cast<const __half*>(w), static_cast<const __half*>(bias), iCout, iCin, iG, b.w_f32, b.bias_f32,
+            b.w_f64, b.bias_f64, adjoint);
     } else {
         eqlin::eqlin_prep_freq_kernel<__nv_bfloat16><<<blocks, threads, 0, st>>>(
             static_cast<const __nv_bfloat16*>(w), static_cast<const __nv_bfloat16*>(bias), iCout, iCin, iG,
@@ -393,12 +412,19 @@ int launch_prep(const Plan& pl, int w_dtype, const void* w, const void* bias, in
     if (b.img) {
         const size_t n = pl.img_alloc_bytes / 2;
         const unsigned b2 = static_cast<unsigned>((n + threads - 1) / threads);
-        if (pl.tm()) {
-            eqlin::eqlin_prep_image_k16_kernel<<<b2, threads, 0, st>>>(b.w_f32, iCout, iCin, iG, pl.nK, pl.rows, n,
-                                                                        b.img);
+        const bool f16 = pl.io == EQLIN_F16;
+        if (pl.tm() && f16) {
+            eqlin::eqlin_prep_image_k16_kernel<__half><<<b2, threads, 0, st>>>(b.w_f32, iCout, iCin, iG, pl.nK,
+                                                                                pl.rows, n, b.img);
+        } else if (pl.tm()) {
+            eqlin::eqlin_prep_image_k16_kernel<__nv_bfloat16><<<b2, threads, 0, st>>>(b.w_f32, iCout, iCin, iG,
+                                                                                       pl.nK, pl.rows, n, b.img);
+        } else if (f16) {
+            eqlin::eqlin_prep_image_kernel<__half><<<b2, threads, 0, st>>>(b.w_f32, iCout, iCin, iG, pl.nK, pl.rows,
+                                                                            n, b.img);
         } else {
-            eqlin::eqlin_prep_image_kernel<<<b2, threads, 0, st>>>(b.w_f32, iCout, iCin, iG, pl.nK, pl.rows, n,
-                                                                    b.img);
+            eqlin::eqlin_prep_image_kernel<__nv_bfloat16><<<b2, threads, 0, st>>>(b.w_f32, iCout, iCin, iG, pl.nK,
+                                                                                   pl.rows, n, b.img);
         }
         e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "weight image launch");
@@ -429,7 +455,9 @@ int launch_forward(const Plan& pl, int64_t Cout, int64_t Cin, int64_t G, int sm_
         cuuint64_t dims[2] = {static_cast<cuuint64_t>(Cin * G), static_cast<cuuint64_t>(N)};
         cuuint64_t strides[1] = {static_cast<cuuint64_t>(Cin * G * 2)};
         cuuint32_t boxdim[2] = {static_cast<cuuint32_t>(pl.box_elems), static_cast<cuuint32_t>(pl.BN)};
-        CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, boxdim,
+        const CUtensorMapDataType dt16 =
+            pl.io == EQLIN_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+        CUresult r = encode(&map, dt16, 2, const_cast<void*>(x), dims, strides, boxdim,
                             estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                             pl.x_swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -447,7 +475,7 @@ int launch_forward(const Plan& pl, int64_t Cout, int64_t Cin, int64_t G, int sm_
             ybox[1] = static_cast<cuuint32_t>(pl.TG);
             yswz = CU_TENSOR_MAP_SWIZZLE_NONE;
         }
-        r = encode(&ymap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, ydims, ystrides, ybox, estr,
+        r = encode(&ymap, dt16, 2, y, ydims, ystrides, ybox, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, yswz, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return fail(EQLIN_ERR_CUDA, "cuTensorMapEncodeTiled failed for y");
@@ -469,14 +497,13 @@ int launch_forward(const Plan& pl, int64_t Cout, int64_t Cin, int64_t G, int sm_
             p.w_region_bytes = pl.w_region_bytes;
             p.w_img_bytes = pl.w_img_bytes;
             p.timeout_ns = timeout_ns;
-            const TmEntry entry = tm_entry_for(iG, pl.streamed());
+            const TmEntry entry = tm_entry_for(iG, pl.streamed(), pl.io);
             if (!entry.launch) return fail(EQLIN_ERR_UNSUPPORTED, "G");
             entry.launch(grid, pl.smem_bytes, st, map, ymap, p);
         } else {
             TcParams p;
             p.w_img = b.img;
             p.bias = b.has_bias ? b.bias_f32 : nullptr;
-            p.y = static_cast<__nv_bfloat16*>(y);
             p.status = b.status;
             p.N = N;
             p.Cout = static_cast<int>(Cout);
@@ -490,7 +517,7 @@ int launch_forward(const Plan& pl, int64_t Cout, int64_t Cin, int64_t G, int sm_
             p.ybufs = pl.ybufs;
             p.w_img_bytes = pl.w_img_bytes;
             p.timeout_ns = timeout_ns;
-            const TcEntry entry = tc_entry_for(iG, pl.streamed(), pl.nacc);
+            const TcEntry entry = tc_entry_for(iG, pl.streamed(), pl.nacc, pl.io);
             if (!entry.launch) return fail(EQLIN_ERR_UNSUPPORTED, "G");
             entry.launch(grid, pl.smem_bytes, st, map, ymap, p);
         }
@@ -504,6 +531,7 @@ int launch_forward(const Plan& pl, int64_t Cout, int64_t Cin, int64_t G, int sm_
 // Tiling of the weight-gradient kernel: a unit is an (MO-row, NI-column) tile of the
 // [Cout x Cin] gradient; the grid is units x token splits (see eqlin_bwd_dw.cuh).
 struct DwPlan {
+    int io = EQLIN_BF16;  // 16-bit element type of x and dy
     int MO = 0, NI = 0, n_ot = 0, n_it = 0, max_splits = 0;
     int cpb_dy = 0, cpb_x = 0;
     int raw_stages = 0, spec_bufs = 0;
@@ -616,30 +644,34 @@ size_t dw_workspace_bytes(const DwPlan& pl, bool f32_path, int64_t Cout, int64_t
            static_cast<size_t>(pl.units()) * (pl.slab_floats + static_cast<size_t>(pl.MO)) * sizeof(double);
 }
 
-template <int G>
+template <int G, class T16>
 void dw_launch(unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& mdy, const CUtensorMap& mx,
                const eqlin::DwParams& p) {
-    launch_fused(eqlin::eqlin_dw_tc_kernel<G>, grid, eqlin::dw::Cfg<G>::kThreads, smem, st, mdy, mx, p);
+    launch_fused(eqlin::eqlin_dw_tc_kernel<G, T16>, grid, eqlin::dw::Cfg<G>::kThreads, smem, st, mdy, mx, p);
 }
 
-void* dw_kernel_for(int G) {
+template <class T16>
+void* dw_kernel_t(int G) {
     switch (G) {
-        case 2: return reinterpret_cast<void*>(&eqlin::eqlin_dw_tc_kernel<2>);
-        case 4: return reinterpret_cast<void*>(&eqlin::eqlin_dw_tc_kernel<4>);
-        case 8: return reinterpret_cast<void*>(&eqlin::eqlin_dw_tc_kernel<8>);
-        case 16: return reinterpret_cast<void*>(&eqlin::eqlin_dw_tc_kernel<16>);
+        case 2: return reinterpret_cast<void*>(&eqlin::eqlin_dw_tc_kernel<2, T16>);
+        case 4: return reinterpret_cast<void*>(&eqlin::eqlin_dw_tc_kernel<4, T16>);
+        case 8: return reinterpret_cast<void*>(&eqlin::eqlin_dw_tc_kernel<8, T16>);
+        case 16: return reinterpret_cast<void*>(&eqlin::eqlin_dw_tc_kernel<16, T16>);
         default: return nullptr;
     }
 }
+void* dw_kernel_for(int G, int io) { return io == EQLIN_F16 ? dw_kernel_t<__half>(G) : dw_kernel_t<__nv_bfloat16>(G); }
 
-int encode_rows_map(CUtensorMap* map, const void* base, int64_t cols, int64_t rows, int box_cols, int box_rows) {
+int encode_rows_map(CUtensorMap* map, const void* base, int64_t cols, int64_t rows, int box_cols, int box_rows,
+                    int io) {
     auto encode = tensor_map_encoder();
     if (!encode) return fail(EQLIN_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
     cuuint32_t estr[2] = {1, 1};
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols * 2)};
     cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
-    CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+    CUresult r = encode(map, io == EQLIN_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                        const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(EQLIN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
@@ -677,9 +709,9 @@ int launch_dw(const DwPlan& pl, bool f32_path, int64_t Cout, int64_t Cin, int64_
         return EQLIN_OK;
     }
     CUtensorMap mdy, mx;
-    int s = encode_rows_map(&mdy, dy, Cout * G, N, pl.cpb_dy * iG, eqlin::dw::kTok);
+    int s = encode_rows_map(&mdy, dy, Cout * G, N, pl.cpb_dy * iG, eqlin::dw::kTok, pl.io);
     if (s != EQLIN_OK) return s;
-    s = encode_rows_map(&mx, x, Cin * G, N, pl.cpb_x * iG, eqlin::dw::kTok);
+    s = encode_rows_map(&mx, x, Cin * G, N, pl.cpb_x * iG, eqlin::dw::kTok, pl.io);
     if (s != EQLIN_OK) return s;
     eqlin::DwParams p;
     p.ws = static_cast<float*>(ws);
@@ -703,10 +735,14 @@ int launch_dw(const DwPlan& pl, bool f32_path, int64_t Cout, int64_t Cin, int64_
     const unsigned grid = static_cast<unsigned>(pl.units() * p.n_splits);
     p.timeout_ns = timeout_ns;
     switch (iG) {
-        case 2: dw_launch<2>(grid, pl.smem_bytes, st, mdy, mx, p); break;
-        case 4: dw_launch<4>(grid, pl.smem_bytes, st, mdy, mx, p); break;
-        case 8: dw_launch<8>(grid, pl.smem_bytes, st, mdy, mx, p); break;
-        default: dw_launch<16>(grid, pl.smem_bytes, st, mdy, mx, p); break;
+        case 2: pl.io == EQLIN_F16 ? dw_launch<2, __half>(grid, pl.smem_bytes, st, mdy, mx, p)
+                                   : dw_launch<2, __nv_bfloat16>(grid, pl.smem_bytes, st, mdy, mx, p); break;
+        case 4: pl.io == EQLIN_F16 ? dw_launch<4, __half>(grid, pl.smem_bytes, st, mdy, mx, p)
+                                   : dw_launch<4, __nv_bfloat16>(grid, pl.smem_bytes, st, mdy, mx, p); break;
+        case 8: pl.io == EQLIN_F16 ? dw_launch<8, __half>(grid, pl.smem_bytes, st, mdy, mx, p)
+                                   : dw_launch<8, __nv_bfloat16>(grid, pl.smem_bytes, st, mdy, mx, p); break;
+        default: pl.io == EQLIN_F16 ? dw_launch<16, __half>(grid, pl.smem_bytes, st, mdy, mx, p)
+                                    : dw_launch<16, __nv_bfloat16>(grid, pl.smem_bytes, st, mdy, mx, p); break;
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "weight-gradient launch");
     eqlin::DwFinalParams f;
@@ -893,10 +929,12 @@ int eqlin_prepare_weights_ex(const void* w, const void* bias, int64_t Cout, int6
         }
         h->has_dx = true;
     }
-    if (io_dtype == EQLIN_BF16) {
+    if (io_dtype != EQLIN_F32) {
         // weight-gradient tiling (host only); a shape without one fails only in eqlin_backward_dw
         if (plan_dw(Cout, Cin, static_cast<int>(G), static_cast<size_t>(optin), sms, &h->dwp) == EQLIN_OK) {
-            e = cudaFuncSetAttribute(dw_kernel_for(static_cast<int>(G)), cudaFuncAttributeMaxDynamicSharedMemorySize,
+            h->dwp.io = io_dtype;
+            e = cudaFuncSetAttribute(dw_kernel_for(static_cast<int>(G), io_dtype),
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(h->dwp.smem_bytes));
             if (e != cudaSuccess) {
                 free_handle(h);
@@ -1110,7 +1148,7 @@ struct NoAllocDevice {
     int sm_count = 0;
     int optin = 0;
     bool cc_ok = false;
-    uint8_t attr_done[kNumPaths][4][2] = {};  // [path][G index][nacc-1]: smem attribute set
+    uint8_t attr_done[kNumPaths][4][2][2] = {};  // [path][G index][nacc-1][fp16 I/O]: smem attribute set
 };
 
 std::mutex g_noalloc_mutex;
@@ -1172,7 +1210,7 @@ extern "C" int eqlin_forward_noalloc(const void* x, const void* w, const void* b
         s = plan_for(Cout, Cin, G, dtype, static_cast<size_t>(d->optin), &plan);
         if (s != EQLIN_OK) return s;
         // kernel shared-memory attribute, once per kernel and device
-        uint8_t& done = d->attr_done[plan.path][g_index(G)][plan.nacc == 1 ? 0 : 1];
+        uint8_t& done = d->attr_done[plan.path][g_index(G)][plan.nacc == 1 ? 0 : 1][dtype == EQLIN_F16 ? 1 : 0];
         if (!done) {
             e = cudaFuncSetAttribute(kernel_for(plan, static_cast<int>(G)),
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(plan.smem_bytes));

@@ -1,4 +1,4 @@
-// eqlin_bwd_dw.cuh -- weight and bias gradients of EQ-Linear (bf16 I/O) on sm_100a.
+// eqlin_bwd_dw.cuh -- weight and bias gradients of EQ-Linear (16-bit I/O) on sm_100a.
 //
 // The page "Flash EQ-Linear: Accelerating Equivariant Linear Layers via Group-wise
 // Discrete Fourier Transform" lists a backward pass among its kernels (section
@@ -51,6 +51,7 @@
 
 #include "eqlin_layout.h"
 #include "group_dft.cuh"
+#include "io16.cuh"
 #include "sm100_ptx.cuh"
 
 namespace eqlin {
@@ -132,10 +133,6 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, int* s
     }
 }
 
-__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&v);
-}
 
 // One unit of the transform: one channel (of the dy tile or of the x tile) x 8 tokens
 // (token group tg of the chunk).  Raw tile layout: boxes of cpb channels, each
@@ -175,7 +172,7 @@ __device__ __forceinline__ void load_unit(const uint8_t* src, int row_bytes, Uni
 // `spec`: plane p of channel c at row r = p*rows_per_plane + c, 16-byte piece tg of the
 // 64-byte row, SWIZZLE_64B (piece j of row r at j ^ ((r >> 1) & 3)).  Returns the sum of
 // plane 0 (the group sums) over the 8 tokens.
-template <int G>
+template <int G, class T16>
 __device__ __forceinline__ float store_unit(const UnitWords<G>& u, uint8_t* spec, int rows_per_plane, int c,
                                             int tg) {
     uint32_t packed[G][4];
@@ -186,13 +183,13 @@ __device__ __forceinline__ float store_unit(const UnitWords<G>& u, uint8_t* spec
 #pragma unroll
         for (int h = 0; h < G / 2; ++h) {
             const uint32_t a = u.w[2 * jp][h], b = u.w[2 * jp + 1][h];
-            v[2 * h] = fx2(__uint_as_float(a << 16), __uint_as_float(b << 16));
-            v[2 * h + 1] = fx2(__uint_as_float(a & 0xFFFF0000u), __uint_as_float(b & 0xFFFF0000u));
+            v[2 * h] = fx2(Io16<T16>::lo(a), Io16<T16>::lo(b));
+            v[2 * h + 1] = fx2(Io16<T16>::hi(a), Io16<T16>::hi(b));
         }
         rdft_planes<G>(v, pl);
         s0 += pl[0].x + pl[0].y;
 #pragma unroll
-        for (int p = 0; p < G; ++p) packed[p][jp] = pack2(pl[p].x, pl[p].y);
+        for (int p = 0; p < G; ++p) packed[p][jp] = Io16<T16>::pack(pl[p].x, pl[p].y);
     }
 #pragma unroll
     for (int p = 0; p < G; ++p) {
@@ -205,7 +202,7 @@ __device__ __forceinline__ float store_unit(const UnitWords<G>& u, uint8_t* spec
 
 }  // namespace dw
 
-template <int G>
+template <int G, class T16>
 __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
     eqlin_dw_tc_kernel(const __grid_constant__ CUtensorMap tmap_dy, const __grid_constant__ CUtensorMap tmap_x,
                        const DwParams p) {
@@ -311,8 +308,8 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
     } else if (warp == dw::kWarpMma) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const uint32_t ID = idesc_bf16_f32(kMmaM, p.NI, false);
-            const uint32_t ID_NEG = idesc_bf16_f32(kMmaM, p.NI, true);
+            const uint32_t ID = idesc_f16kind_f32(kMmaM, p.NI, Io16<T16>::kUmmaFormat, false);
+            const uint32_t ID_NEG = idesc_f16kind_f32(kMmaM, p.NI, Io16<T16>::kUmmaFormat, true);
             const uint32_t s_spec0 = ptx::smem_u32(spec0);
             const uint32_t a_plane16 = static_cast<uint32_t>(p.MO) * kPlaneRowBytes / 16;
             const uint32_t b_plane16 = static_cast<uint32_t>(p.NI) * kPlaneRowBytes / 16;
@@ -394,9 +391,9 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
                 for (int k = 0; k < UPT; ++k) {
                     if (tgs[k] < 0) continue;
                     if (chs[k] < p.MO) {
-                        bias_sm[tgs[k] * p.MO + chs[k]] += dw::store_unit<G>(words[k], spec, p.MO, chs[k], tgs[k]);
+                        bias_sm[tgs[k] * p.MO + chs[k]] += dw::store_unit<G, T16>(words[k], spec, p.MO, chs[k], tgs[k]);
                     } else {
-                        dw::store_unit<G>(words[k], spec + p.a_bytes, p.NI, chs[k] - p.MO, tgs[k]);
+                        dw::store_unit<G, T16>(words[k], spec + p.a_bytes, p.NI, chs[k] - p.MO, tgs[k]);
                     }
                 }
             }

@@ -1,4 +1,4 @@
-// eqlin_fwd_tc.cuh -- fused EQ-Linear forward for bf16 I/O on sm_100a.
+// eqlin_fwd_tc.cuh -- fused EQ-Linear forward for 16-bit (bf16 or fp16) I/O on sm_100a.
 //
 // Operation (page "Flash EQ-Linear: Accelerating Equivariant Linear Layers via
 // Group-wise Discrete Fourier Transform", sections "Percepcion Central" and
@@ -38,6 +38,7 @@
 
 #include "eqlin_layout.h"
 #include "group_dft.cuh"
+#include "io16.cuh"
 #include "sm100_ptx.cuh"
 
 namespace eqlin {
@@ -45,7 +46,6 @@ namespace eqlin {
 struct TcParams {
     const uint8_t* w_img;   // frequency-domain weight image (layout: eqlin_layout.h)
     const float* bias;      // [Cout] fp32, or nullptr
-    __nv_bfloat16* y;       // [N, Cout, G]
     int* status;            // device status word (first error wins)
     long long N;
     int Cout;
@@ -121,15 +121,10 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, Ctl*
     }
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&v);
-}
-
 // ---------------------------------------------------------------- DFT role
 // 128 threads.  Unit = one token row x two adjacent channels (2*G bf16).
 // Lanes 0-15 take row r, lanes 16-31 row r+1; lane&15 selects the channel pair.
-template <int G, int NACC>
+template <int G, int NACC, class T16>
 __device__ __forceinline__ void dft_chunk(uint8_t* xs, int dft_tid) {
     using S = Shape<G, NACC>;
     constexpr int WORDS = G;                         // 32-bit words per unit (2 ch x G x 2 B / 4)
@@ -178,8 +173,8 @@ __device__ __forceinline__ void dft_chunk(uint8_t* xs, int dft_tid) {
 #pragma unroll
         for (int h = 0; h < G / 2; ++h) {
             const uint32_t ua = w[s][h], ub = w[s][G / 2 + h];
-            xab[2 * h] = fx2(__uint_as_float(ua << 16), __uint_as_float(ub << 16));
-            xab[2 * h + 1] = fx2(__uint_as_float(ua & 0xFFFF0000u), __uint_as_float(ub & 0xFFFF0000u));
+            xab[2 * h] = fx2(Io16<T16>::lo(ua), Io16<T16>::lo(ub));
+            xab[2 * h + 1] = fx2(Io16<T16>::hi(ua), Io16<T16>::hi(ub));
         }
         fx2 pab[G];
         rdft_planes<G>(xab, pab);
@@ -187,7 +182,7 @@ __device__ __forceinline__ void dft_chunk(uint8_t* xs, int dft_tid) {
         uint8_t* dst = xs + r * kPlaneRowBytes + phys;
 #pragma unroll
         for (int p = 0; p < G; ++p) {
-            *reinterpret_cast<uint32_t*>(dst + p * S::PLANE_BYTES) = pack_bf16x2(pab[p].x, pab[p].y);
+            *reinterpret_cast<uint32_t*>(dst + p * S::PLANE_BYTES) = Io16<T16>::pack(pab[p].x, pab[p].y);
         }
     }
 }
@@ -198,7 +193,7 @@ __device__ __forceinline__ void dft_chunk(uint8_t* xs, int dft_tid) {
 // The warp stages each group of TG tokens x its 32 output channels (32*G columns,
 // 4 KB) in its own buffer and lane 0 stores it with TMA, so the epilogue warps never
 // wait for one another.  `wstage`: this warp's p.ybufs buffers; `ybuf` alternates.
-template <int G, int NACC>
+template <int G, int NACC, class T16>
 __device__ __forceinline__ void epilogue_tile(const TcParams& p, const CUtensorMap* tmap_y, uint32_t acc,
                                               int q, int half, int lane, long long n0, int oc, uint8_t* wstage,
                                               int& ybuf) {
@@ -241,16 +236,16 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, const CUtensorM
                 RealIdft<G>::run(z, yv);
                 uint8_t* dst = lane_off + t * (YBC * 2);
                 if constexpr (G == 2) {
-                    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(yv[0], yv[1]);
+                    *reinterpret_cast<uint32_t*>(dst) = Io16<T16>::pack(yv[0], yv[1]);
                 } else if constexpr (G == 4) {
                     *reinterpret_cast<uint2*>(dst) =
-                        make_uint2(pack_bf16x2(yv[0], yv[1]), pack_bf16x2(yv[2], yv[3]));
+                        make_uint2(Io16<T16>::pack(yv[0], yv[1]), Io16<T16>::pack(yv[2], yv[3]));
                 } else {
 #pragma unroll
                     for (int c = 0; c < G / 8; ++c) {
                         *reinterpret_cast<uint4*>(dst + 16 * c) = make_uint4(
-                            pack_bf16x2(yv[8 * c + 0], yv[8 * c + 1]), pack_bf16x2(yv[8 * c + 2], yv[8 * c + 3]),
-                            pack_bf16x2(yv[8 * c + 4], yv[8 * c + 5]), pack_bf16x2(yv[8 * c + 6], yv[8 * c + 7]));
+                            Io16<T16>::pack(yv[8 * c + 0], yv[8 * c + 1]), Io16<T16>::pack(yv[8 * c + 2], yv[8 * c + 3]),
+                            Io16<T16>::pack(yv[8 * c + 4], yv[8 * c + 5]), Io16<T16>::pack(yv[8 * c + 6], yv[8 * c + 7]));
                     }
                 }
             }
@@ -278,7 +273,7 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, const CUtensorM
 
 }  // namespace tc
 
-template <int G, bool STREAM_W, int NACC>
+template <int G, bool STREAM_W, int NACC, class T16>
 __global__ void __launch_bounds__(tc::kThreads, 1)
     eqlin_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_y,
                         const TcParams p) {
@@ -409,8 +404,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         if (lane == 0) {
             bool ok = true;
             if constexpr (!STREAM_W) ok = tc::wait_bounded(bar_w_full, 0, ctl, p.status, p.timeout_ns);
-            constexpr uint32_t ID = idesc_bf16_f32(kMmaM, S::BN, false);
-            constexpr uint32_t ID_NEG = idesc_bf16_f32(kMmaM, S::BN, true);
+            constexpr uint32_t ID = idesc_f16kind_f32(kMmaM, S::BN, Io16<T16>::kUmmaFormat, false);
+            constexpr uint32_t ID_NEG = idesc_f16kind_f32(kMmaM, S::BN, Io16<T16>::kUmmaFormat, true);
             int stage = 0;
             uint32_t phase = 0;
             int it = 0;
@@ -495,7 +490,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                     ok = false;
                     break;
                 }
-                tc::dft_chunk<G, NACC>(stage0 + static_cast<size_t>(stage) * STAGE_BYTES, dft_tid);
+                tc::dft_chunk<G, NACC, T16>(stage0 + static_cast<size_t>(stage) * STAGE_BYTES, dft_tid);
                 ptx::fence_proxy_async_smem();
                 ptx::mbar_arrive(bar_xhat(stage));
                 if (++stage == NS) { stage = 0; phase ^= 1u; }
@@ -517,7 +512,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
             const int tile = wk / p.n_oc, oc = wk % p.n_oc;
             // warps whose lane quarter holds no valid output row skip the work
             if (oc * kMmaM + (warp & 3) * 32 < p.Cout) {
-                tc::epilogue_tile<G, NACC>(p, &tmap_y, tmem_base + static_cast<uint32_t>(abuf * S::ACC_COLS),
+                tc::epilogue_tile<G, NACC, T16>(p, &tmap_y, tmem_base + static_cast<uint32_t>(abuf * S::ACC_COLS),
                                            warp & 3, half, lane, static_cast<long long>(tile) * S::BN, oc, wstage,
                                            ybuf);
             }

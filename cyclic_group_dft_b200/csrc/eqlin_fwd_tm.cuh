@@ -92,7 +92,7 @@ struct Cfg {
 // --------------------------------------------------------------- DFT role
 // Unit = one token row x two adjacent channels (2*G bf16).  Lane l: row offset l/8,
 // channel pair l%8; a warp covers 4 rows per step.
-template <int G>
+template <int G, class T16>
 __device__ __forceinline__ void dft_chunk(uint8_t* xs, int dft_tid) {
     using C = Cfg<G>;
     constexpr int WORDS = G;
@@ -146,8 +146,8 @@ __device__ __forceinline__ void dft_chunk(uint8_t* xs, int dft_tid) {
 #pragma unroll
         for (int h = 0; h < G / 2; ++h) {
             const uint32_t ua = w[s][h], ub = w[s][G / 2 + h];
-            xab[2 * h] = fx2(__uint_as_float(ua << 16), __uint_as_float(ub << 16));
-            xab[2 * h + 1] = fx2(__uint_as_float(ua & 0xFFFF0000u), __uint_as_float(ub & 0xFFFF0000u));
+            xab[2 * h] = fx2(Io16<T16>::lo(ua), Io16<T16>::lo(ub));
+            xab[2 * h + 1] = fx2(Io16<T16>::hi(ua), Io16<T16>::hi(ub));
         }
         fx2 pab[G];
         rdft_planes<G>(xab, pab);
@@ -155,7 +155,7 @@ __device__ __forceinline__ void dft_chunk(uint8_t* xs, int dft_tid) {
         uint8_t* dst = xs + r * kRowBytes32 + phys;
 #pragma unroll
         for (int p = 0; p < G; ++p)
-            *reinterpret_cast<uint32_t*>(dst + p * C::PLANE_BYTES) = tc::pack_bf16x2(pab[p].x, pab[p].y);
+            *reinterpret_cast<uint32_t*>(dst + p * C::PLANE_BYTES) = Io16<T16>::pack(pab[p].x, pab[p].y);
     }
 }
 
@@ -167,7 +167,7 @@ __device__ __forceinline__ void dft_chunk(uint8_t* xs, int dft_tid) {
 // [32 tokens x 32 columns] (double-buffered), and lane 0 stores it with TMA; the
 // epilogue warps never wait for one another.  Arrives on `acc_empty` once its last TMEM
 // load has landed.
-template <int G>
+template <int G, class T16>
 __device__ __forceinline__ void epilogue_tile(const TmParams& p, const CUtensorMap* tmap_y, uint32_t tmem,
                                               int q, int half, int lane, long long n0, int oc, uint8_t* wstage,
                                               int& ybuf, uint32_t acc_empty) {
@@ -216,8 +216,8 @@ __device__ __forceinline__ void epilogue_tile(const TmParams& p, const CUtensorM
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             *reinterpret_cast<uint4*>(rowp + ((k ^ swz) * 16)) =
-                make_uint4(tc::pack_bf16x2(yv[8 * k + 0], yv[8 * k + 1]), tc::pack_bf16x2(yv[8 * k + 2], yv[8 * k + 3]),
-                           tc::pack_bf16x2(yv[8 * k + 4], yv[8 * k + 5]), tc::pack_bf16x2(yv[8 * k + 6], yv[8 * k + 7]));
+                make_uint4(Io16<T16>::pack(yv[8 * k + 0], yv[8 * k + 1]), Io16<T16>::pack(yv[8 * k + 2], yv[8 * k + 3]),
+                           Io16<T16>::pack(yv[8 * k + 4], yv[8 * k + 5]), Io16<T16>::pack(yv[8 * k + 6], yv[8 * k + 7]));
         }
         ptx::fence_proxy_async_smem();
         __syncwarp();
@@ -233,7 +233,7 @@ __device__ __forceinline__ void epilogue_tile(const TmParams& p, const CUtensorM
 
 }  // namespace tm
 
-template <int G, bool STREAM_W>
+template <int G, bool STREAM_W, class T16>
 __global__ void __launch_bounds__(tm::Cfg<G>::kThreads, 1)
     eqlin_fwd_tm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_y,
                         const TmParams p) {
@@ -356,8 +356,8 @@ __global__ void __launch_bounds__(tm::Cfg<G>::kThreads, 1)
         if (lane == 0) {
             bool ok = true;
             if constexpr (!STREAM_W) ok = tc::wait_bounded(bar_w_full, 0, ctl, p.status, p.timeout_ns);
-            const uint32_t ID = idesc_bf16_f32(tm::kM, p.NO, false, false);
-            const uint32_t ID_NEG = idesc_bf16_f32(tm::kM, p.NO, false, true);
+            const uint32_t ID = idesc_f16kind_f32(tm::kM, p.NO, Io16<T16>::kUmmaFormat, false, false);
+            const uint32_t ID_NEG = idesc_f16kind_f32(tm::kM, p.NO, Io16<T16>::kUmmaFormat, false, true);
             const uint32_t wplane = static_cast<uint32_t>(p.NO) * kRowBytes32;
             int stage = 0;
             uint32_t phase = 0;
@@ -422,7 +422,7 @@ __global__ void __launch_bounds__(tm::Cfg<G>::kThreads, 1)
                     ok = false;
                     break;
                 }
-                tm::dft_chunk<G>(stage0 + static_cast<size_t>(stage) * stage_bytes, dft_tid);
+                tm::dft_chunk<G, T16>(stage0 + static_cast<size_t>(stage) * stage_bytes, dft_tid);
                 ptx::fence_proxy_async_smem();
                 ptx::mbar_arrive(bar_xhat(stage));
                 if (++stage == NS) { stage = 0; phase ^= 1u; }
@@ -441,7 +441,7 @@ __global__ void __launch_bounds__(tm::Cfg<G>::kThreads, 1)
             if (!ptx::named_bar_and(tm::kBarEpi, tm::kEpiThreads, got)) break;
             ptx::tc_fence_after();
             const int tile = wk / p.n_oc, oc = wk % p.n_oc;
-            tm::epilogue_tile<G>(p, &tmap_y, tmem_base, warp & 3, half, lane,
+            tm::epilogue_tile<G, T16>(p, &tmap_y, tmem_base, warp & 3, half, lane,
                                  static_cast<long long>(tile) * tm::kM, oc, wstage, ybuf, bar_acc_empty);
         }
         // the y stores must be complete (not only read) before the CTA exits

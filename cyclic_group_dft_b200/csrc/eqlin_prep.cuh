@@ -9,10 +9,12 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cstdint>
 
 #include "eqlin_layout.h"
 #include "group_dft.cuh"
+#include "io16.cuh"
 
 namespace eqlin {
 
@@ -25,6 +27,10 @@ __device__ __forceinline__ double load_as_double<float>(const float* p, size_t i
 template <>
 __device__ __forceinline__ double load_as_double<__nv_bfloat16>(const __nv_bfloat16* p, size_t i) {
     return static_cast<double>(__bfloat162float(p[i]));
+}
+template <>
+__device__ __forceinline__ double load_as_double<__half>(const __half* p, size_t i) {
+    return static_cast<double>(__half2float(p[i]));
 }
 
 // One thread per (o, i) of the operator: real DFT of its filter f[o, i, :] in
@@ -70,8 +76,9 @@ __global__ void eqlin_prep_freq_kernel(const T* __restrict__ w, const T* __restr
     }
 }
 
-// One thread per element of the bf16 tensor-core image (see eqlin_layout.h).
-// `rows` rows per sub-block; output chunk oc covers o = oc*128 + r.
+// One thread per element of the 16-bit (T16: bf16 or fp16) tensor-core image (see
+// eqlin_layout.h).  `rows` rows per sub-block; output chunk oc covers o = oc*128 + r.
+template <class T16>
 __global__ void eqlin_prep_image_kernel(const float* __restrict__ w_f32, int Cout, int Cin, int G,
                                         int nK, int rows, size_t n_elems, uint8_t* __restrict__ img) {
     const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -86,11 +93,12 @@ __global__ void eqlin_prep_image_kernel(const float* __restrict__ w_f32, int Cou
     const int i = c * kChunkK + col;
     float v = 0.0f;
     if (o < Cout && i < Cin) v = w_f32[(static_cast<size_t>(p) * Cin + i) * Cout + o];
-    *reinterpret_cast<__nv_bfloat16*>(img + image_offset(sub, rows, r, col)) = __float2bfloat16_rn(v);
+    *reinterpret_cast<T16*>(img + image_offset(sub, rows, r, col)) = Io16<T16>::from_float(v);
 }
 
 // Image for the tokens-on-M kernel (layout: image_offset_k16).  `rows` rows per
 // sub-block; output chunk oc covers o = oc*rows + r.
+template <class T16>
 __global__ void eqlin_prep_image_k16_kernel(const float* __restrict__ w_f32, int Cout, int Cin, int G,
                                             int nK, int rows, size_t n_elems, uint8_t* __restrict__ img) {
     const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -105,7 +113,7 @@ __global__ void eqlin_prep_image_k16_kernel(const float* __restrict__ w_f32, int
     const int i = c * kChunkK16 + col;
     float v = 0.0f;
     if (o < Cout && i < Cin) v = w_f32[(static_cast<size_t>(p) * Cin + i) * Cout + o];
-    *reinterpret_cast<__nv_bfloat16*>(img + image_offset_k16(sub, rows, r, col)) = __float2bfloat16_rn(v);
+    *reinterpret_cast<T16*>(img + image_offset_k16(sub, rows, r, col)) = Io16<T16>::from_float(v);
 }
 
 // ------------------------------------------------------------------ fp32 path

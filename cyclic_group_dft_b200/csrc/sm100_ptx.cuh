@@ -273,16 +273,23 @@ __device__ __forceinline__ uint64_t sdesc_sw64_from_lo(uint32_t lo) {
 
 }  // namespace ptx
 
-// Instruction descriptor for tcgen05.mma kind::f16 with bf16 A/B, fp32 D, both
-// operands K-major.  M in {64,128}, N a multiple of 16 up to 256.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool negate_a, bool negate_b = false) {
+// Instruction descriptor for tcgen05.mma kind::f16 with an fp32 D, both operands
+// K-major.  fmt is the A and B operand format (0 F16, 1 BF16; A and B share it).
+// M in {64,128}, N a multiple of 16 up to 256.
+__host__ __device__ constexpr uint32_t idesc_f16kind_f32(int M, int N, uint32_t fmt, bool negate_a,
+                                                         bool negate_b = false) {
     return (1u << 4)                                  // D format: F32
-           | (1u << 7)                                // A format: BF16
-           | (1u << 10)                               // B format: BF16
+           | (fmt << 7)                               // A format
+           | (fmt << 10)                              // B format
            | ((negate_a ? 1u : 0u) << 13)             // negate A
            | ((negate_b ? 1u : 0u) << 14)             // negate B
            | (static_cast<uint32_t>(N >> 3) << 17)    // N >> 3
            | (static_cast<uint32_t>(M >> 4) << 24);   // M >> 4
+}
+
+// bf16 A and B
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool negate_a, bool negate_b = false) {
+    return idesc_f16kind_f32(M, N, 1u, negate_a, negate_b);
 }
 
 }  // namespace eqlin

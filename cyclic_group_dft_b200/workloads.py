@@ -4,7 +4,7 @@ This module holds shapes, dtypes, distributions and seeds only -- none of the
 layer's arithmetic -- so both the CUDA path and the float64 oracle can be fed
 identical inputs from it.
 
-Five workloads, all EQ-Linear over the cyclic group C_G with layout
+Six workloads, all EQ-Linear over the cyclic group C_G with layout
 x [N, Cin, G], w [Cout, Cin, G], y [N, Cout, G] (G fastest):
 
 ===================  =======  ====  =====  ===  =====  =====================
@@ -15,6 +15,7 @@ p4_c96_bf16          200704   96    96     4    bf16   headline (64*56*56)
 p8_c64_bf16          25088    64    64     8    bf16   p8 group (32*28*28)
 p4_mlp_bf16          65536    192   768    4    bf16   MLP expansion, no bias
 c16_c32_bf16         262144   32    32     16   bf16   C16 group
+p4_c96_f16           200704   96    96     4    fp16   headline shape, FP16 I/O
 ===================  =======  ====  =====  ===  =====  =====================
 
 Distributions: x ~ N(0, 1); w ~ N(0, 1/(Cin*G)); bias ~ N(0, 0.1), where the
@@ -30,7 +31,7 @@ import math
 
 import torch
 
-DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16}
+DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16, "f16": torch.float16}
 
 
 @dataclasses.dataclass(frozen=True)
@@ -40,7 +41,7 @@ class Workload:
     Cin: int
     Cout: int
     G: int
-    io_dtype: str          # "f32" or "bf16"
+    io_dtype: str          # "f32", "bf16" or "f16"
     w_var: float           # variance of w
     bias_var: float | None  # variance of bias; None = no bias (zero)
     seed: int = 0
@@ -70,6 +71,8 @@ WORKLOADS: dict[str, Workload] = {
                  "p4 MLP-expansion EQ-Linear, bf16 I/O, no bias"),
         Workload("c16_c32_bf16", 262144, 32, 32, 16, "bf16", 1.0 / (32 * 16), 0.1, 0,
                  "C16 EQ-Linear, bf16 I/O"),
+        Workload("p4_c96_f16", 64 * 56 * 56, 96, 96, 4, "f16", 1.0 / (96 * 4), 0.1, 0,
+                 "the headline p4 shape with FP16 I/O"),
     ]
 }
 

@@ -29,9 +29,10 @@
  *     a failed call launches nothing and changes nothing.  Nothing throws, aborts
  *     or prints.  eqlin_last_error() describes the latest failure of the
  *     calling thread.
- *   - Supported: G in {2, 4, 8, 16}; Cin, Cout >= 1; for bf16 I/O Cin*G and
- *     Cout*G multiples of 8 (16-byte rows for the TMA engine).  io_dtype EQLIN_BF16 runs the fused
- *     tcgen05 (tensor-core) kernel; EQLIN_F32 runs a fused FFMA kernel.
+ *   - Supported: G in {2, 4, 8, 16}; Cin, Cout >= 1; for 16-bit I/O (bf16 or fp16)
+ *     Cin*G and Cout*G multiples of 8 (16-byte rows for the TMA engine).  io_dtype
+ *     EQLIN_BF16 or EQLIN_F16 runs the fused tcgen05 (tensor-core) kernels with that
+ *     operand type and fp32 accumulation; EQLIN_F32 runs a fused FFMA kernel in float64.
  *   - Requires a compute-capability 10.0 device (B200).
  */
 #ifndef EQLIN_H
@@ -54,7 +55,8 @@ typedef struct eqlin_handle eqlin_handle; /* opaque */
 
 typedef enum {
     EQLIN_F32 = 0,  /* IEEE float32 */
-    EQLIN_BF16 = 1  /* bfloat16 */
+    EQLIN_BF16 = 1, /* bfloat16 */
+    EQLIN_F16 = 2   /* IEEE float16 (the page's FP16 kernels, section "Implementacion") */
 } eqlin_dtype;
 
 typedef enum {
@@ -75,16 +77,17 @@ typedef enum {
  *   w        device, [Cout, Cin, G] of w_dtype.  Read only.
  *   bias     device, [Cout] of w_dtype, or NULL (zero bias).  Read only.
  *   Cout, Cin, G   layer sizes (see "Supported" above).
- *   w_dtype  EQLIN_F32 or EQLIN_BF16: element type of w and bias.
- *   io_dtype EQLIN_F32 or EQLIN_BF16: element type of x and y in eqlin_forward.
+ *   w_dtype  EQLIN_F32, EQLIN_BF16 or EQLIN_F16: element type of w and bias.
+ *   io_dtype EQLIN_F32, EQLIN_BF16 or EQLIN_F16: element type of x and y in
+ *            eqlin_forward (and of dy, dx in the backward calls).
  *   stream   stream the transform runs on; the call synchronises it before
  *            returning, so w and bias may be freed or changed afterwards.
  *   out      host; receives the new handle (set to NULL on failure).
  *
- * The handle owns device memory for the transformed weights (bf16 tensor-core
+ * The handle owns device memory for the transformed weights (16-bit tensor-core
  * image and/or fp32 planes), an fp32 copy of the bias and a device status word.
  * Errors: INVALID_ARG (null w/out, non-positive sizes, unknown dtype),
- * UNSUPPORTED (G not in {2,4,8,16}, Cin*G or Cout*G not a multiple of 8 for bf16 I/O,
+ * UNSUPPORTED (G not in {2,4,8,16}, Cin*G or Cout*G not a multiple of 8 for 16-bit I/O,
  * not an sm_100 device, shape too large for shared memory), MISALIGNED (w or
  * bias not aligned to its element size), OOM, CUDA.
  */
@@ -94,7 +97,7 @@ EQLIN_API int eqlin_prepare_weights(const void* w, const void* bias, int64_t Cou
 /*
  * eqlin_forward -- y = EQ-Linear(x), the whole forward in one fused launch:
  * TMA-staged loads of x, the group DFT in registers, the per-frequency
- * contractions (tcgen05 tensor cores for bf16), the inverse DFT plus bias
+ * contractions (tcgen05 tensor cores for bf16 / fp16), the inverse DFT plus bias
  * written straight to y (sections "Enfoque Algoritmico", "Implementacion").
  *
  *   h        handle from eqlin_prepare_weights.  Not modified; may be shared by
@@ -185,7 +188,7 @@ EQLIN_API int eqlin_check_shape(int64_t Cout, int64_t Cin, int64_t G, int w_dtyp
  *
  *   x, y     device, [N, Cin, G] / [N, Cout, G] of dtype, 16-byte aligned.
  *   w, bias  device, [Cout, Cin, G] / [Cout] of dtype (bias may be NULL).
- *   dtype    EQLIN_BF16 or EQLIN_F32, for all four tensors.
+ *   dtype    EQLIN_BF16, EQLIN_F16 or EQLIN_F32, for all four tensors.
  *   stream   every step (weight transform, forward) is enqueued on it; nothing is
  *            synchronised.
  *
@@ -223,7 +226,7 @@ EQLIN_API int eqlin_forward_noalloc(const void* x, const void* w, const void* bi
  *     filters reflected, f[i,o,m] = w[o,i,(-m) mod G], so the same fused kernels run it
  *     with weights prepared for it.
  *   - dw is a contraction over tokens: a [Cout x N] by [N x Cin] product per frequency,
- *     on tcgen05 for bf16, then an inverse DFT over the group axis.
+ *     on tcgen05 for bf16 / fp16, then an inverse DFT over the group axis.
  */
 
 /* eqlin_prepare_weights_ex flag: also prepare the input-gradient weights, so the
@@ -278,14 +281,14 @@ EQLIN_API int eqlin_backward_dw_workspace_size(const eqlin_handle* h, int64_t N,
  *              16-byte aligned, owned by the caller.  Its contents on entry do not
  *              matter and on exit are unspecified.  Two calls whose work overlaps on
  *              the GPU must not share it.
- *   stream     asynchronous on this stream: 2 launches for bf16 (the tcgen05
- *              contraction with a per-CTA partial sum, then a deterministic
- *              reduction and inverse DFT); for fp32, a clear, a float64 CUDA-core
- *              kernel and a conversion.  Allocates nothing.
+ *   stream     asynchronous on this stream: 3 launches for 16-bit I/O (the tcgen05
+ *              contraction with a per-CTA partial sum, a deterministic reduction of
+ *              the partial sums, the inverse DFT); for fp32, a clear, a float64
+ *              CUDA-core kernel and a conversion.  Allocates nothing.
  *
- * bf16: the spectra are rounded to bf16 for the tensor cores and accumulated in fp32;
- * the partial sums are reduced in float64 in a fixed order, so repeated calls give
- * identical results.  fp32: float64 arithmetic throughout (the order of the float64
+ * 16-bit I/O: the spectra are rounded to the I/O type for the tensor cores and
+ * accumulated in fp32; the partial sums are reduced in float64 in a fixed order, so
+ * repeated calls give identical results.  fp32: float64 arithmetic throughout (the order of the float64
  * additions across token slices may vary).
  * Errors: INVALID_ARG (null handle/dw, N < 0, null x/dy with N > 0, workspace missing or
  * too small, wrong device), MISALIGNED, UNSUPPORTED, CUDA.  Kernel wait timeouts go to

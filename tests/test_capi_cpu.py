@@ -40,6 +40,9 @@ def test_version_and_status_strings():
     ((32, 32, 16, eq.EQLIN_BF16, eq.EQLIN_BF16), eq.EQLIN_OK),
     ((16, 16, 4, eq.EQLIN_F32, eq.EQLIN_F32), eq.EQLIN_OK),
     ((16, 16, 2, eq.EQLIN_F32, eq.EQLIN_BF16), eq.EQLIN_OK),
+    ((96, 96, 4, eq.EQLIN_F16, eq.EQLIN_F16), eq.EQLIN_OK),
+    ((32, 32, 16, eq.EQLIN_F32, eq.EQLIN_F16), eq.EQLIN_OK),
+    ((3, 3, 2, eq.EQLIN_F16, eq.EQLIN_F16), eq.EQLIN_ERR_UNSUPPORTED),     # Cin*G % 8
     ((96, 96, 3, eq.EQLIN_BF16, eq.EQLIN_BF16), eq.EQLIN_ERR_UNSUPPORTED),
     ((96, 96, 32, eq.EQLIN_BF16, eq.EQLIN_BF16), eq.EQLIN_ERR_UNSUPPORTED),
     ((3, 3, 2, eq.EQLIN_BF16, eq.EQLIN_BF16), eq.EQLIN_ERR_UNSUPPORTED),   # Cin*G % 8
@@ -106,7 +109,7 @@ def test_header_matches_binding_constants():
     text = open(_capi.HEADER_PATH).read()
     for name in ("EQLIN_ERR_INVALID_ARG = -1", "EQLIN_ERR_UNSUPPORTED = -2", "EQLIN_ERR_MISALIGNED = -3",
                  "EQLIN_ERR_CUDA = -4", "EQLIN_ERR_OOM = -5", "EQLIN_ERR_TIMEOUT = -6",
-                 "EQLIN_F32 = 0", "EQLIN_BF16 = 1"):
+                 "EQLIN_F32 = 0", "EQLIN_BF16 = 1", "EQLIN_F16 = 2"):
         assert name in text
     for attr, code in eq.ATTRS.items():
         assert f"= {code}" in text

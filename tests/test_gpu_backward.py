@@ -96,7 +96,7 @@ SHAPES = [  # (Cout, Cin, G): odd channel counts, several weight-gradient tiles,
 ]
 
 
-@pytest.mark.parametrize("io", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("io", [torch.bfloat16, torch.float16, torch.float32])
 @pytest.mark.parametrize("Cout,Cin,G", SHAPES)
 def test_backward_shapes(Cout, Cin, G, io):
     gen = torch.Generator().manual_seed(Cout * 1000 + Cin * 10 + G + 77)

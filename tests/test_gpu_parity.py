@@ -6,7 +6,8 @@ on identical seeded inputs.
 * every workload at its full size, on sampled tokens (tokens are independent,
   so the oracle computes just those rows);
 * edge cases: N = 1, N = 0, non-multiple-of-32 channel counts, Cout > 128
-  (weights streamed), every supported G, fp32 and bf16 weights, no bias;
+  (weights streamed), every supported G, fp32 / bf16 / fp16 weights and I/O,
+  no bias;
 * properties: cyclic-shift equivariance, guard bands around y untouched,
   the device status word stays OK, the prepared weights equal the oracle's DFT.
 """
@@ -87,7 +88,7 @@ SHAPES = [  # (Cout, Cin, G): odd channel counts, streamed weights (Cout > 128),
 ]
 
 
-@pytest.mark.parametrize("io", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("io", [torch.bfloat16, torch.float16, torch.float32])
 @pytest.mark.parametrize("Cout,Cin,G", SHAPES)
 def test_shapes_every_group_order(Cout, Cin, G, io):
     gen = torch.Generator().manual_seed(Cout * 1000 + Cin * 10 + G)
@@ -100,20 +101,21 @@ def test_shapes_every_group_order(Cout, Cin, G, io):
     h.close()
 
 
+@pytest.mark.parametrize("io", [torch.bfloat16, torch.float16])
 @pytest.mark.parametrize("kernel", ["tn", "tm"])
 @pytest.mark.parametrize("Cout,Cin,G", SHAPES)
-def test_shapes_both_fused_kernels(Cout, Cin, G, kernel, monkeypatch):
-    """Each fused bf16 kernel (tokens on N, tokens on M) is correct for every
+def test_shapes_both_fused_kernels(Cout, Cin, G, kernel, io, monkeypatch):
+    """Each fused 16-bit kernel (tokens on N, tokens on M) is correct for every
     shape, whichever one the planner would pick by default."""
     monkeypatch.setenv("EQLIN_KERNEL", kernel)
     gen = torch.Generator().manual_seed(Cout * 1000 + Cin * 10 + G + 5)
     N = 517
-    x = torch.randn(N, Cin, G, generator=gen).to(torch.bfloat16)
-    w = (torch.randn(Cout, Cin, G, generator=gen) / np.sqrt(Cin * G)).to(torch.bfloat16)
-    bias = (torch.randn(Cout, generator=gen) * 0.3).to(torch.bfloat16)
-    y, h = _run(x, w, bias, torch.bfloat16)
+    x = torch.randn(N, Cin, G, generator=gen).to(io)
+    w = (torch.randn(Cout, Cin, G, generator=gen) / np.sqrt(Cin * G)).to(io)
+    bias = (torch.randn(Cout, generator=gen) * 0.3).to(io)
+    y, h = _run(x, w, bias, io)
     assert f"tokens_on_{kernel[1]}" in h.path, h.path
-    _assert_parity(torch.bfloat16, y, _ref(x, w, bias), f"Cout={Cout} Cin={Cin} G={G} {kernel}")
+    _assert_parity(io, y, _ref(x, w, bias), f"Cout={Cout} Cin={Cin} G={G} {kernel} {io}")
     h.close()
 
 
