@@ -533,6 +533,7 @@ int launch_forward(const Plan& pl, int64_t Cout, int64_t Cin, int64_t G, int sm_
 struct DwPlan {
     int io = EQLIN_BF16;  // 16-bit element type of x and dy
     int MO = 0, NI = 0, n_ot = 0, n_it = 0, max_splits = 0;
+    int MA = 0, NA = 0;   // 32-channel atoms of the MN-major spectra: ceil(MO / 32), ceil(NI / 32)
     int cpb_dy = 0, cpb_x = 0;
     int raw_stages = 0, spec_bufs = 0;
     uint32_t dy_bytes = 0, raw_bytes = 0, a_bytes = 0, b_bytes = 0, tmem_cols = 0;
@@ -551,13 +552,20 @@ int box_channels(int C, int G) {
     return 0;
 }
 
+// Shared memory of the weight-gradient kernel: raw ring (RS stages of the 32-token dy and
+// x tiles), SB spectra buffers (A: G dy planes of 4 K-groups x MA atoms of 512 B, plus
+// the slack a 128-row MMA reads past the last plane; B: G x planes of 4 x NA atoms),
+// the dbias slots [32 tokens][MO] and the barriers.
 size_t dw_smem(int MO, int NI, int G, int RS, int SB, DwPlan* out) {
+    const int MA = (MO + 31) / 32, NA = (NI + 31) / 32;
     const size_t raw = round_kb(static_cast<size_t>(eqlin::dw::kTok) * (MO + NI) * G * 2);
-    const size_t a = round_kb(static_cast<size_t>(G * MO + (eqlin::kMmaM - MO)) * eqlin::kPlaneRowBytes);
-    const size_t b = round_kb(static_cast<size_t>(G) * NI * eqlin::kPlaneRowBytes);
+    const size_t a = round_kb(static_cast<size_t>(G) * 4 * MA * 512 + static_cast<size_t>(4 - MA) * 512);
+    const size_t b = round_kb(static_cast<size_t>(G) * 4 * NA * 512);
     const size_t total = kSmemAlignSlack + static_cast<size_t>(RS) * raw + static_cast<size_t>(SB) * (a + b) +
-                         static_cast<size_t>(4 * MO) * 4 + 256;
+                         static_cast<size_t>(eqlin::dw::kTok) * MO * 4 + 256;
     if (out) {
+        out->MA = MA;
+        out->NA = NA;
         out->dy_bytes = static_cast<uint32_t>(eqlin::dw::kTok) * MO * G * 2;
         out->raw_bytes = static_cast<uint32_t>(raw);
         out->a_bytes = static_cast<uint32_t>(a);
@@ -619,6 +627,8 @@ int plan_dw(int64_t Cout, int64_t Cin, int G, size_t max_smem, int sm_count, DwP
     pl->max_splits = std::max(1, sm_count / pl->units());
     pl->cpb_dy = box_channels(best_mo, G);
     pl->cpb_x = box_channels(best_ni, G);
+    // the transform's channel pairs never straddle two boxes
+    if (pl->cpb_dy % 2 != 0 || pl->cpb_x % 2 != 0) return fail(EQLIN_ERR_UNSUPPORTED, "odd TMA box width");
     dw_smem(best_mo, best_ni, G, rs, sb, pl);
     int cols = 32;
     while (cols < G * best_ni) cols *= 2;
@@ -732,6 +742,8 @@ int launch_dw(const DwPlan& pl, bool f32_path, int64_t Cout, int64_t Cin, int64_
     p.raw_stages = pl.raw_stages;
     p.spec_bufs = pl.spec_bufs;
     p.slab_floats = pl.slab_floats;
+    p.MA = pl.MA;
+    p.NA = pl.NA;
     const unsigned grid = static_cast<unsigned>(pl.units() * p.n_splits);
     p.timeout_ns = timeout_ns;
     switch (iG) {

@@ -72,28 +72,28 @@ struct DwParams {
     uint32_t tmem_cols;        // power of two >= G * NI
     int raw_stages;            // depth of the raw ring (2 .. kMaxRawStages)
     int spec_bufs;             // spectra buffers (1 or 2)
+    int MA, NA;                // 32-channel atoms per plane row group: ceil(MO / 32), ceil(NI / 32)
     size_t slab_floats;        // G * NI * MO (a CTA's slab holds slab_floats + MO floats)
     unsigned long long timeout_ns;
 };
 
 namespace dw {
 
-constexpr int kTok = 32;           // tokens per chunk (one 64-byte K-major row)
+constexpr int kTok = 32;           // tokens per chunk (4 atoms of 8 K-rows)
 constexpr int kMaxRawStages = 8;   // raw ring depth is a launch parameter (p.raw_stages)
 constexpr int kMaxSpecBufs = 2;
 constexpr int kWarpProducer = 0;
 constexpr int kWarpMma = 1;
 constexpr int kWarpDft0 = 2;
 
-// Transform warps per CTA: 12 (3 per SM sub-partition, to hide the latency of the
-// short dependent DFT chains) where the units of a chunk fill them and the registers
-// allow; 8 for G = 16 (256 units per chunk at most, and the DFT needs the registers).
+// Transform warps per CTA: 16 (4 per SM sub-partition, to hide the latency of the short
+// dependent DFT chains); with the per-token units the transform needs <= 112 registers.
 template <int G>
 struct Cfg {
-    static constexpr int kDftWarps = G == 16 ? 8 : 12;
+    static constexpr int kDftWarps = 16;
     static constexpr int kDftThreads = kDftWarps * 32;
     static constexpr int kThreads = (2 + kDftWarps) * 32;
-    static constexpr int kUnitsPerPass = G >= 8 ? 1 : 2;    // units a thread batches per pass
+    static constexpr int kUnitsPerPass = 16 / G;            // pairs a thread batches per pass
 };
 constexpr int kBarDft = 1;         // named barrier among the DFT warps
 constexpr uint32_t kWaitSleepNs = 20000;
@@ -134,70 +134,52 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, int* s
 }
 
 
-// One unit of the transform: one channel (of the dy tile or of the x tile) x 8 tokens
-// (token group tg of the chunk).  Raw tile layout: boxes of cpb channels, each
-// [32 tokens][cpb*G] bf16.  A thread first loads all of its units of a chunk (load_unit,
-// G/2 words per token) and then transforms and stores them (store_unit), so the shared
-// memory latency of the loads overlaps.
+// One unit of the transform: one token t of the chunk x one channel pair (c, c+1) of
+// the dy tile or of the x tile.  Raw tile layout: boxes of cpb channels (cpb even, so a
+// pair never straddles two boxes), each [32 tokens][cpb*G].  The unit's 2G values are
+// G 32-bit words (channel c in words 0..G/2-1, channel c+1 in the rest).
 template <int G>
-struct UnitWords {
-    uint32_t w[8][G / 2];
-};
-
-template <int G>
-__device__ __forceinline__ void load_unit(const uint8_t* src, int row_bytes, UnitWords<G>& u) {
+__device__ __forceinline__ void load_pair(const uint8_t* src, uint32_t (&w)[G]) {
+    if constexpr (G == 2) {
+        const uint2 v = *reinterpret_cast<const uint2*>(src);
+        w[0] = v.x;
+        w[1] = v.y;
+    } else {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const uint8_t* q = src + j * row_bytes;
-        if constexpr (G == 2) {
-            u.w[j][0] = *reinterpret_cast<const uint32_t*>(q);
-        } else if constexpr (G == 4) {
-            const uint2 v = *reinterpret_cast<const uint2*>(q);
-            u.w[j][0] = v.x;
-            u.w[j][1] = v.y;
-        } else {
-#pragma unroll
-            for (int c = 0; c < G / 8; ++c) {
-                const uint4 v = *reinterpret_cast<const uint4*>(q + 16 * c);
-                u.w[j][4 * c + 0] = v.x;
-                u.w[j][4 * c + 1] = v.y;
-                u.w[j][4 * c + 2] = v.z;
-                u.w[j][4 * c + 3] = v.w;
-            }
+        for (int q = 0; q < G / 4; ++q) {
+            const uint4 v = *reinterpret_cast<const uint4*>(src + 16 * q);
+            w[4 * q + 0] = v.x;
+            w[4 * q + 1] = v.y;
+            w[4 * q + 2] = v.z;
+            w[4 * q + 3] = v.w;
         }
     }
 }
 
-// Real DFT over G of the unit's 8 tokens (token pairs packed as fx2), bf16 planes to
-// `spec`: plane p of channel c at row r = p*rows_per_plane + c, 16-byte piece tg of the
-// 64-byte row, SWIZZLE_64B (piece j of row r at j ^ ((r >> 1) & 3)).  Returns the sum of
-// plane 0 (the group sums) over the 8 tokens.
+// Real DFT over G of the pair (the two channels packed as fx2), stored to the planes in
+// the MN-major SWIZZLE_64B operand layout: plane p at plane0 + p * plane_bytes; in it the
+// 8-row atom (kg = t / 8, ma = c / 32) at kg * sbo + ma * 512 holds row t % 8 = 64 bytes
+// of channels 32ma .. 32ma + 31, 16-byte chunk j of row r stored at chunk j ^ ((r >> 1) & 3).
+// Returns plane 0 (the group sums of the two channels).
 template <int G, class T16>
-__device__ __forceinline__ float store_unit(const UnitWords<G>& u, uint8_t* spec, int rows_per_plane, int c,
-                                            int tg) {
-    uint32_t packed[G][4];
-    float s0 = 0.0f;
+__device__ __forceinline__ fx2 store_pair(const uint32_t (&w)[G], uint8_t* plane0, uint32_t plane_bytes,
+                                          uint32_t sbo, int t, int c) {
+    fx2 v[G], pl[G];
 #pragma unroll
-    for (int jp = 0; jp < 4; ++jp) {
-        fx2 v[G], pl[G];
-#pragma unroll
-        for (int h = 0; h < G / 2; ++h) {
-            const uint32_t a = u.w[2 * jp][h], b = u.w[2 * jp + 1][h];
-            v[2 * h] = fx2(Io16<T16>::lo(a), Io16<T16>::lo(b));
-            v[2 * h + 1] = fx2(Io16<T16>::hi(a), Io16<T16>::hi(b));
-        }
-        rdft_planes<G>(v, pl);
-        s0 += pl[0].x + pl[0].y;
-#pragma unroll
-        for (int p = 0; p < G; ++p) packed[p][jp] = Io16<T16>::pack(pl[p].x, pl[p].y);
+    for (int h = 0; h < G / 2; ++h) {
+        v[2 * h] = fx2(Io16<T16>::lo(w[h]), Io16<T16>::lo(w[G / 2 + h]));
+        v[2 * h + 1] = fx2(Io16<T16>::hi(w[h]), Io16<T16>::hi(w[G / 2 + h]));
     }
+    rdft_planes<G>(v, pl);
+    const int r = t & 7;
+    const uint32_t off = static_cast<uint32_t>(t >> 3) * sbo + static_cast<uint32_t>(c >> 5) * 512u +
+                         static_cast<uint32_t>(r) * 64u +
+                         static_cast<uint32_t>((((c & 31) >> 3) ^ ((r >> 1) & 3)) << 4) +
+                         static_cast<uint32_t>(c & 7) * 2u;
 #pragma unroll
-    for (int p = 0; p < G; ++p) {
-        const int r = p * rows_per_plane + c;
-        uint8_t* dst = spec + static_cast<size_t>(r) * kPlaneRowBytes + ((tg ^ ((r >> 1) & 3)) << 4);
-        *reinterpret_cast<uint4*>(dst) = make_uint4(packed[p][0], packed[p][1], packed[p][2], packed[p][3]);
-    }
-    return s0;
+    for (int p = 0; p < G; ++p)
+        *reinterpret_cast<uint32_t*>(plane0 + p * plane_bytes + off) = Io16<T16>::pack(pl[p].x, pl[p].y);
+    return pl[0];
 }
 
 }  // namespace dw
@@ -213,10 +195,10 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
     uint8_t* raw0 = base;
     uint8_t* spec0 = raw0 + p.raw_stages * p.raw_bytes;
     float* bias_sm = reinterpret_cast<float*>(spec0 + p.spec_bufs * spec_bytes);
-    // bias_sm[tg][c]: group sums of dy channel c over token group tg of every chunk; each
+    // bias_sm[t][c]: group sums of dy channel c at chunk token t, over every chunk; each
     // slot has a single writer (the unit -> thread map is the same for every chunk), so
     // the per-CTA sums are formed in a fixed order
-    uint64_t* bars = reinterpret_cast<uint64_t*>(bias_sm + 4 * p.MO);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(bias_sm + dw::kTok * p.MO);
     const int RS = p.raw_stages, SB = p.spec_bufs;
     dw::Ctl* ctl = reinterpret_cast<dw::Ctl*>(bars + 2 * RS + 2 * SB + 2);
 
@@ -259,12 +241,14 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
     }
     if (warp >= dw::kWarpDft0) {
         const int t = threadIdx.x - dw::kWarpDft0 * 32;
-        for (int c = t; c < 4 * p.MO; c += kDftThreads) bias_sm[c] = 0.0f;
+        for (int c = t; c < dw::kTok * p.MO; c += kDftThreads) bias_sm[c] = 0.0f;
         // A-region tail rows (read by the MMA, never written by the transform): zero
-        const int tail0 = G * p.MO, tail1 = G * p.MO + (kMmaM - p.MO);
+        // A-region slack after the G planes (read by the 128-row MMA of the last plane,
+        // never written by the transform): zero
+        const uint32_t tail0 = static_cast<uint32_t>(G) * 4u * static_cast<uint32_t>(p.MA) * 512u;
         for (int b = 0; b < SB; ++b) {
             uint8_t* a = spec0 + static_cast<size_t>(b) * spec_bytes;
-            for (int idx = tail0 * 4 + t; idx < tail1 * 4; idx += kDftThreads)
+            for (uint32_t idx = tail0 / 16 + t; idx < p.a_bytes / 16; idx += kDftThreads)
                 reinterpret_cast<uint4*>(a)[idx] = make_uint4(0, 0, 0, 0);
         }
         ptx::fence_proxy_async_smem();
@@ -308,11 +292,13 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
     } else if (warp == dw::kWarpMma) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const uint32_t ID = idesc_f16kind_f32(kMmaM, p.NI, Io16<T16>::kUmmaFormat, false);
-            const uint32_t ID_NEG = idesc_f16kind_f32(kMmaM, p.NI, Io16<T16>::kUmmaFormat, true);
+            // both operands MN-major (channels contiguous, tokens along K)
+            const uint32_t ID = idesc_f16kind_f32_mn(kMmaM, p.NI, Io16<T16>::kUmmaFormat, false);
+            const uint32_t ID_NEG = idesc_f16kind_f32_mn(kMmaM, p.NI, Io16<T16>::kUmmaFormat, true);
             const uint32_t s_spec0 = ptx::smem_u32(spec0);
-            const uint32_t a_plane16 = static_cast<uint32_t>(p.MO) * kPlaneRowBytes / 16;
-            const uint32_t b_plane16 = static_cast<uint32_t>(p.NI) * kPlaneRowBytes / 16;
+            const uint32_t sbo_a = static_cast<uint32_t>(p.MA) * 512u, sbo_b = static_cast<uint32_t>(p.NA) * 512u;
+            const uint32_t hi_a = ptx::sdesc_mn_sw64_hi(sbo_a), hi_b = ptx::sdesc_mn_sw64_hi(sbo_b);
+            const uint32_t plane_a16 = 4u * sbo_a / 16u, plane_b16 = 4u * sbo_b / 16u;
             bool ok = true;
             for (int j = 0; j < n_mine; ++j) {
                 const int sb = j % SB;
@@ -323,12 +309,18 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
                 }
                 ptx::tc_fence_after();
                 const uint32_t a_addr = s_spec0 + sb * spec_bytes;
-                const uint32_t a_lo = ptx::sdesc_sw64_lo(a_addr), b_lo = ptx::sdesc_sw64_lo(a_addr + p.a_bytes);
+                const uint32_t a_lo = ptx::sdesc_mn_sw64_lo(a_addr, 512u);
+                const uint32_t b_lo = ptx::sdesc_mn_sw64_lo(a_addr + p.a_bytes, 512u);
 #pragma unroll
                 for (int ks = 0; ks < dw::kTok / 16; ++ks) {
                     const uint32_t acc0 = (j > 0 || ks > 0) ? 1u : 0u;
-                    auto A = [&](int pl) { return ptx::sdesc_sw64_from_lo(a_lo + pl * a_plane16 + ks * 2); };
-                    auto B = [&](int pl) { return ptx::sdesc_sw64_from_lo(b_lo + pl * b_plane16 + ks * 2); };
+                    // K step ks = tokens 16ks .. 16ks+15 = K groups 2ks, 2ks+1
+                    auto A = [&](int pl) {
+                        return ptx::sdesc_from_halves(hi_a, a_lo + pl * plane_a16 + 2 * ks * (sbo_a / 16));
+                    };
+                    auto B = [&](int pl) {
+                        return ptx::sdesc_from_halves(hi_b, b_lo + pl * plane_b16 + 2 * ks * (sbo_b / 16));
+                    };
                     auto D = [&](int pl) { return tmem_base + static_cast<uint32_t>(pl * p.NI); };
                     ptx::umma_f16(D(0), A(0), B(0), ID, acc0);
                     ptx::umma_f16(D(1), A(1), B(1), ID, acc0);
@@ -350,8 +342,12 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
     } else {
         // ------------------------------------------------------------ transform warps
         const int t = threadIdx.x - dw::kWarpDft0 * 32;
-        const int width = p.MO + p.NI;
-        const int n_units = 4 * width;
+        // units: token t x channel pair; the dy pairs of all tokens first, then x's
+        const int pairs_dy = p.MO / 2, pairs_x = p.NI / 2;
+        const int units_dy = dw::kTok * pairs_dy;
+        const int n_units = units_dy + dw::kTok * pairs_x;
+        const uint32_t sbo_a = static_cast<uint32_t>(p.MA) * 512u, sbo_b = static_cast<uint32_t>(p.NA) * 512u;
+        const uint32_t plane_a = 4u * sbo_a, plane_b = 4u * sbo_b;
         bool ok = true;
         for (int j = 0; j < n_mine; ++j) {
             const int s = j % RS, sb = j % SB;
@@ -367,33 +363,36 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
             uint8_t* spec = spec0 + static_cast<size_t>(sb) * spec_bytes;
             constexpr int UPT = dw::Cfg<G>::kUnitsPerPass;
             for (int base = 0; base < n_units; base += kDftThreads * UPT) {
-                dw::UnitWords<G> words[UPT];
-                int chs[UPT], tgs[UPT];
+                uint32_t words[UPT][G];
+                int ts[UPT], cs[UPT];
 #pragma unroll
                 for (int k = 0; k < UPT; ++k) {
                     const int u = base + t + k * kDftThreads;
-                    tgs[k] = -1;
-                    chs[k] = 0;
+                    ts[k] = -1;
+                    cs[k] = 0;
                     if (u < n_units) {
-                        const int tg = u / width, ch = u - tg * width;
-                        const bool is_dy = ch < p.MO;
-                        const int c = is_dy ? ch : ch - p.MO, cpb = is_dy ? p.cpb_dy : p.cpb_x;
+                        const bool is_dy = u < units_dy;
+                        const int v = is_dy ? u : u - units_dy, np = is_dy ? pairs_dy : pairs_x;
+                        const int tok = v / np, c = 2 * (v - tok * np), cpb = is_dy ? p.cpb_dy : p.cpb_x;
                         const int box = c / cpb, row_bytes = cpb * G * 2;
                         const uint8_t* src = raw + (is_dy ? 0u : p.dy_bytes) +
                                              static_cast<size_t>(box) * (dw::kTok * row_bytes) +
-                                             static_cast<size_t>(tg * 8) * row_bytes + (c - box * cpb) * G * 2;
-                        dw::load_unit<G>(src, row_bytes, words[k]);
-                        tgs[k] = tg;
-                        chs[k] = ch;
+                                             static_cast<size_t>(tok) * row_bytes + (c - box * cpb) * G * 2;
+                        dw::load_pair<G>(src, words[k]);
+                        ts[k] = tok;
+                        cs[k] = is_dy ? c : -1 - c;     // x pairs carry -1 - c
                     }
                 }
 #pragma unroll
                 for (int k = 0; k < UPT; ++k) {
-                    if (tgs[k] < 0) continue;
-                    if (chs[k] < p.MO) {
-                        bias_sm[tgs[k] * p.MO + chs[k]] += dw::store_unit<G, T16>(words[k], spec, p.MO, chs[k], tgs[k]);
+                    if (ts[k] < 0) continue;
+                    if (cs[k] >= 0) {
+                        const fx2 s0 = dw::store_pair<G, T16>(words[k], spec, plane_a, sbo_a, ts[k], cs[k]);
+                        float* bs = bias_sm + ts[k] * p.MO + cs[k];
+                        bs[0] += s0.x;
+                        bs[1] += s0.y;
                     } else {
-                        dw::store_unit<G, T16>(words[k], spec + p.a_bytes, p.NI, chs[k] - p.MO, tgs[k]);
+                        dw::store_pair<G, T16>(words[k], spec + p.a_bytes, plane_b, sbo_b, ts[k], -1 - cs[k]);
                     }
                 }
             }
@@ -430,8 +429,11 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
         }
         // dbias partial of this CTA (every CTA writes it; the inverse-DFT kernel reads input tile 0's)
         ptx::named_bar_sync(dw::kBarDft, kDftThreads);
-        for (int c = t; c < p.MO; c += kDftThreads)
-            slab[p.slab_floats + c] = (bias_sm[c] + bias_sm[p.MO + c]) + (bias_sm[2 * p.MO + c] + bias_sm[3 * p.MO + c]);
+        for (int c = t; c < p.MO; c += kDftThreads) {
+            float acc = 0.0f;
+            for (int tok = 0; tok < dw::kTok; ++tok) acc += bias_sm[tok * p.MO + c];
+            slab[p.slab_floats + c] = acc;
+        }
     }
 
     ptx::tc_fence_before();

@@ -271,6 +271,20 @@ __device__ __forceinline__ uint64_t sdesc_sw64_from_lo(uint32_t lo) {
     return (static_cast<uint64_t>(kSdescSw64Hi) << 32) | lo;
 }
 
+// MN-major operand with 64-byte swizzle: each 8-row atom (512 B) holds 8 consecutive
+// K indices as rows of 64 B = 32 consecutive M (or N) elements; lbo = byte stride
+// between atoms along M/N, sbo = byte stride between 8-row groups along K.  Split in
+// halves like the K-major forms: the high half carries sbo, version and layout.
+__device__ __forceinline__ uint32_t sdesc_mn_sw64_lo(uint32_t start, uint32_t lbo) {
+    return ((lbo >> 4) << 16) | (start >> 4);
+}
+__device__ __forceinline__ uint32_t sdesc_mn_sw64_hi(uint32_t sbo) {
+    return ((sbo >> 4) & 0x3FFFu) | (1u << 14) | (4u << 29);
+}
+__device__ __forceinline__ uint64_t sdesc_from_halves(uint32_t hi, uint32_t lo) {
+    return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
 }  // namespace ptx
 
 // Instruction descriptor for tcgen05.mma kind::f16 with an fp32 D, both operands
@@ -285,6 +299,12 @@ __host__ __device__ constexpr uint32_t idesc_f16kind_f32(int M, int N, uint32_t 
            | ((negate_b ? 1u : 0u) << 14)             // negate B
            | (static_cast<uint32_t>(N >> 3) << 17)    // N >> 3
            | (static_cast<uint32_t>(M >> 4) << 24);   // M >> 4
+}
+
+// the same with both operands MN-major (A: M contiguous, B: N contiguous)
+__host__ __device__ constexpr uint32_t idesc_f16kind_f32_mn(int M, int N, uint32_t fmt, bool negate_a,
+                                                            bool negate_b = false) {
+    return idesc_f16kind_f32(M, N, fmt, negate_a, negate_b) | (1u << 15) | (1u << 16);
 }
 
 // bf16 A and B
