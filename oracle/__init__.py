@@ -20,6 +20,8 @@ module only marshals numpy arrays to it.  Functions:
 * :func:`backward_dx`, :func:`backward_dw` -- the gradients of a loss with
   respect to x, and to w and bias, by the chain rule on the definition (the
   backward pass of section "Implementacion");
+* :func:`gelu`, :func:`mlp_forward` -- the MLP block y = L2(GELU(L1(x))) of the
+  network-level results (section "A Nivel de Red"), GELU(v) = v * Phi(v);
 * :func:`dense_flops`, :func:`fourier_flops` -- the operation counts of the
   naive and the Fourier-domain contraction (sections "Enfoque Algoritmico",
   "Especializacion para el Grupo de Rotacion p4").
@@ -49,13 +51,15 @@ def _load():
         lib.eqlin_oracle_irdft_f64.argtypes = [dp, dp, i64, i64, dp]
         lib.eqlin_oracle_backward_dx_f64.argtypes = [dp, dp, i64, i64, i64, i64, dp, ip]
         lib.eqlin_oracle_backward_dw_f64.argtypes = [dp, dp, i64, i64, i64, i64, dp, dp, ip]
+        lib.eqlin_oracle_gelu_f64.argtypes = [dp, i64, dp]
+        lib.eqlin_oracle_mlp_f64.argtypes = [dp, dp, dp, dp, dp, i64, i64, i64, i64, i64, dp, ip]
         lib.eqlin_oracle_num_freqs.argtypes = [i64]
         lib.eqlin_oracle_num_freqs.restype = i64
         lib.eqlin_oracle_max_threads.restype = ctypes.c_int
         for f in ("eqlin_oracle_forward_f64", "eqlin_oracle_forward_fourier_f64",
                   "eqlin_oracle_dense_weight_f64", "eqlin_oracle_rdft_f64",
                   "eqlin_oracle_irdft_f64", "eqlin_oracle_backward_dx_f64",
-                  "eqlin_oracle_backward_dw_f64"):
+                  "eqlin_oracle_backward_dw_f64", "eqlin_oracle_gelu_f64", "eqlin_oracle_mlp_f64"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -148,6 +152,31 @@ def backward_dw(dy, x, threads: int = 0) -> tuple[np.ndarray, np.ndarray]:
                                               int(threads))
     _check(st, "backward_dw")
     return dw, db
+
+
+def gelu(v) -> np.ndarray:
+    """GELU(v) = v * Phi(v) elementwise, Phi the standard normal CDF (erf form), float64."""
+    v = _f64(v)
+    out = np.empty_like(v)
+    _check(_load().eqlin_oracle_gelu_f64(_ptr(v), v.size, _ptr(out)), "gelu")
+    return out
+
+
+def mlp_forward(x, w1, b1, w2, b2, threads: int = 0) -> np.ndarray:
+    """MLP block y = L2(GELU(L1(x))): x [N, Cin, G], w1 [H, Cin, G], b1 [H] or None,
+    w2 [Cout, H, G], b2 [Cout] or None -> y [N, Cout, G], float64."""
+    x, w1, w2 = _f64(x), _f64(w1), _f64(w2)
+    N, Cin, G = x.shape
+    H, Cout = w1.shape[0], w2.shape[0]
+    if w1.shape != (H, Cin, G) or w2.shape != (Cout, H, G):
+        raise ValueError("w1 must be [H, Cin, G] and w2 [Cout, H, G]")
+    c1 = None if b1 is None else _f64(b1).reshape(H)
+    c2 = None if b2 is None else _f64(b2).reshape(Cout)
+    y = np.empty((N, Cout, G), dtype=np.float64)
+    st = _load().eqlin_oracle_mlp_f64(_ptr(x), _ptr(w1), None if c1 is None else _ptr(c1), _ptr(w2),
+                                      None if c2 is None else _ptr(c2), N, Cin, H, Cout, G, _ptr(y), int(threads))
+    _check(st, "mlp_forward")
+    return y
 
 
 def dense_weight(w) -> np.ndarray:

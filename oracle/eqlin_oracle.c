@@ -47,6 +47,18 @@
  *                                   (dx is the transpose of the dense
  *                                   block-circulant matrix applied to dy, a
  *                                   circular correlation along the group axis).
+ *   eqlin_oracle_gelu_f64 /
+ *   eqlin_oracle_mlp_f64            an equivariant MLP block of two EQ-Linear
+ *                                   layers with a pointwise GELU between them,
+ *                                   y = L2(GELU(L1(x))), the block the page's
+ *                                   network-level results (section "A Nivel de
+ *                                   Red": Flash EQ-ViT / EQ-Swin) are built from.
+ *                                   GELU(v) = v * Phi(v), Phi the standard normal
+ *                                   CDF, Phi(v) = (1 + erf(v / sqrt 2)) / 2 (the
+ *                                   exact form; the page does not name a variant).
+ *                                   A pointwise function of each (channel, group
+ *                                   element) commutes with cyclic shifts, so the
+ *                                   block stays equivariant.
  *
  * Readings of points the page leaves open (each is also listed in the design
  * notes of the repository):
@@ -344,4 +356,33 @@ int eqlin_oracle_backward_dw_f64(const double* dy, const double* x,
         }
     }
     return ORACLE_OK;
+}
+
+/* GELU from its definition: v * Phi(v), Phi(v) = (1 + erf(v / sqrt(2))) / 2. */
+static double gelu(double v) { return 0.5 * v * (1.0 + erf(v * 0.70710678118654752440084436210484904)); }
+
+int eqlin_oracle_gelu_f64(const double* v, int64_t n, double* out) {
+    if (n < 0 || (n > 0 && (!v || !out))) return ORACLE_BAD_ARG;
+    for (int64_t k = 0; k < n; ++k) out[k] = gelu(v[k]);
+    return ORACLE_OK;
+}
+
+/*
+ * MLP block y = L2(GELU(L1(x))) with L1 = EQ-Linear(w1 [H, Cin, G], b1 [H] or NULL) and
+ * L2 = EQ-Linear(w2 [Cout, H, G], b2 [Cout] or NULL), each by the definition loops of
+ * eqlin_oracle_forward_f64.  x [N, Cin, G], y [N, Cout, G].
+ */
+int eqlin_oracle_mlp_f64(const double* x, const double* w1, const double* b1, const double* w2,
+                         const double* b2, int64_t N, int64_t Cin, int64_t H, int64_t Cout, int64_t G,
+                         double* y, int nthreads) {
+    if (N < 0 || Cin <= 0 || H <= 0 || Cout <= 0 || G <= 0 || !w1 || !w2) return ORACLE_BAD_ARG;
+    if (N == 0) return ORACLE_OK;
+    if (!x || !y) return ORACLE_BAD_ARG;
+    double* h = (double*)malloc(sizeof(double) * (size_t)(N * H * G));
+    if (!h) return ORACLE_BAD_ARG;
+    int st = eqlin_oracle_forward_f64(x, w1, b1, N, Cin, H, G, h, nthreads);
+    if (st == ORACLE_OK) st = eqlin_oracle_gelu_f64(h, N * H * G, h);
+    if (st == ORACLE_OK) st = eqlin_oracle_forward_f64(h, w2, b2, N, H, Cout, G, y, nthreads);
+    free(h);
+    return st;
 }
