@@ -277,6 +277,8 @@ def main() -> None:
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-mlp-block", action="store_true",
+                    help="skip the extra measurement of the equivariant MLP block L2(GELU(L1(x))), H = 4 C")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the extra measurement of the backward calls (input and weight gradients)")
     ap.add_argument("--tokens", type=int, default=None,
@@ -423,6 +425,38 @@ def main() -> None:
                                 "float64 CUDA-core kernel (clear + kernel + convert)"}
         del dxs
 
+    # ----------------------------------------------------------- MLP block
+    # The equivariant MLP block y = L2(GELU(L1(x))) at the workload's channels with a
+    # 4x hidden layer (16-bit square workloads): two fused launches, GELU in the first
+    # one's epilogue, the hidden activation through HBM.  Timed like the backward calls.
+    mlp = None
+    if not args.no_mlp_block and wl.io_dtype != "f32" and wl.Cin == wl.Cout:
+        H = 4 * wl.Cin
+        w1, b1, w2, b2 = workloads.make_mlp_weights(wl, H)
+        h1 = eq.prepare(w1.to(dev), b1.to(dev), io_dtype=wl.torch_dtype, activation="gelu")
+        h2 = eq.prepare(w2.to(dev), b2.to(dev), io_dtype=wl.torch_dtype)
+        hidden = torch.empty(N, H, wl.G, dtype=wl.torch_dtype, device=dev)
+        Kb = max(10, min(K, 200))
+        for i in range(max(3, args.warmup)):
+            eq.mlp_block(h1, h2, xs[i % n_sets], hidden=hidden, out=ys[i % n_sets], stream=stream)
+        barrier()
+        torch.cuda.synchronize(dev)
+        m0 = torch.cuda.Event(enable_timing=True)
+        m1 = torch.cuda.Event(enable_timing=True)
+        m0.record(stream)
+        for i in range(Kb):
+            eq.mlp_block(h1, h2, xs[i % n_sets], hidden=hidden, out=ys[i % n_sets], stream=stream)
+        m1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        us = 1e3 * reduce_max(m0.elapsed_time(m1), dev) / Kb
+        mlp = {"H": H, "us_per_block": us, "calls": Kb, "launches_per_block": 2,
+               "device_status": max(h1.device_status(), h2.device_status(), key=abs),
+               "tokens_per_s": N / (us * 1e-6)}
+        del hidden
+        h1.close()
+        h2.close()
+
     # ----------------------------------------------------------- CPU baseline
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -459,6 +493,20 @@ def main() -> None:
     roof["tensor_tflops"] = tflops
     roof["tensor_frac"] = tflops / peaks["bf16_tflops"]
 
+    if mlp is not None:
+        e, H = wl.elem_bytes, mlp["H"]
+        # two launches: x in, hidden out and back in, y out, both weight sets
+        mbytes = N * (wl.Cin + 2 * H + wl.Cout) * wl.G * e + 2 * wl.G * wl.Cin * H * e
+        mflops = 2 * N * wl.Cin * H * (2 * wl.G - 2) + 2 * N * H * wl.Cout * (2 * wl.G - 2)
+        t_mh = mbytes / (peaks["hbm_gbs"] * 1e9)
+        t_mt = mflops / (peaks["bf16_tflops"] * 1e12)
+        t = mlp["us_per_block"] * 1e-6
+        mlp.update({"bytes": mbytes, "fourier_flops": mflops, "roofline_time_us": 1e6 * max(t_mh, t_mt),
+                    "bound": "hbm" if t_mh >= t_mt else "tensor", "frac_of_roofline_time": max(t_mh, t_mt) / t,
+                    "fused_block_roofline_us": 1e6 * max(N * (wl.Cin + wl.Cout) * wl.G * e / (peaks["hbm_gbs"] * 1e9),
+                                                         t_mt),
+                    "note": "roofline of the two-launch form (hidden activation through HBM); "
+                            "fused_block_roofline_us is the bound of a single fused kernel"})
     if bwd is not None:
         bb = backward_bytes(wl, N)
         for key in ("dx", "dw"):
@@ -499,6 +547,7 @@ def main() -> None:
         "device_status": status,
         "cpu_baseline": cpu,
         "backward": bwd,
+        "mlp_block": mlp,
     })
     h.close()
 

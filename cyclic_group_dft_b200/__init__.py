@@ -31,6 +31,7 @@ from ._capi import (  # noqa: F401
     EQLIN_F32,
     EQLIN_OK,
     EQLIN_PREPARE_BACKWARD,
+    EQLIN_PREPARE_GELU,
     LIB_PATH,
     PATH_NAMES,
     EqlinError,
@@ -50,6 +51,7 @@ from ._capi import (  # noqa: F401
     eqlin_version,
     header_functions,
     library,
+    mlp_block,
 )
 
 prepare = eqlin_prepare_weights

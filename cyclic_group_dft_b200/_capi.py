@@ -29,10 +29,11 @@ EQLIN_ERR_OOM = -5
 EQLIN_ERR_TIMEOUT = -6
 
 EQLIN_PREPARE_BACKWARD = 1
+EQLIN_PREPARE_GELU = 2
 
 ATTRS = {
     "G": 0, "Cin": 1, "Cout": 2, "io_dtype": 3, "path": 4, "tokens_per_tile": 5,
-    "stages": 6, "smem_bytes": 7, "max_grid": 8, "weight_bytes": 9,
+    "stages": 6, "smem_bytes": 7, "max_grid": 8, "weight_bytes": 9, "activation": 10,
 }
 PATH_NAMES = {0: "tcgen05_tokens_on_n_resident_weights", 1: "tcgen05_tokens_on_n_streamed_weights",
               2: "fp32_fp64_arithmetic", 3: "tcgen05_tokens_on_m_resident_weights",
@@ -211,10 +212,14 @@ class Handle:
 
 
 def eqlin_prepare_weights(w: torch.Tensor, bias: torch.Tensor | None = None,
-                          io_dtype: torch.dtype | None = None, stream=None, backward: bool = False) -> Handle:
+                          io_dtype: torch.dtype | None = None, stream=None, backward: bool = False,
+                          activation: str | None = None) -> Handle:
     """Transform w [Cout, Cin, G] (and bias [Cout]) to the frequency domain on w's device.
     backward=True also prepares the input-gradient weights (eqlin_prepare_weights_ex with
-    EQLIN_PREPARE_BACKWARD), for Handle.backward_dx."""
+    EQLIN_PREPARE_BACKWARD), for Handle.backward_dx.  activation="gelu" makes the forward
+    apply GELU after the bias (EQLIN_PREPARE_GELU)."""
+    if activation not in (None, "gelu"):
+        raise ValueError(f"unsupported activation {activation!r}")
     if w.dim() != 3:
         raise ValueError("w must be [Cout, Cin, G]")
     if w.device.type != "cuda":
@@ -232,7 +237,8 @@ def eqlin_prepare_weights(w: torch.Tensor, bias: torch.Tensor | None = None,
     with torch.cuda.device(w.device):
         st = _lib.eqlin_prepare_weights_ex(
             w.data_ptr(), None if bias is None else bias.data_ptr(), Cout, Cin, G,
-            _TORCH_TO_EQLIN[w.dtype], io, EQLIN_PREPARE_BACKWARD if backward else 0,
+            _TORCH_TO_EQLIN[w.dtype], io,
+            (EQLIN_PREPARE_BACKWARD if backward else 0) | (EQLIN_PREPARE_GELU if activation == "gelu" else 0),
             _stream_ptr(stream), ctypes.byref(out))
     _check(st, "eqlin_prepare_weights_ex")
     return Handle(out.value, w.device)
@@ -314,6 +320,19 @@ def eqlin_backward_dw(h: Handle, x: torch.Tensor, dy: torch.Tensor, with_bias: b
                                       workspace.data_ptr(), workspace.numel(), _stream_ptr(stream)),
                "eqlin_backward_dw")
     return dw, dbias
+
+
+def mlp_block(h1: Handle, h2: Handle, x: torch.Tensor, hidden: torch.Tensor | None = None,
+              out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """The equivariant MLP block y = L2(GELU(L1(x))): a forward of h1 (prepared with
+    activation="gelu") into `hidden` [N, H, G], then a forward of h2.  Two launches on one
+    stream; the second one's prologue overlaps the first one's tail."""
+    if h1.attr("activation") != 1:
+        raise ValueError("h1 must be prepared with activation='gelu'")
+    if h1.Cout != h2.Cin or h1.G != h2.G or h1.io_dtype != h2.io_dtype or h1.device != h2.device:
+        raise ValueError("h1's outputs must match h2's inputs (channels, G, dtype, device)")
+    hidden = eqlin_forward(h1, x, hidden, stream)
+    return eqlin_forward(h2, hidden, out, stream)
 
 
 def eqlin_destroy(h: Handle) -> None:

@@ -385,6 +385,7 @@ struct WeightBuffers {
     double* bias_f64 = nullptr;   // fp32-I/O path only
     int* status = nullptr;
     bool has_bias = false;
+    int act = eqlin::kActNone;   // epilogue activation of the forward (EQLIN_PREPARE_GELU)
 };
 
 // Cout x Cin is the operator's shape.  adjoint: the operator is the layer's input
@@ -442,10 +443,10 @@ int launch_forward(const Plan& pl, int64_t Cout, int64_t Cin, int64_t G, int sm_
         float* yf = static_cast<float*>(y);
         const int iCin = static_cast<int>(Cin), iCout = static_cast<int>(Cout);
         switch (iG) {
-            case 2: eqlin::eqlin_fwd_f32_kernel<2><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, b.w_f64, b.bias_f64, yf, N, iCin, iCout); break;
-            case 4: eqlin::eqlin_fwd_f32_kernel<4><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, b.w_f64, b.bias_f64, yf, N, iCin, iCout); break;
-            case 8: eqlin::eqlin_fwd_f32_kernel<8><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, b.w_f64, b.bias_f64, yf, N, iCin, iCout); break;
-            default: eqlin::eqlin_fwd_f32_kernel<16><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, b.w_f64, b.bias_f64, yf, N, iCin, iCout); break;
+            case 2: eqlin::eqlin_fwd_f32_kernel<2><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, b.w_f64, b.bias_f64, yf, N, iCin, iCout, b.act); break;
+            case 4: eqlin::eqlin_fwd_f32_kernel<4><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, b.w_f64, b.bias_f64, yf, N, iCin, iCout, b.act); break;
+            case 8: eqlin::eqlin_fwd_f32_kernel<8><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, b.w_f64, b.bias_f64, yf, N, iCin, iCout, b.act); break;
+            default: eqlin::eqlin_fwd_f32_kernel<16><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, b.w_f64, b.bias_f64, yf, N, iCin, iCout, b.act); break;
         }
     } else {
         auto encode = tensor_map_encoder();
@@ -497,6 +498,7 @@ int launch_forward(const Plan& pl, int64_t Cout, int64_t Cin, int64_t G, int sm_
             p.w_region_bytes = pl.w_region_bytes;
             p.w_img_bytes = pl.w_img_bytes;
             p.timeout_ns = timeout_ns;
+            p.act = b.act;
             const TmEntry entry = tm_entry_for(iG, pl.streamed(), pl.io);
             if (!entry.launch) return fail(EQLIN_ERR_UNSUPPORTED, "G");
             entry.launch(grid, pl.smem_bytes, st, map, ymap, p);
@@ -517,6 +519,7 @@ int launch_forward(const Plan& pl, int64_t Cout, int64_t Cin, int64_t G, int sm_
             p.ybufs = pl.ybufs;
             p.w_img_bytes = pl.w_img_bytes;
             p.timeout_ns = timeout_ns;
+            p.act = b.act;
             const TcEntry entry = tc_entry_for(iG, pl.streamed(), pl.nacc, pl.io);
             if (!entry.launch) return fail(EQLIN_ERR_UNSUPPORTED, "G");
             entry.launch(grid, pl.smem_bytes, st, map, ymap, p);
@@ -544,12 +547,24 @@ struct DwPlan {
 uint32_t round_kb(size_t v) { return static_cast<uint32_t>((v + 1023) / 1024 * 1024); }
 int round16(int64_t v) { return static_cast<int>((v + 15) / 16 * 16); }
 
-// Channels per TMA box: the largest divisor d of C with d*G <= 256 elements and
-// 16-byte box rows (C is a multiple of 16, so d = 16 always qualifies).
-int box_channels(int C, int G) {
+// Channels per TMA box: the largest divisor d of C with d*G <= 256 elements, 16-byte
+// box rows and d a multiple of `unit` (the channels of one transform unit); C is a
+// multiple of 16, so d = 16 always qualifies.
+int box_channels(int C, int G, int unit) {
     for (int d = C; d >= 1; --d)
-        if (C % d == 0 && d * G <= 256 && (d * G * 2) % 16 == 0) return d;
+        if (C % d == 0 && d % unit == 0 && d * G <= 256 && (d * G * 2) % 16 == 0) return d;
     return 0;
+}
+
+int dw_channels_per_unit(int G) { return G <= 4 ? 8 : (G == 8 ? 4 : 2); }
+
+int max_dw_units(int G) {
+    switch (G) {
+        case 2: return eqlin::dw::Cfg<2>::kMaxPasses * eqlin::dw::Cfg<2>::kDftThreads;
+        case 4: return eqlin::dw::Cfg<4>::kMaxPasses * eqlin::dw::Cfg<4>::kDftThreads;
+        case 8: return eqlin::dw::Cfg<8>::kMaxPasses * eqlin::dw::Cfg<8>::kDftThreads;
+        default: return eqlin::dw::Cfg<16>::kMaxPasses * eqlin::dw::Cfg<16>::kDftThreads;
+    }
 }
 
 // Shared memory of the weight-gradient kernel: raw ring (RS stages of the 32-token dy and
@@ -625,10 +640,13 @@ int plan_dw(int64_t Cout, int64_t Cin, int G, size_t max_smem, int sm_count, DwP
     pl->n_ot = static_cast<int>((Cout + best_mo - 1) / best_mo);
     pl->n_it = static_cast<int>((Cin + best_ni - 1) / best_ni);
     pl->max_splits = std::max(1, sm_count / pl->units());
-    pl->cpb_dy = box_channels(best_mo, G);
-    pl->cpb_x = box_channels(best_ni, G);
-    // the transform's channel pairs never straddle two boxes
-    if (pl->cpb_dy % 2 != 0 || pl->cpb_x % 2 != 0) return fail(EQLIN_ERR_UNSUPPORTED, "odd TMA box width");
+    // a transform unit (dw::Cfg<G>::kChanPerUnit channels) never straddles two boxes
+    const int cpu = dw_channels_per_unit(G);
+    pl->cpb_dy = box_channels(best_mo, G, cpu);
+    pl->cpb_x = box_channels(best_ni, G, cpu);
+    if (pl->cpb_dy == 0 || pl->cpb_x == 0) return fail(EQLIN_ERR_UNSUPPORTED, "no TMA box width for the tile");
+    if (eqlin::dw::kTok * (best_mo + best_ni) / cpu > max_dw_units(G))
+        return fail(EQLIN_ERR_UNSUPPORTED, "weight-gradient tile has more transform units than threads can hold");
     dw_smem(best_mo, best_ni, G, rs, sb, pl);
     int cols = 32;
     while (cols < G * best_ni) cols *= 2;
@@ -838,7 +856,8 @@ int eqlin_prepare_weights_ex(const void* w, const void* bias, int64_t Cout, int6
                              int io_dtype, unsigned flags, void* stream, eqlin_handle** out) {
     if (!out) return fail(EQLIN_ERR_INVALID_ARG, "out is NULL");
     *out = nullptr;
-    if (flags & ~static_cast<unsigned>(EQLIN_PREPARE_BACKWARD)) return fail(EQLIN_ERR_INVALID_ARG, "unknown flags");
+    if (flags & ~static_cast<unsigned>(EQLIN_PREPARE_BACKWARD | EQLIN_PREPARE_GELU))
+        return fail(EQLIN_ERR_INVALID_ARG, "unknown flags");
     if (!w) return fail(EQLIN_ERR_INVALID_ARG, "w is NULL");
     int s = check_shape_impl(Cout, Cin, G, w_dtype, io_dtype);
     if (s != EQLIN_OK) return s;
@@ -873,6 +892,7 @@ int eqlin_prepare_weights_ex(const void* w, const void* bias, int64_t Cout, int6
     h->io_dtype = io_dtype;
     h->plan = plan;
     h->buf.has_bias = bias != nullptr;
+    h->buf.act = (flags & EQLIN_PREPARE_GELU) ? eqlin::kActGelu : eqlin::kActNone;
     const char* sc = std::getenv("EQLIN_SYNC_CHECK");
     h->sync_check = sc && sc[0] == '1';
     if (const char* t = std::getenv("EQLIN_WAIT_TIMEOUT_MS")) {
@@ -1099,6 +1119,7 @@ int eqlin_get_attr(const eqlin_handle* h, int attr, int64_t* value) {
             *value = pl.path == kPathF32 ? static_cast<int64_t>(h->G * h->Cin * h->Cout * 8)
                                          : static_cast<int64_t>(pl.img_alloc_bytes);
             break;
+        case EQLIN_ATTR_ACTIVATION: *value = h->buf.act; break;
         default: return fail(EQLIN_ERR_INVALID_ARG, "unknown attribute");
     }
     return EQLIN_OK;

@@ -22,28 +22,29 @@
 //               N, Cout, Cin).
 //   warp 1      MMA issuer + TMEM owner: per chunk and 16-token K step, tcgen05.mma with
 //               A = DY^ plane [128 rows (MO valid) x 16 tokens], B = X^ plane [NI x 16],
-//               D plane in TMEM (lane = o, column = i):
+//               both MN-major (channels contiguous, tokens along K), D plane in TMEM
+//               (lane = o, column = i):
 //                 D_0 += DY_0 X_0, D_1 += DY_{G/2} X_{G/2},
 //                 Re: D_2k   += DYr Xr + DYi Xi,   Im: D_2k+1 += DYi Xr - DYr Xi
 //               (the minus through the descriptor's negate-A bit).
-//   warps 2..    transpose + DFT (dw::Cfg<G>::kDftWarps warps): a unit of work is one
-//               channel x 8 tokens; the thread
-//               loads the 8 tokens' G-vectors of all its units of the chunk first (lanes =
-//               32 consecutive channels, so the loads are contiguous), then runs the real
-//               DFT over G in fp32 registers (token pairs packed as fx2), packs
-//               each plane's 8 values to bf16 and writes one 16-byte piece per plane
-//               into the K-major SWIZZLE_64B spectra (row = channel, 64-byte row = the
-//               chunk's 32 tokens).  The dy threads also sum plane 0 (the group sum) for
-//               dbias, in a fixed order.  Spectra use p.spec_bufs buffers.
+//   warps 2..   DFT (dw::Cfg<G>::kDftWarps warps): a unit of work is one token x a few
+//               consecutive channels (lanes = consecutive units, so loads and stores
+//               are contiguous); a thread first loads all of its units of a pass, then
+//               runs the real DFT over G in fp32 registers (channel pairs packed as fx2),
+//               packs each plane to the I/O type and writes one store per plane into the
+//               MN-major SWIZZLE_64B spectra.  The dy units also add plane 0 (the group
+//               sum) to a per-token slot for dbias, each slot with a single writer, so the
+//               sums are formed in a fixed order.  Spectra use p.spec_bufs buffers.
 //               After the last chunk the same warps read the TMEM partial dW and write it
 //               to the CTA's slab of the workspace.
 // eqlin_dw_reduce_kernel then sums the slabs of each unit over its token splits in a
 // fixed order (deterministic, float64) and eqlin_dw_idft_kernel<G> runs the inverse real
 // DFT over the planes in float64 and writes dw (fp32) and dbias (fp32).
 //
-// The dy spectra of plane p start at row p*MO of the A region; an MMA reads 128 rows
-// from there, so rows MO..127 of its D are other planes' data (never read back).  The
-// A region holds G*MO + (128 - MO) rows, the tail zeroed once.
+// Spectra layout (one buffer): A = G planes of 4 K-groups x MA atoms of 512 bytes
+// (MA = ceil(MO / 32)), then slack: a 128-row MMA reads 4 atoms along M, so for MO < 128
+// it reads into the next K group (or the slack after the last plane); those D rows are
+// never read back.  B = G planes of 4 x NA atoms (NA = ceil(NI / 32)).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -93,7 +94,14 @@ struct Cfg {
     static constexpr int kDftWarps = 16;
     static constexpr int kDftThreads = kDftWarps * 32;
     static constexpr int kThreads = (2 + kDftWarps) * 32;
-    static constexpr int kUnitsPerPass = 16 / G;            // pairs a thread batches per pass
+    // channels per transform unit: one 16-byte store per plane for G <= 4, 8 bytes for
+    // G = 8, 4 bytes for G = 16 (where the DFT itself dominates and threads are plenty)
+    static constexpr int kChanPerUnit = G <= 4 ? 8 : (G == 8 ? 4 : 2);
+    // units per transform thread and chunk, at most: 32 tokens x (MO + NI) / kChanPerUnit
+    // with MO <= 128 and G * NI <= 512, NI <= 256
+    static constexpr int kMaxUnits = 32 * (128 + (512 / G < 256 ? 512 / G : 256)) / kChanPerUnit;
+    static constexpr int kMaxPasses = (kMaxUnits + kDftThreads - 1) / kDftThreads;
+
 };
 constexpr int kBarDft = 1;         // named barrier among the DFT warps
 constexpr uint32_t kWaitSleepNs = 20000;
@@ -134,52 +142,93 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, int* s
 }
 
 
-// One unit of the transform: one token t of the chunk x one channel pair (c, c+1) of
-// the dy tile or of the x tile.  Raw tile layout: boxes of cpb channels (cpb even, so a
-// pair never straddles two boxes), each [32 tokens][cpb*G].  The unit's 2G values are
-// G 32-bit words (channel c in words 0..G/2-1, channel c+1 in the rest).
-template <int G>
-__device__ __forceinline__ void load_pair(const uint8_t* src, uint32_t (&w)[G]) {
-    if constexpr (G == 2) {
-        const uint2 v = *reinterpret_cast<const uint2*>(src);
-        w[0] = v.x;
-        w[1] = v.y;
-    } else {
+// One unit of the transform: one token t of the chunk x CPU consecutive channels
+// c0 .. c0+CPU-1 of the dy tile or of the x tile (CPU = Cfg<G>::kChanPerUnit).  Raw tile
+// layout: boxes of cpb channels (cpb a multiple of CPU, so a unit never straddles two
+// boxes), each [32 tokens][cpb*G].  The unit's CPU*G values are CPU*G/2 32-bit words,
+// channel c0+j in words j*G/2 .. (j+1)*G/2-1.
+template <int G, int CPU>
+__device__ __forceinline__ void load_unit(const uint8_t* src, int lane, uint32_t (&w)[CPU * G / 2]) {
+    constexpr int BYTES = CPU * G * 2;
+    constexpr int PIECES = BYTES / 16;       // 2 or 4 sixteen-byte pieces
+    static_assert(BYTES == 32 || BYTES == 64, "unit size");
+    // Consecutive lanes hold consecutive units, BYTES apart: loading piece q in step q
+    // would put every lane of a step on the same few banks.  Lane l loads piece
+    // (q + rot) % PIECES in step q instead, rot = (l >> s) % PIECES chosen so that the 32
+    // lanes of a step cover all eight 16-byte bank groups, then rotates back.
+    const int rot = (lane >> (PIECES == 4 ? 1 : 2)) & (PIECES - 1);
+    uint4 ld[PIECES];
 #pragma unroll
-        for (int q = 0; q < G / 4; ++q) {
-            const uint4 v = *reinterpret_cast<const uint4*>(src + 16 * q);
-            w[4 * q + 0] = v.x;
-            w[4 * q + 1] = v.y;
-            w[4 * q + 2] = v.z;
-            w[4 * q + 3] = v.w;
+    for (int q = 0; q < PIECES; ++q) ld[q] = *reinterpret_cast<const uint4*>(src + 16 * ((q + rot) & (PIECES - 1)));
+    // piece k sits in ld[(k - rot) % PIECES]: rotate right by rot (in steps of 1 and 2)
+    if (rot & 1) {
+        const uint4 last = ld[PIECES - 1];
+#pragma unroll
+        for (int k = PIECES - 1; k > 0; --k) ld[k] = ld[k - 1];
+        ld[0] = last;
+    }
+    if constexpr (PIECES == 4) {
+        if (rot & 2) {
+            const uint4 a = ld[0], b = ld[1];
+            ld[0] = ld[2];
+            ld[1] = ld[3];
+            ld[2] = a;
+            ld[3] = b;
         }
+    }
+#pragma unroll
+    for (int k = 0; k < PIECES; ++k) {
+        w[4 * k + 0] = ld[k].x;
+        w[4 * k + 1] = ld[k].y;
+        w[4 * k + 2] = ld[k].z;
+        w[4 * k + 3] = ld[k].w;
     }
 }
 
-// Real DFT over G of the pair (the two channels packed as fx2), stored to the planes in
+// Real DFT over G of the unit's channels (in pairs packed as fx2), stored to the planes in
 // the MN-major SWIZZLE_64B operand layout: plane p at plane0 + p * plane_bytes; in it the
 // 8-row atom (kg = t / 8, ma = c / 32) at kg * sbo + ma * 512 holds row t % 8 = 64 bytes
 // of channels 32ma .. 32ma + 31, 16-byte chunk j of row r stored at chunk j ^ ((r >> 1) & 3).
-// Returns plane 0 (the group sums of the two channels).
-template <int G, class T16>
-__device__ __forceinline__ fx2 store_pair(const uint32_t (&w)[G], uint8_t* plane0, uint32_t plane_bytes,
-                                          uint32_t sbo, int t, int c) {
-    fx2 v[G], pl[G];
+// One store of CPU * 2 bytes per plane.  With with_bias, adds plane 0 (the group sums)
+// to the thread's running dbias sums bias[0..CPU) (kept in registers across chunks).
+template <int G, int CPU, class T16>
+__device__ __forceinline__ void store_unit(const uint32_t (&w)[CPU * G / 2], uint8_t* plane0, uint32_t plane_bytes,
+                                           uint32_t sbo, int t, int c0, float (&bias)[CPU], bool with_bias) {
+    constexpr int H = G / 2;
+    uint32_t packed[G][CPU / 2];
 #pragma unroll
-    for (int h = 0; h < G / 2; ++h) {
-        v[2 * h] = fx2(Io16<T16>::lo(w[h]), Io16<T16>::lo(w[G / 2 + h]));
-        v[2 * h + 1] = fx2(Io16<T16>::hi(w[h]), Io16<T16>::hi(w[G / 2 + h]));
+    for (int j = 0; j < CPU / 2; ++j) {      // channels c0 + 2j, c0 + 2j + 1
+        fx2 v[G], pl[G];
+#pragma unroll
+        for (int h = 0; h < H; ++h) {
+            const uint32_t a = w[(2 * j) * H + h], b = w[(2 * j + 1) * H + h];
+            v[2 * h] = fx2(Io16<T16>::lo(a), Io16<T16>::lo(b));
+            v[2 * h + 1] = fx2(Io16<T16>::hi(a), Io16<T16>::hi(b));
+        }
+        rdft_planes<G>(v, pl);
+        if (with_bias) {
+            bias[2 * j] += pl[0].x;
+            bias[2 * j + 1] += pl[0].y;
+        }
+#pragma unroll
+        for (int p = 0; p < G; ++p) packed[p][j] = Io16<T16>::pack(pl[p].x, pl[p].y);
     }
-    rdft_planes<G>(v, pl);
     const int r = t & 7;
-    const uint32_t off = static_cast<uint32_t>(t >> 3) * sbo + static_cast<uint32_t>(c >> 5) * 512u +
+    const uint32_t off = static_cast<uint32_t>(t >> 3) * sbo + static_cast<uint32_t>(c0 >> 5) * 512u +
                          static_cast<uint32_t>(r) * 64u +
-                         static_cast<uint32_t>((((c & 31) >> 3) ^ ((r >> 1) & 3)) << 4) +
-                         static_cast<uint32_t>(c & 7) * 2u;
+                         static_cast<uint32_t>((((c0 & 31) >> 3) ^ ((r >> 1) & 3)) << 4) +
+                         static_cast<uint32_t>(c0 & 7) * 2u;
 #pragma unroll
-    for (int p = 0; p < G; ++p)
-        *reinterpret_cast<uint32_t*>(plane0 + p * plane_bytes + off) = Io16<T16>::pack(pl[p].x, pl[p].y);
-    return pl[0];
+    for (int p = 0; p < G; ++p) {
+        uint8_t* dst = plane0 + p * plane_bytes + off;
+        if constexpr (CPU == 8) {
+            *reinterpret_cast<uint4*>(dst) = make_uint4(packed[p][0], packed[p][1], packed[p][2], packed[p][3]);
+        } else if constexpr (CPU == 4) {
+            *reinterpret_cast<uint2*>(dst) = make_uint2(packed[p][0], packed[p][1]);
+        } else {
+            *reinterpret_cast<uint32_t*>(dst) = packed[p][0];
+        }
+    }
 }
 
 }  // namespace dw
@@ -241,7 +290,7 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
     }
     if (warp >= dw::kWarpDft0) {
         const int t = threadIdx.x - dw::kWarpDft0 * 32;
-        for (int c = t; c < dw::kTok * p.MO; c += kDftThreads) bias_sm[c] = 0.0f;
+
         // A-region tail rows (read by the MMA, never written by the transform): zero
         // A-region slack after the G planes (read by the 128-row MMA of the last plane,
         // never written by the transform): zero
@@ -342,10 +391,18 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
     } else {
         // ------------------------------------------------------------ transform warps
         const int t = threadIdx.x - dw::kWarpDft0 * 32;
-        // units: token t x channel pair; the dy pairs of all tokens first, then x's
-        const int pairs_dy = p.MO / 2, pairs_x = p.NI / 2;
-        const int units_dy = dw::kTok * pairs_dy;
-        const int n_units = units_dy + dw::kTok * pairs_x;
+        // units: token t x CPU channels; the dy units of all tokens first, then x's.  A
+        // thread handles units t + ps * kDftThreads, the same ones in every chunk, so it
+        // keeps the dbias sums of its dy units in registers (bsum) until the end.
+        constexpr int CPU = dw::Cfg<G>::kChanPerUnit;
+        const int groups_dy = p.MO / CPU, groups_x = p.NI / CPU;
+        const int units_dy = dw::kTok * groups_dy;
+        const int n_units = units_dy + dw::kTok * groups_x;
+        float bsum[dw::Cfg<G>::kMaxPasses][CPU];
+#pragma unroll
+        for (int ps = 0; ps < dw::Cfg<G>::kMaxPasses; ++ps)
+#pragma unroll
+            for (int j = 0; j < CPU; ++j) bsum[ps][j] = 0.0f;
         const uint32_t sbo_a = static_cast<uint32_t>(p.MA) * 512u, sbo_b = static_cast<uint32_t>(p.NA) * 512u;
         const uint32_t plane_a = 4u * sbo_a, plane_b = 4u * sbo_b;
         bool ok = true;
@@ -361,39 +418,23 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
             }
             const uint8_t* raw = raw0 + static_cast<size_t>(s) * p.raw_bytes;
             uint8_t* spec = spec0 + static_cast<size_t>(sb) * spec_bytes;
-            constexpr int UPT = dw::Cfg<G>::kUnitsPerPass;
-            for (int base = 0; base < n_units; base += kDftThreads * UPT) {
-                uint32_t words[UPT][G];
-                int ts[UPT], cs[UPT];
 #pragma unroll
-                for (int k = 0; k < UPT; ++k) {
-                    const int u = base + t + k * kDftThreads;
-                    ts[k] = -1;
-                    cs[k] = 0;
-                    if (u < n_units) {
-                        const bool is_dy = u < units_dy;
-                        const int v = is_dy ? u : u - units_dy, np = is_dy ? pairs_dy : pairs_x;
-                        const int tok = v / np, c = 2 * (v - tok * np), cpb = is_dy ? p.cpb_dy : p.cpb_x;
-                        const int box = c / cpb, row_bytes = cpb * G * 2;
-                        const uint8_t* src = raw + (is_dy ? 0u : p.dy_bytes) +
-                                             static_cast<size_t>(box) * (dw::kTok * row_bytes) +
-                                             static_cast<size_t>(tok) * row_bytes + (c - box * cpb) * G * 2;
-                        dw::load_pair<G>(src, words[k]);
-                        ts[k] = tok;
-                        cs[k] = is_dy ? c : -1 - c;     // x pairs carry -1 - c
-                    }
-                }
-#pragma unroll
-                for (int k = 0; k < UPT; ++k) {
-                    if (ts[k] < 0) continue;
-                    if (cs[k] >= 0) {
-                        const fx2 s0 = dw::store_pair<G, T16>(words[k], spec, plane_a, sbo_a, ts[k], cs[k]);
-                        float* bs = bias_sm + ts[k] * p.MO + cs[k];
-                        bs[0] += s0.x;
-                        bs[1] += s0.y;
-                    } else {
-                        dw::store_pair<G, T16>(words[k], spec + p.a_bytes, plane_b, sbo_b, ts[k], -1 - cs[k]);
-                    }
+            for (int ps = 0; ps < dw::Cfg<G>::kMaxPasses; ++ps) {
+                const int u = t + ps * kDftThreads;
+                if (u >= n_units) break;
+                const bool is_dy = u < units_dy;
+                const int v = is_dy ? u : u - units_dy, ng = is_dy ? groups_dy : groups_x;
+                const int tok = v / ng, c = CPU * (v - tok * ng), cpb = is_dy ? p.cpb_dy : p.cpb_x;
+                const int box = c / cpb, row_bytes = cpb * G * 2;
+                const uint8_t* src = raw + (is_dy ? 0u : p.dy_bytes) +
+                                     static_cast<size_t>(box) * (dw::kTok * row_bytes) +
+                                     static_cast<size_t>(tok) * row_bytes + (c - box * cpb) * G * 2;
+                uint32_t words[CPU * G / 2];
+                dw::load_unit<G, CPU>(src, lane, words);
+                if (is_dy) {
+                    dw::store_unit<G, CPU, T16>(words, spec, plane_a, sbo_a, tok, c, bsum[ps], true);
+                } else {
+                    dw::store_unit<G, CPU, T16>(words, spec + p.a_bytes, plane_b, sbo_b, tok, c, bsum[ps], false);
                 }
             }
             ptx::fence_proxy_async_smem();
@@ -427,7 +468,18 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
                 }
             }
         }
-        // dbias partial of this CTA (every CTA writes it; the inverse-DFT kernel reads input tile 0's)
+        // dbias partial of this CTA (every CTA writes it; the inverse-DFT kernel reads input
+        // tile 0's): each thread's register sums to their slots bias_sm[tok][c], then per
+        // channel the 32 token slots in order
+#pragma unroll
+        for (int ps = 0; ps < dw::Cfg<G>::kMaxPasses; ++ps) {
+            const int u = t + ps * kDftThreads;
+            if (u < units_dy) {
+                const int tok = u / groups_dy, c = CPU * (u - tok * groups_dy);
+#pragma unroll
+                for (int j = 0; j < CPU; ++j) bias_sm[tok * p.MO + c + j] = bsum[ps][j];
+            }
+        }
         ptx::named_bar_sync(dw::kBarDft, kDftThreads);
         for (int c = t; c < p.MO; c += kDftThreads) {
             float acc = 0.0f;

@@ -59,6 +59,7 @@ struct TcParams {
     int ybufs;                // 1 or 2 staging buffers per epilogue warp
     uint32_t w_img_bytes;     // bytes of the resident image to copy
     unsigned long long timeout_ns;
+    int act;                  // epilogue activation after the bias: kActNone or kActGelu
 };
 
 namespace tc {
@@ -234,6 +235,10 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, const CUtensorM
                 for (int pl = 0; pl < G; ++pl) z[pl] = __uint_as_float(r[pl][t]);
                 z[0] += b;  // the DC term appears with weight 1 in every output
                 RealIdft<G>::run(z, yv);
+                if (p.act == kActGelu) {
+#pragma unroll
+                    for (int g = 0; g < G; ++g) yv[g] = gelu(yv[g]);
+                }
                 uint8_t* dst = lane_off + t * (YBC * 2);
                 if constexpr (G == 2) {
                     *reinterpret_cast<uint32_t*>(dst) = Io16<T16>::pack(yv[0], yv[1]);

@@ -50,6 +50,7 @@ struct TmParams {
     uint32_t w_region_bytes;  // resident weights (0 when streamed)
     uint32_t w_img_bytes;
     unsigned long long timeout_ns;
+    int act;                // epilogue activation after the bias: kActNone or kActGelu
 };
 
 namespace tm {
@@ -206,6 +207,10 @@ __device__ __forceinline__ void epilogue_tile(const TmParams& p, const CUtensorM
             for (int gg = 0; gg < G; ++gg) {
                 yv[j * G + gg] = y2[gg].x;
                 yv[(j + 1) * G + gg] = y2[gg].y;
+            }
+            if (p.act == kActGelu) {
+#pragma unroll
+                for (int gg = 0; gg < 2 * G; ++gg) yv[j * G + gg] = gelu(yv[j * G + gg]);
             }
         }
         // this buffer was last stored two groups ago: its TMA read must be complete

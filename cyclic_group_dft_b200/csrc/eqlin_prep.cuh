@@ -130,7 +130,7 @@ template <int G>
 __global__ void __launch_bounds__(kF32Threads)
     eqlin_fwd_f32_kernel(const float* __restrict__ x, const double* __restrict__ w_f64,
                          const double* __restrict__ bias_f64, float* __restrict__ y, long long N,
-                         int Cin, int Cout) {
+                         int Cin, int Cout, int act) {
     extern __shared__ double xs[];  // [kF32Tokens][G][Cin] spectrum of the block's tokens
     const long long n0 = static_cast<long long>(blockIdx.x) * kF32Tokens;
     for (int idx = threadIdx.x; idx < kF32Tokens * Cin; idx += kF32Threads) {
@@ -171,6 +171,10 @@ __global__ void __launch_bounds__(kF32Threads)
     z[0] += bias_f64[o];
     double yv[G];
     RealIdft<G, double>::run(z, yv);
+    if (act == kActGelu) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) yv[g] = gelu(yv[g]);
+    }
     float* dst = y + (n * Cout + o) * G;
     if constexpr (G % 4 == 0) {
 #pragma unroll

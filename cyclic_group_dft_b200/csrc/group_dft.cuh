@@ -214,6 +214,16 @@ struct RealIdft<2, T> {
     }
 };
 
+// GELU(v) = v * Phi(v), Phi the standard normal CDF = (1 + erf(v / sqrt 2)) / 2: the
+// pointwise nonlinearity of the equivariant MLP block (applied per channel and group
+// element, so it commutes with cyclic shifts).  erff / erf are CUDA's.
+__device__ __forceinline__ float gelu(float v) { return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f)); }
+__device__ __forceinline__ double gelu(double v) { return 0.5 * v * (1.0 + erf(v * 0.70710678118654752440)); }
+
+// Epilogue activations (after the bias): 0 = none, 1 = GELU.
+constexpr int kActNone = 0;
+constexpr int kActGelu = 1;
+
 // Forward transform straight into plane order.
 template <int G, typename T>
 __device__ __forceinline__ void rdft_planes(const T (&x)[G], T (&p)[G]) {

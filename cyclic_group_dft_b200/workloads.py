@@ -113,3 +113,19 @@ def sample_tokens(N: int, count: int, seed: int = 0) -> torch.Tensor:
     idx = torch.randperm(N, generator=gen)[: max(count - 2, 0)]
     idx = torch.cat([idx, torch.tensor([0, N - 1])])
     return torch.unique(idx)
+
+
+def make_mlp_weights(wl: Workload, hidden: int, seed: int | None = None):
+    """(w1 [H, Cin, G], b1 [H], w2 [Cout, H, G], b2 [Cout]) for the equivariant MLP block
+    L2(GELU(L1(x))) at the workload's channels, as CPU tensors in the I/O dtype:
+    w1 ~ N(0, 1/(Cin*G)), w2 ~ N(0, 1/(H*G)), biases ~ N(0, 0.1) (second parameter the
+    variance), drawn in that order from one generator (seed + 1000 by default, so
+    they differ from the single-layer weights)."""
+    gen = torch.Generator(device="cpu").manual_seed((wl.seed if seed is None else int(seed)) + 1000)
+    G, H = wl.G, int(hidden)
+    w1 = torch.randn(H, wl.Cin, G, generator=gen) * math.sqrt(1.0 / (wl.Cin * G))
+    b1 = torch.randn(H, generator=gen) * math.sqrt(0.1)
+    w2 = torch.randn(wl.Cout, H, G, generator=gen) * math.sqrt(1.0 / (H * G))
+    b2 = torch.randn(wl.Cout, generator=gen) * math.sqrt(0.1)
+    dt = wl.torch_dtype
+    return w1.to(dt), b1.to(dt), w2.to(dt), b2.to(dt)

@@ -150,7 +150,8 @@ enum {
     EQLIN_ATTR_STAGES = 6,          /* depth of the shared-memory ring */
     EQLIN_ATTR_SMEM_BYTES = 7,      /* dynamic shared memory per CTA */
     EQLIN_ATTR_MAX_GRID = 8,        /* CTAs launched for a large N (one per SM) */
-    EQLIN_ATTR_WEIGHT_BYTES = 9     /* bytes of the frequency-domain weights the kernel reads */
+    EQLIN_ATTR_WEIGHT_BYTES = 9,    /* bytes of the frequency-domain weights the kernel reads */
+    EQLIN_ATTR_ACTIVATION = 10      /* epilogue activation of the forward: 0 none, 1 GELU */
 };
 EQLIN_API int eqlin_get_attr(const eqlin_handle* h, int attr, int64_t* value);
 
@@ -234,10 +235,21 @@ EQLIN_API int eqlin_forward_noalloc(const void* x, const void* w, const void* bi
  * weights. */
 #define EQLIN_PREPARE_BACKWARD 1u
 
+/* eqlin_prepare_weights_ex flag: the forward applies GELU after the bias,
+ * y = GELU(bias + EQ-Linear(x)), GELU(v) = v * Phi(v) with Phi the standard normal
+ * CDF (erf form), in the fused epilogue (fp32 for 16-bit I/O, float64 for fp32 I/O).
+ * It is the first half of the equivariant MLP block L2(GELU(L1(x))) of the page's
+ * network-level results (section "A Nivel de Red"); the block is a forward with a
+ * GELU handle followed by a forward with a plain one.  The backward calls of such a
+ * handle compute the gradients of the linear map (before the activation); the
+ * activation's derivative GELU'(h) dy is the caller's. */
+#define EQLIN_PREPARE_GELU 2u
+
 /*
- * eqlin_prepare_weights_ex -- eqlin_prepare_weights with flags (0 or
- * EQLIN_PREPARE_BACKWARD).  eqlin_prepare_weights(...) is this call with flags 0.
- * Errors: as eqlin_prepare_weights; INVALID_ARG for an unknown flag bit.
+ * eqlin_prepare_weights_ex -- eqlin_prepare_weights with flags (0, or any of
+ * EQLIN_PREPARE_BACKWARD | EQLIN_PREPARE_GELU).  eqlin_prepare_weights(...) is this
+ * call with flags 0.  Errors: as eqlin_prepare_weights; INVALID_ARG for an unknown
+ * flag bit.
  */
 EQLIN_API int eqlin_prepare_weights_ex(const void* w, const void* bias, int64_t Cout, int64_t Cin, int64_t G,
                                        int w_dtype, int io_dtype, unsigned flags, void* stream,

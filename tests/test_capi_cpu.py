@@ -135,3 +135,16 @@ def test_backward_entry_points_reject_bad_arguments_on_host():
 def test_header_declares_the_backward_flag():
     text = open(_capi.HEADER_PATH).read()
     assert f"#define EQLIN_PREPARE_BACKWARD {eq.EQLIN_PREPARE_BACKWARD}u" in text
+
+
+def test_gelu_flag_is_declared_and_accepted_on_host():
+    text = open(_capi.HEADER_PATH).read()
+    assert f"#define EQLIN_PREPARE_GELU {eq.EQLIN_PREPARE_GELU}u" in text
+    assert "EQLIN_ATTR_ACTIVATION = 10" in text
+    lib = eq.library()
+    h = ctypes.c_void_p(1234)
+    # both flags together pass the flag check (then fail on the NULL weight pointer)
+    st = lib.eqlin_prepare_weights_ex(None, None, 8, 8, 4, eq.EQLIN_BF16, eq.EQLIN_BF16,
+                                      eq.EQLIN_PREPARE_BACKWARD | eq.EQLIN_PREPARE_GELU, None,
+                                      ctypes.byref(h))
+    assert st == eq.EQLIN_ERR_INVALID_ARG and "NULL" in eq.eqlin_last_error()
