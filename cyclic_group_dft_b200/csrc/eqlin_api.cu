@@ -386,6 +386,7 @@ struct WeightBuffers {
     int* status = nullptr;
     bool has_bias = false;
     int act = eqlin::kActNone;   // epilogue activation of the forward (EQLIN_PREPARE_GELU)
+    long long inject_stop = -1;  // failure-detection test hook (EQLIN_TEST_STOP_AFTER), -1 = off
 };
 
 // Cout x Cin is the operator's shape.  adjoint: the operator is the layer's input
@@ -499,6 +500,7 @@ int launch_forward(const Plan& pl, int64_t Cout, int64_t Cin, int64_t G, int sm_
             p.w_img_bytes = pl.w_img_bytes;
             p.timeout_ns = timeout_ns;
             p.act = b.act;
+            p.inject_stop = b.inject_stop;
             const TmEntry entry = tm_entry_for(iG, pl.streamed(), pl.io);
             if (!entry.launch) return fail(EQLIN_ERR_UNSUPPORTED, "G");
             entry.launch(grid, pl.smem_bytes, st, map, ymap, p);
@@ -520,6 +522,7 @@ int launch_forward(const Plan& pl, int64_t Cout, int64_t Cin, int64_t G, int sm_
             p.w_img_bytes = pl.w_img_bytes;
             p.timeout_ns = timeout_ns;
             p.act = b.act;
+            p.inject_stop = b.inject_stop;
             const TcEntry entry = tc_entry_for(iG, pl.streamed(), pl.nacc, pl.io);
             if (!entry.launch) return fail(EQLIN_ERR_UNSUPPORTED, "G");
             entry.launch(grid, pl.smem_bytes, st, map, ymap, p);
@@ -893,6 +896,14 @@ int eqlin_prepare_weights_ex(const void* w, const void* bias, int64_t Cout, int6
     h->plan = plan;
     h->buf.has_bias = bias != nullptr;
     h->buf.act = (flags & EQLIN_PREPARE_GELU) ? eqlin::kActGelu : eqlin::kActNone;
+    // Test hook for failure detection (read at prepare, never set outside tests): with
+    // EQLIN_TEST_STOP_AFTER=k the fused kernels' producer stops after issuing k chunks per
+    // CTA, so the consumers' bounded waits run out, the kernel records EQLIN_ERR_TIMEOUT
+    // in the status word and exits cleanly.  No fault, trap or unbounded wait is involved.
+    if (const char* e = std::getenv("EQLIN_TEST_STOP_AFTER")) {
+        const long long k = std::atoll(e);
+        if (k >= 0) h->buf.inject_stop = k;
+    }
     const char* sc = std::getenv("EQLIN_SYNC_CHECK");
     h->sync_check = sc && sc[0] == '1';
     if (const char* t = std::getenv("EQLIN_WAIT_TIMEOUT_MS")) {

@@ -186,14 +186,13 @@ __device__ __forceinline__ void load_unit(const uint8_t* src, int lane, uint32_t
 }
 
 // Real DFT over G of the unit's channels (in pairs packed as fx2), stored to the planes in
-// the MN-major SWIZZLE_64B operand layout: plane p at plane0 + p * plane_bytes; in it the
-// 8-row atom (kg = t / 8, ma = c / 32) at kg * sbo + ma * 512 holds row t % 8 = 64 bytes
-// of channels 32ma .. 32ma + 31, 16-byte chunk j of row r stored at chunk j ^ ((r >> 1) & 3).
-// One store of CPU * 2 bytes per plane.  With with_bias, adds plane 0 (the group sums)
-// to the thread's running dbias sums bias[0..CPU) (kept in registers across chunks).
+// the MN-major SWIZZLE_64B operand layout: plane p of the unit at dst + p * plane_bytes
+// (dst from unit_dst_offset).  One store of CPU * 2 bytes per plane.  With with_bias,
+// adds plane 0 (the group sums) to the thread's running dbias sums bias[0..CPU) (kept in
+// registers across chunks).
 template <int G, int CPU, class T16>
-__device__ __forceinline__ void store_unit(const uint32_t (&w)[CPU * G / 2], uint8_t* plane0, uint32_t plane_bytes,
-                                           uint32_t sbo, int t, int c0, float (&bias)[CPU], bool with_bias) {
+__device__ __forceinline__ void store_unit(const uint32_t (&w)[CPU * G / 2], uint8_t* dst, uint32_t plane_bytes,
+                                           float (&bias)[CPU], bool with_bias) {
     constexpr int H = G / 2;
     uint32_t packed[G][CPU / 2];
 #pragma unroll
@@ -213,22 +212,26 @@ __device__ __forceinline__ void store_unit(const uint32_t (&w)[CPU * G / 2], uin
 #pragma unroll
         for (int p = 0; p < G; ++p) packed[p][j] = Io16<T16>::pack(pl[p].x, pl[p].y);
     }
-    const int r = t & 7;
-    const uint32_t off = static_cast<uint32_t>(t >> 3) * sbo + static_cast<uint32_t>(c0 >> 5) * 512u +
-                         static_cast<uint32_t>(r) * 64u +
-                         static_cast<uint32_t>((((c0 & 31) >> 3) ^ ((r >> 1) & 3)) << 4) +
-                         static_cast<uint32_t>(c0 & 7) * 2u;
 #pragma unroll
     for (int p = 0; p < G; ++p) {
-        uint8_t* dst = plane0 + p * plane_bytes + off;
+        uint8_t* d = dst + p * plane_bytes;
         if constexpr (CPU == 8) {
-            *reinterpret_cast<uint4*>(dst) = make_uint4(packed[p][0], packed[p][1], packed[p][2], packed[p][3]);
+            *reinterpret_cast<uint4*>(d) = make_uint4(packed[p][0], packed[p][1], packed[p][2], packed[p][3]);
         } else if constexpr (CPU == 4) {
-            *reinterpret_cast<uint2*>(dst) = make_uint2(packed[p][0], packed[p][1]);
+            *reinterpret_cast<uint2*>(d) = make_uint2(packed[p][0], packed[p][1]);
         } else {
-            *reinterpret_cast<uint32_t*>(dst) = packed[p][0];
+            *reinterpret_cast<uint32_t*>(d) = packed[p][0];
         }
     }
+}
+
+// Offset of channel c0 of token t in a plane of the MN-major SWIZZLE_64B layout: the 8-row
+// atom (kg = t / 8, ma = c0 / 32) at kg * sbo + ma * 512 holds row t % 8 = 64 bytes of
+// channels 32ma .. 32ma + 31, 16-byte chunk j of row r stored at chunk j ^ ((r >> 1) & 3).
+__device__ __forceinline__ uint32_t unit_dst_offset(int t, int c0, uint32_t sbo) {
+    const int r = t & 7;
+    return static_cast<uint32_t>(t >> 3) * sbo + static_cast<uint32_t>(c0 >> 5) * 512u + static_cast<uint32_t>(r) * 64u +
+           static_cast<uint32_t>((((c0 & 31) >> 3) ^ ((r >> 1) & 3)) << 4) + static_cast<uint32_t>(c0 & 7) * 2u;
 }
 
 }  // namespace dw
@@ -405,37 +408,48 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
             for (int j = 0; j < CPU; ++j) bsum[ps][j] = 0.0f;
         const uint32_t sbo_a = static_cast<uint32_t>(p.MA) * 512u, sbo_b = static_cast<uint32_t>(p.NA) * 512u;
         const uint32_t plane_a = 4u * sbo_a, plane_b = 4u * sbo_b;
+        // the thread's units are the same in every chunk: their source offsets in a raw
+        // stage and destination offsets in a spectra buffer are computed once
+        constexpr int MP = dw::Cfg<G>::kMaxPasses;
+        uint32_t src_off[MP], dst_off[MP];
+        uint32_t dy_mask = 0, valid_mask = 0;
+#pragma unroll
+        for (int ps = 0; ps < MP; ++ps) {
+            const int u = t + ps * kDftThreads;
+            src_off[ps] = dst_off[ps] = 0;
+            if (u < n_units) {
+                const bool is_dy = u < units_dy;
+                const int v = is_dy ? u : u - units_dy, ng = is_dy ? groups_dy : groups_x;
+                const int tok = v / ng, c = CPU * (v - tok * ng), cpb = is_dy ? p.cpb_dy : p.cpb_x;
+                const int box = c / cpb, row_bytes = cpb * G * 2;
+                src_off[ps] = (is_dy ? 0u : p.dy_bytes) + static_cast<uint32_t>(box * (dw::kTok * row_bytes) +
+                                                                                 tok * row_bytes + (c - box * cpb) * G * 2);
+                dst_off[ps] = (is_dy ? 0u : p.a_bytes) + dw::unit_dst_offset(tok, c, is_dy ? sbo_a : sbo_b);
+                valid_mask |= 1u << ps;
+                if (is_dy) dy_mask |= 1u << ps;
+            }
+        }
         bool ok = true;
         for (int j = 0; j < n_mine; ++j) {
             const int s = j % RS, sb = j % SB;
             const uint32_t ph_raw = static_cast<uint32_t>(j / RS) & 1u;
             const uint32_t ph_spec = static_cast<uint32_t>(j / SB) & 1u;
-            bool got = dw::wait_bounded(bar_raw_full(s), ph_raw, ctl, p.status, p.timeout_ns);
-            if (got) got = dw::wait_bounded(bar_spec_empty(sb), ph_spec ^ 1u, ctl, p.status, p.timeout_ns);
-            if (!ptx::named_bar_and(dw::kBarDft, kDftThreads, got)) {
+            // no barrier among the transform warps: each thread waits for itself, and a
+            // timeout (which sets the abort flag for every role) ends the loop for all
+            if (!dw::wait_bounded(bar_raw_full(s), ph_raw, ctl, p.status, p.timeout_ns) ||
+                !dw::wait_bounded(bar_spec_empty(sb), ph_spec ^ 1u, ctl, p.status, p.timeout_ns)) {
                 ok = false;
                 break;
             }
             const uint8_t* raw = raw0 + static_cast<size_t>(s) * p.raw_bytes;
             uint8_t* spec = spec0 + static_cast<size_t>(sb) * spec_bytes;
 #pragma unroll
-            for (int ps = 0; ps < dw::Cfg<G>::kMaxPasses; ++ps) {
-                const int u = t + ps * kDftThreads;
-                if (u >= n_units) break;
-                const bool is_dy = u < units_dy;
-                const int v = is_dy ? u : u - units_dy, ng = is_dy ? groups_dy : groups_x;
-                const int tok = v / ng, c = CPU * (v - tok * ng), cpb = is_dy ? p.cpb_dy : p.cpb_x;
-                const int box = c / cpb, row_bytes = cpb * G * 2;
-                const uint8_t* src = raw + (is_dy ? 0u : p.dy_bytes) +
-                                     static_cast<size_t>(box) * (dw::kTok * row_bytes) +
-                                     static_cast<size_t>(tok) * row_bytes + (c - box * cpb) * G * 2;
+            for (int ps = 0; ps < MP; ++ps) {
+                if (!(valid_mask & (1u << ps))) break;
                 uint32_t words[CPU * G / 2];
-                dw::load_unit<G, CPU>(src, lane, words);
-                if (is_dy) {
-                    dw::store_unit<G, CPU, T16>(words, spec, plane_a, sbo_a, tok, c, bsum[ps], true);
-                } else {
-                    dw::store_unit<G, CPU, T16>(words, spec + p.a_bytes, plane_b, sbo_b, tok, c, bsum[ps], false);
-                }
+                dw::load_unit<G, CPU>(raw + src_off[ps], lane, words);
+                const bool is_dy = dy_mask & (1u << ps);
+                dw::store_unit<G, CPU, T16>(words, spec + dst_off[ps], is_dy ? plane_a : plane_b, bsum[ps], is_dy);
             }
             ptx::fence_proxy_async_smem();
             ptx::mbar_arrive(bar_raw_empty(s));

@@ -50,6 +50,7 @@ struct TmParams {
     uint32_t w_region_bytes;  // resident weights (0 when streamed)
     uint32_t w_img_bytes;
     unsigned long long timeout_ns;
+    long long inject_stop;  // test hook: chunks issued per CTA before the producer stops; -1 = never
     int act;                // epilogue activation after the bias: kActNone or kActGelu
 };
 
@@ -314,6 +315,12 @@ __global__ void __launch_bounds__(tm::Cfg<G>::kThreads, 1)
                 const int n0 = tile * tm::kM;
                 for (int c = 0; c < p.nK; ++c) {
                     if (!tc::wait_bounded(bar_empty(stage), phase ^ 1u, ctl, p.status, p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    // test hook (failure detection): stop issuing after inject_stop chunks, so
+                    // the consumers' bounded waits run out; -1 (always, outside tests) = off
+                    if (issued == p.inject_stop) {
                         ok = false;
                         break;
                     }
