@@ -37,7 +37,7 @@ ATTRS = {
 }
 PATH_NAMES = {0: "tcgen05_tokens_on_n_resident_weights", 1: "tcgen05_tokens_on_n_streamed_weights",
               2: "fp32_fp64_arithmetic", 3: "tcgen05_tokens_on_m_resident_weights",
-              4: "tcgen05_tokens_on_m_streamed_weights"}
+              4: "tcgen05_tokens_on_m_streamed_weights", 5: "tcgen05_tokens_on_n_resident_input"}
 
 _TORCH_TO_EQLIN = {torch.float32: EQLIN_F32, torch.bfloat16: EQLIN_BF16, torch.float16: EQLIN_F16}
 _EQLIN_TO_TORCH = {v: k for k, v in _TORCH_TO_EQLIN.items()}

@@ -18,6 +18,7 @@
 
 #include "eqlin_bwd_dw.cuh"
 #include "eqlin_fwd_tc.cuh"
+#include "eqlin_fwd_tcr.cuh"
 #include "eqlin_fwd_tm.cuh"
 #include "eqlin_layout.h"
 #include "eqlin_prep.cuh"
@@ -38,7 +39,15 @@ constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per boun
 //   0/1  tcgen05, tokens on the MMA N dimension, weights resident / streamed
 //   2    fp32 I/O, float64 CUDA-core kernel
 //   3/4  tcgen05, tokens on the MMA M dimension, weights resident / streamed
-enum Path { kPathResident = 0, kPathStreamed = 1, kPathF32 = 2, kPathTmResident = 3, kPathTmStreamed = 4 };
+//   5    tcgen05, tokens on N, input spectrum resident across output chunks, weights streamed
+enum Path {
+    kPathResident = 0,
+    kPathStreamed = 1,
+    kPathF32 = 2,
+    kPathTmResident = 3,
+    kPathTmStreamed = 4,
+    kPathTnResidentX = 5
+};
 
 thread_local std::string g_last_error;
 
@@ -68,7 +77,8 @@ struct Plan {
     size_t smem_bytes = 0;
     size_t img_alloc_bytes = 0;
     bool tm() const { return path == kPathTmResident || path == kPathTmStreamed; }
-    bool streamed() const { return path == kPathStreamed || path == kPathTmStreamed; }
+    bool tnr() const { return path == kPathTnResidentX; }
+    bool streamed() const { return path == kPathStreamed || path == kPathTmStreamed || path == kPathTnResidentX; }
 };
 
 // ----------------------------------------------------------------- planning
@@ -145,6 +155,43 @@ int plan_tn_g(int64_t Cout, int64_t Cin, size_t max_smem, Plan* pl) {
     return fail(EQLIN_ERR_UNSUPPORTED, "shape does not fit in shared memory");
 }
 
+// Tokens on N with the input spectrum resident: all nK x chunks of a token tile stay in
+// smem while the weight chunks of every output chunk stream through a ring.  Applies
+// when Cout > 128 (several output chunks) and the slots fit with >= 2 ring stages.
+template <int G>
+int plan_tnr_g(int64_t Cout, int64_t Cin, size_t max_smem, Plan* pl) {
+    using S = eqlin::tc::Shape<G, 2>;
+    const int max_stages = std::min(kMaxStages, env_int("EQLIN_MAX_STAGES", kMaxStages));
+    const int nK = static_cast<int>((Cin + eqlin::kChunkK - 1) / eqlin::kChunkK);
+    const int n_oc = static_cast<int>((Cout + eqlin::kMmaM - 1) / eqlin::kMmaM);
+    if (n_oc < 2 || nK > eqlin::tcr::kMaxK) return EQLIN_ERR_UNSUPPORTED;
+    const size_t ybuf = static_cast<size_t>(S::TG) * 32 * G * 2;
+    for (int nb = 2; nb >= 1; --nb) {
+        const size_t fixed = kSmemAlignSlack + kSmemCtlBytes + static_cast<size_t>(eqlin::tc::kEpiWarps) * nb * ybuf +
+                             static_cast<size_t>(nK) * S::XCHUNK_BYTES;
+        if (max_smem <= fixed) continue;
+        const size_t stages = std::min<size_t>(max_stages, (max_smem - fixed) / S::WSTAGE_BYTES);
+        if (stages < static_cast<size_t>(nb == 2 ? 3 : 2)) continue;
+        pl->path = kPathTnResidentX;
+        pl->nacc = 2;
+        pl->nK = nK;
+        pl->n_oc = n_oc;
+        pl->BN = S::BN;
+        pl->TG = S::TG;
+        pl->box_elems = S::BOX_ELEMS;
+        pl->ybufs = nb;
+        pl->ystage_bytes = static_cast<uint32_t>(nb * ybuf);
+        pl->rows = eqlin::kMmaM;
+        pl->stages = static_cast<int>(stages);
+        pl->w_region_bytes = 0;
+        pl->w_img_bytes = 0;
+        pl->img_alloc_bytes = static_cast<size_t>(n_oc) * nK * S::WSTAGE_BYTES;
+        pl->smem_bytes = fixed + stages * S::WSTAGE_BYTES;
+        return EQLIN_OK;
+    }
+    return EQLIN_ERR_UNSUPPORTED;
+}
+
 template <int G>
 int plan_tm_g(int64_t Cout, int64_t Cin, size_t max_smem, Plan* pl) {
     using C = eqlin::tm::Cfg<G>;
@@ -204,9 +251,22 @@ int plan_for(int64_t Cout, int64_t Cin, int64_t G, int io_dtype, size_t max_smem
         return EQLIN_OK;
     }
     bool tm = default_tokens_on_m(static_cast<int>(G));
+    bool tnr_ok = true;   // tokens on N: prefer the resident-input form when it applies
     if (const char* e = std::getenv("EQLIN_KERNEL")) {
         if (std::strcmp(e, "tm") == 0) tm = true;
-        if (std::strcmp(e, "tn") == 0) tm = false;
+        if (std::strcmp(e, "tn") == 0) tm = false, tnr_ok = false;
+        if (std::strcmp(e, "tnr") == 0) tm = false;
+    }
+    if (!tm && tnr_ok) {
+        int r = EQLIN_ERR_UNSUPPORTED;
+        switch (G) {
+            case 2: r = plan_tnr_g<2>(Cout, Cin, max_smem, pl); break;
+            case 4: r = plan_tnr_g<4>(Cout, Cin, max_smem, pl); break;
+            case 8: r = plan_tnr_g<8>(Cout, Cin, max_smem, pl); break;
+            case 16: r = plan_tnr_g<16>(Cout, Cin, max_smem, pl); break;
+            default: break;
+        }
+        if (r == EQLIN_OK) return EQLIN_OK;
     }
     if (tm) {
         switch (G) {
@@ -309,6 +369,25 @@ struct TcEntry {
     TcLaunch launch = nullptr;
     void* kernel = nullptr;
 };
+
+template <int G, class T16>
+void tcr_launch(unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& mx, const CUtensorMap& my,
+                const TcParams& p) {
+    launch_fused(eqlin::eqlin_fwd_tcr_kernel<G, T16>, grid, eqlin::tc::kThreads, smem, st, mx, my, p);
+}
+template <class T16>
+TcEntry tcr_entry_t(int G) {
+    switch (G) {
+        case 2: return {&tcr_launch<2, T16>, reinterpret_cast<void*>(&eqlin::eqlin_fwd_tcr_kernel<2, T16>)};
+        case 4: return {&tcr_launch<4, T16>, reinterpret_cast<void*>(&eqlin::eqlin_fwd_tcr_kernel<4, T16>)};
+        case 8: return {&tcr_launch<8, T16>, reinterpret_cast<void*>(&eqlin::eqlin_fwd_tcr_kernel<8, T16>)};
+        case 16: return {&tcr_launch<16, T16>, reinterpret_cast<void*>(&eqlin::eqlin_fwd_tcr_kernel<16, T16>)};
+        default: return {};
+    }
+}
+TcEntry tcr_entry_for(int G, int io) {
+    return io == EQLIN_F16 ? tcr_entry_t<__half>(G) : tcr_entry_t<__nv_bfloat16>(G);
+}
 struct TmEntry {
     TmLaunch launch = nullptr;
     void* kernel = nullptr;
@@ -369,6 +448,7 @@ void* f32_kernel_for(int G) {
 void* kernel_for(const Plan& pl, int G) {
     if (pl.path == kPathF32) return f32_kernel_for(G);
     if (pl.tm()) return tm_entry_for(G, pl.streamed(), pl.io).kernel;
+    if (pl.tnr()) return tcr_entry_for(G, pl.io).kernel;
     return tc_entry_for(G, pl.streamed(), pl.nacc, pl.io).kernel;
 }
 
@@ -482,7 +562,8 @@ int launch_forward(const Plan& pl, int64_t Cout, int64_t Cin, int64_t G, int sm_
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return fail(EQLIN_ERR_CUDA, "cuTensorMapEncodeTiled failed for y");
         const long long n_tiles = (N + pl.BN - 1) / pl.BN;
-        const int n_work = static_cast<int>(n_tiles * pl.n_oc);
+        // the resident-input kernel's work item is a whole token tile (all output chunks)
+        const int n_work = static_cast<int>(pl.tnr() ? n_tiles : n_tiles * pl.n_oc);
         const unsigned grid = static_cast<unsigned>(std::min<long long>(n_work, sm_count));
         if (pl.tm()) {
             TmParams p;
@@ -523,7 +604,7 @@ int launch_forward(const Plan& pl, int64_t Cout, int64_t Cin, int64_t G, int sm_
             p.timeout_ns = timeout_ns;
             p.act = b.act;
             p.inject_stop = b.inject_stop;
-            const TcEntry entry = tc_entry_for(iG, pl.streamed(), pl.nacc, pl.io);
+            const TcEntry entry = pl.tnr() ? tcr_entry_for(iG, pl.io) : tc_entry_for(iG, pl.streamed(), pl.nacc, pl.io);
             if (!entry.launch) return fail(EQLIN_ERR_UNSUPPORTED, "G");
             entry.launch(grid, pl.smem_bytes, st, map, ymap, p);
         }
@@ -1184,7 +1265,7 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[EQLIN_NOALLOC_S
 namespace {
 
 constexpr int kNoAllocMaxDevices = 64;
-constexpr int kNumPaths = 5;
+constexpr int kNumPaths = 6;
 
 struct NoAllocDevice {
     bool ready = false;

@@ -123,6 +123,18 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, Ctl*
     }
 }
 
+// Bounded wait that ignores the abort flag, for copies or MMAs in flight before exit.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, int* status,
+                                           unsigned long long timeout_ns) {
+    const uint64_t t0 = ptx::globaltimer_ns();
+    while (!ptx::mbar_try_wait(bar, parity)) {
+        if (ptx::globaltimer_ns() - t0 > timeout_ns) {
+            atomicCAS(status, 0, kDeviceErrTimeout);
+            return;
+        }
+    }
+}
+
 // ---------------------------------------------------------------- DFT role
 // 128 threads.  Unit = one token row x two adjacent channels (2*G bf16).
 // Lanes 0-15 take row r, lanes 16-31 row r+1; lane&15 selects the channel pair.

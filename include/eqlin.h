@@ -145,7 +145,9 @@ enum {
     EQLIN_ATTR_IO_DTYPE = 3,
     EQLIN_ATTR_PATH = 4,            /* kernel variant: 0/1 tcgen05 with tokens on the MMA N dimension,
                                        weights resident / streamed; 2 fp32 I/O (float64 arithmetic);
-                                       3/4 tcgen05 with tokens on the MMA M dimension, resident / streamed */
+                                       3/4 tcgen05 with tokens on the MMA M dimension, resident / streamed;
+                                       5 tcgen05 with tokens on N and the input spectrum resident
+                                       across output chunks (Cout > 128), weights streamed */
     EQLIN_ATTR_TOKENS_PER_TILE = 5, /* tokens per work item of the fused kernel */
     EQLIN_ATTR_STAGES = 6,          /* depth of the shared-memory ring */
     EQLIN_ATTR_SMEM_BYTES = 7,      /* dynamic shared memory per CTA */

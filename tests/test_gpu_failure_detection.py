@@ -24,7 +24,7 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
 
 
-@pytest.mark.parametrize("kernel,name", [("tn", "p4_c96_bf16"), ("tm", "c16_c32_bf16")])
+@pytest.mark.parametrize("kernel,name", [("tn", "p4_c96_bf16"), ("tm", "c16_c32_bf16"), ("tnr", "p4_mlp_bf16")])
 def test_wait_timeout_is_reported_and_the_gpu_stays_usable(kernel, name, monkeypatch):
     wl = workloads.WORKLOADS[name]
     x, w, bias = workloads.make_inputs(wl, N=4 * 148 * 128)
@@ -32,7 +32,8 @@ def test_wait_timeout_is_reported_and_the_gpu_stays_usable(kernel, name, monkeyp
     monkeypatch.setenv("EQLIN_KERNEL", kernel)
     monkeypatch.setenv("EQLIN_WAIT_TIMEOUT_MS", "200")
     monkeypatch.setenv("EQLIN_TEST_STOP_AFTER", "3")
-    h = eq.prepare(w.to(DEV), bias.to(DEV), io_dtype=wl.torch_dtype)
+    bd = None if bias is None else bias.to(DEV)
+    h = eq.prepare(w.to(DEV), bd, io_dtype=wl.torch_dtype)
     h.forward(xd)
     torch.cuda.synchronize()                   # the kernel returns: no hang, no fault
     assert h.device_status() == eq.EQLIN_ERR_TIMEOUT
@@ -40,7 +41,7 @@ def test_wait_timeout_is_reported_and_the_gpu_stays_usable(kernel, name, monkeyp
     h.close()
 
     monkeypatch.delenv("EQLIN_TEST_STOP_AFTER")
-    h = eq.prepare(w.to(DEV), bias.to(DEV), io_dtype=wl.torch_dtype)
+    h = eq.prepare(w.to(DEV), bd, io_dtype=wl.torch_dtype)
     y = h.forward(xd)
     torch.cuda.synchronize()
     assert h.device_status() == eq.EQLIN_OK

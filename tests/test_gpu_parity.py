@@ -102,11 +102,12 @@ def test_shapes_every_group_order(Cout, Cin, G, io):
 
 
 @pytest.mark.parametrize("io", [torch.bfloat16, torch.float16])
-@pytest.mark.parametrize("kernel", ["tn", "tm"])
+@pytest.mark.parametrize("kernel", ["tn", "tm", "tnr"])
 @pytest.mark.parametrize("Cout,Cin,G", SHAPES)
 def test_shapes_both_fused_kernels(Cout, Cin, G, kernel, io, monkeypatch):
-    """Each fused 16-bit kernel (tokens on N, tokens on M) is correct for every
-    shape, whichever one the planner would pick by default."""
+    """Each fused 16-bit kernel (tokens on N, tokens on M, tokens on N with the input
+    spectrum resident -- which falls back to tokens on N where it does not apply) is
+    correct for every shape, whichever one the planner would pick by default."""
     monkeypatch.setenv("EQLIN_KERNEL", kernel)
     gen = torch.Generator().manual_seed(Cout * 1000 + Cin * 10 + G + 5)
     N = 517
@@ -119,7 +120,7 @@ def test_shapes_both_fused_kernels(Cout, Cin, G, kernel, io, monkeypatch):
     h.close()
 
 
-@pytest.mark.parametrize("kernel", ["tn", "tm"])
+@pytest.mark.parametrize("kernel", ["tn", "tm", "tnr"])
 @pytest.mark.parametrize("name", ["p4_c96_bf16", "p8_c64_bf16", "p4_mlp_bf16", "c16_c32_bf16"])
 def test_workloads_both_fused_kernels(name, kernel, monkeypatch):
     monkeypatch.setenv("EQLIN_KERNEL", kernel)
