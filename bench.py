@@ -42,8 +42,10 @@ L2_BYTES = 126 * 1024 * 1024
 # device code of each fused kernel: a recorded ncu traffic figure is reported only
 # while these files are unchanged since the capture
 KERNEL_SOURCES = {
-    "eqlin_fwd_tc": ["eqlin_fwd_tc.cuh", "group_dft.cuh", "sm100_ptx.cuh", "eqlin_layout.h"],
-    "eqlin_fwd_tm": ["eqlin_fwd_tm.cuh", "group_dft.cuh", "sm100_ptx.cuh", "eqlin_layout.h"],
+    "eqlin_fwd_tc": ["eqlin_fwd_tc.cuh", "group_dft.cuh", "io16.cuh", "sm100_ptx.cuh", "eqlin_layout.h"],
+    "eqlin_fwd_tm": ["eqlin_fwd_tm.cuh", "group_dft.cuh", "io16.cuh", "sm100_ptx.cuh", "eqlin_layout.h"],
+    "eqlin_fwd_tcr": ["eqlin_fwd_tcr.cuh", "eqlin_fwd_tc.cuh", "group_dft.cuh", "io16.cuh", "sm100_ptx.cuh",
+                      "eqlin_layout.h"],
 }
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "eqlin_fwd_traffic.json")
 

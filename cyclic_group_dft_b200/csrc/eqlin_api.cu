@@ -91,10 +91,24 @@ int env_int(const char* name, int dflt) {
     return v > 0 ? v : dflt;
 }
 
+// How the tokens-on-N epilogue writes y: staged in shared memory for TMA stores, or with
+// plain coalesced stores from registers (a warp writes 32 consecutive channels of a
+// token).  Measured on B200: staging wins at equal ring depth (p4 C96: 61.8 vs 80.1 us);
+// direct stores win where the freed staging space deepens a shallow ring (resident-input
+// kernel, 192 -> 768: 174 vs 210 us with 3 instead of 2 weight stages).
+// EQLIN_YSTORE=tma|direct overrides.
+bool y_direct(bool dflt) {
+    const char* e = std::getenv("EQLIN_YSTORE");
+    if (e && std::strcmp(e, "direct") == 0) return true;
+    if (e && std::strcmp(e, "tma") == 0) return false;
+    return dflt;
+}
+
 template <int G, int NACC>
 int plan_tn_g(int64_t Cout, int64_t Cin, size_t max_smem, Plan* pl) {
     const int max_stages = std::min(kMaxStages, env_int("EQLIN_MAX_STAGES", kMaxStages));
     const int ybufs_env = env_int("EQLIN_YBUFS", 0);
+    const bool direct = y_direct(false);
     using S = eqlin::tc::Shape<G, NACC>;
     pl->nacc = NACC;
     pl->nK = static_cast<int>((Cin + eqlin::kChunkK - 1) / eqlin::kChunkK);
@@ -103,14 +117,14 @@ int plan_tn_g(int64_t Cout, int64_t Cin, size_t max_smem, Plan* pl) {
     pl->TG = S::TG;
     pl->box_elems = S::BOX_ELEMS;
     // y staging: per epilogue warp, ybufs buffers of TG rows x 32*G bf16 columns (4 KB);
-    // double-buffered when at least 5 ring stages still fit
+    // double-buffered when at least 4 ring stages still fit
     const size_t ybuf = static_cast<size_t>(S::TG) * 32 * G * 2;
     auto fixed_for = [&](int nb) {
         return kSmemAlignSlack + kSmemCtlBytes + static_cast<size_t>(eqlin::tc::kEpiWarps) * nb * ybuf;
     };
     pl->ybufs = 2;
-    for (int nb = 2; nb >= 1; --nb) {
-        if (ybufs_env && nb != ybufs_env) continue;
+    for (int nb = direct ? 0 : 2; nb >= (direct ? 0 : 1); --nb) {
+        if (!direct && ybufs_env && nb != ybufs_env) continue;
         const size_t fixed = fixed_for(nb);
         pl->ybufs = nb;
         pl->ystage_bytes = static_cast<uint32_t>(nb * ybuf);
@@ -123,22 +137,22 @@ int plan_tn_g(int64_t Cout, int64_t Cin, size_t max_smem, Plan* pl) {
                                    1023) / 1024 * 1024;
             if (max_smem > fixed + region) {
                 const size_t stages =
-                    std::min<size_t>(max_stages, (max_smem - fixed - region) / S::XCHUNK_BYTES);
-                if (stages >= static_cast<size_t>(nb == 2 && !ybufs_env ? 5 : 2)) {
+                    std::min<size_t>(max_stages, (max_smem - fixed - region) / S::SPEC_BYTES);
+                if (stages >= static_cast<size_t>(nb == 2 && !ybufs_env ? 4 : 2)) {
                     pl->path = kPathResident;
                     pl->rows = rows;
                     pl->stages = static_cast<int>(stages);
                     pl->w_region_bytes = static_cast<uint32_t>(region);
                     pl->w_img_bytes = static_cast<uint32_t>(img);
                     pl->img_alloc_bytes = img;
-                    pl->smem_bytes = fixed + region + stages * S::XCHUNK_BYTES;
+                    pl->smem_bytes = fixed + region + stages * S::SPEC_BYTES;
                     return EQLIN_OK;
                 }
             }
         }
         // weights streamed chunk by chunk next to each x chunk
-        if (pl->n_oc > 1 || nb == 1) {
-            const size_t stage = static_cast<size_t>(S::XCHUNK_BYTES) + S::WSTAGE_BYTES;
+        if (pl->n_oc > 1 || nb <= 1) {
+            const size_t stage = static_cast<size_t>(S::SPEC_BYTES) + S::WSTAGE_BYTES;
             const size_t stages = max_smem > fixed ? std::min<size_t>(max_stages, (max_smem - fixed) / stage) : 0;
             if (stages >= static_cast<size_t>(nb == 2 && !ybufs_env ? 3 : 1)) {
                 pl->path = kPathStreamed;
@@ -166,12 +180,21 @@ int plan_tnr_g(int64_t Cout, int64_t Cin, size_t max_smem, Plan* pl) {
     const int n_oc = static_cast<int>((Cout + eqlin::kMmaM - 1) / eqlin::kMmaM);
     if (n_oc < 2 || nK > eqlin::tcr::kMaxK) return EQLIN_ERR_UNSUPPORTED;
     const size_t ybuf = static_cast<size_t>(S::TG) * 32 * G * 2;
-    for (int nb = 2; nb >= 1; --nb) {
+    // (staging buffers, least ring stages) in order of preference: staged TMA stores with
+    // a ring of >= 3 weight chunks, else direct stores (no staging) with >= 2, else one
+    // staging buffer with 2; EQLIN_YSTORE=tma|direct keeps to one store mode
+    const char* ys = std::getenv("EQLIN_YSTORE");
+    const bool only_direct = ys && std::strcmp(ys, "direct") == 0;
+    const bool only_tma = ys && std::strcmp(ys, "tma") == 0;
+    const int options[5][2] = {{2, 3}, {1, 3}, {0, 2}, {1, 2}, {2, 2}};
+    for (const auto& opt : options) {
+        const int nb = opt[0];
+        if ((only_direct && nb != 0) || (only_tma && nb == 0)) continue;
         const size_t fixed = kSmemAlignSlack + kSmemCtlBytes + static_cast<size_t>(eqlin::tc::kEpiWarps) * nb * ybuf +
-                             static_cast<size_t>(nK) * S::XCHUNK_BYTES;
+                             static_cast<size_t>(nK) * S::SPEC_BYTES;
         if (max_smem <= fixed) continue;
         const size_t stages = std::min<size_t>(max_stages, (max_smem - fixed) / S::WSTAGE_BYTES);
-        if (stages < static_cast<size_t>(nb == 2 ? 3 : 2)) continue;
+        if (stages < static_cast<size_t>(opt[1])) continue;
         pl->path = kPathTnResidentX;
         pl->nacc = 2;
         pl->nK = nK;
@@ -203,7 +226,7 @@ int plan_tm_g(int64_t Cout, int64_t Cin, size_t max_smem, Plan* pl) {
     pl->BN = eqlin::tm::kM;
     pl->box_elems = C::X_BOX;
     pl->x_swizzle128 = C::X_SW128;
-    const size_t wchunk = static_cast<size_t>(G) * no * eqlin::kRowBytes32;   // one (oc, c) weight chunk
+    const size_t wchunk = static_cast<size_t>(eqlin::pair_slots(G)) * no * eqlin::kRowBytes32;  // one (oc, c) chunk
     const size_t fixed = kSmemAlignSlack + kSmemCtlBytes +
                          static_cast<size_t>(eqlin::tm::kYStageBytes);
     if (pl->n_oc == 1) {
@@ -600,6 +623,7 @@ int launch_forward(const Plan& pl, int64_t Cout, int64_t Cin, int64_t G, int sm_
             p.w_region_bytes = pl.w_region_bytes;
             p.ystage_bytes = pl.ystage_bytes;
             p.ybufs = pl.ybufs;
+            p.y = static_cast<uint8_t*>(y);
             p.w_img_bytes = pl.w_img_bytes;
             p.timeout_ns = timeout_ns;
             p.act = b.act;
@@ -1015,8 +1039,10 @@ int eqlin_prepare_weights_ex(const void* w, const void* bias, int64_t Cout, int6
         free_handle(h);
         return s;
     }
+    // The attribute is per kernel, not per handle: allow the device's opt-in maximum, so a
+    // later handle of the same kernel with a smaller plan cannot lower it under this one.
     e = cudaFuncSetAttribute(kernel_for(plan, static_cast<int>(G)), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(plan.smem_bytes));
+                             optin);
     if (e != cudaSuccess) {
         free_handle(h);
         return cuda_fail(e, "cudaFuncSetAttribute");
@@ -1045,7 +1071,7 @@ int eqlin_prepare_weights_ex(const void* w, const void* bias, int64_t Cout, int6
         if (s == EQLIN_OK && (e = cudaStreamSynchronize(st)) != cudaSuccess) s = cuda_fail(e, "input-gradient transform");
         if (s == EQLIN_OK &&
             (e = cudaFuncSetAttribute(kernel_for(pd, static_cast<int>(G)), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      static_cast<int>(pd.smem_bytes))) != cudaSuccess)
+                                      optin)) != cudaSuccess)
             s = cuda_fail(e, "cudaFuncSetAttribute");
         if (s != EQLIN_OK) {
             free_handle(h);
@@ -1058,8 +1084,7 @@ int eqlin_prepare_weights_ex(const void* w, const void* bias, int64_t Cout, int6
         if (plan_dw(Cout, Cin, static_cast<int>(G), static_cast<size_t>(optin), sms, &h->dwp) == EQLIN_OK) {
             h->dwp.io = io_dtype;
             e = cudaFuncSetAttribute(dw_kernel_for(static_cast<int>(G), io_dtype),
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     static_cast<int>(h->dwp.smem_bytes));
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
             if (e != cudaSuccess) {
                 free_handle(h);
                 return cuda_fail(e, "cudaFuncSetAttribute");
@@ -1334,11 +1359,11 @@ extern "C" int eqlin_forward_noalloc(const void* x, const void* w, const void* b
         if (s != EQLIN_OK) return s;
         s = plan_for(Cout, Cin, G, dtype, static_cast<size_t>(d->optin), &plan);
         if (s != EQLIN_OK) return s;
-        // kernel shared-memory attribute, once per kernel and device
+        // kernel shared-memory attribute (the device's opt-in maximum), once per kernel and device
         uint8_t& done = d->attr_done[plan.path][g_index(G)][plan.nacc == 1 ? 0 : 1][dtype == EQLIN_F16 ? 1 : 0];
         if (!done) {
             e = cudaFuncSetAttribute(kernel_for(plan, static_cast<int>(G)),
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(plan.smem_bytes));
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, d->optin);
             if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
             done = 1;
         }

@@ -12,13 +12,16 @@
 //   warp 12     TMA producer: x chunks [BN tokens x 32 channels x G] (16 KB) into a smem
 //               ring (plus the weight chunk when the weights are streamed).
 //   warps 8-11  DFT: read a landed x chunk, real DFT over G in fp32 registers, write the
-//               G frequency planes [BN x 32] bf16 back IN PLACE in the UMMA K-major
-//               SWIZZLE_64B layout (the x chunk and its spectrum have the same size).
+//               spectrum's pair slots [BN x 32] bf16 back IN PLACE in the UMMA K-major
+//               SWIZZLE_64B layout (the stage holds the x chunk and, past its end, the
+//               spectrum's extra -Im slots).
 //   warp 13     MMA issuer (one thread) + TMEM owner: per chunk and frequency,
 //               tcgen05.mma with A = W^ plane [128 out-rows x 32], B = X^ plane [BN x 32],
-//               D in TMEM (lane = output channel, column = token).  Complex frequencies
-//               use four real products; the -Im(W)Im(X) term uses the descriptor's
-//               negate-A bit, so only Re and Im of W^ are stored.  Two accumulators
+//               D in TMEM (lane = output channel, column = token).  A complex frequency
+//               takes two products of N = 2*BN that write its Re and Im planes of D at
+//               once: the DFT stores [-Im, Re, Im] of X^ back to back (pair slots,
+//               eqlin_layout.h), so B = [Xr; Xi] pairs with Wr and B = [-Xi; Xr] with
+//               Wi, and only Re and Im of W^ are stored.  Two accumulators
 //               (G*BN = 256 columns each) alternate between work items, so the MMAs of
 //               one tile overlap the epilogue of the previous one.
 //   warps 0-7   epilogue: tcgen05.ld of all G planes of a token group, inverse real DFT
@@ -45,6 +48,7 @@ namespace eqlin {
 
 struct TcParams {
     const uint8_t* w_img;   // frequency-domain weight image (layout: eqlin_layout.h)
+    uint8_t* y;             // [N, Cout, G] output (direct stores, ybufs == 0)
     const float* bias;      // [Cout] fp32, or nullptr
     int* status;            // device status word (first error wins)
     long long N;
@@ -56,7 +60,7 @@ struct TcParams {
     int stages;             // smem ring depth
     uint32_t w_region_bytes;  // smem reserved for resident weights (0 when streamed)
     uint32_t ystage_bytes;    // y staging per epilogue warp (ybufs buffers of TG x 32*G bf16)
-    int ybufs;                // 1 or 2 staging buffers per epilogue warp
+    int ybufs;                // 1 or 2 staging buffers per epilogue warp; 0 = direct stores
     uint32_t w_img_bytes;     // bytes of the resident image to copy
     unsigned long long timeout_ns;
     long long inject_stop;  // test hook: chunks issued per CTA before the producer stops; -1 = never
@@ -83,7 +87,9 @@ struct Shape {
     static constexpr int kNumAcc = NACC;
     static constexpr int BN = (512 / (G * NACC)) < 128 ? (512 / (G * NACC)) : 128;  // tokens per tile (MMA N)
     static constexpr int PLANE_BYTES = BN * kPlaneRowBytes;          // one frequency plane
-    static constexpr int XCHUNK_BYTES = G * PLANE_BYTES;             // == BN * 32 * G * 2
+    static constexpr int XCHUNK_BYTES = G * PLANE_BYTES;             // == BN * 32 * G * 2 (the x chunk)
+    static constexpr int SLOTS = pair_slots(G);                      // spectrum slots (eqlin_layout.h)
+    static constexpr int SPEC_BYTES = SLOTS * PLANE_BYTES;           // the chunk's spectrum, in place
     static constexpr int XROW_ELEMS = kChunkK * G;                   // one token row of a chunk
     static constexpr int BOX_ELEMS = XROW_ELEMS < 256 ? XROW_ELEMS : 256;
     static constexpr int NBOX = XROW_ELEMS / BOX_ELEMS;
@@ -91,7 +97,7 @@ struct Shape {
     static constexpr int ACC_COLS = G * BN;                          // one accumulator
     static constexpr int TMEM_COLS = 512;
     static constexpr int TG = (64 / G) < BN / 2 ? (64 / G) : BN / 2;  // tokens per epilogue group
-    static_assert(XCHUNK_BYTES % 1024 == 0, "stage alignment");
+    static_assert(XCHUNK_BYTES % 1024 == 0 && SPEC_BYTES % 1024 == 0, "stage alignment");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N");
     static_assert(NACC * ACC_COLS <= TMEM_COLS, "TMEM columns");
     static_assert((BN / 2) % TG == 0, "epilogue groups");
@@ -194,9 +200,18 @@ __device__ __forceinline__ void dft_chunk(uint8_t* xs, int dft_tid) {
         rdft_planes<G>(xab, pab);
         const int phys = (chunk ^ ((r >> 1) & 3)) * 16 + in_chunk;   // SWIZZLE_64B
         uint8_t* dst = xs + r * kPlaneRowBytes + phys;
+        // pair slots: planes 0 and 1, then [-Im, Re, Im] per complex frequency; the sign
+        // flip of the packed pair is exact (rounding to nearest even is symmetric)
+        *reinterpret_cast<uint32_t*>(dst) = Io16<T16>::pack(pab[0].x, pab[0].y);
+        *reinterpret_cast<uint32_t*>(dst + S::PLANE_BYTES) = Io16<T16>::pack(pab[1].x, pab[1].y);
 #pragma unroll
-        for (int p = 0; p < G; ++p) {
-            *reinterpret_cast<uint32_t*>(dst + p * S::PLANE_BYTES) = Io16<T16>::pack(pab[p].x, pab[p].y);
+        for (int k = 1; k < G / 2; ++k) {
+            const uint32_t re = Io16<T16>::pack(pab[2 * k].x, pab[2 * k].y);
+            const uint32_t im = Io16<T16>::pack(pab[2 * k + 1].x, pab[2 * k + 1].y);
+            uint8_t* d = dst + pair_first_slot(k) * S::PLANE_BYTES;
+            *reinterpret_cast<uint32_t*>(d) = im ^ 0x80008000u;
+            *reinterpret_cast<uint32_t*>(d + S::PLANE_BYTES) = re;
+            *reinterpret_cast<uint32_t*>(d + 2 * S::PLANE_BYTES) = im;
         }
     }
 }
@@ -233,6 +248,41 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, const CUtensorM
         ptx::tmem_wait_ld();
 #pragma unroll
         for (int pl = 0; pl < G; ++pl) ptx::tmem_regs_ready<TG>(r[pl]);
+        if (p.ybufs == 0) {
+            // direct stores: lane o writes its G outputs (2G bytes) of each token, so a warp
+            // writes 32 consecutive channels = one contiguous 64G-byte run per token
+            const long long row0 = n0 + t0 + j * TG;
+            if (valid_o) {
+#pragma unroll
+                for (int t = 0; t < TG; ++t) {
+                    if (row0 + t >= p.N) break;
+                    float z[G], yv[G];
+#pragma unroll
+                    for (int pl = 0; pl < G; ++pl) z[pl] = __uint_as_float(r[pl][t]);
+                    z[0] += b;
+                    RealIdft<G>::run(z, yv);
+                    if (p.act == kActGelu) {
+#pragma unroll
+                        for (int g = 0; g < G; ++g) yv[g] = gelu(yv[g]);
+                    }
+                    uint8_t* dst = p.y + ((row0 + t) * p.Cout + o) * (2 * G);
+                    if constexpr (G == 2) {
+                        *reinterpret_cast<uint32_t*>(dst) = Io16<T16>::pack(yv[0], yv[1]);
+                    } else if constexpr (G == 4) {
+                        *reinterpret_cast<uint2*>(dst) =
+                            make_uint2(Io16<T16>::pack(yv[0], yv[1]), Io16<T16>::pack(yv[2], yv[3]));
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < G / 8; ++c) {
+                            *reinterpret_cast<uint4*>(dst + 16 * c) = make_uint4(
+                                Io16<T16>::pack(yv[8 * c + 0], yv[8 * c + 1]), Io16<T16>::pack(yv[8 * c + 2], yv[8 * c + 3]),
+                                Io16<T16>::pack(yv[8 * c + 4], yv[8 * c + 5]), Io16<T16>::pack(yv[8 * c + 6], yv[8 * c + 7]));
+                        }
+                    }
+                }
+            }
+            continue;
+        }
         // the buffer about to be written was stored p.ybufs groups ago: wait until read
         if (lane == 0) {
             if (p.ybufs == 2) ptx::bulk_wait_group_read<1>();
@@ -300,8 +350,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
 
-    constexpr uint32_t STAGE_BYTES = S::XCHUNK_BYTES + (STREAM_W ? S::WSTAGE_BYTES : 0);
-    constexpr uint32_t STAGE_TX = STAGE_BYTES;   // every byte of a stage arrives by copy
+    // a stage: the x chunk, transformed in place into its (larger) spectrum, then the
+    // streamed weight chunk; the copies fill the x chunk and the weight chunk
+    constexpr uint32_t STAGE_BYTES = S::SPEC_BYTES + (STREAM_W ? S::WSTAGE_BYTES : 0);
+    constexpr uint32_t STAGE_TX = S::XCHUNK_BYTES + (STREAM_W ? S::WSTAGE_BYTES : 0);
     const int NS = p.stages;
     uint8_t* ystage0 = smem + p.w_region_bytes;                 // y staging, one area per epilogue warp
     uint8_t* stage0 = ystage0 + tc::kEpiWarps * static_cast<size_t>(p.ystage_bytes);
@@ -389,7 +441,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                                          c * S::XROW_ELEMS + bx * S::BOX_ELEMS, n0, bar_full(stage));
                     }
                     if constexpr (STREAM_W) {
-                        ptx::bulk_load(dst + S::XCHUNK_BYTES,
+                        ptx::bulk_load(dst + S::SPEC_BYTES,
                                        p.w_img + static_cast<size_t>(oc * p.nK + c) * S::WSTAGE_BYTES,
                                        S::WSTAGE_BYTES, bar_full(stage));
                     }
@@ -429,7 +481,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
             bool ok = true;
             if constexpr (!STREAM_W) ok = tc::wait_bounded(bar_w_full, 0, ctl, p.status, p.timeout_ns);
             constexpr uint32_t ID = idesc_f16kind_f32(kMmaM, S::BN, Io16<T16>::kUmmaFormat, false);
-            constexpr uint32_t ID_NEG = idesc_f16kind_f32(kMmaM, S::BN, Io16<T16>::kUmmaFormat, true);
+            // complex products: N = 2*BN, the Re and Im planes of D side by side
+            constexpr uint32_t ID2 = idesc_f16kind_f32(kMmaM, G > 2 ? 2 * S::BN : S::BN, Io16<T16>::kUmmaFormat, false);
             int stage = 0;
             uint32_t phase = 0;
             int it = 0;
@@ -451,7 +504,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                     const uint32_t xb = s_stage0 + stage * STAGE_BYTES;
                     uint32_t wb, wsub;
                     if constexpr (STREAM_W) {
-                        wb = xb + S::XCHUNK_BYTES;
+                        wb = xb + S::SPEC_BYTES;
                         wsub = kMmaM * kPlaneRowBytes;
                     } else {
                         wsub = static_cast<uint32_t>(p.rows) * kPlaneRowBytes;
@@ -468,21 +521,19 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                         auto A = [&](int pl) {
                             return ptx::sdesc_sw64_from_lo(a_lo + static_cast<uint32_t>(pl) * wsub16 + ks * 2);
                         };
-                        auto B = [&](int pl) {
-                            return ptx::sdesc_sw64_from_lo(b_lo + (pl * S::PLANE_BYTES + ks * 32) / 16);
+                        auto B = [&](int slot) {
+                            return ptx::sdesc_sw64_from_lo(b_lo + (slot * S::PLANE_BYTES + ks * 32) / 16);
                         };
                         auto D = [&](int pl) { return acc_base + static_cast<uint32_t>(pl * S::BN); };
                         // real frequencies k = 0 and k = G/2
                         ptx::umma_f16(D(0), A(0), B(0), ID, acc0);
                         ptx::umma_f16(D(1), A(1), B(1), ID, acc0);
-                        // complex frequencies: (Wr + i Wi)(Xr + i Xi)
+                        // complex frequencies: (Wr + i Wi)(Xr + i Xi), two products of N = 2*BN
 #pragma unroll
                         for (int k = 1; k < G / 2; ++k) {
-                            const int pr = 2 * k, pi = 2 * k + 1;
-                            ptx::umma_f16(D(pr), A(pr), B(pr), ID, acc0);      // + Wr Xr
-                            ptx::umma_f16(D(pr), A(pi), B(pi), ID_NEG, 1u);    // - Wi Xi
-                            ptx::umma_f16(D(pi), A(pi), B(pr), ID, acc0);      // + Wi Xr
-                            ptx::umma_f16(D(pi), A(pr), B(pi), ID, 1u);        // + Wr Xi
+                            const int pr = 2 * k, pi = 2 * k + 1, s = pair_first_slot(k);
+                            ptx::umma_f16(D(pr), A(pr), B(s + 1), ID2, acc0);   // [Dr|Di] += Wr [Xr; Xi]
+                            ptx::umma_f16(D(pr), A(pi), B(s), ID2, 1u);         // [Dr|Di] += Wi [-Xi; Xr]
                         }
                     }
                     ptx::umma_commit(bar_empty(stage));   // stage reusable once these finish

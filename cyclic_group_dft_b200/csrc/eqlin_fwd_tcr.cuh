@@ -47,7 +47,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     const int NS = p.stages, nK = p.nK;
     uint8_t* ystage0 = smem;                                          // y staging per epilogue warp
     uint8_t* xslot0 = ystage0 + tc::kEpiWarps * static_cast<size_t>(p.ystage_bytes);
-    uint8_t* wring0 = xslot0 + static_cast<size_t>(nK) * S::XCHUNK_BYTES;
+    uint8_t* wring0 = xslot0 + static_cast<size_t>(nK) * S::SPEC_BYTES;
     uint64_t* bars = reinterpret_cast<uint64_t*>(wring0 + static_cast<size_t>(NS) * S::WSTAGE_BYTES);
     tc::Ctl* ctl = reinterpret_cast<tc::Ctl*>(bars + 2 * tcr::kMaxK + 2 * NS + 6);
 
@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                         ok = false;
                         break;
                     }
-                    const uint32_t dst = s_xslot0 + c * S::XCHUNK_BYTES;
+                    const uint32_t dst = s_xslot0 + c * S::SPEC_BYTES;
                     ptx::mbar_arrive_expect_tx(bar_x_full(c), S::XCHUNK_BYTES);
 #pragma unroll
                     for (int bx = 0; bx < S::NBOX; ++bx)
@@ -164,7 +164,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t ID = idesc_f16kind_f32(kMmaM, S::BN, Io16<T16>::kUmmaFormat, false);
-            constexpr uint32_t ID_NEG = idesc_f16kind_f32(kMmaM, S::BN, Io16<T16>::kUmmaFormat, true);
+            constexpr uint32_t ID2 = idesc_f16kind_f32(kMmaM, G > 2 ? 2 * S::BN : S::BN, Io16<T16>::kUmmaFormat, false);
             constexpr uint32_t wsub16 = (kMmaM * kPlaneRowBytes) >> 4;
             bool ok = true;
             int it = 0, ws = 0, ti = 0;
@@ -191,7 +191,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                         }
                         ptx::tc_fence_after();
                         const uint32_t a_lo = ptx::sdesc_sw64_lo(s_wring0 + ws * S::WSTAGE_BYTES);
-                        const uint32_t b_lo = ptx::sdesc_sw64_lo(s_xslot0 + c * S::XCHUNK_BYTES);
+                        const uint32_t b_lo = ptx::sdesc_sw64_lo(s_xslot0 + c * S::SPEC_BYTES);
                         const uint32_t acc_first = c > 0 ? 1u : 0u;
 #pragma unroll
                         for (int ks = 0; ks < kChunkK / 16; ++ks) {
@@ -199,19 +199,17 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                             auto A = [&](int pl) {
                                 return ptx::sdesc_sw64_from_lo(a_lo + static_cast<uint32_t>(pl) * wsub16 + ks * 2);
                             };
-                            auto B = [&](int pl) {
-                                return ptx::sdesc_sw64_from_lo(b_lo + (pl * S::PLANE_BYTES + ks * 32) / 16);
+                            auto B = [&](int slot) {
+                                return ptx::sdesc_sw64_from_lo(b_lo + (slot * S::PLANE_BYTES + ks * 32) / 16);
                             };
                             auto D = [&](int pl) { return acc_base + static_cast<uint32_t>(pl * S::BN); };
                             ptx::umma_f16(D(0), A(0), B(0), ID, acc0);
                             ptx::umma_f16(D(1), A(1), B(1), ID, acc0);
 #pragma unroll
                             for (int k = 1; k < G / 2; ++k) {
-                                const int pr = 2 * k, pi = 2 * k + 1;
-                                ptx::umma_f16(D(pr), A(pr), B(pr), ID, acc0);      // + Wr Xr
-                                ptx::umma_f16(D(pr), A(pi), B(pi), ID_NEG, 1u);    // - Wi Xi
-                                ptx::umma_f16(D(pi), A(pi), B(pr), ID, acc0);      // + Wi Xr
-                                ptx::umma_f16(D(pi), A(pr), B(pi), ID, 1u);        // + Wr Xi
+                                const int pr = 2 * k, pi = 2 * k + 1, s = pair_first_slot(k);
+                                ptx::umma_f16(D(pr), A(pr), B(s + 1), ID2, acc0);   // [Dr|Di] += Wr [Xr; Xi]
+                                ptx::umma_f16(D(pr), A(pi), B(s), ID2, 1u);         // [Dr|Di] += Wi [-Xi; Xr]
                             }
                         }
                         ptx::umma_commit(bar_w_empty(ws));
@@ -239,7 +237,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                     ok = false;
                     break;
                 }
-                tc::dft_chunk<G, 2, T16>(xslot0 + static_cast<size_t>(c) * S::XCHUNK_BYTES, dft_tid);
+                tc::dft_chunk<G, 2, T16>(xslot0 + static_cast<size_t>(c) * S::SPEC_BYTES, dft_tid);
                 ptx::fence_proxy_async_smem();
                 ptx::mbar_arrive(bar_xhat(c));
             }

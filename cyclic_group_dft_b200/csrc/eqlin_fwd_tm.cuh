@@ -7,7 +7,7 @@
 //   A = X^ plane [128 tokens x 16 channels]  (M = 128 tokens)
 //   B = W^ plane [NO output channels x 16]   (N = NO <= 512/G, a multiple of 32)
 //   D = TMEM, lane = token, column = output channel, one plane per frequency component
-// A work item (128 tokens, NO output channels) needs 2G-2 MMAs per 16 input channels,
+// A work item (128 tokens, NO output channels) needs G MMAs per 16 input channels,
 // independent of how many output channels it covers, so small Cout configurations
 // issue 4-8x fewer MMAs than with tokens on N.  G*NO <= 512 TMEM columns leaves room for
 // one accumulator: the MMAs of a tile wait for the epilogue of the previous tile to
@@ -17,7 +17,9 @@
 //   producer warp    TMA loads of x chunks [128 tokens x 16 channels x G] (+ the weight
 //                    chunk when the weights are streamed) into a smem ring
 //   DW DFT warps     in-place real DFT over G: x chunk -> G planes, K-major SWIZZLE_32B
-//   MMA warp         one thread issues tcgen05.mma (2 real + 4 per complex frequency)
+//   MMA warp         one thread issues tcgen05.mma: 2 real products, and 2 per complex
+//                    frequency, each over the Re and Im planes of D at once (N = 2*NO)
+//                    thanks to the weight image's [-Im, Re, Im] slots (eqlin_layout.h)
 //   8 epilogue warps lane = token; per group of 32/G output channels: tcgen05.ld of the
 //                    G planes, inverse real DFT + bias, bf16, into the warp's own
 //                    SWIZZLE_64B staging tile [32 tokens x 32 columns], TMA store by the
@@ -248,7 +250,8 @@ __global__ void __launch_bounds__(tm::Cfg<G>::kThreads, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
 
-    const uint32_t wstage_bytes = STREAM_W ? static_cast<uint32_t>(G * p.NO * kRowBytes32) : 0u;
+    constexpr int SL = pair_slots(G);
+    const uint32_t wstage_bytes = STREAM_W ? static_cast<uint32_t>(SL * p.NO * kRowBytes32) : 0u;
     const uint32_t stage_bytes = C::XCHUNK_BYTES + wstage_bytes;
     const int NS = p.stages;
     uint8_t* ystage0 = smem + p.w_region_bytes;
@@ -369,7 +372,8 @@ __global__ void __launch_bounds__(tm::Cfg<G>::kThreads, 1)
             bool ok = true;
             if constexpr (!STREAM_W) ok = tc::wait_bounded(bar_w_full, 0, ctl, p.status, p.timeout_ns);
             const uint32_t ID = idesc_f16kind_f32(tm::kM, p.NO, Io16<T16>::kUmmaFormat, false, false);
-            const uint32_t ID_NEG = idesc_f16kind_f32(tm::kM, p.NO, Io16<T16>::kUmmaFormat, false, true);
+            // complex products: N = 2*NO output columns, the Re and Im planes of D side by side
+            const uint32_t ID2 = idesc_f16kind_f32(tm::kM, G > 2 ? 2 * p.NO : p.NO, Io16<T16>::kUmmaFormat, false, false);
             const uint32_t wplane = static_cast<uint32_t>(p.NO) * kRowBytes32;
             int stage = 0;
             uint32_t phase = 0;
@@ -389,7 +393,7 @@ __global__ void __launch_bounds__(tm::Cfg<G>::kThreads, 1)
                     ptx::tc_fence_after();
                     const uint32_t xb = s_stage0 + stage * stage_bytes;
                     const uint32_t wb = STREAM_W ? xb + C::XCHUNK_BYTES
-                                                 : s_w + static_cast<uint32_t>(c * G) * wplane;
+                                                 : s_w + static_cast<uint32_t>(c * SL) * wplane;
                     const uint32_t a_lo = ptx::sdesc_sw32_lo(xb), b_lo = ptx::sdesc_sw32_lo(wb);
                     const uint32_t wplane16 = wplane >> 4;
                     const uint32_t acc0 = c > 0 ? 1u : 0u;
@@ -400,11 +404,9 @@ __global__ void __launch_bounds__(tm::Cfg<G>::kThreads, 1)
                     ptx::umma_f16(D(1), A(1), B(1), ID, acc0);          // k = G/2
 #pragma unroll
                     for (int k = 1; k < G / 2; ++k) {                   // (Xr + i Xi)(Wr + i Wi)
-                        const int pr = 2 * k, pi = 2 * k + 1;
-                        ptx::umma_f16(D(pr), A(pr), B(pr), ID, acc0);       // + Xr Wr
-                        ptx::umma_f16(D(pr), A(pi), B(pi), ID_NEG, 1u);     // - Xi Wi
-                        ptx::umma_f16(D(pi), A(pr), B(pi), ID, acc0);       // + Xr Wi
-                        ptx::umma_f16(D(pi), A(pi), B(pr), ID, 1u);         // + Xi Wr
+                        const int pr = 2 * k, pi = 2 * k + 1, s = pair_first_slot(k);
+                        ptx::umma_f16(D(pr), A(pr), B(s + 1), ID2, acc0);   // [Dr|Di] += Xr [Wr; Wi]
+                        ptx::umma_f16(D(pr), A(pi), B(s), ID2, 1u);         // [Dr|Di] += Xi [-Wi; Wr]
                     }
                     ptx::umma_commit(bar_empty(stage));
                     if (++stage == NS) { stage = 0; phase ^= 1u; }

@@ -38,9 +38,28 @@ __host__ __device__ inline size_t image_offset(size_t sub, int rows, int r, int 
            static_cast<size_t>(piece) * 16 + static_cast<size_t>(col & 7) * 2;
 }
 
+// Slot layout of an MMA operand that pairs the products of a complex frequency.  The
+// slots are: plane 0, plane 1, then for each complex frequency k the three slots
+// [-Im V_k, Re V_k, Im V_k].  They are stored back to back, so [Re V_k; Im V_k] and
+// [-Im V_k; Re V_k] are each one operand of twice the slot's rows, and a complex product
+// (a + ib)(c + id) takes two MMAs that write the Re and Im planes of D side by side:
+//   [D_re | D_im] += a [c; d],   [D_re | D_im] += b [-d; c].
+// The tokens-on-M weight image uses it for W^, the tokens-on-N kernels for X^.
+__host__ __device__ constexpr int pair_slots(int G) { return 2 + 3 * (G / 2 - 1); }
+// first slot of complex frequency k (0 < k < G/2): the -Im slot
+__host__ __device__ constexpr int pair_first_slot(int k) { return 2 + 3 * (k - 1); }
+// frequency plane held by slot s, and its sign
+__host__ __device__ inline int pair_slot_plane(int s, float* sign) {
+    *sign = 1.0f;
+    if (s < 2) return s;
+    const int k = (s - 2) / 3 + 1, j = (s - 2) % 3;
+    if (j == 0) *sign = -1.0f;
+    return j == 1 ? 2 * k : 2 * k + 1;
+}
+
 // Tokens-on-M kernel variant: 16-channel K chunks, rows of 32 bytes, SWIZZLE_32B
 // (16-byte piece j of row r stored at piece j ^ ((r >> 2) & 1)).  Image layout
-// [oc][c][p][r < rows][16].
+// [oc][c][s][r < rows][16] over the pair slots s < pair_slots(G) of W^.
 constexpr int kChunkK16 = 16;
 constexpr int kRowBytes32 = 32;
 __host__ __device__ inline size_t image_offset_k16(size_t sub, int rows, int r, int col) {

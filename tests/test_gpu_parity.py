@@ -120,6 +120,25 @@ def test_shapes_both_fused_kernels(Cout, Cin, G, kernel, io, monkeypatch):
     h.close()
 
 
+@pytest.mark.parametrize("ystore", ["tma", "direct"])
+@pytest.mark.parametrize("Cout,Cin,G", [(50, 40, 4), (96, 96, 4), (200, 32, 4), (130, 96, 4), (96, 96, 2),
+                                        (136, 64, 8), (768, 192, 4)])
+def test_tokens_on_n_store_modes(Cout, Cin, G, ystore, monkeypatch):
+    """Both ways the tokens-on-N epilogues write y (TMA stores of a staged tile, plain
+    coalesced stores), for both tokens-on-N kernels, with a ragged token tail."""
+    monkeypatch.setenv("EQLIN_KERNEL", "tnr")
+    monkeypatch.setenv("EQLIN_YSTORE", ystore)
+    gen = torch.Generator().manual_seed(Cout * 1000 + Cin * 10 + G + 17)
+    N = 1031
+    x = torch.randn(N, Cin, G, generator=gen).to(torch.bfloat16)
+    w = (torch.randn(Cout, Cin, G, generator=gen) / np.sqrt(Cin * G)).to(torch.bfloat16)
+    bias = (torch.randn(Cout, generator=gen) * 0.3).to(torch.bfloat16)
+    y, h = _run(x, w, bias, torch.bfloat16)
+    assert "tokens_on_n" in h.path, h.path
+    _assert_parity(torch.bfloat16, y, _ref(x, w, bias), f"Cout={Cout} Cin={Cin} G={G} {ystore} path={h.path}")
+    h.close()
+
+
 @pytest.mark.parametrize("kernel", ["tn", "tm", "tnr"])
 @pytest.mark.parametrize("name", ["p4_c96_bf16", "p8_c64_bf16", "p4_mlp_bf16", "c16_c32_bf16"])
 def test_workloads_both_fused_kernels(name, kernel, monkeypatch):
@@ -260,3 +279,23 @@ def test_host_buffer_forward_matches_device_forward():
 
 def test_tolerances_are_the_stated_ones():
     assert TOL_F32_MAXREL == 1e-5 and TOL_BF16_NORMWISE == 2e-2
+
+
+def test_handles_sharing_a_kernel_keep_their_shared_memory():
+    """Two handles of one kernel with different shared-memory plans: preparing the second
+    must not shrink what the first one launches with (the limit is per kernel)."""
+    gen = torch.Generator().manual_seed(91)
+    shapes = [(128, 128, 4), (32, 32, 4)]
+    hs, refs, xs = [], [], []
+    for Cout, Cin, G in shapes:
+        x = torch.randn(300, Cin, G, generator=gen).to(torch.bfloat16)
+        w = (torch.randn(Cout, Cin, G, generator=gen) / np.sqrt(Cin * G)).to(torch.bfloat16)
+        hs.append(eq.prepare(w.to(DEV), None))
+        xs.append(x)
+        refs.append(_ref(x, w, None))
+    assert hs[0].path == hs[1].path and hs[0].attr("smem_bytes") != hs[1].attr("smem_bytes")
+    for h, x, ref in zip(hs, xs, refs):
+        y = h.forward(x.to(DEV))
+        torch.cuda.synchronize()
+        _assert_parity(torch.bfloat16, y, ref, f"path={h.path} smem={h.attr('smem_bytes')}")
+        h.close()
