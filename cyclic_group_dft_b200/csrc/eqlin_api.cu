@@ -93,9 +93,10 @@ int env_int(const char* name, int dflt) {
 
 // How the tokens-on-N epilogue writes y: staged in shared memory for TMA stores, or with
 // plain coalesced stores from registers (a warp writes 32 consecutive channels of a
-// token).  Measured on B200: staging wins at equal ring depth (p4 C96: 61.8 vs 80.1 us);
-// direct stores win where the freed staging space deepens a shallow ring (resident-input
-// kernel, 192 -> 768: 174 vs 210 us with 3 instead of 2 weight stages).
+// token).  Measured on B200: staging wins where the output dominates (p4 C96: 62.1 vs
+// 82.8 us); direct stores win where the freed staging space deepens a ring that limits
+// the kernel: many input chunks per work item, or the resident-input kernel's weight ring
+// (192 -> 768: 174 vs 210 us with 3 instead of 2 weight stages).
 // EQLIN_YSTORE=tma|direct overrides.
 bool y_direct(bool dflt) {
     const char* e = std::getenv("EQLIN_YSTORE");
@@ -108,10 +109,12 @@ template <int G, int NACC>
 int plan_tn_g(int64_t Cout, int64_t Cin, size_t max_smem, Plan* pl) {
     const int max_stages = std::min(kMaxStages, env_int("EQLIN_MAX_STAGES", kMaxStages));
     const int ybufs_env = env_int("EQLIN_YBUFS", 0);
-    const bool direct = y_direct(false);
     using S = eqlin::tc::Shape<G, NACC>;
     pl->nacc = NACC;
     pl->nK = static_cast<int>((Cin + eqlin::kChunkK - 1) / eqlin::kChunkK);
+    // direct stores from 8 input chunks on (B200: 256 -> 64 at p4, 126.5 vs 139.4 us;
+    // 384 -> 96, 189.4 vs 206.1 us), staged TMA stores below (96 -> 96: 62.1 vs 82.8 us)
+    const bool direct = y_direct(pl->nK >= 8);
     pl->n_oc = static_cast<int>((Cout + eqlin::kMmaM - 1) / eqlin::kMmaM);
     pl->BN = S::BN;
     pl->TG = S::TG;
@@ -172,13 +175,16 @@ int plan_tn_g(int64_t Cout, int64_t Cin, size_t max_smem, Plan* pl) {
 // Tokens on N with the input spectrum resident: all nK x chunks of a token tile stay in
 // smem while the weight chunks of every output chunk stream through a ring.  Applies
 // when Cout > 128 (several output chunks) and the slots fit with >= 2 ring stages.
+// By default only from 4 input chunks on: below that, re-transforming x per output chunk
+// costs less than the resident form's narrower ring (B200, p4: 96 -> 384, 186.5 us
+// streamed vs 193.5 us; 64 -> 256, 115.7 vs 122.7 us; 128 -> 512, 314.1 vs 290.8 us).
 template <int G>
-int plan_tnr_g(int64_t Cout, int64_t Cin, size_t max_smem, Plan* pl) {
+int plan_tnr_g(int64_t Cout, int64_t Cin, size_t max_smem, bool forced, Plan* pl) {
     using S = eqlin::tc::Shape<G, 2>;
     const int max_stages = std::min(kMaxStages, env_int("EQLIN_MAX_STAGES", kMaxStages));
     const int nK = static_cast<int>((Cin + eqlin::kChunkK - 1) / eqlin::kChunkK);
     const int n_oc = static_cast<int>((Cout + eqlin::kMmaM - 1) / eqlin::kMmaM);
-    if (n_oc < 2 || nK > eqlin::tcr::kMaxK) return EQLIN_ERR_UNSUPPORTED;
+    if (n_oc < 2 || nK > eqlin::tcr::kMaxK || (!forced && nK < 4)) return EQLIN_ERR_UNSUPPORTED;
     const size_t ybuf = static_cast<size_t>(S::TG) * 32 * G * 2;
     // (staging buffers, least ring stages) in order of preference: staged TMA stores with
     // a ring of >= 3 weight chunks, else direct stores (no staging) with >= 2, else one
@@ -275,18 +281,19 @@ int plan_for(int64_t Cout, int64_t Cin, int64_t G, int io_dtype, size_t max_smem
     }
     bool tm = default_tokens_on_m(static_cast<int>(G));
     bool tnr_ok = true;   // tokens on N: prefer the resident-input form when it applies
+    bool tnr_forced = false;
     if (const char* e = std::getenv("EQLIN_KERNEL")) {
         if (std::strcmp(e, "tm") == 0) tm = true;
         if (std::strcmp(e, "tn") == 0) tm = false, tnr_ok = false;
-        if (std::strcmp(e, "tnr") == 0) tm = false;
+        if (std::strcmp(e, "tnr") == 0) tm = false, tnr_forced = true;
     }
     if (!tm && tnr_ok) {
         int r = EQLIN_ERR_UNSUPPORTED;
         switch (G) {
-            case 2: r = plan_tnr_g<2>(Cout, Cin, max_smem, pl); break;
-            case 4: r = plan_tnr_g<4>(Cout, Cin, max_smem, pl); break;
-            case 8: r = plan_tnr_g<8>(Cout, Cin, max_smem, pl); break;
-            case 16: r = plan_tnr_g<16>(Cout, Cin, max_smem, pl); break;
+            case 2: r = plan_tnr_g<2>(Cout, Cin, max_smem, tnr_forced, pl); break;
+            case 4: r = plan_tnr_g<4>(Cout, Cin, max_smem, tnr_forced, pl); break;
+            case 8: r = plan_tnr_g<8>(Cout, Cin, max_smem, tnr_forced, pl); break;
+            case 16: r = plan_tnr_g<16>(Cout, Cin, max_smem, tnr_forced, pl); break;
             default: break;
         }
         if (r == EQLIN_OK) return EQLIN_OK;

@@ -263,7 +263,11 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, const CUtensorM
                     RealIdft<G>::run(z, yv);
                     if (p.act == kActGelu) {
 #pragma unroll
-                        for (int g = 0; g < G; ++g) yv[g] = gelu(yv[g]);
+                        for (int g = 0; g < G; g += 2) {
+                            const fx2 u = gelu2(fx2(yv[g], yv[g + 1]));
+                            yv[g] = u.x;
+                            yv[g + 1] = u.y;
+                        }
                     }
                     uint8_t* dst = p.y + ((row0 + t) * p.Cout + o) * (2 * G);
                     if constexpr (G == 2) {
@@ -300,7 +304,11 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, const CUtensorM
                 RealIdft<G>::run(z, yv);
                 if (p.act == kActGelu) {
 #pragma unroll
-                    for (int g = 0; g < G; ++g) yv[g] = gelu(yv[g]);
+                    for (int g = 0; g < G; g += 2) {
+                        const fx2 u = gelu2(fx2(yv[g], yv[g + 1]));
+                        yv[g] = u.x;
+                        yv[g + 1] = u.y;
+                    }
                 }
                 uint8_t* dst = lane_off + t * (YBC * 2);
                 if constexpr (G == 2) {

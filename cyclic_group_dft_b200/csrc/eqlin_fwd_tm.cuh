@@ -206,14 +206,14 @@ __device__ __forceinline__ void epilogue_tile(const TmParams& p, const CUtensorM
                 z[0] += fx2(o < p.Cout ? __ldg(p.bias + o) : 0.0f, o + 1 < p.Cout ? __ldg(p.bias + o + 1) : 0.0f);
             }
             RealIdft<G, fx2>::run(z, y2);
+            if (p.act == kActGelu) {
+#pragma unroll
+                for (int gg = 0; gg < G; ++gg) y2[gg] = gelu2(y2[gg]);
+            }
 #pragma unroll
             for (int gg = 0; gg < G; ++gg) {
                 yv[j * G + gg] = y2[gg].x;
                 yv[(j + 1) * G + gg] = y2[gg].y;
-            }
-            if (p.act == kActGelu) {
-#pragma unroll
-                for (int gg = 0; gg < 2 * G; ++gg) yv[j * G + gg] = gelu(yv[j * G + gg]);
             }
         }
         // this buffer was last stored two groups ago: its TMA read must be complete

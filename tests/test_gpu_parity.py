@@ -120,6 +120,19 @@ def test_shapes_both_fused_kernels(Cout, Cin, G, kernel, io, monkeypatch):
     h.close()
 
 
+@pytest.mark.parametrize("Cout,Cin,G,path", [
+    (96, 96, 4, "tcgen05_tokens_on_n_resident_weights"), (384, 96, 4, "tcgen05_tokens_on_n_streamed_weights"),
+    (768, 192, 4, "tcgen05_tokens_on_n_resident_input"), (512, 128, 4, "tcgen05_tokens_on_n_resident_input"),
+    (96, 384, 4, "tcgen05_tokens_on_n_streamed_weights"), (64, 64, 8, "tcgen05_tokens_on_m_resident_weights"),
+])
+def test_default_kernel_choice(Cout, Cin, G, path):
+    """The planner's default for 16-bit I/O, so the parity cases cover each form."""
+    w = torch.zeros(Cout, Cin, G, dtype=torch.bfloat16, device=DEV)
+    h = eq.prepare(w, None)
+    assert h.path == path
+    h.close()
+
+
 @pytest.mark.parametrize("ystore", ["tma", "direct"])
 @pytest.mark.parametrize("Cout,Cin,G", [(50, 40, 4), (96, 96, 4), (200, 32, 4), (130, 96, 4), (96, 96, 2),
                                         (136, 64, 8), (768, 192, 4)])
