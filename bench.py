@@ -422,8 +422,8 @@ def main() -> None:
             bwd[key] = {"us_per_call": 1e3 * reduce_max(b0.elapsed_time(b1), dev) / Kb, "calls": Kb}
         bwd["device_status"] = h.device_status()
         bwd["kernels"] = {"dx": "fused forward kernel on the adjoint operator (1 launch)",
-                          "dw": "tcgen05 contraction over tokens + deterministic reduction / inverse DFT "
-                                "(3 launches)" if wl.io_dtype != "f32" else
+                          "dw": "tcgen05 contraction over tokens + deterministic reduction and inverse DFT "
+                                "(2 launches)" if wl.io_dtype != "f32" else
                                 "float64 CUDA-core kernel (clear + kernel + convert)"}
         del dxs
 

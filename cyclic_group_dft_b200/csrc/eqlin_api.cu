@@ -771,8 +771,8 @@ int plan_dw(int64_t Cout, int64_t Cin, int G, size_t max_smem, int sm_count, DwP
 }
 
 // Workspace of one weight-gradient call.  bf16 path: per CTA an fp32 slab ([G][NI][MO]
-// partial planes, then [MO] bias sums), followed (16-byte aligned) by the per-unit
-// float64 sums of those slabs.  fp32 path: a float64 [Cout][Cin][G] + [Cout] accumulator.
+// partial planes, then [MO] bias sums).  fp32 path: a float64 [Cout][Cin][G] + [Cout]
+// accumulator.
 size_t dw_slab_region_bytes(const DwPlan& pl, int64_t N) {
     const long long n_chunks = (N + eqlin::dw::kTok - 1) / eqlin::dw::kTok;
     const long long splits = std::max<long long>(1, std::min<long long>(pl.max_splits, n_chunks));
@@ -783,8 +783,7 @@ size_t dw_slab_region_bytes(const DwPlan& pl, int64_t N) {
 
 size_t dw_workspace_bytes(const DwPlan& pl, bool f32_path, int64_t Cout, int64_t Cin, int64_t G, int64_t N) {
     if (f32_path) return static_cast<size_t>(Cout * Cin * G + Cout) * sizeof(double);
-    return dw_slab_region_bytes(pl, N) +
-           static_cast<size_t>(pl.units()) * (pl.slab_floats + static_cast<size_t>(pl.MO)) * sizeof(double);
+    return dw_slab_region_bytes(pl, N);
 }
 
 template <int G, class T16>
@@ -892,7 +891,6 @@ int launch_dw(const DwPlan& pl, bool f32_path, int64_t Cout, int64_t Cin, int64_
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "weight-gradient launch");
     eqlin::DwFinalParams f;
     f.ws = p.ws;
-    f.P = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + dw_slab_region_bytes(pl, N));
     f.dw = dw;
     f.dbias = dbias;
     f.Cout = iCout;
@@ -902,17 +900,14 @@ int launch_dw(const DwPlan& pl, bool f32_path, int64_t Cout, int64_t Cin, int64_
     f.n_it = pl.n_it;
     f.n_splits = p.n_splits;
     f.slab_floats = pl.slab_floats;
-    const size_t per_unit = (pl.slab_floats + static_cast<size_t>(pl.MO) + 31) / 32;
-    eqlin::eqlin_dw_reduce_kernel<<<static_cast<unsigned>(pl.units() * per_unit), 256, 0, st>>>(f);
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "weight-gradient reduction launch");
-    const unsigned igrid = static_cast<unsigned>((Cout * Cin + 255) / 256);
+    const unsigned fgrid = static_cast<unsigned>(pl.units() * (pl.NI + 1) * ((pl.MO + 31) / 32));
     switch (iG) {
-        case 2: eqlin::eqlin_dw_idft_kernel<2><<<igrid, 256, 0, st>>>(f); break;
-        case 4: eqlin::eqlin_dw_idft_kernel<4><<<igrid, 256, 0, st>>>(f); break;
-        case 8: eqlin::eqlin_dw_idft_kernel<8><<<igrid, 256, 0, st>>>(f); break;
-        default: eqlin::eqlin_dw_idft_kernel<16><<<igrid, 256, 0, st>>>(f); break;
+        case 2: eqlin::eqlin_dw_finish_kernel<2><<<fgrid, 256, 0, st>>>(f); break;
+        case 4: eqlin::eqlin_dw_finish_kernel<4><<<fgrid, 256, 0, st>>>(f); break;
+        case 8: eqlin::eqlin_dw_finish_kernel<8><<<fgrid, 256, 0, st>>>(f); break;
+        default: eqlin::eqlin_dw_finish_kernel<16><<<fgrid, 256, 0, st>>>(f); break;
     }
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "weight-gradient inverse DFT launch");
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "weight-gradient reduction launch");
     return EQLIN_OK;
 }
 

@@ -37,9 +37,9 @@
 //               sums are formed in a fixed order.  Spectra use p.spec_bufs buffers.
 //               After the last chunk the same warps read the TMEM partial dW and write it
 //               to the CTA's slab of the workspace.
-// eqlin_dw_reduce_kernel then sums the slabs of each unit over its token splits in a
-// fixed order (deterministic, float64) and eqlin_dw_idft_kernel<G> runs the inverse real
-// DFT over the planes in float64 and writes dw (fp32) and dbias (fp32).
+// eqlin_dw_finish_kernel<G> then sums the slabs of each unit over its token splits in a
+// fixed order (deterministic, float64), runs the inverse real DFT over the planes in
+// float64 and writes dw (fp32) and dbias (fp32).
 //
 // Spectra layout (one buffer): A = G planes of 4 K-groups x MA atoms of 512 bytes
 // (MA = ceil(MO / 32)), then slack: a 128-row MMA reads 4 atoms along M, so for MO < 128
@@ -511,19 +511,15 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
     }
 }
 
-// Cross-CTA reduction, deterministic, in two small kernels:
-//  eqlin_dw_reduce_kernel  P[u][e] = sum over the unit's token splits s (in a fixed
-//                          order) of slab[u * n_splits + s][e], float64, for every slab
-//                          element e (the G planes and the bias sums).  Block = 32
-//                          consecutive elements; warp w sums splits w, w+8, ... with
-//                          several loads in flight; the 8 warp sums are added in order.
-//  eqlin_dw_idft_kernel    per (o, i): the inverse real DFT over the planes.  With
-//                          P_k = sum_n DY_k conj(X_k) (unscaled transforms),
+// Cross-CTA reduction and inverse DFT, deterministic, in one small kernel.
+// Block = (unit u, column ii of the unit, 32 consecutive rows oo), or the unit's bias
+// sums when ii == NI.  Warp w sums the slabs of splits w, w+8, w+16, ... in that order,
+// float64, for the block's G planes; the 8 warp sums are then added in warp order.
+// With P_k = sum_n DY_k conj(X_k) (unscaled transforms), warp 0 writes
 //   dw[o,i,m] = (1/G) [P_0 + (-1)^m P_{G/2} + 2 sum_{0<k<G/2} Re(P_k e^{+2 pi i m k / G})],
-//                          and dbias[o] from the bias sums of input tile 0.
+// and dbias[o] from the bias sums of the units of input tile 0.
 struct DwFinalParams {
     const float* ws;      // slabs: per CTA [G][NI][MO] then [MO]
-    double* P;            // per unit [G][NI][MO] then [MO]
     float* dw;            // [Cout, Cin, G]
     float* dbias;         // [Cout] or nullptr
     int Cout, Cin;
@@ -531,54 +527,73 @@ struct DwFinalParams {
     size_t slab_floats;   // G * NI * MO
 };
 
-__global__ void __launch_bounds__(256) eqlin_dw_reduce_kernel(const DwFinalParams f) {
-    __shared__ double red[8][32];
-    const size_t stride = f.slab_floats + f.MO;
-    const size_t blocks_per_unit = (stride + 31) / 32;
-    const int unit = static_cast<int>(blockIdx.x / blocks_per_unit);
-    const size_t e = (blockIdx.x % blocks_per_unit) * 32 + (threadIdx.x & 31);
-    const int warp = threadIdx.x >> 5;
-    double acc = 0.0;
-    if (e < stride) {
-        const float* src = f.ws + static_cast<size_t>(unit) * f.n_splits * stride + e;
-        int s = warp;
-        for (; s + 24 < f.n_splits; s += 32) {   // four loads in flight, added in split order
-            const float v0 = src[static_cast<size_t>(s) * stride];
-            const float v1 = src[static_cast<size_t>(s + 8) * stride];
-            const float v2 = src[static_cast<size_t>(s + 16) * stride];
-            const float v3 = src[static_cast<size_t>(s + 24) * stride];
-            acc += v0;
-            acc += v1;
-            acc += v2;
-            acc += v3;
-        }
-        for (; s < f.n_splits; s += 8) acc += src[static_cast<size_t>(s) * stride];
-    }
-    red[warp][threadIdx.x & 31] = acc;
-    __syncthreads();
-    if (warp == 0 && e < stride) {
-        double v = 0.0;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) v += red[w][threadIdx.x];
-        f.P[static_cast<size_t>(unit) * stride + e] = v;
-    }
-}
-
 template <int G>
-__global__ void __launch_bounds__(256) eqlin_dw_idft_kernel(const DwFinalParams f) {
-    const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (idx >= static_cast<long long>(f.Cout) * f.Cin) return;
-    const int o = static_cast<int>(idx % f.Cout), i = static_cast<int>(idx / f.Cout);
-    const int ot = o / f.MO, oo = o - ot * f.MO;
-    const int it = i / f.NI, ii = i - it * f.NI;
+__global__ void __launch_bounds__(256) eqlin_dw_finish_kernel(const DwFinalParams f) {
+    __shared__ double red[8][G][32];
+    const int n_og = (f.MO + 31) / 32;
+    const int per_unit = (f.NI + 1) * n_og;
+    const int unit = static_cast<int>(blockIdx.x) / per_unit;
+    const int rem = static_cast<int>(blockIdx.x) % per_unit;
+    const int ii = rem / n_og, oo = (rem % n_og) * 32 + (threadIdx.x & 31);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const bool bias_blk = ii == f.NI;
     const size_t stride = f.slab_floats + f.MO;
-    const double* P = f.P + static_cast<size_t>(ot * f.n_it + it) * stride;
-    double z[G], out[G];
+    const size_t pstride = static_cast<size_t>(f.NI) * f.MO;   // between planes of a slab
+    double acc[G];
+#pragma unroll
+    for (int pl = 0; pl < G; ++pl) acc[pl] = 0.0;
+    if (oo < f.MO) {
+        const float* src = f.ws + static_cast<size_t>(unit) * f.n_splits * stride +
+                           (bias_blk ? f.slab_floats + oo : static_cast<size_t>(ii) * f.MO + oo);
+        const int nv = bias_blk ? 1 : G;
+        int s = warp;
+        for (; s + 8 < f.n_splits; s += 16) {   // two splits in flight, added in split order
+            float v0[G], v1[G];
+#pragma unroll
+            for (int pl = 0; pl < G; ++pl) {
+                if (pl < nv) {
+                    v0[pl] = src[static_cast<size_t>(s) * stride + pl * pstride];
+                    v1[pl] = src[static_cast<size_t>(s + 8) * stride + pl * pstride];
+                }
+            }
+#pragma unroll
+            for (int pl = 0; pl < G; ++pl) {
+                if (pl < nv) {
+                    acc[pl] += v0[pl];
+                    acc[pl] += v1[pl];
+                }
+            }
+        }
+        for (; s < f.n_splits; s += 8) {
+#pragma unroll
+            for (int pl = 0; pl < G; ++pl)
+                if (pl < nv) acc[pl] += src[static_cast<size_t>(s) * stride + pl * pstride];
+        }
+    }
+#pragma unroll
+    for (int pl = 0; pl < G; ++pl) red[warp][pl][lane] = acc[pl];
+    __syncthreads();
+    if (warp != 0 || oo >= f.MO) return;
+    double z[G];
 #pragma unroll
     for (int pl = 0; pl < G; ++pl) {
-        const double v = P[(static_cast<size_t>(pl) * f.NI + ii) * f.MO + oo];
-        z[pl] = (pl < 2 ? v : 2.0 * v) / G;
+        double v = 0.0;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) v += red[w][pl][lane];
+        z[pl] = v;
     }
+    const int ot = unit / f.n_it, it = unit % f.n_it;
+    const int o = ot * f.MO + oo;
+    if (o >= f.Cout) return;
+    if (bias_blk) {
+        if (f.dbias != nullptr && it == 0) f.dbias[o] = static_cast<float>(z[0]);
+        return;
+    }
+    const int i = it * f.NI + ii;
+    if (i >= f.Cin) return;
+#pragma unroll
+    for (int pl = 0; pl < G; ++pl) z[pl] = (pl < 2 ? z[pl] : 2.0 * z[pl]) / G;
+    double out[G];
     if constexpr (G == 2) {
         out[0] = z[0] + z[1];
         out[1] = z[0] - z[1];
@@ -588,7 +603,6 @@ __global__ void __launch_bounds__(256) eqlin_dw_idft_kernel(const DwFinalParams 
     float* dst = f.dw + (static_cast<size_t>(o) * f.Cin + i) * G;
 #pragma unroll
     for (int m = 0; m < G; ++m) dst[m] = static_cast<float>(out[m]);
-    if (f.dbias != nullptr && i == 0) f.dbias[o] = static_cast<float>(P[f.slab_floats + oo]);
 }
 
 // ------------------------------------------------------------------ fp32 I/O

@@ -295,9 +295,9 @@ EQLIN_API int eqlin_backward_dw_workspace_size(const eqlin_handle* h, int64_t N,
  *              16-byte aligned, owned by the caller.  Its contents on entry do not
  *              matter and on exit are unspecified.  Two calls whose work overlaps on
  *              the GPU must not share it.
- *   stream     asynchronous on this stream: 3 launches for 16-bit I/O (the tcgen05
- *              contraction with a per-CTA partial sum, a deterministic reduction of
- *              the partial sums, the inverse DFT); for fp32, a clear, a float64
+ *   stream     asynchronous on this stream: 2 launches for 16-bit I/O (the tcgen05
+ *              contraction with a per-CTA partial sum, then a deterministic reduction
+ *              of the partial sums fused with the inverse DFT); for fp32, a clear, a float64
  *              CUDA-core kernel and a conversion.  Allocates nothing.
  *
  * 16-bit I/O: the spectra are rounded to the I/O type for the tensor cores and
