@@ -387,7 +387,8 @@ def main() -> None:
         e2e = {"value": aggregate_tokens_per_s(world, E, N, e2e_ms), "unit": "tokens/s", "steps": E,
                "h2d_bytes_per_step": x_pin.numel() * x_pin.element_size(),
                "d2h_bytes_per_step": y_pin.numel() * y_pin.element_size(),
-               "api": "Handle.forward_host (pinned host x -> device -> eqlin_forward -> pinned host y)"}
+               "api": "eqlin_forward_host (C ABI: pinned host x and y, chunked copies in and out "
+                      "overlapping the fused kernel on two streams)"}
 
     # ----------------------------------------------------------- backward calls
     # Measured after the forward's timed region, on the same rotating buffer sets

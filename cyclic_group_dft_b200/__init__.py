@@ -45,6 +45,7 @@ from ._capi import (  # noqa: F401
     eqlin_device_status,
     eqlin_forward,
     eqlin_forward_noalloc,
+    eqlin_forward_host,
     eqlin_last_error,
     eqlin_prepare_weights,
     eqlin_status_string,

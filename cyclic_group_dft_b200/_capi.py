@@ -51,6 +51,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 _vp, _i64, _int = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
 _lib.eqlin_prepare_weights.argtypes = [_vp, _vp, _i64, _i64, _i64, _int, _int, _vp, ctypes.POINTER(_vp)]
 _lib.eqlin_forward.argtypes = [_vp, _vp, _vp, _i64, _vp]
+_lib.eqlin_forward_host.argtypes = [_vp, _vp, _vp, _i64, _vp]
 _lib.eqlin_destroy.argtypes = [_vp]
 _lib.eqlin_device_status.argtypes = [_vp, ctypes.POINTER(_int)]
 _lib.eqlin_get_attr.argtypes = [_vp, _int, ctypes.POINTER(_i64)]
@@ -67,7 +68,7 @@ _lib.eqlin_status_string.restype = ctypes.c_char_p
 _lib.eqlin_last_error.argtypes = []
 _lib.eqlin_last_error.restype = ctypes.c_char_p
 _lib.eqlin_version.argtypes = []
-for _f in ("eqlin_prepare_weights", "eqlin_forward", "eqlin_destroy", "eqlin_device_status",
+for _f in ("eqlin_prepare_weights", "eqlin_forward", "eqlin_forward_host", "eqlin_destroy", "eqlin_device_status",
            "eqlin_get_attr", "eqlin_copy_freq_weights", "eqlin_check_shape", "eqlin_version",
            "eqlin_forward_noalloc", "eqlin_prepare_weights_ex", "eqlin_backward_dx",
            "eqlin_backward_dw_workspace_size", "eqlin_backward_dw"):
@@ -171,19 +172,9 @@ class Handle:
 
     def forward_host(self, x_host: torch.Tensor, out_host: torch.Tensor | None = None,
                      stream=None) -> torch.Tensor:
-        """Forward from and to host memory: copy x in, run, copy y back (synchronous)."""
-        if x_host.device.type != "cpu":
-            raise ValueError("forward_host takes a CPU tensor")
-        with torch.cuda.device(self.device):
-            s = torch.cuda.current_stream() if stream is None else stream
-            with torch.cuda.stream(s):
-                xd = x_host.to(self.device, non_blocking=True)
-                yd = eqlin_forward(self, xd, None, s)
-                if out_host is None:
-                    out_host = torch.empty(yd.shape, dtype=yd.dtype, pin_memory=x_host.is_pinned())
-                out_host.copy_(yd, non_blocking=True)
-            s.synchronize()
-        return out_host
+        """Forward from and to host memory through eqlin_forward_host (chunked copies in
+        and out overlapping the kernels); returns once y is in host memory."""
+        return eqlin_forward_host(self, x_host, out_host, stream)
 
     def device_status(self) -> int:
         return eqlin_device_status(self)
@@ -262,6 +253,30 @@ def eqlin_forward(h: Handle, x: torch.Tensor, y: torch.Tensor | None = None, str
         _check(_lib.eqlin_forward(h.ptr, x.data_ptr(), y.data_ptr(), N, _stream_ptr(stream)),
                "eqlin_forward")
     return y
+
+
+def eqlin_forward_host(h: Handle, x_host: torch.Tensor, y_host: torch.Tensor | None = None,
+                       stream=None) -> torch.Tensor:
+    """y_host [N, Cout, G] = EQ-Linear(x_host [N, Cin, G]), both in host memory (pinned
+    for overlapped copies).  Synchronises the stream before returning."""
+    if x_host.device.type != "cpu":
+        raise ValueError("eqlin_forward_host takes CPU tensors")
+    if x_host.dim() != 3 or x_host.shape[1] != h.Cin or x_host.shape[2] != h.G:
+        raise ValueError(f"x must be [N, {h.Cin}, {h.G}], got {tuple(x_host.shape)}")
+    if x_host.dtype != h.io_dtype or not x_host.is_contiguous():
+        raise ValueError(f"x must be contiguous {h.io_dtype}")
+    N = x_host.shape[0]
+    if y_host is None:
+        y_host = torch.empty((N, h.Cout, h.G), dtype=h.io_dtype, pin_memory=x_host.is_pinned())
+    elif y_host.shape != (N, h.Cout, h.G) or y_host.dtype != h.io_dtype or y_host.device.type != "cpu" \
+            or not y_host.is_contiguous():
+        raise ValueError("y has the wrong shape, dtype, device or layout")
+    with torch.cuda.device(h.device):
+        ptr = _stream_ptr(stream)
+        _check(_lib.eqlin_forward_host(h.ptr, x_host.data_ptr(), y_host.data_ptr(), N, ptr),
+               "eqlin_forward_host")
+        (stream if isinstance(stream, torch.cuda.Stream) else torch.cuda.ExternalStream(ptr)).synchronize()
+    return y_host
 
 
 def _check_rows(t: torch.Tensor, name: str, C: int, h: Handle) -> None:

@@ -926,6 +926,14 @@ struct eqlin_handle {
     DwPlan dwp;          // weight-gradient tiling (bf16 I/O)
     bool sync_check = false;
     unsigned long long timeout_ns = kDefaultTimeoutNs;
+    // eqlin_forward_host: device staging for two chunks, two streams, created on first use
+    std::mutex host_mutex;
+    int64_t host_chunk = 0;                     // tokens per chunk (0: not set up)
+    void* host_x[2] = {nullptr, nullptr};
+    void* host_y[2] = {nullptr, nullptr};
+    cudaStream_t host_st[2] = {nullptr, nullptr};
+    cudaEvent_t host_ev_in = nullptr;
+    cudaEvent_t host_ev_out[2] = {nullptr, nullptr};
 };
 
 namespace {
@@ -943,7 +951,41 @@ void free_handle(eqlin_handle* h) {
     if (h->buf_dx.bias_f32) cudaFree(h->buf_dx.bias_f32);
     if (h->buf_dx.w_f64) cudaFree(h->buf_dx.w_f64);
     if (h->buf_dx.bias_f64) cudaFree(h->buf_dx.bias_f64);
+    for (int k = 0; k < 2; ++k) {
+        if (h->host_x[k]) cudaFree(h->host_x[k]);
+        if (h->host_y[k]) cudaFree(h->host_y[k]);
+        if (h->host_st[k]) cudaStreamDestroy(h->host_st[k]);
+        if (h->host_ev_out[k]) cudaEventDestroy(h->host_ev_out[k]);
+    }
+    if (h->host_ev_in) cudaEventDestroy(h->host_ev_in);
     delete h;
+}
+
+size_t io_elem_bytes(int io) { return io == EQLIN_F32 ? 4 : 2; }
+
+// Staging of eqlin_forward_host: chunks of about 16 MB of x plus y (a multiple of 64
+// tokens), two of each, and two non-blocking streams.  Called with host_mutex held.
+int setup_host_staging(eqlin_handle* h) {
+    if (h->host_chunk > 0) return EQLIN_OK;
+    const size_t e = io_elem_bytes(h->io_dtype);
+    const size_t row_x = static_cast<size_t>(h->Cin * h->G) * e, row_y = static_cast<size_t>(h->Cout * h->G) * e;
+    int64_t tokens = static_cast<int64_t>((size_t(16) << 20) / (row_x + row_y)) / 64 * 64;
+    tokens = std::max<int64_t>(tokens, 64);
+    cudaError_t err;
+    for (int k = 0; k < 2; ++k) {
+        if ((err = cudaMalloc(&h->host_x[k], tokens * row_x)) != cudaSuccess ||
+            (err = cudaMalloc(&h->host_y[k], tokens * row_y)) != cudaSuccess) {
+            cudaGetLastError();
+            return fail(EQLIN_ERR_OOM, "staging allocation for the host-buffer forward");
+        }
+        if ((err = cudaStreamCreateWithFlags(&h->host_st[k], cudaStreamNonBlocking)) != cudaSuccess ||
+            (err = cudaEventCreateWithFlags(&h->host_ev_out[k], cudaEventDisableTiming)) != cudaSuccess)
+            return cuda_fail(err, "host-buffer forward streams");
+    }
+    if ((err = cudaEventCreateWithFlags(&h->host_ev_in, cudaEventDisableTiming)) != cudaSuccess)
+        return cuda_fail(err, "host-buffer forward streams");
+    h->host_chunk = tokens;
+    return EQLIN_OK;
 }
 
 }  // namespace
@@ -1196,6 +1238,61 @@ int eqlin_forward(const eqlin_handle* h, const void* x, void* y, int64_t N, void
         if (e != cudaSuccess) return cuda_fail(e, "forward (EQLIN_SYNC_CHECK)");
         e = cudaMemcpy(&dst, h->buf.status, sizeof(int), cudaMemcpyDeviceToHost);
         if (e != cudaSuccess) return cuda_fail(e, "status read");
+        if (dst != 0) return fail(dst, "device reported an error (status word)");
+    }
+    return EQLIN_OK;
+}
+
+int eqlin_forward_host(eqlin_handle* h, const void* x_host, void* y_host, int64_t N, void* stream) {
+    if (!h) return fail(EQLIN_ERR_INVALID_ARG, "handle is NULL");
+    if (N < 0) return fail(EQLIN_ERR_INVALID_ARG, "N < 0");
+    if (N == 0) return EQLIN_OK;
+    if (!x_host || !y_host) return fail(EQLIN_ERR_INVALID_ARG, "x_host or y_host is NULL");
+    if (N >= (int64_t(1) << 31)) return fail(EQLIN_ERR_UNSUPPORTED, "N must be below 2^31");
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev != h->device) return fail(EQLIN_ERR_INVALID_ARG, "current device differs from the handle's device");
+    std::lock_guard<std::mutex> lock(h->host_mutex);
+    int s = setup_host_staging(h);
+    if (s != EQLIN_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t el = io_elem_bytes(h->io_dtype);
+    const size_t row_x = static_cast<size_t>(h->Cin * h->G) * el, row_y = static_cast<size_t>(h->Cout * h->G) * el;
+    // both internal streams start after the work already queued on the caller's stream
+    if ((e = cudaEventRecord(h->host_ev_in, st)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    for (int k = 0; k < 2; ++k)
+        if ((e = cudaStreamWaitEvent(h->host_st[k], h->host_ev_in, 0)) != cudaSuccess)
+            return cuda_fail(e, "cudaStreamWaitEvent");
+    // chunk i on stream i % 2 with buffers i % 2: a stream's own order protects its
+    // buffers, and the two streams overlap the copies in and out
+    const auto* xb = static_cast<const uint8_t*>(x_host);
+    auto* yb = static_cast<uint8_t*>(y_host);
+    int64_t i = 0;
+    for (int64_t n0 = 0; n0 < N; n0 += h->host_chunk, ++i) {
+        const int k = static_cast<int>(i & 1);
+        const int64_t n = std::min<int64_t>(h->host_chunk, N - n0);
+        cudaStream_t sk = h->host_st[k];
+        if ((e = cudaMemcpyAsync(h->host_x[k], xb + n0 * row_x, n * row_x, cudaMemcpyHostToDevice, sk)) !=
+            cudaSuccess)
+            return cuda_fail(e, "host-to-device copy");
+        s = launch_forward(h->plan, h->Cout, h->Cin, h->G, h->sm_count, h->host_x[k], h->host_y[k], n, h->buf,
+                           h->timeout_ns, sk);
+        if (s != EQLIN_OK) return s;
+        if ((e = cudaMemcpyAsync(yb + n0 * row_y, h->host_y[k], n * row_y, cudaMemcpyDeviceToHost, sk)) !=
+            cudaSuccess)
+            return cuda_fail(e, "device-to-host copy");
+    }
+    for (int k = 0; k < 2; ++k) {
+        if ((e = cudaEventRecord(h->host_ev_out[k], h->host_st[k])) != cudaSuccess ||
+            (e = cudaStreamWaitEvent(st, h->host_ev_out[k], 0)) != cudaSuccess)
+            return cuda_fail(e, "stream join");
+    }
+    if (h->sync_check) {
+        int dst = 0;
+        if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return cuda_fail(e, "forward (EQLIN_SYNC_CHECK)");
+        if ((e = cudaMemcpy(&dst, h->buf.status, sizeof(int), cudaMemcpyDeviceToHost)) != cudaSuccess)
+            return cuda_fail(e, "status read");
         if (dst != 0) return fail(dst, "device reported an error (status word)");
     }
     return EQLIN_OK;

@@ -120,6 +120,31 @@ EQLIN_API int eqlin_prepare_weights(const void* w, const void* bias, int64_t Cou
 EQLIN_API int eqlin_forward(const eqlin_handle* h, const void* x, void* y, int64_t N, void* stream);
 
 /*
+ * eqlin_forward_host -- the same forward with x and y in HOST memory: the library
+ * copies x in, runs the fused kernel and copies y back, chunk by chunk, so that the
+ * host-to-device copy of one chunk, the kernel of another and the device-to-host copy
+ * of a third overlap (two internal streams; full-duplex copies).
+ *
+ *   h        handle from eqlin_prepare_weights.  The first call allocates the handle's
+ *            staging buffers (two chunks of x and of y, about 32 MB) and two streams,
+ *            freed by eqlin_destroy.  Calls on one handle are serialised by the
+ *            library (a mutex for the host side, the internal streams for the GPU).
+ *   x_host   host, [N, Cin, G] of the handle's io_dtype.  Pinned memory (cudaHostAlloc,
+ *            cudaHostRegister, torch pin_memory) lets the copies overlap; pageable
+ *            memory works but the copies then serialise with the host.
+ *   y_host   host, [N, Cout, G] of io_dtype; must not overlap x_host.
+ *   N        number of tokens; N == 0 is a no-op returning EQLIN_OK.  N < 2^31.
+ *   stream   ordering: the work starts after everything already queued on `stream`,
+ *            and `stream` waits for its completion.  Asynchronous: synchronise `stream`
+ *            before reading y_host (or reusing x_host).
+ *
+ * Errors: INVALID_ARG (null handle, N < 0, null x_host/y_host with N > 0, wrong
+ * current device), OOM (staging allocation), CUDA (copy or launch failure).  Device
+ * timeouts are reported as for eqlin_forward.
+ */
+EQLIN_API int eqlin_forward_host(eqlin_handle* h, const void* x_host, void* y_host, int64_t N, void* stream);
+
+/*
  * eqlin_destroy -- free the handle and its device memory.  The caller must
  * ensure no forward using it is still executing (e.g. synchronise the streams).
  * NULL is accepted and ignored.  Returns EQLIN_OK, or CUDA if a free failed.

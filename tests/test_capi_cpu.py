@@ -88,6 +88,8 @@ def test_forward_rejects_bad_arguments_on_host():
     s = ctypes.c_int()
     assert lib.eqlin_device_status(None, ctypes.byref(s)) == eq.EQLIN_ERR_INVALID_ARG
     assert lib.eqlin_copy_freq_weights(None, None, 0) == eq.EQLIN_ERR_INVALID_ARG
+    assert lib.eqlin_forward_host(None, 16, 16, 4, None) == eq.EQLIN_ERR_INVALID_ARG
+    assert "NULL" in eq.eqlin_last_error()
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks behaviour without a GPU")

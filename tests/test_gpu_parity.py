@@ -312,3 +312,25 @@ def test_handles_sharing_a_kernel_keep_their_shared_memory():
         torch.cuda.synchronize()
         _assert_parity(torch.bfloat16, y, ref, f"path={h.path} smem={h.attr('smem_bytes')}")
         h.close()
+
+
+@pytest.mark.parametrize("pinned", [True, False])
+@pytest.mark.parametrize("name,N", [("p4_c96_bf16", 3 * 10880 + 517), ("p4_c96_bf16", 300), ("p4_mlp_bf16", 20000),
+                                    ("c16_c32_bf16", 40000), ("tiny_p4_fp32", 5000)])
+def test_forward_from_host_buffers(name, N, pinned):
+    """eqlin_forward_host: chunked copies in and out around the fused kernel, several
+    chunks with a ragged last one, pinned or pageable host memory; equal to the
+    device-buffer forward bit for bit, and to the oracle within the tolerance."""
+    wl = workloads.WORKLOADS[name]
+    x, w, bias = workloads.make_inputs(wl, seed=21, N=N)
+    h = eq.prepare(w.to(DEV), None if bias is None else bias.to(DEV), io_dtype=wl.torch_dtype)
+    xh = x.pin_memory() if pinned else x.clone()
+    y_host = h.forward_host(xh)
+    y_dev = h.forward(x.to(DEV)).cpu()
+    assert h.device_status() == eq.EQLIN_OK
+    assert torch.equal(y_host, y_dev)
+    idx = workloads.sample_tokens(N, 256, seed=4)
+    _assert_parity(wl.torch_dtype, y_host[idx], _ref(x[idx], w, bias), f"{name} N={N} pinned={pinned}")
+    y2 = h.forward_host(xh, y_host)            # again, into the same output, staging reused
+    assert torch.equal(y2, y_dev)
+    h.close()
