@@ -198,3 +198,24 @@ def test_backward_argument_errors():
     dw_ref, db_ref = oracle.backward_dw(dy, x)
     _assert(torch.bfloat16, dw.cpu(), dw_ref, "dw without the flag")
     h.close()
+
+
+@pytest.mark.parametrize("Cout,Cin,G", [(1, 1, 8), (1, 1, 16), (2, 2, 4), (4, 4, 2), (3, 5, 8), (1024, 1024, 4),
+                                        (64, 2048, 4)])
+def test_backward_edge_channel_counts(Cout, Cin, G):
+    """dx, dw and dbias at the fewest channels a 16-byte row allows and for large layers."""
+    gen = torch.Generator().manual_seed(Cout * 5 + Cin + G)
+    N = 333 if Cout * Cin < 2 ** 17 else 97
+    x = torch.randn(N, Cin, G, generator=gen).to(torch.bfloat16)
+    w = (torch.randn(Cout, Cin, G, generator=gen) / np.sqrt(Cin * G)).to(torch.bfloat16)
+    dy = torch.randn(N, Cout, G, generator=gen).to(torch.bfloat16)
+    h = _prep(w, None, torch.bfloat16)
+    dx = h.backward_dx(dy.to(DEV))
+    dw, db = h.backward_dw(x.to(DEV), dy.to(DEV))
+    torch.cuda.synchronize()
+    assert h.device_status() == eq.EQLIN_OK
+    _assert(torch.bfloat16, dx.cpu(), oracle.backward_dx(dy, w), f"dx {Cout},{Cin},{G}")
+    dw_ref, db_ref = oracle.backward_dw(dy, x)
+    _assert(torch.bfloat16, dw.cpu(), dw_ref, f"dw {Cout},{Cin},{G}")
+    _assert(torch.bfloat16, db.cpu(), db_ref, f"dbias {Cout},{Cin},{G}")
+    h.close()

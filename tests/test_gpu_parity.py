@@ -133,6 +133,29 @@ def test_default_kernel_choice(Cout, Cin, G, path):
     h.close()
 
 
+EDGE_SHAPES = [  # (Cout, Cin, G): the fewest channels 16-byte rows allow, and large layers
+    (1, 1, 8), (1, 1, 16), (2, 2, 4), (4, 4, 2), (8, 4, 2), (4, 1, 8), (3, 5, 8),
+    (1024, 1024, 4), (2048, 64, 8), (64, 2048, 4), (512, 512, 16),
+]
+
+
+@pytest.mark.parametrize("kernel", ["default", "tn", "tm", "tnr"])
+@pytest.mark.parametrize("Cout,Cin,G", EDGE_SHAPES)
+def test_edge_channel_counts(Cout, Cin, G, kernel, monkeypatch):
+    """Smallest channel counts (a 16-byte row), where one 32- or 16-channel chunk is mostly
+    padding, and large layers with many weight chunks, on each fused kernel."""
+    if kernel != "default":
+        monkeypatch.setenv("EQLIN_KERNEL", kernel)
+    gen = torch.Generator().manual_seed(Cout * 7 + Cin * 3 + G)
+    N = 333 if Cout * Cin < 2 ** 17 else 97   # the oracle's definition loop stays a few seconds
+    x = torch.randn(N, Cin, G, generator=gen).to(torch.bfloat16)
+    w = (torch.randn(Cout, Cin, G, generator=gen) / np.sqrt(Cin * G)).to(torch.bfloat16)
+    bias = (torch.randn(Cout, generator=gen) * 0.3).to(torch.bfloat16)
+    y, h = _run(x, w, bias, torch.bfloat16)
+    _assert_parity(torch.bfloat16, y, _ref(x, w, bias), f"Cout={Cout} Cin={Cin} G={G} {kernel} path={h.path}")
+    h.close()
+
+
 @pytest.mark.parametrize("ystore", ["tma", "direct"])
 @pytest.mark.parametrize("Cout,Cin,G", [(50, 40, 4), (96, 96, 4), (200, 32, 4), (130, 96, 4), (96, 96, 2),
                                         (136, 64, 8), (768, 192, 4)])
