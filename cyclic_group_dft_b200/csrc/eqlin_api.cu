@@ -938,6 +938,21 @@ struct eqlin_handle {
 
 namespace {
 
+void release_host_staging(eqlin_handle* h) {
+    for (int k = 0; k < 2; ++k) {
+        if (h->host_x[k]) cudaFree(h->host_x[k]);
+        if (h->host_y[k]) cudaFree(h->host_y[k]);
+        if (h->host_st[k]) cudaStreamDestroy(h->host_st[k]);
+        if (h->host_ev_out[k]) cudaEventDestroy(h->host_ev_out[k]);
+        h->host_x[k] = h->host_y[k] = nullptr;
+        h->host_st[k] = nullptr;
+        h->host_ev_out[k] = nullptr;
+    }
+    if (h->host_ev_in) cudaEventDestroy(h->host_ev_in);
+    h->host_ev_in = nullptr;
+    h->host_chunk = 0;
+}
+
 void free_handle(eqlin_handle* h) {
     if (!h) return;
     if (h->buf.img) cudaFree(h->buf.img);
@@ -951,13 +966,7 @@ void free_handle(eqlin_handle* h) {
     if (h->buf_dx.bias_f32) cudaFree(h->buf_dx.bias_f32);
     if (h->buf_dx.w_f64) cudaFree(h->buf_dx.w_f64);
     if (h->buf_dx.bias_f64) cudaFree(h->buf_dx.bias_f64);
-    for (int k = 0; k < 2; ++k) {
-        if (h->host_x[k]) cudaFree(h->host_x[k]);
-        if (h->host_y[k]) cudaFree(h->host_y[k]);
-        if (h->host_st[k]) cudaStreamDestroy(h->host_st[k]);
-        if (h->host_ev_out[k]) cudaEventDestroy(h->host_ev_out[k]);
-    }
-    if (h->host_ev_in) cudaEventDestroy(h->host_ev_in);
+    release_host_staging(h);
     delete h;
 }
 
@@ -976,14 +985,19 @@ int setup_host_staging(eqlin_handle* h) {
         if ((err = cudaMalloc(&h->host_x[k], tokens * row_x)) != cudaSuccess ||
             (err = cudaMalloc(&h->host_y[k], tokens * row_y)) != cudaSuccess) {
             cudaGetLastError();
+            release_host_staging(h);   // nothing half set up survives a failure
             return fail(EQLIN_ERR_OOM, "staging allocation for the host-buffer forward");
         }
         if ((err = cudaStreamCreateWithFlags(&h->host_st[k], cudaStreamNonBlocking)) != cudaSuccess ||
-            (err = cudaEventCreateWithFlags(&h->host_ev_out[k], cudaEventDisableTiming)) != cudaSuccess)
+            (err = cudaEventCreateWithFlags(&h->host_ev_out[k], cudaEventDisableTiming)) != cudaSuccess) {
+            release_host_staging(h);
             return cuda_fail(err, "host-buffer forward streams");
+        }
     }
-    if ((err = cudaEventCreateWithFlags(&h->host_ev_in, cudaEventDisableTiming)) != cudaSuccess)
+    if ((err = cudaEventCreateWithFlags(&h->host_ev_in, cudaEventDisableTiming)) != cudaSuccess) {
+        release_host_staging(h);
         return cuda_fail(err, "host-buffer forward streams");
+    }
     h->host_chunk = tokens;
     return EQLIN_OK;
 }
