@@ -547,21 +547,21 @@ __global__ void __launch_bounds__(256) eqlin_dw_finish_kernel(const DwFinalParam
                            (bias_blk ? f.slab_floats + oo : static_cast<size_t>(ii) * f.MO + oo);
         const int nv = bias_blk ? 1 : G;
         int s = warp;
-        for (; s + 8 < f.n_splits; s += 16) {   // two splits in flight, added in split order
-            float v0[G], v1[G];
+        // four splits in flight (4G loads per thread), added in split order
+        constexpr int kIn = 4;
+        for (; s + 8 * (kIn - 1) < f.n_splits; s += 8 * kIn) {
+            float v[kIn][G];
 #pragma unroll
-            for (int pl = 0; pl < G; ++pl) {
-                if (pl < nv) {
-                    v0[pl] = src[static_cast<size_t>(s) * stride + pl * pstride];
-                    v1[pl] = src[static_cast<size_t>(s + 8) * stride + pl * pstride];
-                }
+            for (int u = 0; u < kIn; ++u) {
+#pragma unroll
+                for (int pl = 0; pl < G; ++pl)
+                    if (pl < nv) v[u][pl] = src[static_cast<size_t>(s + 8 * u) * stride + pl * pstride];
             }
 #pragma unroll
-            for (int pl = 0; pl < G; ++pl) {
-                if (pl < nv) {
-                    acc[pl] += v0[pl];
-                    acc[pl] += v1[pl];
-                }
+            for (int u = 0; u < kIn; ++u) {
+#pragma unroll
+                for (int pl = 0; pl < G; ++pl)
+                    if (pl < nv) acc[pl] += v[u][pl];
             }
         }
         for (; s < f.n_splits; s += 8) {
