@@ -494,7 +494,8 @@ def main() -> None:
     roof["frac_of_roofline_time"] = max(t_hbm, t_tc) / avg_launch_s
     roof["bytes_per_launch"] = bytes_launch
     roof["tensor_tflops"] = tflops
-    roof["tensor_frac"] = tflops / peaks["bf16_tflops"]
+    roof["tensor_frac"] = tflops / peaks["bf16_tflops"]                       # burst peak: the headline
+    roof["tensor_frac_sustained"] = tflops / peaks["bf16_tflops_sustained"]   # seconds-long GEMM peak
 
     if mlp is not None:
         e, H = wl.elem_bytes, mlp["H"]
