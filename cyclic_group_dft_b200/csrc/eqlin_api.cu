@@ -654,6 +654,7 @@ struct DwPlan {
     int MA = 0, NA = 0;   // 32-channel atoms of the MN-major spectra: ceil(MO / 32), ceil(NI / 32)
     int cpb_dy = 0, cpb_x = 0;
     int raw_stages = 0, spec_bufs = 0;
+    int tok = 0;          // tokens per chunk (dw::Cfg<G>::kTok)
     uint32_t dy_bytes = 0, raw_bytes = 0, a_bytes = 0, b_bytes = 0, tmem_cols = 0;
     size_t smem_bytes = 0, slab_floats = 0;
     int units() const { return n_ot * n_it; }
@@ -685,23 +686,36 @@ int max_dw_units(int G) {
 // Shared memory of the weight-gradient kernel: raw ring (RS stages of the 32-token dy and
 // x tiles), SB spectra buffers (A: G dy planes of 4 K-groups x MA atoms of 512 B, plus
 // the slack a 128-row MMA reads past the last plane; B: G x planes of 4 x NA atoms),
-// the dbias slots [32 tokens][MO] and the barriers.
+// the dbias slots [kTok tokens][MO] and the barriers.
+// tokens per weight-gradient chunk, as the kernel instantiated for G uses them
+int dw_tok(int G) {
+    switch (G) {
+        case 2: return eqlin::dw::Cfg<2>::kTok;
+        case 4: return eqlin::dw::Cfg<4>::kTok;
+        case 8: return eqlin::dw::Cfg<8>::kTok;
+        default: return eqlin::dw::Cfg<16>::kTok;
+    }
+}
+
 size_t dw_smem(int MO, int NI, int G, int RS, int SB, DwPlan* out) {
     const int MA = (MO + 31) / 32, NA = (NI + 31) / 32;
-    const size_t raw = round_kb(static_cast<size_t>(eqlin::dw::kTok) * (MO + NI) * G * 2);
-    const size_t a = round_kb(static_cast<size_t>(G) * 4 * MA * 512 + static_cast<size_t>(4 - MA) * 512);
-    const size_t b = round_kb(static_cast<size_t>(G) * 4 * NA * 512);
+    const size_t raw = round_kb(static_cast<size_t>(dw_tok(G)) * (MO + NI) * G * 2);
+    const int KG = dw_tok(G) / 8;
+    // a 128-row MMA reads 4 atoms along M from each K group, MA of them written
+    const size_t a = round_kb(static_cast<size_t>(G) * KG * MA * 512 + static_cast<size_t>(4 - MA) * 512);
+    const size_t b = round_kb(static_cast<size_t>(G) * KG * NA * 512);
     const size_t total = kSmemAlignSlack + static_cast<size_t>(RS) * raw + static_cast<size_t>(SB) * (a + b) +
-                         static_cast<size_t>(eqlin::dw::kTok) * MO * 4 + 256;
+                         static_cast<size_t>(dw_tok(G)) * MO * 4 + 256;
     if (out) {
         out->MA = MA;
         out->NA = NA;
-        out->dy_bytes = static_cast<uint32_t>(eqlin::dw::kTok) * MO * G * 2;
+        out->dy_bytes = static_cast<uint32_t>(dw_tok(G)) * MO * G * 2;
         out->raw_bytes = static_cast<uint32_t>(raw);
         out->a_bytes = static_cast<uint32_t>(a);
         out->b_bytes = static_cast<uint32_t>(b);
         out->raw_stages = RS;
         out->spec_bufs = SB;
+        out->tok = dw_tok(G);
         out->smem_bytes = total;
     }
     return total;
@@ -760,7 +774,7 @@ int plan_dw(int64_t Cout, int64_t Cin, int G, size_t max_smem, int sm_count, DwP
     pl->cpb_dy = box_channels(best_mo, G, cpu);
     pl->cpb_x = box_channels(best_ni, G, cpu);
     if (pl->cpb_dy == 0 || pl->cpb_x == 0) return fail(EQLIN_ERR_UNSUPPORTED, "no TMA box width for the tile");
-    if (eqlin::dw::kTok * (best_mo + best_ni) / cpu > max_dw_units(G))
+    if (dw_tok(G) * (best_mo + best_ni) / cpu > max_dw_units(G))
         return fail(EQLIN_ERR_UNSUPPORTED, "weight-gradient tile has more transform units than threads can hold");
     dw_smem(best_mo, best_ni, G, rs, sb, pl);
     int cols = 32;
@@ -774,7 +788,7 @@ int plan_dw(int64_t Cout, int64_t Cin, int G, size_t max_smem, int sm_count, DwP
 // partial planes, then [MO] bias sums).  fp32 path: a float64 [Cout][Cin][G] + [Cout]
 // accumulator.
 size_t dw_slab_region_bytes(const DwPlan& pl, int64_t N) {
-    const long long n_chunks = (N + eqlin::dw::kTok - 1) / eqlin::dw::kTok;
+    const long long n_chunks = (N + pl.tok - 1) / pl.tok;
     const long long splits = std::max<long long>(1, std::min<long long>(pl.max_splits, n_chunks));
     const size_t grid = static_cast<size_t>(pl.units()) * static_cast<size_t>(splits);
     const size_t bytes = grid * (pl.slab_floats + static_cast<size_t>(pl.MO)) * sizeof(float);
@@ -851,9 +865,9 @@ int launch_dw(const DwPlan& pl, bool f32_path, int64_t Cout, int64_t Cin, int64_
         return EQLIN_OK;
     }
     CUtensorMap mdy, mx;
-    int s = encode_rows_map(&mdy, dy, Cout * G, N, pl.cpb_dy * iG, eqlin::dw::kTok, pl.io);
+    int s = encode_rows_map(&mdy, dy, Cout * G, N, pl.cpb_dy * iG, dw_tok(G), pl.io);
     if (s != EQLIN_OK) return s;
-    s = encode_rows_map(&mx, x, Cin * G, N, pl.cpb_x * iG, eqlin::dw::kTok, pl.io);
+    s = encode_rows_map(&mx, x, Cin * G, N, pl.cpb_x * iG, dw_tok(G), pl.io);
     if (s != EQLIN_OK) return s;
     eqlin::DwParams p;
     p.ws = static_cast<float*>(ws);
@@ -862,7 +876,7 @@ int launch_dw(const DwPlan& pl, bool f32_path, int64_t Cout, int64_t Cin, int64_
     p.MO = pl.MO;
     p.NI = pl.NI;
     p.n_it = pl.n_it;
-    p.n_chunks = (N + eqlin::dw::kTok - 1) / eqlin::dw::kTok;
+    p.n_chunks = (N + dw_tok(G) - 1) / dw_tok(G);
     p.n_splits = static_cast<int>(std::max<long long>(1, std::min<long long>(pl.max_splits, p.n_chunks)));
     p.cpb_dy = pl.cpb_dy;
     p.cpb_x = pl.cpb_x;

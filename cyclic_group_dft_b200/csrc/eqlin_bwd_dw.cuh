@@ -17,8 +17,8 @@
 // Kernel eqlin_dw_tc_kernel<G>: the grid is units x token splits.  A unit is an
 // (MO-row output tile, NI-column input tile) pair; each CTA owns one unit and a
 // contiguous range of 32-token chunks, and keeps its partial dW in TMEM:
-//   warp 0      TMA producer: per chunk the dy tile [32 tokens x MO*G] and the x tile
-//               [32 tokens x NI*G] into a raw ring of p.raw_stages stages (zero fill past
+//   warp 0      TMA producer: per chunk the dy tile [kTok tokens x MO*G] and the x tile
+//               [kTok tokens x NI*G] into a raw ring of p.raw_stages stages (zero fill past
 //               N, Cout, Cin).
 //   warp 1      MMA issuer + TMEM owner: per chunk and 16-token K step, tcgen05.mma with
 //               A = DY^ plane [128 rows (MO valid) x 16 tokens], B = X^ plane [NI x 16],
@@ -64,9 +64,9 @@ struct DwParams {
     int MO, NI;                // rows / columns of a unit (multiples of 16; MO <= 128, G*NI <= 512)
     int n_it;                  // input tiles per output tile
     int n_splits;              // CTAs per unit (token splits)
-    long long n_chunks;        // ceil(N / 32)
+    long long n_chunks;        // ceil(N / kTok)
     int cpb_dy, cpb_x;         // channels per TMA box of the dy / x tile
-    uint32_t dy_bytes;         // dy part of a raw stage: 32 * MO * G * 2
+    uint32_t dy_bytes;         // dy part of a raw stage: kTok * MO * G * 2
     uint32_t raw_bytes;        // one raw stage: dy part + x part (multiple of 1 KB)
     uint32_t a_bytes;          // A (dy spectra) region of one spectra buffer (multiple of 1 KB)
     uint32_t b_bytes;          // B (x spectra) region (multiple of 1 KB)
@@ -80,7 +80,6 @@ struct DwParams {
 
 namespace dw {
 
-constexpr int kTok = 32;           // tokens per chunk (4 atoms of 8 K-rows)
 constexpr int kMaxRawStages = 8;   // raw ring depth is a launch parameter (p.raw_stages)
 constexpr int kMaxSpecBufs = 2;
 constexpr int kWarpProducer = 0;
@@ -91,15 +90,21 @@ constexpr int kWarpDft0 = 2;
 // dependent DFT chains); with the per-token units the transform needs <= 112 registers.
 template <int G>
 struct Cfg {
+    // tokens per chunk: 32 (two MMA K steps) for G <= 4; 16 for G >= 8, where a token's
+    // raw rows are twice as long, so that the raw ring keeps four or more stages (B200:
+    // weight gradient of C16 C32 218 vs 258 us, p8 C64 30.8 vs 35.0 us; p4 C96 81.4 us with
+    // 32 tokens against 98.4 with 16)
+    static constexpr int kTok = G >= 8 ? 16 : 32;
+    static constexpr int kKGroups = kTok / 8;   // 8-token K groups per spectra plane
     static constexpr int kDftWarps = 16;
     static constexpr int kDftThreads = kDftWarps * 32;
     static constexpr int kThreads = (2 + kDftWarps) * 32;
     // channels per transform unit: one 16-byte store per plane for G <= 4, 8 bytes for
     // G = 8, 4 bytes for G = 16 (where the DFT itself dominates and threads are plenty)
     static constexpr int kChanPerUnit = G <= 4 ? 8 : (G == 8 ? 4 : 2);
-    // units per transform thread and chunk, at most: 32 tokens x (MO + NI) / kChanPerUnit
+    // units per transform thread and chunk, at most: kTok tokens x (MO + NI) / kChanPerUnit
     // with MO <= 128 and G * NI <= 512, NI <= 256
-    static constexpr int kMaxUnits = 32 * (128 + (512 / G < 256 ? 512 / G : 256)) / kChanPerUnit;
+    static constexpr int kMaxUnits = kTok * (128 + (512 / G < 256 ? 512 / G : 256)) / kChanPerUnit;
     static constexpr int kMaxPasses = (kMaxUnits + kDftThreads - 1) / kDftThreads;
 
 };
@@ -145,7 +150,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, int* s
 // One unit of the transform: one token t of the chunk x CPU consecutive channels
 // c0 .. c0+CPU-1 of the dy tile or of the x tile (CPU = Cfg<G>::kChanPerUnit).  Raw tile
 // layout: boxes of cpb channels (cpb a multiple of CPU, so a unit never straddles two
-// boxes), each [32 tokens][cpb*G].  The unit's CPU*G values are CPU*G/2 32-bit words,
+// boxes), each [kTok tokens][cpb*G].  The unit's CPU*G values are CPU*G/2 32-bit words,
 // channel c0+j in words j*G/2 .. (j+1)*G/2-1.
 template <int G, int CPU>
 __device__ __forceinline__ void load_unit(const uint8_t* src, int lane, uint32_t (&w)[CPU * G / 2]) {
@@ -250,7 +255,7 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
     // bias_sm[t][c]: group sums of dy channel c at chunk token t, over every chunk; each
     // slot has a single writer (the unit -> thread map is the same for every chunk), so
     // the per-CTA sums are formed in a fixed order
-    uint64_t* bars = reinterpret_cast<uint64_t*>(bias_sm + dw::kTok * p.MO);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(bias_sm + dw::Cfg<G>::kTok * p.MO);
     const int RS = p.raw_stages, SB = p.spec_bufs;
     dw::Ctl* ctl = reinterpret_cast<dw::Ctl*>(bars + 2 * RS + 2 * SB + 2);
 
@@ -297,7 +302,7 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
         // A-region tail rows (read by the MMA, never written by the transform): zero
         // A-region slack after the G planes (read by the 128-row MMA of the last plane,
         // never written by the transform): zero
-        const uint32_t tail0 = static_cast<uint32_t>(G) * 4u * static_cast<uint32_t>(p.MA) * 512u;
+        const uint32_t tail0 = static_cast<uint32_t>(G) * dw::Cfg<G>::kKGroups * static_cast<uint32_t>(p.MA) * 512u;
         for (int b = 0; b < SB; ++b) {
             uint8_t* a = spec0 + static_cast<size_t>(b) * spec_bytes;
             for (uint32_t idx = tail0 / 16 + t; idx < p.a_bytes / 16; idx += kDftThreads)
@@ -316,15 +321,15 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             const int nb_dy = p.MO / p.cpb_dy, nb_x = p.NI / p.cpb_x;
-            const uint32_t box_dy = dw::kTok * p.cpb_dy * G * 2, box_x = dw::kTok * p.cpb_x * G * 2;
-            const uint32_t tx = p.dy_bytes + dw::kTok * p.NI * G * 2;
+            const uint32_t box_dy = dw::Cfg<G>::kTok * p.cpb_dy * G * 2, box_x = dw::Cfg<G>::kTok * p.cpb_x * G * 2;
+            const uint32_t tx = p.dy_bytes + dw::Cfg<G>::kTok * p.NI * G * 2;
             const uint32_t s_raw0 = ptx::smem_u32(raw0);
             int issued = 0;
             for (int j = 0; j < n_mine; ++j) {
                 const int s = j % RS;
                 const uint32_t ph = static_cast<uint32_t>(j / RS) & 1u;
                 if (!dw::wait_bounded(bar_raw_empty(s), ph ^ 1u, ctl, p.status, p.timeout_ns)) break;
-                const int n0 = static_cast<int>((c_begin + j) * dw::kTok);
+                const int n0 = static_cast<int>((c_begin + j) * dw::Cfg<G>::kTok);
                 const uint32_t dst = s_raw0 + s * p.raw_bytes;
                 ptx::mbar_arrive_expect_tx(bar_raw_full(s), tx);
                 for (int b = 0; b < nb_dy; ++b)
@@ -350,7 +355,7 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
             const uint32_t s_spec0 = ptx::smem_u32(spec0);
             const uint32_t sbo_a = static_cast<uint32_t>(p.MA) * 512u, sbo_b = static_cast<uint32_t>(p.NA) * 512u;
             const uint32_t hi_a = ptx::sdesc_mn_sw64_hi(sbo_a), hi_b = ptx::sdesc_mn_sw64_hi(sbo_b);
-            const uint32_t plane_a16 = 4u * sbo_a / 16u, plane_b16 = 4u * sbo_b / 16u;
+            const uint32_t plane_a16 = dw::Cfg<G>::kKGroups * sbo_a / 16u, plane_b16 = dw::Cfg<G>::kKGroups * sbo_b / 16u;
             bool ok = true;
             for (int j = 0; j < n_mine; ++j) {
                 const int sb = j % SB;
@@ -364,7 +369,7 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
                 const uint32_t a_lo = ptx::sdesc_mn_sw64_lo(a_addr, 512u);
                 const uint32_t b_lo = ptx::sdesc_mn_sw64_lo(a_addr + p.a_bytes, 512u);
 #pragma unroll
-                for (int ks = 0; ks < dw::kTok / 16; ++ks) {
+                for (int ks = 0; ks < dw::Cfg<G>::kTok / 16; ++ks) {
                     const uint32_t acc0 = (j > 0 || ks > 0) ? 1u : 0u;
                     // K step ks = tokens 16ks .. 16ks+15 = K groups 2ks, 2ks+1
                     auto A = [&](int pl) {
@@ -399,15 +404,15 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
         // keeps the dbias sums of its dy units in registers (bsum) until the end.
         constexpr int CPU = dw::Cfg<G>::kChanPerUnit;
         const int groups_dy = p.MO / CPU, groups_x = p.NI / CPU;
-        const int units_dy = dw::kTok * groups_dy;
-        const int n_units = units_dy + dw::kTok * groups_x;
+        const int units_dy = dw::Cfg<G>::kTok * groups_dy;
+        const int n_units = units_dy + dw::Cfg<G>::kTok * groups_x;
         float bsum[dw::Cfg<G>::kMaxPasses][CPU];
 #pragma unroll
         for (int ps = 0; ps < dw::Cfg<G>::kMaxPasses; ++ps)
 #pragma unroll
             for (int j = 0; j < CPU; ++j) bsum[ps][j] = 0.0f;
         const uint32_t sbo_a = static_cast<uint32_t>(p.MA) * 512u, sbo_b = static_cast<uint32_t>(p.NA) * 512u;
-        const uint32_t plane_a = 4u * sbo_a, plane_b = 4u * sbo_b;
+        const uint32_t plane_a = dw::Cfg<G>::kKGroups * sbo_a, plane_b = dw::Cfg<G>::kKGroups * sbo_b;
         // the thread's units are the same in every chunk: their source offsets in a raw
         // stage and destination offsets in a spectra buffer are computed once
         constexpr int MP = dw::Cfg<G>::kMaxPasses;
@@ -422,7 +427,7 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
                 const int v = is_dy ? u : u - units_dy, ng = is_dy ? groups_dy : groups_x;
                 const int tok = v / ng, c = CPU * (v - tok * ng), cpb = is_dy ? p.cpb_dy : p.cpb_x;
                 const int box = c / cpb, row_bytes = cpb * G * 2;
-                src_off[ps] = (is_dy ? 0u : p.dy_bytes) + static_cast<uint32_t>(box * (dw::kTok * row_bytes) +
+                src_off[ps] = (is_dy ? 0u : p.dy_bytes) + static_cast<uint32_t>(box * (dw::Cfg<G>::kTok * row_bytes) +
                                                                                  tok * row_bytes + (c - box * cpb) * G * 2);
                 dst_off[ps] = (is_dy ? 0u : p.a_bytes) + dw::unit_dst_offset(tok, c, is_dy ? sbo_a : sbo_b);
                 valid_mask |= 1u << ps;
@@ -484,7 +489,7 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
         }
         // dbias partial of this CTA (every CTA writes it; the inverse-DFT kernel reads input
         // tile 0's): each thread's register sums to their slots bias_sm[tok][c], then per
-        // channel the 32 token slots in order
+        // channel the kTok token slots in order
 #pragma unroll
         for (int ps = 0; ps < dw::Cfg<G>::kMaxPasses; ++ps) {
             const int u = t + ps * kDftThreads;
@@ -497,7 +502,7 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
         ptx::named_bar_sync(dw::kBarDft, kDftThreads);
         for (int c = t; c < p.MO; c += kDftThreads) {
             float acc = 0.0f;
-            for (int tok = 0; tok < dw::kTok; ++tok) acc += bias_sm[tok * p.MO + c];
+            for (int tok = 0; tok < dw::Cfg<G>::kTok; ++tok) acc += bias_sm[tok * p.MO + c];
             slab[p.slab_floats + c] = acc;
         }
     }
