@@ -46,6 +46,7 @@ from ._capi import (  # noqa: F401
     eqlin_forward,
     eqlin_forward_noalloc,
     eqlin_forward_host,
+    query_plan,
     eqlin_last_error,
     eqlin_prepare_weights,
     eqlin_status_string,

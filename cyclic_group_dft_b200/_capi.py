@@ -34,6 +34,7 @@ EQLIN_PREPARE_GELU = 2
 ATTRS = {
     "G": 0, "Cin": 1, "Cout": 2, "io_dtype": 3, "path": 4, "tokens_per_tile": 5,
     "stages": 6, "smem_bytes": 7, "max_grid": 8, "weight_bytes": 9, "activation": 10,
+    "y_staging": 11, "dw_tile_rows": 12, "dw_tile_cols": 13, "dw_raw_stages": 14, "dw_tokens": 15,
 }
 PATH_NAMES = {0: "tcgen05_tokens_on_n_resident_weights", 1: "tcgen05_tokens_on_n_streamed_weights",
               2: "fp32_fp64_arithmetic", 3: "tcgen05_tokens_on_m_resident_weights",
@@ -52,6 +53,7 @@ _vp, _i64, _int = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
 _lib.eqlin_prepare_weights.argtypes = [_vp, _vp, _i64, _i64, _i64, _int, _int, _vp, ctypes.POINTER(_vp)]
 _lib.eqlin_forward.argtypes = [_vp, _vp, _vp, _i64, _vp]
 _lib.eqlin_forward_host.argtypes = [_vp, _vp, _vp, _i64, _vp]
+_lib.eqlin_query_plan.argtypes = [_i64, _i64, _i64, _int, _int, ctypes.POINTER(_i64)]
 _lib.eqlin_destroy.argtypes = [_vp]
 _lib.eqlin_device_status.argtypes = [_vp, ctypes.POINTER(_int)]
 _lib.eqlin_get_attr.argtypes = [_vp, _int, ctypes.POINTER(_i64)]
@@ -68,7 +70,8 @@ _lib.eqlin_status_string.restype = ctypes.c_char_p
 _lib.eqlin_last_error.argtypes = []
 _lib.eqlin_last_error.restype = ctypes.c_char_p
 _lib.eqlin_version.argtypes = []
-for _f in ("eqlin_prepare_weights", "eqlin_forward", "eqlin_forward_host", "eqlin_destroy", "eqlin_device_status",
+for _f in ("eqlin_prepare_weights", "eqlin_forward", "eqlin_forward_host", "eqlin_query_plan", "eqlin_destroy",
+           "eqlin_device_status",
            "eqlin_get_attr", "eqlin_copy_freq_weights", "eqlin_check_shape", "eqlin_version",
            "eqlin_forward_noalloc", "eqlin_prepare_weights_ex", "eqlin_backward_dx",
            "eqlin_backward_dw_workspace_size", "eqlin_backward_dw"):
@@ -253,6 +256,21 @@ def eqlin_forward(h: Handle, x: torch.Tensor, y: torch.Tensor | None = None, str
         _check(_lib.eqlin_forward(h.ptr, x.data_ptr(), y.data_ptr(), N, _stream_ptr(stream)),
                "eqlin_forward")
     return y
+
+
+def query_plan(Cout: int, Cin: int, G: int, io_dtype=torch.bfloat16) -> dict:
+    """The kernel plan eqlin_prepare_weights would choose for these sizes on a B200 (host
+    only, no GPU): {attribute name: value} via eqlin_query_plan."""
+    io = _TORCH_TO_EQLIN[io_dtype]
+    out = {}
+    v = _i64()
+    for name, a in ATTRS.items():
+        if name == "activation":
+            continue
+        _check(_lib.eqlin_query_plan(Cout, Cin, G, io, a, ctypes.byref(v)), "eqlin_query_plan")
+        out[name] = v.value
+    out["path_name"] = PATH_NAMES.get(out["path"], str(out["path"]))
+    return out
 
 
 def eqlin_forward_host(h: Handle, x_host: torch.Tensor, y_host: torch.Tensor | None = None,

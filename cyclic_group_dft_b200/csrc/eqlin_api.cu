@@ -29,6 +29,7 @@ using eqlin::TmParams;
 namespace {
 
 constexpr size_t kB200SmemOptin = 232448;   // 227 KB opt-in shared memory per CTA on sm_100
+constexpr int kB200SmCount = 148;           // SMs of a B200 (host-only planning queries)
 constexpr size_t kSmemAlignSlack = 1024;    // the kernels round their smem base up to 1 KB
 constexpr size_t kSmemCtlBytes = 512;       // mbarriers + control block
 constexpr int kMaxStages = 12;
@@ -927,6 +928,36 @@ int launch_dw(const DwPlan& pl, bool f32_path, int64_t Cout, int64_t Cin, int64_
 
 }  // namespace
 
+namespace {
+// Attributes that follow from the plans alone (shared by eqlin_get_attr and
+// eqlin_query_plan); false when attr is not one of them.
+bool plan_attr(const Plan& pl, const DwPlan& dwp, int64_t G, int64_t Cin, int64_t Cout, int io_dtype, int attr,
+               int64_t* value) {
+    const bool tn = pl.path == kPathResident || pl.path == kPathStreamed || pl.path == kPathTnResidentX;
+    const bool has_dw = io_dtype != EQLIN_F32 && dwp.MO > 0;
+    switch (attr) {
+        case EQLIN_ATTR_G: *value = G; return true;
+        case EQLIN_ATTR_CIN: *value = Cin; return true;
+        case EQLIN_ATTR_COUT: *value = Cout; return true;
+        case EQLIN_ATTR_IO_DTYPE: *value = io_dtype; return true;
+        case EQLIN_ATTR_PATH: *value = pl.path; return true;
+        case EQLIN_ATTR_TOKENS_PER_TILE: *value = pl.BN; return true;
+        case EQLIN_ATTR_STAGES: *value = pl.stages; return true;
+        case EQLIN_ATTR_SMEM_BYTES: *value = static_cast<int64_t>(pl.smem_bytes); return true;
+        case EQLIN_ATTR_WEIGHT_BYTES:
+            *value = pl.path == kPathF32 ? static_cast<int64_t>(G * Cin * Cout * 8)
+                                         : static_cast<int64_t>(pl.img_alloc_bytes);
+            return true;
+        case EQLIN_ATTR_Y_STAGING: *value = tn ? pl.ybufs : -1; return true;
+        case EQLIN_ATTR_DW_TILE_ROWS: *value = has_dw ? dwp.MO : -1; return true;
+        case EQLIN_ATTR_DW_TILE_COLS: *value = has_dw ? dwp.NI : -1; return true;
+        case EQLIN_ATTR_DW_RAW_STAGES: *value = has_dw ? dwp.raw_stages : -1; return true;
+        case EQLIN_ATTR_DW_TOKENS: *value = has_dw ? dwp.tok : -1; return true;
+        default: return false;
+    }
+}
+}  // namespace
+
 struct eqlin_handle {
     int device = 0;
     int sm_count = 0;
@@ -1349,24 +1380,35 @@ int eqlin_device_status(eqlin_handle* h, int* status_out) {
 int eqlin_get_attr(const eqlin_handle* h, int attr, int64_t* value) {
     if (!h || !value) return fail(EQLIN_ERR_INVALID_ARG, "NULL argument");
     const Plan& pl = h->plan;
+    if (plan_attr(pl, h->dwp, h->G, h->Cin, h->Cout, h->io_dtype, attr, value)) return EQLIN_OK;
     switch (attr) {
         case EQLIN_ATTR_G: *value = h->G; break;
         case EQLIN_ATTR_CIN: *value = h->Cin; break;
         case EQLIN_ATTR_COUT: *value = h->Cout; break;
         case EQLIN_ATTR_IO_DTYPE: *value = h->io_dtype; break;
-        case EQLIN_ATTR_PATH: *value = pl.path; break;
-        case EQLIN_ATTR_TOKENS_PER_TILE: *value = pl.BN; break;
-        case EQLIN_ATTR_STAGES: *value = pl.stages; break;
-        case EQLIN_ATTR_SMEM_BYTES: *value = static_cast<int64_t>(pl.smem_bytes); break;
         case EQLIN_ATTR_MAX_GRID: *value = pl.path == kPathF32 ? -1 : h->sm_count; break;
-        case EQLIN_ATTR_WEIGHT_BYTES:
-            *value = pl.path == kPathF32 ? static_cast<int64_t>(h->G * h->Cin * h->Cout * 8)
-                                         : static_cast<int64_t>(pl.img_alloc_bytes);
-            break;
         case EQLIN_ATTR_ACTIVATION: *value = h->buf.act; break;
         default: return fail(EQLIN_ERR_INVALID_ARG, "unknown attribute");
     }
     return EQLIN_OK;
+}
+
+int eqlin_query_plan(int64_t Cout, int64_t Cin, int64_t G, int io_dtype, int attr, int64_t* value) {
+    if (!value) return fail(EQLIN_ERR_INVALID_ARG, "NULL argument");
+    int s = check_shape_impl(Cout, Cin, G, io_dtype, io_dtype);
+    if (s != EQLIN_OK) return s;
+    Plan pl;
+    if ((s = plan_for(Cout, Cin, G, io_dtype, kB200SmemOptin, &pl)) != EQLIN_OK) return s;
+    DwPlan dwp;
+    if (io_dtype != EQLIN_F32 &&
+        plan_dw(Cout, Cin, static_cast<int>(G), kB200SmemOptin, kB200SmCount, &dwp) != EQLIN_OK)
+        dwp = DwPlan();
+    if (attr == EQLIN_ATTR_MAX_GRID) {
+        *value = pl.path == kPathF32 ? -1 : kB200SmCount;
+        return EQLIN_OK;
+    }
+    if (plan_attr(pl, dwp, G, Cin, Cout, io_dtype, attr, value)) return EQLIN_OK;
+    return fail(EQLIN_ERR_INVALID_ARG, "unknown attribute");
 }
 
 int eqlin_copy_freq_weights(const eqlin_handle* h, float* dst, int64_t count) {

@@ -172,15 +172,33 @@ enum {
                                        weights resident / streamed; 2 fp32 I/O (float64 arithmetic);
                                        3/4 tcgen05 with tokens on the MMA M dimension, resident / streamed;
                                        5 tcgen05 with tokens on N and the input spectrum resident
-                                       across output chunks (Cout > 128), weights streamed */
+                                       across output chunks (Cout > 128 and at least 4 chunks
+                                       of 32 input channels), weights streamed */
     EQLIN_ATTR_TOKENS_PER_TILE = 5, /* tokens per work item of the fused kernel */
     EQLIN_ATTR_STAGES = 6,          /* depth of the shared-memory ring */
     EQLIN_ATTR_SMEM_BYTES = 7,      /* dynamic shared memory per CTA */
     EQLIN_ATTR_MAX_GRID = 8,        /* CTAs launched for a large N (one per SM) */
     EQLIN_ATTR_WEIGHT_BYTES = 9,    /* bytes of the frequency-domain weights the kernel reads */
-    EQLIN_ATTR_ACTIVATION = 10      /* epilogue activation of the forward: 0 none, 1 GELU */
+    EQLIN_ATTR_ACTIVATION = 10,     /* epilogue activation of the forward: 0 none, 1 GELU */
+    EQLIN_ATTR_Y_STAGING = 11,      /* tokens-on-N kernels: y staging buffers per epilogue warp
+                                       (1 or 2, TMA stores), 0 = direct stores from registers;
+                                       -1 for the other kernels */
+    EQLIN_ATTR_DW_TILE_ROWS = 12,   /* weight gradient (16-bit I/O): output rows of a unit */
+    EQLIN_ATTR_DW_TILE_COLS = 13,   /* weight gradient: input columns of a unit */
+    EQLIN_ATTR_DW_RAW_STAGES = 14,  /* weight gradient: depth of the raw dy / x ring */
+    EQLIN_ATTR_DW_TOKENS = 15       /* weight gradient: tokens per chunk */
 };
 EQLIN_API int eqlin_get_attr(const eqlin_handle* h, int attr, int64_t* value);
+
+/*
+ * eqlin_query_plan -- the same properties (EQLIN_ATTR_PATH .. EQLIN_ATTR_DW_TOKENS,
+ * except ACTIVATION) that eqlin_prepare_weights would give a handle of these sizes,
+ * planned on the host for a B200 (227 KB of shared memory per CTA, 148 SMs) under the
+ * current environment overrides.  Host only: no GPU, no allocation.  The weight-gradient
+ * attributes are -1 where no tiling fits (or for fp32 I/O).
+ * Errors: INVALID_ARG / UNSUPPORTED as eqlin_check_shape, INVALID_ARG for an unknown attr.
+ */
+EQLIN_API int eqlin_query_plan(int64_t Cout, int64_t Cin, int64_t G, int io_dtype, int attr, int64_t* value);
 
 /*
  * eqlin_copy_freq_weights -- copy the fp32 frequency-domain weights to host

@@ -150,3 +150,64 @@ def test_gelu_flag_is_declared_and_accepted_on_host():
                                       eq.EQLIN_PREPARE_BACKWARD | eq.EQLIN_PREPARE_GELU, None,
                                       ctypes.byref(h))
     assert st == eq.EQLIN_ERR_INVALID_ARG and "NULL" in eq.eqlin_last_error()
+
+
+# ---------------------------------------------------------------- planner (host only)
+@pytest.mark.parametrize("Cout,Cin,G,path,ystore", [
+    (96, 96, 4, "tcgen05_tokens_on_n_resident_weights", "tma"),      # headline: staged TMA stores
+    (96, 96, 2, "tcgen05_tokens_on_n_resident_weights", "tma"),
+    (384, 96, 4, "tcgen05_tokens_on_n_streamed_weights", "tma"),     # 3 input chunks: no resident input
+    (512, 128, 4, "tcgen05_tokens_on_n_resident_input", "tma"),      # from 4 input chunks on
+    (768, 192, 4, "tcgen05_tokens_on_n_resident_input", "direct"),   # direct stores deepen the ring
+    (96, 384, 4, "tcgen05_tokens_on_n_streamed_weights", "direct"),  # 12 input chunks: direct stores
+    (64, 224, 4, "tcgen05_tokens_on_n_resident_weights", "tma"),     # 7 input chunks: staged
+    (64, 256, 4, "tcgen05_tokens_on_n_resident_weights", "direct"),  # 8 input chunks: direct
+    (64, 64, 8, "tcgen05_tokens_on_m_resident_weights", "none"),
+    (32, 32, 16, "tcgen05_tokens_on_m_resident_weights", "none"),
+])
+def test_planner_kernel_choice(Cout, Cin, G, path, ystore):
+    """The kernel form and store mode the planner picks, from the measured rules."""
+    q = eq.query_plan(Cout, Cin, G)
+    assert q["path_name"] == path
+    mode = {-1: "none", 0: "direct"}.get(q["y_staging"], "tma")
+    assert mode == ystore, q
+
+
+def test_planner_fits_shared_memory_and_tiles():
+    for shape in [(96, 96, 4), (768, 192, 4), (64, 64, 8), (32, 32, 16), (1024, 1024, 4), (1, 1, 8), (8, 16, 2)]:
+        for io in (torch.bfloat16, torch.float16):
+            q = eq.query_plan(*shape, io_dtype=io)
+            assert 0 < q["smem_bytes"] <= 232448
+            assert q["stages"] >= 2 and q["tokens_per_tile"] in (16, 32, 64, 128)
+            assert q["max_grid"] == 148
+
+
+@pytest.mark.parametrize("G,tokens", [(2, 32), (4, 32), (8, 16), (16, 16)])
+def test_planner_weight_gradient_chunks(G, tokens):
+    """Weight-gradient chunks: 32 tokens up to G = 4, 16 from G = 8 on (a deeper raw ring)."""
+    q = eq.query_plan(32, 32, G)
+    assert q["dw_tokens"] == tokens
+    assert q["dw_raw_stages"] >= 2
+    assert q["dw_tile_rows"] % 16 == 0 and q["dw_tile_cols"] % 16 == 0
+
+
+def test_planner_environment_overrides(monkeypatch):
+    monkeypatch.setenv("EQLIN_KERNEL", "tm")
+    assert "tokens_on_m" in eq.query_plan(96, 96, 4)["path_name"]
+    monkeypatch.setenv("EQLIN_KERNEL", "tn")
+    assert eq.query_plan(768, 192, 4)["path_name"] == "tcgen05_tokens_on_n_streamed_weights"
+    monkeypatch.delenv("EQLIN_KERNEL")
+    monkeypatch.setenv("EQLIN_YSTORE", "direct")
+    assert eq.query_plan(96, 96, 4)["y_staging"] == 0
+    monkeypatch.setenv("EQLIN_YSTORE", "tma")
+    assert eq.query_plan(768, 192, 4)["y_staging"] in (1, 2)
+
+
+def test_planner_query_errors():
+    lib = eq.library()
+    v = ctypes.c_int64()
+    assert lib.eqlin_query_plan(96, 96, 3, eq.EQLIN_BF16, 4, ctypes.byref(v)) == eq.EQLIN_ERR_UNSUPPORTED
+    assert lib.eqlin_query_plan(96, 96, 4, eq.EQLIN_BF16, 999, ctypes.byref(v)) == eq.EQLIN_ERR_INVALID_ARG
+    assert lib.eqlin_query_plan(96, 96, 4, eq.EQLIN_BF16, 4, None) == eq.EQLIN_ERR_INVALID_ARG
+    q = eq.query_plan(16, 16, 4, io_dtype=torch.float32)
+    assert q["path_name"] == "fp32_fp64_arithmetic" and q["dw_tokens"] == -1
