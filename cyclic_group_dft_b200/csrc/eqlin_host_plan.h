@@ -395,8 +395,8 @@ size_t dw_smem(int MO, int NI, int G, int RS, int SB, DwPlan* out) {
 // pipeline (2 raw stages, 1 spectra buffer); fewer units = fewer re-reads of x and dy.
 // Ties go to the larger MO (less MMA padding), then the larger NI.  Then the deepest
 // raw ring that fits: with two spectra buffers (the transform of one chunk overlaps the
-// MMAs of the previous one) when that still leaves >= 2 raw stages, else with one.  Tuning overrides: EQLIN_DW_TILE ("MO,NI"), EQLIN_DW_SPEC_BUFS,
-// EQLIN_DW_RAW_STAGES.
+// MMAs of the previous one) when that still leaves >= 2 raw stages, else with one.
+// Tuning overrides: EQLIN_DW_TILE ("MO,NI"), EQLIN_DW_SPEC_BUFS, EQLIN_DW_RAW_STAGES.
 int plan_dw(int64_t Cout, int64_t Cin, int G, size_t max_smem, int sm_count, DwPlan* pl) {
     const int mo_max = std::min(eqlin::kMmaM, round16(Cout));
     const int ni_cap = std::min(256, (512 / G) / 16 * 16);
