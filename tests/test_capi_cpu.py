@@ -211,3 +211,26 @@ def test_planner_query_errors():
     assert lib.eqlin_query_plan(96, 96, 4, eq.EQLIN_BF16, 4, None) == eq.EQLIN_ERR_INVALID_ARG
     q = eq.query_plan(16, 16, 4, io_dtype=torch.float32)
     assert q["path_name"] == "fp32_fp64_arithmetic" and q["dw_tokens"] == -1
+
+
+def test_planner_over_random_shapes():
+    """Every accepted 16-bit shape gets a plan inside the 227 KB opt-in shared memory with at
+    least two ring stages, a tile the kernels support, and a weight-gradient tiling."""
+    import random
+    rnd = random.Random(7)
+    lib = eq.library()
+    checked = 0
+    for _ in range(300):
+        G = rnd.choice([2, 4, 8, 16])
+        step = max(1, 8 // G)                  # 16-byte rows: C*G a multiple of 8
+        Cout = step * rnd.randint(1, 1024 // step)
+        Cin = step * rnd.randint(1, 1024 // step)
+        io = rnd.choice([torch.bfloat16, torch.float16])
+        if lib.eqlin_check_shape(Cout, Cin, G, eq.EQLIN_BF16, eq.EQLIN_BF16) != eq.EQLIN_OK:
+            continue
+        q = eq.query_plan(Cout, Cin, G, io_dtype=io)
+        assert 0 < q["smem_bytes"] <= 232448, (Cout, Cin, G, q)
+        assert q["stages"] >= 1 and q["tokens_per_tile"] in (16, 32, 64, 128), (Cout, Cin, G, q)
+        assert q["dw_tile_rows"] > 0 and q["dw_tile_cols"] > 0 and q["dw_raw_stages"] >= 2, (Cout, Cin, G, q)
+        checked += 1
+    assert checked > 250
