@@ -186,11 +186,14 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ CPU oracle
-def oracle_rate(wl: workloads.Workload, target_s: float, seed: int = 0, cap_tokens: int | None = None):
-    """Time the float64 oracle on a token prefix sized for ~target_s seconds.
+def oracle_rate(wl: workloads.Workload, target_s: float, seed: int = 0, cap_tokens: int | None = None,
+                threads: int | None = None):
+    """Time the float64 oracle on a token prefix sized for ~target_s seconds, on `threads`
+    host threads (default: every core this process may run on).
     Returns (tokens/s, tokens, seconds, threads)."""
     import oracle
-    threads = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    if threads is None:
+        threads = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
     x, w, bias = workloads.make_inputs(wl, seed=seed, N=64)
     xf, wf = x.double().numpy(), w.double().numpy()
     bf = None if bias is None else bias.double().numpy()
@@ -464,8 +467,11 @@ def main() -> None:
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, n_s, dt, threads = oracle_rate(wl, args.cpu_seconds)
+        rate1, n1, dt1, _ = oracle_rate(wl, min(args.cpu_seconds, 5.0), threads=1)
         cpu = {"value": rate, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-               "sample": f"{n_s} of {wl.N} tokens of {wl.name} in {dt:.1f} s (float64 definition loops, OpenMP over tokens)"}
+               "sample": f"{n_s} of {wl.N} tokens of {wl.name} in {dt:.1f} s (float64 definition loops, OpenMP over tokens)",
+               "single_core": {"value": rate1, "unit": "tokens/s", "cores": 1,
+                               "sample": f"{n1} of {wl.N} tokens in {dt1:.1f} s"}}
 
     if world > 1:
         torch.distributed.barrier()

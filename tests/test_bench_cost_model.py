@@ -51,3 +51,12 @@ def test_fourier_share_of_the_dense_count():
     for name, ratio in (("p4_c96_bf16", 6 / 16), ("p8_c64_bf16", 14 / 64), ("c16_c32_bf16", 30 / 256)):
         wl = workloads.WORKLOADS[name]
         assert b.fourier_flops(wl, wl.N) / b.dense_equivalent_flops(wl, wl.N) == pytest.approx(ratio, rel=1e-12)
+
+
+def test_oracle_rate_reports_its_threads():
+    """The CPU baseline's timing helper: a bounded sample, on the threads asked for."""
+    b = _bench()
+    from cyclic_group_dft_b200 import workloads
+    wl = workloads.WORKLOADS["tiny_p4_fp32"]
+    rate, n, dt, threads = b.oracle_rate(wl, 0.05, threads=1)
+    assert threads == 1 and 64 <= n <= wl.N and rate > 0 and dt > 0
