@@ -3,19 +3,27 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl eqlin|reference]
 
-One step = one eqlin_forward over the whole workload batch (weights prepared
-once, outside the timed region; inputs already resident in HBM).  Prints ONE
-JSON line (rank 0): tokens/s over all ranks, ms per step, the roofline of the
-fused kernel (algorithmic bytes / HBM peak, Fourier FLOPs / bf16 tensor peak),
-clocks sampled during the timed region, an end-to-end figure through the host
-buffer API, and the CPU float64 oracle's throughput on a bounded sample.
+One step = one eqlin_forward over the whole batch of the headline workload (p4,
+Cin = Cout = 96, N = 64*56*56 tokens, bf16 I/O): weights prepared once, outside the
+timed region; inputs already resident in HBM.  Prints ONE JSON line (rank 0):
+tokens/s over all ranks, ms per step, the roofline of the fused kernel (algorithmic
+bytes / HBM peak, Fourier FLOPs / bf16 tensor peak), clocks sampled during the timed
+region, an end-to-end figure through the host-buffer API, and the CPU float64
+oracle's throughput on a bounded sample.
+
+The same line carries a ``workloads`` object with every synthetic workload
+(tiny p4 fp32, p4 C96, p8 C64, p4 MLP 192->768, C16 C32), each measured in this run
+the same way: us per launch over back-to-back launches, tokens/s, roofline,
+dense-equivalent TFLOP/s, the backward calls, and the oracle on a bounded sample of
+that workload.  The other workloads run first, the headline last.
 
 Multi-GPU (torchrun): every rank runs the full workload on its own GPU (tokens
 are independent, no collective on the data path): weak scaling; the timed
 region is bracketed by barriers and the slowest rank's time is used.
 
 --impl reference times the float64 CPU oracle on the host cores instead (the
-method's plain definition), on bounded token samples of the same workload.
+method's plain definition), on bounded token samples of the same workload.  That
+arm never loads the CUDA library.
 """
 from __future__ import annotations
 
@@ -34,16 +42,20 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+# the package loads libeqlin.so lazily: importing the input generators maps no CUDA code
 from cyclic_group_dft_b200 import workloads  # noqa: E402
 
 METRIC = "EQ-Linear tokens/s and % of roofline (HBM vs bf16 TC), p4 Cin=Cout=96"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_BYTES = 126 * 1024 * 1024
+# the synthetic workloads of the method's configurations, measured in every run
+BENCH_WORKLOADS = ("tiny_p4_fp32", "p4_c96_bf16", "p8_c64_bf16", "p4_mlp_bf16", "c16_c32_bf16")
 # device code of each fused kernel: a recorded ncu traffic figure is reported only
 # while these files are unchanged since the capture
 KERNEL_SOURCES = {
     "eqlin_fwd_tc": ["eqlin_fwd_tc.cuh", "group_dft.cuh", "io16.cuh", "sm100_ptx.cuh", "eqlin_layout.h"],
-    "eqlin_fwd_tm": ["eqlin_fwd_tm.cuh", "group_dft.cuh", "io16.cuh", "sm100_ptx.cuh", "eqlin_layout.h"],
+    "eqlin_fwd_tm": ["eqlin_fwd_tm.cuh", "eqlin_fwd_tc.cuh", "group_dft.cuh", "io16.cuh", "sm100_ptx.cuh",
+                     "eqlin_layout.h"],
     "eqlin_fwd_tcr": ["eqlin_fwd_tcr.cuh", "eqlin_fwd_tc.cuh", "group_dft.cuh", "io16.cuh", "sm100_ptx.cuh",
                       "eqlin_layout.h"],
 }
@@ -103,8 +115,11 @@ def kernel_source_hash(kernel: str) -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str):
-    """DRAM bytes per launch from a committed ncu capture, if the kernel is unchanged since."""
+def recorded_traffic(workload: str) -> dict | None:
+    """DRAM reads plus L2 write bytes per launch from a committed ncu capture, if the
+    kernel is unchanged since.  Reads are counted at DRAM; writes are counted as they
+    enter L2 (every byte of y the kernel stores), because part of y is still dirty in
+    L2 when the kernel ends and its DRAM write-back falls outside the kernel."""
     try:
         with open(TRAFFIC_FILE) as f:
             d = json.load(f)
@@ -115,7 +130,27 @@ def recorded_traffic(workload: str):
         return None
     if entry.get("source_hash") != kernel_source_hash(entry["kernel"]):
         return None
-    return entry.get("dram_bytes_per_launch")
+    if "dram_read_bytes_per_launch" not in entry or "l2_write_bytes_per_launch" not in entry:
+        return None
+    return {"bytes": entry["dram_read_bytes_per_launch"] + entry["l2_write_bytes_per_launch"],
+            "dram_read": entry["dram_read_bytes_per_launch"], "l2_write": entry["l2_write_bytes_per_launch"],
+            "kernel": entry["kernel"]}
+
+
+def rotating_sets(wl: workloads.Workload, N: int) -> tuple[int, int]:
+    """(bytes of one x/y set, number of sets): enough sets that consecutive launches
+    never find their inputs in L2."""
+    set_bytes = N * (wl.Cin + wl.Cout) * wl.G * wl.elem_bytes
+    return set_bytes, max(2, math.ceil(2 * L2_BYTES / set_bytes))
+
+
+def line_config(wl: workloads.Workload, world: int) -> dict:
+    """The `config` of the JSON line: the workload and how it is run, identical in the
+    GPU and the reference arm (kernel details are reported apart, under `kernel`)."""
+    set_bytes, n_sets = rotating_sets(wl, wl.N)
+    return {"workload": wl.name, "N": wl.N, "Cin": wl.Cin, "Cout": wl.Cout, "G": wl.G, "io": wl.io_dtype,
+            "global_batch": world * wl.N, "parallelism": f"replicas{world}" if world > 1 else "single",
+            "l2": f"inputs larger than L2; {n_sets} rotating x/y sets of {set_bytes / 1e6:.0f} MB"}
 
 
 # ------------------------------------------------------------------ clocks
@@ -210,6 +245,18 @@ def oracle_rate(wl: workloads.Workload, target_s: float, seed: int = 0, cap_toke
     return n / dt, n, dt, threads
 
 
+def cpu_baseline(wl: workloads.Workload, seconds: float, single_core_seconds: float = 0.0) -> dict:
+    rate, n_s, dt, threads = oracle_rate(wl, seconds)
+    out = {"value": rate, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+           "sample": f"{n_s} of {wl.N} tokens of {wl.name} in {dt:.1f} s (float64 definition loops, "
+                     f"OpenMP over tokens)"}
+    if single_core_seconds > 0:
+        rate1, n1, dt1, _ = oracle_rate(wl, single_core_seconds, threads=1)
+        out["single_core"] = {"value": rate1, "unit": "tokens/s", "cores": 1,
+                              "sample": f"{n1} of {wl.N} tokens in {dt1:.1f} s"}
+    return out
+
+
 # ------------------------------------------------------------------ helpers
 def reduce_max(value: float, device) -> float:
     """Max of `value` over all ranks (identity without a process group).  Every rank
@@ -239,6 +286,40 @@ def emit(d: dict) -> None:
     print(json.dumps(d), flush=True)
 
 
+def roofline(wl: workloads.Workload, N: int, avg_launch_s: float, peaks: dict, peak_kind: str) -> dict:
+    """Roofline of one launch: algorithmic bytes and Fourier FLOPs against the measured
+    HBM copy peak and bf16 tensor peak; the bound is the slower of the two."""
+    bytes_launch = algorithmic_bytes(wl, N)
+    flops_launch = fourier_flops(wl, N)
+    gbs = bytes_launch / avg_launch_s / 1e9
+    tflops = flops_launch / avg_launch_s / 1e12
+    t_hbm = bytes_launch / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops_launch / (peaks["bf16_tflops"] * 1e12)
+    if t_hbm >= t_tc:
+        roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": gbs / peaks["hbm_gbs"]}
+    else:
+        roof = {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": tflops / peaks["bf16_tflops"]}
+    tr = recorded_traffic(wl.name) if N == wl.N else None
+    roof["traffic"] = None if tr is None else tr["bytes"]
+    if tr is not None:
+        roof["traffic_detail"] = {"dram_read": tr["dram_read"], "l2_write": tr["l2_write"],
+                                  "over_algorithmic": tr["bytes"] / bytes_launch, "kernel": tr["kernel"],
+                                  "source": "ncu capture (profiles/eqlin_fwd_traffic.json): dram__bytes_read.sum "
+                                            "+ 32 * lts__t_sectors_op_write.sum, scaled to a full launch"}
+    roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback"
+    roof["roofline_time_us"] = 1e6 * max(t_hbm, t_tc)
+    roof["kernel_us"] = 1e6 * avg_launch_s
+    roof["frac_of_roofline_time"] = max(t_hbm, t_tc) / avg_launch_s
+    roof["bytes_per_launch"] = bytes_launch
+    roof["fourier_flops_per_launch"] = flops_launch
+    roof["tensor_tflops"] = tflops
+    roof["tensor_frac"] = tflops / peaks["bf16_tflops"]                       # burst peak: the headline
+    roof["tensor_frac_sustained"] = tflops / peaks["bf16_tflops_sustained"]   # seconds-long GEMM peak
+    return roof
+
+
 def run_reference(args, wl) -> None:
     world, rank, _ = dist_info()
     if rank != 0:
@@ -258,103 +339,96 @@ def run_reference(args, wl) -> None:
         oracle.forward(xf, wf, bf, threads=threads)
     dt = time.perf_counter() - t0
     value = args.steps * n / dt
-    sample = f"{n} of {wl.N} tokens per step (tokens are independent; rate scales linearly)"
+    sample = (f"{n} of {wl.N} tokens of {wl.name} per step (tokens are independent: the whole batch takes "
+              f"N / {n} times as long)")
     emit({
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * dt / args.steps * wl.N / n, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "N": wl.N, "Cin": wl.Cin, "Cout": wl.Cout, "G": wl.G,
-                   "io": wl.io_dtype},
+        "config": line_config(wl, args.gpus),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     })
 
 
-def main() -> None:
-    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default=workloads.HEADLINE, choices=sorted(workloads.WORKLOADS))
-    ap.add_argument("--impl", default="eqlin", choices=["eqlin", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=20)
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-mlp-block", action="store_true",
-                    help="skip the extra measurement of the equivariant MLP block L2(GELU(L1(x))), H = 4 C")
-    ap.add_argument("--no-backward", action="store_true",
-                    help="skip the extra measurement of the backward calls (input and weight gradients)")
-    ap.add_argument("--tokens", type=int, default=None,
-                    help="override the workload's token count (profiling a smaller case)")
-    args = ap.parse_args()
-    args.warmup = max(args.warmup, 3)
-    wl = workloads.WORKLOADS[args.workload]
-    if args.tokens is not None:
-        wl = wl.with_n(args.tokens)
+# ------------------------------------------------------------------ GPU arm
+class Ctx:
+    def __init__(self, eq, dev, world, stream, peaks, peak_kind):
+        self.eq, self.dev, self.world, self.stream = eq, dev, world, stream
+        self.peaks, self.peak_kind = peaks, peak_kind
 
-    if args.impl == "reference":
-        run_reference(args, wl)
-        return
-
-    import cyclic_group_dft_b200 as eq
-
-    world, rank, local = dist_info()
-    if world > 1:
-        import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local))
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-
-    x_cpu, w, bias = workloads.make_inputs(wl)
-    h = eq.prepare(w.to(dev), None if bias is None else bias.to(dev), io_dtype=wl.torch_dtype,
-                   backward=not args.no_backward)
-    N = wl.N
-    set_bytes = N * (wl.Cin + wl.Cout) * wl.G * wl.elem_bytes
-    n_sets = max(2, math.ceil(2 * L2_BYTES / set_bytes))
-    xs = [x_cpu.to(dev) for _ in range(n_sets)]
-    ys = [torch.empty(N, wl.Cout, wl.G, dtype=wl.torch_dtype, device=dev) for _ in range(n_sets)]
-    stream = torch.cuda.current_stream(dev)
-
-    def barrier():
-        if world > 1:
+    def barrier(self):
+        if self.world > 1:
             torch.distributed.barrier()
 
-    for i in range(args.warmup):
+
+def time_back_to_back(ctx: Ctx, fn, K: int, clocks: ClockSampler | None = None) -> float:
+    """Elapsed ms (max over ranks) of K calls of fn(i) between two events on the
+    launching stream, with no event between the calls."""
+    ctx.barrier()
+    torch.cuda.synchronize(ctx.dev)
+    if clocks is not None:
+        clocks.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(ctx.stream)
+    for i in range(K):
+        fn(i)
+    t1.record(ctx.stream)
+    torch.cuda.synchronize(ctx.dev)
+    if clocks is not None:
+        clocks.stop()
+    ctx.barrier()
+    return reduce_max(t0.elapsed_time(t1), ctx.dev)
+
+
+def measure_workload(ctx: Ctx, wl: workloads.Workload, K: int, warmup: int, headline: bool, args) -> dict:
+    """One workload: K back-to-back forward launches (timed), a per-launch pass, the
+    backward calls, and (headline only) the end-to-end host-buffer figure, the MLP
+    block and the clocks of the timed region."""
+    eq, dev, stream = ctx.eq, ctx.dev, ctx.stream
+    x_cpu, w, bias = workloads.make_inputs(wl)
+    backward = not args.no_backward
+    h = eq.prepare(w.to(dev), None if bias is None else bias.to(dev), io_dtype=wl.torch_dtype, backward=backward)
+    N = wl.N
+    _, n_sets = rotating_sets(wl, N)
+    xs = [x_cpu.to(dev) for _ in range(n_sets)]
+    ys = [torch.empty(N, wl.Cout, wl.G, dtype=wl.torch_dtype, device=dev) for _ in range(n_sets)]
+
+    def fwd(i):
         h.forward(xs[i % n_sets], out=ys[i % n_sets], stream=stream)
+
+    for i in range(warmup):
+        fwd(i)
     torch.cuda.synchronize(dev)
     if h.device_status() != eq.EQLIN_OK:
-        raise RuntimeError("device status not OK after warm-up")
+        raise RuntimeError(f"{wl.name}: device status not OK after warm-up")
 
-    # ----------------------------------------------------------- timed region
+    # ------------------------------------------------------- timed region
     # K back-to-back steps, one fused launch each, bracketed by two events on the
     # launching stream.  No event sits between the launches: an event there would end
     # the overlap of one launch's tail with the next one's prologue (programmatic
     # dependent launch), which is how the kernel runs in a real stream of layers.
     # The average launch duration of the kernel is therefore elapsed / K.
-    K = args.steps
-    clocks = ClockSampler(dev.index)
-    barrier()
-    torch.cuda.synchronize(dev)
-    clocks.start()
-    t_begin = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    t_begin.record(stream)
-    for i in range(K):
-        h.forward(xs[i % n_sets], out=ys[i % n_sets], stream=stream)
-    t_end.record(stream)
-    torch.cuda.synchronize(dev)
-    clocks.stop()
-    barrier()
-    elapsed_ms = t_begin.elapsed_time(t_end)
+    clocks = ClockSampler(dev.index) if headline else None
+    elapsed_ms = time_back_to_back(ctx, fwd, K, clocks)
     status = h.device_status()
-
-    elapsed_ms = reduce_max(elapsed_ms, dev)
-    value = aggregate_tokens_per_s(world, K, N, elapsed_ms)
     avg_launch_s = elapsed_ms / K / 1e3
+    out = {"N": N, "Cin": wl.Cin, "Cout": wl.Cout, "G": wl.G, "io": wl.io_dtype,
+           "kernel": {"path": h.path, "stages": h.attr("stages"), "tokens_per_tile": h.attr("tokens_per_tile")},
+           "steps": K, "elapsed_ms": elapsed_ms, "us_per_launch": 1e3 * elapsed_ms / K,
+           "tokens_per_s": aggregate_tokens_per_s(ctx.world, K, N, elapsed_ms),
+           "roofline": roofline(wl, N, avg_launch_s, ctx.peaks, ctx.peak_kind),
+           "dense_equivalent_tflops": dense_equivalent_flops(wl, N) / avg_launch_s / 1e12,
+           "device_status": status}
+    if algorithmic_bytes(wl, N) / (ctx.peaks["hbm_gbs"] * 1e9) < 2e-6:
+        out["roofline"]["note"] = ("launch-bound: the roofline time is below the ~2 us cost of one kernel "
+                                   "launch, so the fraction measures launch latency, not the kernel's "
+                                   "arithmetic or memory traffic")
+    if clocks is not None:
+        out["clocks"] = clocks.summary()
 
     # Launch-duration distribution, outside the timed region: an event pair around
     # each launch (which serialises the launches, so each one also pays its own
@@ -364,42 +438,34 @@ def main() -> None:
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(KL)]
     for i in range(KL):
         starts[i].record(stream)
-        h.forward(xs[i % n_sets], out=ys[i % n_sets], stream=stream)
+        fwd(i)
         ends[i].record(stream)
     torch.cuda.synchronize(dev)
     launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    out["launch_us"] = {"mean": 1e3 * statistics.mean(launch_ms), "median": 1e3 * statistics.median(launch_ms),
+                        "min": 1e3 * min(launch_ms), "max": 1e3 * max(launch_ms), "launches": len(launch_ms),
+                        "note": "each launch bracketed by its own events (serialised), outside the timed region"}
 
-    # ----------------------------------------------------------- end to end
-    E = args.e2e_steps
-    e2e = None
-    if E > 0:
+    # ------------------------------------------------------- end to end (headline)
+    if headline and args.e2e_steps > 0:
+        E = args.e2e_steps
         x_pin = x_cpu.pin_memory()
         y_pin = torch.empty(N, wl.Cout, wl.G, dtype=wl.torch_dtype).pin_memory()
         h.forward_host(x_pin, y_pin)  # warm the path
-        barrier()
-        torch.cuda.synchronize(dev)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(E):
-            h.forward_host(x_pin, y_pin, stream=stream)
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        barrier()
-        e2e_ms = reduce_max(e0.elapsed_time(e1), dev)
-        e2e = {"value": aggregate_tokens_per_s(world, E, N, e2e_ms), "unit": "tokens/s", "steps": E,
-               "h2d_bytes_per_step": x_pin.numel() * x_pin.element_size(),
-               "d2h_bytes_per_step": y_pin.numel() * y_pin.element_size(),
-               "api": "eqlin_forward_host (C ABI: pinned host x and y, chunked copies in and out "
-                      "overlapping the fused kernel on two streams)"}
+        e2e_ms = time_back_to_back(ctx, lambda i: h.forward_host(x_pin, y_pin, stream=stream), E)
+        out["e2e"] = {"value": aggregate_tokens_per_s(ctx.world, E, N, e2e_ms), "unit": "tokens/s", "steps": E,
+                      "h2d_bytes_per_step": x_pin.numel() * x_pin.element_size(),
+                      "d2h_bytes_per_step": y_pin.numel() * y_pin.element_size(),
+                      "api": "eqlin_forward_host (C ABI: pinned host x and y, chunked copies in and out "
+                             "overlapping the fused kernel on two streams)"}
+        del x_pin, y_pin
 
-    # ----------------------------------------------------------- backward calls
-    # Measured after the forward's timed region, on the same rotating buffer sets
-    # (the forward outputs stand in for dy): us per call from CUDA events around
-    # Kb back-to-back calls, against the same roofline model as the forward.
-    bwd = None
-    if not args.no_backward:
-        Kb = max(10, min(K, 200))
+    # ------------------------------------------------------- backward calls
+    # Measured after the forward's timed region, on the same rotating buffer sets (the
+    # forward outputs stand in for dy): us per call from CUDA events around Kb
+    # back-to-back calls, against the same roofline model as the forward.
+    if backward:
+        Kb = max(10, min(max(K, 100), 200))
         dxs = [torch.empty(N, wl.Cin, wl.G, dtype=wl.torch_dtype, device=dev) for _ in range(n_sets)]
         dw_t = torch.empty(wl.Cout, wl.Cin, wl.G, dtype=torch.float32, device=dev)
         db_t = torch.empty(wl.Cout, dtype=torch.float32, device=dev)
@@ -410,68 +476,132 @@ def main() -> None:
                                                  dw=dw_t, dbias=db_t, workspace=ws_t),
         }
         bwd = {}
+        bb = backward_bytes(wl, N)
+        t_tc = fourier_flops(wl, N) / (ctx.peaks["bf16_tflops"] * 1e12)
         for key, fn in calls.items():
-            for i in range(max(3, args.warmup)):
+            for i in range(max(3, warmup)):
                 fn(i)
-            barrier()
-            torch.cuda.synchronize(dev)
-            b0 = torch.cuda.Event(enable_timing=True)
-            b1 = torch.cuda.Event(enable_timing=True)
-            b0.record(stream)
-            for i in range(Kb):
-                fn(i)
-            b1.record(stream)
-            torch.cuda.synchronize(dev)
-            barrier()
-            bwd[key] = {"us_per_call": 1e3 * reduce_max(b0.elapsed_time(b1), dev) / Kb, "calls": Kb}
+            ms = time_back_to_back(ctx, fn, Kb)
+            t = ms / Kb * 1e-3
+            t_h = bb[key] / (ctx.peaks["hbm_gbs"] * 1e9)
+            t_roof = max(t_h, t_tc)
+            bwd[key] = {"us_per_call": 1e6 * t, "calls": Kb, "bytes": bb[key], "roofline_time_us": 1e6 * t_roof,
+                        "bound": "hbm" if t_h >= t_tc else "tensor", "frac_of_roofline_time": t_roof / t,
+                        "tokens_per_s": N / t}
         bwd["device_status"] = h.device_status()
         bwd["kernels"] = {"dx": "fused forward kernel on the adjoint operator (1 launch)",
                           "dw": "tcgen05 contraction over tokens + deterministic reduction and inverse DFT "
                                 "(2 launches)" if wl.io_dtype != "f32" else
                                 "float64 CUDA-core kernel (clear + kernel + convert)"}
-        del dxs
+        out["backward"] = bwd
+        del dxs, ws_t
 
-    # ----------------------------------------------------------- MLP block
+    # ------------------------------------------------------- MLP block (headline)
     # The equivariant MLP block y = L2(GELU(L1(x))) at the workload's channels with a
-    # 4x hidden layer (16-bit square workloads): two fused launches, GELU in the first
-    # one's epilogue, the hidden activation through HBM.  Timed like the backward calls.
-    mlp = None
-    if not args.no_mlp_block and wl.io_dtype != "f32" and wl.Cin == wl.Cout:
+    # 4x hidden layer: two fused launches, GELU in the first one's epilogue, the hidden
+    # activation through HBM.  Timed like the backward calls.
+    if headline and not args.no_mlp_block and wl.io_dtype != "f32" and wl.Cin == wl.Cout:
         H = 4 * wl.Cin
         w1, b1, w2, b2 = workloads.make_mlp_weights(wl, H)
         h1 = eq.prepare(w1.to(dev), b1.to(dev), io_dtype=wl.torch_dtype, activation="gelu")
         h2 = eq.prepare(w2.to(dev), b2.to(dev), io_dtype=wl.torch_dtype)
         hidden = torch.empty(N, H, wl.G, dtype=wl.torch_dtype, device=dev)
-        Kb = max(10, min(K, 200))
-        for i in range(max(3, args.warmup)):
+
+        def blk(i):
             eq.mlp_block(h1, h2, xs[i % n_sets], hidden=hidden, out=ys[i % n_sets], stream=stream)
-        barrier()
-        torch.cuda.synchronize(dev)
-        m0 = torch.cuda.Event(enable_timing=True)
-        m1 = torch.cuda.Event(enable_timing=True)
-        m0.record(stream)
-        for i in range(Kb):
-            eq.mlp_block(h1, h2, xs[i % n_sets], hidden=hidden, out=ys[i % n_sets], stream=stream)
-        m1.record(stream)
-        torch.cuda.synchronize(dev)
-        barrier()
-        us = 1e3 * reduce_max(m0.elapsed_time(m1), dev) / Kb
-        mlp = {"H": H, "us_per_block": us, "calls": Kb, "launches_per_block": 2,
-               "device_status": max(h1.device_status(), h2.device_status(), key=abs),
-               "tokens_per_s": N / (us * 1e-6)}
+
+        Kb = max(10, min(max(K, 100), 200))
+        for i in range(max(3, warmup)):
+            blk(i)
+        us = 1e3 * time_back_to_back(ctx, blk, Kb) / Kb
+        e, peaks = wl.elem_bytes, ctx.peaks
+        # two launches: x in, hidden out and back in, y out, both weight sets
+        mbytes = N * (wl.Cin + 2 * H + wl.Cout) * wl.G * e + 2 * wl.G * wl.Cin * H * e
+        mflops = 2 * N * wl.Cin * H * (2 * wl.G - 2) + 2 * N * H * wl.Cout * (2 * wl.G - 2)
+        t_mh = mbytes / (peaks["hbm_gbs"] * 1e9)
+        t_mt = mflops / (peaks["bf16_tflops"] * 1e12)
+        out["mlp_block"] = {
+            "H": H, "us_per_block": us, "calls": Kb, "launches_per_block": 2,
+            "device_status": max(h1.device_status(), h2.device_status(), key=abs),
+            "tokens_per_s": N / (us * 1e-6), "bytes": mbytes, "fourier_flops": mflops,
+            "roofline_time_us": 1e6 * max(t_mh, t_mt), "bound": "hbm" if t_mh >= t_mt else "tensor",
+            "frac_of_roofline_time": max(t_mh, t_mt) / (us * 1e-6),
+            "fused_block_roofline_us": 1e6 * max(N * (wl.Cin + wl.Cout) * wl.G * e / (peaks["hbm_gbs"] * 1e9), t_mt),
+            "note": "roofline of the two-launch form (hidden activation through HBM); "
+                    "fused_block_roofline_us is the bound of a single fused kernel"}
         del hidden
         h1.close()
         h2.close()
 
-    # ----------------------------------------------------------- CPU baseline
+    h.close()
+    del xs, ys
+    torch.cuda.empty_cache()
+    return out
+
+
+def main() -> None:
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=workloads.HEADLINE, choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--impl", default="eqlin", choices=["eqlin", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="oracle sample of the headline workload, seconds on all cores")
+    ap.add_argument("--cpu-seconds-other", type=float, default=3.0,
+                    help="oracle sample of each other workload, seconds on all cores")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", action="store_true",
+                    help="measure only --workload (no workloads object)")
+    ap.add_argument("--no-mlp-block", action="store_true",
+                    help="skip the extra measurement of the equivariant MLP block L2(GELU(L1(x))), H = 4 C")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip the extra measurement of the backward calls (input and weight gradients)")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override the workload's token count (profiling a smaller case; implies --only)")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    wl = workloads.WORKLOADS[args.workload]
+    if args.tokens is not None:
+        wl = wl.with_n(args.tokens)
+        args.only = True
+
+    if args.impl == "reference":
+        run_reference(args, wl)
+        return
+
+    import cyclic_group_dft_b200 as eq
+    eq.library()   # the CUDA library; fails loudly when it is missing
+
+    world, rank, local = dist_info()
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks, peak_kind = load_peaks()
+    ctx = Ctx(eq, dev, world, torch.cuda.current_stream(dev), peaks, peak_kind)
+
+    # every other workload first (each step count at least 100 launches: their launches
+    # are short), the headline last with exactly --steps timed launches
+    results = {}
+    if not args.only:
+        for name in BENCH_WORKLOADS:
+            if name == wl.name:
+                continue
+            results[name] = measure_workload(ctx, workloads.WORKLOADS[name], max(args.steps, 100), args.warmup,
+                                             False, args)
+    head = measure_workload(ctx, wl, args.steps, args.warmup, True, args)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, n_s, dt, threads = oracle_rate(wl, args.cpu_seconds)
-        rate1, n1, dt1, _ = oracle_rate(wl, min(args.cpu_seconds, 5.0), threads=1)
-        cpu = {"value": rate, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-               "sample": f"{n_s} of {wl.N} tokens of {wl.name} in {dt:.1f} s (float64 definition loops, OpenMP over tokens)",
-               "single_core": {"value": rate1, "unit": "tokens/s", "cores": 1,
-                               "sample": f"{n1} of {wl.N} tokens in {dt1:.1f} s"}}
+        cpu = cpu_baseline(wl, args.cpu_seconds, min(args.cpu_seconds, 5.0))
+        for name, r in results.items():
+            r["cpu_baseline"] = cpu_baseline(workloads.WORKLOADS[name], args.cpu_seconds_other)
+        head["cpu_baseline"] = cpu
 
     if world > 1:
         torch.distributed.barrier()
@@ -479,87 +609,41 @@ def main() -> None:
     if rank != 0:
         return
 
-    peaks, peak_kind = load_peaks()
-    bytes_launch = algorithmic_bytes(wl, N)
-    flops_launch = fourier_flops(wl, N)
-    gbs = bytes_launch / avg_launch_s / 1e9
-    tflops = flops_launch / avg_launch_s / 1e12
-    t_hbm = bytes_launch / (peaks["hbm_gbs"] * 1e9)
-    t_tc = flops_launch / (peaks["bf16_tflops"] * 1e12)
-    bound = "hbm" if t_hbm >= t_tc else "tensor"
-    if bound == "hbm":
-        roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": gbs / peaks["hbm_gbs"]}
+    if not args.only:
+        ordered = {name: head if name == wl.name else results[name] for name in BENCH_WORKLOADS}
+        wl_obj = {name: {k: v for k, v in r.items() if k not in ("e2e", "mlp_block", "clocks")}
+                  for name, r in ordered.items()}
     else:
-        roof = {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": tflops / peaks["bf16_tflops"]}
-    roof["traffic"] = recorded_traffic(wl.name)
-    roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback"
-    roof["roofline_time_us"] = 1e6 * max(t_hbm, t_tc)
-    roof["kernel_us"] = 1e6 * avg_launch_s
-    roof["frac_of_roofline_time"] = max(t_hbm, t_tc) / avg_launch_s
-    roof["bytes_per_launch"] = bytes_launch
-    roof["tensor_tflops"] = tflops
-    roof["tensor_frac"] = tflops / peaks["bf16_tflops"]                       # burst peak: the headline
-    roof["tensor_frac_sustained"] = tflops / peaks["bf16_tflops_sustained"]   # seconds-long GEMM peak
+        wl_obj = None
 
-    if mlp is not None:
-        e, H = wl.elem_bytes, mlp["H"]
-        # two launches: x in, hidden out and back in, y out, both weight sets
-        mbytes = N * (wl.Cin + 2 * H + wl.Cout) * wl.G * e + 2 * wl.G * wl.Cin * H * e
-        mflops = 2 * N * wl.Cin * H * (2 * wl.G - 2) + 2 * N * H * wl.Cout * (2 * wl.G - 2)
-        t_mh = mbytes / (peaks["hbm_gbs"] * 1e9)
-        t_mt = mflops / (peaks["bf16_tflops"] * 1e12)
-        t = mlp["us_per_block"] * 1e-6
-        mlp.update({"bytes": mbytes, "fourier_flops": mflops, "roofline_time_us": 1e6 * max(t_mh, t_mt),
-                    "bound": "hbm" if t_mh >= t_mt else "tensor", "frac_of_roofline_time": max(t_mh, t_mt) / t,
-                    "fused_block_roofline_us": 1e6 * max(N * (wl.Cin + wl.Cout) * wl.G * e / (peaks["hbm_gbs"] * 1e9),
-                                                         t_mt),
-                    "note": "roofline of the two-launch form (hidden activation through HBM); "
-                            "fused_block_roofline_us is the bound of a single fused kernel"})
-    if bwd is not None:
-        bb = backward_bytes(wl, N)
-        for key in ("dx", "dw"):
-            t = bwd[key]["us_per_call"] * 1e-6
-            t_h = bb[key] / (peaks["hbm_gbs"] * 1e9)
-            t_roof = max(t_h, t_tc)
-            bwd[key].update({"bytes": bb[key], "roofline_time_us": 1e6 * t_roof,
-                             "bound": "hbm" if t_h >= t_tc else "tensor",
-                             "frac_of_roofline_time": t_roof / t, "tokens_per_s": N / t})
-
-    emit({
+    line = {
         "metric": METRIC,
-        "value": value,
+        "value": head["tokens_per_s"],
         "unit": "tokens/s",
         "n_gpus": world,
-        "steps": K,
+        "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": elapsed_ms / K,
+        "ms_per_step": head["elapsed_ms"] / args.steps,
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": wl.io_dtype,
         "data": "synthetic",
-        "config": {
-            "workload": wl.name, "N": N, "Cin": wl.Cin, "Cout": wl.Cout, "G": wl.G, "io": wl.io_dtype,
-            "global_batch": world * N, "parallelism": f"replicas{world}" if world > 1 else "single",
-            "l2": f"inputs larger than L2; {n_sets} rotating x/y sets of {set_bytes / 1e6:.0f} MB",
-            "kernel_path": h.path, "stages": h.attr("stages"), "tokens_per_tile": h.attr("tokens_per_tile"),
-        },
-        "roofline": roof,
-        "dense_equivalent_tflops": dense_equivalent_flops(wl, N) / avg_launch_s / 1e12,
-        "launch_us": {"mean": 1e3 * statistics.mean(launch_ms), "median": 1e3 * statistics.median(launch_ms),
-                      "min": 1e3 * min(launch_ms), "max": 1e3 * max(launch_ms), "launches": len(launch_ms),
-                      "note": "each launch bracketed by its own events (serialised), outside the timed region"},
-        "clocks": clocks.summary(),
-        "e2e": e2e,
-        "gpu_launches": K,
-        "device_status": status,
+        "config": line_config(wl, world),
+        "kernel": head["kernel"],
+        "roofline": head["roofline"],
+        "dense_equivalent_tflops": head["dense_equivalent_tflops"],
+        "launch_us": head["launch_us"],
+        "clocks": head.get("clocks"),
+        "e2e": head.get("e2e"),
+        "gpu_launches": args.steps,
+        "device_status": head["device_status"],
         "cpu_baseline": cpu,
-        "backward": bwd,
-        "mlp_block": mlp,
-    })
-    h.close()
+        "backward": head.get("backward"),
+        "mlp_block": head.get("mlp_block"),
+        "workloads": wl_obj,
+    }
+    emit(line)
 
 
 if __name__ == "__main__":

@@ -406,6 +406,10 @@ def eqlin_forward_noalloc(x: torch.Tensor, w: torch.Tensor, bias: torch.Tensor |
         raise ValueError("bias must be a contiguous [Cout] tensor of x's dtype")
     if y is None:
         y = torch.empty((N, Cout, G), dtype=x.dtype, device=x.device)
+    elif y.shape != (N, Cout, G) or y.dtype != x.dtype or y.device != x.device or not y.is_contiguous():
+        raise ValueError(f"y must be a contiguous [{N}, {Cout}, {G}] tensor of x's dtype on x's device")
+    if bias is not None and bias.device != x.device:
+        raise ValueError("bias must be on x's device")
     with torch.cuda.device(x.device):
         _check(_lib.eqlin_forward_noalloc(x.data_ptr(), w.data_ptr(), None if bias is None else bias.data_ptr(),
                                           y.data_ptr(), N, Cout, Cin, G, _TORCH_TO_EQLIN[x.dtype],

@@ -175,6 +175,7 @@ int eqlin_prepare_weights_ex(const void* w, const void* bias, int64_t Cout, int6
     h->io_dtype = io_dtype;
     h->plan = plan;
     h->buf.has_bias = bias != nullptr;
+    h->buf.w_early = true;   // prepare synchronises its stream before any forward can use them
     h->buf.act = (flags & EQLIN_PREPARE_GELU) ? eqlin::kActGelu : eqlin::kActNone;
     // Test hook for failure detection (read at prepare, never set outside tests): with
     // EQLIN_TEST_STOP_AFTER=k the fused kernels' producer stops after issuing k chunks per
@@ -233,6 +234,7 @@ int eqlin_prepare_weights_ex(const void* w, const void* bias, int64_t Cout, int6
         const Plan& pd = h->plan_dx;
         d.status = b.status;
         d.has_bias = false;
+        d.w_early = true;
         if (cudaMalloc(&d.w_f32, wf_bytes) != cudaSuccess ||
             cudaMalloc(&d.bias_f32, static_cast<size_t>(Cin) * sizeof(float)) != cudaSuccess ||
             (pd.path == kPathF32 && (cudaMalloc(&d.w_f64, wf_bytes * 2) != cudaSuccess ||
@@ -642,6 +644,7 @@ extern "C" int eqlin_forward_noalloc(const void* x, const void* w, const void* b
     b.bias_f64 = plan.path == kPathF32 ? reinterpret_cast<double*>(sc + off_bd) : nullptr;
     b.img = plan.path == kPathF32 ? nullptr : sc + off_img;
     b.has_bias = bias != nullptr;
+    b.w_early = false;   // the weight transform below writes them in the same stream
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
     // the status word keeps the previous call's value: clear it

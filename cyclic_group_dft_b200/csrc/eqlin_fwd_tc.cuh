@@ -65,6 +65,11 @@ struct TcParams {
     unsigned long long timeout_ns;
     long long inject_stop;  // test hook: chunks issued per CTA before the producer stops; -1 = never
     int act;                  // epilogue activation after the bias: kActNone or kActGelu
+    // 1: the weights (and bias) were complete before the previous kernel of the stream was
+    // launched (a handle's weights: prepare synchronises its stream), so their loads may
+    // start before griddepcontrol.wait and overlap the previous kernel's tail.  0: they may
+    // be written by the previous kernel of the stream; every load waits.
+    int w_early;
 };
 
 namespace tc {
@@ -407,8 +412,20 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem_base = ctl->tmem_base;
+    // resident weights: one bulk copy per 32 KB, completing on bar_w_full
+    auto load_weights = [&]() {
+        ptx::mbar_arrive_expect_tx(bar_w_full, p.w_img_bytes);
+        for (uint32_t off = 0; off < p.w_img_bytes; off += 32768u) {
+            const uint32_t n = min(32768u, p.w_img_bytes - off);
+            ptx::bulk_load(s_w + off, p.w_img + off, n, bar_w_full);
+        }
+    };
+    // weights that no kernel of the stream writes are staged while the previous kernel drains
+    if constexpr (!STREAM_W) {
+        if (p.w_early && warp == tc::kWarpProducer && lane == 0) load_weights();
+    }
     // The next forward of the stream may begin launching (its CTAs take an SM as one of
-    // ours exits); every global access below waits until the previous kernel of the
+    // ours exits); every access to x and y below waits until the previous kernel of the
     // stream has completed, so y / x aliasing between consecutive calls stays safe.
     ptx::grid_launch_dependents();
     ptx::grid_dependency_wait();
@@ -417,11 +434,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             if constexpr (!STREAM_W) {
-                ptx::mbar_arrive_expect_tx(bar_w_full, p.w_img_bytes);
-                for (uint32_t off = 0; off < p.w_img_bytes; off += 32768u) {
-                    const uint32_t n = min(32768u, p.w_img_bytes - off);
-                    ptx::bulk_load(s_w + off, p.w_img + off, n, bar_w_full);
-                }
+                if (!p.w_early) load_weights();
             }
             int stage = 0;
             uint32_t phase = 0;

@@ -93,6 +93,19 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem_base = ctl->tmem_base;
+    // Weights that no kernel of the stream writes (p.w_early): the first ring stages are
+    // filled with the first tile's weight chunks while the previous kernel drains.  The
+    // ring order is the same as below, which then skips issuing those chunks.
+    int w_prefilled = 0;
+    if (p.w_early && warp == tc::kWarpProducer && lane == 0 && blockIdx.x < p.n_work) {
+        const int pre = min(NS, p.n_oc * nK);
+        for (int j = 0; j < pre; ++j) {
+            ptx::mbar_arrive_expect_tx(bar_w_full(j), S::WSTAGE_BYTES);
+            ptx::bulk_load(s_wring0 + j * S::WSTAGE_BYTES, p.w_img + static_cast<size_t>(j) * S::WSTAGE_BYTES,
+                           S::WSTAGE_BYTES, bar_w_full(j));
+        }
+        w_prefilled = pre;
+    }
     ptx::grid_launch_dependents();
     ptx::grid_dependency_wait();
 
@@ -134,6 +147,11 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                 ++tiles_loaded;
                 for (int oc = 0; ok && oc < p.n_oc; ++oc) {
                     for (int c = 0; c < nK; ++c) {
+                        if (issued_w < w_prefilled) {   // issued before griddepcontrol.wait
+                            ++issued_w;
+                            if (++ws == NS) { ws = 0; wph ^= 1u; }
+                            continue;
+                        }
                         if (!tc::wait_bounded(bar_w_empty(ws), wph ^ 1u, ctl, p.status, p.timeout_ns)) {
                             ok = false;
                             break;
@@ -154,8 +172,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                 const int uses = tiles_loaded + (c < last_tile_chunks && last_tile_chunks < nK ? 1 : 0);
                 if (uses > 0) tc::drain_wait(bar_x_full(c), static_cast<uint32_t>((uses - 1) & 1), p.status, p.timeout_ns);
             }
+            // chunks prefilled before the wait are in flight even if the loop stopped early
+            const long long w_total = issued_w > w_prefilled ? issued_w : w_prefilled;
             for (int s = 0; s < NS; ++s) {
-                const long long times = issued_w > s ? (issued_w - s + NS - 1) / NS : 0;
+                const long long times = w_total > s ? (w_total - s + NS - 1) / NS : 0;
                 if (times > 0)
                     tc::drain_wait(bar_w_full(s), static_cast<uint32_t>((times - 1) & 1), p.status, p.timeout_ns);
             }

@@ -167,6 +167,11 @@ struct WeightBuffers {
     bool has_bias = false;
     int act = eqlin::kActNone;   // epilogue activation of the forward (EQLIN_PREPARE_GELU)
     long long inject_stop = -1;  // failure-detection test hook (EQLIN_TEST_STOP_AFTER), -1 = off
+    // The weights were complete before any forward using them was queued (a handle's:
+    // prepare synchronises its stream), so the fused kernels may load them before
+    // griddepcontrol.wait.  False for weights a kernel of the same stream writes just
+    // before the forward (the allocation-free entry point's scratch).
+    bool w_early = false;
 };
 
 // Cout x Cin is the operator's shape.  adjoint: the operator is the layer's input
@@ -282,6 +287,7 @@ int launch_forward(const Plan& pl, int64_t Cout, int64_t Cin, int64_t G, int sm_
             p.timeout_ns = timeout_ns;
             p.act = b.act;
             p.inject_stop = b.inject_stop;
+            p.w_early = b.w_early ? 1 : 0;
             const TmEntry entry = tm_entry_for(iG, pl.streamed(), pl.io);
             if (!entry.launch) return fail(EQLIN_ERR_UNSUPPORTED, "G");
             entry.launch(grid, pl.smem_bytes, st, map, ymap, p);
@@ -305,6 +311,7 @@ int launch_forward(const Plan& pl, int64_t Cout, int64_t Cin, int64_t G, int sm_
             p.timeout_ns = timeout_ns;
             p.act = b.act;
             p.inject_stop = b.inject_stop;
+            p.w_early = b.w_early ? 1 : 0;
             const TcEntry entry = pl.tnr() ? tcr_entry_for(iG, pl.io) : tc_entry_for(iG, pl.streamed(), pl.nacc, pl.io);
             if (!entry.launch) return fail(EQLIN_ERR_UNSUPPORTED, "G");
             entry.launch(grid, pl.smem_bytes, st, map, ymap, p);
