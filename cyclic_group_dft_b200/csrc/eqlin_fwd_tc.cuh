@@ -70,6 +70,10 @@ struct TcParams {
     // start before griddepcontrol.wait and overlap the previous kernel's tail.  0: they may
     // be written by the previous kernel of the stream; every load waits.
     int w_early;
+    // L2 prefetch distance of the producer, in this CTA's work items: while loading item
+    // i it asks the TMA unit to bring item i + pf into L2, so more of x is in flight than
+    // the shared-memory ring holds.  0 = off.
+    int pf;
 };
 
 namespace tc {
@@ -440,9 +444,20 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
             uint32_t phase = 0;
             long long issued = 0;
             bool ok = true;
+            // x chunks of work item wk into L2 (a hint: the loads below still bring them)
+            auto prefetch_item = [&](long long wk) {
+                if (wk >= p.n_work) return;
+                const int n0 = static_cast<int>(wk / p.n_oc) * S::BN;
+                for (int c = 0; c < p.nK; ++c)
+#pragma unroll
+                    for (int bx = 0; bx < S::NBOX; ++bx)
+                        ptx::tma_prefetch_l2_2d(&tmap_x, c * S::XROW_ELEMS + bx * S::BOX_ELEMS, n0);
+            };
+            for (int j = 1; j < p.pf; ++j) prefetch_item(blockIdx.x + static_cast<long long>(j) * gridDim.x);
             for (int wk = blockIdx.x; ok && wk < p.n_work; wk += gridDim.x) {
                 const int tile = wk / p.n_oc, oc = wk % p.n_oc;
                 const int n0 = tile * S::BN;
+                if (p.pf > 0) prefetch_item(wk + static_cast<long long>(p.pf) * gridDim.x);
                 for (int c = 0; c < p.nK; ++c) {
                     if (!tc::wait_bounded(bar_empty(stage), phase ^ 1u, ctl, p.status, p.timeout_ns)) {
                         ok = false;

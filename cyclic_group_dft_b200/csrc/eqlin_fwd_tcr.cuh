@@ -119,7 +119,18 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
             uint32_t wph = 0;
             bool ok = true;
             int ti = 0;
+            // x chunks of token tile t into L2 (a hint: the loads below still bring them)
+            auto prefetch_tile = [&](long long t) {
+                if (t >= p.n_work) return;
+                const int n0 = static_cast<int>(t) * S::BN;
+                for (int c = 0; c < nK; ++c)
+#pragma unroll
+                    for (int bx = 0; bx < S::NBOX; ++bx)
+                        ptx::tma_prefetch_l2_2d(&tmap_x, c * S::XROW_ELEMS + bx * S::BOX_ELEMS, n0);
+            };
+            for (int j = 1; j < p.pf; ++j) prefetch_tile(blockIdx.x + static_cast<long long>(j) * gridDim.x);
             for (int tile = blockIdx.x; ok && tile < p.n_work; tile += gridDim.x, ++ti) {
+                if (p.pf > 0) prefetch_tile(tile + static_cast<long long>(p.pf) * gridDim.x);
                 // the slots are free once every MMA of the previous tile has completed
                 if (!tc::wait_bounded(bar_x_free, (static_cast<uint32_t>(ti) & 1u) ^ 1u, ctl, p.status,
                                       p.timeout_ns)) {

@@ -55,6 +55,7 @@ struct TmParams {
     long long inject_stop;  // test hook: chunks issued per CTA before the producer stops; -1 = never
     int act;                // epilogue activation after the bias: kActNone or kActGelu
     int w_early;            // weights may be loaded before griddepcontrol.wait (TcParams::w_early)
+    int pf;                 // L2 prefetch distance in work items (TcParams::pf), 0 = off
 };
 
 namespace tm {
@@ -321,9 +322,20 @@ __global__ void __launch_bounds__(tm::Cfg<G>::kThreads, 1)
             uint32_t phase = 0;
             long long issued = 0;
             bool ok = true;
+            // x chunks of work item wk into L2 (a hint: the loads below still bring them)
+            auto prefetch_item = [&](long long wk) {
+                if (wk >= p.n_work) return;
+                const int n0 = static_cast<int>(wk / p.n_oc) * tm::kM;
+                for (int c = 0; c < p.nK; ++c)
+#pragma unroll
+                    for (int bx = 0; bx < C::X_NBOX; ++bx)
+                        ptx::tma_prefetch_l2_2d(&tmap_x, c * C::XROW_ELEMS + bx * C::X_BOX, n0);
+            };
+            for (int j = 1; j < p.pf; ++j) prefetch_item(blockIdx.x + static_cast<long long>(j) * gridDim.x);
             for (int wk = blockIdx.x; ok && wk < p.n_work; wk += gridDim.x) {
                 const int tile = wk / p.n_oc, oc = wk % p.n_oc;
                 const int n0 = tile * tm::kM;
+                if (p.pf > 0) prefetch_item(wk + static_cast<long long>(p.pf) * gridDim.x);
                 for (int c = 0; c < p.nK; ++c) {
                     if (!tc::wait_bounded(bar_empty(stage), phase ^ 1u, ctl, p.status, p.timeout_ns)) {
                         ok = false;

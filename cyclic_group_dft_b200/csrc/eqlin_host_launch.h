@@ -154,6 +154,20 @@ void* kernel_for(const Plan& pl, int G) {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// L2 prefetch distance of the fused kernels' producer, in work items of the CTA.
+// EQLIN_PREFETCH=k overrides (0 turns the prefetch off).
+int prefetch_distance() {
+    static const int d = [] {
+        const char* e = std::getenv("EQLIN_PREFETCH");
+        if (e && *e) {
+            const int v = std::atoi(e);
+            if (v >= 0 && v <= 16) return v;
+        }
+        return kDefaultPrefetch;
+    }();
+    return d;
+}
+
 // ------------------------------------------------------------------ launches
 // Buffers of the frequency-domain weights (owned by a handle or carved from the
 // allocation-free scratch array).
@@ -288,6 +302,7 @@ int launch_forward(const Plan& pl, int64_t Cout, int64_t Cin, int64_t G, int sm_
             p.act = b.act;
             p.inject_stop = b.inject_stop;
             p.w_early = b.w_early ? 1 : 0;
+            p.pf = prefetch_distance();
             const TmEntry entry = tm_entry_for(iG, pl.streamed(), pl.io);
             if (!entry.launch) return fail(EQLIN_ERR_UNSUPPORTED, "G");
             entry.launch(grid, pl.smem_bytes, st, map, ymap, p);
@@ -312,6 +327,7 @@ int launch_forward(const Plan& pl, int64_t Cout, int64_t Cin, int64_t G, int sm_
             p.act = b.act;
             p.inject_stop = b.inject_stop;
             p.w_early = b.w_early ? 1 : 0;
+            p.pf = prefetch_distance();
             const TcEntry entry = pl.tnr() ? tcr_entry_for(iG, pl.io) : tc_entry_for(iG, pl.streamed(), pl.nacc, pl.io);
             if (!entry.launch) return fail(EQLIN_ERR_UNSUPPORTED, "G");
             entry.launch(grid, pl.smem_bytes, st, map, ymap, p);

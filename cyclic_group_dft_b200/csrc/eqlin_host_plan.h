@@ -14,6 +14,7 @@ constexpr size_t kSmemCtlBytes = 512;       // mbarriers + control block
 constexpr int kMaxStages = 12;
 constexpr int64_t kMaxChannels = 1 << 16;
 constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per bounded wait
+constexpr int kDefaultPrefetch = 2;   // L2 prefetch distance of the fused kernels (work items)
 
 // Kernel variants (EQLIN_ATTR_PATH):
 //   0/1  tcgen05, tokens on the MMA N dimension, weights resident / streamed
