@@ -64,6 +64,10 @@ _EXPORTS = (
     "header_functions",
     "library",
     "mlp_block",
+    "MlpHandle",
+    "eqlin_mlp_prepare",
+    "eqlin_mlp_forward",
+    "eqlin_mlp_query",
 )
 
 __all__ = list(_EXPORTS) + ["prepare", "workloads"]

@@ -65,6 +65,11 @@ _lib.eqlin_prepare_weights_ex.argtypes = [_vp, _vp, _i64, _i64, _i64, _int, _int
 _lib.eqlin_backward_dx.argtypes = [_vp, _vp, _vp, _i64, _vp]
 _lib.eqlin_backward_dw_workspace_size.argtypes = [_vp, _i64, ctypes.POINTER(ctypes.c_size_t)]
 _lib.eqlin_backward_dw.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _vp, ctypes.c_size_t, _vp]
+_lib.eqlin_mlp_prepare.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _int, _int, _vp, ctypes.POINTER(_vp)]
+_lib.eqlin_mlp_forward.argtypes = [_vp, _vp, _vp, _i64, _vp]
+_lib.eqlin_mlp_device_status.argtypes = [_vp, ctypes.POINTER(_int)]
+_lib.eqlin_mlp_destroy.argtypes = [_vp]
+_lib.eqlin_mlp_query.argtypes = [_i64, _i64, _i64, _i64, _int, ctypes.POINTER(_i64), ctypes.POINTER(_i64)]
 _lib.eqlin_status_string.argtypes = [_int]
 _lib.eqlin_status_string.restype = ctypes.c_char_p
 _lib.eqlin_last_error.argtypes = []
@@ -74,7 +79,8 @@ for _f in ("eqlin_prepare_weights", "eqlin_forward", "eqlin_forward_host", "eqli
            "eqlin_device_status",
            "eqlin_get_attr", "eqlin_copy_freq_weights", "eqlin_check_shape", "eqlin_version",
            "eqlin_forward_noalloc", "eqlin_prepare_weights_ex", "eqlin_backward_dx",
-           "eqlin_backward_dw_workspace_size", "eqlin_backward_dw"):
+           "eqlin_backward_dw_workspace_size", "eqlin_backward_dw", "eqlin_mlp_prepare", "eqlin_mlp_forward",
+           "eqlin_mlp_device_status", "eqlin_mlp_destroy", "eqlin_mlp_query"):
     getattr(_lib, _f).restype = _int
 
 
@@ -366,6 +372,108 @@ def mlp_block(h1: Handle, h2: Handle, x: torch.Tensor, hidden: torch.Tensor | No
         raise ValueError("h1's outputs must match h2's inputs (channels, G, dtype, device)")
     hidden = eqlin_forward(h1, x, hidden, stream)
     return eqlin_forward(h2, hidden, out, stream)
+
+
+class MlpHandle:
+    """Both weight sets of an equivariant MLP block y = L2(GELU(L1(x))), transformed for
+    the single fused kernel (eqlin_mlp_prepare; owns device memory)."""
+
+    def __init__(self, ptr: int, device: torch.device, Cin: int, H: int, Cout: int, G: int, io_dtype: torch.dtype):
+        self._ptr = ptr
+        self.device = device
+        self.Cin, self.H, self.Cout, self.G, self.io_dtype = Cin, H, Cout, G, io_dtype
+
+    @property
+    def ptr(self) -> int:
+        if not self._ptr:
+            raise EqlinError(EQLIN_ERR_INVALID_ARG, "MLP handle already destroyed")
+        return self._ptr
+
+    def forward(self, x: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        return eqlin_mlp_forward(self, x, out, stream)
+
+    def device_status(self) -> int:
+        v = ctypes.c_int()
+        with torch.cuda.device(self.device):
+            _check(_lib.eqlin_mlp_device_status(self.ptr, ctypes.byref(v)), "eqlin_mlp_device_status")
+        return int(v.value)
+
+    def close(self) -> None:
+        if self._ptr:
+            p, self._ptr = self._ptr, None
+            _check(_lib.eqlin_mlp_destroy(p), "eqlin_mlp_destroy")
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def __del__(self):
+        try:
+            if self._ptr and _lib is not None:
+                _lib.eqlin_mlp_destroy(self._ptr)
+                self._ptr = None
+        except Exception:
+            pass
+
+
+def eqlin_mlp_query(Cin: int, H: int, Cout: int, G: int, io_dtype=torch.bfloat16) -> dict | None:
+    """Host only: {"stages", "smem_bytes"} of the fused MLP block's kernel for these sizes on
+    a B200, or None when the fused block does not support them."""
+    st, sm = _i64(), _i64()
+    s = _lib.eqlin_mlp_query(Cin, H, Cout, G, _as_code(io_dtype), ctypes.byref(st), ctypes.byref(sm))
+    if s != EQLIN_OK:
+        return None
+    return {"stages": int(st.value), "smem_bytes": int(sm.value)}
+
+
+def eqlin_mlp_prepare(w1: torch.Tensor, b1: torch.Tensor | None, w2: torch.Tensor, b2: torch.Tensor | None,
+                      io_dtype: torch.dtype | None = None, stream=None) -> MlpHandle:
+    """Transform the weights of y = L2(GELU(L1(x))) for the fused kernel: w1 [H, Cin, G],
+    b1 [H] or None, w2 [Cout, H, G], b2 [Cout] or None, all CUDA tensors of one dtype."""
+    if w1.dim() != 3 or w2.dim() != 3 or w2.shape[1] != w1.shape[0] or w2.shape[2] != w1.shape[2]:
+        raise ValueError("w1 must be [H, Cin, G] and w2 [Cout, H, G]")
+    if w1.device.type != "cuda" or w2.device != w1.device:
+        raise ValueError("w1 and w2 must be CUDA tensors on one device")
+    if w1.dtype not in _TORCH_TO_EQLIN or w2.dtype != w1.dtype:
+        raise ValueError("w1 and w2 must share a supported dtype")
+    H, Cin, G = w1.shape
+    Cout = w2.shape[0]
+    w1, w2 = w1.contiguous(), w2.contiguous()
+    bs = []
+    for b, n in ((b1, H), (b2, Cout)):
+        if b is not None:
+            if b.shape != (n,) or b.device != w1.device:
+                raise ValueError("biases must be [H] and [Cout] on the weights' device")
+            b = b.to(w1.dtype).contiguous()
+        bs.append(b)
+    io = w1.dtype if io_dtype is None else io_dtype
+    out = ctypes.c_void_p()
+    with torch.cuda.device(w1.device):
+        st = _lib.eqlin_mlp_prepare(w1.data_ptr(), None if bs[0] is None else bs[0].data_ptr(), w2.data_ptr(),
+                                    None if bs[1] is None else bs[1].data_ptr(), Cin, H, Cout, G,
+                                    _TORCH_TO_EQLIN[w1.dtype], _TORCH_TO_EQLIN[io], _stream_ptr(stream),
+                                    ctypes.byref(out))
+    _check(st, "eqlin_mlp_prepare")
+    return MlpHandle(out.value, w1.device, Cin, H, Cout, G, io)
+
+
+def eqlin_mlp_forward(m: MlpHandle, x: torch.Tensor, y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y [N, Cout, G] = L2(GELU(L1(x [N, Cin, G]))) in one fused launch."""
+    if x.dim() != 3 or x.shape[1] != m.Cin or x.shape[2] != m.G:
+        raise ValueError(f"x must be [N, {m.Cin}, {m.G}], got {tuple(x.shape)}")
+    if x.device != m.device or x.dtype != m.io_dtype or not x.is_contiguous():
+        raise ValueError(f"x must be a contiguous {m.io_dtype} tensor on {m.device}")
+    N = x.shape[0]
+    if y is None:
+        y = torch.empty((N, m.Cout, m.G), dtype=m.io_dtype, device=m.device)
+    elif y.shape != (N, m.Cout, m.G) or y.dtype != m.io_dtype or y.device != m.device or not y.is_contiguous():
+        raise ValueError("y has the wrong shape, dtype, device or layout")
+    with torch.cuda.device(m.device):
+        _check(_lib.eqlin_mlp_forward(m.ptr, x.data_ptr(), y.data_ptr(), N, _stream_ptr(stream)),
+               "eqlin_mlp_forward")
+    return y
 
 
 def eqlin_destroy(h: Handle) -> None:

@@ -22,6 +22,7 @@
 #include "eqlin_fwd_tcr.cuh"
 #include "eqlin_fwd_tm.cuh"
 #include "eqlin_layout.h"
+#include "eqlin_mlp.cuh"
 #include "eqlin_prep.cuh"
 
 using eqlin::TcParams;
@@ -29,6 +30,7 @@ using eqlin::TmParams;
 
 #include "eqlin_host_plan.h"
 #include "eqlin_host_launch.h"
+#include "eqlin_host_mlp.h"
 
 struct eqlin_handle {
     int device = 0;
@@ -654,3 +656,184 @@ extern "C" int eqlin_forward_noalloc(const void* x, const void* w, const void* b
     if (s != EQLIN_OK) return s;
     return launch_forward(plan, Cout, Cin, G, d->sm_count, x, y, N, b, kDefaultTimeoutNs, st);
 }
+
+// ---------------------------------------------------------------------------------
+// The MLP block as one fused launch (eqlin_mlp_*).
+
+struct eqlin_mlp {
+    int device = 0;
+    int sm_count = 0;
+    int64_t Cin = 0, H = 0, Cout = 0, G = 0;
+    int io_dtype = 0;
+    MlpPlan plan;
+    WeightBuffers b1, b2;   // layer 1 ([H x Cin]) and layer 2 ([Cout x H]); b1 owns the status word
+    bool sync_check = false;
+    unsigned long long timeout_ns = kDefaultTimeoutNs;
+};
+
+namespace {
+
+void free_mlp(eqlin_mlp* m) {
+    if (!m) return;
+    for (WeightBuffers* b : {&m->b1, &m->b2}) {
+        if (b->img) cudaFree(b->img);
+        if (b->w_f32) cudaFree(b->w_f32);
+        if (b->bias_f32) cudaFree(b->bias_f32);
+        if (b->w_f64) cudaFree(b->w_f64);
+        if (b->bias_f64) cudaFree(b->bias_f64);
+    }
+    if (m->b1.status) cudaFree(m->b1.status);
+    delete m;
+}
+
+int alloc_layer(const Plan& lp, int64_t O, int64_t I, int64_t G, WeightBuffers& b) {
+    const size_t planes = static_cast<size_t>(G) * I * O;
+    if (cudaMalloc(&b.w_f32, planes * sizeof(float)) != cudaSuccess ||
+        cudaMalloc(&b.bias_f32, static_cast<size_t>(O) * sizeof(float)) != cudaSuccess ||
+        (lp.path == kPathF32 && (cudaMalloc(&b.w_f64, planes * sizeof(double)) != cudaSuccess ||
+                                 cudaMalloc(&b.bias_f64, static_cast<size_t>(O) * sizeof(double)) != cudaSuccess)) ||
+        (lp.img_alloc_bytes && cudaMalloc(&b.img, lp.img_alloc_bytes) != cudaSuccess)) {
+        cudaGetLastError();
+        return fail(EQLIN_ERR_OOM, "device allocation for the MLP block's transformed weights");
+    }
+    return EQLIN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int eqlin_mlp_query(int64_t Cin, int64_t H, int64_t Cout, int64_t G, int io_dtype, int64_t* stages,
+                    int64_t* smem_bytes) {
+    MlpPlan pl;
+    const int s = plan_mlp(Cin, H, Cout, G, io_dtype, kB200SmemOptin, &pl);
+    if (s != EQLIN_OK) return s;
+    if (stages) *stages = pl.stages;
+    if (smem_bytes) *smem_bytes = static_cast<int64_t>(pl.smem_bytes);
+    return EQLIN_OK;
+}
+
+int eqlin_mlp_prepare(const void* w1, const void* b1, const void* w2, const void* b2, int64_t Cin, int64_t H,
+                      int64_t Cout, int64_t G, int w_dtype, int io_dtype, void* stream, eqlin_mlp** out) {
+    if (!out) return fail(EQLIN_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    if (!w1 || !w2) return fail(EQLIN_ERR_INVALID_ARG, "w1 or w2 is NULL");
+    int s = check_shape_impl(H, Cin, G, w_dtype, io_dtype);
+    if (s == EQLIN_OK) s = check_shape_impl(Cout, H, G, w_dtype, io_dtype);
+    if (s != EQLIN_OK) return s;
+    const size_t welt = w_dtype == EQLIN_F32 ? 4 : 2;
+    if (!aligned(w1, welt) || !aligned(w2, welt) || (b1 && !aligned(b1, welt)) || (b2 && !aligned(b2, welt)))
+        return fail(EQLIN_ERR_MISALIGNED, "weights / biases not aligned to their element size");
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    int major = 0, minor = 0, sms = 0, optin = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
+        return cuda_fail(e, "device query");
+    if (major != 10 || minor != 0) return fail(EQLIN_ERR_UNSUPPORTED, "needs a compute capability 10.0 (sm_100a) device");
+    MlpPlan plan;
+    s = plan_mlp(Cin, H, Cout, G, io_dtype, static_cast<size_t>(optin), &plan);
+    if (s != EQLIN_OK) return s;
+
+    eqlin_mlp* m = new (std::nothrow) eqlin_mlp();
+    if (!m) return fail(EQLIN_ERR_OOM, "host allocation");
+    m->device = dev;
+    m->sm_count = sms;
+    m->Cin = Cin;
+    m->H = H;
+    m->Cout = Cout;
+    m->G = G;
+    m->io_dtype = io_dtype;
+    m->plan = plan;
+    m->b1.has_bias = b1 != nullptr;
+    m->b2.has_bias = b2 != nullptr;
+    m->b1.w_early = m->b2.w_early = true;   // prepare synchronises its stream before any forward
+    if (const char* t = std::getenv("EQLIN_TEST_STOP_AFTER")) {   // failure-detection test hook
+        const long long k = std::atoll(t);
+        if (k >= 0) m->b1.inject_stop = k;
+    }
+    const char* sc = std::getenv("EQLIN_SYNC_CHECK");
+    m->sync_check = sc && sc[0] == '1';
+    if (const char* t = std::getenv("EQLIN_WAIT_TIMEOUT_MS")) {
+        const long long ms = std::atoll(t);
+        if (ms > 0) m->timeout_ns = static_cast<unsigned long long>(ms) * 1000000ull;
+    }
+    if ((s = alloc_layer(plan.layer1, H, Cin, G, m->b1)) != EQLIN_OK ||
+        (s = alloc_layer(plan.layer2, Cout, H, G, m->b2)) != EQLIN_OK) {
+        free_mlp(m);
+        return s;
+    }
+    if (cudaMalloc(&m->b1.status, 256) != cudaSuccess) {
+        cudaGetLastError();
+        free_mlp(m);
+        return fail(EQLIN_ERR_OOM, "device allocation for the status word");
+    }
+    m->b2.status = m->b1.status;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((e = cudaMemsetAsync(m->b1.status, 0, 256, st)) != cudaSuccess) {
+        free_mlp(m);
+        return cuda_fail(e, "status init");
+    }
+    s = launch_prep(plan.layer1, w_dtype, w1, b1, H, Cin, G, m->b1, st);
+    if (s == EQLIN_OK) s = launch_prep(plan.layer2, w_dtype, w2, b2, Cout, H, G, m->b2, st);
+    if (s == EQLIN_OK && (e = cudaStreamSynchronize(st)) != cudaSuccess) s = cuda_fail(e, "MLP weight transform");
+    if (s == EQLIN_OK &&
+        (e = cudaFuncSetAttribute(mlp_kernel_for(static_cast<int>(G), io_dtype),
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, optin)) != cudaSuccess)
+        s = cuda_fail(e, "cudaFuncSetAttribute");
+    if (s != EQLIN_OK) {
+        free_mlp(m);
+        return s;
+    }
+    *out = m;
+    return EQLIN_OK;
+}
+
+int eqlin_mlp_forward(const eqlin_mlp* m, const void* x, void* y, int64_t N, void* stream) {
+    if (!m) return fail(EQLIN_ERR_INVALID_ARG, "handle is NULL");
+    if (N < 0) return fail(EQLIN_ERR_INVALID_ARG, "N < 0");
+    if (N == 0) return EQLIN_OK;
+    if (!x || !y) return fail(EQLIN_ERR_INVALID_ARG, "x or y is NULL");
+    if (N >= (int64_t(1) << 31)) return fail(EQLIN_ERR_UNSUPPORTED, "N must be below 2^31");
+    if (!aligned(x, 16) || !aligned(y, 16)) return fail(EQLIN_ERR_MISALIGNED, "x and y must be 16-byte aligned");
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev != m->device) return fail(EQLIN_ERR_INVALID_ARG, "current device differs from the handle's device");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int s = launch_mlp(m->plan, m->Cin, m->H, m->Cout, m->G, m->sm_count, x, y, N, m->b1, m->b2, m->timeout_ns, st);
+    if (s != EQLIN_OK) return s;
+    if (m->sync_check) {
+        int dst = 0;
+        if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return cuda_fail(e, "MLP forward (EQLIN_SYNC_CHECK)");
+        if ((e = cudaMemcpy(&dst, m->b1.status, sizeof(int), cudaMemcpyDeviceToHost)) != cudaSuccess)
+            return cuda_fail(e, "status read");
+        if (dst != 0) return fail(dst, "device reported an error (status word)");
+    }
+    return EQLIN_OK;
+}
+
+int eqlin_mlp_device_status(eqlin_mlp* m, int* status_out) {
+    if (!m || !status_out) return fail(EQLIN_ERR_INVALID_ARG, "NULL argument");
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    int v = 0;
+    if ((e = cudaMemcpy(&v, m->b1.status, sizeof(int), cudaMemcpyDeviceToHost)) != cudaSuccess)
+        return cuda_fail(e, "status read");
+    if ((e = cudaMemset(m->b1.status, 0, sizeof(int))) != cudaSuccess) return cuda_fail(e, "status clear");
+    *status_out = v;
+    return EQLIN_OK;
+}
+
+int eqlin_mlp_destroy(eqlin_mlp* m) {
+    if (!m) return EQLIN_OK;
+    free_mlp(m);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFree");
+    return EQLIN_OK;
+}
+
+}  // extern "C"

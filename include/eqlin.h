@@ -354,6 +354,55 @@ EQLIN_API int eqlin_backward_dw_workspace_size(const eqlin_handle* h, int64_t N,
 EQLIN_API int eqlin_backward_dw(const eqlin_handle* h, const void* x, const void* dy, float* dw, float* dbias,
                                 int64_t N, void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * The equivariant MLP block y = L2(GELU(L1(x))) in ONE fused launch.  Page "Flash
+ * EQ-Linear: ...", section "A Nivel de Red": the network-level gains come from networks
+ * built of EQ-Linear layers; section "Implementacion": the Fourier fragments stay on chip
+ * between the steps.  Here the hidden activation [N, H, G] never reaches global memory:
+ * per token tile the kernel transforms x once, and for each 128-channel chunk of the hidden
+ * layer runs the layer-1 contraction (tensor cores), bias, GELU (erf form, as
+ * EQLIN_PREPARE_GELU) and the group DFT of the result in registers, then accumulates the
+ * layer-2 contraction; the output epilogue adds b2 and writes y.  GELU acts pointwise in
+ * the group domain, so the block is equivariant.
+ *
+ * eqlin_mlp_prepare -- transform both weight sets once per weight update.
+ *   w1, b1   device, [H, Cin, G] and [H] (b1 may be NULL) of w_dtype.
+ *   w2, b2   device, [Cout, H, G] and [Cout] (b2 may be NULL) of w_dtype.
+ *   Cin, H, Cout, G   block sizes; the same "Supported" rules as one layer for each
+ *            layer ([H x Cin] and [Cout x H]), and further, for 16-bit I/O, Cout <= 128
+ *            (one output chunk) and Cin small enough that the input spectrum of a token
+ *            tile stays in shared memory (Cin <= 256, less for large G; UNSUPPORTED
+ *            otherwise).  For fp32 I/O: 8 * G * (Cin + H) doubles of shared memory.
+ *   w_dtype, io_dtype, stream   as eqlin_prepare_weights (the call synchronises stream).
+ *   out      host; receives the handle (NULL on failure).
+ * The handle owns the two transformed weight sets, fp32 copies of the biases and a
+ * device status word.  Errors: as eqlin_prepare_weights.
+ *
+ * eqlin_mlp_forward -- y [N, Cout, G] = L2(GELU(L1(x [N, Cin, G]))), one launch,
+ * asynchronous on `stream`, allocates nothing.  x and y: device, io_dtype, 16-byte aligned,
+ * not overlapping.  16-bit I/O: tcgen05 tensor cores with fp32 accumulation; the hidden
+ * spectrum is rounded to the I/O type for the second contraction (the two-launch block
+ * rounds the hidden activation instead).  fp32 I/O: float64 throughout, y rounded once.
+ * N == 0 is a no-op; N < 2^31.  Errors: as eqlin_forward; kernel wait timeouts go to the
+ * handle's device status word (eqlin_mlp_device_status).
+ *
+ * eqlin_mlp_query -- host only: EQLIN_OK if the fused block supports these sizes (and then
+ * the weight-ring depth and the dynamic shared memory of its kernel on a B200), else the
+ * status eqlin_mlp_prepare would return.  stages and smem_bytes may be NULL.
+ */
+typedef struct eqlin_mlp eqlin_mlp; /* opaque */
+
+EQLIN_API int eqlin_mlp_prepare(const void* w1, const void* b1, const void* w2, const void* b2, int64_t Cin,
+                                int64_t H, int64_t Cout, int64_t G, int w_dtype, int io_dtype, void* stream,
+                                eqlin_mlp** out);
+EQLIN_API int eqlin_mlp_forward(const eqlin_mlp* m, const void* x, void* y, int64_t N, void* stream);
+/* Reads and clears the block's device status word (synchronises the device). */
+EQLIN_API int eqlin_mlp_device_status(eqlin_mlp* m, int* status_out);
+/* Frees the handle's device memory; no forward using it may still be in flight.  NULL is a no-op. */
+EQLIN_API int eqlin_mlp_destroy(eqlin_mlp* m);
+EQLIN_API int eqlin_mlp_query(int64_t Cin, int64_t H, int64_t Cout, int64_t G, int io_dtype, int64_t* stages,
+                              int64_t* smem_bytes);
+
 /* Static description of a status code ("ok", "invalid argument", ...). */
 EQLIN_API const char* eqlin_status_string(int status);
 

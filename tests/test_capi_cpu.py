@@ -234,3 +234,23 @@ def test_planner_over_random_shapes():
         assert q["dw_tile_rows"] > 0 and q["dw_tile_cols"] > 0 and q["dw_raw_stages"] >= 2, (Cout, Cin, G, q)
         checked += 1
     assert checked > 250
+
+
+def test_fused_mlp_block_planner():
+    """eqlin_mlp_query (host only): the fused MLP block's supported sizes and its ring."""
+    for Cin, H, Cout, G in [(96, 384, 96, 4), (64, 256, 64, 8), (32, 128, 32, 16), (48, 80, 24, 2), (256, 64, 16, 2)]:
+        for io in (torch.bfloat16, torch.float16):
+            q = eq.eqlin_mlp_query(Cin, H, Cout, G, io)
+            assert q is not None and 2 <= q["stages"] <= 12 and q["smem_bytes"] <= 232448, (Cin, H, Cout, G, q)
+        assert eq.eqlin_mlp_query(Cin, H, Cout, G, torch.float32) is not None
+    # one output chunk only; the input spectrum of a tile must stay in shared memory
+    assert eq.eqlin_mlp_query(96, 384, 136, 4) is None
+    assert eq.eqlin_mlp_query(288, 64, 64, 4) is None
+    assert eq.eqlin_mlp_query(256, 64, 64, 16) is None
+    # the single-layer shape rules apply to both layers
+    assert eq.eqlin_mlp_query(96, 382, 96, 4) is not None       # H*G = 1528, a multiple of 8
+    assert eq.eqlin_mlp_query(96, 381, 96, 2) is None           # H*G = 762 is not
+    assert eq.eqlin_mlp_query(96, 384, 96, 3) is None
+    # fp32: 8 tokens' spectra of the input and the hidden layer in shared memory
+    assert eq.eqlin_mlp_query(96, 384, 96, 4, torch.float32) is not None
+    assert eq.eqlin_mlp_query(512, 4096, 96, 4, torch.float32) is None

@@ -97,3 +97,124 @@ def test_mlp_block_rejects_mismatched_handles():
         eq.mlp_block(h1, h1, x.to(DEV))             # 384 outputs into a 96-input layer
     for h in (plain, h2, h1):
         h.close()
+
+
+# ----------------------------------------------------------------------------------
+# The block as ONE fused launch (eqlin_mlp_prepare / eqlin_mlp_forward): the hidden
+# activation never leaves the SM.  For 16-bit I/O the hidden SPECTRUM is rounded to the
+# I/O type for the second contraction (instead of the hidden activation), so the same
+# doubled per-layer bound applies; for fp32 I/O the block runs in float64 throughout and
+# rounds y once, so the 1e-5 elementwise bound holds against the all-float64 oracle.
+
+FUSED_SHAPES = [(96, 384, 96, 4), (64, 256, 64, 8), (32, 128, 32, 16), (48, 80, 24, 2), (40, 200, 50, 4),
+                (96, 384, 128, 4), (256, 64, 16, 2), (24, 40, 8, 16)]
+
+
+def _fused_check(io, got, ref):
+    if io == torch.float32:
+        e = f32_maxrel(got, ref)
+        return e, e <= 1e-5
+    bound = 2 * (F16_DERIVED if io == torch.float16 else BF16_DERIVED)
+    e = normwise(got, ref)
+    return e, e <= min(bound, TOL_BF16_NORMWISE)
+
+
+@pytest.mark.parametrize("io", [torch.bfloat16, torch.float16, torch.float32])
+@pytest.mark.parametrize("Cin,H,Cout,G", FUSED_SHAPES)
+def test_fused_mlp_block(Cin, H, Cout, G, io):
+    x, w1, b1, w2, b2 = _block(1031, Cin, H, Cout, G, io, Cin * 7 + H + G + 1)
+    m = eq.eqlin_mlp_prepare(w1.to(DEV), b1.to(DEV), w2.to(DEV), b2.to(DEV))
+    y = m.forward(x.to(DEV))
+    torch.cuda.synchronize()
+    assert m.device_status() == eq.EQLIN_OK
+    e, ok = _fused_check(io, y.float().cpu().numpy(), oracle.mlp_forward(x, w1, b1, w2, b2))
+    assert ok, e
+    m.close()
+
+
+@pytest.mark.parametrize("io", [torch.bfloat16, torch.float32])
+def test_fused_mlp_block_no_bias_and_ragged_n(io):
+    x, w1, _, w2, _ = _block(300, 96, 384, 96, 4, io, 11)
+    m = eq.eqlin_mlp_prepare(w1.to(DEV), None, w2.to(DEV), None)
+    for N in (1, 2, 63, 64, 65, 129, 300):
+        y = m.forward(x[:N].contiguous().to(DEV))
+        torch.cuda.synchronize()
+        e, ok = _fused_check(io, y.float().cpu().numpy(), oracle.mlp_forward(x[:N], w1, None, w2, None))
+        assert ok, (N, e)
+    assert m.forward(x[:0].contiguous().to(DEV)).shape == (0, 96, 4)
+    m.close()
+
+
+@pytest.mark.parametrize("Cin,H,Cout,G", [(96, 384, 96, 4), (64, 256, 64, 8), (32, 128, 32, 16)])
+def test_fused_mlp_block_many_waves_sampled(Cin, H, Cout, G):
+    """Several persistent waves (every CTA loops over tiles), checked on sampled tokens."""
+    from cyclic_group_dft_b200 import workloads
+    io = torch.bfloat16
+    N = 3 * 148 * (256 // G) + 77
+    x, w1, b1, w2, b2 = _block(N, Cin, H, Cout, G, io, 23 + G)
+    m = eq.eqlin_mlp_prepare(w1.to(DEV), b1.to(DEV), w2.to(DEV), b2.to(DEV))
+    y = m.forward(x.to(DEV)).float().cpu()
+    torch.cuda.synchronize()
+    assert m.device_status() == eq.EQLIN_OK
+    idx = workloads.sample_tokens(N, 600, seed=G)
+    e, ok = _fused_check(io, y[idx].numpy(), oracle.mlp_forward(x[idx], w1, b1, w2, b2))
+    assert ok, e
+    y2 = m.forward(x.to(DEV)).float().cpu()
+    assert torch.equal(y, y2)   # deterministic
+    m.close()
+
+
+def test_fused_mlp_block_is_equivariant_on_gpu():
+    x, w1, b1, w2, b2 = _block(512, 96, 384, 96, 4, torch.float32, 5)
+    m = eq.eqlin_mlp_prepare(w1.to(DEV), b1.to(DEV), w2.to(DEV), b2.to(DEV))
+    y = m.forward(x.to(DEV)).cpu().double().numpy()
+    for s in range(4):
+        ys = m.forward(torch.roll(x, s, dims=-1).to(DEV)).cpu().double().numpy()
+        assert np.abs(ys - np.roll(y, s, axis=-1)).max() <= 1e-5 * np.abs(y).max()
+    m.close()
+
+
+def test_fused_mlp_block_rejects_what_it_does_not_support():
+    x, w1, b1, w2, b2 = _block(16, 96, 384, 200, 4, torch.bfloat16, 6)
+    assert eq.eqlin_mlp_query(96, 384, 200, 4) is None             # Cout > 128: two launches instead
+    with pytest.raises(eq.EqlinError) as e:
+        eq.eqlin_mlp_prepare(w1.to(DEV), b1.to(DEV), w2.to(DEV), b2.to(DEV))
+    assert e.value.status == eq.EQLIN_ERR_UNSUPPORTED
+    x, w1, b1, w2, b2 = _block(16, 96, 384, 96, 4, torch.bfloat16, 6)
+    m = eq.eqlin_mlp_prepare(w1.to(DEV), b1.to(DEV), w2.to(DEV), b2.to(DEV))
+    xd = x.to(DEV)
+    lib = eq.library()
+    y = torch.empty(16, 96, 4, dtype=torch.bfloat16, device=DEV)
+    stream = torch.cuda.current_stream().cuda_stream
+    assert lib.eqlin_mlp_forward(m.ptr, xd.data_ptr() + 2, y.data_ptr(), 15, stream) == eq.EQLIN_ERR_MISALIGNED
+    assert lib.eqlin_mlp_forward(m.ptr, xd.data_ptr(), y.data_ptr(), -1, stream) == eq.EQLIN_ERR_INVALID_ARG
+    with pytest.raises(ValueError):
+        m.forward(x.float().to(DEV))
+    m.close()
+
+
+def test_fused_mlp_block_timeout_is_reported(monkeypatch):
+    """The producer stops after 3 input chunks (test hook): the consumers' bounded waits
+    run out, the kernel returns with EQLIN_ERR_TIMEOUT in the status word, and the next
+    block computes correctly."""
+    N = 4 * 148 * 64
+    x, w1, b1, w2, b2 = _block(N, 96, 384, 96, 4, torch.bfloat16, 8)
+    monkeypatch.setenv("EQLIN_WAIT_TIMEOUT_MS", "200")
+    monkeypatch.setenv("EQLIN_TEST_STOP_AFTER", "3")
+    m = eq.eqlin_mlp_prepare(w1.to(DEV), b1.to(DEV), w2.to(DEV), b2.to(DEV))
+    xd = x.to(DEV)
+    m.forward(xd)
+    torch.cuda.synchronize()
+    assert m.device_status() == eq.EQLIN_ERR_TIMEOUT
+    assert m.device_status() == eq.EQLIN_OK
+    m.close()
+    monkeypatch.delenv("EQLIN_TEST_STOP_AFTER")
+    m = eq.eqlin_mlp_prepare(w1.to(DEV), b1.to(DEV), w2.to(DEV), b2.to(DEV))
+    y = m.forward(xd).float().cpu()
+    torch.cuda.synchronize()
+    assert m.device_status() == eq.EQLIN_OK
+    from cyclic_group_dft_b200 import workloads
+    idx = workloads.sample_tokens(N, 256, seed=4)
+    e, ok = _fused_check(torch.bfloat16, y[idx].numpy(), oracle.mlp_forward(x[idx], w1, b1, w2, b2))
+    assert ok, e
+    m.close()
