@@ -60,3 +60,29 @@ def test_oracle_rate_reports_its_threads():
     wl = workloads.WORKLOADS["tiny_p4_fp32"]
     rate, n, dt, threads = b.oracle_rate(wl, 0.05, threads=1)
     assert threads == 1 and 64 <= n <= wl.N and rate > 0 and dt > 0
+
+
+def test_reference_arm_maps_no_cuda_library():
+    """bench.py --impl reference times the float64 oracle only: importing the bench, the
+    seeded input generators and the oracle maps the oracle's library, never libeqlin.so."""
+    import subprocess
+    code = ("import sys; sys.argv = ['bench.py']; sys.path.insert(0, %r); import bench, oracle; "
+            "from cyclic_group_dft_b200 import workloads; "
+            "x, w, b = workloads.make_inputs(workloads.WORKLOADS['tiny_p4_fp32'], N=8); "
+            "oracle.forward(x, w, b); maps = open('/proc/self/maps').read(); "
+            "print(int('libeqlin.so' in maps), int('eqlin_oracle' in maps))") % ROOT
+    out = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr
+    assert out.stdout.split()[-2:] == ["0", "1"], out.stdout
+
+
+def test_both_arms_share_the_config():
+    """The GPU line and the reference line carry the same `config` (line_config)."""
+    b = _bench()
+    from cyclic_group_dft_b200 import workloads
+    wl = workloads.WORKLOADS["p4_c96_bf16"]
+    c = b.line_config(wl, 1)
+    assert c == b.line_config(wl, 1)
+    assert set(c) == {"workload", "N", "Cin", "Cout", "G", "io", "global_batch", "parallelism", "l2"}
+    assert c["N"] == 64 * 56 * 56 and c["workload"] == "p4_c96_bf16"
+    assert b.BENCH_WORKLOADS == ("tiny_p4_fp32", "p4_c96_bf16", "p8_c64_bf16", "p4_mlp_bf16", "c16_c32_bf16")
