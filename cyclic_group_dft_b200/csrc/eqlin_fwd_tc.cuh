@@ -74,6 +74,9 @@ struct TcParams {
     // i it asks the TMA unit to bring item i + pf into L2, so more of x is in flight than
     // the shared-memory ring holds.  0 = off.
     int pf;
+    // 1: copies carry L2 eviction priorities: the weights (re-read by every CTA) evict
+    // last, x and y (streamed once) evict first.  0: plain copies.
+    int l2hint;
 };
 
 namespace tc {
@@ -248,6 +251,7 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, const CUtensorM
     const uint32_t lane_addr = acc + (static_cast<uint32_t>(q * 32) << 16);
     const int t0 = half * (S::BN / 2);
     const int col = lane * G;                               // first staged column of this lane
+    const uint64_t pol_y = p.l2hint ? ptx::l2_policy_evict_first() : 0ull;
     uint8_t* lane_off0 = wstage + (col / YBC) * BOX_BYTES + (col % YBC) * 2;
 #pragma unroll 1
     for (int j = 0; j < S::BN / 2 / TG; ++j) {
@@ -347,7 +351,8 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, const CUtensorM
                 for (int bx = 0; bx < NYB; ++bx) {
                     const int o_first = oc * kMmaM + q * 32 + bx * (YBC / G);
                     if (o_first < p.Cout)
-                        ptx::tma_store_2d(tmap_y, src + bx * BOX_BYTES, o_first * G, static_cast<int>(row));
+                        ptx::tma_store_2d_h(tmap_y, src + bx * BOX_BYTES, o_first * G, static_cast<int>(row),
+                                            p.l2hint != 0, pol_y);
                 }
             }
             ptx::bulk_commit_group();
@@ -416,12 +421,14 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem_base = ctl->tmem_base;
+    const bool hint = p.l2hint != 0;
+    const uint64_t pol_w = hint ? ptx::l2_policy_evict_last() : 0ull, pol_x = hint ? ptx::l2_policy_evict_first() : 0ull;
     // resident weights: one bulk copy per 32 KB, completing on bar_w_full
     auto load_weights = [&]() {
         ptx::mbar_arrive_expect_tx(bar_w_full, p.w_img_bytes);
         for (uint32_t off = 0; off < p.w_img_bytes; off += 32768u) {
             const uint32_t n = min(32768u, p.w_img_bytes - off);
-            ptx::bulk_load(s_w + off, p.w_img + off, n, bar_w_full);
+            ptx::bulk_load_h(s_w + off, p.w_img + off, n, bar_w_full, hint, pol_w);
         }
     };
     // weights that no kernel of the stream writes are staged while the previous kernel drains
@@ -473,13 +480,13 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                     ptx::mbar_arrive_expect_tx(bar_full(stage), STAGE_TX);
 #pragma unroll
                     for (int bx = 0; bx < S::NBOX; ++bx) {
-                        ptx::tma_load_2d(dst + bx * (S::BN * S::BOX_ELEMS * 2), &tmap_x,
-                                         c * S::XROW_ELEMS + bx * S::BOX_ELEMS, n0, bar_full(stage));
+                        ptx::tma_load_2d_h(dst + bx * (S::BN * S::BOX_ELEMS * 2), &tmap_x,
+                                           c * S::XROW_ELEMS + bx * S::BOX_ELEMS, n0, bar_full(stage), hint, pol_x);
                     }
                     if constexpr (STREAM_W) {
-                        ptx::bulk_load(dst + S::SPEC_BYTES,
-                                       p.w_img + static_cast<size_t>(oc * p.nK + c) * S::WSTAGE_BYTES,
-                                       S::WSTAGE_BYTES, bar_full(stage));
+                        ptx::bulk_load_h(dst + S::SPEC_BYTES,
+                                         p.w_img + static_cast<size_t>(oc * p.nK + c) * S::WSTAGE_BYTES,
+                                         S::WSTAGE_BYTES, bar_full(stage), hint, pol_w);
                     }
                     ++issued;
                     if (++stage == NS) { stage = 0; phase ^= 1u; }

@@ -93,6 +93,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem_base = ctl->tmem_base;
+    const bool hint = p.l2hint != 0;
+    const uint64_t pol_w = hint ? ptx::l2_policy_evict_last() : 0ull, pol_x = hint ? ptx::l2_policy_evict_first() : 0ull;
     // Weights that no kernel of the stream writes (p.w_early): the first ring stages are
     // filled with the first tile's weight chunks while the previous kernel drains.  The
     // ring order is the same as below, which then skips issuing those chunks.
@@ -101,8 +103,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         const int pre = min(NS, p.n_oc * nK);
         for (int j = 0; j < pre; ++j) {
             ptx::mbar_arrive_expect_tx(bar_w_full(j), S::WSTAGE_BYTES);
-            ptx::bulk_load(s_wring0 + j * S::WSTAGE_BYTES, p.w_img + static_cast<size_t>(j) * S::WSTAGE_BYTES,
-                           S::WSTAGE_BYTES, bar_w_full(j));
+            ptx::bulk_load_h(s_wring0 + j * S::WSTAGE_BYTES, p.w_img + static_cast<size_t>(j) * S::WSTAGE_BYTES,
+                             S::WSTAGE_BYTES, bar_w_full(j), hint, pol_w);
         }
         w_prefilled = pre;
     }
@@ -149,8 +151,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                     ptx::mbar_arrive_expect_tx(bar_x_full(c), S::XCHUNK_BYTES);
 #pragma unroll
                     for (int bx = 0; bx < S::NBOX; ++bx)
-                        ptx::tma_load_2d(dst + bx * (S::BN * S::BOX_ELEMS * 2), &tmap_x,
-                                         c * S::XROW_ELEMS + bx * S::BOX_ELEMS, n0, bar_x_full(c));
+                        ptx::tma_load_2d_h(dst + bx * (S::BN * S::BOX_ELEMS * 2), &tmap_x,
+                                           c * S::XROW_ELEMS + bx * S::BOX_ELEMS, n0, bar_x_full(c), hint, pol_x);
                     ++issued_x;
                     ++last_tile_chunks;
                 }
@@ -168,9 +170,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                             break;
                         }
                         ptx::mbar_arrive_expect_tx(bar_w_full(ws), S::WSTAGE_BYTES);
-                        ptx::bulk_load(s_wring0 + ws * S::WSTAGE_BYTES,
+                        ptx::bulk_load_h(s_wring0 + ws * S::WSTAGE_BYTES,
                                        p.w_img + static_cast<size_t>(oc * nK + c) * S::WSTAGE_BYTES,
-                                       S::WSTAGE_BYTES, bar_w_full(ws));
+                                       S::WSTAGE_BYTES, bar_w_full(ws), hint, pol_w);
                         ++issued_w;
                         if (++ws == NS) { ws = 0; wph ^= 1u; }
                     }

@@ -56,6 +56,7 @@ struct TmParams {
     int act;                // epilogue activation after the bias: kActNone or kActGelu
     int w_early;            // weights may be loaded before griddepcontrol.wait (TcParams::w_early)
     int pf;                 // L2 prefetch distance in work items (TcParams::pf), 0 = off
+    int l2hint;             // L2 eviction priorities on the copies (TcParams::l2hint)
 };
 
 namespace tm {
@@ -183,6 +184,7 @@ __device__ __forceinline__ void epilogue_tile(const TmParams& p, const CUtensorM
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const long long row0 = n0 + q * 32;            // first token of this warp's rows
     const int swz = (lane >> 1) & 3;               // SWIZZLE_64B of the staging rows
+    const uint64_t pol_y = p.l2hint ? ptx::l2_policy_evict_first() : 0ull;
 #pragma unroll 1
     for (int g = 0; g < n_groups; ++g) {
         const int o_loc0 = half * (p.NO / 2) + g * OG;
@@ -234,7 +236,7 @@ __device__ __forceinline__ void epilogue_tile(const TmParams& p, const CUtensorM
         if (lane == 0) {
             // a store only starts inside the tensor; its clipped parts are not written
             if (row0 < p.N && o0 < p.Cout)
-                ptx::tma_store_2d(tmap_y, ptx::smem_u32(buf), o0 * G, static_cast<int>(row0));
+                ptx::tma_store_2d_h(tmap_y, ptx::smem_u32(buf), o0 * G, static_cast<int>(row0), p.l2hint != 0, pol_y);
             ptx::bulk_commit_group();
         }
         ybuf ^= 1;
@@ -297,10 +299,12 @@ __global__ void __launch_bounds__(tm::Cfg<G>::kThreads, 1)
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem_base = ctl->tmem_base;
+    const bool hint = p.l2hint != 0;
+    const uint64_t pol_w = hint ? ptx::l2_policy_evict_last() : 0ull, pol_x = hint ? ptx::l2_policy_evict_first() : 0ull;
     auto load_weights = [&]() {
         ptx::mbar_arrive_expect_tx(bar_w_full, p.w_img_bytes);
         for (uint32_t off = 0; off < p.w_img_bytes; off += 32768u)
-            ptx::bulk_load(s_w + off, p.w_img + off, min(32768u, p.w_img_bytes - off), bar_w_full);
+            ptx::bulk_load_h(s_w + off, p.w_img + off, min(32768u, p.w_img_bytes - off), bar_w_full, hint, pol_w);
     };
     // weights that no kernel of the stream writes are staged while the previous kernel drains
     if constexpr (!STREAM_W) {
@@ -351,12 +355,12 @@ __global__ void __launch_bounds__(tm::Cfg<G>::kThreads, 1)
                     ptx::mbar_arrive_expect_tx(bar_full(stage), stage_bytes);
 #pragma unroll
                     for (int bx = 0; bx < C::X_NBOX; ++bx)
-                        ptx::tma_load_2d(dst + bx * C::X_BOX_BYTES, &tmap_x, c * C::XROW_ELEMS + bx * C::X_BOX, n0,
-                                         bar_full(stage));
+                        ptx::tma_load_2d_h(dst + bx * C::X_BOX_BYTES, &tmap_x, c * C::XROW_ELEMS + bx * C::X_BOX, n0,
+                                           bar_full(stage), hint, pol_x);
                     if constexpr (STREAM_W) {
-                        ptx::bulk_load(dst + C::XCHUNK_BYTES,
-                                       p.w_img + static_cast<size_t>(oc * p.nK + c) * wstage_bytes, wstage_bytes,
-                                       bar_full(stage));
+                        ptx::bulk_load_h(dst + C::XCHUNK_BYTES,
+                                         p.w_img + static_cast<size_t>(oc * p.nK + c) * wstage_bytes, wstage_bytes,
+                                         bar_full(stage), hint, pol_w);
                     }
                     ++issued;
                     if (++stage == NS) { stage = 0; phase ^= 1u; }

@@ -154,6 +154,16 @@ void* kernel_for(const Plan& pl, int G) {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// L2 eviction priorities on the fused kernels' copies (weights evict last, x and y evict
+// first).  EQLIN_L2HINT=0 turns them off.
+bool l2_hint() {
+    static const bool on = [] {
+        const char* e = std::getenv("EQLIN_L2HINT");
+        return e && *e ? e[0] != '0' : kDefaultL2Hint;
+    }();
+    return on;
+}
+
 // L2 prefetch distance of the fused kernels' producer, in work items of the CTA.
 // EQLIN_PREFETCH=k overrides (0 turns the prefetch off).
 int prefetch_distance() {
@@ -303,6 +313,7 @@ int launch_forward(const Plan& pl, int64_t Cout, int64_t Cin, int64_t G, int sm_
             p.inject_stop = b.inject_stop;
             p.w_early = b.w_early ? 1 : 0;
             p.pf = prefetch_distance();
+            p.l2hint = l2_hint() ? 1 : 0;
             const TmEntry entry = tm_entry_for(iG, pl.streamed(), pl.io);
             if (!entry.launch) return fail(EQLIN_ERR_UNSUPPORTED, "G");
             entry.launch(grid, pl.smem_bytes, st, map, ymap, p);
@@ -328,6 +339,7 @@ int launch_forward(const Plan& pl, int64_t Cout, int64_t Cin, int64_t G, int sm_
             p.inject_stop = b.inject_stop;
             p.w_early = b.w_early ? 1 : 0;
             p.pf = prefetch_distance();
+            p.l2hint = l2_hint() ? 1 : 0;
             const TcEntry entry = pl.tnr() ? tcr_entry_for(iG, pl.io) : tc_entry_for(iG, pl.streamed(), pl.nacc, pl.io);
             if (!entry.launch) return fail(EQLIN_ERR_UNSUPPORTED, "G");
             entry.launch(grid, pl.smem_bytes, st, map, ymap, p);

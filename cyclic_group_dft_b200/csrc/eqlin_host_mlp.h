@@ -165,6 +165,7 @@ int launch_mlp(const MlpPlan& pl, int64_t Cin, int64_t H, int64_t Cout, int64_t 
         p.inject_stop = b1.inject_stop;
         p.w_early = (b1.w_early && b2.w_early) ? 1 : 0;
         p.pf = prefetch_distance();
+        p.l2hint = l2_hint() ? 1 : 0;
         const unsigned grid = static_cast<unsigned>(std::min<long long>(p.n_tiles, sm_count));
         const bool f16 = pl.io == EQLIN_F16;
         switch (iG) {

@@ -14,7 +14,11 @@ constexpr size_t kSmemCtlBytes = 512;       // mbarriers + control block
 constexpr int kMaxStages = 12;
 constexpr int64_t kMaxChannels = 1 << 16;
 constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per bounded wait
-constexpr int kDefaultPrefetch = 2;   // L2 prefetch distance of the fused kernels (work items)
+// L2 prefetch distance of the fused kernels (work items).  Off: on B200 every workload was
+// slower with it (200 back-to-back launches, distance 2 / 0: p4 C96 63.1 / 62.1 us, p8 C64
+// 24.2 / 22.8, p4 192->768 189.6 / 181.5, C16 C32 153.4 / 145.6).
+constexpr int kDefaultPrefetch = 0;
+constexpr bool kDefaultL2Hint = true;   // L2 eviction priorities on the fused kernels' copies
 
 // Kernel variants (EQLIN_ATTR_PATH):
 //   0/1  tcgen05, tokens on the MMA N dimension, weights resident / streamed

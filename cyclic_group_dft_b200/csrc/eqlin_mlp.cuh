@@ -26,11 +26,13 @@
 // Roles per CTA (one per SM, persistent over token tiles):
 //   warp 12     producer: x chunks of a tile (TMA) into resident slots, weight units into
 //               the ring (bulk copies)
-//   warps 8-11  DFT of each x chunk in place (tc::dft_chunk)
+//   warps 8-11  DFT of each x chunk in place (tc::dft_chunk), then a third of each hidden
+//               chunk's epilogue with the epilogue warps
 //   warp 13     MMA issuer + TMEM owner.  Per tile: for each hidden chunk hc, the layer-1
 //               products into acc1, then (once the epilogue has written H^ of hc-1) the
 //               layer-2 products of hc-1 into acc2
-//   warps 0-7   epilogue: hidden chunks (acc1 -> H^) and, per tile, the output (acc2 -> y)
+//   warps 0-7   epilogue: two thirds of each hidden chunk (acc1 -> H^) and, per tile, the
+//               output (acc2 -> y)
 // Waits are bounded as in eqlin_fwd_tc.cuh.
 #pragma once
 
@@ -64,6 +66,7 @@ struct MlpParams {
     long long inject_stop;   // test hook: x chunks issued per CTA before the producer stops; -1 = never
     int w_early;             // weights may be loaded before griddepcontrol.wait (TcParams::w_early)
     int pf;                  // L2 prefetch distance of x, in tiles of this CTA (0 = off)
+    int l2hint;              // L2 eviction priorities on the copies (TcParams::l2hint)
 };
 
 namespace mlp {
@@ -78,8 +81,13 @@ struct Cfg {
     using S = tc::Shape<G, 2>;
     static constexpr int kUnits = G / 2;               // weight units per 32-channel chunk
     static constexpr int TGM = 32 / G;                 // tokens per TMEM load of a hidden chunk
-    static constexpr int NGR = (S::BN / 2) / TGM;      // such groups per epilogue warp and chunk
-    static_assert(TGM % 2 == 0 && (S::BN / 2) % TGM == 0, "hidden epilogue groups");
+    static constexpr int NGR = S::BN / TGM;            // such groups per token tile (8)
+    // The hidden epilogue runs on 12 warps, 3 per TMEM lane quarter: the 8 epilogue warps
+    // and the 4 DFT warps (which transform x once per tile and are free otherwise).  Warp
+    // part j in {0, 1, 2} of a quarter takes groups j, j + 3, j + 6.
+    static constexpr int kParts = 3;
+    static constexpr int kHiddenThreads = 4 * kParts * 32;
+    static_assert(TGM % 2 == 0 && S::BN % TGM == 0, "hidden epilogue groups");
 };
 
 // Weight unit u of a 32-channel chunk: planes 0 and 1 (the real frequencies 0 and G/2)
@@ -105,14 +113,14 @@ __device__ __forceinline__ void issue_unit(int u, uint32_t d_base, uint32_t a_lo
     }
 }
 
-// Epilogue of one hidden chunk, warp (q, half): hidden rows 32q .. 32q+31 of the chunk
-// (TMEM lane quarter q, one row per lane), tokens [half*BN/2, (half+1)*BN/2).  Per pair
-// of tokens (packed as fx2): irDFT of the G planes + b1, GELU, rDFT, and the G spectrum
-// values written as the pair slots of H^ into K32 chunk q of `hbuf` (lane = K column, one
-// 2-byte store per token and slot: a warp fills one 64-byte row).  Arrives on
+// Epilogue of one hidden chunk, warp (q, part): hidden rows 32q .. 32q+31 of the chunk
+// (TMEM lane quarter q, one row per lane), token groups part, part + 3, ... of TGM tokens.
+// Per pair of tokens (packed as fx2): irDFT of the G planes + b1, GELU, rDFT, and the G
+// spectrum values written as the pair slots of H^ into K32 chunk q of `hbuf` (lane = K
+// column, one 2-byte store per token and slot: a warp fills one 64-byte row).  Arrives on
 // `acc1_empty` once its last TMEM load has landed.
 template <int G, class T16>
-__device__ __forceinline__ void hidden_chunk(const MlpParams& p, uint32_t acc1, int q, int half, int lane, int hc,
+__device__ __forceinline__ void hidden_chunk(const MlpParams& p, uint32_t acc1, int q, int part, int lane, int hc,
                                              uint8_t* hbuf, uint32_t acc1_empty) {
     using C = Cfg<G>;
     using S = typename C::S;
@@ -121,18 +129,17 @@ __device__ __forceinline__ void hidden_chunk(const MlpParams& p, uint32_t acc1, 
     const bool chunk_used = hc * kHK + q < p.nK2;               // layer 2 reads this K32 chunk
     const float b = (p.b1 != nullptr && j < p.H) ? p.b1[j] : 0.0f;
     const uint32_t lane_addr = acc1 + (static_cast<uint32_t>(q * 32) << 16);
-    const int t0 = half * (S::BN / 2);
     uint8_t* hsub = hbuf + static_cast<size_t>(q) * S::SPEC_BYTES;
     const int piece = lane >> 3, in_piece = (lane & 7) * 2;
 #pragma unroll 1
-    for (int g = 0; g < C::NGR; ++g) {
+    for (int g = part; g < C::NGR; g += C::kParts) {
         uint32_t r[G][TGM];
 #pragma unroll
-        for (int pl = 0; pl < G; ++pl) ptx::tmem_ld_32x32b<TGM>(lane_addr + pl * S::BN + t0 + g * TGM, r[pl]);
+        for (int pl = 0; pl < G; ++pl) ptx::tmem_ld_32x32b<TGM>(lane_addr + pl * S::BN + g * TGM, r[pl]);
         ptx::tmem_wait_ld();
 #pragma unroll
         for (int pl = 0; pl < G; ++pl) ptx::tmem_regs_ready<TGM>(r[pl]);
-        if (g == C::NGR - 1) {
+        if (g + C::kParts >= C::NGR) {
             ptx::tc_fence_before();
             ptx::mbar_arrive(acc1_empty);   // acc1 no longer needed by this thread
         }
@@ -148,7 +155,7 @@ __device__ __forceinline__ void hidden_chunk(const MlpParams& p, uint32_t acc1, 
             for (int gg = 0; gg < G; ++gg) hv[gg] = gelu2(hv[gg]);
             rdft_planes<G>(hv, sp);
             // rows tt (even) and tt + 1 share the SWIZZLE_64B piece permutation
-            const int tt = t0 + g * TGM + t;
+            const int tt = g * TGM + t;
             uint8_t* row = hsub + tt * kPlaneRowBytes + ((piece ^ ((tt >> 1) & 3)) << 4) + in_piece;
             auto put = [&](int slot, uint32_t w) {
                 uint8_t* d = row + slot * S::PLANE_BYTES;
@@ -217,8 +224,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
             ptx::mbar_init(bar_w_empty(s), 1);
         }
         ptx::mbar_init(bar_acc1_full, 1);
-        ptx::mbar_init(bar_acc1_empty, tc::kEpiThreads);
-        ptx::mbar_init(bar_h_full, tc::kEpiThreads);
+        ptx::mbar_init(bar_acc1_empty, C::kHiddenThreads);
+        ptx::mbar_init(bar_h_full, C::kHiddenThreads);
         ptx::mbar_init(bar_h_empty, 1);
         ptx::mbar_init(bar_acc2_full, 1);
         ptx::mbar_init(bar_acc2_empty, tc::kEpiThreads);
@@ -237,6 +244,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     ptx::tc_fence_after();
     const uint32_t tmem_base = ctl->tmem_base;
     const uint32_t acc1 = tmem_base, acc2 = tmem_base + static_cast<uint32_t>(S::ACC_COLS);
+    const bool hint = p.l2hint != 0;
+    const uint64_t pol_w = hint ? ptx::l2_policy_evict_last() : 0ull, pol_x = hint ? ptx::l2_policy_evict_first() : 0ull;
 
     // source of weight unit i (0 <= i < units_per_tile) of a tile, and its bytes
     auto unit_src = [&](int i, uint32_t* bytes) -> const uint8_t* {
@@ -271,7 +280,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
             uint32_t bytes;
             const uint8_t* src = unit_src(j, &bytes);
             ptx::mbar_arrive_expect_tx(bar_w_full(j), bytes);
-            ptx::bulk_load(s_wring0 + j * mlp::kUnitBytes, src, bytes, bar_w_full(j));
+            ptx::bulk_load_h(s_wring0 + j * mlp::kUnitBytes, src, bytes, bar_w_full(j), hint, pol_w);
         }
         w_prefilled = pre;
     }
@@ -314,8 +323,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                     ptx::mbar_arrive_expect_tx(bar_x_full(c), S::XCHUNK_BYTES);
 #pragma unroll
                     for (int bx = 0; bx < S::NBOX; ++bx)
-                        ptx::tma_load_2d(dst + bx * (S::BN * S::BOX_ELEMS * 2), &tmap_x,
-                                         c * S::XROW_ELEMS + bx * S::BOX_ELEMS, n0, bar_x_full(c));
+                        ptx::tma_load_2d_h(dst + bx * (S::BN * S::BOX_ELEMS * 2), &tmap_x,
+                                           c * S::XROW_ELEMS + bx * S::BOX_ELEMS, n0, bar_x_full(c), hint, pol_x);
                     ++issued_x;
                     ++last_tile_chunks;
                 }
@@ -334,7 +343,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                     uint32_t bytes;
                     const uint8_t* src = unit_src(i, &bytes);
                     ptx::mbar_arrive_expect_tx(bar_w_full(ws), bytes);
-                    ptx::bulk_load(s_wring0 + ws * mlp::kUnitBytes, src, bytes, bar_w_full(ws));
+                    ptx::bulk_load_h(s_wring0 + ws * mlp::kUnitBytes, src, bytes, bar_w_full(ws), hint, pol_w);
                     ++issued_w;
                     if (++ws == NS) { ws = 0; wph ^= 1u; }
                 }
@@ -437,10 +446,12 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         }
     } else if (warp >= tc::kWarpDft0) {
         // ------------------------------------------------------------ DFT warps
+        // per tile: the x chunks' DFT, then their part of each hidden chunk's epilogue
         const int dft_tid = threadIdx.x - tc::kWarpDft0 * 32;
+        long long uc = 0;
+        bool ok = true;
         int ti = 0;
-        for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++ti) {
-            bool ok = true;
+        for (int tile = blockIdx.x; ok && tile < p.n_tiles; tile += gridDim.x, ++ti) {
             for (int c = 0; c < nK1; ++c) {
                 const bool got = tc::wait_bounded(bar_x_full(c), static_cast<uint32_t>(ti) & 1u, ctl, p.status,
                                                   p.timeout_ns);
@@ -452,7 +463,19 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                 ptx::fence_proxy_async_smem();
                 ptx::mbar_arrive(bar_xhat(c));
             }
-            if (!ok) break;
+            for (int hc = 0; ok && hc < p.n_hc; ++hc, ++uc) {
+                bool got = tc::wait_bounded(bar_acc1_full, static_cast<uint32_t>(uc & 1), ctl, p.status, p.timeout_ns);
+                got = got && tc::wait_bounded(bar_h_empty, static_cast<uint32_t>(uc & 1) ^ 1u, ctl, p.status,
+                                              p.timeout_ns);
+                if (!ptx::named_bar_and(tc::kBarDft, 128, got)) {
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+                mlp::hidden_chunk<G, T16>(p, acc1, warp & 3, 2, lane, hc, hbuf, bar_acc1_empty);
+                ptx::fence_proxy_async_smem();   // H^ visible to the tensor cores
+                ptx::mbar_arrive(bar_h_full);
+            }
         }
     } else {
         // ------------------------------------------------------------ epilogue warps
@@ -478,7 +501,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                     break;
                 }
                 ptx::tc_fence_after();
-                mlp::hidden_chunk<G, T16>(p, acc1, q, half, lane, hc, hbuf, bar_acc1_empty);
+                mlp::hidden_chunk<G, T16>(p, acc1, q, half, lane, hc, hbuf, bar_acc1_empty);   // parts 0, 1
                 ptx::fence_proxy_async_smem();   // H^ visible to the tensor cores
                 ptx::mbar_arrive(bar_h_full);
             }

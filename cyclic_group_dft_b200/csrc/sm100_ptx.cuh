@@ -119,6 +119,35 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, uint32_t src,
                  "r"(c0), "r"(c1), "r"(src)
                  : "memory");
 }
+// L2 eviction-priority policies for the cache-hinted copies below: data read again soon
+// (weights shared by every CTA) is kept in L2 before data streamed once (x, y).
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+// tma_load_2d with an L2 cache policy
+__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap* m, int32_t c0, int32_t c1,
+                                                 uint32_t bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(bar), "l"(policy)
+        : "memory");
+}
+// tma_store_2d with an L2 cache policy
+__device__ __forceinline__ void tma_store_2d_hint(const CUtensorMap* m, uint32_t src, int32_t c0, int32_t c1,
+                                                  uint64_t policy) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%1, %2}], [%3], %4;" ::"l"(
+                     reinterpret_cast<uint64_t>(m)),
+                 "r"(c0), "r"(c1), "r"(src), "l"(policy)
+                 : "memory");
+}
 // Hint: bring the 2-D box at (c0, c1) of the tensor into L2 (no shared memory, no
 // completion to wait for; parts of the box outside the tensor are not fetched).
 __device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* m, int32_t c0, int32_t c1) {
@@ -148,6 +177,31 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
             "r"(dst),
         "l"(src), "r"(bytes), "r"(bar)
         : "memory");
+}
+// bulk_load with an L2 cache policy
+__device__ __forceinline__ void bulk_load_hint(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar,
+                                               uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::
+            "r"(dst),
+        "l"(src), "r"(bytes), "r"(bar), "l"(policy)
+        : "memory");
+}
+// The copies above with an optional L2 policy (hint == false: the plain form).
+__device__ __forceinline__ void bulk_load_h(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar, bool hint,
+                                            uint64_t policy) {
+    if (hint) bulk_load_hint(dst, src, bytes, bar, policy);
+    else bulk_load(dst, src, bytes, bar);
+}
+__device__ __forceinline__ void tma_load_2d_h(uint32_t dst, const CUtensorMap* m, int32_t c0, int32_t c1, uint32_t bar,
+                                              bool hint, uint64_t policy) {
+    if (hint) tma_load_2d_hint(dst, m, c0, c1, bar, policy);
+    else tma_load_2d(dst, m, c0, c1, bar);
+}
+__device__ __forceinline__ void tma_store_2d_h(const CUtensorMap* m, uint32_t src, int32_t c0, int32_t c1, bool hint,
+                                               uint64_t policy) {
+    if (hint) tma_store_2d_hint(m, src, c0, c1, policy);
+    else tma_store_2d(m, src, c0, c1);
 }
 // Make this thread's generic-proxy shared-memory writes visible to the async proxy
 // (tensor-core operand reads, later TMA writes).
