@@ -117,9 +117,9 @@ def kernel_source_hash(kernel: str) -> str:
 
 def recorded_traffic(workload: str) -> dict | None:
     """DRAM reads plus L2 write bytes per launch from a committed ncu capture, if the
-    kernel is unchanged since.  Reads are counted at DRAM; writes are counted as they
-    enter L2 (every byte of y the kernel stores), because part of y is still dirty in
-    L2 when the kernel ends and its DRAM write-back falls outside the kernel."""
+    kernel is unchanged since.  Reads are counted at DRAM; writes are the sectors the SMs
+    write into L2 (every byte the kernel stores), because part of y is still dirty in L2
+    when the kernel ends and its DRAM write-back falls outside the kernel."""
     try:
         with open(TRAFFIC_FILE) as f:
             d = json.load(f)
@@ -307,7 +307,8 @@ def roofline(wl: workloads.Workload, N: int, avg_launch_s: float, peaks: dict, p
         roof["traffic_detail"] = {"dram_read": tr["dram_read"], "l2_write": tr["l2_write"],
                                   "over_algorithmic": tr["bytes"] / bytes_launch, "kernel": tr["kernel"],
                                   "source": "ncu capture (profiles/eqlin_fwd_traffic.json): dram__bytes_read.sum "
-                                            "+ 32 * lts__t_sectors_op_write.sum, scaled to a full launch"}
+                                            "+ 32 * lts__t_sectors_srcunit_tex_op_write.sum (bytes the SMs "
+                                            "write into L2), scaled to a full launch by tokens"}
     roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback"
     roof["roofline_time_us"] = 1e6 * max(t_hbm, t_tc)
     roof["kernel_us"] = 1e6 * avg_launch_s
