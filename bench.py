@@ -356,7 +356,7 @@ def run_reference(args, wl) -> None:
 
 # ------------------------------------------------------------------ GPU arm
 class Ctx:
-    def __init__(self, eq, dev, world, stream, peaks, peak_kind, graph=True):
+    def __init__(self, eq, dev, world, stream, peaks, peak_kind, graph=False):
         self.eq, self.dev, self.world, self.stream = eq, dev, world, stream
         self.peaks, self.peak_kind = peaks, peak_kind
         self.graph = graph
@@ -435,34 +435,7 @@ def measure_workload(ctx: Ctx, wl: workloads.Workload, K: int, warmup: int, head
     if h.device_status() != eq.EQLIN_OK:
         raise RuntimeError(f"{wl.name}: device status not OK after warm-up")
 
-    # ------------------------------------------------------- timed region
-    # K back-to-back steps, one fused launch each, bracketed by two events on the
-    # launching stream.  No event sits between the launches: an event there would end
-    # the overlap of one launch's tail with the next one's prologue (programmatic
-    # dependent launch), which is how the kernel runs in a real stream of layers.
-    # The average launch duration of the kernel is therefore elapsed / K.
-    clocks = ClockSampler(dev.index) if headline else None
-    elapsed_ms = time_back_to_back(ctx, fwd, K, clocks, graph=ctx.graph)
-    status = h.device_status()
-    avg_launch_s = elapsed_ms / K / 1e3
-    # the same K launches issued one by one from the host (no graph), for comparison
-    stream_ms = time_back_to_back(ctx, fwd, K, graph=False) if ctx.graph else elapsed_ms
-    out = {"N": N, "Cin": wl.Cin, "Cout": wl.Cout, "G": wl.G, "io": wl.io_dtype,
-           "kernel": {"path": h.path, "stages": h.attr("stages"), "tokens_per_tile": h.attr("tokens_per_tile")},
-           "steps": K, "elapsed_ms": elapsed_ms, "us_per_launch": 1e3 * elapsed_ms / K,
-           "timing": "one CUDA-graph replay of the K launches" if ctx.graph else "K launches from the host",
-           "us_per_launch_host_launches": 1e3 * stream_ms / K,
-           "tokens_per_s": aggregate_tokens_per_s(ctx.world, K, N, elapsed_ms),
-           "roofline": roofline(wl, N, avg_launch_s, ctx.peaks, ctx.peak_kind),
-           "dense_equivalent_tflops": dense_equivalent_flops(wl, N) / avg_launch_s / 1e12,
-           "device_status": status}
-    if algorithmic_bytes(wl, N) / (ctx.peaks["hbm_gbs"] * 1e9) < 2e-6:
-        out["roofline"]["note"] = ("launch-bound: the roofline time is below the ~2 us cost of one kernel "
-                                   "launch, so the fraction measures launch latency, not the kernel's "
-                                   "arithmetic or memory traffic")
-    if clocks is not None:
-        out["clocks"] = clocks.summary()
-
+    out = {}
     # Launch-duration distribution, outside the timed region: an event pair around
     # each launch (which serialises the launches, so each one also pays its own
     # prologue and tail).
@@ -479,22 +452,8 @@ def measure_workload(ctx: Ctx, wl: workloads.Workload, K: int, warmup: int, head
                         "min": 1e3 * min(launch_ms), "max": 1e3 * max(launch_ms), "launches": len(launch_ms),
                         "note": "each launch bracketed by its own events (serialised), outside the timed region"}
 
-    # ------------------------------------------------------- end to end (headline)
-    if headline and args.e2e_steps > 0:
-        E = args.e2e_steps
-        x_pin = x_cpu.pin_memory()
-        y_pin = torch.empty(N, wl.Cout, wl.G, dtype=wl.torch_dtype).pin_memory()
-        h.forward_host(x_pin, y_pin)  # warm the path
-        e2e_ms = time_back_to_back(ctx, lambda i, st: h.forward_host(x_pin, y_pin, stream=st), E, graph=False)
-        out["e2e"] = {"value": aggregate_tokens_per_s(ctx.world, E, N, e2e_ms), "unit": "tokens/s", "steps": E,
-                      "h2d_bytes_per_step": x_pin.numel() * x_pin.element_size(),
-                      "d2h_bytes_per_step": y_pin.numel() * y_pin.element_size(),
-                      "api": "eqlin_forward_host (C ABI: pinned host x and y, chunked copies in and out "
-                             "overlapping the fused kernel on two streams)"}
-        del x_pin, y_pin
-
     # ------------------------------------------------------- backward calls
-    # Measured after the forward's timed region, on the same rotating buffer sets (the
+    # Measured before the forward's timed region, on the same rotating buffer sets (the
     # forward outputs stand in for dy): us per call from CUDA events around Kb
     # back-to-back calls, against the same roofline model as the forward.
     if backward:
@@ -537,6 +496,51 @@ def measure_workload(ctx: Ctx, wl: workloads.Workload, K: int, warmup: int, head
     # through HBM) is timed beside it for comparison.
     if not args.no_mlp_block and wl.io_dtype != "f32" and wl.Cin == wl.Cout:
         out["mlp_block"] = measure_mlp_block(ctx, wl, xs, ys, n_sets, K, warmup)
+
+    # ------------------------------------------------------- timed region
+    # Last, after the workload's other measurements have kept the GPU busy, W warm-up
+    # launches and then K back-to-back steps, one fused launch each, bracketed by two events on the
+    # launching stream.  No event sits between the launches: an event there would end
+    # the overlap of one launch's tail with the next one's prologue (programmatic
+    # dependent launch), which is how the kernel runs in a real stream of layers.
+    # The average launch duration of the kernel is therefore elapsed / K.
+    for i in range(warmup):
+        fwd(i)
+    clocks = ClockSampler(dev.index) if headline else None
+    elapsed_ms = time_back_to_back(ctx, fwd, K, clocks, graph=ctx.graph)
+    status = h.device_status()
+    avg_launch_s = elapsed_ms / K / 1e3
+    # with --graph, the same K launches issued one by one from the host, for comparison
+    stream_ms = time_back_to_back(ctx, fwd, K, graph=False) if ctx.graph else elapsed_ms
+    out.update({"N": N, "Cin": wl.Cin, "Cout": wl.Cout, "G": wl.G, "io": wl.io_dtype,
+           "kernel": {"path": h.path, "stages": h.attr("stages"), "tokens_per_tile": h.attr("tokens_per_tile")},
+           "steps": K, "elapsed_ms": elapsed_ms, "us_per_launch": 1e3 * elapsed_ms / K,
+           "timing": "one CUDA-graph replay of the K launches" if ctx.graph else "K launches from the host",
+           "us_per_launch_host_launches": 1e3 * stream_ms / K,
+           "tokens_per_s": aggregate_tokens_per_s(ctx.world, K, N, elapsed_ms),
+           "roofline": roofline(wl, N, avg_launch_s, ctx.peaks, ctx.peak_kind),
+           "dense_equivalent_tflops": dense_equivalent_flops(wl, N) / avg_launch_s / 1e12,
+           "device_status": status})
+    if algorithmic_bytes(wl, N) / (ctx.peaks["hbm_gbs"] * 1e9) < 2e-6:
+        out["roofline"]["note"] = ("launch-bound: the roofline time is below the ~2 us cost of one kernel "
+                                   "launch, so the fraction measures launch latency, not the kernel's "
+                                   "arithmetic or memory traffic")
+    if clocks is not None:
+        out["clocks"] = clocks.summary()
+
+    # ------------------------------------------------------- end to end (headline)
+    if headline and args.e2e_steps > 0:
+        E = args.e2e_steps
+        x_pin = x_cpu.pin_memory()
+        y_pin = torch.empty(N, wl.Cout, wl.G, dtype=wl.torch_dtype).pin_memory()
+        h.forward_host(x_pin, y_pin)  # warm the path
+        e2e_ms = time_back_to_back(ctx, lambda i, st: h.forward_host(x_pin, y_pin, stream=st), E, graph=False)
+        out["e2e"] = {"value": aggregate_tokens_per_s(ctx.world, E, N, e2e_ms), "unit": "tokens/s", "steps": E,
+                      "h2d_bytes_per_step": x_pin.numel() * x_pin.element_size(),
+                      "d2h_bytes_per_step": y_pin.numel() * y_pin.element_size(),
+                      "api": "eqlin_forward_host (C ABI: pinned host x and y, chunked copies in and out "
+                             "overlapping the fused kernel on two streams)"}
+        del x_pin, y_pin
 
     h.close()
     del xs, ys
@@ -601,8 +605,9 @@ def main() -> None:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", action="store_true",
                     help="measure only --workload (no workloads object)")
-    ap.add_argument("--no-graph", action="store_true",
-                    help="time launches issued one by one from the host instead of a CUDA-graph replay")
+    ap.add_argument("--graph", action="store_true",
+                    help="time one CUDA-graph replay of the K launches instead of K launches from the host "
+                         "(the graph is replayed once, untimed, to upload it)")
     ap.add_argument("--no-mlp-block", action="store_true",
                     help="skip the extra measurement of the equivariant MLP block L2(GELU(L1(x))), H = 4 C")
     ap.add_argument("--no-backward", action="store_true",
@@ -632,7 +637,7 @@ def main() -> None:
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     peaks, peak_kind = load_peaks()
-    ctx = Ctx(eq, dev, world, torch.cuda.current_stream(dev), peaks, peak_kind, graph=not args.no_graph)
+    ctx = Ctx(eq, dev, world, torch.cuda.current_stream(dev), peaks, peak_kind, graph=args.graph)
 
     # every other workload first (each step count at least 100 launches: their launches
     # are short), the headline last with exactly --steps timed launches
