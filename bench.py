@@ -15,7 +15,7 @@ The same line carries a ``workloads`` object with every synthetic workload
 (tiny p4 fp32, p4 C96, p8 C64, p4 MLP 192->768, C16 C32), each measured in this run
 the same way: us per launch over back-to-back launches, tokens/s, roofline,
 dense-equivalent TFLOP/s, the backward calls, and the oracle on a bounded sample of
-that workload.  The other workloads run first, the headline last.
+that workload.  The headline runs first, then the other workloads.
 
 Multi-GPU (torchrun): every rank runs the full workload on its own GPU (tokens
 are independent, no collective on the data path): weak scaling; the timed
@@ -417,9 +417,9 @@ def setup_workload(ctx: Ctx, wl: workloads.Workload, args) -> dict:
 
 def measure_workload(ctx: Ctx, wl: workloads.Workload, K: int, warmup: int, headline: bool, args,
                      setup: dict | None = None) -> dict:
-    """One workload: K back-to-back forward launches (timed), a per-launch pass, the
-    backward calls, the MLP block, and (headline only) the end-to-end host-buffer figure
-    and the clocks of the timed region."""
+    """One workload: K back-to-back forward launches (timed, first), a per-launch pass,
+    (headline only) the end-to-end host-buffer figure and the clocks of the timed region,
+    then the backward calls and the MLP block."""
     eq, dev, stream = ctx.eq, ctx.dev, ctx.stream
     su = setup if setup is not None else setup_workload(ctx, wl, args)
     x_cpu, h, xs, ys, n_sets = su["x_cpu"], su["h"], su["xs"], su["ys"], su["n_sets"]
@@ -449,6 +449,40 @@ def measure_workload(ctx: Ctx, wl: workloads.Workload, K: int, warmup: int, head
         raise RuntimeError(f"{wl.name}: device status not OK after warm-up")
 
     out = {}
+    # ------------------------------------------------------- timed region
+    # First, on a GPU that this process has not yet loaded for seconds (a long load makes
+    # the same launches a few percent slower): W warm-up launches and then K back-to-back
+    # steps, one fused launch each, bracketed by two events on the
+    # launching stream.  No event sits between the launches: an event there would end
+    # the overlap of one launch's tail with the next one's prologue (programmatic
+    # dependent launch), which is how the kernel runs in a real stream of layers.
+    # The average launch duration of the kernel is therefore elapsed / K.
+    for i in range(warmup):
+        fwd(i)
+    clocks = ClockSampler(dev.index) if headline else None
+    elapsed_ms = time_back_to_back(ctx, fwd_c, K, clocks, graph=ctx.graph)
+    if any(rc != eq.EQLIN_OK for rc in rcs):
+        raise RuntimeError(f"{wl.name}: eqlin_forward returned {sorted(set(rcs))}")
+    status = h.device_status()
+    avg_launch_s = elapsed_ms / K / 1e3
+    # with --graph, the same K launches issued one by one from the host, for comparison
+    stream_ms = time_back_to_back(ctx, fwd_c, K, graph=False) if ctx.graph else elapsed_ms
+    out.update({"N": N, "Cin": wl.Cin, "Cout": wl.Cout, "G": wl.G, "io": wl.io_dtype,
+           "kernel": {"path": h.path, "stages": h.attr("stages"), "tokens_per_tile": h.attr("tokens_per_tile")},
+           "steps": K, "elapsed_ms": elapsed_ms, "us_per_launch": 1e3 * elapsed_ms / K,
+           "timing": "one CUDA-graph replay of the K launches" if ctx.graph else "K launches from the host",
+           "us_per_launch_host_launches": 1e3 * stream_ms / K,
+           "tokens_per_s": aggregate_tokens_per_s(ctx.world, K, N, elapsed_ms),
+           "roofline": roofline(wl, N, avg_launch_s, ctx.peaks, ctx.peak_kind),
+           "dense_equivalent_tflops": dense_equivalent_flops(wl, N) / avg_launch_s / 1e12,
+           "device_status": status})
+    if algorithmic_bytes(wl, N) / (ctx.peaks["hbm_gbs"] * 1e9) < 2e-6:
+        out["roofline"]["note"] = ("launch-bound: the roofline time is below the ~2 us cost of one kernel "
+                                   "launch, so the fraction measures launch latency, not the kernel's "
+                                   "arithmetic or memory traffic")
+    if clocks is not None:
+        out["clocks"] = clocks.summary()
+
     # Launch-duration distribution, outside the timed region: an event pair around
     # each launch (which serialises the launches, so each one also pays its own
     # prologue and tail).
@@ -465,8 +499,22 @@ def measure_workload(ctx: Ctx, wl: workloads.Workload, K: int, warmup: int, head
                         "min": 1e3 * min(launch_ms), "max": 1e3 * max(launch_ms), "launches": len(launch_ms),
                         "note": "each launch bracketed by its own events (serialised), outside the timed region"}
 
+    # ------------------------------------------------------- end to end (headline)
+    if headline and args.e2e_steps > 0:
+        E = args.e2e_steps
+        x_pin = x_cpu.pin_memory()
+        y_pin = torch.empty(N, wl.Cout, wl.G, dtype=wl.torch_dtype).pin_memory()
+        h.forward_host(x_pin, y_pin)  # warm the path
+        e2e_ms = time_back_to_back(ctx, lambda i, st: h.forward_host(x_pin, y_pin, stream=st), E, graph=False)
+        out["e2e"] = {"value": aggregate_tokens_per_s(ctx.world, E, N, e2e_ms), "unit": "tokens/s", "steps": E,
+                      "h2d_bytes_per_step": x_pin.numel() * x_pin.element_size(),
+                      "d2h_bytes_per_step": y_pin.numel() * y_pin.element_size(),
+                      "api": "eqlin_forward_host (C ABI: pinned host x and y, chunked copies in and out "
+                             "overlapping the fused kernel on two streams)"}
+        del x_pin, y_pin
+
     # ------------------------------------------------------- backward calls
-    # Measured before the forward's timed region, on the same rotating buffer sets (the
+    # Measured after the forward's timed region, on the same rotating buffer sets (the
     # forward outputs stand in for dy): us per call from CUDA events around Kb
     # back-to-back calls, against the same roofline model as the forward.
     if backward:
@@ -509,53 +557,6 @@ def measure_workload(ctx: Ctx, wl: workloads.Workload, K: int, warmup: int, head
     # through HBM) is timed beside it for comparison.
     if not args.no_mlp_block and wl.io_dtype != "f32" and wl.Cin == wl.Cout:
         out["mlp_block"] = measure_mlp_block(ctx, wl, xs, ys, n_sets, K, warmup)
-
-    # ------------------------------------------------------- timed region
-    # Last, after the workload's other measurements have kept the GPU busy, W warm-up
-    # launches and then K back-to-back steps, one fused launch each, bracketed by two events on the
-    # launching stream.  No event sits between the launches: an event there would end
-    # the overlap of one launch's tail with the next one's prologue (programmatic
-    # dependent launch), which is how the kernel runs in a real stream of layers.
-    # The average launch duration of the kernel is therefore elapsed / K.
-    for i in range(warmup):
-        fwd(i)
-    clocks = ClockSampler(dev.index) if headline else None
-    elapsed_ms = time_back_to_back(ctx, fwd_c, K, clocks, graph=ctx.graph)
-    if any(rc != eq.EQLIN_OK for rc in rcs):
-        raise RuntimeError(f"{wl.name}: eqlin_forward returned {sorted(set(rcs))}")
-    status = h.device_status()
-    avg_launch_s = elapsed_ms / K / 1e3
-    # with --graph, the same K launches issued one by one from the host, for comparison
-    stream_ms = time_back_to_back(ctx, fwd_c, K, graph=False) if ctx.graph else elapsed_ms
-    out.update({"N": N, "Cin": wl.Cin, "Cout": wl.Cout, "G": wl.G, "io": wl.io_dtype,
-           "kernel": {"path": h.path, "stages": h.attr("stages"), "tokens_per_tile": h.attr("tokens_per_tile")},
-           "steps": K, "elapsed_ms": elapsed_ms, "us_per_launch": 1e3 * elapsed_ms / K,
-           "timing": "one CUDA-graph replay of the K launches" if ctx.graph else "K launches from the host",
-           "us_per_launch_host_launches": 1e3 * stream_ms / K,
-           "tokens_per_s": aggregate_tokens_per_s(ctx.world, K, N, elapsed_ms),
-           "roofline": roofline(wl, N, avg_launch_s, ctx.peaks, ctx.peak_kind),
-           "dense_equivalent_tflops": dense_equivalent_flops(wl, N) / avg_launch_s / 1e12,
-           "device_status": status})
-    if algorithmic_bytes(wl, N) / (ctx.peaks["hbm_gbs"] * 1e9) < 2e-6:
-        out["roofline"]["note"] = ("launch-bound: the roofline time is below the ~2 us cost of one kernel "
-                                   "launch, so the fraction measures launch latency, not the kernel's "
-                                   "arithmetic or memory traffic")
-    if clocks is not None:
-        out["clocks"] = clocks.summary()
-
-    # ------------------------------------------------------- end to end (headline)
-    if headline and args.e2e_steps > 0:
-        E = args.e2e_steps
-        x_pin = x_cpu.pin_memory()
-        y_pin = torch.empty(N, wl.Cout, wl.G, dtype=wl.torch_dtype).pin_memory()
-        h.forward_host(x_pin, y_pin)  # warm the path
-        e2e_ms = time_back_to_back(ctx, lambda i, st: h.forward_host(x_pin, y_pin, stream=st), E, graph=False)
-        out["e2e"] = {"value": aggregate_tokens_per_s(ctx.world, E, N, e2e_ms), "unit": "tokens/s", "steps": E,
-                      "h2d_bytes_per_step": x_pin.numel() * x_pin.element_size(),
-                      "d2h_bytes_per_step": y_pin.numel() * y_pin.element_size(),
-                      "api": "eqlin_forward_host (C ABI: pinned host x and y, chunked copies in and out "
-                             "overlapping the fused kernel on two streams)"}
-        del x_pin, y_pin
 
     h.close()
     del xs, ys
@@ -656,9 +657,9 @@ def main() -> None:
 
     # every other workload first (each step count at least 100 launches: their launches
     # are short), the headline last with exactly --steps timed launches
-    # the headline's inputs and handle are ready before the other workloads run, so its
-    # warm-up and timed launches follow them with no idle gap on the GPU
-    head_setup = setup_workload(ctx, wl, args)
+    # the headline first, then every other workload (each step count at least 100 launches:
+    # their launches are short)
+    head = measure_workload(ctx, wl, args.steps, args.warmup, True, args)
     results = {}
     if not args.only:
         for name in BENCH_WORKLOADS:
@@ -666,7 +667,6 @@ def main() -> None:
                 continue
             results[name] = measure_workload(ctx, workloads.WORKLOADS[name], max(args.steps, 100), args.warmup,
                                              False, args)
-    head = measure_workload(ctx, wl, args.steps, args.warmup, True, args, setup=head_setup)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

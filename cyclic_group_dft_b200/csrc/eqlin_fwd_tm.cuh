@@ -169,77 +169,90 @@ __device__ __forceinline__ void dft_chunk(uint8_t* xs, int dft_tid) {
 // ------------------------------------------------------------ epilogue role
 // Warp (q, half): tokens 32q..32q+31 (TMEM lane quarter q), output channels
 // [half*NO/2, (half+1)*NO/2) of the work item, in groups of OG = 32/G channels.
-// Per group: tcgen05.ld of the G planes, inverse real DFT + bias (channel pairs packed
-// as fx2), bf16, one 64-byte row per lane into the warp's own SWIZZLE_64B staging tile
-// [32 tokens x 32 columns] (double-buffered), and lane 0 stores it with TMA; the
-// epilogue warps never wait for one another.  Arrives on `acc_empty` once its last TMEM
-// load has landed.
+// TMEM is read in batches of EB groups (EB = 2 for G <= 8: G x 2*OG = 64 registers), so a
+// warp waits for half as many TMEM loads; the batch's biases are loaded before the wait.
+// Per group: inverse real DFT + bias (channel pairs packed as fx2), bf16, one 64-byte row
+// per lane into the warp's own SWIZZLE_64B staging tile [32 tokens x 32 columns]
+// (double-buffered), and lane 0 stores it with TMA; the epilogue warps never wait for one
+// another.  Arrives on `acc_empty` once its last TMEM load has landed.
 template <int G, class T16>
 __device__ __forceinline__ void epilogue_tile(const TmParams& p, const CUtensorMap* tmap_y, uint32_t tmem,
                                               int q, int half, int lane, long long n0, int oc, uint8_t* wstage,
                                               int& ybuf, uint32_t acc_empty) {
     using C = Cfg<G>;
     constexpr int OG = C::OG;
+    constexpr int EB = G <= 8 ? 2 : 1;             // groups per TMEM load batch
     const int n_groups = (p.NO / 2) / OG;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const long long row0 = n0 + q * 32;            // first token of this warp's rows
     const int swz = (lane >> 1) & 3;               // SWIZZLE_64B of the staging rows
     const uint64_t pol_y = p.l2hint ? ptx::l2_policy_evict_first() : 0ull;
 #pragma unroll 1
-    for (int g = 0; g < n_groups; ++g) {
-        const int o_loc0 = half * (p.NO / 2) + g * OG;
-        uint32_t r[G][OG];
+    for (int g0 = 0; g0 < n_groups; g0 += EB) {
+        const int o_loc0 = half * (p.NO / 2) + g0 * OG;
+        // biases of the batch's channels (0 past Cout or without bias), before the TMEM wait
+        float bv[EB * OG];
 #pragma unroll
-        for (int pl = 0; pl < G; ++pl) ptx::tmem_ld_32x32b<OG>(lane_addr + pl * p.NO + o_loc0, r[pl]);
+        for (int j = 0; j < EB * OG; ++j) {
+            const int o = oc * p.NO + o_loc0 + j;
+            bv[j] = (p.bias != nullptr && o < p.Cout) ? __ldg(p.bias + o) : 0.0f;
+        }
+        // a batch past the last group reads accumulator columns that are never used
+        // (inside the 512 allocated: (G-1)*NO + NO/2 + EB*OG <= 512 for every plan)
+        uint32_t r[G][EB * OG];
+#pragma unroll
+        for (int pl = 0; pl < G; ++pl) ptx::tmem_ld_32x32b<EB * OG>(lane_addr + pl * p.NO + o_loc0, r[pl]);
         ptx::tmem_wait_ld();
 #pragma unroll
-        for (int pl = 0; pl < G; ++pl) ptx::tmem_regs_ready<OG>(r[pl]);
-        if (g == n_groups - 1) {
+        for (int pl = 0; pl < G; ++pl) ptx::tmem_regs_ready<EB * OG>(r[pl]);
+        if (g0 + EB >= n_groups) {
             ptx::tc_fence_before();
             ptx::mbar_arrive(acc_empty);           // TMEM no longer needed by this thread
         }
-        const int o0 = oc * p.NO + o_loc0;
-        float yv[OG * G];
 #pragma unroll
-        for (int j = 0; j < OG; j += 2) {
-            fx2 z[G], y2[G];
+        for (int gi = 0; gi < EB; ++gi) {
+            if (g0 + gi >= n_groups) break;
+            const int o0 = oc * p.NO + o_loc0 + gi * OG;
+            // the lane's staging row: OG channels x G outputs, channel-major, packed in pairs
+            uint32_t pk[OG * G / 2];
 #pragma unroll
-            for (int pl = 0; pl < G; ++pl) z[pl] = fx2(__uint_as_float(r[pl][j]), __uint_as_float(r[pl][j + 1]));
-            const int o = o0 + j;
-            if (p.bias != nullptr) {
-                z[0] += fx2(o < p.Cout ? __ldg(p.bias + o) : 0.0f, o + 1 < p.Cout ? __ldg(p.bias + o + 1) : 0.0f);
+            for (int j = 0; j < OG; j += 2) {
+                fx2 z[G], y2[G];
+#pragma unroll
+                for (int pl = 0; pl < G; ++pl)
+                    z[pl] = fx2(__uint_as_float(r[pl][gi * OG + j]), __uint_as_float(r[pl][gi * OG + j + 1]));
+                z[0] += fx2(bv[gi * OG + j], bv[gi * OG + j + 1]);
+                RealIdft<G, fx2>::run(z, y2);
+                if (p.act == kActGelu) {
+#pragma unroll
+                    for (int gg = 0; gg < G; ++gg) y2[gg] = gelu2(y2[gg]);
+                }
+#pragma unroll
+                for (int gg = 0; gg < G; gg += 2) {
+                    pk[(j * G + gg) / 2] = Io16<T16>::pack(y2[gg].x, y2[gg + 1].x);
+                    pk[((j + 1) * G + gg) / 2] = Io16<T16>::pack(y2[gg].y, y2[gg + 1].y);
+                }
             }
-            RealIdft<G, fx2>::run(z, y2);
-            if (p.act == kActGelu) {
+            // this buffer was last stored two groups ago: its TMA read must be complete
+            if (lane == 0) ptx::bulk_wait_group_read<1>();
+            __syncwarp();
+            uint8_t* buf = wstage + static_cast<size_t>(ybuf) * kYWarpBufBytes;
+            uint8_t* rowp = buf + lane * (kYCols * 2);
 #pragma unroll
-                for (int gg = 0; gg < G; ++gg) y2[gg] = gelu2(y2[gg]);
+            for (int k = 0; k < 4; ++k)
+                *reinterpret_cast<uint4*>(rowp + ((k ^ swz) * 16)) =
+                    make_uint4(pk[4 * k + 0], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                // a store only starts inside the tensor; its clipped parts are not written
+                if (row0 < p.N && o0 < p.Cout)
+                    ptx::tma_store_2d_h(tmap_y, ptx::smem_u32(buf), o0 * G, static_cast<int>(row0), p.l2hint != 0,
+                                        pol_y);
+                ptx::bulk_commit_group();
             }
-#pragma unroll
-            for (int gg = 0; gg < G; ++gg) {
-                yv[j * G + gg] = y2[gg].x;
-                yv[(j + 1) * G + gg] = y2[gg].y;
-            }
+            ybuf ^= 1;
         }
-        // this buffer was last stored two groups ago: its TMA read must be complete
-        if (lane == 0) ptx::bulk_wait_group_read<1>();
-        __syncwarp();
-        uint8_t* buf = wstage + static_cast<size_t>(ybuf) * kYWarpBufBytes;
-        uint8_t* rowp = buf + lane * (kYCols * 2);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            *reinterpret_cast<uint4*>(rowp + ((k ^ swz) * 16)) =
-                make_uint4(Io16<T16>::pack(yv[8 * k + 0], yv[8 * k + 1]), Io16<T16>::pack(yv[8 * k + 2], yv[8 * k + 3]),
-                           Io16<T16>::pack(yv[8 * k + 4], yv[8 * k + 5]), Io16<T16>::pack(yv[8 * k + 6], yv[8 * k + 7]));
-        }
-        ptx::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-            // a store only starts inside the tensor; its clipped parts are not written
-            if (row0 < p.N && o0 < p.Cout)
-                ptx::tma_store_2d_h(tmap_y, ptx::smem_u32(buf), o0 * G, static_cast<int>(row0), p.l2hint != 0, pol_y);
-            ptx::bulk_commit_group();
-        }
-        ybuf ^= 1;
     }
 }
 
