@@ -643,8 +643,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
             if (q < p.yq && oc * kMmaM + q * 32 < p.Cout) {
                 const uint32_t acc = tmem_base + static_cast<uint32_t>(abuf * S::ACC_COLS);
                 const long long n0 = static_cast<long long>(tile) * S::BN;
-                if (p.ysub == 2)
-                    tc::epilogue_tile<G, NACC, T16, 2>(p, &tmap_y, acc, q, half, lane, n0, oc, wstage, ybuf);
+                // the two-piece form exists for G <= 4 only (the planner offers it there)
+                if (G <= 4 && p.ysub == 2)
+                    tc::epilogue_tile<G, NACC, T16, (G <= 4 ? 2 : 1)>(p, &tmap_y, acc, q, half, lane, n0, oc, wstage,
+                                                                     ybuf);
                 else
                     tc::epilogue_tile<G, NACC, T16, 1>(p, &tmap_y, acc, q, half, lane, n0, oc, wstage, ybuf);
             }

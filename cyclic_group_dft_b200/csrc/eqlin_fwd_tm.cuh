@@ -16,7 +16,10 @@
 // Roles per CTA (one per SM, persistent):
 //   producer warp    TMA loads of x chunks [128 tokens x 16 channels x G] (+ the weight
 //                    chunk when the weights are streamed) into a smem ring
-//   DW DFT warps     in-place real DFT over G: x chunk -> G planes, K-major SWIZZLE_32B
+//   DW DFT warps     in-place real DFT over G: x chunk -> G planes, K-major SWIZZLE_32B,
+//                    laid out so that each 8-row group of the spectrum replaces the same
+//                    rows of the input (tm::SpecLayout): a warp transforms whole groups
+//                    and orders only its own reads before its writes
 //   MMA warp         one thread issues tcgen05.mma: 2 real products, and 2 per complex
 //                    frequency, each over the Re and Im planes of D at once (N = 2*NO)
 //                    thanks to the weight image's [-Im, Re, Im] slots (eqlin_layout.h)
@@ -74,7 +77,7 @@ constexpr int kYStageBytes = kEpiWarps * kYWarpBufs * kYWarpBufBytes;   // 32 KB
 
 template <int G>
 struct Cfg {
-    static constexpr int DW = G == 16 ? 8 : 4;               // DFT warps
+    static constexpr int DW = 4;                              // DFT warps
     static constexpr int kDftThreads = DW * 32;
     static constexpr int kWarpDft0 = kEpiWarps;
     static constexpr int kWarpProducer = kEpiWarps + DW;
@@ -96,73 +99,116 @@ struct Cfg {
     static_assert(XCHUNK_BYTES % 1024 == 0, "stage alignment");
 };
 
+// Spectrum layout of a chunk (the MMA's A operand, K-major SWIZZLE_32B): plane p's
+// 8-row atoms (8 tokens x 16 channels, 256 B) sit SBO bytes apart, inside x box p / PPB
+// at byte (p % PPB) * 256 of each 8-row block of that box.  The x chunk lands as boxes of
+// [128 rows x BOX_ROW bytes], so rows 8g..8g+7 of every plane occupy exactly the bytes of
+// input rows 8g..8g+7: the transform of an 8-row group writes over its own input only.
+template <int G>
+struct SpecLayout {
+    static constexpr int BOX_ROW = Cfg<G>::X_BOX * 2;          // bytes of one x box row
+    static constexpr int PPB = BOX_ROW / kRowBytes32;          // planes per box
+    static constexpr int SBO = 8 * BOX_ROW;                    // bytes between 8-row atoms
+    static_assert(PPB * 256 == SBO && SBO % 16 == 0, "spectrum atoms tile the x boxes");
+    static constexpr uint32_t plane_offset(int p) {
+        return static_cast<uint32_t>((p / PPB) * Cfg<G>::X_BOX_BYTES + (p % PPB) * 256);
+    }
+};
+
+// The A-operand descriptor's constant half for SpecLayout<G> (SBO, version, SWIZZLE_32B).
+template <int G>
+constexpr uint32_t spec_desc_hi() {
+    return (static_cast<uint32_t>(SpecLayout<G>::SBO) >> 4) | (1u << 14) | (6u << 29);
+}
+
 // --------------------------------------------------------------- DFT role
-// Unit = one token row x two adjacent channels (2*G bf16).  Lane l: row offset l/8,
-// channel pair l%8; a warp covers 4 rows per step.
+// Unit = one token row x two adjacent channels (2*G 16-bit values).  Warp w transforms the
+// 8-row groups w, w + DW, ...; a group's 64 units are one warp's (two per lane), so a
+// __syncwarp between its reads and its in-place writes is the only ordering the
+// transform needs.  Lane mapping, chosen so that the 8 lanes of each 16-byte load pass
+// hit 8 different bank groups: with SWIZZLE_128B boxes (G >= 8) lane l takes row
+// 8g + l%8 and channel pairs l/8 and 4 + l/8 (one pair, eight rows per pass: eight
+// different swizzle slots); with unswizzled boxes it takes pair l%8 of rows 8g + l/8 and
+// 8g + 4 + l/8 (one row's contiguous units per pass).  The 32-bit spectrum stores are
+// conflict-free either way.
+template <int G>
+__device__ __forceinline__ int dft_row(int g, int s, int lane) {
+    return Cfg<G>::X_SW128 ? 8 * g + (lane & 7) : 8 * g + 4 * s + (lane >> 3);
+}
+template <int G>
+__device__ __forceinline__ int dft_pair(int s, int lane) {
+    return Cfg<G>::X_SW128 ? (lane >> 3) + 4 * s : (lane & 7);
+}
+
 template <int G, class T16>
 __device__ __forceinline__ void dft_chunk(uint8_t* xs, int dft_tid) {
     using C = Cfg<G>;
+    using L = SpecLayout<G>;
     constexpr int WORDS = G;
-    constexpr int ROWS_PER_STEP = C::kDftThreads / 8;
-    constexpr int STEPS = kM / ROWS_PER_STEP;
+    constexpr int GROUPS = kM / 8;
     const int warp = dft_tid >> 5, lane = dft_tid & 31;
-    const int pair = lane & 7;
-    const int row0 = warp * 4 + (lane >> 3);
-    const uint8_t* src0 = xs + pair * (4 * G);
-    uint32_t w[STEPS][WORDS];
+#pragma unroll 1
+    for (int g = warp; g < GROUPS; g += C::DW) {
+        uint32_t w[2][WORDS];
 #pragma unroll
-    for (int s = 0; s < STEPS; ++s) {
-        const uint8_t* src = src0 + (row0 + s * ROWS_PER_STEP) * (C::XROW_ELEMS * 2);
-        if constexpr (C::X_SW128) {
-            // 16-byte piece c of the unit: logical byte offset pair*4G + 16c in the row,
-            // box off/128, piece (off/16)%8 stored at piece ^ (row % 8)
-            const int r = row0 + s * ROWS_PER_STEP;
+        for (int s = 0; s < 2; ++s) {
+            const int r = dft_row<G>(g, s, lane);
+            const int pair = dft_pair<G>(s, lane);
+            if constexpr (C::X_SW128) {
+                // 16-byte piece c of the unit: logical byte offset pair*4G + 16c in the row,
+                // box off/128, piece (off/16)%8 stored at piece ^ (row % 8)
 #pragma unroll
-            for (int c = 0; c < WORDS / 4; ++c) {
-                const int off = pair * (4 * G) + 16 * c;
-                const uint8_t* q = xs + (off >> 7) * C::X_BOX_BYTES + r * 128 + ((((off >> 4) & 7) ^ (r & 7)) << 4);
-                const uint4 v = *reinterpret_cast<const uint4*>(q);
-                w[s][4 * c + 0] = v.x;
-                w[s][4 * c + 1] = v.y;
-                w[s][4 * c + 2] = v.z;
-                w[s][4 * c + 3] = v.w;
-            }
-        } else if constexpr (WORDS == 2) {
-            const uint2 v = *reinterpret_cast<const uint2*>(src);
-            w[s][0] = v.x;
-            w[s][1] = v.y;
-        } else {
+                for (int c = 0; c < WORDS / 4; ++c) {
+                    const int off = pair * (4 * G) + 16 * c;
+                    const uint8_t* q =
+                        xs + (off >> 7) * C::X_BOX_BYTES + r * 128 + ((((off >> 4) & 7) ^ (r & 7)) << 4);
+                    const uint4 v = *reinterpret_cast<const uint4*>(q);
+                    w[s][4 * c + 0] = v.x;
+                    w[s][4 * c + 1] = v.y;
+                    w[s][4 * c + 2] = v.z;
+                    w[s][4 * c + 3] = v.w;
+                }
+            } else {
+                const uint8_t* src = xs + r * L::BOX_ROW + pair * (4 * G);
+                if constexpr (WORDS == 2) {
+                    const uint2 v = *reinterpret_cast<const uint2*>(src);
+                    w[s][0] = v.x;
+                    w[s][1] = v.y;
+                } else {
 #pragma unroll
-            for (int c = 0; c < WORDS / 4; ++c) {
-                const uint4 v = *reinterpret_cast<const uint4*>(src + 16 * c);
-                w[s][4 * c + 0] = v.x;
-                w[s][4 * c + 1] = v.y;
-                w[s][4 * c + 2] = v.z;
-                w[s][4 * c + 3] = v.w;
+                    for (int c = 0; c < WORDS / 4; ++c) {
+                        const uint4 v = *reinterpret_cast<const uint4*>(src + 16 * c);
+                        w[s][4 * c + 0] = v.x;
+                        w[s][4 * c + 1] = v.y;
+                        w[s][4 * c + 2] = v.z;
+                        w[s][4 * c + 3] = v.w;
+                    }
+                }
             }
         }
-    }
-    ptx::named_bar_sync(kBarDft, C::kDftThreads);   // all reads before any in-place write
-    const int in_piece = (pair & 3) * 4;
+        __syncwarp();   // the group's reads before any of its in-place writes
 #pragma unroll
-    for (int s = 0; s < STEPS; ++s) {
-        const int r = row0 + s * ROWS_PER_STEP;
-        // the unit's two channels (a: words 0..G/2-1, b: words G/2..G-1) transformed as
-        // one packed pair
-        fx2 xab[G];
+        for (int s = 0; s < 2; ++s) {
+            const int r = dft_row<G>(g, s, lane);
+            const int pair = dft_pair<G>(s, lane);
+            const int in_piece = (pair & 3) * 4;
+            // the unit's two channels (a: words 0..G/2-1, b: words G/2..G-1) transformed as
+            // one packed pair
+            fx2 xab[G];
 #pragma unroll
-        for (int h = 0; h < G / 2; ++h) {
-            const uint32_t ua = w[s][h], ub = w[s][G / 2 + h];
-            xab[2 * h] = fx2(Io16<T16>::lo(ua), Io16<T16>::lo(ub));
-            xab[2 * h + 1] = fx2(Io16<T16>::hi(ua), Io16<T16>::hi(ub));
+            for (int h = 0; h < G / 2; ++h) {
+                const uint32_t ua = w[s][h], ub = w[s][G / 2 + h];
+                xab[2 * h] = fx2(Io16<T16>::lo(ua), Io16<T16>::lo(ub));
+                xab[2 * h + 1] = fx2(Io16<T16>::hi(ua), Io16<T16>::hi(ub));
+            }
+            fx2 pab[G];
+            rdft_planes<G>(xab, pab);
+            const int phys = ((pair >> 2) ^ ((r >> 2) & 1)) * 16 + in_piece;   // SWIZZLE_32B
+            uint8_t* dst = xs + g * L::SBO + (r & 7) * kRowBytes32 + phys;
+#pragma unroll
+            for (int p = 0; p < G; ++p)
+                *reinterpret_cast<uint32_t*>(dst + L::plane_offset(p)) = Io16<T16>::pack(pab[p].x, pab[p].y);
         }
-        fx2 pab[G];
-        rdft_planes<G>(xab, pab);
-        const int phys = ((pair >> 2) ^ ((r >> 2) & 1)) * 16 + in_piece;   // SWIZZLE_32B
-        uint8_t* dst = xs + r * kRowBytes32 + phys;
-#pragma unroll
-        for (int p = 0; p < G; ++p)
-            *reinterpret_cast<uint32_t*>(dst + p * C::PLANE_BYTES) = Io16<T16>::pack(pab[p].x, pab[p].y);
     }
 }
 
@@ -434,7 +480,10 @@ __global__ void __launch_bounds__(tm::Cfg<G>::kThreads, 1)
                     const uint32_t a_lo = ptx::sdesc_sw32_lo(xb), b_lo = ptx::sdesc_sw32_lo(wb);
                     const uint32_t wplane16 = wplane >> 4;
                     const uint32_t acc0 = c > 0 ? 1u : 0u;
-                    auto A = [&](int pl) { return ptx::sdesc_sw32_from_lo(a_lo + (pl * C::PLANE_BYTES) / 16); };
+                    auto A = [&](int pl) {
+                        return ptx::sdesc_from_halves(tm::spec_desc_hi<G>(),
+                                                      a_lo + tm::SpecLayout<G>::plane_offset(pl) / 16);
+                    };
                     auto B = [&](int pl) { return ptx::sdesc_sw32_from_lo(b_lo + static_cast<uint32_t>(pl) * wplane16); };
                     auto D = [&](int pl) { return tmem_base + static_cast<uint32_t>(pl * p.NO); };
                     ptx::umma_f16(D(0), A(0), B(0), ID, acc0);          // k = 0

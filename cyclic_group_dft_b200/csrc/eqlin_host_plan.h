@@ -113,8 +113,9 @@ int plan_tn_g(int64_t Cout, int64_t Cin, size_t max_smem, Plan* pl) {
     // The kernel's input ring is latency-bound: each x chunk's stage stays busy for its
     // load, DFT and MMAs, so stages, not bandwidth, set the rate (B200, p4 C96: 3 stages
     // 72.5 us, 4 stages 65.1 us).  Staging each epilogue group as two pieces of TG/2
-    // rows halves the staging space.
-    pl->ysub = env_int("EQLIN_YSUB", kDefaultYSub) == 2 && S::TG % 2 == 0 ? 2 : 1;
+    // rows halves the staging space (G <= 4 only; p4 C96 measured slower with it: 72.0 us
+    // with 6 stages against 65.3 us with 5, so it is off by default).
+    pl->ysub = env_int("EQLIN_YSUB", kDefaultYSub) == 2 && G <= 4 && S::TG % 2 == 0 ? 2 : 1;
     pl->TG = S::TG / pl->ysub;
     // y staging: per active epilogue warp, ybufs buffers of TG/ysub rows x 32*G 16-bit
     // columns; double-buffered when at least 4 ring stages still fit
