@@ -77,7 +77,11 @@ constexpr int kYStageBytes = kEpiWarps * kYWarpBufs * kYWarpBufBytes;   // 32 KB
 
 template <int G>
 struct Cfg {
-    static constexpr int DW = 4;                              // DFT warps
+    // DFT warps: at most 6 keep the CTA at 16 warps (128 registers per thread; 18 warps
+    // would cap it at 96).  B200: p8 C64 20.8 us with 6, 21.2 us with 4; C16 C32 123.2 us
+    // with 4, 129.8 us with 6 (its DFT warps then share two SM partitions with epilogue
+    // warps, whose G = 16 inverse transforms are as long as the DFT's)
+    static constexpr int DW = G == 16 ? 4 : 6;
     static constexpr int kDftThreads = DW * 32;
     static constexpr int kWarpDft0 = kEpiWarps;
     static constexpr int kWarpProducer = kEpiWarps + DW;
@@ -215,8 +219,8 @@ __device__ __forceinline__ void dft_chunk(uint8_t* xs, int dft_tid) {
 // ------------------------------------------------------------ epilogue role
 // Warp (q, half): tokens 32q..32q+31 (TMEM lane quarter q), output channels
 // [half*NO/2, (half+1)*NO/2) of the work item, in groups of OG = 32/G channels.
-// TMEM is read in batches of EB groups (EB = 2 for G <= 8: G x 2*OG = 64 registers), so a
-// warp waits for half as many TMEM loads; the batch's biases are loaded before the wait.
+// TMEM is read in batches of EB = 2 groups (G x 2*OG = 64 registers), so a warp waits for
+// half as many TMEM loads; the batch's biases are loaded before the wait.
 // Per group: inverse real DFT + bias (channel pairs packed as fx2), bf16, one 64-byte row
 // per lane into the warp's own SWIZZLE_64B staging tile [32 tokens x 32 columns]
 // (double-buffered), and lane 0 stores it with TMA; the epilogue warps never wait for one
@@ -227,7 +231,7 @@ __device__ __forceinline__ void epilogue_tile(const TmParams& p, const CUtensorM
                                               int& ybuf, uint32_t acc_empty) {
     using C = Cfg<G>;
     constexpr int OG = C::OG;
-    constexpr int EB = G <= 8 ? 2 : 1;             // groups per TMEM load batch
+    constexpr int EB = 2;                          // groups per TMEM load batch
     const int n_groups = (p.NO / 2) / OG;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const long long row0 = n0 + q * 32;            // first token of this warp's rows
