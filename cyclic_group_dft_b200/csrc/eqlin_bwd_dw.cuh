@@ -19,7 +19,8 @@
 // contiguous range of 32-token chunks, and keeps its partial dW in TMEM:
 //   warp 0      TMA producer: per chunk the dy tile [kTok tokens x MO*G] and the x tile
 //               [kTok tokens x NI*G] into a raw ring of p.raw_stages stages (zero fill past
-//               N, Cout, Cin).
+//               N, Cout, Cin), as boxes of kTok rows x kRowBytes (128 B, SWIZZLE_128B; 64 B,
+//               SWIZZLE_64B at G = 2).
 //   warp 1      MMA issuer + TMEM owner: per chunk and 16-token K step, tcgen05.mma with
 //               A = DY^ plane [128 rows (MO valid) x 16 tokens], B = X^ plane [NI x 16],
 //               both MN-major (channels contiguous, tokens along K), D plane in TMEM
@@ -28,8 +29,9 @@
 //                 Re: D_2k   += DYr Xr + DYi Xi,   Im: D_2k+1 += DYi Xr - DYr Xi
 //               (the minus through the descriptor's negate-A bit).
 //   warps 2..   DFT (dw::Cfg<G>::kDftWarps warps): a unit of work is one token x a few
-//               consecutive channels (lanes = consecutive units, so loads and stores
-//               are contiguous); a thread first loads all of its units of a pass, then
+//               consecutive channels; the 8 lanes of each 16-byte load pass take one
+//               channel group of 8 consecutive tokens, which the swizzled boxes spread
+//               over 8 bank groups (dw::unit_token); a thread first loads all of its units of a pass, then
 //               runs the real DFT over G in fp32 registers (channel pairs packed as fx2),
 //               packs each plane to the I/O type and writes one store per plane into the
 //               MN-major SWIZZLE_64B spectra.  The dy units also add plane 0 (the group
@@ -106,6 +108,11 @@ struct Cfg {
     // with MO <= 128 and G * NI <= 512, NI <= 256
     static constexpr int kMaxUnits = kTok * (128 + (512 / G < 256 ? 512 / G : 256)) / kChanPerUnit;
     static constexpr int kMaxPasses = (kMaxUnits + kDftThreads - 1) / kDftThreads;
+    // raw box rows: 128 B (SWIZZLE_128B) of kBoxChannels channels x G, 64 B (SWIZZLE_64B)
+    // at G = 2; a unit (kChanPerUnit channels, 32 or 64 bytes) never straddles two boxes
+    static constexpr int kRowBytes = G == 2 ? 64 : 128;
+    static constexpr int kBoxChannels = kRowBytes / (2 * G);
+    static_assert(kBoxChannels % kChanPerUnit == 0, "units inside boxes");
 
 };
 constexpr int kBarDft = 1;         // named barrier among the DFT warps
@@ -148,46 +155,33 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, int* s
 
 
 // One unit of the transform: one token t of the chunk x CPU consecutive channels
-// c0 .. c0+CPU-1 of the dy tile or of the x tile (CPU = Cfg<G>::kChanPerUnit).  Raw tile
-// layout: boxes of cpb channels (cpb a multiple of CPU, so a unit never straddles two
-// boxes), each [kTok tokens][cpb*G].  The unit's CPU*G values are CPU*G/2 32-bit words,
-// channel c0+j in words j*G/2 .. (j+1)*G/2-1.
+// c0 .. c0+CPU-1 of the dy tile or of the x tile (CPU = Cfg<G>::kChanPerUnit).  `row` is
+// the token's row of the box holding the unit; the unit's k-th 16-byte piece is logical
+// piece lc + k of the row, stored at piece (lc + k) ^ key (key = t % 8 for 128-byte
+// SWIZZLE_128B rows, (t / 2) % 4 for 64-byte SWIZZLE_64B rows).  The unit's CPU*G values
+// are CPU*G/2 32-bit words, channel c0+j in words j*G/2 .. (j+1)*G/2-1.
 template <int G, int CPU>
-__device__ __forceinline__ void load_unit(const uint8_t* src, int lane, uint32_t (&w)[CPU * G / 2]) {
+__device__ __forceinline__ void load_unit(const uint8_t* row, int lc, int key, uint32_t (&w)[CPU * G / 2]) {
     constexpr int BYTES = CPU * G * 2;
     constexpr int PIECES = BYTES / 16;       // 2 or 4 sixteen-byte pieces
     static_assert(BYTES == 32 || BYTES == 64, "unit size");
-    // Consecutive lanes hold consecutive units, BYTES apart: loading piece q in step q
-    // would put every lane of a step on the same few banks.  Lane l loads piece
-    // (q + rot) % PIECES in step q instead, rot = (l >> s) % PIECES chosen so that the 32
-    // lanes of a step cover all eight 16-byte bank groups, then rotates back.
-    const int rot = (lane >> (PIECES == 4 ? 1 : 2)) & (PIECES - 1);
-    uint4 ld[PIECES];
-#pragma unroll
-    for (int q = 0; q < PIECES; ++q) ld[q] = *reinterpret_cast<const uint4*>(src + 16 * ((q + rot) & (PIECES - 1)));
-    // piece k sits in ld[(k - rot) % PIECES]: rotate right by rot (in steps of 1 and 2)
-    if (rot & 1) {
-        const uint4 last = ld[PIECES - 1];
-#pragma unroll
-        for (int k = PIECES - 1; k > 0; --k) ld[k] = ld[k - 1];
-        ld[0] = last;
-    }
-    if constexpr (PIECES == 4) {
-        if (rot & 2) {
-            const uint4 a = ld[0], b = ld[1];
-            ld[0] = ld[2];
-            ld[1] = ld[3];
-            ld[2] = a;
-            ld[3] = b;
-        }
-    }
 #pragma unroll
     for (int k = 0; k < PIECES; ++k) {
-        w[4 * k + 0] = ld[k].x;
-        w[4 * k + 1] = ld[k].y;
-        w[4 * k + 2] = ld[k].z;
-        w[4 * k + 3] = ld[k].w;
+        const uint4 v = *reinterpret_cast<const uint4*>(row + 16 * ((lc + k) ^ key));
+        w[4 * k + 0] = v.x;
+        w[4 * k + 1] = v.y;
+        w[4 * k + 2] = v.z;
+        w[4 * k + 3] = v.w;
     }
+}
+
+// Token and channel group of unit v of a tile with ng groups of CPU channels per token:
+// v = ((token / 8) * ng + group) * 8 + token % 8, so consecutive lanes take 8 consecutive
+// tokens of one group, then the next group.
+__device__ __forceinline__ void unit_token(int v, int ng, int& tok, int& grp) {
+    const int rest = v >> 3;
+    grp = rest % ng;
+    tok = (rest / ng) * 8 + (v & 7);
 }
 
 // Real DFT over G of the unit's channels (in pairs packed as fx2), stored to the planes in
@@ -247,7 +241,7 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
                        const DwParams p) {
     constexpr int kDftThreads = dw::Cfg<G>::kDftThreads;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* base = ptx::smem_align_1k(smem_raw);
     const uint32_t spec_bytes = p.a_bytes + p.b_bytes;
     uint8_t* raw0 = base;
     uint8_t* spec0 = raw0 + p.raw_stages * p.raw_bytes;
@@ -417,18 +411,25 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
         // stage and destination offsets in a spectra buffer are computed once
         constexpr int MP = dw::Cfg<G>::kMaxPasses;
         uint32_t src_off[MP], dst_off[MP];
+        uint8_t lc_key[MP];
         uint32_t dy_mask = 0, valid_mask = 0;
 #pragma unroll
         for (int ps = 0; ps < MP; ++ps) {
             const int u = t + ps * kDftThreads;
             src_off[ps] = dst_off[ps] = 0;
+            lc_key[ps] = 0;
             if (u < n_units) {
                 const bool is_dy = u < units_dy;
                 const int v = is_dy ? u : u - units_dy, ng = is_dy ? groups_dy : groups_x;
-                const int tok = v / ng, c = CPU * (v - tok * ng), cpb = is_dy ? p.cpb_dy : p.cpb_x;
-                const int box = c / cpb, row_bytes = cpb * G * 2;
-                src_off[ps] = (is_dy ? 0u : p.dy_bytes) + static_cast<uint32_t>(box * (dw::Cfg<G>::kTok * row_bytes) +
-                                                                                 tok * row_bytes + (c - box * cpb) * G * 2);
+                int tok, grp;
+                dw::unit_token(v, ng, tok, grp);
+                const int c = CPU * grp;
+                constexpr int RB = dw::Cfg<G>::kRowBytes, CPB = dw::Cfg<G>::kBoxChannels;
+                const int box = c / CPB;
+                src_off[ps] = (is_dy ? 0u : p.dy_bytes) + static_cast<uint32_t>(box * (dw::Cfg<G>::kTok * RB) + tok * RB);
+                const int lc = (c - box * CPB) * G * 2 / 16;
+                const int key = RB == 128 ? (tok & 7) : ((tok >> 1) & 3);
+                lc_key[ps] = static_cast<uint8_t>(lc | (key << 4));
                 dst_off[ps] = (is_dy ? 0u : p.a_bytes) + dw::unit_dst_offset(tok, c, is_dy ? sbo_a : sbo_b);
                 valid_mask |= 1u << ps;
                 if (is_dy) dy_mask |= 1u << ps;
@@ -452,7 +453,7 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
             for (int ps = 0; ps < MP; ++ps) {
                 if (!(valid_mask & (1u << ps))) break;
                 uint32_t words[CPU * G / 2];
-                dw::load_unit<G, CPU>(raw + src_off[ps], lane, words);
+                dw::load_unit<G, CPU>(raw + src_off[ps], lc_key[ps] & 15, lc_key[ps] >> 4, words);
                 const bool is_dy = dy_mask & (1u << ps);
                 dw::store_unit<G, CPU, T16>(words, spec + dst_off[ps], is_dy ? plane_a : plane_b, bsum[ps], is_dy);
             }
@@ -494,7 +495,9 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
         for (int ps = 0; ps < dw::Cfg<G>::kMaxPasses; ++ps) {
             const int u = t + ps * kDftThreads;
             if (u < units_dy) {
-                const int tok = u / groups_dy, c = CPU * (u - tok * groups_dy);
+                int tok, grp;
+                dw::unit_token(u, groups_dy, tok, grp);
+                const int c = CPU * grp;
 #pragma unroll
                 for (int j = 0; j < CPU; ++j) bias_sm[tok * p.MO + c + j] = bsum[ps][j];
             }

@@ -379,8 +379,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                         const TcParams p) {
     using S = tc::Shape<G, NACC>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* smem = ptx::smem_align_1k(smem_raw);
 
     // a stage: the x chunk, transformed in place into its (larger) spectrum, then the
     // streamed weight chunk; the copies fill the x chunk and the weight chunk

@@ -314,8 +314,7 @@ __global__ void __launch_bounds__(tm::Cfg<G>::kThreads, 1)
                         const TmParams p) {
     using C = tm::Cfg<G>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* smem = ptx::smem_align_1k(smem_raw);
 
     constexpr int SL = pair_slots(G);
     const uint32_t wstage_bytes = STREAM_W ? static_cast<uint32_t>(SL * p.NO * kRowBytes32) : 0u;

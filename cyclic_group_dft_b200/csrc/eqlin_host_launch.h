@@ -371,7 +371,7 @@ void* dw_kernel_t(int G) {
 void* dw_kernel_for(int G, int io) { return io == EQLIN_F16 ? dw_kernel_t<__half>(G) : dw_kernel_t<__nv_bfloat16>(G); }
 
 int encode_rows_map(CUtensorMap* map, const void* base, int64_t cols, int64_t rows, int box_cols, int box_rows,
-                    int io) {
+                    int io, CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE) {
     auto encode = tensor_map_encoder();
     if (!encode) return fail(EQLIN_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
     cuuint32_t estr[2] = {1, 1};
@@ -380,7 +380,7 @@ int encode_rows_map(CUtensorMap* map, const void* base, int64_t cols, int64_t ro
     cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
     CUresult r = encode(map, io == EQLIN_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                         const_cast<void*>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(EQLIN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
     return EQLIN_OK;
@@ -417,9 +417,10 @@ int launch_dw(const DwPlan& pl, bool f32_path, int64_t Cout, int64_t Cin, int64_
         return EQLIN_OK;
     }
     CUtensorMap mdy, mx;
-    int s = encode_rows_map(&mdy, dy, Cout * G, N, pl.cpb_dy * iG, dw_tok(G), pl.io);
+    const CUtensorMapSwizzle swz = iG == 2 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+    int s = encode_rows_map(&mdy, dy, Cout * G, N, pl.cpb_dy * iG, dw_tok(G), pl.io, swz);
     if (s != EQLIN_OK) return s;
-    s = encode_rows_map(&mx, x, Cin * G, N, pl.cpb_x * iG, dw_tok(G), pl.io);
+    s = encode_rows_map(&mx, x, Cin * G, N, pl.cpb_x * iG, dw_tok(G), pl.io, swz);
     if (s != EQLIN_OK) return s;
     eqlin::DwParams p;
     p.ws = static_cast<float*>(ws);

@@ -353,15 +353,6 @@ struct DwPlan {
 uint32_t round_kb(size_t v) { return static_cast<uint32_t>((v + 1023) / 1024 * 1024); }
 int round16(int64_t v) { return static_cast<int>((v + 15) / 16 * 16); }
 
-// Channels per TMA box: the largest divisor d of C with d*G <= 256 elements, 16-byte
-// box rows and d a multiple of `unit` (the channels of one transform unit); C is a
-// multiple of 16, so d = 16 always qualifies.
-int box_channels(int C, int G, int unit) {
-    for (int d = C; d >= 1; --d)
-        if (C % d == 0 && d % unit == 0 && d * G <= 256 && (d * G * 2) % 16 == 0) return d;
-    return 0;
-}
-
 int dw_channels_per_unit(int G) { return G <= 4 ? 8 : (G == 8 ? 4 : 2); }
 
 int max_dw_units(int G) {
@@ -412,8 +403,10 @@ size_t dw_smem(int MO, int NI, int G, int RS, int SB, DwPlan* out) {
 }
 
 // Pick the tile with the fewest units that fits shared memory with the minimum
-// pipeline (2 raw stages, 1 spectra buffer); fewer units = fewer re-reads of x and dy.
-// Ties go to the larger MO (less MMA padding), then the larger NI.  Then the deepest
+// pipeline (2 raw stages, 1 spectra buffer) and whose transform units the threads can
+// hold; fewer units = fewer re-reads of x and dy.  Ties go to the least padded area (192
+// input channels as 2 x 96, not 128 + 64: B200, weight gradient of the 192 -> 768 layer
+// 341 us against 386 us), then to the larger MO (less MMA padding), then the larger NI.  Then the deepest
 // raw ring that fits: with two spectra buffers (the transform of one chunk overlaps the
 // MMAs of the previous one) when that still leaves >= 2 raw stages, else with one.
 // Tuning overrides: EQLIN_DW_TILE ("MO,NI"), EQLIN_DW_SPEC_BUFS, EQLIN_DW_RAW_STAGES.
@@ -421,14 +414,18 @@ int plan_dw(int64_t Cout, int64_t Cin, int G, size_t max_smem, int sm_count, DwP
     const int mo_max = std::min(eqlin::kMmaM, round16(Cout));
     const int ni_cap = std::min(256, (512 / G) / 16 * 16);
     const int ni_max = std::min(ni_cap, round16(Cin));
-    long long best_units = -1;
+    long long best_units = -1, best_area = 0;
     int best_mo = 0, best_ni = 0;
+    const int cpu = dw_channels_per_unit(G);
     for (int mo = mo_max; mo >= 16; mo -= 16) {
         for (int ni = ni_max; ni >= 16; ni -= 16) {
+            if (dw_tok(G) * (mo + ni) / cpu > max_dw_units(G)) continue;
             if (dw_smem(mo, ni, G, 2, 1, nullptr) > max_smem) continue;
-            const long long units = ((Cout + mo - 1) / mo) * ((Cin + ni - 1) / ni);
-            if (best_units < 0 || units < best_units) {
+            const long long n_ot = (Cout + mo - 1) / mo, n_it = (Cin + ni - 1) / ni;
+            const long long units = n_ot * n_it, area = n_ot * mo * n_it * ni;
+            if (best_units < 0 || units < best_units || (units == best_units && area < best_area)) {
                 best_units = units;
+                best_area = area;
                 best_mo = mo;
                 best_ni = ni;
             }
@@ -438,7 +435,8 @@ int plan_dw(int64_t Cout, int64_t Cin, int G, size_t max_smem, int sm_count, DwP
     if (const char* e = std::getenv("EQLIN_DW_TILE")) {  // "MO,NI" tuning override
         int mo = 0, ni = 0;
         if (std::sscanf(e, "%d,%d", &mo, &ni) == 2 && mo >= 16 && mo <= mo_max && mo % 16 == 0 && ni >= 16 &&
-            ni <= ni_max && ni % 16 == 0 && dw_smem(mo, ni, G, 2, 1, nullptr) <= max_smem) {
+            ni <= ni_max && ni % 16 == 0 && dw_smem(mo, ni, G, 2, 1, nullptr) <= max_smem &&
+            dw_tok(G) * (mo + ni) / cpu <= max_dw_units(G)) {
             best_mo = mo;
             best_ni = ni;
         }
@@ -460,10 +458,11 @@ int plan_dw(int64_t Cout, int64_t Cin, int G, size_t max_smem, int sm_count, DwP
     pl->n_it = static_cast<int>((Cin + best_ni - 1) / best_ni);
     pl->max_splits = std::max(1, sm_count / pl->units());
     // a transform unit (dw::Cfg<G>::kChanPerUnit channels) never straddles two boxes
-    const int cpu = dw_channels_per_unit(G);
-    pl->cpb_dy = box_channels(best_mo, G, cpu);
-    pl->cpb_x = box_channels(best_ni, G, cpu);
-    if (pl->cpb_dy == 0 || pl->cpb_x == 0) return fail(EQLIN_ERR_UNSUPPORTED, "no TMA box width for the tile");
+    // raw boxes of 128-byte rows (64 at G = 2), swizzled (dw::Cfg<G>::kRowBytes): MO and NI,
+    // multiples of 16, are multiples of the box's channels
+    pl->cpb_dy = pl->cpb_x = (G == 2 ? 64 : 128) / (2 * G);
+    if (best_mo % pl->cpb_dy != 0 || best_ni % pl->cpb_x != 0 || pl->cpb_dy % cpu != 0)
+        return fail(EQLIN_ERR_UNSUPPORTED, "no TMA box width for the tile");
     if (dw_tok(G) * (best_mo + best_ni) / cpu > max_dw_units(G))
         return fail(EQLIN_ERR_UNSUPPORTED, "weight-gradient tile has more transform units than threads can hold");
     dw_smem(best_mo, best_ni, G, rs, sb, pl);

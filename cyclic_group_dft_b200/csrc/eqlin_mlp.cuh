@@ -186,8 +186,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     using S = typename C::S;
     constexpr int U = C::kUnits;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* smem = ptx::smem_align_1k(smem_raw);
 
     const int NS = p.stages, nK1 = p.nK1;
     uint8_t* xslot0 = smem;                                                   // nK1 x chunks / X^

@@ -15,6 +15,14 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// Dynamic shared memory rounded up to a 1 KB boundary by pointer arithmetic on the
+// __shared__ array itself.  Every pointer derived from the result stays in the shared
+// state space, so the compiler emits shared-memory loads and stores for it; rounding
+// through an integer would turn all of them into generic accesses.
+__device__ __forceinline__ uint8_t* smem_align_1k(uint8_t* raw) {
+    return raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);
+}
+
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
