@@ -522,7 +522,10 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
 // Cross-CTA reduction and inverse DFT, deterministic, in one small kernel.
 // Block = (unit u, column ii of the unit, 32 consecutive rows oo), or the unit's bias
 // sums when ii == NI.  Warp w sums the slabs of splits w, w+8, w+16, ... in that order,
-// float64, for the block's G planes; the 8 warp sums are then added in warp order.
+// float64, for the block's G planes, with kIn splits (kIn * G loads per thread) in
+// flight per round trip; the 8 warp sums are then added in warp order.  Launched as a
+// programmatic dependent of the main kernel: its blocks start as that kernel's CTAs
+// exit and wait (griddepcontrol.wait) for all of its slabs before reading them.
 // With P_k = sum_n DY_k conj(X_k) (unscaled transforms), warp 0 writes
 //   dw[o,i,m] = (1/G) [P_0 + (-1)^m P_{G/2} + 2 sum_{0<k<G/2} Re(P_k e^{+2 pi i m k / G})],
 // and dbias[o] from the bias sums of the units of input tile 0.
@@ -538,6 +541,8 @@ struct DwFinalParams {
 template <int G>
 __global__ void __launch_bounds__(256) eqlin_dw_finish_kernel(const DwFinalParams f) {
     __shared__ double red[8][G][32];
+    ptx::grid_launch_dependents();
+    ptx::grid_dependency_wait();
     const int n_og = (f.MO + 31) / 32;
     const int per_unit = (f.NI + 1) * n_og;
     const int unit = static_cast<int>(blockIdx.x) / per_unit;
@@ -555,8 +560,8 @@ __global__ void __launch_bounds__(256) eqlin_dw_finish_kernel(const DwFinalParam
                            (bias_blk ? f.slab_floats + oo : static_cast<size_t>(ii) * f.MO + oo);
         const int nv = bias_blk ? 1 : G;
         int s = warp;
-        // four splits in flight (4G loads per thread), added in split order
-        constexpr int kIn = 4;
+        // kIn splits in flight (kIn * G <= 32 loads per thread), added in split order
+        constexpr int kIn = 32 / G > 2 ? 32 / G : 2;
         for (; s + 8 * (kIn - 1) < f.n_splits; s += 8 * kIn) {
             float v[kIn][G];
 #pragma unroll

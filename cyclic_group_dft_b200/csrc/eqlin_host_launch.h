@@ -468,12 +468,24 @@ int launch_dw(const DwPlan& pl, bool f32_path, int64_t Cout, int64_t Cin, int64_
     f.n_splits = p.n_splits;
     f.slab_floats = pl.slab_floats;
     const unsigned fgrid = static_cast<unsigned>(pl.units() * (pl.NI + 1) * ((pl.MO + 31) / 32));
+    // a programmatic dependent of the main kernel (its blocks wait for the slabs)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(fgrid);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = use_pdl() ? 1 : 0;
     switch (iG) {
-        case 2: eqlin::eqlin_dw_finish_kernel<2><<<fgrid, 256, 0, st>>>(f); break;
-        case 4: eqlin::eqlin_dw_finish_kernel<4><<<fgrid, 256, 0, st>>>(f); break;
-        case 8: eqlin::eqlin_dw_finish_kernel<8><<<fgrid, 256, 0, st>>>(f); break;
-        default: eqlin::eqlin_dw_finish_kernel<16><<<fgrid, 256, 0, st>>>(f); break;
+        case 2: e = cudaLaunchKernelEx(&cfg, eqlin::eqlin_dw_finish_kernel<2>, f); break;
+        case 4: e = cudaLaunchKernelEx(&cfg, eqlin::eqlin_dw_finish_kernel<4>, f); break;
+        case 8: e = cudaLaunchKernelEx(&cfg, eqlin::eqlin_dw_finish_kernel<8>, f); break;
+        default: e = cudaLaunchKernelEx(&cfg, eqlin::eqlin_dw_finish_kernel<16>, f); break;
     }
+    if (e != cudaSuccess) return cuda_fail(e, "weight-gradient reduction launch");
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "weight-gradient reduction launch");
     return EQLIN_OK;
 }
