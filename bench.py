@@ -155,9 +155,18 @@ def line_config(wl: workloads.Workload, world: int) -> dict:
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    """Samples SM clock and clock-event reasons through NVML in a thread."""
+    """Samples SM clock and clock-event reasons through NVML: once before the warm-up
+    launches (begin), every period_s in a thread while the timed region runs, and once
+    right after it (stop).  The first in-region sample comes one period after the start:
+    an NVML query just before or while the kernels run slows them (B200, p4 C96, 20
+    back-to-back launches: 62.4 us per launch with 10 ms sampling from the start against
+    60.2 us without; 61.8 us with one query just before the start), so a region shorter
+    than one period is bracketed by the samples around it instead.  Construct it (NVML
+    initialisation) before the warm-up too: a host delay between the warm-up and the
+    timed region lets the GPU idle, and the region then starts slow (63.0 us after a
+    20 ms pause)."""
 
-    def __init__(self, device_index: int, period_s: float = 0.01):
+    def __init__(self, device_index: int, period_s: float = 0.05):
         self.samples: list[tuple[int, int]] = []
         self.max_mhz = None
         self.error = None
@@ -191,13 +200,15 @@ class ClockSampler:
             self.error = str(exc)
 
     def _run(self):
-        while not self._stop.is_set():
+        while not self._stop.wait(self.period):
             self._sample()
-            self._stop.wait(self.period)
+
+    def begin(self):
+        if self._nvml is not None:
+            self._sample()
 
     def start(self):
         if self._nvml is not None:
-            self._sample()
             self._thread = threading.Thread(target=self._run, daemon=True)
             self._thread.start()
 
@@ -217,7 +228,9 @@ class ClockSampler:
             bits |= r
         reasons = [name for bit, name in REASON_BITS.items() if bits & bit and name != "gpu_idle"]
         return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": reasons,
-                "samples": len(self.samples)}
+                "samples": len(self.samples),
+                "sampling": f"NVML, before the warm-up launches, right after the timed region and every "
+                            f"{self.period * 1e3:.0f} ms inside it"}
 
 
 # ------------------------------------------------------------------ CPU oracle
@@ -457,9 +470,11 @@ def measure_workload(ctx: Ctx, wl: workloads.Workload, K: int, warmup: int, head
     # the overlap of one launch's tail with the next one's prologue (programmatic
     # dependent launch), which is how the kernel runs in a real stream of layers.
     # The average launch duration of the kernel is therefore elapsed / K.
+    clocks = ClockSampler(dev.index) if headline else None
+    if clocks is not None:
+        clocks.begin()
     for i in range(warmup):
         fwd(i)
-    clocks = ClockSampler(dev.index) if headline else None
     elapsed_ms = time_back_to_back(ctx, fwd_c, K, clocks, graph=ctx.graph)
     if any(rc != eq.EQLIN_OK for rc in rcs):
         raise RuntimeError(f"{wl.name}: eqlin_forward returned {sorted(set(rcs))}")
