@@ -20,9 +20,11 @@
 //                    laid out so that each 8-row group of the spectrum replaces the same
 //                    rows of the input (tm::SpecLayout): a warp transforms whole groups
 //                    and orders only its own reads before its writes
-//   MMA warp         one thread issues tcgen05.mma: 2 real products, and 2 per complex
-//                    frequency, each over the Re and Im planes of D at once (N = 2*NO)
-//                    thanks to the weight image's [-Im, Re, Im] slots (eqlin_layout.h)
+//   MMA warp         one thread issues tcgen05.mma: 2 real products, and per complex
+//                    frequency Xr [Wr | Wi] over the Re and Im planes of D at once
+//                    (N = 2*NO), then for G <= 8 Xi (-Wi) into Re (the negate-B bit) and
+//                    Xi Wr into Im (N = NO), for G = 16 Xi [-Wi | Wr] from the weight
+//                    image's pair slots (eqlin_layout.h, tm_weight_slots)
 //   8 epilogue warps lane = token; per group of 32/G output channels: tcgen05.ld of the
 //                    G planes, inverse real DFT + bias, bf16, into the warp's own
 //                    SWIZZLE_64B staging tile [32 tokens x 32 columns], TMA store by the
@@ -316,7 +318,7 @@ __global__ void __launch_bounds__(tm::Cfg<G>::kThreads, 1)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = ptx::smem_align_1k(smem_raw);
 
-    constexpr int SL = pair_slots(G);
+    constexpr int SL = tm_weight_slots(G);
     const uint32_t wstage_bytes = STREAM_W ? static_cast<uint32_t>(SL * p.NO * kRowBytes32) : 0u;
     const uint32_t stage_bytes = C::XCHUNK_BYTES + wstage_bytes;
     const int NS = p.stages;
@@ -458,6 +460,7 @@ __global__ void __launch_bounds__(tm::Cfg<G>::kThreads, 1)
             bool ok = true;
             if constexpr (!STREAM_W) ok = tc::wait_bounded(bar_w_full, 0, ctl, p.status, p.timeout_ns);
             const uint32_t ID = idesc_f16kind_f32(tm::kM, p.NO, Io16<T16>::kUmmaFormat, false, false);
+            const uint32_t ID_NEGB = idesc_f16kind_f32(tm::kM, p.NO, Io16<T16>::kUmmaFormat, false, true);
             // complex products: N = 2*NO output columns, the Re and Im planes of D side by side
             const uint32_t ID2 = idesc_f16kind_f32(tm::kM, G > 2 ? 2 * p.NO : p.NO, Io16<T16>::kUmmaFormat, false, false);
             const uint32_t wplane = static_cast<uint32_t>(p.NO) * kRowBytes32;
@@ -493,9 +496,16 @@ __global__ void __launch_bounds__(tm::Cfg<G>::kThreads, 1)
                     ptx::umma_f16(D(1), A(1), B(1), ID, acc0);          // k = G/2
 #pragma unroll
                     for (int k = 1; k < G / 2; ++k) {                   // (Xr + i Xi)(Wr + i Wi)
-                        const int pr = 2 * k, pi = 2 * k + 1, s = pair_first_slot(k);
-                        ptx::umma_f16(D(pr), A(pr), B(s + 1), ID2, acc0);   // [Dr|Di] += Xr [Wr; Wi]
-                        ptx::umma_f16(D(pr), A(pi), B(s), ID2, 1u);         // [Dr|Di] += Xi [-Wi; Wr]
+                        const int pr = 2 * k, pi = 2 * k + 1;
+                        if constexpr (tm_pair_slots(G)) {
+                            const int s = pair_first_slot(k);
+                            ptx::umma_f16(D(pr), A(pr), B(s + 1), ID2, acc0);   // [Dr|Di] += Xr [Wr; Wi]
+                            ptx::umma_f16(D(pr), A(pi), B(s), ID2, 1u);         // [Dr|Di] += Xi [-Wi; Wr]
+                        } else {
+                            ptx::umma_f16(D(pr), A(pr), B(pr), ID2, acc0);      // [Dr|Di] += Xr [Wr; Wi]
+                            ptx::umma_f16(D(pr), A(pi), B(pi), ID_NEGB, 1u);    // Dr += Xi (-Wi)
+                            ptx::umma_f16(D(pi), A(pi), B(pr), ID, 1u);         // Di += Xi Wr
+                        }
                     }
                     ptx::umma_commit(bar_empty(stage));
                     if (++stage == NS) { stage = 0; phase ^= 1u; }

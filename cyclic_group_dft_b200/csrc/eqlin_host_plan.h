@@ -232,7 +232,7 @@ int plan_tm_g(int64_t Cout, int64_t Cin, size_t max_smem, Plan* pl) {
     pl->BN = eqlin::tm::kM;
     pl->box_elems = C::X_BOX;
     pl->x_swizzle128 = C::X_SW128;
-    const size_t wchunk = static_cast<size_t>(eqlin::pair_slots(G)) * no * eqlin::kRowBytes32;  // one (oc, c) chunk
+    const size_t wchunk = static_cast<size_t>(eqlin::tm_weight_slots(G)) * no * eqlin::kRowBytes32;  // one (oc, c) chunk
     const size_t fixed = kSmemAlignSlack + kSmemCtlBytes +
                          static_cast<size_t>(eqlin::tm::kYStageBytes);
     if (pl->n_oc == 1) {

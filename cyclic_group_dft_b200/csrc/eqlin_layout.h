@@ -44,7 +44,7 @@ __host__ __device__ inline size_t image_offset(size_t sub, int rows, int r, int 
 // [-Im V_k; Re V_k] are each one operand of twice the slot's rows, and a complex product
 // (a + ib)(c + id) takes two MMAs that write the Re and Im planes of D side by side:
 //   [D_re | D_im] += a [c; d],   [D_re | D_im] += b [-d; c].
-// The tokens-on-M weight image uses it for W^, the tokens-on-N kernels for X^.
+// The tokens-on-N kernels use it for X^.
 __host__ __device__ constexpr int pair_slots(int G) { return 2 + 3 * (G / 2 - 1); }
 // first slot of complex frequency k (0 < k < G/2): the -Im slot
 __host__ __device__ constexpr int pair_first_slot(int k) { return 2 + 3 * (k - 1); }
@@ -59,7 +59,15 @@ __host__ __device__ inline int pair_slot_plane(int s, float* sign) {
 
 // Tokens-on-M kernel variant: 16-channel K chunks, rows of 32 bytes, SWIZZLE_32B
 // (16-byte piece j of row r stored at piece j ^ ((r >> 2) & 1)).  Image layout
-// [oc][c][s][r < rows][16] over the pair slots s < pair_slots(G) of W^.
+// [oc][c][s][r < rows][16] over the weight slots s:
+//  - G <= 8: the G planes of W^ in plane order (Re and Im of a complex frequency adjacent,
+//    so [Re W_k | Im W_k] is one operand of twice the rows; the -Im W_k factor of a
+//    complex product comes from the MMA's negate-B bit, one more MMA per frequency);
+//  - G = 16: the pair slots above, so each complex product is two MMAs.
+// B200: p8 C64 19.3 us with plane order (a fourth ring stage fits) against 19.6 us;
+// C16 C32 112.5 us with plane order against 110.6 us.
+__host__ __device__ constexpr bool tm_pair_slots(int G) { return G > 8; }
+__host__ __device__ constexpr int tm_weight_slots(int G) { return tm_pair_slots(G) ? pair_slots(G) : G; }
 constexpr int kChunkK16 = 16;
 constexpr int kRowBytes32 = 32;
 __host__ __device__ inline size_t image_offset_k16(size_t sub, int rows, int r, int col) {

@@ -96,14 +96,14 @@ __global__ void eqlin_prep_image_kernel(const float* __restrict__ w_f32, int Cou
     *reinterpret_cast<T16*>(img + image_offset(sub, rows, r, col)) = Io16<T16>::from_float(v);
 }
 
-// Image for the tokens-on-M kernel (layout: image_offset_k16 over the weight slots of
-// pair_slots).  `rows` rows per sub-block; output chunk oc covers o = oc*rows + r.
+// Image for the tokens-on-M kernel (layout: image_offset_k16 over the weight slots,
+// tm_weight_slots).  `rows` rows per sub-block; output chunk oc covers o = oc*rows + r.
 template <class T16>
 __global__ void eqlin_prep_image_k16_kernel(const float* __restrict__ w_f32, int Cout, int Cin, int G,
                                             int nK, int rows, size_t n_elems, uint8_t* __restrict__ img) {
     const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (idx >= n_elems) return;
-    const int SL = pair_slots(G);
+    const int SL = tm_weight_slots(G);
     const int col = static_cast<int>(idx % kChunkK16);
     const int r = static_cast<int>((idx / kChunkK16) % rows);
     const size_t sub = idx / (static_cast<size_t>(kChunkK16) * rows);
@@ -112,8 +112,8 @@ __global__ void eqlin_prep_image_k16_kernel(const float* __restrict__ w_f32, int
     const int oc = static_cast<int>(sub / (static_cast<size_t>(SL) * nK));
     const int o = oc * rows + r;
     const int i = c * kChunkK16 + col;
-    float sign;
-    const int p = pair_slot_plane(slot, &sign);
+    float sign = 1.0f;
+    const int p = tm_pair_slots(G) ? pair_slot_plane(slot, &sign) : slot;
     float v = 0.0f;
     if (o < Cout && i < Cin) v = sign * w_f32[(static_cast<size_t>(p) * Cin + i) * Cout + o];
     *reinterpret_cast<T16*>(img + image_offset_k16(sub, rows, r, col)) = Io16<T16>::from_float(v);
