@@ -59,9 +59,8 @@ struct TcParams {
     int n_work;             // n_tiles * n_oc
     int stages;             // smem ring depth
     uint32_t w_region_bytes;  // smem reserved for resident weights (0 when streamed)
-    uint32_t ystage_bytes;    // y staging per epilogue warp (ybufs buffers of TG/ysub x 32*G bf16)
+    uint32_t ystage_bytes;    // y staging per epilogue warp (ybufs buffers of TG x 32*G bf16)
     int ybufs;                // 1 or 2 staging buffers per epilogue warp; 0 = direct stores
-    int ysub;                 // 1 or 2 staged TMA stores per epilogue group (rows TG / ysub each)
     int yq;                   // TMEM lane quarters that hold output rows, each with staging (1..4)
     uint32_t w_img_bytes;     // bytes of the resident image to copy
     unsigned long long timeout_ns;
@@ -234,22 +233,19 @@ __device__ __forceinline__ void dft_chunk(uint8_t* xs, int dft_tid) {
 // Warp (q, half): TMEM lane quarter q (output rows 32q..32q+31 of the chunk), tokens
 // [half*BN/2, (half+1)*BN/2) of the tile held in accumulator `acc` (column base).
 // The warp reads a group of TG tokens x its 32 output channels (32*G columns) from
-// TMEM, stages it in SUB pieces of TG/SUB rows in its own buffers and lane 0 stores
-// each piece with TMA, so the epilogue warps never wait for one another.  `wstage`:
-// this warp's p.ybufs buffers; `ybuf` alternates.  Smaller pieces need less staging
-// space, which the kernel gives to its input ring.
-template <int G, int NACC, class T16, int SUB = 1>
+// TMEM, stages it in its own buffer and lane 0 stores it with TMA, so the epilogue
+// warps never wait for one another.  `wstage`: this warp's p.ybufs buffers; `ybuf`
+// alternates.
+template <int G, int NACC, class T16>
 __device__ __forceinline__ void epilogue_tile(const TcParams& p, const CUtensorMap* tmap_y, uint32_t acc,
                                               int q, int half, int lane, long long n0, int oc, uint8_t* wstage,
                                               int& ybuf) {
     using S = Shape<G, NACC>;
     constexpr int TG = S::TG;
-    constexpr int TR = TG / SUB;                            // rows of one staged piece
-    static_assert(SUB >= 1 && TG % SUB == 0, "staged pieces");
     constexpr int WCOLS = 32 * G;                           // y columns of the warp's 32 outputs
     constexpr int YBC = WCOLS < kYBoxCols2 ? WCOLS : kYBoxCols2;  // TMA box columns
     constexpr int NYB = WCOLS / YBC;
-    constexpr int BOX_BYTES = TR * YBC * 2;
+    constexpr int BOX_BYTES = TG * YBC * 2;
     const int o_local = q * 32 + lane;
     const int o = oc * kMmaM + o_local;
     const bool valid_o = o < p.Cout;
@@ -306,68 +302,64 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, const CUtensorM
             }
             continue;
         }
-#pragma unroll
-        for (int sb = 0; sb < SUB; ++sb) {
-            // the buffer about to be written was stored p.ybufs pieces ago: wait until read
-            if (lane == 0) {
-                if (p.ybufs == 2) ptx::bulk_wait_group_read<1>();
-                else ptx::bulk_wait_group_read<0>();
-            }
-            __syncwarp();
-            uint8_t* lane_off = lane_off0 + static_cast<size_t>(ybuf) * (NYB * BOX_BYTES);
-            if (valid_o) {
-#pragma unroll
-                for (int tr = 0; tr < TR; ++tr) {
-                    const int t = sb * TR + tr;
-                    float z[G], yv[G];
-#pragma unroll
-                    for (int pl = 0; pl < G; ++pl) z[pl] = __uint_as_float(r[pl][t]);
-                    z[0] += b;  // the DC term appears with weight 1 in every output
-                    RealIdft<G>::run(z, yv);
-                    if (p.act == kActGelu) {
-#pragma unroll
-                        for (int g = 0; g < G; g += 2) {
-                            const fx2 u = gelu2(fx2(yv[g], yv[g + 1]));
-                            yv[g] = u.x;
-                            yv[g + 1] = u.y;
-                        }
-                    }
-                    uint8_t* dst = lane_off + tr * (YBC * 2);
-                    if constexpr (G == 2) {
-                        *reinterpret_cast<uint32_t*>(dst) = Io16<T16>::pack(yv[0], yv[1]);
-                    } else if constexpr (G == 4) {
-                        *reinterpret_cast<uint2*>(dst) =
-                            make_uint2(Io16<T16>::pack(yv[0], yv[1]), Io16<T16>::pack(yv[2], yv[3]));
-                    } else {
-#pragma unroll
-                        for (int c = 0; c < G / 8; ++c) {
-                            *reinterpret_cast<uint4*>(dst + 16 * c) = make_uint4(
-                                Io16<T16>::pack(yv[8 * c + 0], yv[8 * c + 1]), Io16<T16>::pack(yv[8 * c + 2], yv[8 * c + 3]),
-                                Io16<T16>::pack(yv[8 * c + 4], yv[8 * c + 5]), Io16<T16>::pack(yv[8 * c + 6], yv[8 * c + 7]));
-                        }
-                    }
-                }
-            }
-            ptx::fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                // every store starts inside the tensor: rows past N and columns past Cout*G
-                // of a started box are clipped, boxes that would start outside are skipped
-                const long long row = n0 + t0 + j * TG + sb * TR;
-                if (row < p.N) {
-                    const uint32_t src = ptx::smem_u32(wstage + static_cast<size_t>(ybuf) * (NYB * BOX_BYTES));
-#pragma unroll
-                    for (int bx = 0; bx < NYB; ++bx) {
-                        const int o_first = oc * kMmaM + q * 32 + bx * (YBC / G);
-                        if (o_first < p.Cout)
-                            ptx::tma_store_2d_h(tmap_y, src + bx * BOX_BYTES, o_first * G, static_cast<int>(row),
-                                                p.l2hint != 0, pol_y);
-                    }
-                }
-                ptx::bulk_commit_group();
-            }
-            if (p.ybufs == 2) ybuf ^= 1;
+        // the buffer about to be written was stored p.ybufs groups ago: wait until read
+        if (lane == 0) {
+            if (p.ybufs == 2) ptx::bulk_wait_group_read<1>();
+            else ptx::bulk_wait_group_read<0>();
         }
+        __syncwarp();
+        uint8_t* lane_off = lane_off0 + static_cast<size_t>(ybuf) * (NYB * BOX_BYTES);
+        if (valid_o) {
+#pragma unroll
+            for (int t = 0; t < TG; ++t) {
+                float z[G], yv[G];
+#pragma unroll
+                for (int pl = 0; pl < G; ++pl) z[pl] = __uint_as_float(r[pl][t]);
+                z[0] += b;  // the DC term appears with weight 1 in every output
+                RealIdft<G>::run(z, yv);
+                if (p.act == kActGelu) {
+#pragma unroll
+                    for (int g = 0; g < G; g += 2) {
+                        const fx2 u = gelu2(fx2(yv[g], yv[g + 1]));
+                        yv[g] = u.x;
+                        yv[g + 1] = u.y;
+                    }
+                }
+                uint8_t* dst = lane_off + t * (YBC * 2);
+                if constexpr (G == 2) {
+                    *reinterpret_cast<uint32_t*>(dst) = Io16<T16>::pack(yv[0], yv[1]);
+                } else if constexpr (G == 4) {
+                    *reinterpret_cast<uint2*>(dst) =
+                        make_uint2(Io16<T16>::pack(yv[0], yv[1]), Io16<T16>::pack(yv[2], yv[3]));
+                } else {
+#pragma unroll
+                    for (int c = 0; c < G / 8; ++c) {
+                        *reinterpret_cast<uint4*>(dst + 16 * c) = make_uint4(
+                            Io16<T16>::pack(yv[8 * c + 0], yv[8 * c + 1]), Io16<T16>::pack(yv[8 * c + 2], yv[8 * c + 3]),
+                            Io16<T16>::pack(yv[8 * c + 4], yv[8 * c + 5]), Io16<T16>::pack(yv[8 * c + 6], yv[8 * c + 7]));
+                    }
+                }
+            }
+        }
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            // every store starts inside the tensor: rows past N and columns past Cout*G
+            // of a started box are clipped, boxes that would start outside are skipped
+            const long long row = n0 + t0 + j * TG;
+            if (row < p.N) {
+                const uint32_t src = ptx::smem_u32(wstage + static_cast<size_t>(ybuf) * (NYB * BOX_BYTES));
+#pragma unroll
+                for (int bx = 0; bx < NYB; ++bx) {
+                    const int o_first = oc * kMmaM + q * 32 + bx * (YBC / G);
+                    if (o_first < p.Cout)
+                        ptx::tma_store_2d_h(tmap_y, src + bx * BOX_BYTES, o_first * G, static_cast<int>(row),
+                                            p.l2hint != 0, pol_y);
+                }
+            }
+            ptx::bulk_commit_group();
+        }
+        if (p.ybufs == 2) ybuf ^= 1;
     }
 }
 
@@ -642,12 +634,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
             if (q < p.yq && oc * kMmaM + q * 32 < p.Cout) {
                 const uint32_t acc = tmem_base + static_cast<uint32_t>(abuf * S::ACC_COLS);
                 const long long n0 = static_cast<long long>(tile) * S::BN;
-                // the two-piece form exists for G <= 4 only (the planner offers it there)
-                if (G <= 4 && p.ysub == 2)
-                    tc::epilogue_tile<G, NACC, T16, (G <= 4 ? 2 : 1)>(p, &tmap_y, acc, q, half, lane, n0, oc, wstage,
-                                                                     ybuf);
-                else
-                    tc::epilogue_tile<G, NACC, T16, 1>(p, &tmap_y, acc, q, half, lane, n0, oc, wstage, ybuf);
+                tc::epilogue_tile<G, NACC, T16>(p, &tmap_y, acc, q, half, lane, n0, oc, wstage, ybuf);
             }
             ptx::tc_fence_before();
             ptx::mbar_arrive(bar_acc_empty(abuf));

@@ -332,7 +332,6 @@ int launch_forward(const Plan& pl, int64_t Cout, int64_t Cin, int64_t G, int sm_
             p.w_region_bytes = pl.w_region_bytes;
             p.ystage_bytes = pl.ystage_bytes;
             p.ybufs = pl.ybufs;
-            p.ysub = pl.ysub;
             p.yq = pl.yq;
             p.y = static_cast<uint8_t*>(y);
             p.w_img_bytes = pl.w_img_bytes;

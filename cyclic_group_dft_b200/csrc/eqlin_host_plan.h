@@ -11,7 +11,6 @@ constexpr size_t kB200SmemOptin = 232448;   // 227 KB opt-in shared memory per C
 constexpr int kB200SmCount = 148;           // SMs of a B200 (host-only planning queries)
 constexpr size_t kSmemAlignSlack = 1024;    // the kernels round their smem base up to 1 KB
 constexpr size_t kSmemCtlBytes = 512;       // mbarriers + control block
-constexpr int kDefaultYSub = 1;             // staged y stores per tokens-on-N epilogue group
 constexpr int kMaxStages = 12;
 constexpr int64_t kMaxChannels = 1 << 16;
 constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per bounded wait
@@ -55,9 +54,8 @@ struct Plan {
     int n_oc = 0;        // output chunks
     int BN = 0;          // tokens per work item
     int stages = 0;
-    int TG = 0;          // y TMA store box rows (tokens-on-N): the epilogue group's tokens / ysub
+    int TG = 0;          // y TMA store box rows (tokens-on-N): the epilogue group's tokens
     int ybufs = 0;       // y staging buffers per epilogue warp (tokens-on-N)
-    int ysub = 1;        // staged y stores per epilogue group (tokens-on-N)
     int yq = 4;          // TMEM lane quarters with output rows, each given y staging (tokens-on-N)
     int box_elems = 0;   // x TMA box columns
     bool x_swizzle128 = false;  // x boxes land SWIZZLE_128B (tokens-on-M, G >= 8)
@@ -71,8 +69,7 @@ struct Plan {
 
 // ----------------------------------------------------------------- planning
 // Tuning overrides read from the environment: EQLIN_MAX_STAGES caps the ring depth,
-// EQLIN_YBUFS (1 or 2) fixes the tokens-on-N y staging depth, EQLIN_YSUB (1 or 2) the
-// staged stores per epilogue group.
+// EQLIN_YBUFS (1 or 2) fixes the tokens-on-N y staging depth.
 int env_int(const char* name, int dflt) {
     const char* e = std::getenv(name);
     if (!e || !*e) return dflt;
@@ -110,15 +107,10 @@ int plan_tn_g(int64_t Cout, int64_t Cin, size_t max_smem, Plan* pl) {
     // Only the TMEM lane quarters that hold output rows get y staging (Cout = 96 leaves the
     // fourth one empty), and the freed space deepens the input ring.
     pl->yq = pl->n_oc == 1 ? static_cast<int>((Cout + 31) / 32) : 4;
-    // The kernel's input ring is latency-bound: each x chunk's stage stays busy for its
-    // load, DFT and MMAs, so stages, not bandwidth, set the rate (B200, p4 C96: 3 stages
-    // 72.5 us, 4 stages 65.1 us).  Staging each epilogue group as two pieces of TG/2
-    // rows halves the staging space (G <= 4 only; p4 C96 measured slower with it: 72.0 us
-    // with 6 stages against 65.3 us with 5, so it is off by default).
-    pl->ysub = env_int("EQLIN_YSUB", kDefaultYSub) == 2 && G <= 4 && S::TG % 2 == 0 ? 2 : 1;
-    pl->TG = S::TG / pl->ysub;
-    // y staging: per active epilogue warp, ybufs buffers of TG/ysub rows x 32*G 16-bit
-    // columns; double-buffered when at least 4 ring stages still fit
+    pl->TG = S::TG;
+    // y staging: per active epilogue warp, ybufs buffers of TG rows x 32*G 16-bit columns;
+    // double-buffered when at least 4 ring stages still fit (B200, p4 C96: 3 stages 72.5 us,
+    // 4 stages 60.9 us, 5 stages 60.1 us)
     const size_t ybuf = static_cast<size_t>(pl->TG) * 32 * G * 2;
     auto fixed_for = [&](int nb) {
         return kSmemAlignSlack + kSmemCtlBytes + static_cast<size_t>(2 * pl->yq) * nb * ybuf;
@@ -205,7 +197,6 @@ int plan_tnr_g(int64_t Cout, int64_t Cin, size_t max_smem, bool forced, Plan* pl
         pl->n_oc = n_oc;
         pl->BN = S::BN;
         pl->TG = S::TG;
-        pl->ysub = 1;
         pl->yq = 4;
         pl->box_elems = S::BOX_ELEMS;
         pl->ybufs = nb;

@@ -156,17 +156,15 @@ def test_edge_channel_counts(Cout, Cin, G, kernel, monkeypatch):
     h.close()
 
 
-@pytest.mark.parametrize("ystore", ["tma", "tma_pieces", "direct"])
+@pytest.mark.parametrize("ystore", ["tma", "direct"])
 @pytest.mark.parametrize("Cout,Cin,G", [(50, 40, 4), (96, 96, 4), (200, 32, 4), (130, 96, 4), (96, 96, 2),
                                         (136, 64, 8), (768, 192, 4), (70, 64, 4), (16, 32, 16)])
 def test_tokens_on_n_store_modes(Cout, Cin, G, ystore, monkeypatch):
-    """Every way the tokens-on-N epilogues write y (TMA stores of a staged group, of a
-    group staged as two pieces, plain coalesced stores), for both tokens-on-N kernels,
-    with a ragged token tail.  Cout = 50, 70, 96 and 16 leave TMEM lane quarters empty,
-    which get no staging."""
+    """Both ways the tokens-on-N epilogues write y (TMA stores of a staged group, plain
+    coalesced stores), for both tokens-on-N kernels, with a ragged token tail.  Cout = 50,
+    70, 96 and 16 leave TMEM lane quarters empty, which get no staging."""
     monkeypatch.setenv("EQLIN_KERNEL", "tnr")
-    monkeypatch.setenv("EQLIN_YSTORE", "direct" if ystore == "direct" else "tma")
-    monkeypatch.setenv("EQLIN_YSUB", "2" if ystore == "tma_pieces" else "1")
+    monkeypatch.setenv("EQLIN_YSTORE", ystore)
     gen = torch.Generator().manual_seed(Cout * 1000 + Cin * 10 + G + 17)
     N = 1031
     x = torch.randn(N, Cin, G, generator=gen).to(torch.bfloat16)
