@@ -415,6 +415,41 @@ def time_back_to_back(ctx: Ctx, fn, K: int, clocks: ClockSampler | None = None, 
     return reduce_max(t0.elapsed_time(t1), ctx.dev)
 
 
+def host_link_rates(dev, x_pin, x_dev, y_dev, y_pin, N: int, reps: int = 3) -> dict:
+    """The host link's own rates for the bytes e2e moves: one pinned host -> device copy of
+    x, one device -> host copy of y, and both at once on two streams (the host-buffer path
+    overlaps them), each the best of `reps`, from CUDA events.  `bound_tokens_per_s` is the
+    e2e rate the concurrent copies alone allow."""
+    main = torch.cuda.current_stream(dev)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
+    def timed(use_in: bool, use_out: bool) -> float:
+        best = float("inf")
+        for _ in range(reps):
+            torch.cuda.synchronize(dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(main)
+            for st, use, fn in ((s_in, use_in, lambda: x_dev.copy_(x_pin, non_blocking=True)),
+                                (s_out, use_out, lambda: y_pin.copy_(y_dev, non_blocking=True))):
+                if use:
+                    st.wait_event(e0)
+                    with torch.cuda.stream(st):
+                        fn()
+                    done = torch.cuda.Event()
+                    done.record(st)
+                    main.wait_event(done)
+            e1.record(main)
+            torch.cuda.synchronize(dev)
+            best = min(best, e0.elapsed_time(e1) * 1e-3)
+        return best
+
+    bx, by = x_pin.numel() * x_pin.element_size(), y_pin.numel() * y_pin.element_size()
+    t_in, t_out, t_both = timed(True, False), timed(False, True), timed(True, True)
+    return {"h2d_gbs": bx / t_in / 1e9, "d2h_gbs": by / t_out / 1e9, "both_s": t_both,
+            "both_gbs": (bx + by) / t_both / 1e9, "bound_tokens_per_s": N / t_both,
+            "method": "pinned cudaMemcpyAsync of the step's x and y, best of 3, CUDA events"}
+
+
 def setup_workload(ctx: Ctx, wl: workloads.Workload, args) -> dict:
     """Seeded inputs on the host, the prepared handle and the rotating x/y sets on the
     device (everything a workload's measurement needs, before any of it is timed)."""
@@ -525,7 +560,8 @@ def measure_workload(ctx: Ctx, wl: workloads.Workload, K: int, warmup: int, head
                       "h2d_bytes_per_step": x_pin.numel() * x_pin.element_size(),
                       "d2h_bytes_per_step": y_pin.numel() * y_pin.element_size(),
                       "api": "eqlin_forward_host (C ABI: pinned host x and y, chunked copies in and out "
-                             "overlapping the fused kernel on two streams)"}
+                             "overlapping the fused kernel on two streams)",
+                      "link": host_link_rates(dev, x_pin, xs[0], ys[0], y_pin, N)}
         del x_pin, y_pin
 
     # ------------------------------------------------------- backward calls

@@ -86,3 +86,30 @@ def test_both_arms_share_the_config():
     assert set(c) == {"workload", "N", "Cin", "Cout", "G", "io", "global_batch", "parallelism", "l2"}
     assert c["N"] == 64 * 56 * 56 and c["workload"] == "p4_c96_bf16"
     assert b.BENCH_WORKLOADS == ("tiny_p4_fp32", "p4_c96_bf16", "p8_c64_bf16", "p4_mlp_bf16", "c16_c32_bf16")
+
+
+def test_clock_sampler_stays_out_of_short_timed_regions(monkeypatch):
+    """The clock sampler queries NVML before the warm-up (begin) and right after the timed
+    region (stop); while the region runs its thread waits one period before its first
+    query, so a region shorter than the period sees no query.  A fake NVML counts them."""
+    import threading
+    import types
+    calls = []
+    fake = types.SimpleNamespace(
+        NVML_CLOCK_SM=0,
+        nvmlInit=lambda: None,
+        nvmlDeviceGetHandleByIndex=lambda i: "h",
+        nvmlDeviceGetMaxClockInfo=lambda h, c: 1965,
+        nvmlDeviceGetClockInfo=lambda h, c: calls.append(threading.current_thread().name) or 1965,
+        nvmlDeviceGetCurrentClocksEventReasons=lambda h: 0,
+    )
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    b = _bench()
+    c = b.ClockSampler(0, period_s=0.5)
+    c.begin()
+    assert len(calls) == 1
+    c.start()
+    c.stop()                      # a region far shorter than the period
+    assert len(calls) == 2        # begin and stop only: nothing from the thread
+    s = c.summary()
+    assert s["sm_mhz"] == 1965 and s["samples"] == 2 and "before the warm-up" in s["sampling"]

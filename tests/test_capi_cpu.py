@@ -191,6 +191,33 @@ def test_planner_weight_gradient_chunks(G, tokens):
     assert q["dw_tile_rows"] % 16 == 0 and q["dw_tile_cols"] % 16 == 0
 
 
+@pytest.mark.parametrize("Cout,Cin,G,rows,cols", [(96, 96, 4, 96, 96), (768, 192, 4, 128, 96),
+                                                    (192, 768, 4, 96, 128), (64, 64, 8, 64, 64),
+                                                    (32, 32, 16, 32, 32)])
+def test_planner_weight_gradient_tiles(Cout, Cin, G, rows, cols):
+    """Weight-gradient tiles: the fewest units, then the least padded area (192 input
+    channels as 2 x 96, not 128 + 64)."""
+    q = eq.query_plan(Cout, Cin, G)
+    assert (q["dw_tile_rows"], q["dw_tile_cols"]) == (rows, cols)
+
+
+def test_planner_tokens_on_m_weight_image():
+    """Tokens-on-M weight image: the G planes in plane order up to G = 8 (p8 C64: 64 KB, so
+    four 32 KB ring stages fit), the pair slots at G = 16 (C16 C32: 23 slots, 46 KB)."""
+    q = eq.query_plan(64, 64, 8)
+    assert "tokens_on_m" in q["path_name"] and q["weight_bytes"] == 8 * 64 * 32 * 4 and q["stages"] == 4
+    q = eq.query_plan(32, 32, 16)
+    assert "tokens_on_m" in q["path_name"] and q["weight_bytes"] == 23 * 32 * 32 * 2
+
+
+def test_planner_y_staging_only_for_used_lane_quarters():
+    """Tokens-on-N with one output chunk: Cout = 96 uses 3 of the 4 TMEM lane quarters, so
+    only 3 x 2 warps get y staging and the input ring gets a fifth stage."""
+    q = eq.query_plan(96, 96, 4)
+    assert q["path_name"] == "tcgen05_tokens_on_n_resident_weights"
+    assert q["stages"] == 5 and q["y_staging"] == 2
+
+
 def test_planner_environment_overrides(monkeypatch):
     monkeypatch.setenv("EQLIN_KERNEL", "tm")
     assert "tokens_on_m" in eq.query_plan(96, 96, 4)["path_name"]
