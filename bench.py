@@ -155,16 +155,16 @@ def line_config(wl: workloads.Workload, world: int) -> dict:
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    """Samples SM clock and clock-event reasons through NVML: once before the warm-up
-    launches (begin), every period_s in a thread while the timed region runs, and once
-    right after it (stop).  The first in-region sample comes one period after the start:
-    an NVML query just before or while the kernels run slows them (B200, p4 C96, 20
-    back-to-back launches: 62.4 us per launch with 10 ms sampling from the start against
-    60.2 us without; 61.8 us with one query just before the start), so a region shorter
-    than one period is bracketed by the samples around it instead.  Construct it (NVML
-    initialisation) before the warm-up too: a host delay between the warm-up and the
-    timed region lets the GPU idle, and the region then starts slow (63.0 us after a
-    20 ms pause)."""
+    """Samples SM clock and clock-event reasons through NVML: every period_s in a thread
+    while the timed region runs (the first one period after its start) and once right
+    after it (stop).  An NVML query just before or while the kernels run slows them
+    (B200, p4 C96, 20 back-to-back launches: 62.4 us per launch with 10 ms sampling from
+    the start against 60.2 us without, 61.8 us with one query just before the start, still
+    1 us slower with one query before the 5 warm-up launches), so a region shorter than
+    one period is represented by the sample taken right after it.  Construct it (NVML
+    initialisation) before the warm-up: a host delay between the warm-up and the timed
+    region lets the GPU idle, and the region then starts slow (63.0 us after a 20 ms
+    pause)."""
 
     def __init__(self, device_index: int, period_s: float = 0.05):
         self.samples: list[tuple[int, int]] = []
@@ -203,10 +203,6 @@ class ClockSampler:
         while not self._stop.wait(self.period):
             self._sample()
 
-    def begin(self):
-        if self._nvml is not None:
-            self._sample()
-
     def start(self):
         if self._nvml is not None:
             self._thread = threading.Thread(target=self._run, daemon=True)
@@ -229,8 +225,8 @@ class ClockSampler:
         reasons = [name for bit, name in REASON_BITS.items() if bits & bit and name != "gpu_idle"]
         return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": reasons,
                 "samples": len(self.samples),
-                "sampling": f"NVML, before the warm-up launches, right after the timed region and every "
-                            f"{self.period * 1e3:.0f} ms inside it"}
+                "sampling": f"NVML, every {self.period * 1e3:.0f} ms inside the timed region (the first one "
+                            "period after its start) and right after it"}
 
 
 # ------------------------------------------------------------------ CPU oracle
@@ -506,8 +502,6 @@ def measure_workload(ctx: Ctx, wl: workloads.Workload, K: int, warmup: int, head
     # dependent launch), which is how the kernel runs in a real stream of layers.
     # The average launch duration of the kernel is therefore elapsed / K.
     clocks = ClockSampler(dev.index) if headline else None
-    if clocks is not None:
-        clocks.begin()
     for i in range(warmup):
         fwd(i)
     elapsed_ms = time_back_to_back(ctx, fwd_c, K, clocks, graph=ctx.graph)

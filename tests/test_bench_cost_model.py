@@ -89,9 +89,9 @@ def test_both_arms_share_the_config():
 
 
 def test_clock_sampler_stays_out_of_short_timed_regions(monkeypatch):
-    """The clock sampler queries NVML before the warm-up (begin) and right after the timed
-    region (stop); while the region runs its thread waits one period before its first
-    query, so a region shorter than the period sees no query.  A fake NVML counts them."""
+    """The clock sampler queries NVML right after the timed region (stop); while the region
+    runs its thread waits one period before its first query, so a region shorter than the
+    period sees no query at all.  A fake NVML counts them."""
     import threading
     import types
     calls = []
@@ -106,10 +106,15 @@ def test_clock_sampler_stays_out_of_short_timed_regions(monkeypatch):
     monkeypatch.setitem(sys.modules, "pynvml", fake)
     b = _bench()
     c = b.ClockSampler(0, period_s=0.5)
-    c.begin()
-    assert len(calls) == 1
+    assert not calls              # constructing it queries no clock
     c.start()
     c.stop()                      # a region far shorter than the period
-    assert len(calls) == 2        # begin and stop only: nothing from the thread
+    assert len(calls) == 1        # the sample right after the region only
     s = c.summary()
-    assert s["sm_mhz"] == 1965 and s["samples"] == 2 and "before the warm-up" in s["sampling"]
+    assert s["sm_mhz"] == 1965 and s["samples"] == 1 and "right after it" in s["sampling"]
+    calls.clear()
+    c = b.ClockSampler(0, period_s=0.01)
+    c.start()
+    threading.Event().wait(0.1)   # a region of ten periods is sampled inside
+    c.stop()
+    assert len(calls) >= 5
