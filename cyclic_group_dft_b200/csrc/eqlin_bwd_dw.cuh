@@ -521,9 +521,11 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
 
 // Cross-CTA reduction and inverse DFT, deterministic, in one small kernel.
 // Block = (unit u, column ii of the unit, 32 consecutive rows oo), or the unit's bias
-// sums when ii == NI.  Warp w sums the slabs of splits w, w+8, w+16, ... in that order,
-// float64, for the block's G planes, with kIn splits (kIn * G loads per thread) in
-// flight per round trip; the 8 warp sums are then added in warp order.  Launched as a
+// sums when ii == NI.  Warp w of the block's W warps sums the slabs of splits w, w+W,
+// w+2W, ... in that order, float64, for the block's G planes, with kIn splits (kIn * G
+// loads per thread) in flight per round trip; the W warp sums are then added in warp
+// order.  W = 16 (8 at G = 16, whose float64 partial sums would not fit 48 KB of static
+// shared memory): 148 splits then take one round trip per warp, not three.  Launched as a
 // programmatic dependent of the main kernel: its blocks start as that kernel's CTAs
 // exit and wait (griddepcontrol.wait) for all of its slabs before reading them.
 // With P_k = sum_n DY_k conj(X_k) (unscaled transforms), warp 0 writes
@@ -539,8 +541,12 @@ struct DwFinalParams {
 };
 
 template <int G>
-__global__ void __launch_bounds__(256) eqlin_dw_finish_kernel(const DwFinalParams f) {
-    __shared__ double red[8][G][32];
+constexpr int dw_finish_warps() { return G <= 8 ? 16 : 8; }
+
+template <int G>
+__global__ void __launch_bounds__(dw_finish_warps<G>() * 32) eqlin_dw_finish_kernel(const DwFinalParams f) {
+    constexpr int W = dw_finish_warps<G>();
+    __shared__ double red[W][G][32];
     ptx::grid_launch_dependents();
     ptx::grid_dependency_wait();
     const int n_og = (f.MO + 31) / 32;
@@ -562,13 +568,13 @@ __global__ void __launch_bounds__(256) eqlin_dw_finish_kernel(const DwFinalParam
         int s = warp;
         // kIn splits in flight (kIn * G <= 32 loads per thread), added in split order
         constexpr int kIn = 32 / G > 2 ? 32 / G : 2;
-        for (; s + 8 * (kIn - 1) < f.n_splits; s += 8 * kIn) {
+        for (; s + W * (kIn - 1) < f.n_splits; s += W * kIn) {
             float v[kIn][G];
 #pragma unroll
             for (int u = 0; u < kIn; ++u) {
 #pragma unroll
                 for (int pl = 0; pl < G; ++pl)
-                    if (pl < nv) v[u][pl] = src[static_cast<size_t>(s + 8 * u) * stride + pl * pstride];
+                    if (pl < nv) v[u][pl] = src[static_cast<size_t>(s + W * u) * stride + pl * pstride];
             }
 #pragma unroll
             for (int u = 0; u < kIn; ++u) {
@@ -577,7 +583,7 @@ __global__ void __launch_bounds__(256) eqlin_dw_finish_kernel(const DwFinalParam
                     if (pl < nv) acc[pl] += v[u][pl];
             }
         }
-        for (; s < f.n_splits; s += 8) {
+        for (; s < f.n_splits; s += W) {
 #pragma unroll
             for (int pl = 0; pl < G; ++pl)
                 if (pl < nv) acc[pl] += src[static_cast<size_t>(s) * stride + pl * pstride];
@@ -592,7 +598,7 @@ __global__ void __launch_bounds__(256) eqlin_dw_finish_kernel(const DwFinalParam
     for (int pl = 0; pl < G; ++pl) {
         double v = 0.0;
 #pragma unroll
-        for (int w = 0; w < 8; ++w) v += red[w][pl][lane];
+        for (int w = 0; w < W; ++w) v += red[w][pl][lane];
         z[pl] = v;
     }
     const int ot = unit / f.n_it, it = unit % f.n_it;

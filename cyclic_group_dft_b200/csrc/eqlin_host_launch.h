@@ -470,7 +470,7 @@ int launch_dw(const DwPlan& pl, bool f32_path, int64_t Cout, int64_t Cin, int64_
     // a programmatic dependent of the main kernel (its blocks wait for the slabs)
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(fgrid);
-    cfg.blockDim = dim3(256);
+    cfg.blockDim = dim3(iG <= 8 ? 16 * 32 : 8 * 32);   // eqlin::dw_finish_warps<G>() warps
     cfg.dynamicSmemBytes = 0;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];

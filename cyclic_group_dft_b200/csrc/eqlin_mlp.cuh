@@ -533,7 +533,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
 // once.  Warp = token; lanes stride over the hidden channels, then over the outputs.
 // w1_f64 [G][Cin][H] and w2_f64 [G][H][Cout] are the scaled planes of eqlin_layout.h.
 template <int G>
-__global__ void __launch_bounds__(kF32Threads)
+__global__ void __launch_bounds__(kF32Threads, 1)
     eqlin_mlp_f32_kernel(const float* __restrict__ x, const double* __restrict__ w1_f64,
                          const double* __restrict__ b1_f64, const double* __restrict__ w2_f64,
                          const double* __restrict__ b2_f64, float* __restrict__ y, long long N, int Cin, int H,
