@@ -524,8 +524,8 @@ __global__ void __launch_bounds__(dw::Cfg<G>::kThreads, 1)
 // sums when ii == NI.  Warp w of the block's W warps sums the slabs of splits w, w+W,
 // w+2W, ... in that order, float64, for the block's G planes, with kIn splits (kIn * G
 // loads per thread) in flight per round trip; the W warp sums are then added in warp
-// order.  W = 16 (8 at G = 16, whose float64 partial sums would not fit 48 KB of static
-// shared memory): 148 splits then take one round trip per warp, not three.  Launched as a
+// order.  W = 16: 148 splits then take one round trip per warp, not three.  The W x G x 32
+// float64 warp sums live in dynamic shared memory (64 KB at G = 16).  Launched as a
 // programmatic dependent of the main kernel: its blocks start as that kernel's CTAs
 // exit and wait (griddepcontrol.wait) for all of its slabs before reading them.
 // With P_k = sum_n DY_k conj(X_k) (unscaled transforms), warp 0 writes
@@ -540,13 +540,13 @@ struct DwFinalParams {
     size_t slab_floats;   // G * NI * MO
 };
 
-template <int G>
-constexpr int dw_finish_warps() { return G <= 8 ? 16 : 8; }
+constexpr int kDwFinishWarps = 16;
 
 template <int G>
-__global__ void __launch_bounds__(dw_finish_warps<G>() * 32) eqlin_dw_finish_kernel(const DwFinalParams f) {
-    constexpr int W = dw_finish_warps<G>();
-    __shared__ double red[W][G][32];
+__global__ void __launch_bounds__(kDwFinishWarps * 32) eqlin_dw_finish_kernel(const DwFinalParams f) {
+    constexpr int W = kDwFinishWarps;
+    extern __shared__ double red_sm[];   // [W][G][32]
+    auto red = [&](int w, int pl) -> double& { return red_sm[(w * G + pl) * 32 + (threadIdx.x & 31)]; };
     ptx::grid_launch_dependents();
     ptx::grid_dependency_wait();
     const int n_og = (f.MO + 31) / 32;
@@ -590,7 +590,7 @@ __global__ void __launch_bounds__(dw_finish_warps<G>() * 32) eqlin_dw_finish_ker
         }
     }
 #pragma unroll
-    for (int pl = 0; pl < G; ++pl) red[warp][pl][lane] = acc[pl];
+    for (int pl = 0; pl < G; ++pl) red(warp, pl) = acc[pl];
     __syncthreads();
     if (warp != 0 || oo >= f.MO) return;
     double z[G];
@@ -598,7 +598,7 @@ __global__ void __launch_bounds__(dw_finish_warps<G>() * 32) eqlin_dw_finish_ker
     for (int pl = 0; pl < G; ++pl) {
         double v = 0.0;
 #pragma unroll
-        for (int w = 0; w < W; ++w) v += red[w][pl][lane];
+        for (int w = 0; w < W; ++w) v += red(w, pl);
         z[pl] = v;
     }
     const int ot = unit / f.n_it, it = unit % f.n_it;

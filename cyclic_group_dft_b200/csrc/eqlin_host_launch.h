@@ -470,14 +470,19 @@ int launch_dw(const DwPlan& pl, bool f32_path, int64_t Cout, int64_t Cin, int64_
     // a programmatic dependent of the main kernel (its blocks wait for the slabs)
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(fgrid);
-    cfg.blockDim = dim3(iG <= 8 ? 16 * 32 : 8 * 32);   // eqlin::dw_finish_warps<G>() warps
-    cfg.dynamicSmemBytes = 0;
+    cfg.blockDim = dim3(eqlin::kDwFinishWarps * 32);
+    cfg.dynamicSmemBytes = static_cast<size_t>(eqlin::kDwFinishWarps) * iG * 32 * sizeof(double);
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = use_pdl() ? 1 : 0;
+    // 64 KB of warp sums at G = 16: above the default 48 KB, opted in on the current device
+    if (iG == 16 && (e = cudaFuncSetAttribute(eqlin::eqlin_dw_finish_kernel<16>,
+                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              static_cast<int>(cfg.dynamicSmemBytes))) != cudaSuccess)
+        return cuda_fail(e, "cudaFuncSetAttribute (weight-gradient reduction)");
     switch (iG) {
         case 2: e = cudaLaunchKernelEx(&cfg, eqlin::eqlin_dw_finish_kernel<2>, f); break;
         case 4: e = cudaLaunchKernelEx(&cfg, eqlin::eqlin_dw_finish_kernel<4>, f); break;
