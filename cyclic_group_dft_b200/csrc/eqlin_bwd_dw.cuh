@@ -554,7 +554,7 @@ __global__ void __launch_bounds__(kDwFinishWarps * 32) eqlin_dw_finish_kernel(co
     const int unit = static_cast<int>(blockIdx.x) / per_unit;
     const int rem = static_cast<int>(blockIdx.x) % per_unit;
     const int ii = rem / n_og, oo = (rem % n_og) * 32 + (threadIdx.x & 31);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
     const bool bias_blk = ii == f.NI;
     const size_t stride = f.slab_floats + f.MO;
     const size_t pstride = static_cast<size_t>(f.NI) * f.MO;   // between planes of a slab

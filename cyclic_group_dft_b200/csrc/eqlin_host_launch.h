@@ -252,12 +252,24 @@ int launch_forward(const Plan& pl, int64_t Cout, int64_t Cin, int64_t G, int sm_
         const float* xf = static_cast<const float*>(x);
         float* yf = static_cast<float*>(y);
         const int iCin = static_cast<int>(Cin), iCout = static_cast<int>(Cout);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = grid;
+        cfg.blockDim = dim3(eqlin::kF32Threads);
+        cfg.dynamicSmemBytes = pl.smem_bytes;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = use_pdl() ? 1 : 0;
+        cudaError_t e;
         switch (iG) {
-            case 2: eqlin::eqlin_fwd_f32_kernel<2><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, b.w_f64, b.bias_f64, yf, N, iCin, iCout, b.act); break;
-            case 4: eqlin::eqlin_fwd_f32_kernel<4><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, b.w_f64, b.bias_f64, yf, N, iCin, iCout, b.act); break;
-            case 8: eqlin::eqlin_fwd_f32_kernel<8><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, b.w_f64, b.bias_f64, yf, N, iCin, iCout, b.act); break;
-            default: eqlin::eqlin_fwd_f32_kernel<16><<<grid, eqlin::kF32Threads, pl.smem_bytes, st>>>(xf, b.w_f64, b.bias_f64, yf, N, iCin, iCout, b.act); break;
+            case 2: e = cudaLaunchKernelEx(&cfg, eqlin::eqlin_fwd_f32_kernel<2>, xf, b.w_f64, b.bias_f64, yf, N, iCin, iCout, b.act); break;
+            case 4: e = cudaLaunchKernelEx(&cfg, eqlin::eqlin_fwd_f32_kernel<4>, xf, b.w_f64, b.bias_f64, yf, N, iCin, iCout, b.act); break;
+            case 8: e = cudaLaunchKernelEx(&cfg, eqlin::eqlin_fwd_f32_kernel<8>, xf, b.w_f64, b.bias_f64, yf, N, iCin, iCout, b.act); break;
+            default: e = cudaLaunchKernelEx(&cfg, eqlin::eqlin_fwd_f32_kernel<16>, xf, b.w_f64, b.bias_f64, yf, N, iCin, iCout, b.act); break;
         }
+        if (e != cudaSuccess) return cuda_fail(e, "fp32 forward launch");
     } else {
         auto encode = tensor_map_encoder();
         if (!encode) return fail(EQLIN_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");

@@ -15,6 +15,7 @@
 #include "eqlin_layout.h"
 #include "group_dft.cuh"
 #include "io16.cuh"
+#include "sm100_ptx.cuh"
 
 namespace eqlin {
 
@@ -135,6 +136,10 @@ __global__ void __launch_bounds__(kF32Threads)
                          const double* __restrict__ bias_f64, float* __restrict__ y, long long N,
                          int Cin, int Cout, int act) {
     extern __shared__ double xs[];  // [kF32Tokens][G][Cin] spectrum of the block's tokens
+    // launched as a programmatic dependent: the next kernel of the stream may start its
+    // blocks as these exit, and x and y are touched only once the previous one has completed
+    ptx::grid_launch_dependents();
+    ptx::grid_dependency_wait();
     const long long n0 = static_cast<long long>(blockIdx.x) * kF32Tokens;
     for (int idx = threadIdx.x; idx < kF32Tokens * Cin; idx += kF32Threads) {
         const int t = idx / Cin, i = idx % Cin;
