@@ -224,9 +224,11 @@ __device__ __forceinline__ void dft_chunk(uint8_t* xs, int dft_tid) {
 // TMEM is read in batches of EB = 2 groups (G x 2*OG = 64 registers), so a warp waits for
 // half as many TMEM loads; the batch's biases are loaded before the wait.
 // Per group: inverse real DFT + bias (channel pairs packed as fx2), bf16, one 64-byte row
-// per lane into the warp's own SWIZZLE_64B staging tile [32 tokens x 32 columns]
-// (double-buffered), and lane 0 stores it with TMA; the epilogue warps never wait for one
-// another.  Arrives on `acc_empty` once its last TMEM load has landed.
+// per lane into a SWIZZLE_64B staging tile [32 tokens x 32 columns] of the warp's own; a
+// batch's EB groups take the warp's EB tiles, then one proxy fence and lane 0's TMA stores
+// of all of them under one commit group (so the next batch waits once for the previous
+// batch's tiles to be read); the epilogue warps never wait for one another.  Arrives on
+// `acc_empty` once its last TMEM load has landed.
 template <int G, class T16>
 __device__ __forceinline__ void epilogue_tile(const TmParams& p, const CUtensorMap* tmap_y, uint32_t tmem,
                                               int q, int half, int lane, long long n0, int oc, uint8_t* wstage,
@@ -234,6 +236,7 @@ __device__ __forceinline__ void epilogue_tile(const TmParams& p, const CUtensorM
     using C = Cfg<G>;
     constexpr int OG = C::OG;
     constexpr int EB = 2;                          // groups per TMEM load batch
+    static_assert(EB <= kYWarpBufs, "a batch's groups take the warp's staging tiles");
     const int n_groups = (p.NO / 2) / OG;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const long long row0 = n0 + q * 32;            // first token of this warp's rows
@@ -264,7 +267,6 @@ __device__ __forceinline__ void epilogue_tile(const TmParams& p, const CUtensorM
 #pragma unroll
         for (int gi = 0; gi < EB; ++gi) {
             if (g0 + gi >= n_groups) break;
-            const int o0 = oc * p.NO + o_loc0 + gi * OG;
             // the lane's staging row: OG channels x G outputs, channel-major, packed in pairs
             uint32_t pk[OG * G / 2];
 #pragma unroll
@@ -285,27 +287,32 @@ __device__ __forceinline__ void epilogue_tile(const TmParams& p, const CUtensorM
                     pk[((j + 1) * G + gg) / 2] = Io16<T16>::pack(y2[gg].y, y2[gg + 1].y);
                 }
             }
-            // this buffer was last stored two groups ago: its TMA read must be complete
-            if (lane == 0) ptx::bulk_wait_group_read<1>();
-            __syncwarp();
-            uint8_t* buf = wstage + static_cast<size_t>(ybuf) * kYWarpBufBytes;
-            uint8_t* rowp = buf + lane * (kYCols * 2);
+            if (gi == 0) {
+                // the previous batch's tiles (one commit group) must have been read
+                if (lane == 0) ptx::bulk_wait_group_read<0>();
+                __syncwarp();
+            }
+            uint8_t* rowp = wstage + static_cast<size_t>(gi) * kYWarpBufBytes + lane * (kYCols * 2);
 #pragma unroll
             for (int k = 0; k < 4; ++k)
                 *reinterpret_cast<uint4*>(rowp + ((k ^ swz) * 16)) =
                     make_uint4(pk[4 * k + 0], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
-            ptx::fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
+        }
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+#pragma unroll
+            for (int gi = 0; gi < EB; ++gi) {
+                const int o0 = oc * p.NO + o_loc0 + gi * OG;
                 // a store only starts inside the tensor; its clipped parts are not written
-                if (row0 < p.N && o0 < p.Cout)
-                    ptx::tma_store_2d_h(tmap_y, ptx::smem_u32(buf), o0 * G, static_cast<int>(row0), p.l2hint != 0,
-                                        pol_y);
-                ptx::bulk_commit_group();
+                if (g0 + gi < n_groups && row0 < p.N && o0 < p.Cout)
+                    ptx::tma_store_2d_h(tmap_y, ptx::smem_u32(wstage + static_cast<size_t>(gi) * kYWarpBufBytes),
+                                        o0 * G, static_cast<int>(row0), p.l2hint != 0, pol_y);
             }
-            ybuf ^= 1;
+            ptx::bulk_commit_group();
         }
     }
+    (void)ybuf;
 }
 
 }  // namespace tm
