@@ -45,31 +45,47 @@ struct eqlin_handle {
     DwPlan dwp;          // weight-gradient tiling (bf16 I/O)
     bool sync_check = false;
     unsigned long long timeout_ns = kDefaultTimeoutNs;
-    // eqlin_forward_host: device staging for two chunks, two streams, created on first use
+    // eqlin_forward_host: device staging for kHostBufs chunks and three streams (copies
+    // in, kernels, copies out), created on first use
+    static constexpr int kHostBufs = 4;
     std::mutex host_mutex;
     int64_t host_chunk = 0;                     // tokens per chunk (0: not set up)
-    void* host_x[2] = {nullptr, nullptr};
-    void* host_y[2] = {nullptr, nullptr};
-    cudaStream_t host_st[2] = {nullptr, nullptr};
-    cudaEvent_t host_ev_in = nullptr;
-    cudaEvent_t host_ev_out[2] = {nullptr, nullptr};
+    int64_t host_seq = 0;                       // chunks issued so far, over all calls
+    void* host_x[kHostBufs] = {};
+    void* host_y[kHostBufs] = {};
+    cudaStream_t host_in = nullptr, host_run = nullptr, host_out = nullptr;
+    cudaEvent_t host_ev_start = nullptr, host_ev_done = nullptr;
+    cudaEvent_t host_ev_in[kHostBufs] = {};    // chunk's x copied in
+    cudaEvent_t host_ev_run[kHostBufs] = {};   // chunk's kernel done (x buffer free, y ready)
+    cudaEvent_t host_ev_out[kHostBufs] = {};   // chunk's y copied out (y buffer free)
 };
 
 namespace {
 
 void release_host_staging(eqlin_handle* h) {
-    for (int k = 0; k < 2; ++k) {
+    auto free_event = [](cudaEvent_t& ev) {
+        if (ev) cudaEventDestroy(ev);
+        ev = nullptr;
+    };
+    auto free_stream = [](cudaStream_t& st) {
+        if (st) cudaStreamDestroy(st);
+        st = nullptr;
+    };
+    for (int k = 0; k < eqlin_handle::kHostBufs; ++k) {
         if (h->host_x[k]) cudaFree(h->host_x[k]);
         if (h->host_y[k]) cudaFree(h->host_y[k]);
-        if (h->host_st[k]) cudaStreamDestroy(h->host_st[k]);
-        if (h->host_ev_out[k]) cudaEventDestroy(h->host_ev_out[k]);
         h->host_x[k] = h->host_y[k] = nullptr;
-        h->host_st[k] = nullptr;
-        h->host_ev_out[k] = nullptr;
+        free_event(h->host_ev_in[k]);
+        free_event(h->host_ev_run[k]);
+        free_event(h->host_ev_out[k]);
     }
-    if (h->host_ev_in) cudaEventDestroy(h->host_ev_in);
-    h->host_ev_in = nullptr;
+    free_stream(h->host_in);
+    free_stream(h->host_run);
+    free_stream(h->host_out);
+    free_event(h->host_ev_start);
+    free_event(h->host_ev_done);
     h->host_chunk = 0;
+    h->host_seq = 0;
 }
 
 void free_handle(eqlin_handle* h) {
@@ -91,29 +107,33 @@ void free_handle(eqlin_handle* h) {
 
 size_t io_elem_bytes(int io) { return io == EQLIN_F32 ? 4 : 2; }
 
-// Staging of eqlin_forward_host: chunks of about 16 MB of x plus y (a multiple of 64
-// tokens), two of each, and two non-blocking streams.  Called with host_mutex held.
+// Staging of eqlin_forward_host: kHostBufs chunks of about 16 MB of x plus y (a multiple
+// of 64 tokens) and three non-blocking streams.  Measured on B200 at p4 C96 (200704
+// tokens, pinned host memory): each chunk costs about 20 us beyond its copies, so 4 and
+// 8 MB chunks were slower (4.0e7 and 4.9e7 tokens/s against 5.4e7 on one box); 64 MB
+// chunks lose on the pipeline's fill and drain.  Called with host_mutex held.
 int setup_host_staging(eqlin_handle* h) {
     if (h->host_chunk > 0) return EQLIN_OK;
     const size_t e = io_elem_bytes(h->io_dtype);
     const size_t row_x = static_cast<size_t>(h->Cin * h->G) * e, row_y = static_cast<size_t>(h->Cout * h->G) * e;
     int64_t tokens = static_cast<int64_t>((size_t(16) << 20) / (row_x + row_y)) / 64 * 64;
     tokens = std::max<int64_t>(tokens, 64);
-    cudaError_t err;
-    for (int k = 0; k < 2; ++k) {
-        if ((err = cudaMalloc(&h->host_x[k], tokens * row_x)) != cudaSuccess ||
-            (err = cudaMalloc(&h->host_y[k], tokens * row_y)) != cudaSuccess) {
+    cudaError_t err = cudaSuccess;
+    for (int k = 0; k < eqlin_handle::kHostBufs; ++k) {
+        if (cudaMalloc(&h->host_x[k], tokens * row_x) != cudaSuccess ||
+            cudaMalloc(&h->host_y[k], tokens * row_y) != cudaSuccess) {
             cudaGetLastError();
             release_host_staging(h);   // nothing half set up survives a failure
             return fail(EQLIN_ERR_OOM, "staging allocation for the host-buffer forward");
         }
-        if ((err = cudaStreamCreateWithFlags(&h->host_st[k], cudaStreamNonBlocking)) != cudaSuccess ||
-            (err = cudaEventCreateWithFlags(&h->host_ev_out[k], cudaEventDisableTiming)) != cudaSuccess) {
-            release_host_staging(h);
-            return cuda_fail(err, "host-buffer forward streams");
-        }
+        for (cudaEvent_t* ev : {&h->host_ev_in[k], &h->host_ev_run[k], &h->host_ev_out[k]})
+            if (err == cudaSuccess) err = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
     }
-    if ((err = cudaEventCreateWithFlags(&h->host_ev_in, cudaEventDisableTiming)) != cudaSuccess) {
+    for (cudaStream_t* st : {&h->host_in, &h->host_run, &h->host_out})
+        if (err == cudaSuccess) err = cudaStreamCreateWithFlags(st, cudaStreamNonBlocking);
+    for (cudaEvent_t* ev : {&h->host_ev_start, &h->host_ev_done})
+        if (err == cudaSuccess) err = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+    if (err != cudaSuccess) {
         release_host_staging(h);
         return cuda_fail(err, "host-buffer forward streams");
     }
@@ -394,35 +414,49 @@ int eqlin_forward_host(eqlin_handle* h, const void* x_host, void* y_host, int64_
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const size_t el = io_elem_bytes(h->io_dtype);
     const size_t row_x = static_cast<size_t>(h->Cin * h->G) * el, row_y = static_cast<size_t>(h->Cout * h->G) * el;
-    // both internal streams start after the work already queued on the caller's stream
-    if ((e = cudaEventRecord(h->host_ev_in, st)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-    for (int k = 0; k < 2; ++k)
-        if ((e = cudaStreamWaitEvent(h->host_st[k], h->host_ev_in, 0)) != cudaSuccess)
+    // the internal streams start after the work already queued on the caller's stream
+    if ((e = cudaEventRecord(h->host_ev_start, st)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    for (cudaStream_t si : {h->host_in, h->host_run, h->host_out})
+        if ((e = cudaStreamWaitEvent(si, h->host_ev_start, 0)) != cudaSuccess)
             return cuda_fail(e, "cudaStreamWaitEvent");
-    // chunk i on stream i % 2 with buffers i % 2: a stream's own order protects its
-    // buffers, and the two streams overlap the copies in and out
+    // Chunk i (counted over all calls on the handle, so that a call on another stream
+    // cannot overwrite buffers the previous one still uses) takes buffers
+    // b = i mod kHostBufs.  Copies in, kernels and copies out each have a stream of their
+    // own, so the two copy directions run back to back on their engines; events carry
+    // the dependencies: the kernel of chunk i waits for its x and for the copy out of
+    // chunk i - kHostBufs (the y buffer), the copy in of chunk i for the kernel of chunk
+    // i - kHostBufs (the x buffer), the copy out for the kernel.
     const auto* xb = static_cast<const uint8_t*>(x_host);
     auto* yb = static_cast<uint8_t*>(y_host);
-    int64_t i = 0;
-    for (int64_t n0 = 0; n0 < N; n0 += h->host_chunk, ++i) {
-        const int k = static_cast<int>(i & 1);
+    auto wait = [&](cudaStream_t si, cudaEvent_t ev) { return cudaStreamWaitEvent(si, ev, 0); };
+    for (int64_t n0 = 0; n0 < N; n0 += h->host_chunk) {
+        const int64_t i = h->host_seq++;
+        const int b = static_cast<int>(i % eqlin_handle::kHostBufs);
+        const bool reuse = i >= eqlin_handle::kHostBufs;
         const int64_t n = std::min<int64_t>(h->host_chunk, N - n0);
-        cudaStream_t sk = h->host_st[k];
-        if ((e = cudaMemcpyAsync(h->host_x[k], xb + n0 * row_x, n * row_x, cudaMemcpyHostToDevice, sk)) !=
-            cudaSuccess)
+        if ((reuse && (e = wait(h->host_in, h->host_ev_run[b])) != cudaSuccess) ||
+            (e = cudaMemcpyAsync(h->host_x[b], xb + n0 * row_x, n * row_x, cudaMemcpyHostToDevice, h->host_in)) !=
+                cudaSuccess ||
+            (e = cudaEventRecord(h->host_ev_in[b], h->host_in)) != cudaSuccess)
             return cuda_fail(e, "host-to-device copy");
-        s = launch_forward(h->plan, h->Cout, h->Cin, h->G, h->sm_count, h->host_x[k], h->host_y[k], n, h->buf,
-                           h->timeout_ns, sk);
+        if ((e = wait(h->host_run, h->host_ev_in[b])) != cudaSuccess ||
+            (reuse && (e = wait(h->host_run, h->host_ev_out[b])) != cudaSuccess))
+            return cuda_fail(e, "cudaStreamWaitEvent");
+        s = launch_forward(h->plan, h->Cout, h->Cin, h->G, h->sm_count, h->host_x[b], h->host_y[b], n, h->buf,
+                           h->timeout_ns, h->host_run);
         if (s != EQLIN_OK) return s;
-        if ((e = cudaMemcpyAsync(yb + n0 * row_y, h->host_y[k], n * row_y, cudaMemcpyDeviceToHost, sk)) !=
-            cudaSuccess)
+        if ((e = cudaEventRecord(h->host_ev_run[b], h->host_run)) != cudaSuccess ||
+            (e = wait(h->host_out, h->host_ev_run[b])) != cudaSuccess ||
+            (e = cudaMemcpyAsync(yb + n0 * row_y, h->host_y[b], n * row_y, cudaMemcpyDeviceToHost, h->host_out)) !=
+                cudaSuccess ||
+            (e = cudaEventRecord(h->host_ev_out[b], h->host_out)) != cudaSuccess)
             return cuda_fail(e, "device-to-host copy");
     }
-    for (int k = 0; k < 2; ++k) {
-        if ((e = cudaEventRecord(h->host_ev_out[k], h->host_st[k])) != cudaSuccess ||
-            (e = cudaStreamWaitEvent(st, h->host_ev_out[k], 0)) != cudaSuccess)
-            return cuda_fail(e, "stream join");
-    }
+    // every copy out follows its kernel, which follows its copy in: the caller's stream
+    // waits for the last copy out
+    if ((e = cudaEventRecord(h->host_ev_done, h->host_out)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(st, h->host_ev_done, 0)) != cudaSuccess)
+        return cuda_fail(e, "stream join");
     if (h->sync_check) {
         int dst = 0;
         if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return cuda_fail(e, "forward (EQLIN_SYNC_CHECK)");

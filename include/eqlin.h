@@ -123,10 +123,11 @@ EQLIN_API int eqlin_forward(const eqlin_handle* h, const void* x, void* y, int64
  * eqlin_forward_host -- the same forward with x and y in HOST memory: the library
  * copies x in, runs the fused kernel and copies y back, chunk by chunk, so that the
  * host-to-device copy of one chunk, the kernel of another and the device-to-host copy
- * of a third overlap (two internal streams; full-duplex copies).
+ * of a third overlap (three internal streams: copies in, kernels, copies out;
+ * full-duplex copies).
  *
  *   h        handle from eqlin_prepare_weights.  The first call allocates the handle's
- *            staging buffers (two chunks of x and of y, about 32 MB) and two streams,
+ *            staging buffers (four chunks of x and of y, about 64 MB) and three streams,
  *            freed by eqlin_destroy.  Calls on one handle are serialised by the
  *            library (a mutex for the host side, the internal streams for the GPU).
  *   x_host   host, [N, Cin, G] of the handle's io_dtype.  Pinned memory (cudaHostAlloc,

@@ -314,6 +314,32 @@ def test_host_buffer_forward_matches_device_forward():
     h.close()
 
 
+def test_host_buffer_forward_on_two_streams():
+    """Two host-buffer calls on one handle, issued on two streams without a synchronisation
+    between them, each over more chunks than the handle has staging buffers: the second
+    call's copies must wait for the first call's use of the shared buffers, so both
+    results equal the device-buffer forward."""
+    wl = workloads.WORKLOADS["p4_c96_bf16"]
+    N = 6 * 10880 + 300                       # 10880 tokens per chunk at p4 C96: 7 chunks
+    x1, w, bias = workloads.make_inputs(wl, seed=31, N=N)
+    x2, _, _ = workloads.make_inputs(wl, seed=32, N=N)
+    h = _prep(w, bias, wl.torch_dtype)
+    ref1, ref2 = h.forward(x1.to(DEV)).cpu(), h.forward(x2.to(DEV)).cpu()
+    xs = [x1.pin_memory(), x2.pin_memory()]
+    ys = [torch.empty(N, wl.Cout, wl.G, dtype=wl.torch_dtype, pin_memory=True) for _ in range(2)]
+    streams = [torch.cuda.Stream(DEV), torch.cuda.Stream(DEV)]
+    lib = eq.library()
+    torch.cuda.synchronize()
+    for k in range(2):
+        st = lib.eqlin_forward_host(h.ptr, xs[k].data_ptr(), ys[k].data_ptr(), N, streams[k].cuda_stream)
+        assert st == eq.EQLIN_OK
+    for s_ in streams:
+        s_.synchronize()
+    assert h.device_status() == eq.EQLIN_OK
+    assert torch.equal(ys[0], ref1) and torch.equal(ys[1], ref2)
+    h.close()
+
+
 def test_tolerances_are_the_stated_ones():
     assert TOL_F32_MAXREL == 1e-5 and TOL_BF16_NORMWISE == 2e-2
 
