@@ -14,8 +14,10 @@ oracle's throughput on a bounded sample.
 The same line carries a ``workloads`` object with every synthetic workload
 (tiny p4 fp32, p4 C96, p8 C64, p4 MLP 192->768, C16 C32), each measured in this run
 the same way: us per launch over back-to-back launches, tokens/s, roofline,
-dense-equivalent TFLOP/s, the backward calls, and the oracle on a bounded sample of
-that workload.  The headline runs first, then the other workloads.
+dense-equivalent TFLOP/s, the backward calls, the MLP block, the pages' dense
+baseline as context (one cuBLAS GEMM on the replicated group-circulant weight), and
+the oracle on a bounded sample of that workload.  The headline runs first, then the
+other workloads.
 
 Multi-GPU (torchrun): every rank runs the full workload on its own GPU (tokens
 are independent, no collective on the data path): weak scaling; the timed
@@ -456,7 +458,7 @@ def setup_workload(ctx: Ctx, wl: workloads.Workload, args) -> dict:
     _, n_sets = rotating_sets(wl, wl.N)
     xs = [x_cpu.to(dev) for _ in range(n_sets)]
     ys = [torch.empty(wl.N, wl.Cout, wl.G, dtype=wl.torch_dtype, device=dev) for _ in range(n_sets)]
-    return {"x_cpu": x_cpu, "h": h, "xs": xs, "ys": ys, "n_sets": n_sets}
+    return {"x_cpu": x_cpu, "w": w, "bias": bias, "h": h, "xs": xs, "ys": ys, "n_sets": n_sets}
 
 
 def measure_workload(ctx: Ctx, wl: workloads.Workload, K: int, warmup: int, headline: bool, args,
@@ -603,10 +605,51 @@ def measure_workload(ctx: Ctx, wl: workloads.Workload, K: int, warmup: int, head
     if not args.no_mlp_block and wl.io_dtype != "f32" and wl.Cin == wl.Cout:
         out["mlp_block"] = measure_mlp_block(ctx, wl, xs, ys, n_sets, K, warmup)
 
+    # ------------------------------------------------------- dense baseline (context)
+    if not args.no_dense_context and wl.io_dtype != "f32":
+        out["dense_context"] = measure_dense_context(ctx, wl, su["w"], su["bias"], h, xs, n_sets, K, warmup,
+                                                     out["us_per_launch"])
+
     h.close()
     del xs, ys
     torch.cuda.empty_cache()
     return out
+
+
+def measure_dense_context(ctx: Ctx, wl: workloads.Workload, w, bias, h, xs, n_sets: int, K: int, warmup: int,
+                          fused_us: float) -> dict:
+    """The pages' baseline, for context: the layer as one dense GEMM over the replicated
+    weight ("Declaracion del Problema": the group-circulant matrix M[(o,g),(i,h)] =
+    w[o,i,(g-h) mod G], built on the device by indexing, then torch's F.linear, a cuBLAS
+    bf16 GEMM with fp32 accumulation), timed like the fused kernel: K back-to-back calls
+    between two events on rotating x sets.  Its output is compared with the fused
+    kernel's (relative norm difference), which checks the matrix's convention."""
+    import torch.nn.functional as F
+    dev, stream = ctx.dev, ctx.stream
+    G, N = wl.G, wl.N
+    wd = w.to(dev)
+    gi = torch.arange(G, device=dev)
+    idx = (gi.view(G, 1) - gi.view(1, G)) % G                      # [g, h] -> (g - h) mod G
+    M = wd[:, :, idx].permute(0, 2, 1, 3).reshape(wl.Cout * G, wl.Cin * G).contiguous()
+    bd = None if bias is None else bias.to(dev).repeat_interleave(G)
+    x2 = [t.view(N, wl.Cin * G) for t in xs]
+    for i in range(max(3, warmup)):
+        F.linear(x2[i % n_sets], M, bd)
+    res = {}
+
+    def run(i, st=stream):
+        res["y"] = F.linear(x2[i % n_sets], M, bd)
+
+    ms = time_back_to_back(ctx, run, K, graph=False)
+    us = 1e3 * ms / K
+    y_d = res["y"].float()
+    y_f = h.forward(xs[(K - 1) % n_sets], stream=stream).view(N, wl.Cout * G).float()
+    diff = ((y_d - y_f).norm() / y_f.norm()).item()
+    dense_fl = 2.0 * N * (wl.Cin * G) * (wl.Cout * G)
+    return {"us_per_call": us, "calls": K, "dense_flops": dense_fl, "dense_tflops": dense_fl / (us * 1e-6) / 1e12,
+            "fused_over_dense_speedup": us / fused_us, "rel_diff_vs_fused": diff,
+            "what": "F.linear on the replicated group-circulant [Cout*G, Cin*G] matrix (cuBLAS, bf16 in, fp32 "
+                    "accumulate); the x sets rotate as in the fused timing; context, not a target"}
 
 
 def measure_mlp_block(ctx: Ctx, wl: workloads.Workload, xs, ys, n_sets: int, K: int, warmup: int) -> dict:
@@ -671,6 +714,9 @@ def main() -> None:
                          "(the graph is replayed once, untimed, to upload it)")
     ap.add_argument("--no-mlp-block", action="store_true",
                     help="skip the extra measurement of the equivariant MLP block L2(GELU(L1(x))), H = 4 C")
+    ap.add_argument("--no-dense-context", action="store_true",
+                    help="skip the pages' baseline, one dense cuBLAS GEMM on the replicated weight, timed "
+                         "as context (dense_context in each 16-bit workload)")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the extra measurement of the backward calls (input and weight gradients)")
     ap.add_argument("--tokens", type=int, default=None,
@@ -760,6 +806,7 @@ def main() -> None:
         "cpu_baseline": cpu,
         "backward": head.get("backward"),
         "mlp_block": head.get("mlp_block"),
+        "dense_context": head.get("dense_context"),
         "workloads": wl_obj,
     }
     emit(line)
