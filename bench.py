@@ -620,11 +620,12 @@ def measure_dense_context(ctx: Ctx, wl: workloads.Workload, w, bias, h, xs, n_se
                           fused_us: float) -> dict:
     """The pages' baseline, for context: the layer as one dense GEMM over the replicated
     weight ("Declaracion del Problema": the group-circulant matrix M[(o,g),(i,h)] =
-    w[o,i,(g-h) mod G], built on the device by indexing, then torch's F.linear, a cuBLAS
-    bf16 GEMM with fp32 accumulation), timed like the fused kernel: K back-to-back calls
-    between two events on rotating x sets.  Its output is compared with the fused
-    kernel's (relative norm difference), which checks the matrix's convention."""
-    import torch.nn.functional as F
+    w[o,i,(g-h) mod G], built on the device by indexing, then the GEMM F.linear runs,
+    y = x M^T + b, as torch.addmm (torch.mm without bias) into preallocated outputs: a
+    cuBLAS bf16 GEMM with fp32 accumulation and no allocation in the timed loop), timed
+    like the fused kernel: K back-to-back calls between two events on rotating x/y sets.
+    Its output is compared with the fused kernel's (relative norm difference), which
+    checks the matrix's convention."""
     dev, stream = ctx.dev, ctx.stream
     G, N = wl.G, wl.N
     wd = w.to(dev)
@@ -633,23 +634,28 @@ def measure_dense_context(ctx: Ctx, wl: workloads.Workload, w, bias, h, xs, n_se
     M = wd[:, :, idx].permute(0, 2, 1, 3).reshape(wl.Cout * G, wl.Cin * G).contiguous()
     bd = None if bias is None else bias.to(dev).repeat_interleave(G)
     x2 = [t.view(N, wl.Cin * G) for t in xs]
-    for i in range(max(3, warmup)):
-        F.linear(x2[i % n_sets], M, bd)
-    res = {}
+    y2 = [torch.empty(N, wl.Cout * G, dtype=wl.torch_dtype, device=dev) for _ in range(n_sets)]
+    Mt = M.t()
 
     def run(i, st=stream):
-        res["y"] = F.linear(x2[i % n_sets], M, bd)
+        if bd is None:
+            torch.mm(x2[i % n_sets], Mt, out=y2[i % n_sets])
+        else:
+            torch.addmm(bd, x2[i % n_sets], Mt, out=y2[i % n_sets])
 
+    for i in range(max(3, warmup)):
+        run(i)
     ms = time_back_to_back(ctx, run, K, graph=False)
     us = 1e3 * ms / K
-    y_d = res["y"].float()
+    y_d = y2[(K - 1) % n_sets].float()
     y_f = h.forward(xs[(K - 1) % n_sets], stream=stream).view(N, wl.Cout * G).float()
     diff = ((y_d - y_f).norm() / y_f.norm()).item()
     dense_fl = 2.0 * N * (wl.Cin * G) * (wl.Cout * G)
     return {"us_per_call": us, "calls": K, "dense_flops": dense_fl, "dense_tflops": dense_fl / (us * 1e-6) / 1e12,
             "fused_over_dense_speedup": us / fused_us, "rel_diff_vs_fused": diff,
-            "what": "F.linear on the replicated group-circulant [Cout*G, Cin*G] matrix (cuBLAS, bf16 in, fp32 "
-                    "accumulate); the x sets rotate as in the fused timing; context, not a target"}
+            "what": "the GEMM of F.linear (torch.addmm / torch.mm into preallocated outputs) on the replicated "
+                    "group-circulant [Cout*G, Cin*G] matrix: cuBLAS, bf16 in, fp32 accumulate; x/y sets rotate "
+                    "as in the fused timing; context, not a target"}
 
 
 def measure_mlp_block(ctx: Ctx, wl: workloads.Workload, xs, ys, n_sets: int, K: int, warmup: int) -> dict:
