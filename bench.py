@@ -616,6 +616,16 @@ def measure_workload(ctx: Ctx, wl: workloads.Workload, K: int, warmup: int, head
     return out
 
 
+def group_circulant_matrix(w: torch.Tensor) -> torch.Tensor:
+    """The replicated dense weight of the pages' baseline ("Declaracion del Problema"):
+    M[(o,g),(i,h)] = w[o,i,(g-h) mod G] as a [Cout*G, Cin*G] matrix, built by indexing on
+    w's device, so that y[n] = M x[n] over the flattened [Cin*G] token."""
+    Cout, Cin, G = w.shape
+    gi = torch.arange(G, device=w.device)
+    idx = (gi.view(G, 1) - gi.view(1, G)) % G                      # [g, h] -> (g - h) mod G
+    return w[:, :, idx].permute(0, 2, 1, 3).reshape(Cout * G, Cin * G).contiguous()
+
+
 def measure_dense_context(ctx: Ctx, wl: workloads.Workload, w, bias, h, xs, n_sets: int, K: int, warmup: int,
                           fused_us: float) -> dict:
     """The pages' baseline, for context: the layer as one dense GEMM over the replicated
@@ -628,10 +638,7 @@ def measure_dense_context(ctx: Ctx, wl: workloads.Workload, w, bias, h, xs, n_se
     checks the matrix's convention."""
     dev, stream = ctx.dev, ctx.stream
     G, N = wl.G, wl.N
-    wd = w.to(dev)
-    gi = torch.arange(G, device=dev)
-    idx = (gi.view(G, 1) - gi.view(1, G)) % G                      # [g, h] -> (g - h) mod G
-    M = wd[:, :, idx].permute(0, 2, 1, 3).reshape(wl.Cout * G, wl.Cin * G).contiguous()
+    M = group_circulant_matrix(w.to(dev))
     bd = None if bias is None else bias.to(dev).repeat_interleave(G)
     x2 = [t.view(N, wl.Cin * G) for t in xs]
     y2 = [torch.empty(N, wl.Cout * G, dtype=wl.torch_dtype, device=dev) for _ in range(n_sets)]

@@ -118,3 +118,22 @@ def test_clock_sampler_stays_out_of_short_timed_regions(monkeypatch):
     threading.Event().wait(0.1)   # a region of ten periods is sampled inside
     c.stop()
     assert len(calls) >= 5
+
+
+@pytest.mark.parametrize("Cout,Cin,G", [(3, 5, 2), (4, 3, 4), (2, 3, 8), (3, 2, 16)])
+def test_dense_baseline_matrix_is_the_oracle_one(Cout, Cin, G):
+    """The dense baseline the bench times beside the fused kernel multiplies by the same
+    replicated group-circulant matrix as the oracle's dense_weight, and that matrix
+    reproduces the oracle's forward."""
+    import numpy as np
+    import torch
+
+    import oracle
+    b = _bench()
+    gen = torch.Generator().manual_seed(Cout * 100 + Cin * 10 + G)
+    w = torch.randn(Cout, Cin, G, generator=gen, dtype=torch.float64)
+    x = torch.randn(7, Cin, G, generator=gen, dtype=torch.float64)
+    M = b.group_circulant_matrix(w)
+    assert np.array_equal(M.numpy(), oracle.dense_weight(w.numpy()))
+    y = (x.reshape(7, Cin * G) @ M.T).reshape(7, Cout, G)
+    np.testing.assert_allclose(y.numpy(), oracle.forward(x.numpy(), w.numpy()), rtol=1e-12, atol=1e-12)
