@@ -183,7 +183,8 @@ int eqlin_prepare_weights_ex(const void* w, const void* bias, int64_t Cout, int6
         return fail(EQLIN_ERR_UNSUPPORTED, "needs a compute capability 10.0 (sm_100a) device");
 
     Plan plan;
-    s = plan_for(Cout, Cin, G, io_dtype, static_cast<size_t>(optin), &plan);
+    s = plan_for(Cout, Cin, G, io_dtype, static_cast<size_t>(optin), &plan,
+                 (flags & EQLIN_PREPARE_GELU) ? eqlin::kActGelu : eqlin::kActNone);
     if (s != EQLIN_OK) return s;
 
     eqlin_handle* h = new (std::nothrow) eqlin_handle();

@@ -260,7 +260,14 @@ int plan_tm_g(int64_t Cout, int64_t Cin, size_t max_smem, Plan* pl) {
 // double-buffered tokens-on-N kernel stays ahead (p4 C96: 70.1 vs 76.6 us).
 bool default_tokens_on_m(int G) { return G >= 8; }
 
-int plan_for(int64_t Cout, int64_t Cin, int64_t G, int io_dtype, size_t max_smem, Plan* pl) {
+// `act`: the forward's epilogue activation.  With GELU the epilogue is ALU-bound, and the
+// resident-input form (x transformed once per tile, not once per output chunk) wins from 2
+// input chunks on and for G = 8 too (B200, 20 GELU layers back to back: p4 96 -> 384 309.2
+// vs 324.6 us streamed, 64 -> 256 206.6 vs 210.5, 96 -> 256 211.8 vs 219.5; G = 8 64 -> 256
+// 59.0 vs 67.8 us tokens on M at N = 25088, 198.2 vs 231.2 at 100352), while without an
+// activation the rules below stand (96 -> 384: 191.4 vs 180.2 us).
+int plan_for(int64_t Cout, int64_t Cin, int64_t G, int io_dtype, size_t max_smem, Plan* pl,
+             int act = eqlin::kActNone) {
     pl->io = io_dtype;
     if (io_dtype == EQLIN_F32) {
         const size_t smem = static_cast<size_t>(eqlin::kF32Tokens) * G * Cin * sizeof(double);
@@ -273,10 +280,20 @@ int plan_for(int64_t Cout, int64_t Cin, int64_t G, int io_dtype, size_t max_smem
     bool tm = default_tokens_on_m(static_cast<int>(G));
     bool tnr_ok = true;   // tokens on N: prefer the resident-input form when it applies
     bool tnr_forced = false;
+    const bool gelu_tnr = act == eqlin::kActGelu && G <= 8 && Cout > eqlin::kMmaM && Cin > eqlin::kChunkK;
     if (const char* e = std::getenv("EQLIN_KERNEL")) {
         if (std::strcmp(e, "tm") == 0) tm = true;
         if (std::strcmp(e, "tn") == 0) tm = false, tnr_ok = false;
         if (std::strcmp(e, "tnr") == 0) tm = false, tnr_forced = true;
+    } else if (gelu_tnr) {
+        int r = EQLIN_ERR_UNSUPPORTED;
+        switch (G) {
+            case 2: r = plan_tnr_g<2>(Cout, Cin, max_smem, true, pl); break;
+            case 4: r = plan_tnr_g<4>(Cout, Cin, max_smem, true, pl); break;
+            case 8: r = plan_tnr_g<8>(Cout, Cin, max_smem, true, pl); break;
+            default: break;
+        }
+        if (r == EQLIN_OK) return EQLIN_OK;
     }
     if (!tm && tnr_ok) {
         int r = EQLIN_ERR_UNSUPPORTED;

@@ -193,7 +193,9 @@ EQLIN_API int eqlin_get_attr(const eqlin_handle* h, int attr, int64_t* value);
 
 /*
  * eqlin_query_plan -- the same properties (EQLIN_ATTR_PATH .. EQLIN_ATTR_DW_TOKENS,
- * except ACTIVATION) that eqlin_prepare_weights would give a handle of these sizes,
+ * except ACTIVATION) that eqlin_prepare_weights would give a handle of these sizes
+ * without an activation (a GELU handle with Cout > 128 and G <= 8 takes the tokens-on-N
+ * kernel with the input spectrum resident wherever it fits),
  * planned on the host for a B200 (227 KB of shared memory per CTA, 148 SMs) under the
  * current environment overrides.  Host only: no GPU, no allocation.  The weight-gradient
  * attributes are -1 where no tiling fits (or for fp32 I/O).

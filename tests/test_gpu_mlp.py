@@ -37,7 +37,8 @@ def _block(N, Cin, H, Cout, G, io, seed):
 
 
 @pytest.mark.parametrize("io", [torch.bfloat16, torch.float16, torch.float32])
-@pytest.mark.parametrize("Cout,Cin,G", [(96, 96, 4), (64, 64, 8), (32, 32, 16), (50, 40, 4), (200, 32, 4)])
+@pytest.mark.parametrize("Cout,Cin,G", [(96, 96, 4), (64, 64, 8), (32, 32, 16), (50, 40, 4), (200, 32, 4),
+                                        (384, 96, 4), (256, 64, 8), (136, 40, 2), (160, 96, 4)])
 def test_gelu_epilogue(Cout, Cin, G, io):
     x, w, b, _, _ = _block(517, Cin, Cout, Cout, G, io, Cout + Cin + G)
     h = eq.prepare(w.to(DEV), b.to(DEV), io_dtype=io, activation="gelu")
@@ -49,6 +50,27 @@ def test_gelu_epilogue(Cout, Cin, G, io):
     r = check(io, y.cpu(), ref)
     assert r["ok"], r
     h.close()
+
+
+RES_X, STREAMED, RES_W = ("tcgen05_tokens_on_n_resident_input", "tcgen05_tokens_on_n_streamed_weights",
+                           "tcgen05_tokens_on_n_resident_weights")
+TM_STREAMED = "tcgen05_tokens_on_m_streamed_weights"
+
+
+@pytest.mark.parametrize("Cout,Cin,G,gelu_path,plain_path", [
+    (384, 96, 4, RES_X, STREAMED), (256, 64, 8, RES_X, TM_STREAMED), (136, 40, 2, RES_X, STREAMED),
+    (384, 32, 4, STREAMED, STREAMED), (128, 96, 4, RES_W, RES_W), (128, 32, 16, TM_STREAMED, TM_STREAMED),
+])
+def test_gelu_layers_take_the_resident_input_kernel(Cout, Cin, G, gelu_path, plain_path):
+    """A GELU layer with several output chunks (Cout > 128), G <= 8 and at least two
+    input chunks takes the tokens-on-N kernel with the input spectrum resident: its
+    epilogue is ALU-bound, and transforming x once per tile rather than once per output
+    chunk pays there.  The same layer without an activation keeps its own kernel."""
+    w = torch.zeros(Cout, Cin, G, dtype=torch.bfloat16, device=DEV)
+    h, h_plain = eq.prepare(w, None, activation="gelu"), eq.prepare(w, None)
+    assert (h.path, h_plain.path) == (gelu_path, plain_path)
+    h.close()
+    h_plain.close()
 
 
 @pytest.mark.parametrize("io", [torch.bfloat16, torch.float16, torch.float32])
