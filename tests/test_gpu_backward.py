@@ -219,3 +219,50 @@ def test_backward_edge_channel_counts(Cout, Cin, G):
     _assert(torch.bfloat16, dw.cpu(), dw_ref, f"dw {Cout},{Cin},{G}")
     _assert(torch.bfloat16, db.cpu(), db_ref, f"dbias {Cout},{Cin},{G}")
     h.close()
+
+
+def test_forward_backward_and_mlp_block_replay_from_a_cuda_graph():
+    """The calls a training or serving step makes -- the forward, dx, dw + dbias (two
+    launches, the second a programmatic dependent) and the fused MLP block -- captured once
+    into a CUDA graph on a side stream and replayed: every replay equals the calls made
+    one by one, bit for bit."""
+    wl = workloads.WORKLOADS["p4_c96_bf16"]
+    N = 3 * 148 * 64 + 77
+    x, w, bias = workloads.make_inputs(wl, seed=41, N=N)
+    dev = torch.device(DEV)
+    h = eq.prepare(w.to(dev), bias.to(dev), io_dtype=wl.torch_dtype, backward=True)
+    H = 4 * wl.Cin
+    w1, b1, w2, b2 = workloads.make_mlp_weights(wl, H)
+    m = eq.eqlin_mlp_prepare(w1.to(dev), b1.to(dev), w2.to(dev), b2.to(dev))
+    xd = x.to(dev)
+    y = torch.empty(N, wl.Cout, wl.G, dtype=wl.torch_dtype, device=dev)
+    dx = torch.empty(N, wl.Cin, wl.G, dtype=wl.torch_dtype, device=dev)
+    dw = torch.empty(wl.Cout, wl.Cin, wl.G, dtype=torch.float32, device=dev)
+    db = torch.empty(wl.Cout, dtype=torch.float32, device=dev)
+    ym = torch.empty(N, wl.Cout, wl.G, dtype=wl.torch_dtype, device=dev)
+    ws = torch.empty(max(16, eq.eqlin_backward_dw_workspace_size(h, N)), dtype=torch.uint8, device=dev)
+
+    def step(st):
+        h.forward(xd, out=y, stream=st)
+        h.backward_dx(y, out=dx, stream=st)
+        eq.eqlin_backward_dw(h, xd, y, stream=st, dw=dw, dbias=db, workspace=ws)
+        m.forward(xd, out=ym, stream=st)
+
+    side = torch.cuda.Stream(dev)
+    step(side)
+    side.synchronize()
+    ref = [t.clone() for t in (y, dx, dw, db, ym)]
+    for t in (y, dx, dw, db, ym):
+        t.zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        step(side)
+    for _ in range(2):
+        g.replay()
+        torch.cuda.synchronize()
+        for got, want in zip((y, dx, dw, db, ym), ref):
+            assert torch.equal(got, want)
+    assert h.device_status() == eq.EQLIN_OK and m.device_status() == eq.EQLIN_OK
+    del g
+    h.close()
+    m.close()
