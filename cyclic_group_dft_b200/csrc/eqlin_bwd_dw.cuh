@@ -566,8 +566,11 @@ __global__ void __launch_bounds__(kDwFinishWarps * 32) eqlin_dw_finish_kernel(co
                            (bias_blk ? f.slab_floats + oo : static_cast<size_t>(ii) * f.MO + oo);
         const int nv = bias_blk ? 1 : G;
         int s = warp;
-        // kIn splits in flight (kIn * G <= 32 loads per thread), added in split order
-        constexpr int kIn = 32 / G > 2 ? 32 / G : 2;
+        // kIn splits in flight per round trip, added in split order.  32 / G loads per
+        // thread for G <= 8 keeps the block at 64-66 registers, so two blocks share an SM
+        // (10 splits at G = 4, one round trip for 148 splits, took 76 registers and measured
+        // 73.3 against 71.0 us at p4 C96); G = 16 takes 4 (128 registers, unspilled)
+        constexpr int kIn = G == 16 ? 4 : 32 / G;
         for (; s + W * (kIn - 1) < f.n_splits; s += W * kIn) {
             float v[kIn][G];
 #pragma unroll
@@ -597,8 +600,8 @@ __global__ void __launch_bounds__(kDwFinishWarps * 32) eqlin_dw_finish_kernel(co
 #pragma unroll
     for (int pl = 0; pl < G; ++pl) {
         double v = 0.0;
-#pragma unroll
-        for (int w = 0; w < W; ++w) v += red(w, pl);
+#pragma unroll 4
+        for (int w = 0; w < W; ++w) v += red(w, pl);   // in warp order (deterministic)
         z[pl] = v;
     }
     const int ot = unit / f.n_it, it = unit % f.n_it;
