@@ -340,6 +340,31 @@ def test_host_buffer_forward_on_two_streams():
     h.close()
 
 
+@pytest.mark.parametrize("name", ["p4_c96_bf16", "p8_c64_bf16", "p4_mlp_bf16"])
+def test_concurrent_forwards_of_one_handle_on_two_streams(name):
+    """A prepared handle is read-only on the forward path (weights, bias, plan), so
+    forwards of one handle issued on two streams at once, with no synchronisation between
+    them, give the same outputs as the same calls made one after the other."""
+    wl = workloads.WORKLOADS[name]
+    N = 3 * 148 * 64 + 123
+    xa, w, bias = workloads.make_inputs(wl, seed=51, N=N)
+    xb, _, _ = workloads.make_inputs(wl, seed=52, N=N)
+    h = _prep(w, bias, wl.torch_dtype)
+    xs = [xa.to(DEV), xb.to(DEV)]
+    serial = [h.forward(t).clone() for t in xs]
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(DEV), torch.cuda.Stream(DEV)]
+    outs = [torch.empty_like(serial[0]) for _ in range(2)]
+    for rep in range(3):
+        for k in range(2):
+            h.forward(xs[k], out=outs[k], stream=streams[k])
+        for s_ in streams:
+            s_.synchronize()
+        assert torch.equal(outs[0], serial[0]) and torch.equal(outs[1], serial[1])
+    assert h.device_status() == eq.EQLIN_OK
+    h.close()
+
+
 def test_tolerances_are_the_stated_ones():
     assert TOL_F32_MAXREL == 1e-5 and TOL_BF16_NORMWISE == 2e-2
 
