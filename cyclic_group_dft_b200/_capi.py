@@ -299,8 +299,23 @@ def eqlin_forward_host(h: Handle, x_host: torch.Tensor, y_host: torch.Tensor | N
         ptr = _stream_ptr(stream)
         _check(_lib.eqlin_forward_host(h.ptr, x_host.data_ptr(), y_host.data_ptr(), N, ptr),
                "eqlin_forward_host")
-        (stream if isinstance(stream, torch.cuda.Stream) else torch.cuda.ExternalStream(ptr)).synchronize()
+        _synchronize(stream, ptr)
     return y_host
+
+
+def _synchronize(stream, ptr: int) -> None:
+    """Block until the work queued on the call's stream is done.  A torch Stream (or None,
+    the current stream) synchronises itself; a raw pointer goes through ExternalStream,
+    except 0, the legacy default stream, which ExternalStream(0) does not wait for (measured
+    on B200: the call returned before its copies out in 99 of 100 trials)."""
+    if isinstance(stream, torch.cuda.Stream):
+        stream.synchronize()
+    elif stream is None:
+        torch.cuda.current_stream().synchronize()
+    elif ptr == 0:
+        torch.cuda.default_stream().synchronize()
+    else:
+        torch.cuda.ExternalStream(ptr).synchronize()
 
 
 def _check_rows(t: torch.Tensor, name: str, C: int, h: Handle) -> None:

@@ -314,6 +314,28 @@ def test_host_buffer_forward_matches_device_forward():
     h.close()
 
 
+@pytest.mark.parametrize("which", ["none", "torch_stream", "raw_default_pointer"])
+def test_host_buffer_forward_returns_with_y_in_place(which):
+    """The binding's forward_host returns only once y is in host memory, whichever way the
+    stream is given (None = the current stream, a torch Stream, or the raw pointer 0 of the
+    legacy default stream): a NaN-filled pinned output holds the device forward's values
+    right after the call, with no synchronisation by the caller."""
+    wl = workloads.WORKLOADS["p4_c96_bf16"]
+    x, w, bias = workloads.make_inputs(wl, seed=61, N=2048)
+    h = _prep(w, bias, wl.torch_dtype)
+    ref = h.forward(x.to(DEV)).cpu()
+    xp = x.pin_memory()
+    side = torch.cuda.Stream(DEV)
+    stream = {"none": None, "torch_stream": side, "raw_default_pointer": 0}[which]
+    for _ in range(20):
+        yp = torch.full((2048, wl.Cout, wl.G), float("nan"), dtype=wl.torch_dtype).pin_memory()
+        torch.cuda.synchronize()
+        out = h.forward_host(xp, yp, stream=stream)
+        snap = out.clone()                      # before any synchronisation of ours
+        assert torch.equal(snap, ref)
+    h.close()
+
+
 def test_host_buffer_forward_on_two_streams():
     """Two host-buffer calls on one handle, issued on two streams without a synchronisation
     between them, each over more chunks than the handle has staging buffers: the second
