@@ -566,11 +566,12 @@ __global__ void __launch_bounds__(kDwFinishWarps * 32) eqlin_dw_finish_kernel(co
                            (bias_blk ? f.slab_floats + oo : static_cast<size_t>(ii) * f.MO + oo);
         const int nv = bias_blk ? 1 : G;
         int s = warp;
-        // kIn splits in flight per round trip, added in split order.  32 / G loads per
-        // thread for G <= 8 keeps the block at 64-66 registers, so two blocks share an SM
-        // (10 splits at G = 4, one round trip for 148 splits, took 76 registers and measured
-        // 73.3 against 71.0 us at p4 C96); G = 16 takes 4 (128 registers, unspilled)
-        constexpr int kIn = G == 16 ? 4 : 32 / G;
+        // kIn splits in flight per round trip, added in split order.  Measured on B200
+        // (weight gradient, reduction included): G = 4 with 8 (64 registers, two blocks per
+        // SM) 71.0 us at p4 C96, with 10 (76 registers) 73.3; G = 8 with 8 (122 registers)
+        // 26.4 us at p8 C64, with 4 30.7; G = 16 with 4 (128 registers) 176.1 us at C16,
+        // with 2 (and the spills of a fully unrolled warp sum) 177.7
+        constexpr int kIn = G <= 4 ? 32 / G : (G == 8 ? 8 : 4);
         for (; s + W * (kIn - 1) < f.n_splits; s += W * kIn) {
             float v[kIn][G];
 #pragma unroll
@@ -597,10 +598,12 @@ __global__ void __launch_bounds__(kDwFinishWarps * 32) eqlin_dw_finish_kernel(co
     __syncthreads();
     if (warp != 0 || oo >= f.MO) return;
     double z[G];
+    // fully unrolled, the warp sum's G x W shared loads spill at G >= 8 (512 and 1564 B)
+    constexpr int kSumUnroll = G <= 4 ? W : 4;
 #pragma unroll
     for (int pl = 0; pl < G; ++pl) {
         double v = 0.0;
-#pragma unroll 4
+#pragma unroll kSumUnroll
         for (int w = 0; w < W; ++w) v += red(w, pl);   // in warp order (deterministic)
         z[pl] = v;
     }
