@@ -430,11 +430,22 @@ int eqlin_forward_host(eqlin_handle* h, const void* x_host, void* y_host, int64_
     const auto* xb = static_cast<const uint8_t*>(x_host);
     auto* yb = static_cast<uint8_t*>(y_host);
     auto wait = [&](cudaStream_t si, cudaEvent_t ev) { return cudaStreamWaitEvent(si, ev, 0); };
-    for (int64_t n0 = 0; n0 < N; n0 += h->host_chunk) {
+    // Chunk sizes ramp: c/8, c/4, c/2, then c, and what is left at the end is halved down
+    // to c/8, so the first copy in and the last copy out, which run alone, are short.
+    const int64_t c = h->host_chunk;
+    auto next_chunk = [c](int64_t j, int64_t rem) {
+        int64_t sz = j < 3 ? std::max<int64_t>(64, c >> (3 - j)) : c;
+        if (rem < 2 * sz) sz = (rem + 1) / 2;
+        sz = (sz + 63) / 64 * 64;
+        if (sz < c / 8 || sz >= rem) sz = rem;
+        return std::min(sz, rem);
+    };
+    int64_t n = 0;
+    for (int64_t n0 = 0, j = 0; n0 < N; n0 += n, ++j) {
+        n = next_chunk(j, N - n0);
         const int64_t i = h->host_seq++;
         const int b = static_cast<int>(i % eqlin_handle::kHostBufs);
         const bool reuse = i >= eqlin_handle::kHostBufs;
-        const int64_t n = std::min<int64_t>(h->host_chunk, N - n0);
         if ((reuse && (e = wait(h->host_in, h->host_ev_run[b])) != cudaSuccess) ||
             (e = cudaMemcpyAsync(h->host_x[b], xb + n0 * row_x, n * row_x, cudaMemcpyHostToDevice, h->host_in)) !=
                 cudaSuccess ||

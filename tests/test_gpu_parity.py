@@ -342,7 +342,7 @@ def test_host_buffer_forward_on_two_streams():
     call's copies must wait for the first call's use of the shared buffers, so both
     results equal the device-buffer forward."""
     wl = workloads.WORKLOADS["p4_c96_bf16"]
-    N = 6 * 10880 + 300                       # 10880 tokens per chunk at p4 C96: 7 chunks
+    N = 6 * 10880 + 300                       # 10880 tokens per full chunk at p4 C96: > 4 chunks
     x1, w, bias = workloads.make_inputs(wl, seed=31, N=N)
     x2, _, _ = workloads.make_inputs(wl, seed=32, N=N)
     h = _prep(w, bias, wl.torch_dtype)
